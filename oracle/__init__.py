@@ -1,0 +1,209 @@
+"""fp64 CPU oracle for causal linear attention with per-head decay (LASP / LASP-2).
+
+TEST INFRASTRUCTURE. Only ``tests/``, ``__graft_entry__.smoke()`` and the
+``cpu_baseline`` / ``--impl reference`` legs of ``bench.py`` may import this
+package. It shares no code with ``sequence_linear_attention_b200`` and never
+imports it; the CUDA library never calls into it.
+
+The arithmetic lives in ``lasp_oracle.c`` (plain C, double precision, one loop
+nest per definition); this module compiles it with gcc on first use and wraps
+it with ctypes. Each wrapper states the passage it follows:
+
+* :func:`fwd` -- LASP page, section 3.2, Eq. 4-6 (token recurrence).
+* :func:`bwd` -- LASP page, section 3.2, Eq. 12-13 (reverse recurrence).
+* :func:`chunk_states` -- LASP page, Eq. 10 / Algorithm 2 (forward memory
+  state of one chunk) and Eq. 20 / Algorithm 3 (gradient state); LASP-2 review
+  page, "The reading": M_t summarises chunk t.
+* :func:`state_scan` -- LASP-2 review page, "Core claim": prefix sum of the
+  gathered states (forward), suffix sum of dM_t (backward); decay lambda^C per
+  chunk from LASP Eq. 10 / Eq. 20.
+* :func:`state_snapshots` -- LASP page, section 3.4 "KV State Caching": the
+  chunk-boundary states of the recurrences.
+
+Inputs are float32 arrays shaped [B, N, H, d] (any strides, feature axis
+contiguous). Values that came from bf16 are exact in float32 and double, so the
+oracle sees exactly what the GPU sees. Outputs are float64.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "lasp_oracle.c")
+_LIB = os.path.join(_HERE, "liblasp_oracle.so")
+_CFLAGS = ["-O3", "-fopenmp", "-fPIC", "-shared", "-ffp-contract=off", "-std=c11"]
+_lock = threading.Lock()
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile lasp_oracle.c into liblasp_oracle.so (portable x86-64 code)."""
+    stale = (not os.path.exists(_LIB)) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC)
+    if force or stale:
+        tmp = _LIB + f".tmp{os.getpid()}"
+        subprocess.run(["gcc", *_CFLAGS, _SRC, "-o", tmp, "-lm"], check=True)
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+_P = ctypes.c_void_p
+_L = ctypes.c_long
+_I = ctypes.c_int
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is None:
+            lib = ctypes.CDLL(build())
+            lib.oracle_fwd.argtypes = [_P, _P, _P, _L, _L, _L, _P, _P, _P, _L, _L, _L, _P, _I, _L, _I, _I]
+            lib.oracle_bwd.argtypes = [_P, _P, _P, _P, _L, _L, _L, _P, _P, _P,
+                                       _P, _P, _P, _L, _L, _L, _P, _I, _L, _I, _I]
+            lib.oracle_chunk_states.argtypes = [_P, _P, _L, _L, _L, _P, _P, _I, _L, _I, _I, _L, _I]
+            lib.oracle_state_scan.argtypes = [_P, _P, _P, _P, _P, _I, _L, _I, _I, _L, _I]
+            lib.oracle_state_snapshots.argtypes = [_P, _P, _L, _L, _L, _P, _P, _P, _I, _L, _I, _I, _L, _I]
+            lib.oracle_num_threads.restype = _I
+            for f in (lib.oracle_fwd, lib.oracle_bwd, lib.oracle_chunk_states,
+                      lib.oracle_state_scan, lib.oracle_state_snapshots):
+                f.restype = None
+            _lib = lib
+    return _lib
+
+
+def num_threads() -> int:
+    """OpenMP threads the oracle uses (OMP_NUM_THREADS, else all cores)."""
+    return int(_load().oracle_num_threads())
+
+
+def _view(x: np.ndarray, same_as: np.ndarray | None = None):
+    """(pointer, sb, sn, sh) in elements for a [B, N, H, d] float32 view."""
+    if x.dtype != np.float32 or x.ndim != 4 or x.strides[3] != 4:
+        raise ValueError("token tensors must be float32 [B, N, H, d] with a contiguous feature axis")
+    if same_as is not None and (x.shape != same_as.shape or x.strides != same_as.strides):
+        raise ValueError("token tensors must share shape and strides")
+    sb, sn, sh, _ = (s // 4 for s in x.strides)
+    return x.ctypes.data, sb, sn, sh
+
+
+def _lam(lam, H):
+    if lam is None:
+        return None, None
+    a = np.ascontiguousarray(np.asarray(lam, dtype=np.float64).reshape(H))
+    return a, a.ctypes.data
+
+
+def _state(x, shape):
+    if x is None:
+        return None, None
+    a = np.ascontiguousarray(np.asarray(x, dtype=np.float64))
+    if a.shape != shape:
+        raise ValueError(f"state must have shape {shape}, got {a.shape}")
+    return a, a.ctypes.data
+
+
+def _ptr(a):
+    return None if a is None else a.ctypes.data
+
+
+def fwd(q, k, v, lam=None, init=None, want_final=False):
+    """o_s = q_s kv_s with kv_s = lam*kv_{s-1} + k_s^T v_s (LASP Eq. 4-6).
+
+    ``lam``: per-head decay [H] or None (lambda = 1). ``init``: [B, H, d, d]
+    state entering token 0, or None. Returns o (float64 [B, N, H, d]) and, if
+    ``want_final``, the state after the last token as well.
+    """
+    B, N, H, d = q.shape
+    pq, sb, sn, sh = _view(q)
+    _view(k, q), _view(v, q)
+    la, pl = _lam(lam, H)
+    ia, pi = _state(init, (B, H, d, d))
+    o = np.empty((B, N, H, d), np.float64)
+    fin = np.empty((B, H, d, d), np.float64) if want_final else None
+    _load().oracle_fwd(pq, k.ctypes.data, v.ctypes.data, sb, sn, sh, pl, pi,
+                       o.ctypes.data, N * H * d, H * d, d, _ptr(fin), B, N, H, d)
+    return (o, fin) if want_final else o
+
+
+def bwd(q, k, v, do, lam=None, init=None, dstate_in=None, want_dinit=False):
+    """Gradients of sum(o * do) by the reverse recurrence (LASP Eq. 12-13).
+
+    ``dstate_in``: [B, H, d, d] gradient state entering the last token from
+    beyond the sequence end (0 if None). Returns dq, dk, dv (float64
+    [B, N, H, d]) and, if ``want_dinit``, the gradient w.r.t. ``init``.
+    """
+    B, N, H, d = q.shape
+    pq, sb, sn, sh = _view(q)
+    for t in (k, v, do):
+        _view(t, q)
+    la, pl = _lam(lam, H)
+    ia, pi = _state(init, (B, H, d, d))
+    fa, pf = _state(dstate_in, (B, H, d, d))
+    dq = np.empty((B, N, H, d), np.float64)
+    dk = np.empty_like(dq)
+    dv = np.empty_like(dq)
+    dinit = np.empty((B, H, d, d), np.float64) if want_dinit else None
+    _load().oracle_bwd(pq, k.ctypes.data, v.ctypes.data, do.ctypes.data, sb, sn, sh, pl, pi, pf,
+                       dq.ctypes.data, dk.ctypes.data, dv.ctypes.data, N * H * d, H * d, d,
+                       _ptr(dinit), B, N, H, d)
+    return (dq, dk, dv, dinit) if want_dinit else (dq, dk, dv)
+
+
+def chunk_states(a, b, lam, C, kind=0):
+    """Per-chunk states M [B, T, H, d, d] from their definition.
+
+    kind 0: M_c = sum_t lam^(C-1-t) a_t^T b_t with (a, b) = (k, v)  (LASP Eq. 10).
+    kind 1: M_c = sum_t lam^(t+1)   a_t^T b_t with (a, b) = (q, do) (LASP Eq. 20).
+    """
+    B, N, H, d = a.shape
+    if N % C:
+        raise ValueError("C must divide N")
+    pa, sb, sn, sh = _view(a)
+    _view(b, a)
+    la, pl = _lam(lam, H)
+    M = np.empty((B, N // C, H, d, d), np.float64)
+    _load().oracle_chunk_states(pa, b.ctypes.data, sb, sn, sh, pl, M.ctypes.data, B, N, H, d, C, kind)
+    return M
+
+
+def state_scan(M, lam, C, init=None, reverse=False):
+    """Exclusive decayed prefix (reverse=False) or suffix (reverse=True) scan.
+
+    prefix: P_0 = init, P_c = lam^C P_{c-1} + M_{c-1}; total = lam^C P_{T-1} + M_{T-1}
+    suffix: R_{T-1} = init, R_c = lam^C R_{c+1} + M_{c+1}; total = lam^C R_0 + M_0
+    Returns (P, total) in float64.
+    """
+    M = np.ascontiguousarray(np.asarray(M, dtype=np.float64))
+    B, T, H, d, _ = M.shape
+    la, pl = _lam(lam, H)
+    ia, pi = _state(init, (B, H, d, d))
+    P = np.empty_like(M)
+    tot = np.empty((B, H, d, d), np.float64)
+    _load().oracle_state_scan(M.ctypes.data, P.ctypes.data, pl, pi, tot.ctypes.data,
+                              B, T, H, d, C, int(bool(reverse)))
+    return P, tot
+
+
+def state_snapshots(a, b, lam, C, init=None, kind=0):
+    """Chunk-boundary states of the token recurrences, [B, T, H, d, d].
+
+    kind 0, (a, b) = (k, v): P_c = kv_{cC-1}, the state entering chunk c.
+    kind 1, (a, b) = (q, do): R_c = gradient state chunk c receives from the
+    tokens after it; ``init`` is then the gradient state entering from beyond
+    the sequence end.
+    """
+    B, N, H, d = a.shape
+    if N % C:
+        raise ValueError("C must divide N")
+    pa, sb, sn, sh = _view(a)
+    _view(b, a)
+    la, pl = _lam(lam, H)
+    ia, pi = _state(init, (B, H, d, d))
+    P = np.empty((B, N // C, H, d, d), np.float64)
+    _load().oracle_state_snapshots(pa, b.ctypes.data, sb, sn, sh, pl, pi, P.ctypes.data,
+                                   B, N, H, d, C, kind)
+    return P

@@ -1,0 +1,313 @@
+/*
+ * lasp_oracle.c -- fp64 CPU oracle for causal linear attention with a per-head
+ * decay, as LASP / LASP-2 compute it.
+ *
+ * TEST INFRASTRUCTURE. Only the tests, the smoke check and the CPU-baseline leg
+ * of the benchmark use this file. It shares no code, header, table or helper
+ * with the CUDA library, and the CUDA library never calls it.
+ *
+ * Sources (page: "Linear Attention Sequence Parallelism" (LASP), v3 full text):
+ *   - Eq. 4-6  (section 3.2, forward): kv_s = lambda*kv_{s-1} + k_s v_s^T,
+ *              o_s^T = q_s^T kv_s, kv_0 = 0.
+ *   - Eq. 12-13 (section 3.2, backward): dq_s^T = do_s^T kv_s^T,
+ *              dk_s^T = v_s^T dkv_s^T, dv_s^T = k_s^T dkv_s,
+ *              dkv_s = sum_{i>=s} lambda^{i-s} q_i do_i^T.
+ *   - Eq. 10 and Algorithm 2 (chunk state update): KV_t = lambda^C KV_{t-1}
+ *              + (diag{lambda^{C-1},...,1} K_t)^T V_t.
+ *   - Eq. 20 and Algorithm 3 (gradient state): dKV_t = lambda^C dKV_{t+1}
+ *              + (Lambda Q_t)^T dO_t with Lambda = diag{lambda,...,lambda^C}.
+ * Page "LASP-2" (pith.science review), "The reading" / "Core claim": each chunk
+ * is summarised by M_t; a prefix sum over the gathered states gives
+ * M_{1:t-1} in the forward pass, a suffix sum over dM_t in the backward pass.
+ *
+ * Conventions (0-based): per (b, h), tokens s = 0..N-1; chunk c = 0..T-1 with
+ * T = N / C; s = c*C + j.  Norm(.) is omitted as on the LASP page (section
+ * 3.2, "To streamline derivations ...").  No feature map, no 1/sqrt(d).
+ *
+ * Tensor arguments are views: a base pointer plus element strides for the
+ * batch, token and head indices (sb, sn, sh); the feature index is contiguous.
+ * Inputs are float32 (bf16- or fp32-valued data are exact in float32 and in
+ * double); all arithmetic and all outputs are double.
+ *
+ * Every function is plain loops over the definition.  Work is split across
+ * OpenMP threads by (b, h) and by blocks of state rows or columns; this only
+ * decides which thread evaluates an output element, never the order of the
+ * terms summed into it, so results are bit-identical for any thread count.
+ */
+#include <math.h>
+#include <stdlib.h>
+#include <string.h>
+
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+#define BLK 32 /* rows or columns of the d x d state owned by one task */
+
+static double lam_of(const double *lam, int h) { return lam ? lam[h] : 1.0; }
+
+static const float *tok(const float *x, long sb, long sn, long sh, int b, long n, int h) {
+  return x + (long)b * sb + n * sn + (long)h * sh;
+}
+static double *tokd(double *x, long sb, long sn, long sh, int b, long n, int h) {
+  return x + (long)b * sb + n * sn + (long)h * sh;
+}
+
+/* State arrays [B, H, d, d] (entering or leaving states) and [B, T, H, d, d]. */
+static const double *st_bh(const double *x, int H, int d, int b, int h) {
+  return x + ((long)b * H + h) * d * d;
+}
+static double *st_bh_w(double *x, int H, int d, int b, int h) {
+  return x + ((long)b * H + h) * d * d;
+}
+static long st_btc(int T, int H, int d, int b, long c, int h) {
+  return (((long)b * T + c) * H + h) * (long)d * d;
+}
+
+/*
+ * Forward recurrence, Eq. 5:  S <- lambda*S + k_s v_s^T ;  o_s = q_s S.
+ * S starts at init[b,h] (the state entering token 0) or 0.
+ * Task = (b, h, block of S columns j0..j1): column j of o only needs column j
+ * of S.  If final_state is given, it receives S after token N-1.
+ */
+void oracle_fwd(const float *q, const float *k, const float *v, long sb, long sn, long sh,
+                const double *lam, const double *init,
+                double *o, long ob, long on, long oh,
+                double *final_state, int B, long N, int H, int d) {
+  int nblk = (d + BLK - 1) / BLK;
+  long ntask = (long)B * H * nblk;
+#pragma omp parallel for schedule(dynamic, 1)
+  for (long task = 0; task < ntask; ++task) {
+    int blk = (int)(task % nblk);
+    int h = (int)((task / nblk) % H);
+    int b = (int)(task / ((long)nblk * H));
+    int j0 = blk * BLK, j1 = j0 + BLK < d ? j0 + BLK : d;
+    double l = lam_of(lam, h);
+    double *S = (double *)calloc((size_t)d * d, sizeof(double));
+    if (init) memcpy(S, st_bh(init, H, d, b, h), sizeof(double) * d * d);
+    for (long s = 0; s < N; ++s) {
+      const float *qs = tok(q, sb, sn, sh, b, s, h);
+      const float *ks = tok(k, sb, sn, sh, b, s, h);
+      const float *vs = tok(v, sb, sn, sh, b, s, h);
+      double *os = tokd(o, ob, on, oh, b, s, h);
+      for (int i = 0; i < d; ++i)
+        for (int j = j0; j < j1; ++j) S[i * d + j] = l * S[i * d + j] + (double)ks[i] * vs[j];
+      for (int j = j0; j < j1; ++j) {
+        double acc = 0.0;
+        for (int i = 0; i < d; ++i) acc += (double)qs[i] * S[i * d + j];
+        os[j] = acc;
+      }
+    }
+    if (final_state) {
+      double *F = st_bh_w(final_state, H, d, b, h);
+      for (int i = 0; i < d; ++i)
+        for (int j = j0; j < j1; ++j) F[i * d + j] = S[i * d + j];
+    }
+    free(S);
+  }
+}
+
+/*
+ * Backward recurrences, Eq. 12-13.
+ *   dq_s[i] = sum_j kv_s[i][j] do_s[j]          (forward sweep, S rows i)
+ *   dkv_s   = q_s do_s^T + lambda * dkv_{s+1}     (reverse sweep)
+ *   dk_s[i] = sum_j dkv_s[i][j] v_s[j]          (reverse sweep, G rows i)
+ *   dv_s[j] = sum_i k_s[i] dkv_s[i][j]          (reverse sweep, G columns j)
+ * The reverse sweep starts from dstate_in[b,h] (the gradient state that
+ * enters token N-1 from tokens beyond the sequence end, i.e. dkv_{N-1} =
+ * q_{N-1} do_{N-1}^T + dstate_in) or 0; init (the forward entering state)
+ * enters kv_s as in oracle_fwd.  If dinit is given it receives the gradient
+ * of sum(o * do) with respect to init: lambda * dkv_0.
+ * Tasks: (b, h, sweep, block); sweep 0 = dq (row blocks of S),
+ * 1 = dk (row blocks of G), 2 = dv and dinit (column blocks of G).
+ */
+void oracle_bwd(const float *q, const float *k, const float *v, const float *dout,
+                long sb, long sn, long sh, const double *lam, const double *init,
+                const double *dstate_in,
+                double *dq, double *dk, double *dv, long gb, long gn, long gh,
+                double *dinit, int B, long N, int H, int d) {
+  int nblk = (d + BLK - 1) / BLK;
+  long ntask = (long)B * H * 3 * nblk;
+#pragma omp parallel for schedule(dynamic, 1)
+  for (long task = 0; task < ntask; ++task) {
+    int blk = (int)(task % nblk);
+    int sweep = (int)((task / nblk) % 3);
+    int h = (int)((task / (3L * nblk)) % H);
+    int b = (int)(task / (3L * nblk * H));
+    int r0 = blk * BLK, r1 = r0 + BLK < d ? r0 + BLK : d;
+    double l = lam_of(lam, h);
+    double *S = (double *)calloc((size_t)d * d, sizeof(double));
+    if (sweep == 0) {
+      if (init) memcpy(S, st_bh(init, H, d, b, h), sizeof(double) * d * d);
+      for (long s = 0; s < N; ++s) {
+        const float *ks = tok(k, sb, sn, sh, b, s, h);
+        const float *vs = tok(v, sb, sn, sh, b, s, h);
+        const float *ds = tok(dout, sb, sn, sh, b, s, h);
+        double *dqs = tokd(dq, gb, gn, gh, b, s, h);
+        for (int i = r0; i < r1; ++i) {
+          double acc = 0.0;
+          for (int j = 0; j < d; ++j) {
+            S[i * d + j] = l * S[i * d + j] + (double)ks[i] * vs[j];
+            acc += S[i * d + j] * ds[j];
+          }
+          dqs[i] = acc;
+        }
+      }
+    } else {
+      double *G = S; /* dkv, exclusive of the current token until it is added */
+      if (dstate_in) memcpy(G, st_bh(dstate_in, H, d, b, h), sizeof(double) * d * d);
+      for (long s = N - 1; s >= 0; --s) {
+        const float *qs = tok(q, sb, sn, sh, b, s, h);
+        const float *ks = tok(k, sb, sn, sh, b, s, h);
+        const float *vs = tok(v, sb, sn, sh, b, s, h);
+        const float *ds = tok(dout, sb, sn, sh, b, s, h);
+        if (sweep == 1) {
+          double *dks = tokd(dk, gb, gn, gh, b, s, h);
+          for (int i = r0; i < r1; ++i) {
+            double acc = 0.0;
+            for (int j = 0; j < d; ++j) {
+              G[i * d + j] += (double)qs[i] * ds[j];
+              acc += G[i * d + j] * vs[j];
+            }
+            dks[i] = acc;
+            for (int j = 0; j < d; ++j) G[i * d + j] *= l;
+          }
+        } else {
+          double *dvs = tokd(dv, gb, gn, gh, b, s, h);
+          for (int i = 0; i < d; ++i)
+            for (int j = r0; j < r1; ++j) G[i * d + j] += (double)qs[i] * ds[j];
+          for (int j = r0; j < r1; ++j) {
+            double acc = 0.0;
+            for (int i = 0; i < d; ++i) acc += (double)ks[i] * G[i * d + j];
+            dvs[j] = acc;
+          }
+          for (int i = 0; i < d; ++i)
+            for (int j = r0; j < r1; ++j) G[i * d + j] *= l;
+        }
+      }
+      if (sweep == 2 && dinit) {
+        double *D = st_bh_w(dinit, H, d, b, h);
+        for (int i = 0; i < d; ++i)
+          for (int j = r0; j < r1; ++j) D[i * d + j] = G[i * d + j];
+      }
+    }
+    free(S);
+  }
+}
+
+/*
+ * Per-chunk states, written out from their definition.
+ *   kind 0 (forward memory state, Eq. 10 / Algorithm 2):
+ *       M_c[i][j] = sum_{t=0}^{C-1} lambda^{C-1-t} a_{cC+t}[i] b_{cC+t}[j]
+ *       with (a, b) = (k, v).
+ *   kind 1 (gradient state, Eq. 20 / Algorithm 3, term (Lambda Q_t)^T dO_t):
+ *       M_c[i][j] = sum_{t=0}^{C-1} lambda^{t+1} a_{cC+t}[i] b_{cC+t}[j]
+ *       with (a, b) = (q, do).
+ * M is [B, T, H, d, d], T = N / C (the caller guarantees C divides N).
+ */
+void oracle_chunk_states(const float *a, const float *bm, long sb, long sn, long sh,
+                         const double *lam, double *M, int B, long N, int H, int d,
+                         long C, int kind) {
+  long T = N / C;
+  long ntask = (long)B * T * H;
+#pragma omp parallel for schedule(dynamic, 1)
+  for (long task = 0; task < ntask; ++task) {
+    int h = (int)(task % H);
+    long c = (task / H) % T;
+    int b = (int)(task / ((long)H * T));
+    double l = lam_of(lam, h);
+    double *Mc = M + st_btc((int)T, H, d, b, c, h);
+    for (long e = 0; e < (long)d * d; ++e) Mc[e] = 0.0;
+    for (long t = 0; t < C; ++t) {
+      double w = kind == 0 ? pow(l, (double)(C - 1 - t)) : pow(l, (double)(t + 1));
+      const float *as = tok(a, sb, sn, sh, b, c * C + t, h);
+      const float *bs = tok(bm, sb, sn, sh, b, c * C + t, h);
+      for (int i = 0; i < d; ++i)
+        for (int j = 0; j < d; ++j) Mc[i * d + j] += w * (double)as[i] * bs[j];
+    }
+  }
+}
+
+/*
+ * Decayed scans over chunk states (LASP-2: prefix sum of the gathered M_t in
+ * the forward pass, suffix sum of dM_t in the backward pass; LASP Eq. 10 and
+ * Eq. 20 give the decay lambda^C per chunk).
+ *   reverse = 0:  P_0 = init (or 0);      P_c = lambda^C P_{c-1} + M_{c-1};
+ *                 total = lambda^C P_{T-1} + M_{T-1}.
+ *   reverse = 1:  R_{T-1} = init (or 0);  R_c = lambda^C R_{c+1} + M_{c+1};
+ *                 total = lambda^C R_0 + M_0.
+ * M and P are [B, T, H, d, d]; init and total are [B, H, d, d].
+ */
+void oracle_state_scan(const double *M, double *P, const double *lam, const double *init,
+                       double *total, int B, long T, int H, int d, long C, int reverse) {
+  long ntask = (long)B * H;
+#pragma omp parallel for schedule(dynamic, 1)
+  for (long task = 0; task < ntask; ++task) {
+    int h = (int)(task % H);
+    int b = (int)(task / H);
+    double g = pow(lam_of(lam, h), (double)C);
+    double *acc = (double *)calloc((size_t)d * d, sizeof(double));
+    if (init) memcpy(acc, st_bh(init, H, d, b, h), sizeof(double) * d * d);
+    for (long n = 0; n < T; ++n) {
+      long c = reverse ? T - 1 - n : n;
+      const double *Mc = M + st_btc((int)T, H, d, b, c, h);
+      double *Pc = P + st_btc((int)T, H, d, b, c, h);
+      for (long e = 0; e < (long)d * d; ++e) Pc[e] = acc[e];
+      for (long e = 0; e < (long)d * d; ++e) acc[e] = g * acc[e] + Mc[e];
+    }
+    if (total) memcpy(st_bh_w(total, H, d, b, h), acc, sizeof(double) * d * d);
+    free(acc);
+  }
+}
+
+/*
+ * State snapshots from the token recurrences (the state the pages cache for
+ * the backward pass, "KV state caching", section 3.4):
+ *   kind 0:  P_c = kv_{cC-1}, the forward state after the last token before
+ *            chunk c (P_0 = init or 0), run token by token with Eq. 5.
+ *   kind 1:  R_c = sum_{s >= (c+1)C} lambda^{s-(c+1)C+1} q_s do_s^T
+ *            + lambda^{N-(c+1)C} dstate_in, the gradient state that chunk c
+ *            receives from the tokens after it, run token by token with Eq. 13.
+ * (a, b) = (k, v) for kind 0 and (q, do) for kind 1; P is [B, T, H, d, d].
+ */
+void oracle_state_snapshots(const float *a, const float *bm, long sb, long sn, long sh,
+                            const double *lam, const double *init, double *P,
+                            int B, long N, int H, int d, long C, int kind) {
+  long T = N / C;
+  long ntask = (long)B * H;
+#pragma omp parallel for schedule(dynamic, 1)
+  for (long task = 0; task < ntask; ++task) {
+    int h = (int)(task % H);
+    int b = (int)(task / H);
+    double l = lam_of(lam, h);
+    double *S = (double *)calloc((size_t)d * d, sizeof(double));
+    if (init) memcpy(S, st_bh(init, H, d, b, h), sizeof(double) * d * d);
+    if (kind == 0) {
+      for (long s = 0; s < N; ++s) {
+        if (s % C == 0) memcpy(P + st_btc((int)T, H, d, b, s / C, h), S, sizeof(double) * d * d);
+        const float *as = tok(a, sb, sn, sh, b, s, h);
+        const float *bs = tok(bm, sb, sn, sh, b, s, h);
+        for (int i = 0; i < d; ++i)
+          for (int j = 0; j < d; ++j) S[i * d + j] = l * S[i * d + j] + (double)as[i] * bs[j];
+      }
+    } else {
+      /* S holds the exclusive suffix state at token s (terms from tokens > s). */
+      for (long s = N - 1; s >= 0; --s) {
+        if (s % C == C - 1) memcpy(P + st_btc((int)T, H, d, b, s / C, h), S, sizeof(double) * d * d);
+        const float *as = tok(a, sb, sn, sh, b, s, h);
+        const float *bs = tok(bm, sb, sn, sh, b, s, h);
+        for (int i = 0; i < d; ++i)
+          for (int j = 0; j < d; ++j) S[i * d + j] = l * (S[i * d + j] + (double)as[i] * bs[j]);
+      }
+    }
+    free(S);
+  }
+}
+
+int oracle_num_threads(void) {
+#ifdef _OPENMP
+  return omp_get_max_threads();
+#else
+  return 1;
+#endif
+}
