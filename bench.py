@@ -1,0 +1,387 @@
+"""Benchmark: chunked causal linear attention forward + backward on B200.
+
+One step = one pass of the whole hot path over one batch of synthetic input:
+chunk states, exclusive prefix, output (the forward pass), gradient states,
+exclusive suffix, dQ/dK/dV (the backward pass). The step issues these six
+library calls on one stream -- the same kernels lasp_fwd and lasp_bwd issue --
+with CUDA events between them, so each kernel's duration is measured live.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload NAME]
+
+Prints one JSON line (rank 0). With N > 1 (launched by torch.distributed.run)
+every rank runs the same workload on its own GPU with no data exchange
+(independent sequences: weak scaling); the step time is the max over ranks.
+`--impl reference` times the fp64 CPU oracle on the host cores instead.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from sequence_linear_attention_b200 import inputs as lasp_inputs  # noqa: E402
+
+METRIC = "linear-attn fwd+bwd tokens/s (H16 d128 N64K bf16); % of bf16 tensor peak"
+DEFAULT_WORKLOAD = "decayed_bf16_N64K"
+KERNELS = ("chunk_states", "state_prefix", "chunk_out", "chunk_dstates", "state_suffix", "chunk_grads")
+
+
+# ------------------------------------------------------------ algorithmic work
+def algorithmic_bytes(name: str, tokens_heads: int, d: int, C: int, elem: int) -> float:
+    """Bytes each kernel must move, per launch: token tensors once, states once.
+
+    Per token-head, with e = element size and s = d*d*4/C (one fp32 state per
+    chunk spread over its C tokens):
+      chunk_states / chunk_dstates: read 2 token rows, write one state  = 2de + s
+      state_prefix / state_suffix:  read and write one state            = 2s
+      chunk_out:   read q, k, v and P, write o                         = 4de + s
+      chunk_grads: read q, k, v, dO, P and R, write dq, dk, dv          = 7de + 2s
+    """
+    s = d * d * 4 / C
+    per = {"chunk_states": 2 * d * elem + s, "chunk_dstates": 2 * d * elem + s,
+           "state_prefix": 2 * s, "state_suffix": 2 * s,
+           "chunk_out": 4 * d * elem + s, "chunk_grads": 7 * d * elem + 2 * s}[name]
+    return per * tokens_heads
+
+
+def flops_per_step(tokens_heads: int, d: int, C: int) -> float:
+    """fwd 2(2Cd + 2d^2) and bwd 2(5Cd + 4d^2) FLOPs per token-head."""
+    return tokens_heads * (2 * (2 * C * d + 2 * d * d) + 2 * (5 * C * d + 4 * d * d))
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            j = json.load(f)
+        return dict(hbm=float(j["hbm_gbs"]), bf16=float(j["bf16_tflops"]),
+                    bf16_sustained=float(j.get("bf16_tflops_sustained", j["bf16_tflops"])), source="measured")
+    except Exception:
+        return dict(hbm=6650.0, bf16=1590.0, bf16_sustained=1400.0, source="fallback")
+
+
+# ---------------------------------------------------------------- distributed
+def dist_setup():
+    """(rank, world, local_rank). Initialises torch.distributed when WORLD_SIZE > 1."""
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        backend = os.environ.get("LASP_BENCH_BACKEND", "nccl")
+        dist.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=120))
+    return rank, world, local
+
+
+def max_over_ranks(x: float, world: int, device=None) -> float:
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world: int, device=None):
+    if world > 1:
+        import torch.distributed as dist
+        if device is not None and dist.get_backend() == "nccl":
+            dist.barrier(device_ids=[device.index])
+        else:
+            dist.barrier()
+
+
+def aggregate(units_per_rank: float, seconds_per_rank: float, world: int, device=None) -> tuple[float, float]:
+    """Whole-job throughput: all ranks' units over the slowest rank's time."""
+    t = max_over_ranks(seconds_per_rank, world, device)
+    return units_per_rank * world / t, t
+
+
+# ---------------------------------------------------------------------- clocks
+class ClockSampler:
+    """Samples SM clocks and throttle reasons with nvidia-smi while running."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.idx = gpu_index
+        self.proc = None
+        self.out = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.idx), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            time.sleep(0.25)
+            self.proc.terminate()
+            try:
+                self.out, _ = self.proc.communicate(timeout=5)
+            except Exception:
+                self.proc.kill()
+                self.out = ""
+
+    def summary(self):
+        if not self.out:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"]}
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.out.strip().splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax = float(parts[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": smax, "reasons": sorted(reasons)}
+        loaded = [x for x in sm if smax and x > 0.5 * smax] or sm
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": smax, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ GPU arm
+def run_gpu(args, rank, world, local):
+    import torch
+    import sequence_linear_attention_b200 as lasp
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    w = lasp_inputs.WORKLOADS[args.workload]
+    B, N, H, d, C = w["B"], w["N"], w["H"], w["d"], w["C"]
+    bf16 = w["bf16"]
+    tdtype = torch.bfloat16 if bf16 else torch.float32
+    elem = 2 if bf16 else 4
+    T = N // C
+    inp = lasp_inputs.make_inputs(B, N, H, d, seed=w["seed"] + 7919 * rank, bf16=bf16, decayed=w["decayed"])
+
+    def host_tensor(x):
+        if bf16:
+            return torch.from_numpy(np.ascontiguousarray(x).view(np.int16)).view(torch.bfloat16)
+        return torch.from_numpy(np.ascontiguousarray(x, dtype=np.float32))
+
+    host = {n: host_tensor(inp[n]).pin_memory() for n in ("q", "k", "v", "do")}
+    dv_ = {n: host[n].to(dev) for n in host}
+    q, k, v, do = dv_["q"], dv_["k"], dv_["v"], dv_["do"]
+    decay = None if inp["lam"] is None else torch.from_numpy(inp["lam"]).to(dev)
+    o, dq, dk, dvv = (torch.empty_like(q) for _ in range(4))
+    P = torch.empty((B, T, H, d, d), dtype=torch.float32, device=dev)
+    R = torch.empty_like(P)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(evs=None):
+        def mark(i):
+            if evs is not None:
+                evs[i].record(stream)
+        mark(0)
+        lasp.lasp_chunk_states(None, k, v, decay, P, C)
+        mark(1)
+        lasp.lasp_state_prefix(P, P, decay, C)
+        mark(2)
+        lasp.lasp_chunk_out(q, k, v, decay, P, o, C)
+        mark(3)
+        lasp.lasp_chunk_dstates(q, do, decay, R, C)
+        mark(4)
+        lasp.lasp_state_prefix(R, R, decay, C, reverse=True)
+        mark(5)
+        lasp.lasp_chunk_grads(q, k, v, do, decay, P, R, dq, dk, dvv, C)
+        mark(6)
+
+    for _ in range(args.warmup):
+        step()
+    st, site = lasp.lasp_check_device_status()
+    if st != 0:
+        raise RuntimeError(f"device status {lasp.lasp_status_string(st)} at site {site}")
+
+    events = [[torch.cuda.Event(enable_timing=True) for _ in range(7)] for _ in range(args.steps)]
+    torch.cuda.synchronize(dev)
+    barrier(world, dev)
+    torch.cuda.synchronize(dev)
+    with ClockSampler(local) as clk:
+        for i in range(args.steps):
+            step(events[i])
+        torch.cuda.synchronize(dev)
+    barrier(world, dev)
+    torch.cuda.synchronize(dev)
+    per_kernel = {n: [] for n in KERNELS}
+    total_ms = 0.0
+    for evs in events:
+        total_ms += evs[0].elapsed_time(evs[6])
+        for j, n in enumerate(KERNELS):
+            per_kernel[n].append(evs[j].elapsed_time(evs[j + 1]))
+    tokens = B * N
+    value, t_max = aggregate(tokens * args.steps, total_ms / 1e3, world, dev)
+    ms_per_step = t_max * 1e3 / args.steps
+
+    # end to end through the public API: pinned host -> device, fwd, bwd, device -> host
+    outs_host = {n: torch.empty_like(host["q"]).pin_memory() for n in ("o", "dq", "dk", "dv")}
+    e2e_steps = max(1, min(args.steps, 5))
+
+    def e2e_step():
+        for n in ("q", "k", "v", "do"):
+            dv_[n].copy_(host[n], non_blocking=True)
+        lasp.lasp_fwd(q, k, v, decay, o, C, P)
+        lasp.lasp_bwd(q, k, v, decay, do, dq, dk, dvv, C, P, R)
+        for n, t in (("o", o), ("dq", dq), ("dk", dk), ("dv", dvv)):
+            outs_host[n].copy_(t, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize(dev)
+    barrier(world, dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_value, _ = aggregate(tokens * e2e_steps, e0.elapsed_time(e1) / 1e3, world, dev)
+    st, site = lasp.lasp_check_device_status()
+    if st != 0:
+        raise RuntimeError(f"device status {lasp.lasp_status_string(st)} at site {site}")
+
+    peaks = load_peaks()
+    th = tokens * H
+    avg = {n: statistics.mean(per_kernel[n]) for n in KERNELS}
+    top = max(KERNELS, key=lambda n: avg[n])
+    achieved = algorithmic_bytes(top, th, d, C, elem) / (avg[top] / 1e3) / 1e9
+    kernel_table = {n: {"ms": round(avg[n], 4),
+                        "GBps": round(algorithmic_bytes(n, th, d, C, elem) / (avg[n] / 1e3) / 1e9, 1),
+                        "hbm_frac": round(algorithmic_bytes(n, th, d, C, elem) / (avg[n] / 1e3) / 1e9
+                                          / peaks["hbm"], 4)} for n in KERNELS}
+    flops = flops_per_step(th, d, C)
+    tflops = flops / (ms_per_step / 1e3) / 1e12
+    line = {
+        "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16" if bf16 else "f32", "data": "synthetic (seeded normal q,k,v,dO; no dataset)",
+        "config": {"workload": args.workload, "B": B, "H": H, "N": N, "d": d, "C": C,
+                   "decay": "per-head 1-2^-(5+8h/H)" if w["decayed"] else "none",
+                   "l2": "inputs larger than L2 (q, k, v, dO are 4 x %d MiB)" % (B * N * H * d * elem >> 20),
+                   "parallelism": f"replicas x{world} (independent sequences, no collective)"},
+        "tflops": round(tflops, 2),
+        "tensor_peak_frac": round(tflops / peaks["bf16_sustained"], 4),
+        "roofline": {"bound": "hbm", "kernel": top, "achieved": round(achieved, 1), "peak": peaks["hbm"],
+                     "unit": "GB/s", "frac": round(achieved / peaks["hbm"], 4), "traffic": None,
+                     "peak_source": peaks["source"]},
+        "kernels": kernel_table,
+        "e2e": {"value": round(e2e_value, 1), "unit": "tokens/s",
+                "h2d_bytes_per_step": 4 * B * N * H * d * elem, "d2h_bytes_per_step": 4 * B * N * H * d * elem,
+                "api": "lasp_fwd + lasp_bwd with pinned host buffers"},
+        "gpu_launches": 6 * args.steps,
+        "clocks": clk.summary(),
+    }
+    return line
+
+
+# ------------------------------------------------------------------ CPU oracle
+def oracle_sample(args, tokens: int):
+    """A bounded sample of the workload for the fp64 oracle: all heads, the
+    first `tokens` positions of batch 0 (per-token work does not depend on N)."""
+    w = lasp_inputs.WORKLOADS[args.workload]
+    inp = lasp_inputs.make_inputs(1, tokens, w["H"], w["d"], seed=w["seed"], bf16=w["bf16"], decayed=w["decayed"])
+    return [lasp_inputs.as_f32(inp[n], w["bf16"]) for n in ("q", "k", "v", "do")] + [inp["lam"]]
+
+
+def time_oracle(args, tokens: int, reps: int = 1):
+    import oracle
+    q, k, v, do, lam = oracle_sample(args, tokens)
+    oracle.build()
+    t0 = time.perf_counter()
+    for _ in range(reps):
+        oracle.fwd(q, k, v, lam)
+        oracle.bwd(q, k, v, do, lam)
+    return tokens * reps / (time.perf_counter() - t0), oracle.num_threads()
+
+
+def cpu_baseline(args):
+    # about 10-30 s of host work: all heads over 32768 positions of the workload
+    tokens = 32768
+    value, cores = time_oracle(args, tokens)
+    return {"value": round(value, 1), "unit": "tokens/s", "cores": cores, "kind": "oracle",
+            "sample": f"fp64 oracle fwd+bwd, batch 0, all heads, first {tokens} positions"}
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return None
+    tokens = 2048
+    import oracle
+    q, k, v, do, lam = oracle_sample(args, tokens)
+    oracle.build()
+    for _ in range(args.warmup):
+        oracle.fwd(q, k, v, lam)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle.fwd(q, k, v, lam)
+        oracle.bwd(q, k, v, do, lam)
+    dt = time.perf_counter() - t0
+    value = tokens * args.steps / dt
+    w = lasp_inputs.WORKLOADS[args.workload]
+    sample = f"fp64 oracle fwd+bwd, batch 0, all heads, first {tokens} positions per step"
+    return {
+        "impl": "reference", "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(dt * 1e3 / args.steps, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": {"workload": args.workload, "B": w["B"], "H": w["H"], "N": w["N"],
+                                         "d": w["d"], "C": w["C"]},
+        "cpu_baseline": {"value": round(value, 1), "unit": "tokens/s", "kind": "oracle",
+                         "cores": __import__("oracle").num_threads(), "sample": sample},
+        "e2e": {"value": round(value, 1), "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(lasp_inputs.WORKLOADS))
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    rank, world, local = dist_setup()
+    try:
+        if args.impl == "reference":
+            line = run_reference(args, rank, world)
+        else:
+            line = run_gpu(args, rank, world, local)
+            if rank == 0 and world == 1 and not args.no_cpu_baseline:
+                line["cpu_baseline"] = cpu_baseline(args)
+        if rank == 0 and line is not None:
+            print(json.dumps(line), flush=True)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,220 @@
+/*
+ * lasp.h -- C ABI of the B200 library for chunked causal linear attention
+ * with a per-head decay: the single-GPU hot path of LASP / LASP-2.
+ *
+ * What is computed (page "Linear Attention Sequence Parallelism" (LASP), v3,
+ * section 3.2; page "LASP-2" (pith.science review), "The reading"):
+ * for every batch b and head h, tokens s = 0..N-1,
+ *     kv_s = lambda_h kv_{s-1} + k_s^T v_s        (LASP Eq. 5-6, kv_{-1} = init)
+ *     o_s  = q_s kv_s                              (LASP Eq. 4-5)
+ * and the gradients of sum(o * dO) (LASP Eq. 12-13). Norm(.) after attention
+ * is not applied (LASP section 3.2 omits it in the derivation); there is no
+ * feature map and no 1/sqrt(d) scale.
+ *
+ * The sequence is cut into chunks of C tokens (LASP Algorithm 1, C = N/T);
+ * chunk c (0-based) holds tokens c*C .. c*C+C-1.
+ *
+ * Layouts (all row-major, C order):
+ *   token tensors q, k, v, o, dout, dq, dk, dv:  [B, N, H, d]
+ *       element type: float (LASP_F32) or bfloat16 (LASP_BF16), the same for all.
+ *   state arrays (always float32):  [B, T, H, d, d], T = N / C, or [B, H, d, d]
+ *       for a single state per (b, h); element [i][j] pairs key/query feature i
+ *       with value/output feature j, e.g. M_c[i][j] = sum_t w_t k_t[i] v_t[j].
+ *   decay: float[H], lambda_h in (0, 1], or NULL for lambda = 1 (ordinary
+ *       linear attention, LASP section 3.2). NULL and an all-ones array give
+ *       bit-identical results.
+ *
+ * Pointers: every pointer is a DEVICE pointer owned by the caller; the library
+ * never allocates, frees or keeps a pointer after the call returns. All
+ * tensors must be 16-byte aligned and must not overlap unless stated.
+ *
+ * Execution: every compute call is asynchronous and stream-ordered on
+ * `stream` (a cudaStream_t; NULL = the legacy default stream). Arguments are
+ * validated on the host before anything is launched; a non-zero status means
+ * nothing was launched. Conditions only the device can see (a decay value
+ * outside (0, 1], a wait that exceeded its time limit) are recorded in a
+ * per-device status word read by lasp_check_device_status().
+ *
+ * Supported sizes: B, H >= 1; N >= 0 (N = 0 launches nothing); d in
+ * {32, 64, 128}; 1 <= C, C divides N. Larger T * H * d * d products are limited
+ * only by device memory.
+ */
+#ifndef LASP_H
+#define LASP_H
+
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define LASP_API __attribute__((visibility("default")))
+#else
+#define LASP_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  LASP_OK = 0,
+  LASP_ERR_INVALID_ARG = 1, /* bad size, NULL required pointer, bad dtype */
+  LASP_ERR_UNSUPPORTED = 2, /* a size this build has no kernel for (e.g. d = 96) */
+  LASP_ERR_MISALIGNED = 3,  /* a pointer not 16-byte aligned */
+  LASP_ERR_CUDA = 4,        /* a CUDA runtime error (launch failure, no device) */
+  LASP_ERR_TIMEOUT = 5      /* a device-side wait exceeded its limit */
+} lasp_status;
+
+typedef enum { LASP_F32 = 0, LASP_BF16 = 1 } lasp_dtype;
+
+/*
+ * lasp_fwd -- forward pass (LASP Algorithm 2; LASP-2 "The reading": chunk
+ * states, prefix over chunk states, intra + inter output).
+ *   o[b, s, h, :] = q_s kv_s, with kv_{-1} = init_state[b, h] (or 0).
+ * Steps (each a kernel): chunk states M_c = sum_j lambda^{C-1-j} k_j^T v_j
+ * (LASP Eq. 10) into state_cache; exclusive decayed prefix over chunks in
+ * place, P_c = lambda^C P_{c-1} + M_{c-1}, P_0 = init (LASP-2 prefix sum);
+ * output O_c = [(Q_c K_c^T) . Mask] V_c + Lambda Q_c P_c (LASP Eq. 7, 9, 11).
+ *   q, k, v:      in,  [B, N, H, d] of `dtype`.
+ *   decay:        in,  float[H] or NULL.
+ *   o:            out, [B, N, H, d] of `dtype`.
+ *   state_cache:  out, float [B, N/C, H, d, d]; receives P_c, the state that
+ *                 enters chunk c (LASP section 3.4 "KV State Caching"), which
+ *                 lasp_bwd reads. Required.
+ *   init_state:   in,  float [B, H, d, d] or NULL: the state entering token 0
+ *                 (the prefix of the shards before this one in the LASP-2
+ *                 decomposition).
+ */
+LASP_API int lasp_fwd(const void* q, const void* k, const void* v, const float* decay, void* o,
+             int B, int H, int64_t N, int d, int C, int dtype,
+             float* state_cache, const float* init_state, void* stream);
+
+/*
+ * lasp_bwd -- backward pass (LASP Algorithm 3; LASP-2 suffix sum of dM_t).
+ * Gradients of sum(o * dout) with respect to q, k, v.
+ * Steps: gradient chunk states dM_c = sum_j lambda^{j+1} q_j^T do_j
+ * (LASP Eq. 20 term (Lambda Q_t)^T dO_t) into dstate_ws; exclusive decayed
+ * suffix in place, R_c = lambda^C R_{c+1} + dM_{c+1}, R_{T-1} = dstate_in;
+ * then dQ, dK, dV per chunk:
+ *   dQ_c = [(dO_c V_c^T) . Mask] K_c + Lambda dO_c P_c^T         (Eq. 14, 16)
+ *   dK_c = [(dO_c V_c^T) . Mask]^T Q_c + lambda^C Lambda^-1 V_c R_c^T (Eq. 17, 19)
+ *   dV_c = [(Q_c K_c^T) . Mask]^T dO_c + lambda^C Lambda^-1 K_c R_c   (Eq. 22, 23)
+ *   q, k, v, dout:  in,  [B, N, H, d] of `dtype`.
+ *   dq, dk, dv:     out, [B, N, H, d] of `dtype`.
+ *   state_cache:    in,  the P array lasp_fwd wrote for the same q, k, v,
+ *                   decay, C and init_state. Required.
+ *   dstate_ws:      out, float [B, N/C, H, d, d]; receives R_c, the gradient
+ *                   state chunk c receives from the tokens after it. Required.
+ *   init_state:     in,  as given to lasp_fwd (only its effect through
+ *                   state_cache matters; may be NULL).
+ *   dstate_in:      in,  float [B, H, d, d] or NULL: gradient state entering the
+ *                   last token from tokens after the sequence (LASP-2 suffix of
+ *                   the later shards).
+ *   dinit_state:    out, float [B, H, d, d] or NULL: gradient of the loss with
+ *                   respect to init_state, lambda^C R_0 + dM_0 (the dstate_in of
+ *                   the previous shard).
+ */
+LASP_API int lasp_bwd(const void* q, const void* k, const void* v, const float* decay, const void* dout,
+             void* dq, void* dk, void* dv, int B, int H, int64_t N, int d, int C, int dtype,
+             const float* state_cache, float* dstate_ws, const float* init_state,
+             const float* dstate_in, float* dinit_state, void* stream);
+
+/*
+ * lasp_chunk_states -- per-chunk memory states (LASP Eq. 10, Algorithm 2 step
+ * 16 with KV_{t-1} = 0; LASP-2 "The reading": M_t summarises chunk t):
+ *   M[b, c, h][i][j] = sum_{j'=0}^{C-1} lambda_h^{C-1-j'} k_{cC+j'}[i] v_{cC+j'}[j].
+ *   q:  unused, may be NULL (kept so the call mirrors lasp_fwd).
+ *   k, v:  in, [B, N, H, d] of `dtype`.   M: out, float [B, N/C, H, d, d].
+ * C may be as large as N (one state per sequence: the LASP-2 shard state).
+ */
+LASP_API int lasp_chunk_states(const void* q, const void* k, const void* v, const float* decay, float* M,
+                      int B, int H, int64_t N, int d, int C, int dtype, void* stream);
+
+/*
+ * lasp_chunk_dstates -- per-chunk gradient states (LASP Eq. 20, Algorithm 3
+ * step 18 with dKV_{t+1} = 0):
+ *   dM[b, c, h][i][j] = sum_{j'=0}^{C-1} lambda_h^{j'+1} q_{cC+j'}[i] do_{cC+j'}[j].
+ *   q, dout: in, [B, N, H, d] of `dtype`.   dM: out, float [B, N/C, H, d, d].
+ */
+LASP_API int lasp_chunk_dstates(const void* q, const void* dout, const float* decay, float* dM,
+                       int B, int H, int64_t N, int d, int C, int dtype, void* stream);
+
+/*
+ * lasp_state_prefix -- exclusive decayed scan over chunk states (LASP-2:
+ * prefix sum of the gathered M_t in the forward pass, suffix sum of dM_t in
+ * the backward pass; LASP Eq. 10 / Eq. 20 give the per-chunk decay lambda^C).
+ *   reverse = 0:  P_0 = init; P_c = lambda^C P_{c-1} + M_{c-1};
+ *                 total = lambda^C P_{T-1} + M_{T-1}  (state after the last chunk)
+ *   reverse = 1:  R_{T-1} = init; R_c = lambda^C R_{c+1} + M_{c+1};
+ *                 total = lambda^C R_0 + M_0
+ *   M:        in,  float [B, T, H, d, d].
+ *   Mprefix:  out, float [B, T, H, d, d]; may be the same pointer as M (in place).
+ *   init:     in,  float [B, H, d, d] or NULL (zero).
+ *   total:    out, float [B, H, d, d] or NULL.
+ *   C:        chunk length in tokens, >= 1 (the decay step is lambda^C).
+ */
+LASP_API int lasp_state_prefix(const float* M, float* Mprefix, const float* decay, const float* init,
+                      float* total, int B, int T, int H, int d, int64_t C, int reverse,
+                      void* stream);
+
+/*
+ * lasp_chunk_out -- the output step of lasp_fwd on its own (LASP Eq. 7, 9, 11;
+ * Algorithm 2 steps 9, 14, 15), given the chunk-entering states P:
+ *   O_c[j] = sum_{i<=j} lambda^{j-i} (q_j . k_i) v_i + lambda^{j+1} q_j P_c.
+ *   q, k, v: in, [B, N, H, d] of `dtype`.   P: in, float [B, N/C, H, d, d].
+ *   o: out, [B, N, H, d] of `dtype`.
+ * lasp_fwd = lasp_chunk_states, lasp_state_prefix (in place), lasp_chunk_out.
+ */
+LASP_API int lasp_chunk_out(const void* q, const void* k, const void* v, const float* decay, const float* P,
+                            void* o, int B, int H, int64_t N, int d, int C, int dtype, void* stream);
+
+/*
+ * lasp_chunk_grads -- the dQ/dK/dV step of lasp_bwd on its own (LASP Eq. 14,
+ * 16, 17, 19, 22, 23; Algorithm 3 steps 7-17), given the chunk-entering
+ * states P (from the forward pass) and the gradient states R:
+ *   dQ_c[j] = sum_{i<=j} lambda^{j-i} (do_j . v_i) k_i + lambda^{j+1} do_j P_c^T
+ *   dK_c[j] = sum_{i>=j} lambda^{i-j} (do_i . v_j) q_i + lambda^{C-1-j} v_j R_c^T
+ *   dV_c[j] = sum_{i>=j} lambda^{i-j} (q_i . k_j) do_i + lambda^{C-1-j} k_j R_c
+ *   q, k, v, dout: in, [B, N, H, d]; P, R: in, float [B, N/C, H, d, d];
+ *   dq, dk, dv: out, [B, N, H, d], all of `dtype`.
+ * lasp_bwd = lasp_chunk_dstates, lasp_state_prefix (reverse, in place),
+ * lasp_chunk_grads.
+ */
+LASP_API int lasp_chunk_grads(const void* q, const void* k, const void* v, const void* dout, const float* decay,
+                              const float* P, const float* R, void* dq, void* dk, void* dv, int B, int H,
+                              int64_t N, int d, int C, int dtype, void* stream);
+
+/*
+ * lasp_check_device_status -- synchronizes `stream`, then returns and clears
+ * the first error any kernel of this library recorded on the current device
+ * (LASP_OK if none; LASP_ERR_TIMEOUT for a wait that ran out;
+ * LASP_ERR_INVALID_ARG for a decay outside (0, 1]; LASP_ERR_CUDA if the
+ * synchronization itself failed). `site` (may be NULL) receives the code of
+ * the place that recorded it.
+ */
+LASP_API int lasp_check_device_status(void* stream, int* site);
+
+/* Human-readable name of a status code (static storage). */
+LASP_API const char* lasp_status_string(int status);
+
+/*
+ * lasp_set_wait_limit_ns -- sets, for the current device, the time after which
+ * a spin-wait inside a kernel gives up, records LASP_ERR_TIMEOUT and lets the
+ * kernel return (default 2e9 ns). Synchronous. Used by tests.
+ */
+LASP_API int lasp_set_wait_limit_ns(uint64_t limit_ns);
+
+/*
+ * lasp_wait_probe -- launches one CTA that waits on a barrier nothing arrives
+ * on, with the current wait limit, then returns. Lets tests check, without a
+ * fault, that a wait that runs out ends with LASP_ERR_TIMEOUT in the status
+ * word. Asynchronous on `stream`.
+ */
+LASP_API int lasp_wait_probe(void* stream);
+
+/* Library version, major * 10000 + minor * 100 + patch. */
+LASP_API int lasp_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LASP_H */

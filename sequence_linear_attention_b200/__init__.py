@@ -1,0 +1,199 @@
+"""B200 chunked causal linear attention (the LASP / LASP-2 hot path).
+
+A thin ctypes binding over ``liblasp.so``, whose C ABI is declared in
+``include/lasp.h``. Every function here has the name of its C entry point and
+only marshals arguments: torch tensors supply device pointers and sizes, the
+current CUDA stream is passed along, and a non-zero status raises
+:class:`LaspError`. All arithmetic runs in the library's CUDA kernels; there is
+no CPU path. If the library has not been built, the first call raises.
+
+Token tensors are contiguous [B, N, H, d] (float32 or bfloat16, all the same);
+state arrays are contiguous float32 [B, N/C, H, d, d] or [B, H, d, d]; decay is
+a float32 [H] device tensor or None (lambda = 1).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+__all__ = [
+    "LaspError", "library_path", "lasp_fwd", "lasp_bwd", "lasp_chunk_states", "lasp_chunk_dstates",
+    "lasp_chunk_out", "lasp_chunk_grads",
+    "lasp_state_prefix", "lasp_check_device_status", "lasp_set_wait_limit_ns", "lasp_wait_probe",
+    "lasp_status_string", "lasp_version",
+]
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_LIB_PATH = os.path.join(_HERE, "liblasp.so")
+_lib = None
+_lock = threading.Lock()
+
+LASP_F32, LASP_BF16 = 0, 1
+_STATUS = ["LASP_OK", "LASP_ERR_INVALID_ARG", "LASP_ERR_UNSUPPORTED", "LASP_ERR_MISALIGNED",
+           "LASP_ERR_CUDA", "LASP_ERR_TIMEOUT"]
+
+
+class LaspError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        name = _STATUS[status] if 0 <= status < len(_STATUS) else f"status {status}"
+        super().__init__(f"{where}: {name}")
+
+
+def library_path() -> str:
+    return _LIB_PATH
+
+
+def _load():
+    global _lib
+    if _lib is not None:
+        return _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(_LIB_PATH):
+                raise RuntimeError(
+                    f"{_LIB_PATH} is missing: build it with `python -m sequence_linear_attention_b200.build`")
+            lib = ctypes.CDLL(_LIB_PATH)
+            P, I, L, U64 = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_uint64
+            lib.lasp_fwd.argtypes = [P, P, P, P, P, I, I, L, I, I, I, P, P, P]
+            lib.lasp_bwd.argtypes = [P, P, P, P, P, P, P, P, I, I, L, I, I, I, P, P, P, P, P, P]
+            lib.lasp_chunk_states.argtypes = [P, P, P, P, P, I, I, L, I, I, I, P]
+            lib.lasp_chunk_dstates.argtypes = [P, P, P, P, I, I, L, I, I, I, P]
+            lib.lasp_chunk_out.argtypes = [P, P, P, P, P, P, I, I, L, I, I, I, P]
+            lib.lasp_chunk_grads.argtypes = [P, P, P, P, P, P, P, P, P, P, I, I, L, I, I, I, P]
+            lib.lasp_state_prefix.argtypes = [P, P, P, P, P, I, I, I, I, L, I, P]
+            lib.lasp_check_device_status.argtypes = [P, ctypes.POINTER(I)]
+            lib.lasp_set_wait_limit_ns.argtypes = [U64]
+            lib.lasp_wait_probe.argtypes = [P]
+            lib.lasp_status_string.argtypes = [I]
+            lib.lasp_status_string.restype = ctypes.c_char_p
+            for f in (lib.lasp_fwd, lib.lasp_bwd, lib.lasp_chunk_states, lib.lasp_chunk_dstates,
+                      lib.lasp_chunk_out, lib.lasp_chunk_grads,
+                      lib.lasp_state_prefix, lib.lasp_check_device_status, lib.lasp_set_wait_limit_ns,
+                      lib.lasp_wait_probe, lib.lasp_version):
+                f.restype = I
+            _lib = lib
+    return _lib
+
+
+# ----------------------------------------------------------------- marshalling
+def _ptr(t):
+    return None if t is None else t.data_ptr()
+
+
+def _stream(stream, like):
+    if stream is not None:
+        return stream if isinstance(stream, int) else stream.cuda_stream
+    import torch
+    return torch.cuda.current_stream(like.device).cuda_stream
+
+
+def _dtype_code(t):
+    import torch
+    if t.dtype == torch.float32:
+        return LASP_F32
+    if t.dtype == torch.bfloat16:
+        return LASP_BF16
+    raise TypeError(f"token tensors must be float32 or bfloat16, got {t.dtype}")
+
+
+def _tokens(*ts):
+    ref = ts[0]
+    if ref.dim() != 4:
+        raise ValueError("token tensors must be [B, N, H, d]")
+    for t in ts:
+        if t is None:
+            continue
+        if tuple(t.shape) != tuple(ref.shape) or t.dtype != ref.dtype or not t.is_contiguous() or not t.is_cuda:
+            raise ValueError("token tensors must be contiguous CUDA tensors of one shape and dtype")
+    B, N, H, d = ref.shape
+    return B, N, H, d, _dtype_code(ref)
+
+
+def _check(status, where):
+    if status != 0:
+        raise LaspError(status, where)
+
+
+# ---------------------------------------------------------------- entry points
+def lasp_fwd(q, k, v, decay, o, C, state_cache, init_state=None, stream=None):
+    """o = causal linear attention of (q, k, v); state_cache receives P_c. See lasp.h."""
+    B, N, H, d, dt = _tokens(q, k, v, o)
+    _check(_load().lasp_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(decay), _ptr(o), B, H, N, d, C, dt,
+                            _ptr(state_cache), _ptr(init_state), _stream(stream, q)), "lasp_fwd")
+
+
+def lasp_bwd(q, k, v, decay, dout, dq, dk, dv, C, state_cache, dstate_ws, init_state=None,
+             dstate_in=None, dinit_state=None, stream=None):
+    """dq, dk, dv of sum(o * dout); dstate_ws receives R_c. See lasp.h."""
+    B, N, H, d, dt = _tokens(q, k, v, dout, dq, dk, dv)
+    _check(_load().lasp_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(decay), _ptr(dout), _ptr(dq), _ptr(dk), _ptr(dv),
+                            B, H, N, d, C, dt, _ptr(state_cache), _ptr(dstate_ws), _ptr(init_state),
+                            _ptr(dstate_in), _ptr(dinit_state), _stream(stream, q)), "lasp_bwd")
+
+
+def lasp_chunk_states(q, k, v, decay, M, C, stream=None):
+    """M[b, c, h] = sum_j lambda^(C-1-j) k_j^T v_j. See lasp.h."""
+    B, N, H, d, dt = _tokens(k, v)
+    _check(_load().lasp_chunk_states(_ptr(q), _ptr(k), _ptr(v), _ptr(decay), _ptr(M), B, H, N, d, C, dt,
+                                     _stream(stream, k)), "lasp_chunk_states")
+
+
+def lasp_chunk_dstates(q, dout, decay, dM, C, stream=None):
+    """dM[b, c, h] = sum_j lambda^(j+1) q_j^T do_j. See lasp.h."""
+    B, N, H, d, dt = _tokens(q, dout)
+    _check(_load().lasp_chunk_dstates(_ptr(q), _ptr(dout), _ptr(decay), _ptr(dM), B, H, N, d, C, dt,
+                                      _stream(stream, q)), "lasp_chunk_dstates")
+
+
+def lasp_chunk_out(q, k, v, decay, P, o, C, stream=None):
+    """The output step alone: o from (q, k, v) and the chunk-entering states P. See lasp.h."""
+    B, N, H, d, dt = _tokens(q, k, v, o)
+    _check(_load().lasp_chunk_out(_ptr(q), _ptr(k), _ptr(v), _ptr(decay), _ptr(P), _ptr(o), B, H, N, d, C, dt,
+                                  _stream(stream, q)), "lasp_chunk_out")
+
+
+def lasp_chunk_grads(q, k, v, dout, decay, P, R, dq, dk, dv, C, stream=None):
+    """The dQ/dK/dV step alone, from the states P and R. See lasp.h."""
+    B, N, H, d, dt = _tokens(q, k, v, dout, dq, dk, dv)
+    _check(_load().lasp_chunk_grads(_ptr(q), _ptr(k), _ptr(v), _ptr(dout), _ptr(decay), _ptr(P), _ptr(R),
+                                    _ptr(dq), _ptr(dk), _ptr(dv), B, H, N, d, C, dt, _stream(stream, q)),
+           "lasp_chunk_grads")
+
+
+def lasp_state_prefix(M, Mprefix, decay, C, init=None, total=None, reverse=False, stream=None):
+    """Exclusive decayed prefix (or suffix) over chunk states [B, T, H, d, d]. See lasp.h."""
+    if M.dim() != 5:
+        raise ValueError("M must be [B, T, H, d, d]")
+    B, T, H, d, _ = M.shape
+    _check(_load().lasp_state_prefix(_ptr(M), _ptr(Mprefix), _ptr(decay), _ptr(init), _ptr(total),
+                                     B, T, H, d, int(C), int(bool(reverse)), _stream(stream, M)),
+           "lasp_state_prefix")
+
+
+def lasp_check_device_status(stream=None, device=None):
+    """(status, site): synchronizes the stream, returns and clears the device status word."""
+    import torch
+    s = stream if stream is not None else torch.cuda.current_stream(device).cuda_stream
+    site = ctypes.c_int(0)
+    st = _load().lasp_check_device_status(s if isinstance(s, int) else s.cuda_stream, ctypes.byref(site))
+    return st, site.value
+
+
+def lasp_set_wait_limit_ns(limit_ns: int):
+    _check(_load().lasp_set_wait_limit_ns(int(limit_ns)), "lasp_set_wait_limit_ns")
+
+
+def lasp_wait_probe(stream=None):
+    import torch
+    s = stream if stream is not None else torch.cuda.current_stream().cuda_stream
+    _check(_load().lasp_wait_probe(s if isinstance(s, int) else s.cuda_stream), "lasp_wait_probe")
+
+
+def lasp_status_string(status: int) -> str:
+    return _load().lasp_status_string(int(status)).decode()
+
+
+def lasp_version() -> int:
+    return int(_load().lasp_version())

@@ -1,0 +1,81 @@
+// Exclusive decayed scan over per-chunk d x d states (LASP-2: prefix sum of
+// the gathered M_t in the forward pass, suffix sum of dM_t in the backward
+// pass; LASP Eq. 10 and Eq. 20 give the per-chunk decay lambda^C).
+//
+//   forward:  P_0 = init,     P_c = g P_{c-1} + M_{c-1},  g = lambda^C
+//   reverse:  R_{T-1} = init, R_c = g R_{c+1} + M_{c+1}
+//
+// The scan is pure HBM traffic: every state element is read once and written
+// once. One thread owns one float4 of the d*d state of one (b, h) and walks the
+// chunks in order; the loads of a group of kUnroll chunks do not depend on the
+// recurrence, so they are all issued before the group's FMAs, keeping
+// kUnroll * 16 bytes in flight per thread. Consecutive threads own consecutive
+// float4s of one state, so every warp access is a fully coalesced 512-byte run.
+// M and P may be the same array: each element is loaded before it is stored,
+// by the same thread.
+#include "kernels.h"
+#include "lasp_common.cuh"
+
+namespace lasp {
+namespace scan_detail {
+
+constexpr int kUnroll = 16;
+constexpr int kThreads = 256;
+
+__device__ __forceinline__ float4 fma4(float g, float4 a, float4 m) {
+  return make_float4(fmaf(g, a.x, m.x), fmaf(g, a.y, m.y), fmaf(g, a.z, m.z), fmaf(g, a.w, m.w));
+}
+
+__global__ void __launch_bounds__(kThreads) state_scan_kernel(const float4* M, float4* P, const float* decay,
+                                                              const float4* __restrict__ init,
+                                                              float4* __restrict__ total, int H, int T,
+                                                              int dd4, int64_t n_threads, float Cf,
+                                                              int reverse) {
+  const int64_t idx = (int64_t)blockIdx.x * kThreads + threadIdx.x;
+  if (idx >= n_threads) return;
+  const int e = (int)(idx % dd4);
+  const int h = (int)((idx / dd4) % H);
+  const int64_t b = idx / ((int64_t)dd4 * H);
+  const float g = decay_pow(log2f(load_decay(decay, h)), Cf);
+  const int64_t bh = b * H + h;
+  float4 acc = init ? init[bh * dd4 + e] : make_float4(0.f, 0.f, 0.f, 0.f);
+  const int64_t cstride = (int64_t)H * dd4;  // float4s between chunk c and c+1
+  const int64_t base = (b * T * H + h) * (int64_t)dd4 + e;
+  const int64_t step = reverse ? -cstride : cstride;
+  int64_t off = reverse ? base + (int64_t)(T - 1) * cstride : base;
+  int n = 0;
+  for (; n + kUnroll <= T; n += kUnroll) {
+    float4 m[kUnroll];
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) m[u] = __ldcs(M + off + u * step);
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+      __stcs(P + off + u * step, acc);
+      acc = fma4(g, acc, m[u]);
+    }
+    off += kUnroll * step;
+  }
+  for (; n < T; ++n) {
+    float4 m = __ldcs(M + off);
+    __stcs(P + off, acc);
+    acc = fma4(g, acc, m);
+    off += step;
+  }
+  if (total) total[bh * dd4 + e] = acc;
+}
+
+}  // namespace scan_detail
+using namespace scan_detail;
+
+cudaError_t launch_state_scan(const float* M, float* P, const float* decay, const float* init, float* total,
+                              int B, int T, int H, int d, int64_t C, int reverse, cudaStream_t st) {
+  const int dd4 = d * d / 4;
+  const int64_t n_threads = (int64_t)B * H * dd4;
+  const int64_t blocks = (n_threads + kThreads - 1) / kThreads;
+  state_scan_kernel<<<(unsigned)blocks, kThreads, 0, st>>>(
+      (const float4*)M, (float4*)P, decay, (const float4*)init, (float4*)total, H, T, dd4, n_threads,
+      (float)C, reverse);
+  return cudaGetLastError();
+}
+
+}  // namespace lasp

@@ -1,0 +1,27 @@
+// Internal launchers behind the C ABI of include/lasp.h. Each returns the
+// cudaError_t of its launch; arguments are already validated by lasp_api.cu.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace lasp {
+
+// Exclusive decayed scan over chunk states (k_state_scan.cu).
+cudaError_t launch_state_scan(const float* M, float* P, const float* decay, const float* init, float* total,
+                              int B, int T, int H, int d, int64_t C, int reverse, cudaStream_t st);
+
+// CUDA-core kernels, any d in {32, 64, 128} and any C (k_simt.cu).
+// kind 0: M_c = sum lambda^{C-1-t} a_t^T b_t ; kind 1: sum lambda^{t+1} a_t^T b_t.
+cudaError_t simt_chunk_states(const void* a, const void* b, const float* decay, float* M, int B, int H,
+                              int64_t N, int d, int C, int kind, int dtype, cudaStream_t st);
+cudaError_t simt_chunk_out(const void* q, const void* k, const void* v, const float* decay, const float* P,
+                           void* o, int B, int H, int64_t N, int d, int C, int dtype, cudaStream_t st);
+cudaError_t simt_chunk_bwd(const void* q, const void* k, const void* v, const void* dout, const float* decay,
+                           const float* P, const float* Rs, void* dq, void* dk, void* dv, int B, int H,
+                           int64_t N, int d, int C, int dtype, cudaStream_t st);
+
+// One CTA waiting on a barrier nothing completes; ends by the wait limit.
+cudaError_t launch_wait_probe(cudaStream_t st);
+
+}  // namespace lasp

@@ -1,0 +1,202 @@
+// C ABI of include/lasp.h: host-side validation and dispatch to the kernels.
+// Nothing here allocates memory; every launch goes to the caller's stream.
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "kernels.h"
+#include "lasp_common.cuh"
+#include "sm100.cuh"
+#include "tc_kernels.h"
+
+namespace lasp {
+
+namespace api_detail {
+
+__global__ void wait_probe_kernel() {
+  __shared__ __align__(8) uint64_t bar;
+  if (threadIdx.x == 0) {
+    sm100::mbar_init(&bar, 1);
+    sm100::fence_mbar_init();
+    // Nothing arrives on the barrier: the wait can only end by its limit.
+    sm100::mbar_wait(&bar, 0, SITE_PROBE);
+  }
+}
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+inline int check_ptrs(std::initializer_list<const void*> required, std::initializer_list<const void*> optional) {
+  for (const void* p : required) {
+    if (p == nullptr) return LASP_ERR_INVALID_ARG;
+    if (!aligned16(p)) return LASP_ERR_MISALIGNED;
+  }
+  for (const void* p : optional)
+    if (p != nullptr && !aligned16(p)) return LASP_ERR_MISALIGNED;
+  return LASP_OK;
+}
+
+inline int check_sizes(int B, int H, int64_t N, int d, int64_t C, int dtype) {
+  if (dtype != LASP_F32 && dtype != LASP_BF16) return LASP_ERR_INVALID_ARG;
+  if (B < 1 || H < 1 || N < 0 || C < 1) return LASP_ERR_INVALID_ARG;
+  if (B > 65535 || H > 65535) return LASP_ERR_UNSUPPORTED;  // grid y / z limits
+  if (d != 32 && d != 64 && d != 128) return LASP_ERR_UNSUPPORTED;
+  if (N % C != 0) return LASP_ERR_INVALID_ARG;
+  if (N / C > INT32_MAX) return LASP_ERR_UNSUPPORTED;
+  return LASP_OK;
+}
+
+inline int cuda_status(cudaError_t e) { return e == cudaSuccess ? LASP_OK : LASP_ERR_CUDA; }
+
+// The tensor-core kernels take bf16 with d in {64, 128} and C a multiple of 16;
+// everything else runs on the CUDA-core kernels.
+inline bool tc_states_ok(int dtype, int d, int64_t C) {
+  return dtype == LASP_BF16 && (d == 64 || d == 128) && C % 16 == 0;
+}
+
+int chunk_states_impl(const void* a, const void* b, const float* decay, float* M, int B, int H, int64_t N, int d,
+                      int C, int dtype, int kind, cudaStream_t st) {
+  if (tc_states_ok(dtype, d, C)) return cuda_status(tc_chunk_states(a, b, decay, M, B, H, N, d, C, kind, st));
+  return cuda_status(simt_chunk_states(a, b, decay, M, B, H, N, d, C, kind, dtype, st));
+}
+
+int chunk_out_impl(const void* q, const void* k, const void* v, const float* decay, const float* P, void* o, int B,
+                   int H, int64_t N, int d, int C, int dtype, cudaStream_t st) {
+  if (tc_out_ok(dtype, d, C)) return cuda_status(tc_chunk_out(q, k, v, decay, P, o, B, H, N, d, C, st));
+  return cuda_status(simt_chunk_out(q, k, v, decay, P, o, B, H, N, d, C, dtype, st));
+}
+
+int chunk_grads_impl(const void* q, const void* k, const void* v, const void* dout, const float* decay,
+                     const float* P, const float* R, void* dq, void* dk, void* dv, int B, int H, int64_t N, int d,
+                     int C, int dtype, cudaStream_t st) {
+  if (tc_bwd_ok(dtype, d, C)) return cuda_status(tc_chunk_bwd(q, k, v, dout, decay, P, R, dq, dk, dv, B, H, N, d, C, st));
+  return cuda_status(simt_chunk_bwd(q, k, v, dout, decay, P, R, dq, dk, dv, B, H, N, d, C, dtype, st));
+}
+
+}  // namespace api_detail
+}  // namespace lasp
+
+using namespace lasp;
+using namespace lasp::api_detail;
+
+extern "C" {
+
+int lasp_version(void) { return 100; }
+
+const char* lasp_status_string(int status) {
+  switch (status) {
+    case LASP_OK: return "LASP_OK";
+    case LASP_ERR_INVALID_ARG: return "LASP_ERR_INVALID_ARG";
+    case LASP_ERR_UNSUPPORTED: return "LASP_ERR_UNSUPPORTED";
+    case LASP_ERR_MISALIGNED: return "LASP_ERR_MISALIGNED";
+    case LASP_ERR_CUDA: return "LASP_ERR_CUDA";
+    case LASP_ERR_TIMEOUT: return "LASP_ERR_TIMEOUT";
+    default: return "LASP_ERR_UNKNOWN";
+  }
+}
+
+int lasp_chunk_states(const void* q, const void* k, const void* v, const float* decay, float* M, int B, int H,
+                      int64_t N, int d, int C, int dtype, void* stream) {
+  (void)q;
+  int s = check_sizes(B, H, N, d, C, dtype);
+  if (s) return s;
+  if (N == 0) return LASP_OK;
+  if ((s = check_ptrs({k, v, M}, {decay}))) return s;
+  return chunk_states_impl(k, v, decay, M, B, H, N, d, C, dtype, 0, (cudaStream_t)stream);
+}
+
+int lasp_chunk_dstates(const void* q, const void* dout, const float* decay, float* dM, int B, int H, int64_t N,
+                       int d, int C, int dtype, void* stream) {
+  int s = check_sizes(B, H, N, d, C, dtype);
+  if (s) return s;
+  if (N == 0) return LASP_OK;
+  if ((s = check_ptrs({q, dout, dM}, {decay}))) return s;
+  return chunk_states_impl(q, dout, decay, dM, B, H, N, d, C, dtype, 1, (cudaStream_t)stream);
+}
+
+int lasp_state_prefix(const float* M, float* Mprefix, const float* decay, const float* init, float* total, int B,
+                      int T, int H, int d, int64_t C, int reverse, void* stream) {
+  if (B < 1 || H < 1 || T < 0 || C < 1 || (reverse != 0 && reverse != 1)) return LASP_ERR_INVALID_ARG;
+  if (d != 32 && d != 64 && d != 128) return LASP_ERR_UNSUPPORTED;
+  if (C > (int64_t)1 << 24) return LASP_ERR_UNSUPPORTED;  // lambda^C exponent kept exact in fp32
+  if (T > 0) {
+    int s = check_ptrs({M, Mprefix}, {decay, init, total});
+    if (s) return s;
+  } else {
+    int s = check_ptrs({}, {decay, init, total});
+    if (s) return s;
+    if (total == nullptr) return LASP_OK;
+  }
+  return cuda_status(launch_state_scan(M, Mprefix, decay, init, total, B, T, H, d, C, reverse, (cudaStream_t)stream));
+}
+
+int lasp_fwd(const void* q, const void* k, const void* v, const float* decay, void* o, int B, int H, int64_t N,
+             int d, int C, int dtype, float* state_cache, const float* init_state, void* stream) {
+  int s = check_sizes(B, H, N, d, C, dtype);
+  if (s) return s;
+  if (N == 0) return LASP_OK;
+  if ((s = check_ptrs({q, k, v, o, state_cache}, {decay, init_state}))) return s;
+  cudaStream_t st = (cudaStream_t)stream;
+  const int T = (int)(N / C);
+  // 1. chunk states M_c into the cache; 2. exclusive prefix in place -> P_c; 3. output.
+  if ((s = chunk_states_impl(k, v, decay, state_cache, B, H, N, d, C, dtype, 0, st))) return s;
+  if ((s = cuda_status(launch_state_scan(state_cache, state_cache, decay, init_state, nullptr, B, T, H, d, C, 0, st))))
+    return s;
+  return chunk_out_impl(q, k, v, decay, state_cache, o, B, H, N, d, C, dtype, st);
+}
+
+int lasp_chunk_out(const void* q, const void* k, const void* v, const float* decay, const float* P, void* o, int B,
+                   int H, int64_t N, int d, int C, int dtype, void* stream) {
+  int s = check_sizes(B, H, N, d, C, dtype);
+  if (s) return s;
+  if (N == 0) return LASP_OK;
+  if ((s = check_ptrs({q, k, v, P, o}, {decay}))) return s;
+  return chunk_out_impl(q, k, v, decay, P, o, B, H, N, d, C, dtype, (cudaStream_t)stream);
+}
+
+int lasp_chunk_grads(const void* q, const void* k, const void* v, const void* dout, const float* decay,
+                     const float* P, const float* R, void* dq, void* dk, void* dv, int B, int H, int64_t N, int d,
+                     int C, int dtype, void* stream) {
+  int s = check_sizes(B, H, N, d, C, dtype);
+  if (s) return s;
+  if (N == 0) return LASP_OK;
+  if ((s = check_ptrs({q, k, v, dout, P, R, dq, dk, dv}, {decay}))) return s;
+  return chunk_grads_impl(q, k, v, dout, decay, P, R, dq, dk, dv, B, H, N, d, C, dtype, (cudaStream_t)stream);
+}
+
+int lasp_bwd(const void* q, const void* k, const void* v, const float* decay, const void* dout, void* dq, void* dk,
+             void* dv, int B, int H, int64_t N, int d, int C, int dtype, const float* state_cache, float* dstate_ws,
+             const float* init_state, const float* dstate_in, float* dinit_state, void* stream) {
+  (void)init_state;
+  int s = check_sizes(B, H, N, d, C, dtype);
+  if (s) return s;
+  if (N == 0) return LASP_OK;
+  if ((s = check_ptrs({q, k, v, dout, dq, dk, dv, state_cache, dstate_ws}, {decay, init_state, dstate_in, dinit_state})))
+    return s;
+  cudaStream_t st = (cudaStream_t)stream;
+  const int T = (int)(N / C);
+  // 1. gradient chunk states dM_c; 2. exclusive suffix in place -> R_c; 3. dQ, dK, dV.
+  if ((s = chunk_states_impl(q, dout, decay, dstate_ws, B, H, N, d, C, dtype, 1, st))) return s;
+  if ((s = cuda_status(launch_state_scan(dstate_ws, dstate_ws, decay, dstate_in, dinit_state, B, T, H, d, C, 1, st))))
+    return s;
+  return chunk_grads_impl(q, k, v, dout, decay, state_cache, dstate_ws, dq, dk, dv, B, H, N, d, C, dtype, st);
+}
+
+int lasp_check_device_status(void* stream, int* site) {
+  if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return LASP_ERR_CUDA;
+  unsigned int word = 0, zero = 0;
+  if (cudaMemcpyFromSymbol(&word, g_device_status, sizeof(word)) != cudaSuccess) return LASP_ERR_CUDA;
+  if (word != 0 && cudaMemcpyToSymbol(g_device_status, &zero, sizeof(zero)) != cudaSuccess) return LASP_ERR_CUDA;
+  if (site) *site = (int)(word & 0xFFFFu);
+  return (int)(word >> 16);
+}
+
+int lasp_set_wait_limit_ns(uint64_t limit_ns) {
+  unsigned long long v = limit_ns;
+  return cuda_status(cudaMemcpyToSymbol(g_wait_limit_ns, &v, sizeof(v)));
+}
+
+int lasp_wait_probe(void* stream) {
+  wait_probe_kernel<<<1, 32, 0, (cudaStream_t)stream>>>();
+  return cuda_status(cudaGetLastError());
+}
+
+}  // extern "C"

@@ -1,0 +1,6 @@
+// The whole library is one translation unit, so that the per-device status
+// word and wait limit (lasp_common.cuh) need no relocatable device code.
+#include "lasp_api.cu"
+#include "k_state_scan.cu"
+#include "k_simt.cu"
+#include "k_tc_stubs.cu"

@@ -1,0 +1,24 @@
+// Tensor-core (tcgen05 / TMEM / TMA) kernels for bf16 inputs, and the
+// predicates that say which sizes they take. The CUDA-core kernels of
+// k_simt.cu serve every other size.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace lasp {
+
+// Chunk states on tensor cores: bf16, d in {64, 128}, C a multiple of 16.
+cudaError_t tc_chunk_states(const void* a, const void* b, const float* decay, float* M, int B, int H, int64_t N,
+                            int d, int C, int kind, cudaStream_t st);
+
+bool tc_out_ok(int dtype, int d, int64_t C);
+cudaError_t tc_chunk_out(const void* q, const void* k, const void* v, const float* decay, const float* P, void* o,
+                         int B, int H, int64_t N, int d, int C, cudaStream_t st);
+
+bool tc_bwd_ok(int dtype, int d, int64_t C);
+cudaError_t tc_chunk_bwd(const void* q, const void* k, const void* v, const void* dout, const float* decay,
+                         const float* P, const float* Rs, void* dq, void* dk, void* dv, int B, int H, int64_t N,
+                         int d, int C, cudaStream_t st);
+
+}  // namespace lasp

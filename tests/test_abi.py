@@ -1,0 +1,117 @@
+"""The C-ABI library without a GPU: it loads, exports every entry point that
+include/lasp.h declares, and rejects bad arguments on the host before any
+launch (these calls never reach the device, so they run on a CPU-only host)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import sequence_linear_attention_b200 as lasp
+from sequence_linear_attention_b200 import build as lasp_build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "lasp.h")
+
+OK, INVALID, UNSUPPORTED, MISALIGNED = 0, 1, 2, 3
+F32, BF16 = 0, 1
+A = 1 << 20  # a fake, 16-byte aligned device address; validation never dereferences it
+
+
+def _declared():
+    src = open(HEADER).read()
+    return sorted(set(re.findall(r"LASP_API\s+[\w\s\*]+?\b(lasp_\w+)\s*\(", src)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    lasp_build.build()
+    return lasp._load()
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = _declared()
+    assert {"lasp_fwd", "lasp_bwd", "lasp_chunk_states", "lasp_state_prefix"} <= set(names)
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_status_strings(lib):
+    assert lasp.lasp_status_string(0) == "LASP_OK"
+    assert lasp.lasp_status_string(5) == "LASP_ERR_TIMEOUT"
+    assert lasp.lasp_status_string(99) == "LASP_ERR_UNKNOWN"
+    assert lasp.lasp_version() >= 100
+
+
+def _fwd(lib, q=A, k=A, v=A, decay=None, o=A, B=1, H=2, N=256, d=32, C=64, dt=F32, cache=A, init=None):
+    return lib.lasp_fwd(q, k, v, decay, o, B, H, N, d, C, dt, cache, init, None)
+
+
+def _bwd(lib, B=1, H=2, N=256, d=32, C=64, dt=BF16, ptrs=None):
+    p = dict(q=A, k=A, v=A, decay=None, do=A, dq=A, dk=A, dv=A, cache=A, ws=A, init=None, din=None, dinit=None)
+    p.update(ptrs or {})
+    return lib.lasp_bwd(p["q"], p["k"], p["v"], p["decay"], p["do"], p["dq"], p["dk"], p["dv"], B, H, N, d, C, dt,
+                        p["cache"], p["ws"], p["init"], p["din"], p["dinit"], None)
+
+
+def test_fwd_rejects_bad_sizes(lib):
+    assert _fwd(lib, N=250) == INVALID          # C does not divide N
+    assert _fwd(lib, C=0) == INVALID
+    assert _fwd(lib, B=0) == INVALID
+    assert _fwd(lib, H=0) == INVALID
+    assert _fwd(lib, N=-64) == INVALID
+    assert _fwd(lib, d=96) == UNSUPPORTED
+    assert _fwd(lib, d=256) == UNSUPPORTED
+    assert _fwd(lib, dt=7) == INVALID
+    assert _fwd(lib, B=70000) == UNSUPPORTED
+
+
+def test_fwd_rejects_bad_pointers(lib):
+    assert _fwd(lib, q=None) == INVALID
+    assert _fwd(lib, cache=None) == INVALID
+    assert _fwd(lib, o=A + 8) == MISALIGNED
+    assert _fwd(lib, decay=A + 4) == MISALIGNED
+    assert _fwd(lib, init=A + 2) == MISALIGNED
+
+
+def test_empty_sequence_launches_nothing(lib):
+    # N = 0 is valid and returns before touching the device (no GPU here)
+    assert _fwd(lib, N=0) == OK
+    assert _bwd(lib, N=0) == OK
+    assert lib.lasp_chunk_states(None, A, A, None, A, 1, 2, 0, 64, 16, BF16, None) == OK
+
+
+def test_bwd_rejects_bad_arguments(lib):
+    assert _bwd(lib, ptrs={"ws": None}) == INVALID
+    assert _bwd(lib, ptrs={"dk": A + 1}) == MISALIGNED
+    assert _bwd(lib, ptrs={"dinit": A + 12}) == MISALIGNED
+    assert _bwd(lib, N=100, C=64) == INVALID
+
+
+def test_state_prefix_rejects_bad_arguments(lib):
+    f = lib.lasp_state_prefix
+    assert f(A, A, None, None, None, 1, 4, 2, 64, 128, 2, None) == INVALID   # reverse must be 0 or 1
+    assert f(A, A, None, None, None, 1, -1, 2, 64, 128, 0, None) == INVALID
+    assert f(A, A, None, None, None, 1, 4, 2, 48, 128, 0, None) == UNSUPPORTED
+    assert f(None, A, None, None, None, 1, 4, 2, 64, 128, 0, None) == INVALID
+    assert f(A, A, None, None, None, 1, 4, 2, 64, 0, 0, None) == INVALID
+    assert f(A, A + 4, None, None, None, 1, 4, 2, 64, 128, 0, None) == MISALIGNED
+    assert f(None, None, None, None, None, 1, 0, 2, 64, 128, 0, None) == OK  # T = 0, nothing to write
+
+
+def test_chunk_states_rejects_bad_arguments(lib):
+    f = lib.lasp_chunk_states
+    assert f(None, None, A, None, A, 1, 2, 256, 64, 64, BF16, None) == INVALID
+    assert f(None, A, A, None, A, 1, 2, 256, 64, 48, BF16, None) == INVALID   # 48 does not divide 256
+    assert f(None, A, A + 2, None, A, 1, 2, 256, 64, 64, BF16, None) == MISALIGNED
+    g = lib.lasp_chunk_dstates
+    assert g(A, None, None, A, 1, 2, 256, 64, 64, BF16, None) == INVALID
+
+
+def test_binding_marshals_only(lib):
+    import inspect
+    src = inspect.getsource(lasp)
+    # the binding never falls back to torch arithmetic or to the oracle
+    for forbidden in ("oracle", "einsum", "matmul", "cumsum", "@"):
+        assert forbidden not in src.replace("@property", ""), forbidden
+    assert ctypes.CDLL(lasp.library_path())
