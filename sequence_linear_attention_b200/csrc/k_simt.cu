@@ -265,26 +265,25 @@ cudaError_t launch_bwd(const void* q, const void* k, const void* v, const void* 
 }
 
 }  // namespace simt_detail
-using namespace simt_detail;
 
 cudaError_t simt_chunk_states(const void* a, const void* b, const float* decay, float* M, int B, int H,
                               int64_t N, int d, int C, int kind, int dtype, cudaStream_t st) {
-  return dtype == LASP_F32 ? launch_states<float>(a, b, decay, M, B, H, N, d, C, kind, st)
-                           : launch_states<__nv_bfloat16>(a, b, decay, M, B, H, N, d, C, kind, st);
+  return dtype == LASP_F32 ? simt_detail::launch_states<float>(a, b, decay, M, B, H, N, d, C, kind, st)
+                           : simt_detail::launch_states<__nv_bfloat16>(a, b, decay, M, B, H, N, d, C, kind, st);
 }
 
 cudaError_t simt_chunk_out(const void* q, const void* k, const void* v, const float* decay, const float* P,
                            void* o, int B, int H, int64_t N, int d, int C, int dtype, cudaStream_t st) {
-  return dtype == LASP_F32 ? launch_out<float>(q, k, v, decay, P, o, B, H, N, d, C, st)
-                           : launch_out<__nv_bfloat16>(q, k, v, decay, P, o, B, H, N, d, C, st);
+  return dtype == LASP_F32 ? simt_detail::launch_out<float>(q, k, v, decay, P, o, B, H, N, d, C, st)
+                           : simt_detail::launch_out<__nv_bfloat16>(q, k, v, decay, P, o, B, H, N, d, C, st);
 }
 
 cudaError_t simt_chunk_bwd(const void* q, const void* k, const void* v, const void* dout, const float* decay,
                            const float* P, const float* Rs, void* dq, void* dk, void* dv, int B, int H,
                            int64_t N, int d, int C, int dtype, cudaStream_t st) {
   return dtype == LASP_F32
-             ? launch_bwd<float>(q, k, v, dout, decay, P, Rs, dq, dk, dv, B, H, N, d, C, st)
-             : launch_bwd<__nv_bfloat16>(q, k, v, dout, decay, P, Rs, dq, dk, dv, B, H, N, d, C, st);
+             ? simt_detail::launch_bwd<float>(q, k, v, dout, decay, P, Rs, dq, dk, dv, B, H, N, d, C, st)
+             : simt_detail::launch_bwd<__nv_bfloat16>(q, k, v, dout, decay, P, Rs, dq, dk, dv, B, H, N, d, C, st);
 }
 
 }  // namespace lasp

@@ -65,14 +65,13 @@ __global__ void __launch_bounds__(kThreads) state_scan_kernel(const float4* M, f
 }
 
 }  // namespace scan_detail
-using namespace scan_detail;
 
 cudaError_t launch_state_scan(const float* M, float* P, const float* decay, const float* init, float* total,
                               int B, int T, int H, int d, int64_t C, int reverse, cudaStream_t st) {
   const int dd4 = d * d / 4;
   const int64_t n_threads = (int64_t)B * H * dd4;
-  const int64_t blocks = (n_threads + kThreads - 1) / kThreads;
-  state_scan_kernel<<<(unsigned)blocks, kThreads, 0, st>>>(
+  const int64_t blocks = (n_threads + scan_detail::kThreads - 1) / scan_detail::kThreads;
+  scan_detail::state_scan_kernel<<<(unsigned)blocks, scan_detail::kThreads, 0, st>>>(
       (const float4*)M, (float4*)P, decay, (const float4*)init, (float4*)total, H, T, dd4, n_threads,
       (float)C, reverse);
   return cudaGetLastError();

@@ -46,12 +46,6 @@ inline int check_sizes(int B, int H, int64_t N, int d, int64_t C, int dtype) {
 
 inline int cuda_status(cudaError_t e) { return e == cudaSuccess ? LASP_OK : LASP_ERR_CUDA; }
 
-// The tensor-core kernels take bf16 with d in {64, 128} and C a multiple of 16;
-// everything else runs on the CUDA-core kernels.
-inline bool tc_states_ok(int dtype, int d, int64_t C) {
-  return dtype == LASP_BF16 && (d == 64 || d == 128) && C % 16 == 0;
-}
-
 int chunk_states_impl(const void* a, const void* b, const float* decay, float* M, int B, int H, int64_t N, int d,
                       int C, int dtype, int kind, cudaStream_t st) {
   if (tc_states_ok(dtype, d, C)) return cuda_status(tc_chunk_states(a, b, decay, M, B, H, N, d, C, kind, st));

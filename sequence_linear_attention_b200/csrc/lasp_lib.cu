@@ -3,4 +3,5 @@
 #include "lasp_api.cu"
 #include "k_state_scan.cu"
 #include "k_simt.cu"
+#include "k_tc_states.cu"
 #include "k_tc_stubs.cu"

@@ -8,7 +8,9 @@
 
 namespace lasp {
 
-// Chunk states on tensor cores: bf16, d in {64, 128}, C a multiple of 16.
+// Chunk states on tensor cores: bf16, d = 128, C a multiple of 16. The
+// CUDA-core kernels take every size for which a predicate is false.
+bool tc_states_ok(int dtype, int d, int64_t C);
 cudaError_t tc_chunk_states(const void* a, const void* b, const float* decay, float* M, int B, int H, int64_t N,
                             int d, int C, int kind, cudaStream_t st);
 

@@ -51,14 +51,17 @@ def host_f32(inp: dict, name: str) -> np.ndarray:
     return lasp_inputs.as_f32(inp[name], inp["bf16"])
 
 
-def run_fwd_bwd(inp: dict, C: int, init=None, dstate_in=None, want_dinit=False, decay_override="keep"):
+_KEEP = object()
+
+
+def run_fwd_bwd(inp: dict, C: int, init=None, dstate_in=None, want_dinit=False, decay_override=_KEEP):
     """Runs lasp_fwd and lasp_bwd on the device; returns a dict of device tensors."""
     import torch
     import sequence_linear_attention_b200 as lasp
     bf16 = inp["bf16"]
     q, k, v, do = (to_device(inp[n], bf16) for n in ("q", "k", "v", "do"))
     B, N, H, d = q.shape
-    lam = inp["lam"] if decay_override == "keep" else decay_override
+    lam = inp["lam"] if decay_override is _KEEP else decay_override
     decay = decay_device(lam)
     T = N // C
     o = torch.empty_like(q)
