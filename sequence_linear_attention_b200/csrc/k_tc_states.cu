@@ -44,7 +44,21 @@ __device__ __forceinline__ uint32_t bf16x2_scale(uint32_t x, float w) {
   return *reinterpret_cast<uint32_t*>(&r);
 }
 
-__global__ void __launch_bounds__(kThreads) chunk_states_tc(const __grid_constant__ CUtensorMap map_a,
+// Issues the four TMA boxes of stage `stage` (A and B, two 64-feature boxes
+// each) into slot stage & 1.
+__device__ __forceinline__ void issue_stage(uint8_t* tiles, uint32_t tile_bytes, Smem* s, const CUtensorMap* map_a,
+                                            const CUtensorMap* map_b, int stage, int row, int h, int b) {
+  const int slot = stage & 1;
+  uint8_t* a = tiles + (size_t)slot * 2 * tile_bytes;
+  uint8_t* bb = a + tile_bytes;
+  mbar_arrive_expect_tx(&s->full[slot], 2 * tile_bytes);
+  tma_load_4d(a, map_a, &s->full[slot], 0, h, row, b);
+  tma_load_4d(a + tile_bytes / 2, map_a, &s->full[slot], 64, h, row, b);
+  tma_load_4d(bb, map_b, &s->full[slot], 0, h, row, b);
+  tma_load_4d(bb + tile_bytes / 2, map_b, &s->full[slot], 64, h, row, b);
+}
+
+__global__ void __launch_bounds__(kThreads, 1) chunk_states_tc(const __grid_constant__ CUtensorMap map_a,
                                                             const __grid_constant__ CUtensorMap map_b,
                                                             const float* decay, float* __restrict__ M, int H,
                                                             int C, int KB, int kind) {
@@ -62,20 +76,6 @@ __global__ void __launch_bounds__(kThreads) chunk_states_tc(const __grid_constan
   const float lam = load_decay(decay, h);
   const float l2 = log2f(lam);
   const bool scale = lam != 1.0f;
-
-  auto slot_a = [&](int slot) { return tiles + (size_t)slot * 2 * tile_bytes; };
-  auto slot_b = [&](int slot) { return tiles + (size_t)slot * 2 * tile_bytes + tile_bytes; };
-  auto issue_load = [&](int stage) {
-    const int slot = stage & 1;
-    const int row = c * C + stage * KB;
-    mbar_arrive_expect_tx(&s->full[slot], 4 * (tile_bytes / 2));
-    uint8_t* a = slot_a(slot);
-    uint8_t* bb = slot_b(slot);
-    tma_load_4d(a, &map_a, &s->full[slot], 0, h, row, b);
-    tma_load_4d(a + tile_bytes / 2, &map_a, &s->full[slot], 64, h, row, b);
-    tma_load_4d(bb, &map_b, &s->full[slot], 0, h, row, b);
-    tma_load_4d(bb + tile_bytes / 2, &map_b, &s->full[slot], 64, h, row, b);
-  };
 
   if (tid == 0) {
     prefetch_tmap(&map_a);
@@ -98,8 +98,8 @@ __global__ void __launch_bounds__(kThreads) chunk_states_tc(const __grid_constan
   const uint32_t tmem = s->tmem_base;
 
   if (tid == 0) {
-    issue_load(0);
-    if (nstages > 1) issue_load(1);
+    issue_stage(tiles, tile_bytes, s, &map_a, &map_b, 0, c * C, h, b);
+    if (nstages > 1) issue_stage(tiles, tile_bytes, s, &map_a, &map_b, 1, c * C + KB, h, b);
   }
 
   constexpr uint32_t idesc = idesc_bf16(128, 128, 1, 1);
@@ -110,7 +110,7 @@ __global__ void __launch_bounds__(kThreads) chunk_states_tc(const __grid_constan
     if (scale) {
       // scale row r of A by w_{k*KB + r}; the row of a 16-byte chunk is its
       // byte offset / 128 in either 64-feature box, whatever the swizzle
-      uint4* a = reinterpret_cast<uint4*>(slot_a(slot));
+      uint4* a = reinterpret_cast<uint4*>(tiles + (size_t)slot * 2 * tile_bytes);
       const int nchunks = KB * 16;
       for (int g = tid; g < nchunks; g += kThreads) {
         const int r = (g % (KB * 8)) / 8;
@@ -129,7 +129,7 @@ __global__ void __launch_bounds__(kThreads) chunk_states_tc(const __grid_constan
     if (s->abort) break;
     if (tid == 0) {
       tc_fence_after();
-      const uint32_t a0 = smem_u32(slot_a(slot)), b0 = smem_u32(slot_b(slot));
+      const uint32_t a0 = smem_u32(tiles + (size_t)slot * 2 * tile_bytes), b0 = a0 + tile_bytes;
       for (int j = 0; j < KB / 16; ++j) {
         const uint64_t ad = sw128_desc(a0 + j * 2048, KB * 128, 1024);
         const uint64_t bd = sw128_desc(b0 + j * 2048, KB * 128, 1024);
@@ -138,7 +138,8 @@ __global__ void __launch_bounds__(kThreads) chunk_states_tc(const __grid_constan
       mma_commit(k + 1 < nstages ? &s->empty[slot] : &s->done);
       if (k + 2 < nstages) {
         // the slot is refilled once the MMAs that read it have completed
-        if (mbar_wait(&s->empty[slot], par, SITE_STATES_MMA)) issue_load(k + 2);
+        if (mbar_wait(&s->empty[slot], par, SITE_STATES_MMA))
+          issue_stage(tiles, tile_bytes, s, &map_a, &map_b, k + 2, c * C + (k + 2) * KB, h, b);
         else s->abort = 1;
       }
     }
@@ -149,7 +150,7 @@ __global__ void __launch_bounds__(kThreads) chunk_states_tc(const __grid_constan
   if (ok) {
     const int row = warp * 32 + lane;
     float* out = M + ((((int64_t)b * T + c) * H + h) * kD + row) * kD;
-#pragma unroll
+#pragma unroll 1
     for (int cc = 0; cc < kD / 32; ++cc) {
       uint32_t r[32];
       tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16) + cc * 32, r);

@@ -4,4 +4,5 @@
 #include "k_state_scan.cu"
 #include "k_simt.cu"
 #include "k_tc_states.cu"
-#include "k_tc_stubs.cu"
+#include "k_tc_out.cu"
+#include "k_tc_bwd.cu"
