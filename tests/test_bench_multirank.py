@@ -1,0 +1,52 @@
+"""bench.py's multi-rank plumbing on CPU: two gloo ranks, the step time is the
+max over ranks and the throughput counts every rank's tokens."""
+import os
+import socket
+import sys
+
+import pytest
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _worker(rank, world, port, out):
+    os.environ.update(RANK=str(rank), WORLD_SIZE=str(world), LOCAL_RANK=str(rank), MASTER_ADDR="127.0.0.1",
+                      MASTER_PORT=str(port), LASP_BENCH_BACKEND="gloo")
+    sys.path.insert(0, ROOT)
+    import bench
+    import torch.distributed as dist
+    r, w, _ = bench.dist_setup()
+    try:
+        seconds = 1.0 + r  # rank 1 is the slow one
+        value, t = bench.aggregate(1000.0, seconds, w)
+        bench.barrier(w)
+        out[r] = (value, t)
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.timeout(120)
+def test_two_gloo_ranks_take_the_slowest_rank():
+    ctx = mp.get_context("spawn")
+    with ctx.Manager() as m:
+        out = m.dict()
+        mp.start_processes(_worker, args=(2, _free_port(), out), nprocs=2, join=True, start_method="spawn")
+        res = dict(out)
+    for r in (0, 1):
+        value, t = res[r]
+        assert t == 2.0
+        assert value == pytest.approx(2 * 1000.0 / 2.0)
+
+
+def test_single_rank_needs_no_process_group():
+    sys.path.insert(0, ROOT)
+    import bench
+    assert bench.aggregate(500.0, 0.5, 1) == (1000.0, 0.5)
+    assert bench.algorithmic_bytes("state_prefix", 1, 128, 128, 2) == 2 * 128 * 128 * 4 / 128
