@@ -183,6 +183,34 @@ LASP_API int lasp_chunk_grads(const void* q, const void* k, const void* v, const
                               int64_t N, int d, int C, int dtype, void* stream);
 
 /*
+ * lasp_bwd_noalloc -- lasp_bwd without the caller-provided workspace.
+ * The pages have no counterpart to this call; it exists for callers that
+ * cannot allocate device memory: a plain C program or plug-in with no device
+ * allocator of its own, or a host application whose memory pool already owns
+ * all of the device memory, so that a cudaMalloc would fail (and would
+ * synchronize the device if it succeeded).
+ * It computes exactly what lasp_bwd computes, with the same arguments except
+ * dstate_ws: the gradient states R live in a fixed 32 MiB array compiled into
+ * the library (LASP_NOALLOC_SCRATCH_BYTES), which every GPU that loads the
+ * library holds until the process exits. The call allocates nothing.
+ *   Limit: B * (N / C) * H * d * d * 4 <= LASP_NOALLOC_SCRATCH_BYTES (for
+ *   d = 128: at most 512 chunk-head states); larger problems return
+ *   LASP_ERR_UNSUPPORTED before anything is launched.
+ *   Set-up: the first call on each device looks up the device address of the
+ *   array, with that device current, and caches it; make that first call
+ *   before any stream capture.
+ *   Sharing: every call uses the same array, which keeps the last call's
+ *   contents (nothing in it needs to start at zero). Calls that overlap on the
+ *   GPU (on different streams, or from different threads) race on it and must
+ *   be serialized by the caller.
+ */
+#define LASP_NOALLOC_SCRATCH_BYTES (32u << 20)
+LASP_API int lasp_bwd_noalloc(const void* q, const void* k, const void* v, const float* decay, const void* dout,
+                              void* dq, void* dk, void* dv, int B, int H, int64_t N, int d, int C, int dtype,
+                              const float* state_cache, const float* dstate_in, float* dinit_state,
+                              void* stream);
+
+/*
  * lasp_check_device_status -- synchronizes `stream`, then returns and clears
  * the first error any kernel of this library recorded on the current device
  * (LASP_OK if none; LASP_ERR_TIMEOUT for a wait that ran out;

@@ -19,7 +19,7 @@ import threading
 
 __all__ = [
     "LaspError", "library_path", "lasp_fwd", "lasp_bwd", "lasp_chunk_states", "lasp_chunk_dstates",
-    "lasp_chunk_out", "lasp_chunk_grads",
+    "lasp_chunk_out", "lasp_chunk_grads", "lasp_bwd_noalloc",
     "lasp_state_prefix", "lasp_check_device_status", "lasp_set_wait_limit_ns", "lasp_wait_probe",
     "lasp_status_string", "lasp_version",
 ]
@@ -60,6 +60,7 @@ def _load():
             lib.lasp_bwd.argtypes = [P, P, P, P, P, P, P, P, I, I, L, I, I, I, P, P, P, P, P, P]
             lib.lasp_chunk_states.argtypes = [P, P, P, P, P, I, I, L, I, I, I, P]
             lib.lasp_chunk_dstates.argtypes = [P, P, P, P, I, I, L, I, I, I, P]
+            lib.lasp_bwd_noalloc.argtypes = [P, P, P, P, P, P, P, P, I, I, L, I, I, I, P, P, P, P]
             lib.lasp_chunk_out.argtypes = [P, P, P, P, P, P, I, I, L, I, I, I, P]
             lib.lasp_chunk_grads.argtypes = [P, P, P, P, P, P, P, P, P, P, I, I, L, I, I, I, P]
             lib.lasp_state_prefix.argtypes = [P, P, P, P, P, I, I, I, I, L, I, P]
@@ -69,7 +70,7 @@ def _load():
             lib.lasp_status_string.argtypes = [I]
             lib.lasp_status_string.restype = ctypes.c_char_p
             for f in (lib.lasp_fwd, lib.lasp_bwd, lib.lasp_chunk_states, lib.lasp_chunk_dstates,
-                      lib.lasp_chunk_out, lib.lasp_chunk_grads,
+                      lib.lasp_chunk_out, lib.lasp_chunk_grads, lib.lasp_bwd_noalloc,
                       lib.lasp_state_prefix, lib.lasp_check_device_status, lib.lasp_set_wait_limit_ns,
                       lib.lasp_wait_probe, lib.lasp_version):
                 f.restype = I
@@ -131,6 +132,16 @@ def lasp_bwd(q, k, v, decay, dout, dq, dk, dv, C, state_cache, dstate_ws, init_s
     _check(_load().lasp_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(decay), _ptr(dout), _ptr(dq), _ptr(dk), _ptr(dv),
                             B, H, N, d, C, dt, _ptr(state_cache), _ptr(dstate_ws), _ptr(init_state),
                             _ptr(dstate_in), _ptr(dinit_state), _stream(stream, q)), "lasp_bwd")
+
+
+def lasp_bwd_noalloc(q, k, v, decay, dout, dq, dk, dv, C, state_cache, dstate_in=None, dinit_state=None,
+                     stream=None):
+    """lasp_bwd for callers that cannot allocate: the gradient-state workspace is
+    a fixed array inside the library (see lasp.h for its limit and sharing rules)."""
+    B, N, H, d, dt = _tokens(q, k, v, dout, dq, dk, dv)
+    _check(_load().lasp_bwd_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(decay), _ptr(dout), _ptr(dq), _ptr(dk),
+                                    _ptr(dv), B, H, N, d, C, dt, _ptr(state_cache), _ptr(dstate_in),
+                                    _ptr(dinit_state), _stream(stream, q)), "lasp_bwd_noalloc")
 
 
 def lasp_chunk_states(q, k, v, decay, M, C, stream=None):

@@ -6,3 +6,4 @@
 #include "k_tc_states.cu"
 #include "k_tc_out.cu"
 #include "k_tc_bwd.cu"
+#include "lasp_noalloc.cu"
