@@ -20,7 +20,7 @@ namespace lasp {
 namespace scan_detail {
 
 constexpr int kUnroll = 16;
-constexpr int kThreads = 256;
+constexpr int kThreads = 64;  // small blocks spread the work evenly over the SMs
 
 __device__ __forceinline__ float4 fma4(float g, float4 a, float4 m) {
   return make_float4(fmaf(g, a.x, m.x), fmaf(g, a.y, m.y), fmaf(g, a.z, m.z), fmaf(g, a.w, m.w));

@@ -57,12 +57,21 @@ __device__ __forceinline__ void st_tile16(uint8_t* tile, int row, int col, uint4
 
 // fp32 d x d state [m][e] -> bf16 tile (row m, column e), all 128 threads.
 __device__ __forceinline__ void load_state_tile(uint8_t* tile, const float* src, int warp, int lane) {
+  // each warp converts rows warp, warp + 4, ...; all 16 loads of a batch are in flight together
   const float4* p = reinterpret_cast<const float4*>(src);
-  for (int r = warp; r < kD; r += kThreads / 32) {
-    const float4 x = __ldcs(p + r * (kD / 4) + lane);
-    const int col = lane * 4;
-    const uint32_t off = (col >> 6) * kBox + sw128_offset(r, (col & 63) >> 3) + (col & 7) * 2;
-    *reinterpret_cast<uint2*>(tile + off) = make_uint2(pack_bf16(x.x, x.y), pack_bf16(x.z, x.w));
+  constexpr int kBatch = 16;
+  const int col = lane * 4;
+#pragma unroll
+  for (int r0 = 0; r0 < kD / 4; r0 += kBatch) {
+    float4 x[kBatch];
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) x[u] = __ldcs(p + (warp + 4 * (r0 + u)) * (kD / 4) + lane);
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) {
+      const int r = warp + 4 * (r0 + u);
+      const uint32_t off = (col >> 6) * kBox + sw128_offset(r, (col & 63) >> 3) + (col & 7) * 2;
+      *reinterpret_cast<uint2*>(tile + off) = make_uint2(pack_bf16(x[u].x, x[u].y), pack_bf16(x[u].z, x[u].w));
+    }
   }
 }
 

@@ -110,12 +110,21 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_out_tc(const __grid_constan
   {
     const int c0 = row0 / C;
     const float4* Pc = reinterpret_cast<const float4*>(P + ((((int64_t)b * T + c0) * H + h) * kD) * kD);
-    for (int r = warp; r < kD; r += kThreads / 32) {
-      const float4 x = __ldcs(Pc + r * (kD / 4) + lane);
-      const int col = lane * 4;
-      uint8_t* box = sP + (col >> 6) * kBox;
-      const uint32_t off = sw128_offset(r, (col & 63) >> 3) + (col & 7) * 2;
-      *reinterpret_cast<uint2*>(box + off) = make_uint2(pack_bf16(x.x, x.y), pack_bf16(x.z, x.w));
+    // each warp converts rows warp, warp + 4, ...; all 16 loads of a batch are
+    // in flight together
+    constexpr int kBatch = 16;
+    const int col = lane * 4;
+#pragma unroll
+    for (int r0 = 0; r0 < kD / 4; r0 += kBatch) {
+      float4 x[kBatch];
+#pragma unroll
+      for (int u = 0; u < kBatch; ++u) x[u] = __ldcs(Pc + (warp + 4 * (r0 + u)) * (kD / 4) + lane);
+#pragma unroll
+      for (int u = 0; u < kBatch; ++u) {
+        const int r = warp + 4 * (r0 + u);
+        const uint32_t off = (col >> 6) * kBox + sw128_offset(r, (col & 63) >> 3) + (col & 7) * 2;
+        *reinterpret_cast<uint2*>(sP + off) = make_uint2(pack_bf16(x[u].x, x[u].y), pack_bf16(x[u].z, x[u].w));
+      }
     }
     fence_async_smem();
   }
