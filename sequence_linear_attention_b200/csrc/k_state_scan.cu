@@ -8,8 +8,8 @@
 // The scan is pure HBM traffic: every state element is read once and written
 // once. One thread owns one float4 of the d*d state of one (b, h) and walks the
 // chunks in order; the loads of a group of kUnroll chunks do not depend on the
-// recurrence, so they are all issued before the group's FMAs, keeping
-// kUnroll * 16 bytes in flight per thread. Consecutive threads own consecutive
+// recurrence, so they are issued one group ahead of the FMAs and stores,
+// keeping up to 2 * kUnroll * 16 bytes in flight per thread. Consecutive threads own consecutive
 // float4s of one state, so every warp access is a fully coalesced 512-byte run.
 // M and P may be the same array: each element is loaded before it is stored,
 // by the same thread.
@@ -19,7 +19,7 @@
 namespace lasp {
 namespace scan_detail {
 
-constexpr int kUnroll = 16;
+constexpr int kUnroll = 8;
 constexpr int kThreads = 64;  // small blocks spread the work evenly over the SMs
 
 __device__ __forceinline__ float4 fma4(float g, float4 a, float4 m) {
@@ -43,18 +43,33 @@ __global__ void __launch_bounds__(kThreads) state_scan_kernel(const float4* M, f
   const int64_t base = (b * T * H + h) * (int64_t)dd4 + e;
   const int64_t step = reverse ? -cstride : cstride;
   int64_t off = reverse ? base + (int64_t)(T - 1) * cstride : base;
-  int n = 0;
-  for (; n + kUnroll <= T; n += kUnroll) {
-    float4 m[kUnroll];
+  // software pipeline: the loads of group g + 1 are issued before group g is
+  // scanned and stored, so a group's worth of loads is always in flight
+  const int ngroups = T / kUnroll;
+  float4 cur[kUnroll];
+  if (ngroups > 0) {
 #pragma unroll
-    for (int u = 0; u < kUnroll; ++u) m[u] = __ldcs(M + off + u * step);
+    for (int u = 0; u < kUnroll; ++u) cur[u] = __ldcs(M + off + u * step);
+  }
+  for (int gi = 0; gi < ngroups; ++gi) {
+    const bool more = gi + 1 < ngroups;
+    float4 nxt[kUnroll];
+    if (more) {
+#pragma unroll
+      for (int u = 0; u < kUnroll; ++u) nxt[u] = __ldcs(M + off + (kUnroll + u) * step);
+    }
 #pragma unroll
     for (int u = 0; u < kUnroll; ++u) {
       __stcs(P + off + u * step, acc);
-      acc = fma4(g, acc, m[u]);
+      acc = fma4(g, acc, cur[u]);
     }
     off += kUnroll * step;
+    if (more) {
+#pragma unroll
+      for (int u = 0; u < kUnroll; ++u) cur[u] = nxt[u];
+    }
   }
+  int n = ngroups * kUnroll;
   for (; n < T; ++n) {
     float4 m = __ldcs(M + off);
     __stcs(P + off, acc);

@@ -10,9 +10,12 @@
 // over the whole tile regroup the per-chunk intra and inter terms (LASP Eq. 8,
 // 15, 18, 21).
 //
-// One CTA per (tile, head, batch), 128 threads (thread i owns row i in every
-// epilogue). Shared memory holds seven 32 KB bf16 tiles: Q, K, V, dO (TMA,
-// 128-byte swizzle), X (P, later R, converted from fp32), dP' and S'. Each
+// One CTA per (tile, head, batch), 256 threads; in every epilogue warp w owns
+// the TMEM lanes (rows) 32*(w%4).. and the column half w/4. Shared memory holds
+// seven 32 KB bf16 tiles: Q, K, V, dO (TMA, 128-byte swizzle), X (P, later R,
+// converted from fp32), dP' and S'. R arrives at the start by one bulk copy
+// into the dP'/S' space (64 KB of fp32, idle until epilogue 1) and moves to
+// registers before epilogue 1, so no global load waits in mid-kernel. Each
 // stored tile serves both as a K-major and as an MN-major operand, so no
 // transposed copy is made: dP' [i][j] is the K-major A of dP' K and the
 // MN-major A of dP'^T Q, and so on. The 512 TMEM columns hold four 128-column
@@ -34,13 +37,15 @@ using namespace sm100;
 
 constexpr int kD = 128;
 constexpr int kTile = 128;
-constexpr int kThreads = 128;
+constexpr int kThreads = 256;
+constexpr int kWarps = kThreads / 32;
+constexpr int kRowsPerWarp = 128 / kWarps;
 constexpr uint32_t kTileBytes = kTile * kD * 2;
 constexpr uint32_t kBox = kTileBytes / 2;
 constexpr uint32_t kTmemCols = 512;
 
 struct Smem {
-  uint64_t load, mma1a, mma1b, mma2, mma3;
+  uint64_t load, rload, mma1a, mma1b, mma2, mma3;
   uint32_t tmem_base;
   int abort;
   float pw[kTile];
@@ -55,24 +60,23 @@ __device__ __forceinline__ void st_tile16(uint8_t* tile, int row, int col, uint4
   *reinterpret_cast<uint4*>(tile + (col >> 6) * kBox + sw128_offset(row, (col & 63) >> 3)) = v;
 }
 
-// fp32 d x d state [m][e] -> bf16 tile (row m, column e), all 128 threads.
-__device__ __forceinline__ void load_state_tile(uint8_t* tile, const float* src, int warp, int lane) {
-  // each warp converts rows warp, warp + 4, ...; all 16 loads of a batch are in flight together
-  const float4* p = reinterpret_cast<const float4*>(src);
-  constexpr int kBatch = 16;
+// Row r of a d x d fp32 state [m][e], float4 `lane` (columns 4*lane..4*lane+3),
+// written as bf16 into the operand tile (row m, column e).
+__device__ __forceinline__ void put_state_row(uint8_t* tile, int r, int lane, float4 x) {
   const int col = lane * 4;
+  const uint32_t off = (col >> 6) * kBox + sw128_offset(r, (col & 63) >> 3) + (col & 7) * 2;
+  *reinterpret_cast<uint2*>(tile + off) = make_uint2(pack_bf16(x.x, x.y), pack_bf16(x.z, x.w));
+}
+
+// fp32 d x d state in global memory -> bf16 tile. Warp w converts rows w,
+// w + 8, ...; all of its loads are in flight together.
+__device__ __forceinline__ void load_state_tile(uint8_t* tile, const float* src, int warp, int lane) {
+  const float4* p = reinterpret_cast<const float4*>(src);
+  float4 x[kRowsPerWarp];
 #pragma unroll
-  for (int r0 = 0; r0 < kD / 4; r0 += kBatch) {
-    float4 x[kBatch];
+  for (int u = 0; u < kRowsPerWarp; ++u) x[u] = __ldcs(p + (warp + kWarps * u) * (kD / 4) + lane);
 #pragma unroll
-    for (int u = 0; u < kBatch; ++u) x[u] = __ldcs(p + (warp + 4 * (r0 + u)) * (kD / 4) + lane);
-#pragma unroll
-    for (int u = 0; u < kBatch; ++u) {
-      const int r = warp + 4 * (r0 + u);
-      const uint32_t off = (col >> 6) * kBox + sw128_offset(r, (col & 63) >> 3) + (col & 7) * 2;
-      *reinterpret_cast<uint2*>(tile + off) = make_uint2(pack_bf16(x[u].x, x[u].y), pack_bf16(x[u].z, x[u].w));
-    }
-  }
+  for (int u = 0; u < kRowsPerWarp; ++u) put_state_row(tile, warp + kWarps * u, lane, x[u]);
 }
 
 // K-major operand descriptor for K step kk (16 elements) of a 128 x 128 tile.
@@ -116,6 +120,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_bwd_tc(const __grid_constan
     prefetch_tmap(&map_v);
     prefetch_tmap(&map_do);
     mbar_init(&s->load, 1);
+    mbar_init(&s->rload, 1);
     mbar_init(&s->mma1a, 1);
     mbar_init(&s->mma1b, 1);
     mbar_init(&s->mma2, 1);
@@ -123,7 +128,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_bwd_tc(const __grid_constan
     s->abort = 0;
     fence_mbar_init();
   }
-  s->pw[tid] = decay_pow(l2, (float)tid);
+  if (tid < kTile) s->pw[tid] = decay_pow(l2, (float)tid);
   if (warp == 0) {
     tmem_alloc(&s->tmem_base, kTmemCols);
     tmem_relinquish();
@@ -132,7 +137,8 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_bwd_tc(const __grid_constan
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = s->tmem_base;
-  const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
+  const uint32_t lane_base = tmem + ((uint32_t)((warp & 3) * 32) << 16);
+  const int half = warp >> 2;  // column half of every epilogue
   const uint32_t T0 = 0, T1 = 128, T2 = 256, T3 = 384;
 
   if (tid == 0) {
@@ -147,6 +153,13 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_bwd_tc(const __grid_constan
     tma_load_4d(sD + kBox, &map_do, &s->load, 64, h, row0, b);
   }
   const int c_first = row0 / C, c_last = (row0 + last) / C;
+  if (tid == 32) {
+    // R of the tile's last chunk, fp32, into the (still unused) dP'/S' space
+    const float* Rc = R + ((((int64_t)b * T + c_last) * H + h) * kD) * kD;
+    mbar_arrive_expect_tx(&s->rload, kD * kD * 4);
+    for (int part = 0; part < 4; ++part)
+      bulk_load(sA + part * (kD * kD), Rc + part * (kD * kD / 4), kD * kD, &s->rload);
+  }
   load_state_tile(sX, P + ((((int64_t)b * T + c_first) * H + h) * kD) * kD, warp, lane);
   fence_async_smem();
   __syncthreads();
@@ -171,12 +184,23 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_bwd_tc(const __grid_constan
     }
   }
 
-  // ---- epilogue 1: masks, dP' -> sA, S' -> sB (row i = tid)
-  const int i = tid;
+  // ---- R (fp32, in the dP'/S' space) -> registers; that space is then free
+  float4 rreg[kRowsPerWarp];
+  if (mbar_wait(&s->rload, 0, SITE_BWD_TMA)) {
+    const float4* rs4 = reinterpret_cast<const float4*>(sA);
+#pragma unroll
+    for (int u = 0; u < kRowsPerWarp; ++u) rreg[u] = rs4[(warp + kWarps * u) * (kD / 4) + lane];
+  } else {
+    s->abort = 1;
+  }
+  __syncthreads();
+
+  // ---- epilogue 1: masks, dP' -> sA, S' -> sB (row i, column half `half`)
+  const int i = (warp & 3) * 32 + lane;
   if (mbar_wait(&s->mma1a, 0, SITE_BWD_MMA)) {
     tc_fence_after();
 #pragma unroll 1
-    for (int cc = 0; cc < kTile / 32; ++cc) {
+    for (int cc = 2 * half; cc < 2 * half + 2; ++cc) {
       uint32_t rp[32], rs[32];
       tmem_ld32(lane_base + T0 + cc * 32, rp);
       tmem_ld32(lane_base + T1 + cc * 32, rs);
@@ -199,10 +223,17 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_bwd_tc(const __grid_constan
                              pack_bf16(fs[6], fs[7])));
       }
     }
-    fence_async_smem();
   } else {
     s->abort = 1;
   }
+  // X is free once dQ_inter has read P: R (bf16) replaces it
+  if (mbar_wait(&s->mma1b, 0, SITE_BWD_MMA)) {
+#pragma unroll
+    for (int u = 0; u < kRowsPerWarp; ++u) put_state_row(sX, warp + kWarps * u, lane, rreg[u]);
+  } else {
+    s->abort = 1;
+  }
+  fence_async_smem();
   tc_fence_before();
   __syncthreads();
   if (s->abort) goto cleanup;
@@ -213,11 +244,6 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_bwd_tc(const __grid_constan
     for (int kk = 0; kk < kTile / 16; ++kk) mma_bf16(tmem + T3, kmaj(aA, kk), mnmaj(aK, kk), id_kn, kk != 0);
     mma_commit(&s->mma2);
   }
-  // X is free once dQ_inter has read P: bring in R of the tile's last chunk
-  if (!mbar_wait(&s->mma1b, 0, SITE_BWD_MMA)) s->abort = 1;
-  load_state_tile(sX, R + ((((int64_t)b * T + c_last) * H + h) * kD) * kD, warp, lane);
-  fence_async_smem();
-
   // ---- epilogue 2: dQ = T3 + lambda^{i+1} T2, stored straight to global
   if (!s->abort && mbar_wait(&s->mma2, 0, SITE_BWD_MMA)) {
     tc_fence_after();
@@ -225,7 +251,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_bwd_tc(const __grid_constan
     const bool valid = i <= last;
     __nv_bfloat16* out = dq + (((int64_t)b * N + row0 + i) * H + h) * kD;
 #pragma unroll 1
-    for (int cc = 0; cc < kD / 32; ++cc) {
+    for (int cc = 2 * half; cc < 2 * half + 2; ++cc) {
       uint32_t ra[32], re[32];
       tmem_ld32(lane_base + T3 + cc * 32, ra);
       tmem_ld32(lane_base + T2 + cc * 32, re);
@@ -259,13 +285,13 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_bwd_tc(const __grid_constan
     mma_commit(&s->mma3);
   }
 
-  // ---- epilogue 3: row j = tid; dK -> sA, dV -> sB, then TMA stores
+  // ---- epilogue 3: row j, column half `half`; dK -> sA, dV -> sB, then TMA stores
   if (mbar_wait(&s->mma3, 0, SITE_BWD_MMA)) {
     tc_fence_after();
-    const int j = tid;
+    const int j = i;
     const float wj = j <= last ? decay_pow(l2, (float)(last - j)) : 0.f;
 #pragma unroll 1
-    for (int cc = 0; cc < kD / 32; ++cc) {
+    for (int cc = 2 * half; cc < 2 * half + 2; ++cc) {
       uint32_t ka[32], ke[32];
       tmem_ld32(lane_base + T0 + cc * 32, ka);
       tmem_ld32(lane_base + T2 + cc * 32, ke);

@@ -7,7 +7,9 @@
 // as the per-chunk intra terms plus the inter terms of the chunks inside it
 // (LASP Eq. 8 regrouped), so only the first chunk's P is read.
 //
-// One CTA per (tile, head, batch), 128 threads; thread i owns output row i.
+// One CTA per (tile, head, batch), 256 threads. In the epilogues warp w reads
+// TMEM lanes 32*(w%4).. (the rows it may access) and the column half w/4, so
+// the two warpgroups share every epilogue.
 //  1. thread 0: TMA loads Q, K, V (128 x 128 bf16, two 64-feature boxes each,
 //     128-byte swizzle); all threads: P (fp32, 64 KB) -> bf16 into shared
 //     memory as an MN-major operand.
@@ -29,7 +31,7 @@ using namespace sm100;
 
 constexpr int kD = 128;
 constexpr int kTile = 128;
-constexpr int kThreads = 128;
+constexpr int kThreads = 256;
 constexpr uint32_t kTileBytes = kTile * kD * 2;  // 32 KB: two 16 KB boxes
 constexpr uint32_t kBox = kTileBytes / 2;
 constexpr uint32_t kTmemCols = 512;
@@ -86,7 +88,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_out_tc(const __grid_constan
     s->abort = 0;
     fence_mbar_init();
   }
-  s->pw[tid] = decay_pow(l2, (float)tid);
+  if (tid < kTile) s->pw[tid] = decay_pow(l2, (float)tid);
   if (warp == 0) {
     tmem_alloc(&s->tmem_base, kTmemCols);
     tmem_relinquish();
@@ -110,18 +112,16 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_out_tc(const __grid_constan
   {
     const int c0 = row0 / C;
     const float4* Pc = reinterpret_cast<const float4*>(P + ((((int64_t)b * T + c0) * H + h) * kD) * kD);
-    // each warp converts rows warp, warp + 4, ...; all 16 loads of a batch are
-    // in flight together
-    constexpr int kBatch = 16;
+    // warp w converts rows w, w + 8, ...: all 16 of its loads are in flight together
+    constexpr int kWarps = kThreads / 32, kRows = kD / kWarps;
     const int col = lane * 4;
+    {
+      float4 x[kRows];
 #pragma unroll
-    for (int r0 = 0; r0 < kD / 4; r0 += kBatch) {
-      float4 x[kBatch];
+      for (int u = 0; u < kRows; ++u) x[u] = __ldcs(Pc + (warp + kWarps * u) * (kD / 4) + lane);
 #pragma unroll
-      for (int u = 0; u < kBatch; ++u) x[u] = __ldcs(Pc + (warp + 4 * (r0 + u)) * (kD / 4) + lane);
-#pragma unroll
-      for (int u = 0; u < kBatch; ++u) {
-        const int r = warp + 4 * (r0 + u);
+      for (int u = 0; u < kRows; ++u) {
+        const int r = warp + kWarps * u;
         const uint32_t off = (col >> 6) * kBox + sw128_offset(r, (col & 63) >> 3) + (col & 7) * 2;
         *reinterpret_cast<uint2*>(sP + off) = make_uint2(pack_bf16(x[u].x, x[u].y), pack_bf16(x[u].z, x[u].w));
       }
@@ -153,14 +153,15 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_out_tc(const __grid_constan
     }
   }
 
-  // S' = Mask . S, row i = tid, written over the K tile as a K-major A operand
-  const int i = tid;
+  // S' = Mask . S, written over the K tile as a K-major A operand; this thread
+  // owns row i and the column half `half`
+  const int i = (warp & 3) * 32 + lane, half = warp >> 2;
   bool ok = mbar_wait(&s->s_done, 0, SITE_OUT_MMA);
   tc_fence_after();
   if (ok) {
-    const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
+    const uint32_t lane_base = tmem + ((uint32_t)((warp & 3) * 32) << 16);
 #pragma unroll 1
-    for (int cc = 0; cc < kTile / 32; ++cc) {
+    for (int cc = 2 * half; cc < 2 * half + 2; ++cc) {
       uint32_t r[32];
       tmem_ld32(lane_base + kColS + cc * 32, r);
       tmem_ld_wait();
@@ -199,9 +200,9 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_out_tc(const __grid_constan
   tc_fence_after();
   if (ok) {
     const float wi = decay_pow(l2, (float)(i + 1));
-    const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
+    const uint32_t lane_base = tmem + ((uint32_t)((warp & 3) * 32) << 16);
 #pragma unroll 1
-    for (int cc = 0; cc < kD / 32; ++cc) {
+    for (int cc = 2 * half; cc < 2 * half + 2; ++cc) {
       uint32_t a[32], e[32];
       tmem_ld32(lane_base + kColIntra + cc * 32, a);
       tmem_ld32(lane_base + kColInter + cc * 32, e);
