@@ -30,7 +30,8 @@ __global__ void __launch_bounds__(kThreads) state_scan_kernel(const float4* M, f
                                                               const float4* __restrict__ init,
                                                               float4* __restrict__ total, int H, int T,
                                                               int dd4, int64_t n_threads, float Cf,
-                                                              int reverse) {
+                                                              int reverse, int64_t t_slots, int slot_stride,
+                                                              int slot_offset) {
   const int64_t idx = (int64_t)blockIdx.x * kThreads + threadIdx.x;
   if (idx >= n_threads) return;
   const int e = (int)(idx % dd4);
@@ -39,8 +40,9 @@ __global__ void __launch_bounds__(kThreads) state_scan_kernel(const float4* M, f
   const float g = decay_pow(log2f(load_decay(decay, h)), Cf);
   const int64_t bh = b * H + h;
   float4 acc = init ? init[bh * dd4 + e] : make_float4(0.f, 0.f, 0.f, 0.f);
-  const int64_t cstride = (int64_t)H * dd4;  // float4s between chunk c and c+1
-  const int64_t base = (b * T * H + h) * (int64_t)dd4 + e;
+  // scan element c lives in slot c * slot_stride + slot_offset of an array of t_slots states
+  const int64_t cstride = (int64_t)slot_stride * H * dd4;  // float4s between element c and c+1
+  const int64_t base = ((b * t_slots + slot_offset) * H + h) * (int64_t)dd4 + e;
   const int64_t step = reverse ? -cstride : cstride;
   int64_t off = reverse ? base + (int64_t)(T - 1) * cstride : base;
   // software pipeline: the loads of group g + 1 are issued before group g is
@@ -81,15 +83,21 @@ __global__ void __launch_bounds__(kThreads) state_scan_kernel(const float4* M, f
 
 }  // namespace scan_detail
 
-cudaError_t launch_state_scan(const float* M, float* P, const float* decay, const float* init, float* total,
-                              int B, int T, int H, int d, int64_t C, int reverse, cudaStream_t st) {
+cudaError_t launch_state_scan_slots(const float* M, float* P, const float* decay, const float* init, float* total,
+                                    int B, int T, int H, int d, int64_t C, int reverse, int64_t t_slots,
+                                    int slot_stride, int slot_offset, cudaStream_t st) {
   const int dd4 = d * d / 4;
   const int64_t n_threads = (int64_t)B * H * dd4;
   const int64_t blocks = (n_threads + scan_detail::kThreads - 1) / scan_detail::kThreads;
   scan_detail::state_scan_kernel<<<(unsigned)blocks, scan_detail::kThreads, 0, st>>>(
       (const float4*)M, (float4*)P, decay, (const float4*)init, (float4*)total, H, T, dd4, n_threads,
-      (float)C, reverse);
+      (float)C, reverse, t_slots, slot_stride, slot_offset);
   return cudaGetLastError();
+}
+
+cudaError_t launch_state_scan(const float* M, float* P, const float* decay, const float* init, float* total,
+                              int B, int T, int H, int d, int64_t C, int reverse, cudaStream_t st) {
+  return launch_state_scan_slots(M, P, decay, init, total, B, T, H, d, C, reverse, T, 1, 0, st);
 }
 
 }  // namespace lasp

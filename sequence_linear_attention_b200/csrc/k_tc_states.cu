@@ -61,7 +61,8 @@ __device__ __forceinline__ void issue_stage(uint8_t* tiles, uint32_t tile_bytes,
 __global__ void __launch_bounds__(kThreads, 1) chunk_states_tc(const __grid_constant__ CUtensorMap map_a,
                                                             const __grid_constant__ CUtensorMap map_b,
                                                             const float* decay, float* __restrict__ M, int H,
-                                                            int C, int KB, int kind) {
+                                                            int C, int KB, int kind, int64_t t_out,
+                                                            int slot_stride, int slot_offset) {
   extern __shared__ uint8_t smem_raw[];
   // tiles need 1024-byte alignment for the 128-byte swizzle atoms
   uint8_t* tiles = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
@@ -72,7 +73,6 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_states_tc(const __grid_cons
 
   const int c = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int64_t T = gridDim.x;
   const float lam = load_decay(decay, h);
   const float l2 = log2f(lam);
   const bool scale = lam != 1.0f;
@@ -149,7 +149,9 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_states_tc(const __grid_cons
   tc_fence_after();
   if (ok) {
     const int row = warp * 32 + lane;
-    float* out = M + ((((int64_t)b * T + c) * H + h) * kD + row) * kD;
+    // chunk c's state goes to slot c * slot_stride + slot_offset of an array with t_out slots
+    const int64_t slot = (int64_t)c * slot_stride + slot_offset;
+    float* out = M + ((((int64_t)b * t_out + slot) * H + h) * kD + row) * kD;
 #pragma unroll 1
     for (int cc = 0; cc < kD / 32; ++cc) {
       uint32_t r[32];
@@ -179,8 +181,9 @@ bool tc_states_ok(int dtype, int d, int64_t C) {
   return dtype == LASP_BF16 && d == tc_states_detail::kD && C % 16 == 0;
 }
 
-cudaError_t tc_chunk_states(const void* a, const void* bm, const float* decay, float* M, int B, int H, int64_t N,
-                            int d, int C, int kind, cudaStream_t st) {
+cudaError_t tc_chunk_states_slots(const void* a, const void* bm, const float* decay, float* M, int B, int H,
+                                  int64_t N, int d, int C, int kind, int64_t t_out, int slot_stride, int slot_offset,
+                                  cudaStream_t st) {
   using namespace tc_states_detail;
   const int KB = stage_rows(C);
   CUtensorMap ma, mb;
@@ -191,8 +194,13 @@ cudaError_t tc_chunk_states(const void* a, const void* bm, const float* decay, f
   cudaError_t e = cudaFuncSetAttribute(chunk_states_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   dim3 grid((unsigned)(N / C), H, B);
-  chunk_states_tc<<<grid, kThreads, smem, st>>>(ma, mb, decay, M, H, C, KB, kind);
+  chunk_states_tc<<<grid, kThreads, smem, st>>>(ma, mb, decay, M, H, C, KB, kind, t_out, slot_stride, slot_offset);
   return cudaGetLastError();
+}
+
+cudaError_t tc_chunk_states(const void* a, const void* bm, const float* decay, float* M, int B, int H, int64_t N,
+                            int d, int C, int kind, cudaStream_t st) {
+  return tc_chunk_states_slots(a, bm, decay, M, B, H, N, d, C, kind, N / C, 1, 0, st);
 }
 
 }  // namespace lasp

@@ -11,6 +11,12 @@ namespace lasp {
 cudaError_t launch_state_scan(const float* M, float* P, const float* decay, const float* init, float* total,
                               int B, int T, int H, int d, int64_t C, int reverse, cudaStream_t st);
 
+// The same scan over every slot_stride-th state of an array of t_slots states,
+// starting at slot slot_offset (segment states stored inside a chunk array).
+cudaError_t launch_state_scan_slots(const float* M, float* P, const float* decay, const float* init, float* total,
+                                    int B, int T, int H, int d, int64_t C, int reverse, int64_t t_slots,
+                                    int slot_stride, int slot_offset, cudaStream_t st);
+
 // CUDA-core kernels, any d in {32, 64, 128} and any C (k_simt.cu).
 // kind 0: M_c = sum lambda^{C-1-t} a_t^T b_t ; kind 1: sum lambda^{t+1} a_t^T b_t.
 cudaError_t simt_chunk_states(const void* a, const void* b, const float* decay, float* M, int B, int H,

@@ -52,6 +52,13 @@ int chunk_states_impl(const void* a, const void* b, const float* decay, float* M
   return cuda_status(simt_chunk_states(a, b, decay, M, B, H, N, d, C, kind, dtype, st));
 }
 
+int num_sms_current_device() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) return 148;
+  return n;
+}
+
 int chunk_out_impl(const void* q, const void* k, const void* v, const float* decay, const float* P, void* o, int B,
                    int H, int64_t N, int d, int C, int dtype, cudaStream_t st) {
   if (tc_out_ok(dtype, d, C)) return cuda_status(tc_chunk_out(q, k, v, decay, P, o, B, H, N, d, C, st));
@@ -130,6 +137,19 @@ int lasp_fwd(const void* q, const void* k, const void* v, const float* decay, vo
   if ((s = check_ptrs({q, k, v, o, state_cache}, {decay, init_state}))) return s;
   cudaStream_t st = (cudaStream_t)stream;
   const int T = (int)(N / C);
+  if (tc_fwd_walk_ok(dtype, d, C)) {
+    // segments of G tokens: their states go to the slots of their first chunks,
+    // the exclusive prefix over segments turns them into P of those chunks, and
+    // the walk carries the state through each segment, filling the other slots
+    const int G = walk_segment_tokens(N, C);
+    const int stride = G / C;
+    if ((s = cuda_status(tc_chunk_states_slots(k, v, decay, state_cache, B, H, N, d, G, 0, T, stride, 0, st))))
+      return s;
+    if ((s = cuda_status(launch_state_scan_slots(state_cache, state_cache, decay, init_state, nullptr, B,
+                                                 (int)(N / G), H, d, G, 0, T, stride, 0, st))))
+      return s;
+    return cuda_status(tc_fwd_walk(q, k, v, decay, state_cache, o, B, H, N, d, C, G, num_sms_current_device(), st));
+  }
   // 1. chunk states M_c into the cache; 2. exclusive prefix in place -> P_c; 3. output.
   if ((s = chunk_states_impl(k, v, decay, state_cache, B, H, N, d, C, dtype, 0, st))) return s;
   if ((s = cuda_status(launch_state_scan(state_cache, state_cache, decay, init_state, nullptr, B, T, H, d, C, 0, st))))

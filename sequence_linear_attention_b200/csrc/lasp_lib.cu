@@ -5,5 +5,6 @@
 #include "k_simt.cu"
 #include "k_tc_states.cu"
 #include "k_tc_out.cu"
+#include "k_tc_fwd_walk.cu"
 #include "k_tc_bwd.cu"
 #include "lasp_noalloc.cu"

@@ -14,6 +14,21 @@ bool tc_states_ok(int dtype, int d, int64_t C);
 cudaError_t tc_chunk_states(const void* a, const void* b, const float* decay, float* M, int B, int H, int64_t N,
                             int d, int C, int kind, cudaStream_t st);
 
+// The same, writing chunk c's state to slot c * slot_stride + slot_offset of
+// an array of t_out states per (b, h).
+cudaError_t tc_chunk_states_slots(const void* a, const void* b, const float* decay, float* M, int B, int H,
+                                  int64_t N, int d, int C, int kind, int64_t t_out, int slot_stride, int slot_offset,
+                                  cudaStream_t st);
+
+// Forward walk over segments of G tokens with the state on chip (bf16,
+// d = 128, C a multiple of 128, G a multiple of C dividing N). P must hold,
+// in the slot of each segment's first chunk, the state entering that segment;
+// the walk fills the other chunks' slots and writes o.
+bool tc_fwd_walk_ok(int dtype, int d, int64_t C);
+int walk_segment_tokens(int64_t N, int C);
+cudaError_t tc_fwd_walk(const void* q, const void* k, const void* v, const float* decay, float* P, void* o, int B,
+                        int H, int64_t N, int d, int C, int G, int num_sms, cudaStream_t st);
+
 bool tc_out_ok(int dtype, int d, int64_t C);
 cudaError_t tc_chunk_out(const void* q, const void* k, const void* v, const float* decay, const float* P, void* o,
                          int B, int H, int64_t N, int d, int C, cudaStream_t st);

@@ -42,6 +42,9 @@ SMALL = [
     (1, 2, 96, 64, 24, True, True),      # C not a multiple of 16
     (1, 2, 128, 128, 128, True, True),   # a single chunk
     (2, 2, 64, 64, 1, False, True),      # C = 1: pure inter-chunk
+    (1, 2, 2048, 128, 128, True, True),  # forward walk over two 1024-token segments
+    (2, 3, 1536, 128, 256, True, True),  # chunks of two tiles
+    (1, 2, 1024, 128, 512, True, False),
 ]
 
 
@@ -52,11 +55,11 @@ def test_small_shapes_against_oracle(B, H, N, d, C, bf16, decayed):
     _compare(gpu, _oracle_all(inp, C), bf16)
 
 
-@pytest.mark.parametrize("bf16", [False, True])
-def test_entering_states_against_oracle(bf16):
+@pytest.mark.parametrize("bf16,N,C", [(False, 256, 64), (True, 256, 64), (True, 2048, 128)])
+def test_entering_states_against_oracle(bf16, N, C):
     """init_state (the forward state entering token 0) and dstate_in (the
     gradient state entering from beyond the end), plus dinit_state."""
-    B, H, N, d, C = 2, 3, 256, 128 if bf16 else 32, 64
+    B, H, d = 2, 3, 128 if bf16 else 32
     inp = lasp_inputs.make_inputs(B, N, H, d, seed=77, bf16=bf16, decayed=True)
     rng = np.random.default_rng(78)
     init = (rng.standard_normal((B, H, d, d)) * 0.2).astype(np.float32)
