@@ -1,10 +1,10 @@
 """Benchmark: chunked causal linear attention forward + backward on B200.
 
 One step = one pass of the whole hot path over one batch of synthetic input:
-chunk states, exclusive prefix, output (the forward pass), gradient states,
-exclusive suffix, dQ/dK/dV (the backward pass). The step issues these six
-library calls on one stream -- the same kernels lasp_fwd and lasp_bwd issue --
-with CUDA events between them, so each kernel's duration is measured live.
+lasp_fwd (states, prefix, output) then lasp_bwd (gradient states, suffix,
+dQ/dK/dV), as a user calls them. The library's trace brackets each of its
+kernel launches with CUDA events on the same stream, so every kernel's
+duration is measured live inside the timed region.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                     [--workload NAME]
@@ -33,24 +33,35 @@ from sequence_linear_attention_b200 import inputs as lasp_inputs  # noqa: E402
 
 METRIC = "linear-attn fwd+bwd tokens/s (H16 d128 N64K bf16); % of bf16 tensor peak"
 DEFAULT_WORKLOAD = "decayed_bf16_N64K"
-KERNELS = ("chunk_states", "state_prefix", "chunk_out", "chunk_dstates", "state_suffix", "chunk_grads")
 
 
 # ------------------------------------------------------------ algorithmic work
-def algorithmic_bytes(name: str, tokens_heads: int, d: int, C: int, elem: int) -> float:
-    """Bytes each kernel must move, per launch: token tensors once, states once.
+def algorithmic_bytes(name: str, tokens_heads: int, d: int, C: int, G: int, elem: int) -> float:
+    """Bytes a kernel must move per launch: each token tensor once, each state once.
 
-    Per token-head, with e = element size and s = d*d*4/C (one fp32 state per
-    chunk spread over its C tokens):
-      chunk_states / chunk_dstates: read 2 token rows, write one state  = 2de + s
-      state_prefix / state_suffix:  read and write one state            = 2s
-      chunk_out:   read q, k, v and P, write o                         = 4de + s
-      chunk_grads: read q, k, v, dO, P and R, write dq, dk, dv          = 7de + 2s
+    Per token-head, with e = element size, s = 4 d^2 (one fp32 state), C the
+    chunk and G the segment length in tokens:
+      chunk_states_* (M_c or dM_c):  read 2 token rows, write s/C        = 2de + s/C
+      segment_states_tc:             read 2 token rows, write s/G        = 2de + s/G
+      state_scan:                    read and write s/C                  = 2s/C
+      segment_scan:                  read and write s/G                  = 2s/G
+      chunk_out_*:                   read q, k, v and P, write o         = 4de + s/C
+      fwd_walk_tc:  read q, k, v and the segment's P (s/G), write o and
+                    the other chunks' P (s/C - s/G)                      = 4de + s/C
+      chunk_bwd_*:  read q, k, v, dO, P and R, write dq, dk, dv          = 7de + 2s/C
+      bwd_walk_tc:  read q, k, v, dO, P and the segment's R (s/G), write
+                    dq, dk, dv and the other chunks' R (s/C - s/G)       = 7de + 2s/C
     """
-    s = d * d * 4 / C
-    per = {"chunk_states": 2 * d * elem + s, "chunk_dstates": 2 * d * elem + s,
-           "state_prefix": 2 * s, "state_suffix": 2 * s,
-           "chunk_out": 4 * d * elem + s, "chunk_grads": 7 * d * elem + 2 * s}[name]
+    s = 4 * d * d
+    de = d * elem
+    per = {
+        "chunk_states_tc": 2 * de + s / C, "chunk_states_simt": 2 * de + s / C,
+        "segment_states_tc": 2 * de + s / G,
+        "state_scan": 2 * s / C, "segment_scan": 2 * s / G,
+        "chunk_out_tc": 4 * de + s / C, "chunk_out_simt": 4 * de + s / C, "fwd_walk_tc": 4 * de + s / C,
+        "chunk_bwd_tc": 7 * de + 2 * s / C, "chunk_bwd_simt": 7 * de + 2 * s / C,
+        "bwd_walk_tc": 7 * de + 2 * s / C,
+    }[name]
     return per * tokens_heads
 
 
@@ -193,24 +204,11 @@ def run_gpu(args, rank, world, local):
     P = torch.empty((B, T, H, d, d), dtype=torch.float32, device=dev)
     R = torch.empty_like(P)
     stream = torch.cuda.current_stream(dev)
+    G = lasp.lasp_segment_tokens(N, C, d, 1 if bf16 else 0)
 
-    def step(evs=None):
-        def mark(i):
-            if evs is not None:
-                evs[i].record(stream)
-        mark(0)
-        lasp.lasp_chunk_states(None, k, v, decay, P, C)
-        mark(1)
-        lasp.lasp_state_prefix(P, P, decay, C)
-        mark(2)
-        lasp.lasp_chunk_out(q, k, v, decay, P, o, C)
-        mark(3)
-        lasp.lasp_chunk_dstates(q, do, decay, R, C)
-        mark(4)
-        lasp.lasp_state_prefix(R, R, decay, C, reverse=True)
-        mark(5)
-        lasp.lasp_chunk_grads(q, k, v, do, decay, P, R, dq, dk, dvv, C)
-        mark(6)
+    def step():
+        lasp.lasp_fwd(q, k, v, decay, o, C, P)
+        lasp.lasp_bwd(q, k, v, decay, do, dq, dk, dvv, C, P, R)
 
     for _ in range(args.warmup):
         step()
@@ -218,22 +216,27 @@ def run_gpu(args, rank, world, local):
     if st != 0:
         raise RuntimeError(f"device status {lasp.lasp_status_string(st)} at site {site}")
 
-    events = [[torch.cuda.Event(enable_timing=True) for _ in range(7)] for _ in range(args.steps)]
+    # the library brackets each of its kernel launches with CUDA events on this
+    # stream, so every kernel's duration is measured inside the timed region
+    events = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    lasp.lasp_trace_enable(16 * args.steps + 16)
     torch.cuda.synchronize(dev)
     barrier(world, dev)
     torch.cuda.synchronize(dev)
     with ClockSampler(local) as clk:
         for i in range(args.steps):
-            step(events[i])
+            events[i][0].record(stream)
+            step()
+            events[i][1].record(stream)
         torch.cuda.synchronize(dev)
     barrier(world, dev)
     torch.cuda.synchronize(dev)
-    per_kernel = {n: [] for n in KERNELS}
-    total_ms = 0.0
-    for evs in events:
-        total_ms += evs[0].elapsed_time(evs[6])
-        for j, n in enumerate(KERNELS):
-            per_kernel[n].append(evs[j].elapsed_time(evs[j + 1]))
+    trace = lasp.lasp_trace_read(16 * args.steps + 16)
+    lasp.lasp_trace_enable(0)
+    per_kernel = {}
+    for name, ms in trace:
+        per_kernel.setdefault(name, []).append(ms)
+    total_ms = sum(a.elapsed_time(b) for a, b in events)
     tokens = B * N
     value, t_max = aggregate(tokens * args.steps, total_ms / 1e3, world, dev)
     ms_per_step = t_max * 1e3 / args.steps
@@ -266,13 +269,15 @@ def run_gpu(args, rank, world, local):
 
     peaks = load_peaks()
     th = tokens * H
-    avg = {n: statistics.mean(per_kernel[n]) for n in KERNELS}
-    top = max(KERNELS, key=lambda n: avg[n])
-    achieved = algorithmic_bytes(top, th, d, C, elem) / (avg[top] / 1e3) / 1e9
-    kernel_table = {n: {"ms": round(avg[n], 4),
-                        "GBps": round(algorithmic_bytes(n, th, d, C, elem) / (avg[n] / 1e3) / 1e9, 1),
-                        "hbm_frac": round(algorithmic_bytes(n, th, d, C, elem) / (avg[n] / 1e3) / 1e9
-                                          / peaks["hbm"], 4)} for n in KERNELS}
+    names = list(per_kernel)
+    top = max(names, key=lambda n: sum(per_kernel[n]))
+    kernel_table = {}
+    for n in names:
+        mean = statistics.mean(per_kernel[n])
+        gbps = algorithmic_bytes(n, th, d, C, G, elem) / (mean / 1e3) / 1e9
+        kernel_table[n] = {"launches_per_step": len(per_kernel[n]) / args.steps, "ms": round(mean, 4),
+                           "GBps": round(gbps, 1), "hbm_frac": round(gbps / peaks["hbm"], 4)}
+    achieved = kernel_table[top]["GBps"]
     flops = flops_per_step(th, d, C)
     tflops = flops / (ms_per_step / 1e3) / 1e12
     line = {
@@ -280,7 +285,7 @@ def run_gpu(args, rank, world, local):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "bf16" if bf16 else "f32", "data": "synthetic (seeded normal q,k,v,dO; no dataset)",
-        "config": {"workload": args.workload, "B": B, "H": H, "N": N, "d": d, "C": C,
+        "config": {"workload": args.workload, "B": B, "H": H, "N": N, "d": d, "C": C, "segment": G,
                    "decay": "per-head 1-2^-(5+8h/H)" if w["decayed"] else "none",
                    "l2": "inputs larger than L2 (q, k, v, dO are 4 x %d MiB)" % (B * N * H * d * elem >> 20),
                    "parallelism": f"replicas x{world} (independent sequences, no collective)"},
@@ -293,7 +298,7 @@ def run_gpu(args, rank, world, local):
         "e2e": {"value": round(e2e_value, 1), "unit": "tokens/s",
                 "h2d_bytes_per_step": 4 * B * N * H * d * elem, "d2h_bytes_per_step": 4 * B * N * H * d * elem,
                 "api": "lasp_fwd + lasp_bwd with pinned host buffers"},
-        "gpu_launches": 6 * args.steps,
+        "gpu_launches": len(trace),
         "clocks": clk.summary(),
     }
     return line

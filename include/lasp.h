@@ -224,6 +224,31 @@ LASP_API int lasp_check_device_status(void* stream, int* site);
 LASP_API const char* lasp_status_string(int status);
 
 /*
+ * Tracing (a measurement aid; the pages have no counterpart). While enabled,
+ * the library brackets each of its kernel launches with two CUDA events on
+ * the launch's stream, for up to `capacity` launches.
+ *   lasp_trace_enable(capacity): creates the events (no device memory); 0
+ *     turns tracing off. Resets the record. Not for concurrent callers.
+ *   lasp_trace_read(ids, ms, capacity): waits for the recorded launches,
+ *     writes each one's kernel id and duration in milliseconds, clears the
+ *     record and returns how many it wrote (a negative status on error).
+ *   lasp_kernel_name(id): the kernel's name (static storage).
+ */
+LASP_API int lasp_trace_enable(int capacity);
+LASP_API int lasp_trace_read(int* kernel_ids, float* ms, int capacity);
+LASP_API const char* lasp_kernel_name(int kernel_id);
+
+/*
+ * lasp_segment_tokens -- the segment length G (tokens) that lasp_fwd uses for
+ * a problem of N tokens with chunk size C, head dimension d and `dtype`: the
+ * per-segment states and their prefix go to the state_cache slots of each
+ * segment's first chunk and a walk carries the state through the segment.
+ * Equals C when lasp_fwd computes every chunk state separately; 0 for
+ * invalid sizes.
+ */
+LASP_API int lasp_segment_tokens(int64_t N, int C, int d, int dtype);
+
+/*
  * lasp_set_wait_limit_ns -- sets, for the current device, the time after which
  * a spin-wait inside a kernel gives up, records LASP_ERR_TIMEOUT and lets the
  * kernel return (default 2e9 ns). Synchronous. Used by tests.

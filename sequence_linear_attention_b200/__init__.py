@@ -21,7 +21,8 @@ __all__ = [
     "LaspError", "library_path", "lasp_fwd", "lasp_bwd", "lasp_chunk_states", "lasp_chunk_dstates",
     "lasp_chunk_out", "lasp_chunk_grads", "lasp_bwd_noalloc",
     "lasp_state_prefix", "lasp_check_device_status", "lasp_set_wait_limit_ns", "lasp_wait_probe",
-    "lasp_status_string", "lasp_version",
+    "lasp_status_string", "lasp_version", "lasp_trace_enable", "lasp_trace_read", "lasp_kernel_name",
+    "lasp_segment_tokens",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -67,12 +68,18 @@ def _load():
             lib.lasp_check_device_status.argtypes = [P, ctypes.POINTER(I)]
             lib.lasp_set_wait_limit_ns.argtypes = [U64]
             lib.lasp_wait_probe.argtypes = [P]
+            lib.lasp_trace_enable.argtypes = [I]
+            lib.lasp_trace_read.argtypes = [P, P, I]
+            lib.lasp_kernel_name.argtypes = [I]
+            lib.lasp_kernel_name.restype = ctypes.c_char_p
+            lib.lasp_segment_tokens.argtypes = [L, I, I, I]
             lib.lasp_status_string.argtypes = [I]
             lib.lasp_status_string.restype = ctypes.c_char_p
             for f in (lib.lasp_fwd, lib.lasp_bwd, lib.lasp_chunk_states, lib.lasp_chunk_dstates,
                       lib.lasp_chunk_out, lib.lasp_chunk_grads, lib.lasp_bwd_noalloc,
                       lib.lasp_state_prefix, lib.lasp_check_device_status, lib.lasp_set_wait_limit_ns,
-                      lib.lasp_wait_probe, lib.lasp_version):
+                      lib.lasp_wait_probe, lib.lasp_version, lib.lasp_trace_enable, lib.lasp_trace_read,
+                      lib.lasp_segment_tokens):
                 f.restype = I
             _lib = lib
     return _lib
@@ -200,6 +207,30 @@ def lasp_wait_probe(stream=None):
     import torch
     s = stream if stream is not None else torch.cuda.current_stream().cuda_stream
     _check(_load().lasp_wait_probe(s if isinstance(s, int) else s.cuda_stream), "lasp_wait_probe")
+
+
+def lasp_trace_enable(capacity: int):
+    """Bracket each library kernel launch with CUDA events (up to `capacity`); 0 turns it off."""
+    _check(_load().lasp_trace_enable(int(capacity)), "lasp_trace_enable")
+
+
+def lasp_trace_read(capacity: int = 4096):
+    """[(kernel_name, milliseconds)] of the launches recorded since the last read."""
+    ids = (ctypes.c_int * capacity)()
+    ms = (ctypes.c_float * capacity)()
+    n = _load().lasp_trace_read(ids, ms, capacity)
+    if n < 0:
+        raise LaspError(-n, "lasp_trace_read")
+    return [(lasp_kernel_name(ids[i]), float(ms[i])) for i in range(n)]
+
+
+def lasp_kernel_name(kernel_id: int) -> str:
+    return _load().lasp_kernel_name(int(kernel_id)).decode()
+
+
+def lasp_segment_tokens(N: int, C: int, d: int, dtype_code: int) -> int:
+    """Segment length lasp_fwd uses (see lasp.h)."""
+    return int(_load().lasp_segment_tokens(int(N), int(C), int(d), int(dtype_code)))
 
 
 def lasp_status_string(status: int) -> str:

@@ -3,6 +3,9 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <mutex>
+#include <vector>
+
 #include "kernels.h"
 #include "lasp_common.cuh"
 #include "sm100.cuh"
@@ -11,6 +14,46 @@
 namespace lasp {
 
 namespace api_detail {
+
+// ---------------------------------------------------------------- tracing
+// Kernel identities reported by lasp_trace_read / lasp_kernel_name.
+enum KernelId : int {
+  K_STATES_TC = 1,      // per-chunk states, tensor cores
+  K_STATES_SIMT = 2,    // per-chunk states, CUDA cores
+  K_SCAN = 3,           // per-chunk prefix / suffix
+  K_OUT_TC = 4,         // output, one tile per CTA
+  K_OUT_SIMT = 5,
+  K_BWD_TC = 6,         // dQ/dK/dV, one tile per CTA
+  K_BWD_SIMT = 7,
+  K_FWD_WALK = 8,       // output walk over segments
+  K_BWD_WALK = 9,       // dQ/dK/dV walk over segments
+  K_SEG_STATES = 10,    // segment states (tensor cores)
+  K_SEG_SCAN = 11,      // prefix / suffix over segments
+  K_PROBE = 12,
+  K_COUNT
+};
+
+struct Trace {
+  std::mutex mu;
+  std::vector<cudaEvent_t> ev;
+  std::vector<int> ids;
+  int n = 0;
+  int cap = 0;
+};
+Trace g_trace;
+
+// Runs `launch`; while tracing is on, brackets it with two events on `st`.
+template <class F>
+cudaError_t traced(int id, cudaStream_t st, F&& launch) {
+  if (g_trace.cap == 0) return launch();
+  std::lock_guard<std::mutex> lock(g_trace.mu);
+  if (g_trace.n >= g_trace.cap) return launch();
+  cudaEventRecord(g_trace.ev[2 * g_trace.n], st);
+  cudaError_t e = launch();
+  cudaEventRecord(g_trace.ev[2 * g_trace.n + 1], st);
+  g_trace.ids[g_trace.n++] = id;
+  return e;
+}
 
 __global__ void wait_probe_kernel() {
   __shared__ __align__(8) uint64_t bar;
@@ -48,8 +91,16 @@ inline int cuda_status(cudaError_t e) { return e == cudaSuccess ? LASP_OK : LASP
 
 int chunk_states_impl(const void* a, const void* b, const float* decay, float* M, int B, int H, int64_t N, int d,
                       int C, int dtype, int kind, cudaStream_t st) {
-  if (tc_states_ok(dtype, d, C)) return cuda_status(tc_chunk_states(a, b, decay, M, B, H, N, d, C, kind, st));
-  return cuda_status(simt_chunk_states(a, b, decay, M, B, H, N, d, C, kind, dtype, st));
+  if (tc_states_ok(dtype, d, C))
+    return cuda_status(traced(K_STATES_TC, st, [&] { return tc_chunk_states(a, b, decay, M, B, H, N, d, C, kind, st); }));
+  return cuda_status(
+      traced(K_STATES_SIMT, st, [&] { return simt_chunk_states(a, b, decay, M, B, H, N, d, C, kind, dtype, st); }));
+}
+
+int scan_impl(int id, const float* M, float* P, const float* decay, const float* init, float* total, int B, int T,
+              int H, int d, int64_t C, int reverse, cudaStream_t st) {
+  return cuda_status(
+      traced(id, st, [&] { return launch_state_scan(M, P, decay, init, total, B, T, H, d, C, reverse, st); }));
 }
 
 int num_sms_current_device() {
@@ -61,15 +112,20 @@ int num_sms_current_device() {
 
 int chunk_out_impl(const void* q, const void* k, const void* v, const float* decay, const float* P, void* o, int B,
                    int H, int64_t N, int d, int C, int dtype, cudaStream_t st) {
-  if (tc_out_ok(dtype, d, C)) return cuda_status(tc_chunk_out(q, k, v, decay, P, o, B, H, N, d, C, st));
-  return cuda_status(simt_chunk_out(q, k, v, decay, P, o, B, H, N, d, C, dtype, st));
+  if (tc_out_ok(dtype, d, C))
+    return cuda_status(traced(K_OUT_TC, st, [&] { return tc_chunk_out(q, k, v, decay, P, o, B, H, N, d, C, st); }));
+  return cuda_status(
+      traced(K_OUT_SIMT, st, [&] { return simt_chunk_out(q, k, v, decay, P, o, B, H, N, d, C, dtype, st); }));
 }
 
 int chunk_grads_impl(const void* q, const void* k, const void* v, const void* dout, const float* decay,
                      const float* P, const float* R, void* dq, void* dk, void* dv, int B, int H, int64_t N, int d,
                      int C, int dtype, cudaStream_t st) {
-  if (tc_bwd_ok(dtype, d, C)) return cuda_status(tc_chunk_bwd(q, k, v, dout, decay, P, R, dq, dk, dv, B, H, N, d, C, st));
-  return cuda_status(simt_chunk_bwd(q, k, v, dout, decay, P, R, dq, dk, dv, B, H, N, d, C, dtype, st));
+  if (tc_bwd_ok(dtype, d, C))
+    return cuda_status(
+        traced(K_BWD_TC, st, [&] { return tc_chunk_bwd(q, k, v, dout, decay, P, R, dq, dk, dv, B, H, N, d, C, st); }));
+  return cuda_status(traced(
+      K_BWD_SIMT, st, [&] { return simt_chunk_bwd(q, k, v, dout, decay, P, R, dq, dk, dv, B, H, N, d, C, dtype, st); }));
 }
 
 }  // namespace api_detail
@@ -126,7 +182,7 @@ int lasp_state_prefix(const float* M, float* Mprefix, const float* decay, const 
     if (s) return s;
     if (total == nullptr) return LASP_OK;
   }
-  return cuda_status(launch_state_scan(M, Mprefix, decay, init, total, B, T, H, d, C, reverse, (cudaStream_t)stream));
+  return scan_impl(K_SCAN, M, Mprefix, decay, init, total, B, T, H, d, C, reverse, (cudaStream_t)stream);
 }
 
 int lasp_fwd(const void* q, const void* k, const void* v, const float* decay, void* o, int B, int H, int64_t N,
@@ -143,17 +199,23 @@ int lasp_fwd(const void* q, const void* k, const void* v, const float* decay, vo
     // the walk carries the state through each segment, filling the other slots
     const int G = walk_segment_tokens(N, C);
     const int stride = G / C;
-    if ((s = cuda_status(tc_chunk_states_slots(k, v, decay, state_cache, B, H, N, d, G, 0, T, stride, 0, st))))
+    if ((s = cuda_status(traced(K_SEG_STATES, st, [&] {
+           return tc_chunk_states_slots(k, v, decay, state_cache, B, H, N, d, G, 0, T, stride, 0, st);
+         }))))
       return s;
-    if ((s = cuda_status(launch_state_scan_slots(state_cache, state_cache, decay, init_state, nullptr, B,
-                                                 (int)(N / G), H, d, G, 0, T, stride, 0, st))))
+    if ((s = cuda_status(traced(K_SEG_SCAN, st, [&] {
+           return launch_state_scan_slots(state_cache, state_cache, decay, init_state, nullptr, B, (int)(N / G), H, d,
+                                          G, 0, T, stride, 0, st);
+         }))))
       return s;
-    return cuda_status(tc_fwd_walk(q, k, v, decay, state_cache, o, B, H, N, d, C, G, num_sms_current_device(), st));
+    const int sms = num_sms_current_device();
+    return cuda_status(traced(K_FWD_WALK, st, [&] {
+      return tc_fwd_walk(q, k, v, decay, state_cache, o, B, H, N, d, C, G, sms, st);
+    }));
   }
   // 1. chunk states M_c into the cache; 2. exclusive prefix in place -> P_c; 3. output.
   if ((s = chunk_states_impl(k, v, decay, state_cache, B, H, N, d, C, dtype, 0, st))) return s;
-  if ((s = cuda_status(launch_state_scan(state_cache, state_cache, decay, init_state, nullptr, B, T, H, d, C, 0, st))))
-    return s;
+  if ((s = scan_impl(K_SCAN, state_cache, state_cache, decay, init_state, nullptr, B, T, H, d, C, 0, st))) return s;
   return chunk_out_impl(q, k, v, decay, state_cache, o, B, H, N, d, C, dtype, st);
 }
 
@@ -189,8 +251,7 @@ int lasp_bwd(const void* q, const void* k, const void* v, const float* decay, co
   const int T = (int)(N / C);
   // 1. gradient chunk states dM_c; 2. exclusive suffix in place -> R_c; 3. dQ, dK, dV.
   if ((s = chunk_states_impl(q, dout, decay, dstate_ws, B, H, N, d, C, dtype, 1, st))) return s;
-  if ((s = cuda_status(launch_state_scan(dstate_ws, dstate_ws, decay, dstate_in, dinit_state, B, T, H, d, C, 1, st))))
-    return s;
+  if ((s = scan_impl(K_SCAN, dstate_ws, dstate_ws, decay, dstate_in, dinit_state, B, T, H, d, C, 1, st))) return s;
   return chunk_grads_impl(q, k, v, dout, decay, state_cache, dstate_ws, dq, dk, dv, B, H, N, d, C, dtype, st);
 }
 
@@ -203,14 +264,75 @@ int lasp_check_device_status(void* stream, int* site) {
   return (int)(word >> 16);
 }
 
+int lasp_trace_enable(int capacity) {
+  if (capacity < 0) return LASP_ERR_INVALID_ARG;
+  std::lock_guard<std::mutex> lock(g_trace.mu);
+  for (cudaEvent_t e : g_trace.ev) cudaEventDestroy(e);
+  g_trace.ev.clear();
+  g_trace.ids.assign(capacity, 0);
+  g_trace.n = 0;
+  g_trace.cap = 0;
+  for (int i = 0; i < 2 * capacity; ++i) {
+    cudaEvent_t e;
+    if (cudaEventCreate(&e) != cudaSuccess) {
+      for (cudaEvent_t x : g_trace.ev) cudaEventDestroy(x);
+      g_trace.ev.clear();
+      return LASP_ERR_CUDA;
+    }
+    g_trace.ev.push_back(e);
+  }
+  g_trace.cap = capacity;
+  return LASP_OK;
+}
+
+int lasp_trace_read(int* kernel_ids, float* ms, int capacity) {
+  if (capacity < 0 || (capacity > 0 && (kernel_ids == nullptr || ms == nullptr))) return -LASP_ERR_INVALID_ARG;
+  std::lock_guard<std::mutex> lock(g_trace.mu);
+  const int n = g_trace.n < capacity ? g_trace.n : capacity;
+  for (int i = 0; i < n; ++i) {
+    if (cudaEventSynchronize(g_trace.ev[2 * i + 1]) != cudaSuccess ||
+        cudaEventElapsedTime(&ms[i], g_trace.ev[2 * i], g_trace.ev[2 * i + 1]) != cudaSuccess)
+      return -LASP_ERR_CUDA;
+    kernel_ids[i] = g_trace.ids[i];
+  }
+  g_trace.n = 0;
+  return n;
+}
+
+const char* lasp_kernel_name(int id) {
+  switch (id) {
+    case K_STATES_TC: return "chunk_states_tc";
+    case K_STATES_SIMT: return "chunk_states_simt";
+    case K_SCAN: return "state_scan";
+    case K_OUT_TC: return "chunk_out_tc";
+    case K_OUT_SIMT: return "chunk_out_simt";
+    case K_BWD_TC: return "chunk_bwd_tc";
+    case K_BWD_SIMT: return "chunk_bwd_simt";
+    case K_FWD_WALK: return "fwd_walk_tc";
+    case K_BWD_WALK: return "bwd_walk_tc";
+    case K_SEG_STATES: return "segment_states_tc";
+    case K_SEG_SCAN: return "segment_scan";
+    case K_PROBE: return "wait_probe";
+    default: return "unknown";
+  }
+}
+
+int lasp_segment_tokens(int64_t N, int C, int d, int dtype) {
+  if (N <= 0 || C < 1 || N % C != 0) return 0;
+  return tc_fwd_walk_ok(dtype, d, C) ? walk_segment_tokens(N, C) : C;
+}
+
 int lasp_set_wait_limit_ns(uint64_t limit_ns) {
   unsigned long long v = limit_ns;
   return cuda_status(cudaMemcpyToSymbol(g_wait_limit_ns, &v, sizeof(v)));
 }
 
 int lasp_wait_probe(void* stream) {
-  wait_probe_kernel<<<1, 32, 0, (cudaStream_t)stream>>>();
-  return cuda_status(cudaGetLastError());
+  cudaStream_t st = (cudaStream_t)stream;
+  return cuda_status(traced(K_PROBE, st, [&] {
+    wait_probe_kernel<<<1, 32, 0, st>>>();
+    return cudaGetLastError();
+  }));
 }
 
 }  // extern "C"

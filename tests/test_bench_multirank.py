@@ -49,4 +49,5 @@ def test_single_rank_needs_no_process_group():
     sys.path.insert(0, ROOT)
     import bench
     assert bench.aggregate(500.0, 0.5, 1) == (1000.0, 0.5)
-    assert bench.algorithmic_bytes("state_prefix", 1, 128, 128, 2) == 2 * 128 * 128 * 4 / 128
+    assert bench.algorithmic_bytes("state_scan", 1, 128, 128, 1024, 2) == 2 * 128 * 128 * 4 / 128
+    assert bench.algorithmic_bytes("fwd_walk_tc", 1, 128, 128, 1024, 2) == 4 * 128 * 2 + 128 * 128 * 4 / 128
