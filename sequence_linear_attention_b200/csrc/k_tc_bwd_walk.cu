@@ -1,0 +1,454 @@
+// Backward pass over segments with the gradient state kept on chip: the
+// mirror of the forward walk (LASP Algorithm 3 steps 12-20, dKV_t =
+// lambda^C dKV_{t+1} + (Lambda Q_t)^T dO_t, walked from the last chunk to the
+// first; LASP-2 review, "Core claim": suffix over the gradient states),
+// bf16, d = 128, chunk C = 128 = one tile.
+//
+// Before this kernel, the segment gradient states and an exclusive suffix
+// over them put, in the R slot of each segment's last chunk, the gradient
+// state entering that chunk from the tokens after the segment. One persistent
+// CTA (256 threads) takes segments in turn and walks their chunks backward,
+// holding R (fp32) in TMEM; P of each chunk comes from the forward pass's
+// state cache. Per chunk c (LASP Eq. 14-23):
+//
+//   MMA 1:  T0 = dO V^T,  T1 = Q K^T,  T2 = dO P^T
+//   epi 1:  dP' = Mask . T0 -> A,  S' = Mask . T1 -> B;  R -> R cache slot,
+//           R -> bf16 X (replacing P),  R <- lambda^128 R in TMEM;
+//           V <- diag(lambda^{127-j}) V in place
+//   MMA 2:  T0 = dP' K
+//   epi 2:  dQ = T0 + lambda^{i+1} T2 -> global;  K <- diag(lambda^{127-j}) K
+//   MMA 3:  T0 = dP'^T Q + V~ R^T  (dK),  T1 = S'^T dO + K~ R  (dV)
+//   epi 3:  dK -> A, dV -> B (TMA stores);  Q <- diag(lambda^{j+1}) Q
+//   MMA 4:  R += Q~^T dO          (the state for chunk c - 1)
+//
+// The decays of the dK/dV inter terms ride on the bf16 operands V~ and K~ so
+// both terms share an accumulator; the dQ inter term keeps its fp32 row
+// scaling. The next chunk's K and V are loaded as soon as MMA 3 has read
+// them, its Q and dO once MMA 4 has. In every epilogue warp w owns TMEM lanes
+// (rows) 32*(w%4).. and the column half w/4.
+#include <algorithm>
+
+#include "kernels.h"
+#include "lasp_common.cuh"
+#include "sm100.cuh"
+#include "tc_kernels.h"
+#include "tma_host.h"
+
+namespace lasp {
+namespace tc_bwd_walk_detail {
+
+using namespace sm100;
+
+constexpr int kD = 128;
+constexpr int kTile = 128;
+constexpr int kThreads = 256;
+constexpr int kWarps = kThreads / 32;
+constexpr uint32_t kTileBytes = kTile * kD * 2;
+constexpr uint32_t kBox = kTileBytes / 2;
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t T0 = 0, T1 = 128, T2 = 256, TR = 384;
+
+struct Smem {
+  uint64_t ld_kv, ld_qd;
+  uint64_t c1, c2, c3, c4;
+  uint32_t tmem_base;
+  int abort;
+  float pw[kTile];
+};
+
+__device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
+  __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+__device__ __forceinline__ uint32_t scale_bf16x2(uint32_t x, float w) {
+  __nv_bfloat162 h = *reinterpret_cast<__nv_bfloat162*>(&x);
+  float2 f = __bfloat1622float2(h);
+  return pack_bf16(f.x * w, f.y * w);
+}
+__device__ __forceinline__ void st_tile16(uint8_t* tile, int row, int col, uint4 v) {
+  *reinterpret_cast<uint4*>(tile + (col >> 6) * kBox + sw128_offset(row, (col & 63) >> 3)) = v;
+}
+__device__ __forceinline__ void st_row32_bf16(uint8_t* tile, int row, int col, const float* v) {
+#pragma unroll
+  for (int q = 0; q < 4; ++q)
+    st_tile16(tile, row, col + q * 8,
+              make_uint4(pack_bf16(v[8 * q], v[8 * q + 1]), pack_bf16(v[8 * q + 2], v[8 * q + 3]),
+                         pack_bf16(v[8 * q + 4], v[8 * q + 5]), pack_bf16(v[8 * q + 6], v[8 * q + 7])));
+}
+__device__ __forceinline__ uint64_t kmaj(uint32_t tile, int kk) {
+  return sw128_desc(tile + (kk >> 2) * kBox + (kk & 3) * 32, 16, 1024);
+}
+__device__ __forceinline__ uint64_t mnmaj(uint32_t tile, int kk) { return sw128_desc(tile + kk * 2048, kBox, 1024); }
+
+// Scales row r of a 128 x 128 bf16 tile by w[r] (w indexed through `pw` with
+// `flip`: w = pw[flip ? 127 - r : r] * post), in place; all threads.
+__device__ __forceinline__ void scale_rows(uint8_t* tile, const float* pw, bool flip, float post, int tid) {
+  uint4* t4 = reinterpret_cast<uint4*>(tile);
+#pragma unroll 2
+  for (int g = tid; g < kTile * 16; g += kThreads) {
+    const int r = (g & (kTile * 8 - 1)) >> 3;
+    const float w = pw[flip ? kTile - 1 - r : r] * post;
+    uint4 x = t4[g];
+    x.x = scale_bf16x2(x.x, w);
+    x.y = scale_bf16x2(x.y, w);
+    x.z = scale_bf16x2(x.z, w);
+    x.w = scale_bf16x2(x.w, w);
+    t4[g] = x;
+  }
+}
+
+struct Item {
+  int b, h, seg;
+};
+__device__ __forceinline__ Item item_of(int64_t w, int H, int nseg) {
+  Item it;
+  it.seg = (int)(w % nseg);
+  it.h = (int)((w / nseg) % H);
+  it.b = (int)(w / ((int64_t)nseg * H));
+  return it;
+}
+
+__global__ void __launch_bounds__(kThreads, 1) bwd_walk_tc(
+    const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
+    const __grid_constant__ CUtensorMap map_v, const __grid_constant__ CUtensorMap map_do,
+    const __grid_constant__ CUtensorMap map_dk, const __grid_constant__ CUtensorMap map_dv, const float* decay,
+    const float* __restrict__ P, float* __restrict__ R, __nv_bfloat16* __restrict__ dq, int H, int64_t N, int T,
+    int G, int nseg, int64_t nitems) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* base = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  uint8_t* sQ = base;
+  uint8_t* sK = base + 1 * kTileBytes;
+  uint8_t* sV = base + 2 * kTileBytes;
+  uint8_t* sD = base + 3 * kTileBytes;
+  uint8_t* sX = base + 4 * kTileBytes;  // P, then R (bf16)
+  uint8_t* sA = base + 5 * kTileBytes;  // dP', then dK out
+  uint8_t* sB = base + 6 * kTileBytes;  // S',  then dV out
+  Smem* s = reinterpret_cast<Smem*>(base + 7 * kTileBytes);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int i = (warp & 3) * 32 + lane;
+  const int half = warp >> 2;
+  const int tiles = G / kTile;
+
+  if (tid == 0) {
+    prefetch_tmap(&map_q);
+    prefetch_tmap(&map_k);
+    prefetch_tmap(&map_v);
+    prefetch_tmap(&map_do);
+    mbar_init(&s->ld_kv, 1);
+    mbar_init(&s->ld_qd, 1);
+    mbar_init(&s->c1, 1);
+    mbar_init(&s->c2, 1);
+    mbar_init(&s->c3, 1);
+    mbar_init(&s->c4, 1);
+    s->abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(&s->tmem_base, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = s->tmem_base;
+  const uint32_t lane_base = tmem + ((uint32_t)((warp & 3) * 32) << 16);
+
+  auto load_kv = [&](const Item& it, int t) {
+    const int row = it.seg * G + t * kTile;
+    mbar_arrive_expect_tx(&s->ld_kv, 2 * kTileBytes);
+    tma_load_4d(sK, &map_k, &s->ld_kv, 0, it.h, row, it.b);
+    tma_load_4d(sK + kBox, &map_k, &s->ld_kv, 64, it.h, row, it.b);
+    tma_load_4d(sV, &map_v, &s->ld_kv, 0, it.h, row, it.b);
+    tma_load_4d(sV + kBox, &map_v, &s->ld_kv, 64, it.h, row, it.b);
+  };
+  auto load_qd = [&](const Item& it, int t) {
+    const int row = it.seg * G + t * kTile;
+    mbar_arrive_expect_tx(&s->ld_qd, 2 * kTileBytes);
+    tma_load_4d(sQ, &map_q, &s->ld_qd, 0, it.h, row, it.b);
+    tma_load_4d(sQ + kBox, &map_q, &s->ld_qd, 64, it.h, row, it.b);
+    tma_load_4d(sD, &map_do, &s->ld_qd, 0, it.h, row, it.b);
+    tma_load_4d(sD + kBox, &map_do, &s->ld_qd, 64, it.h, row, it.b);
+  };
+
+  if (tid == 0 && (int64_t)blockIdx.x < nitems) {
+    const Item first = item_of(blockIdx.x, H, nseg);
+    load_kv(first, tiles - 1);
+    load_qd(first, tiles - 1);
+  }
+
+  constexpr uint32_t id_kk = idesc_bf16(128, 128, 0, 0);
+  constexpr uint32_t id_kn = idesc_bf16(128, 128, 0, 1);
+  constexpr uint32_t id_nn = idesc_bf16(128, 128, 1, 1);
+  const uint32_t aQ = smem_u32(sQ), aK = smem_u32(sK), aV = smem_u32(sV), aD = smem_u32(sD);
+  const uint32_t aX = smem_u32(sX), aA = smem_u32(sA), aB = smem_u32(sB);
+  uint32_t it = 0;
+  bool stop = false;
+
+  for (int64_t w = blockIdx.x; w < nitems && !stop; w += gridDim.x) {
+    const Item item = item_of(w, H, nseg);
+    const float lam = load_decay(decay, item.h);
+    const float l2 = log2f(lam);
+    const bool scale = lam != 1.0f;
+    const float g_tile = decay_pow(l2, (float)kTile);
+    // the previous segment's last MMA 4 writes TMEM R: let it finish before R is replaced
+    if (it > 0 && !mbar_wait(&s->c4, (it - 1) & 1u, SITE_BWD_MMA)) s->abort = 1;
+    tc_fence_after();
+    if (tid < kTile) s->pw[tid] = decay_pow(l2, (float)tid);
+    {
+      // R entering the segment's last chunk -> TMEM R
+      const int64_t slot = (int64_t)item.seg * (G / kTile) + tiles - 1;
+      const float4* src = reinterpret_cast<const float4*>(
+          R + ((((int64_t)item.b * T + slot) * H + item.h) * kD + i) * kD + half * 64);
+#pragma unroll
+      for (int c2 = 0; c2 < 2; ++c2) {
+        uint32_t r[32];
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          const float4 x = __ldcs(src + c2 * 8 + q);
+          r[4 * q] = __float_as_uint(x.x);
+          r[4 * q + 1] = __float_as_uint(x.y);
+          r[4 * q + 2] = __float_as_uint(x.z);
+          r[4 * q + 3] = __float_as_uint(x.w);
+        }
+        tmem_st32(lane_base + TR + half * 64 + c2 * 32, r);
+      }
+      tmem_st_wait();
+    }
+    tc_fence_before();
+    __syncthreads();
+
+    for (int t = tiles - 1; t >= 0; --t, ++it) {
+      const uint32_t par = it & 1u;
+      const int row0 = item.seg * G + t * kTile;
+      const int64_t c = row0 / kTile;  // chunk index (C = tile)
+
+      // P of this chunk -> bf16 X (X's previous content, R, was read by the previous MMA 3)
+      {
+        const float4* src = reinterpret_cast<const float4*>(P + (((int64_t)item.b * T + c) * H + item.h) * kD * kD);
+        float4 x[kD / kWarps];
+#pragma unroll
+        for (int u = 0; u < kD / kWarps; ++u) x[u] = __ldcs(src + (warp + kWarps * u) * (kD / 4) + lane);
+#pragma unroll
+        for (int u = 0; u < kD / kWarps; ++u) {
+          const int r = warp + kWarps * u, col = lane * 4;
+          const uint32_t off = (col >> 6) * kBox + sw128_offset(r, (col & 63) >> 3) + (col & 7) * 2;
+          *reinterpret_cast<uint2*>(sX + off) = make_uint2(pack_bf16(x[u].x, x[u].y), pack_bf16(x[u].z, x[u].w));
+        }
+        fence_async_smem();
+      }
+      // the previous chunk's dK/dV stores must have left A and B
+      if (tid == 0) tma_store_wait_read0();
+      __syncthreads();
+
+      // ---- MMA 1
+      if (tid == 0) {
+        if (mbar_wait(&s->ld_kv, par, SITE_BWD_TMA) && mbar_wait(&s->ld_qd, par, SITE_BWD_TMA)) {
+          tc_fence_after();
+          for (int kk = 0; kk < kD / 16; ++kk) mma_bf16(tmem + T0, kmaj(aD, kk), kmaj(aV, kk), id_kk, kk != 0);
+          for (int kk = 0; kk < kD / 16; ++kk) mma_bf16(tmem + T1, kmaj(aQ, kk), kmaj(aK, kk), id_kk, kk != 0);
+          for (int kk = 0; kk < kD / 16; ++kk) mma_bf16(tmem + T2, kmaj(aD, kk), kmaj(aX, kk), id_kk, kk != 0);
+          mma_commit(&s->c1);
+        } else {
+          s->abort = 1;
+        }
+      }
+
+      // ---- epilogue 1
+      if (mbar_wait(&s->c1, par, SITE_BWD_MMA)) {
+        tc_fence_after();
+#pragma unroll 1
+        for (int cc = 2 * half; cc < 2 * half + 2; ++cc) {
+          uint32_t rp[32], rs[32];
+          tmem_ld32(lane_base + T0 + cc * 32, rp);
+          tmem_ld32(lane_base + T1 + cc * 32, rs);
+          tmem_ld_wait();
+          float fp[32], fs[32];
+#pragma unroll
+          for (int q = 0; q < 32; ++q) {
+            const int j = cc * 32 + q;
+            const float wgt = j <= i ? s->pw[i - j] : 0.f;
+            fp[q] = __uint_as_float(rp[q]) * wgt;
+            fs[q] = __uint_as_float(rs[q]) * wgt;
+          }
+          st_row32_bf16(sA, i, cc * 32, fp);
+          st_row32_bf16(sB, i, cc * 32, fs);
+        }
+        // R of this chunk: to the R cache (the segment's last slot has it already),
+        // to bf16 X (MMA 1 has read P), and pre-scaled by lambda^128 for MMA 4
+        const bool write_r = t < tiles - 1;
+        float* dst = R + (((((int64_t)item.b * T + c) * H + item.h) * kD + i) * kD) + half * 64;
+#pragma unroll 1
+        for (int c2 = 0; c2 < 2; ++c2) {
+          uint32_t r[32];
+          tmem_ld32(lane_base + TR + half * 64 + c2 * 32, r);
+          tmem_ld_wait();
+          float f[32];
+#pragma unroll
+          for (int q = 0; q < 32; ++q) f[q] = __uint_as_float(r[q]);
+          if (write_r) {
+            float4* d4 = reinterpret_cast<float4*>(dst + c2 * 32);
+#pragma unroll
+            for (int q = 0; q < 8; ++q) __stcs(d4 + q, make_float4(f[4 * q], f[4 * q + 1], f[4 * q + 2], f[4 * q + 3]));
+          }
+          st_row32_bf16(sX, i, half * 64 + c2 * 32, f);
+          if (scale) {
+#pragma unroll
+            for (int q = 0; q < 32; ++q) r[q] = __float_as_uint(f[q] * g_tile);
+            tmem_st32(lane_base + TR + half * 64 + c2 * 32, r);
+          }
+        }
+        if (scale) {
+          tmem_st_wait();
+          scale_rows(sV, s->pw, true, 1.f, tid);  // V~ = diag(lambda^{127-j}) V
+        }
+        fence_async_smem();
+      } else {
+        s->abort = 1;
+      }
+      tc_fence_before();
+      __syncthreads();
+      if (s->abort) {
+        stop = true;
+        break;
+      }
+
+      // ---- MMA 2: dQ_intra = dP' K
+      if (tid == 0) {
+        tc_fence_after();
+        for (int kk = 0; kk < kTile / 16; ++kk) mma_bf16(tmem + T0, kmaj(aA, kk), mnmaj(aK, kk), id_kn, kk != 0);
+        mma_commit(&s->c2);
+      }
+      // ---- epilogue 2: dQ
+      if (mbar_wait(&s->c2, par, SITE_BWD_MMA)) {
+        tc_fence_after();
+        const float wi = decay_pow(l2, (float)(i + 1));
+        __nv_bfloat16* out = dq + (((int64_t)item.b * N + row0 + i) * H + item.h) * kD;
+#pragma unroll 1
+        for (int cc = 2 * half; cc < 2 * half + 2; ++cc) {
+          uint32_t ra[32], re[32];
+          tmem_ld32(lane_base + T0 + cc * 32, ra);
+          tmem_ld32(lane_base + T2 + cc * 32, re);
+          tmem_ld_wait();
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            float o[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) o[u] = fmaf(wi, __uint_as_float(re[q * 8 + u]), __uint_as_float(ra[q * 8 + u]));
+            *reinterpret_cast<uint4*>(out + cc * 32 + q * 8) =
+                make_uint4(pack_bf16(o[0], o[1]), pack_bf16(o[2], o[3]), pack_bf16(o[4], o[5]), pack_bf16(o[6], o[7]));
+          }
+        }
+        if (scale) scale_rows(sK, s->pw, true, 1.f, tid);  // K~ = diag(lambda^{127-j}) K
+        fence_async_smem();
+      } else {
+        s->abort = 1;
+      }
+      tc_fence_before();
+      __syncthreads();
+      if (s->abort) {
+        stop = true;
+        break;
+      }
+
+      // ---- MMA 3: dK = dP'^T Q + V~ R^T, dV = S'^T dO + K~ R
+      if (tid == 0) {
+        tc_fence_after();
+        for (int kk = 0; kk < kTile / 16; ++kk) mma_bf16(tmem + T0, mnmaj(aA, kk), mnmaj(aQ, kk), id_nn, kk != 0);
+        for (int kk = 0; kk < kD / 16; ++kk) mma_bf16(tmem + T0, kmaj(aV, kk), kmaj(aX, kk), id_kk, 1);
+        for (int kk = 0; kk < kTile / 16; ++kk) mma_bf16(tmem + T1, mnmaj(aB, kk), mnmaj(aD, kk), id_nn, kk != 0);
+        for (int kk = 0; kk < kD / 16; ++kk) mma_bf16(tmem + T1, kmaj(aK, kk), mnmaj(aX, kk), id_kn, 1);
+        mma_commit(&s->c3);
+      }
+      // ---- epilogue 3: dK -> A, dV -> B; Q~ = diag(lambda^{j+1}) Q
+      if (mbar_wait(&s->c3, par, SITE_BWD_MMA)) {
+        tc_fence_after();
+#pragma unroll 1
+        for (int cc = 2 * half; cc < 2 * half + 2; ++cc) {
+          uint32_t ka[32], va[32];
+          tmem_ld32(lane_base + T0 + cc * 32, ka);
+          tmem_ld32(lane_base + T1 + cc * 32, va);
+          tmem_ld_wait();
+          float fk[32], fv[32];
+#pragma unroll
+          for (int q = 0; q < 32; ++q) {
+            fk[q] = __uint_as_float(ka[q]);
+            fv[q] = __uint_as_float(va[q]);
+          }
+          st_row32_bf16(sA, i, cc * 32, fk);
+          st_row32_bf16(sB, i, cc * 32, fv);
+        }
+        if (scale) scale_rows(sQ, s->pw, false, lam, tid);  // lambda^{j+1} = pw[j] * lambda
+        fence_async_smem();
+      } else {
+        s->abort = 1;
+      }
+      tc_fence_before();
+      __syncthreads();
+      if (s->abort) {
+        stop = true;
+        break;
+      }
+
+      if (tid == 0) {
+        tc_fence_after();
+        // ---- MMA 4: R += Q~^T dO (TMEM R was pre-scaled by lambda^128 in epilogue 1)
+        for (int kk = 0; kk < kTile / 16; ++kk) mma_bf16(tmem + TR, mnmaj(aQ, kk), mnmaj(aD, kk), id_nn, 1);
+        mma_commit(&s->c4);
+        tma_store_4d(&map_dk, sA, 0, item.h, row0, item.b);
+        tma_store_4d(&map_dk, sA + kBox, 64, item.h, row0, item.b);
+        tma_store_4d(&map_dv, sB, 0, item.h, row0, item.b);
+        tma_store_4d(&map_dv, sB + kBox, 64, item.h, row0, item.b);
+        tma_store_commit();
+        // next chunk of this CTA's stream: K, V are free now, Q and dO once MMA 4 is done
+        Item nx = item;
+        int nt = t - 1;
+        bool has_next = true;
+        if (nt < 0) {
+          has_next = w + gridDim.x < nitems;
+          if (has_next) {
+            nx = item_of(w + gridDim.x, H, nseg);
+            nt = tiles - 1;
+          }
+        }
+        if (has_next) {
+          load_kv(nx, nt);
+          if (mbar_wait(&s->c4, par, SITE_BWD_MMA)) load_qd(nx, nt);
+          else s->abort = 1;
+        }
+      }
+    }
+  }
+  if (tid == 0) tma_store_wait0();
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) tmem_dealloc(tmem, kTmemCols);
+}
+
+}  // namespace tc_bwd_walk_detail
+
+bool tc_bwd_walk_ok(int dtype, int d, int64_t C) {
+  return dtype == LASP_BF16 && d == tc_bwd_walk_detail::kD && C == tc_bwd_walk_detail::kTile;
+}
+
+cudaError_t tc_bwd_walk(const void* q, const void* k, const void* v, const void* dout, const float* decay,
+                        const float* P, float* R, void* dq, void* dk, void* dv, int B, int H, int64_t N, int d, int C,
+                        int G, int num_sms, cudaStream_t st) {
+  using namespace tc_bwd_walk_detail;
+  CUtensorMap mq, mk, mv, mdo, mdk, mdv;
+  if (!make_token_map(&mq, q, B, H, N, d, kTile) || !make_token_map(&mk, k, B, H, N, d, kTile) ||
+      !make_token_map(&mv, v, B, H, N, d, kTile) || !make_token_map(&mdo, dout, B, H, N, d, kTile) ||
+      !make_token_map(&mdk, dk, B, H, N, d, kTile) || !make_token_map(&mdv, dv, B, H, N, d, kTile))
+    return cudaErrorInvalidValue;
+  const size_t smem = 1024 + 7 * (size_t)kTileBytes + sizeof(Smem);
+  cudaError_t e = cudaFuncSetAttribute(bwd_walk_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  const int nseg = (int)(N / G);
+  const int64_t nitems = (int64_t)B * H * nseg;
+  const unsigned grid = (unsigned)std::min<int64_t>(nitems, num_sms);
+  bwd_walk_tc<<<grid, kThreads, smem, st>>>(mq, mk, mv, mdo, mdk, mdv, decay, P, R, (__nv_bfloat16*)dq, H, N,
+                                            (int)(N / C), G, nseg, nitems);
+  return cudaGetLastError();
+}
+
+}  // namespace lasp

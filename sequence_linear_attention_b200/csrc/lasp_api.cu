@@ -249,6 +249,27 @@ int lasp_bwd(const void* q, const void* k, const void* v, const float* decay, co
     return s;
   cudaStream_t st = (cudaStream_t)stream;
   const int T = (int)(N / C);
+  if (tc_bwd_walk_ok(dtype, d, C)) {
+    // segments of G tokens: their gradient states go to the slots of their last
+    // chunks, the exclusive suffix over segments turns them into R of those
+    // chunks (and gives dinit), and the walk carries R backward through each
+    // segment, filling the other slots
+    const int G = walk_segment_tokens(N, C);
+    const int stride = G / C;
+    if ((s = cuda_status(traced(K_SEG_STATES, st, [&] {
+           return tc_chunk_states_slots(q, dout, decay, dstate_ws, B, H, N, d, G, 1, T, stride, stride - 1, st);
+         }))))
+      return s;
+    if ((s = cuda_status(traced(K_SEG_SCAN, st, [&] {
+           return launch_state_scan_slots(dstate_ws, dstate_ws, decay, dstate_in, dinit_state, B, (int)(N / G), H, d,
+                                          G, 1, T, stride, stride - 1, st);
+         }))))
+      return s;
+    const int sms = num_sms_current_device();
+    return cuda_status(traced(K_BWD_WALK, st, [&] {
+      return tc_bwd_walk(q, k, v, dout, decay, state_cache, dstate_ws, dq, dk, dv, B, H, N, d, C, G, sms, st);
+    }));
+  }
   // 1. gradient chunk states dM_c; 2. exclusive suffix in place -> R_c; 3. dQ, dK, dV.
   if ((s = chunk_states_impl(q, dout, decay, dstate_ws, B, H, N, d, C, dtype, 1, st))) return s;
   if ((s = scan_impl(K_SCAN, dstate_ws, dstate_ws, decay, dstate_in, dinit_state, B, T, H, d, C, 1, st))) return s;

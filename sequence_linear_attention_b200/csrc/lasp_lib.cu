@@ -7,4 +7,5 @@
 #include "k_tc_out.cu"
 #include "k_tc_fwd_walk.cu"
 #include "k_tc_bwd.cu"
+#include "k_tc_bwd_walk.cu"
 #include "lasp_noalloc.cu"

@@ -29,6 +29,15 @@ int walk_segment_tokens(int64_t N, int C);
 cudaError_t tc_fwd_walk(const void* q, const void* k, const void* v, const float* decay, float* P, void* o, int B,
                         int H, int64_t N, int d, int C, int G, int num_sms, cudaStream_t st);
 
+// Backward walk over segments with the gradient state on chip (bf16, d = 128,
+// C = 128). R must hold, in the slot of each segment's last chunk, the
+// gradient state entering that chunk; the walk fills the other chunks' R
+// slots and writes dq, dk, dv. P is the forward state cache.
+bool tc_bwd_walk_ok(int dtype, int d, int64_t C);
+cudaError_t tc_bwd_walk(const void* q, const void* k, const void* v, const void* dout, const float* decay,
+                        const float* P, float* R, void* dq, void* dk, void* dv, int B, int H, int64_t N, int d, int C,
+                        int G, int num_sms, cudaStream_t st);
+
 bool tc_out_ok(int dtype, int d, int64_t C);
 cudaError_t tc_chunk_out(const void* q, const void* k, const void* v, const float* decay, const float* P, void* o,
                          int B, int H, int64_t N, int d, int C, cudaStream_t st);

@@ -45,6 +45,7 @@ SMALL = [
     (1, 2, 2048, 128, 128, True, True),  # forward walk over two 1024-token segments
     (2, 3, 1536, 128, 256, True, True),  # chunks of two tiles
     (1, 2, 1024, 128, 512, True, False),
+    (2, 150, 1024, 128, 128, True, True),  # more segments than SMs: each CTA walks several
 ]
 
 
