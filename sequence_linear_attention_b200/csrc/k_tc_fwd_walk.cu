@@ -221,19 +221,26 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_walk_tc(const __grid_constant
       // ---- epilogue A
       if (mbar_wait(&s->mma1, it & 1u, SITE_OUT_MMA)) {
         tc_fence_after();
-        // S' = Mask . S into the Q buffer (Q has been read by both MMAs)
-#pragma unroll 1
-        for (int cc = 2 * half; cc < 2 * half + 2; ++cc) {
-          uint32_t r[32];
-          tmem_ld32(lane_base + TS + cc * 32, r);
+        // S' = Mask . S into the Q buffer (Q has been read by both MMAs); both
+        // TMEM loads are in flight before the one wait
+        {
+          uint32_t r0[32], r1[32];
+          tmem_ld32(lane_base + TS + (2 * half) * 32, r0);
+          tmem_ld32(lane_base + TS + (2 * half + 1) * 32, r1);
           tmem_ld_wait();
           float w32[32];
 #pragma unroll
           for (int q = 0; q < 32; ++q) {
-            const int j = cc * 32 + q;
-            w32[q] = j <= i ? __uint_as_float(r[q]) * s->pw[i - j] : 0.f;
+            const int j = 2 * half * 32 + q;
+            w32[q] = j <= i ? __uint_as_float(r0[q]) * s->pw[i - j] : 0.f;
           }
-          st_row32_bf16(sQ, i, cc * 32, w32);
+          st_row32_bf16(sQ, i, 2 * half * 32, w32);
+#pragma unroll
+          for (int q = 0; q < 32; ++q) {
+            const int j = (2 * half + 1) * 32 + q;
+            w32[q] = j <= i ? __uint_as_float(r1[q]) * s->pw[i - j] : 0.f;
+          }
+          st_row32_bf16(sQ, i, (2 * half + 1) * 32, w32);
         }
         // K~ = diag(lambda^{127-j}) K, in place (K has been read by the S MMA)
         if (scale) {
@@ -254,22 +261,23 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_walk_tc(const __grid_constant
         const bool write_cache = t > 0 && (t * kTile) % C == 0;
         if (write_cache || scale) {
           float* dst = P + ((((int64_t)item.b * T + row0 / C) * H + item.h) * kD + i) * kD + half * 64;
-#pragma unroll 1
+          uint32_t r[2][32];
+          tmem_ld32(lane_base + TP + half * 64, r[0]);
+          tmem_ld32(lane_base + TP + half * 64 + 32, r[1]);
+          tmem_ld_wait();
+#pragma unroll
           for (int c2 = 0; c2 < 2; ++c2) {
-            uint32_t r[32];
-            tmem_ld32(lane_base + TP + half * 64 + c2 * 32, r);
-            tmem_ld_wait();
             if (write_cache) {
               float4* d4 = reinterpret_cast<float4*>(dst + c2 * 32);
 #pragma unroll
               for (int q = 0; q < 8; ++q)
-                __stcs(d4 + q, make_float4(__uint_as_float(r[4 * q]), __uint_as_float(r[4 * q + 1]),
-                                           __uint_as_float(r[4 * q + 2]), __uint_as_float(r[4 * q + 3])));
+                __stcs(d4 + q, make_float4(__uint_as_float(r[c2][4 * q]), __uint_as_float(r[c2][4 * q + 1]),
+                                           __uint_as_float(r[c2][4 * q + 2]), __uint_as_float(r[c2][4 * q + 3])));
             }
             if (scale) {
 #pragma unroll
-              for (int q = 0; q < 32; ++q) r[q] = __float_as_uint(__uint_as_float(r[q]) * g_tile);
-              tmem_st32(lane_base + TP + half * 64 + c2 * 32, r);
+              for (int q = 0; q < 32; ++q) r[c2][q] = __float_as_uint(__uint_as_float(r[c2][q]) * g_tile);
+              tmem_st32(lane_base + TP + half * 64 + c2 * 32, r[c2]);
             }
           }
           tmem_st_wait();
@@ -298,26 +306,34 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_walk_tc(const __grid_constant
       if (mbar_wait(&s->mma2, it & 1u, SITE_OUT_MMA)) {
         tc_fence_after();
         const float wi = decay_pow(l2, (float)(i + 1));
-#pragma unroll 1
-        for (int cc = 2 * half; cc < 2 * half + 2; ++cc) {
-          uint32_t a[32], e[32];
-          tmem_ld32(lane_base + TO + cc * 32, a);
-          tmem_ld32(lane_base + TI + cc * 32, e);
+        {
+          // O = O_intra + lambda^{i+1} O_inter, both column chunks' loads in flight together
+          uint32_t a0[32], e0[32], a1[32], e1[32];
+          tmem_ld32(lane_base + TO + (2 * half) * 32, a0);
+          tmem_ld32(lane_base + TI + (2 * half) * 32, e0);
+          tmem_ld32(lane_base + TO + (2 * half + 1) * 32, a1);
+          tmem_ld32(lane_base + TI + (2 * half + 1) * 32, e1);
           tmem_ld_wait();
           float o[32];
 #pragma unroll
-          for (int q = 0; q < 32; ++q) o[q] = fmaf(wi, __uint_as_float(e[q]), __uint_as_float(a[q]));
-          st_row32_bf16(sK, i, cc * 32, o);  // output staging over K~
+          for (int q = 0; q < 32; ++q) o[q] = fmaf(wi, __uint_as_float(e0[q]), __uint_as_float(a0[q]));
+          st_row32_bf16(sK, i, 2 * half * 32, o);  // output staging over K~
+#pragma unroll
+          for (int q = 0; q < 32; ++q) o[q] = fmaf(wi, __uint_as_float(e1[q]), __uint_as_float(a1[q]));
+          st_row32_bf16(sK, i, (2 * half + 1) * 32, o);
         }
-#pragma unroll 1
-        for (int cc = 2 * half; cc < 2 * half + 2; ++cc) {
-          uint32_t r[32];
-          tmem_ld32(lane_base + TP + cc * 32, r);
+        {
+          uint32_t r0[32], r1[32];
+          tmem_ld32(lane_base + TP + (2 * half) * 32, r0);
+          tmem_ld32(lane_base + TP + (2 * half + 1) * 32, r1);
           tmem_ld_wait();
           float p[32];
 #pragma unroll
-          for (int q = 0; q < 32; ++q) p[q] = __uint_as_float(r[q]);
-          st_row32_bf16(sP, i, cc * 32, p);
+          for (int q = 0; q < 32; ++q) p[q] = __uint_as_float(r0[q]);
+          st_row32_bf16(sP, i, 2 * half * 32, p);
+#pragma unroll
+          for (int q = 0; q < 32; ++q) p[q] = __uint_as_float(r1[q]);
+          st_row32_bf16(sP, i, (2 * half + 1) * 32, p);
         }
         fence_async_smem();
       } else {

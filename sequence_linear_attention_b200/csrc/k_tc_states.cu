@@ -3,7 +3,7 @@
 //   M_c = (diag(w) A_c)^T B_c,   A_c, B_c = C x d token tiles of chunk c,
 //   w_t = lambda^{C-1-t} (kind 0, (A, B) = (K, V)) or lambda^{t+1} (kind 1, (Q, dO)).
 //
-// One CTA per (chunk, head, batch), 128 threads. The chunk is consumed in
+// One CTA per (chunk, head, batch), 256 threads. The chunk is consumed in
 // stages of KB tokens (KB = 128, or the largest of 64/32/16 dividing C). Per
 // stage: TMA brings A and B (KB rows x 128 features, two 64-feature boxes each,
 // 128-byte swizzle) into a shared-memory slot; when lambda != 1 the four warps
@@ -11,9 +11,12 @@
 // tcgen05.mma (M = N = 128 features, K = 16 tokens) that accumulate M_c in
 // TMEM. Both operands are MN-major: the tiles arrive token-major with features
 // contiguous, which is exactly A^T and B with the reduced (token) index as the
-// slow one. Two slots let the next stage's loads run under the current
-// stage's scaling and MMAs. The epilogue reads the 128 x 128 fp32 accumulator
-// from TMEM (thread i owns row i) and writes the state row by row.
+// slow one. Up to three slots keep two stages' loads in flight under the
+// current stage's scaling and MMAs. The epilogue reads the 128 x 128 fp32
+// accumulator from TMEM (warp w: rows 32*(w%4).., column half w/4) and writes
+// the state row by row.
+#include <algorithm>
+
 #include "kernels.h"
 #include "lasp_common.cuh"
 #include "sm100.cuh"
@@ -26,12 +29,13 @@ namespace tc_states_detail {
 using namespace sm100;
 
 constexpr int kD = 128;           // head dimension handled here
-constexpr int kThreads = 128;
+constexpr int kThreads = 256;
+constexpr int kMaxSlots = 3;
 constexpr uint32_t kTmemCols = 128;  // one 128 x 128 fp32 accumulator
 
 struct Smem {
-  uint64_t full[2];
-  uint64_t empty[2];
+  uint64_t full[kMaxSlots];
+  uint64_t empty[kMaxSlots];
   uint64_t done;
   uint32_t tmem_base;
   int abort;
@@ -44,11 +48,10 @@ __device__ __forceinline__ uint32_t bf16x2_scale(uint32_t x, float w) {
   return *reinterpret_cast<uint32_t*>(&r);
 }
 
-// Issues the four TMA boxes of stage `stage` (A and B, two 64-feature boxes
-// each) into slot stage & 1.
+// Issues the four TMA boxes of one stage (A and B, two 64-feature boxes each)
+// into `slot`.
 __device__ __forceinline__ void issue_stage(uint8_t* tiles, uint32_t tile_bytes, Smem* s, const CUtensorMap* map_a,
-                                            const CUtensorMap* map_b, int stage, int row, int h, int b) {
-  const int slot = stage & 1;
+                                            const CUtensorMap* map_b, int slot, int row, int h, int b) {
   uint8_t* a = tiles + (size_t)slot * 2 * tile_bytes;
   uint8_t* bb = a + tile_bytes;
   mbar_arrive_expect_tx(&s->full[slot], 2 * tile_bytes);
@@ -67,7 +70,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_states_tc(const __grid_cons
   // tiles need 1024-byte alignment for the 128-byte swizzle atoms
   uint8_t* tiles = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   const int nstages = C / KB;
-  const int nslots = nstages > 1 ? 2 : 1;
+  const int nslots = nstages < kMaxSlots ? nstages : kMaxSlots;
   const uint32_t tile_bytes = (uint32_t)KB * 256;  // KB rows x 128 features x bf16
   Smem* s = reinterpret_cast<Smem*>(tiles + nslots * 2 * tile_bytes);
 
@@ -80,10 +83,10 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_states_tc(const __grid_cons
   if (tid == 0) {
     prefetch_tmap(&map_a);
     prefetch_tmap(&map_b);
-    mbar_init(&s->full[0], 1);
-    mbar_init(&s->full[1], 1);
-    mbar_init(&s->empty[0], 1);
-    mbar_init(&s->empty[1], 1);
+    for (int q = 0; q < kMaxSlots; ++q) {
+      mbar_init(&s->full[q], 1);
+      mbar_init(&s->empty[q], 1);
+    }
     mbar_init(&s->done, 1);
     s->abort = 0;
     fence_mbar_init();
@@ -98,14 +101,13 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_states_tc(const __grid_cons
   const uint32_t tmem = s->tmem_base;
 
   if (tid == 0) {
-    issue_stage(tiles, tile_bytes, s, &map_a, &map_b, 0, c * C, h, b);
-    if (nstages > 1) issue_stage(tiles, tile_bytes, s, &map_a, &map_b, 1, c * C + KB, h, b);
+    for (int k = 0; k < nslots; ++k) issue_stage(tiles, tile_bytes, s, &map_a, &map_b, k, c * C + k * KB, h, b);
   }
 
   constexpr uint32_t idesc = idesc_bf16(128, 128, 1, 1);
   for (int k = 0; k < nstages; ++k) {
-    const int slot = k & 1;
-    const uint32_t par = (uint32_t)(k >> 1) & 1u;
+    const int slot = k % nslots;
+    const uint32_t par = (uint32_t)(k / nslots) & 1u;
     if (!mbar_wait(&s->full[slot], par, SITE_STATES_TMA)) s->abort = 1;
     if (scale) {
       // scale row r of A by w_{k*KB + r}; the row of a 16-byte chunk is its
@@ -136,11 +138,15 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_states_tc(const __grid_cons
         mma_bf16(tmem, ad, bd, idesc, (k | j) != 0);
       }
       mma_commit(k + 1 < nstages ? &s->empty[slot] : &s->done);
-      if (k + 2 < nstages) {
-        // the slot is refilled once the MMAs that read it have completed
-        if (mbar_wait(&s->empty[slot], par, SITE_STATES_MMA))
-          issue_stage(tiles, tile_bytes, s, &map_a, &map_b, k + 2, c * C + (k + 2) * KB, h, b);
-        else s->abort = 1;
+      // refill the slot of the previous stage (its MMAs were issued one stage
+      // ago), keeping nslots - 1 stages in flight while this one is consumed
+      const int kr = k - 1 + nslots;
+      if (k >= 1 && kr < nstages) {
+        const int pslot = (k - 1) % nslots;
+        if (mbar_wait(&s->empty[pslot], (uint32_t)((k - 1) / nslots) & 1u, SITE_STATES_MMA))
+          issue_stage(tiles, tile_bytes, s, &map_a, &map_b, pslot, c * C + kr * KB, h, b);
+        else
+          s->abort = 1;
       }
     }
   }
@@ -148,14 +154,15 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_states_tc(const __grid_cons
   const bool ok = !s->abort && mbar_wait(&s->done, 0, SITE_STATES_MMA);
   tc_fence_after();
   if (ok) {
-    const int row = warp * 32 + lane;
+    // warp w reads TMEM lanes (rows) 32*(w%4).. and the column half w/4
+    const int row = (warp & 3) * 32 + lane, half = warp >> 2;
     // chunk c's state goes to slot c * slot_stride + slot_offset of an array with t_out slots
     const int64_t slot = (int64_t)c * slot_stride + slot_offset;
     float* out = M + ((((int64_t)b * t_out + slot) * H + h) * kD + row) * kD;
 #pragma unroll 1
-    for (int cc = 0; cc < kD / 32; ++cc) {
+    for (int cc = 2 * half; cc < 2 * half + 2; ++cc) {
       uint32_t r[32];
-      tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16) + cc * 32, r);
+      tmem_ld32(tmem + ((uint32_t)((warp & 3) * 32) << 16) + cc * 32, r);
       tmem_ld_wait();
       float4* o4 = reinterpret_cast<float4*>(out + cc * 32);
 #pragma unroll
@@ -189,7 +196,7 @@ cudaError_t tc_chunk_states_slots(const void* a, const void* bm, const float* de
   CUtensorMap ma, mb;
   if (!make_token_map(&ma, a, B, H, N, d, KB) || !make_token_map(&mb, bm, B, H, N, d, KB))
     return cudaErrorInvalidValue;
-  const int nslots = C / KB > 1 ? 2 : 1;
+  const int nslots = std::min(C / KB, kMaxSlots);
   const size_t smem = 1024 + (size_t)nslots * 2 * KB * 256 + sizeof(Smem);
   cudaError_t e = cudaFuncSetAttribute(chunk_states_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
