@@ -24,7 +24,8 @@
 // The decays of the dK/dV inter terms ride on the bf16 operands V~ and K~ so
 // both terms share an accumulator; the dQ inter term keeps its fp32 row
 // scaling. The next chunk's K and V are loaded as soon as MMA 3 has read
-// them, its Q and dO once MMA 4 has. In every epilogue warp w owns TMEM lanes
+// them, its P (fp32, by bulk copy into A and B) once the dK/dV stores have
+// left those tiles, its Q and dO once MMA 4 has. In every epilogue warp w owns TMEM lanes
 // (rows) 32*(w%4).. and the column half w/4.
 #include <algorithm>
 
@@ -49,7 +50,7 @@ constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t T0 = 0, T1 = 128, T2 = 256, TR = 384;
 
 struct Smem {
-  uint64_t ld_kv, ld_qd;
+  uint64_t ld_kv, ld_qd, ld_p;
   uint64_t c1, c2, c3, c4;
   uint32_t tmem_base;
   int abort;
@@ -137,6 +138,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_walk_tc(
     prefetch_tmap(&map_do);
     mbar_init(&s->ld_kv, 1);
     mbar_init(&s->ld_qd, 1);
+    mbar_init(&s->ld_p, 1);
     mbar_init(&s->c1, 1);
     mbar_init(&s->c2, 1);
     mbar_init(&s->c3, 1);
@@ -171,10 +173,20 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_walk_tc(
     tma_load_4d(sD + kBox, &map_do, &s->ld_qd, 64, it.h, row, it.b);
   };
 
+  // P of a chunk (fp32, 64 KB) -> the A and B tiles, which are idle between a
+  // chunk's dK/dV stores and the next chunk's epilogue 1
+  auto load_p = [&](const Item& it, int t) {
+    const int64_t c = ((int64_t)it.seg * G + (int64_t)t * kTile) / kTile;
+    const float* src = P + (((int64_t)it.b * T + c) * H + it.h) * kD * kD;
+    mbar_arrive_expect_tx(&s->ld_p, kD * kD * 4);
+    for (int part = 0; part < 4; ++part) bulk_load(sA + part * (kD * kD), src + part * (kD * kD / 4), kD * kD, &s->ld_p);
+  };
+
   if (tid == 0 && (int64_t)blockIdx.x < nitems) {
     const Item first = item_of(blockIdx.x, H, nseg);
     load_kv(first, tiles - 1);
     load_qd(first, tiles - 1);
+    load_p(first, tiles - 1);
   }
 
   constexpr uint32_t id_kk = idesc_bf16(128, 128, 0, 0);
@@ -223,22 +235,21 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_walk_tc(
       const int row0 = item.seg * G + t * kTile;
       const int64_t c = row0 / kTile;  // chunk index (C = tile)
 
-      // P of this chunk -> bf16 X (X's previous content, R, was read by the previous MMA 3)
-      {
-        const float4* src = reinterpret_cast<const float4*>(P + (((int64_t)item.b * T + c) * H + item.h) * kD * kD);
-        float4 x[kD / kWarps];
-#pragma unroll
-        for (int u = 0; u < kD / kWarps; ++u) x[u] = __ldcs(src + (warp + kWarps * u) * (kD / 4) + lane);
-#pragma unroll
+      // P of this chunk (fp32 in A and B) -> bf16 X; X's previous content, R,
+      // was read by the previous MMA 3
+      if (mbar_wait(&s->ld_p, par, SITE_BWD_TMA)) {
+        const float4* src = reinterpret_cast<const float4*>(sA);
+#pragma unroll 4
         for (int u = 0; u < kD / kWarps; ++u) {
           const int r = warp + kWarps * u, col = lane * 4;
+          const float4 x = src[r * (kD / 4) + lane];
           const uint32_t off = (col >> 6) * kBox + sw128_offset(r, (col & 63) >> 3) + (col & 7) * 2;
-          *reinterpret_cast<uint2*>(sX + off) = make_uint2(pack_bf16(x[u].x, x[u].y), pack_bf16(x[u].z, x[u].w));
+          *reinterpret_cast<uint2*>(sX + off) = make_uint2(pack_bf16(x.x, x.y), pack_bf16(x.z, x.w));
         }
         fence_async_smem();
+      } else {
+        s->abort = 1;
       }
-      // the previous chunk's dK/dV stores must have left A and B
-      if (tid == 0) tma_store_wait_read0();
       __syncthreads();
 
       // ---- MMA 1
@@ -413,6 +424,8 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_walk_tc(
         }
         if (has_next) {
           load_kv(nx, nt);
+          tma_store_wait_read0();  // the dK/dV stores have left A and B
+          load_p(nx, nt);
           if (mbar_wait(&s->c4, par, SITE_BWD_MMA)) load_qd(nx, nt);
           else s->abort = 1;
         }
