@@ -76,9 +76,14 @@ typedef enum { LASP_F32 = 0, LASP_BF16 = 1 } lasp_dtype;
  *   q, k, v:      in,  [B, N, H, d] of `dtype`.
  *   decay:        in,  float[H] or NULL.
  *   o:            out, [B, N, H, d] of `dtype`.
- *   state_cache:  out, float [B, N/C, H, d, d]; receives P_c, the state that
- *                 enters chunk c (LASP section 3.4 "KV State Caching"), which
- *                 lasp_bwd reads. Required.
+ *   state_cache:  out, B * (N/C) * H * d * d floats (16-byte aligned): the
+ *                 cache of chunk-entering states P_c that lasp_bwd reads (LASP
+ *                 section 3.4 "KV State Caching"), one d x d slot per (b, c, h).
+ *                 Its encoding inside a slot is internal to the library (fp32
+ *                 P_c, or, for bf16 with d = 128 and C = 128, the bf16 operand
+ *                 tile of P_c); pass it unchanged to lasp_bwd with the same
+ *                 sizes. The per-chunk states themselves are exposed by
+ *                 lasp_chunk_states + lasp_state_prefix. Required.
  *   init_state:   in,  float [B, H, d, d] or NULL: the state entering token 0
  *                 (the prefix of the shards before this one in the LASP-2
  *                 decomposition).
@@ -99,10 +104,13 @@ LASP_API int lasp_fwd(const void* q, const void* k, const void* v, const float* 
  *   dV_c = [(Q_c K_c^T) . Mask]^T dO_c + lambda^C Lambda^-1 K_c R_c   (Eq. 22, 23)
  *   q, k, v, dout:  in,  [B, N, H, d] of `dtype`.
  *   dq, dk, dv:     out, [B, N, H, d] of `dtype`.
- *   state_cache:    in,  the P array lasp_fwd wrote for the same q, k, v,
+ *   state_cache:    in,  the cache lasp_fwd wrote for the same q, k, v,
  *                   decay, C and init_state. Required.
- *   dstate_ws:      out, float [B, N/C, H, d, d]; receives R_c, the gradient
- *                   state chunk c receives from the tokens after it. Required.
+ *   dstate_ws:      workspace, B * (N/C) * H * d * d floats (16-byte aligned)
+ *                   for the gradient states R_c (the gradient state chunk c
+ *                   receives from the tokens after it); its contents on return
+ *                   are unspecified (lasp_chunk_dstates + lasp_state_prefix
+ *                   expose R_c). Required.
  *   init_state:     in,  as given to lasp_fwd (only its effect through
  *                   state_cache matters; may be NULL).
  *   dstate_in:      in,  float [B, H, d, d] or NULL: gradient state entering the
@@ -190,7 +198,7 @@ LASP_API int lasp_chunk_grads(const void* q, const void* k, const void* v, const
  * all of the device memory, so that a cudaMalloc would fail (and would
  * synchronize the device if it succeeded).
  * It computes exactly what lasp_bwd computes, with the same arguments except
- * dstate_ws: the gradient states R live in a fixed 32 MiB array compiled into
+ * dstate_ws: the gradient-state workspace lives in a fixed 32 MiB array compiled into
  * the library (LASP_NOALLOC_SCRATCH_BYTES), which every GPU that loads the
  * library holds until the process exits. The call allocates nothing.
  *   Limit: B * (N / C) * H * d * d * 4 <= LASP_NOALLOC_SCRATCH_BYTES (for

@@ -8,11 +8,11 @@
 // over them put, in the R slot of each segment's last chunk, the gradient
 // state entering that chunk from the tokens after the segment. One persistent
 // CTA (256 threads) takes segments in turn and walks their chunks backward,
-// holding R (fp32) in TMEM; P of each chunk comes from the forward pass's
-// state cache. Per chunk c (LASP Eq. 14-23):
+// holding R (fp32) in TMEM; P of each chunk comes from the forward walk's
+// cache as a ready bf16 operand tile. Per chunk c (LASP Eq. 14-23):
 //
 //   MMA 1:  T0 = dO V^T,  T1 = Q K^T,  T2 = dO P^T
-//   epi 1:  dP' = Mask . T0 -> A,  S' = Mask . T1 -> B;  R -> R cache slot,
+//   epi 1:  dP' = Mask . T0 -> A,  S' = Mask . T1 -> B;
 //           R -> bf16 X (replacing P),  R <- lambda^128 R in TMEM;
 //           V <- diag(lambda^{127-j}) V in place
 //   MMA 2:  T0 = dP' K
@@ -23,9 +23,9 @@
 //
 // The decays of the dK/dV inter terms ride on the bf16 operands V~ and K~ so
 // both terms share an accumulator; the dQ inter term keeps its fp32 row
-// scaling. The next chunk's K and V are loaded as soon as MMA 3 has read
-// them, its P (fp32, by bulk copy into A and B) once the dK/dV stores have
-// left those tiles, its Q and dO once MMA 4 has. In every epilogue warp w owns TMEM lanes
+// scaling. The next chunk's K, V and P are loaded as soon as MMA 3 has read
+// the buffers they replace, its Q and dO once MMA 4 has. R is not stored per
+// chunk: only the segment-level slots of the workspace are used. In every epilogue warp w owns TMEM lanes
 // (rows) 32*(w%4).. and the column half w/4.
 #include <algorithm>
 
@@ -173,13 +173,13 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_walk_tc(
     tma_load_4d(sD + kBox, &map_do, &s->ld_qd, 64, it.h, row, it.b);
   };
 
-  // P of a chunk (fp32, 64 KB) -> the A and B tiles, which are idle between a
-  // chunk's dK/dV stores and the next chunk's epilogue 1
+  // P of a chunk: the forward walk stored it in the chunk's cache slot as the
+  // bf16 operand tile (128-byte swizzled), so it is copied into X as is
   auto load_p = [&](const Item& it, int t) {
     const int64_t c = ((int64_t)it.seg * G + (int64_t)t * kTile) / kTile;
     const float* src = P + (((int64_t)it.b * T + c) * H + it.h) * kD * kD;
-    mbar_arrive_expect_tx(&s->ld_p, kD * kD * 4);
-    for (int part = 0; part < 4; ++part) bulk_load(sA + part * (kD * kD), src + part * (kD * kD / 4), kD * kD, &s->ld_p);
+    mbar_arrive_expect_tx(&s->ld_p, kTileBytes);
+    bulk_load(sX, src, kTileBytes, &s->ld_p);
   };
 
   if (tid == 0 && (int64_t)blockIdx.x < nitems) {
@@ -235,26 +235,14 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_walk_tc(
       const int row0 = item.seg * G + t * kTile;
       const int64_t c = row0 / kTile;  // chunk index (C = tile)
 
-      // P of this chunk (fp32 in A and B) -> bf16 X; X's previous content, R,
-      // was read by the previous MMA 3
-      if (mbar_wait(&s->ld_p, par, SITE_BWD_TMA)) {
-        const float4* src = reinterpret_cast<const float4*>(sA);
-#pragma unroll 4
-        for (int u = 0; u < kD / kWarps; ++u) {
-          const int r = warp + kWarps * u, col = lane * 4;
-          const float4 x = src[r * (kD / 4) + lane];
-          const uint32_t off = (col >> 6) * kBox + sw128_offset(r, (col & 63) >> 3) + (col & 7) * 2;
-          *reinterpret_cast<uint2*>(sX + off) = make_uint2(pack_bf16(x.x, x.y), pack_bf16(x.z, x.w));
-        }
-        fence_async_smem();
-      } else {
-        s->abort = 1;
-      }
+      // the previous chunk's dK/dV stores must have left A and B before epilogue 1
+      if (tid == 0) tma_store_wait_read0();
       __syncthreads();
 
       // ---- MMA 1
       if (tid == 0) {
-        if (mbar_wait(&s->ld_kv, par, SITE_BWD_TMA) && mbar_wait(&s->ld_qd, par, SITE_BWD_TMA)) {
+        if (mbar_wait(&s->ld_kv, par, SITE_BWD_TMA) && mbar_wait(&s->ld_qd, par, SITE_BWD_TMA) &&
+            mbar_wait(&s->ld_p, par, SITE_BWD_TMA)) {
           tc_fence_after();
           for (int kk = 0; kk < kD / 16; ++kk) mma_bf16(tmem + T0, kmaj(aD, kk), kmaj(aV, kk), id_kk, kk != 0);
           for (int kk = 0; kk < kD / 16; ++kk) mma_bf16(tmem + T1, kmaj(aQ, kk), kmaj(aK, kk), id_kk, kk != 0);
@@ -285,28 +273,23 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_walk_tc(
           st_row32_bf16(sA, i, cc * 32, fp);
           st_row32_bf16(sB, i, cc * 32, fs);
         }
-        // R of this chunk: to the R cache (the segment's last slot has it already),
-        // to bf16 X (MMA 1 has read P), and pre-scaled by lambda^128 for MMA 4
-        const bool write_r = t < tiles - 1;
-        float* dst = R + (((((int64_t)item.b * T + c) * H + item.h) * kD + i) * kD) + half * 64;
-#pragma unroll 1
-        for (int c2 = 0; c2 < 2; ++c2) {
-          uint32_t r[32];
-          tmem_ld32(lane_base + TR + half * 64 + c2 * 32, r);
+        // R of this chunk -> bf16 X (MMA 1 has read P) and pre-scaled by lambda^128 for MMA 4
+        {
+          uint32_t r[2][32];
+          tmem_ld32(lane_base + TR + half * 64, r[0]);
+          tmem_ld32(lane_base + TR + half * 64 + 32, r[1]);
           tmem_ld_wait();
-          float f[32];
 #pragma unroll
-          for (int q = 0; q < 32; ++q) f[q] = __uint_as_float(r[q]);
-          if (write_r) {
-            float4* d4 = reinterpret_cast<float4*>(dst + c2 * 32);
+          for (int c2 = 0; c2 < 2; ++c2) {
+            float f[32];
 #pragma unroll
-            for (int q = 0; q < 8; ++q) __stcs(d4 + q, make_float4(f[4 * q], f[4 * q + 1], f[4 * q + 2], f[4 * q + 3]));
-          }
-          st_row32_bf16(sX, i, half * 64 + c2 * 32, f);
-          if (scale) {
+            for (int q = 0; q < 32; ++q) f[q] = __uint_as_float(r[c2][q]);
+            st_row32_bf16(sX, i, half * 64 + c2 * 32, f);
+            if (scale) {
 #pragma unroll
-            for (int q = 0; q < 32; ++q) r[q] = __float_as_uint(f[q] * g_tile);
-            tmem_st32(lane_base + TR + half * 64 + c2 * 32, r);
+              for (int q = 0; q < 32; ++q) r[c2][q] = __float_as_uint(f[q] * g_tile);
+              tmem_st32(lane_base + TR + half * 64 + c2 * 32, r[c2]);
+            }
           }
         }
         if (scale) {
@@ -424,8 +407,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_walk_tc(
         }
         if (has_next) {
           load_kv(nx, nt);
-          tma_store_wait_read0();  // the dK/dV stores have left A and B
-          load_p(nx, nt);
+          load_p(nx, nt);  // X (R) has been read by MMA 3
           if (mbar_wait(&s->c4, par, SITE_BWD_MMA)) load_qd(nx, nt);
           else s->abort = 1;
         }

@@ -13,13 +13,16 @@
 //
 //   MMA 1:  S = Q K^T (TMEM S),  O_inter = Q P_bf16 (TMEM I)
 //   epi A:  S' = Mask . S -> bf16 over Q;  K~ = diag(lambda^{127-j}) K in place;
-//           P -> state cache (at chunk starts);  P <- lambda^128 P in TMEM
+//           P <- lambda^128 P in TMEM (and, for C > 128, P -> fp32 cache at chunk starts)
 //   MMA 2:  O_intra = S' V (TMEM O);  P += K~^T V (TMEM P)
 //   epi B:  O = O_intra + lambda^{i+1} O_inter -> bf16 over K~ -> TMA store;
 //           P -> bf16 operand for the next tile
 //
-// Two sets of Q/K/V buffers alternate: while a tile is computed, the next
-// tile's loads (possibly of the next segment) are in flight. In every epilogue
+// With C = 128 each tile starts a chunk, and the bf16 operand tile of the
+// entering state (already in shared memory for O_inter) goes to the chunk's
+// cache slot by one bulk copy; the backward walk loads it back as is. Two sets
+// of Q/K/V buffers alternate: while a tile is computed, the next tile's loads
+// (possibly of the next segment) are in flight. In every epilogue
 // warp w owns TMEM lanes (rows) 32*(w%4).. and the column half w/4.
 #include <algorithm>
 
@@ -92,7 +95,8 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_walk_tc(const __grid_constant
                                                             const __grid_constant__ CUtensorMap map_v,
                                                             const __grid_constant__ CUtensorMap map_o,
                                                             const float* decay, float* __restrict__ P, int H,
-                                                            int T, int C, int G, int nseg, int64_t nitems) {
+                                                            int T, int C, int G, int nseg, int64_t nitems,
+                                                            int cache_bf16) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   uint8_t* sP = base + 6 * kTileBytes;
@@ -191,6 +195,13 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_walk_tc(const __grid_constant
       uint8_t* sV = sQ + 2 * kTileBytes;
       const int row0 = item.seg * G + t * kTile;
 
+      if (tid == 0 && cache_bf16) {
+        // the bf16 operand tile of the state entering this chunk, as it sits in
+        // shared memory, is the cache entry the backward pass loads back
+        uint8_t* slot = reinterpret_cast<uint8_t*>(P + (((int64_t)item.b * T + row0 / C) * H + item.h) * kD * kD);
+        bulk_store(slot, sP, kTileBytes);
+        tma_store_commit();
+      }
       if (tid == 0) {
         // prefetch the next tile of this CTA's stream into the other set; its
         // K buffer may still be the source of the previous tile's TMA store
@@ -258,7 +269,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_walk_tc(const __grid_constant
           }
         }
         // the state entering this tile: into the cache at chunk starts, then pre-scaled by lambda^128
-        const bool write_cache = t > 0 && (t * kTile) % C == 0;
+        const bool write_cache = !cache_bf16 && t > 0 && (t * kTile) % C == 0;
         if (write_cache || scale) {
           float* dst = P + ((((int64_t)item.b * T + row0 / C) * H + item.h) * kD + i) * kD + half * 64;
           uint32_t r[2][32];
@@ -286,6 +297,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_walk_tc(const __grid_constant
       } else {
         s->abort = 1;
       }
+      if (tid == 0 && cache_bf16) tma_store_wait_read0();  // epilogue B rewrites sP
       tc_fence_before();
       __syncthreads();
       if (s->abort) {
@@ -385,7 +397,11 @@ cudaError_t tc_fwd_walk(const void* q, const void* k, const void* v, const float
   const int nseg = (int)(N / G);
   const int64_t nitems = (int64_t)B * H * nseg;
   const unsigned grid = (unsigned)std::min<int64_t>(nitems, num_sms);
-  fwd_walk_tc<<<grid, kThreads, smem, st>>>(mq, mk, mv, mo, decay, P, H, (int)(N / C), C, G, nseg, nitems);
+  // with C = 128 the backward walk reads the cache: it gets each chunk's state
+  // as the bf16 operand tile; otherwise the cache holds fp32 states
+  const int cache_bf16 = C == kTile ? 1 : 0;
+  fwd_walk_tc<<<grid, kThreads, smem, st>>>(mq, mk, mv, mo, decay, P, H, (int)(N / C), C, G, nseg, nitems,
+                                           cache_bf16);
   return cudaGetLastError();
 }
 

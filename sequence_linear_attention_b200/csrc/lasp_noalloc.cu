@@ -60,8 +60,19 @@ extern "C" int lasp_bwd_noalloc(const void* q, const void* k, const void* v, con
   float* R = nullptr;
   if ((s = noalloc_detail::scratch_for_current_device(&R))) return s;
   cudaStream_t st = (cudaStream_t)stream;
-  // the same three steps as lasp_bwd, with the workspace in the fixed array;
-  // every element of R is written before it is read, so nothing is cleared
+  // the same steps as lasp_bwd, with the workspace in the fixed array; every
+  // element of R that is read is written first, so nothing is cleared
+  if (tc_bwd_walk_ok(dtype, d, C)) {
+    const int G = walk_segment_tokens(N, C);
+    const int stride = G / C;
+    if ((s = cuda_status(tc_chunk_states_slots(q, dout, decay, R, B, H, N, d, G, 1, T, stride, stride - 1, st))))
+      return s;
+    if ((s = cuda_status(launch_state_scan_slots(R, R, decay, dstate_in, dinit_state, B, (int)(N / G), H, d, G, 1, T,
+                                                 stride, stride - 1, st))))
+      return s;
+    return cuda_status(tc_bwd_walk(q, k, v, dout, decay, state_cache, R, dq, dk, dv, B, H, N, d, C, G,
+                                   num_sms_current_device(), st));
+  }
   if ((s = chunk_states_impl(q, dout, decay, R, B, H, N, d, C, dtype, 1, st))) return s;
   if ((s = cuda_status(launch_state_scan(R, R, decay, dstate_in, dinit_state, B, T, H, d, C, 1, st)))) return s;
   return chunk_grads_impl(q, k, v, dout, decay, state_cache, R, dq, dk, dv, B, H, N, d, C, dtype, st);

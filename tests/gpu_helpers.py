@@ -77,3 +77,23 @@ def run_fwd_bwd(inp: dict, C: int, init=None, dstate_in=None, want_dinit=False, 
     status, site = lasp.lasp_check_device_status()
     assert status == 0, (status, site)
     return dict(o=o, dq=dq, dk=dk, dv=dv, P=cache, R=ws, dinit=dinit)
+
+
+def run_states(inp: dict, C: int, P, R, init=None, dstate_in=None):
+    """P_c and R_c through the exposed state entry points (lasp_chunk_states /
+    lasp_chunk_dstates, then lasp_state_prefix forward / reverse), into the
+    given [B, N/C, H, d, d] fp32 device buffers."""
+    import torch
+    import sequence_linear_attention_b200 as lasp
+    bf16 = inp["bf16"]
+    q, k, v, do = (to_device(inp[n], bf16) for n in ("q", "k", "v", "do"))
+    decay = decay_device(inp["lam"])
+    init_t = None if init is None else torch.from_numpy(np.asarray(init, np.float32)).cuda()
+    din_t = None if dstate_in is None else torch.from_numpy(np.asarray(dstate_in, np.float32)).cuda()
+    lasp.lasp_chunk_states(None, k, v, decay, P, C)
+    lasp.lasp_state_prefix(P, P, decay, C, init=init_t)
+    lasp.lasp_chunk_dstates(q, do, decay, R, C)
+    lasp.lasp_state_prefix(R, R, decay, C, init=din_t, reverse=True)
+    status, site = lasp.lasp_check_device_status()
+    assert status == 0, (status, site)
+    return dict(P=P, R=R)

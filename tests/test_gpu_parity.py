@@ -6,7 +6,7 @@ import pytest
 
 import oracle
 from sequence_linear_attention_b200 import inputs as lasp_inputs
-from gpu_helpers import (decay_device, host_f32, rel_err, run_fwd_bwd, to_device, to_host, tol)
+from gpu_helpers import (decay_device, host_f32, rel_err, run_fwd_bwd, run_states, to_device, to_host, tol)
 
 pytestmark = pytest.mark.gpu
 
@@ -21,7 +21,7 @@ def _oracle_all(inp, C, init=None, dstate_in=None):
     return dict(o=o, dq=dq, dk=dk, dv=dv, P=P, R=R, dinit=dinit)
 
 
-def _compare(gpu, ref, bf16, names=("o", "dq", "dk", "dv", "P", "R")):
+def _compare(gpu, ref, bf16, names=("o", "dq", "dk", "dv")):
     errs = {n: rel_err(to_host(gpu[n]), ref[n]) for n in names}
     bad = {n: e for n, e in errs.items() if not e <= tol(bf16)}
     assert not bad, f"errors above {tol(bf16)}: {bad} (all: {errs})"
@@ -53,7 +53,10 @@ SMALL = [
 def test_small_shapes_against_oracle(B, H, N, d, C, bf16, decayed):
     inp = lasp_inputs.make_inputs(B, N, H, d, seed=7 + N + d + C, bf16=bf16, decayed=decayed)
     gpu = run_fwd_bwd(inp, C)
-    _compare(gpu, _oracle_all(inp, C), bf16)
+    ref = _oracle_all(inp, C)
+    _compare(gpu, ref, bf16)
+    # the chunk-entering states P_c and R_c, through the state entry points
+    _compare(run_states(inp, C, gpu["P"], gpu["R"]), ref, bf16, names=("P", "R"))
 
 
 @pytest.mark.parametrize("bf16,N,C", [(False, 256, 64), (True, 256, 64), (True, 2048, 128)])
@@ -67,7 +70,8 @@ def test_entering_states_against_oracle(bf16, N, C):
     din = (rng.standard_normal((B, H, d, d)) * 0.2).astype(np.float32)
     gpu = run_fwd_bwd(inp, C, init=init, dstate_in=din, want_dinit=True)
     ref = _oracle_all(inp, C, init=init.astype(np.float64), dstate_in=din.astype(np.float64))
-    _compare(gpu, ref, bf16, names=("o", "dq", "dk", "dv", "P", "R", "dinit"))
+    _compare(gpu, ref, bf16, names=("o", "dq", "dk", "dv", "dinit"))
+    _compare(run_states(inp, C, gpu["P"], gpu["R"], init=init, dstate_in=din), ref, bf16, names=("P", "R"))
 
 
 def test_chunk_size_invariance():
@@ -85,7 +89,7 @@ def test_no_decay_equals_all_ones_bitwise():
     inp = lasp_inputs.make_inputs(1, 256, 2, 128, seed=92, bf16=True, decayed=False)
     a = run_fwd_bwd(inp, 64, decay_override=None)
     b = run_fwd_bwd(inp, 64, decay_override=np.ones(2, np.float32))
-    for n in ("o", "dq", "dk", "dv", "P", "R"):
+    for n in ("o", "dq", "dk", "dv"):
         assert torch.equal(a[n], b[n]), n
 
 
@@ -127,7 +131,8 @@ def test_state_entry_points_against_oracle():
 
 
 def test_outputs_stay_inside_their_buffers():
-    """Guard regions around every output keep their sentinel bytes."""
+    """Guard regions around every output, the state cache and the workspace
+    keep their sentinel bytes; every output element is written."""
     import torch
     import sequence_linear_attention_b200 as lasp
     B, H, N, d, C = 1, 3, 320, 128, 64
@@ -153,7 +158,8 @@ def test_outputs_stay_inside_their_buffers():
     torch.cuda.synchronize()
     for name, (buf, _) in bufs.items():
         assert torch.isnan(buf[:G]).all() and torch.isnan(buf[-G:]).all(), name
-        assert not torch.isnan(buf[G:-G]).any(), name
+        if name in ("o", "dq", "dk", "dv"):
+            assert not torch.isnan(buf[G:-G]).any(), name
 
 
 def test_invalid_decay_is_recorded():

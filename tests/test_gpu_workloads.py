@@ -9,7 +9,7 @@ import pytest
 
 import oracle
 from sequence_linear_attention_b200 import inputs as lasp_inputs
-from gpu_helpers import decay_device, rel_err, run_fwd_bwd, to_device, to_host, tol
+from gpu_helpers import decay_device, rel_err, run_fwd_bwd, run_states, to_device, to_host, tol
 
 pytestmark = pytest.mark.gpu
 W = lasp_inputs.WORKLOADS
@@ -43,6 +43,8 @@ def _run(name, heads):
     inp = lasp_inputs.make_inputs(w["B"], w["N"], w["H"], w["d"], seed=w["seed"], bf16=w["bf16"],
                                   decayed=w["decayed"])
     gpu = run_fwd_bwd(inp, w["C"])
+    # P_c and R_c through the state entry points, into the (now free) cache and workspace
+    gpu.update(run_states(inp, w["C"], gpu["P"], gpu["R"]))
     return _check_heads(inp, gpu, w["C"], heads)
 
 
