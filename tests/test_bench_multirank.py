@@ -50,4 +50,6 @@ def test_single_rank_needs_no_process_group():
     import bench
     assert bench.aggregate(500.0, 0.5, 1) == (1000.0, 0.5)
     assert bench.algorithmic_bytes("state_scan", 1, 128, 128, 1024, 2) == 2 * 128 * 128 * 4 / 128
-    assert bench.algorithmic_bytes("fwd_walk_tc", 1, 128, 128, 1024, 2) == 4 * 128 * 2 + 128 * 128 * 4 / 128
+    s4 = 4 * 128 * 128
+    assert bench.algorithmic_bytes("fwd_walk_tc", 1, 128, 128, 1024, 2) == 4 * 128 * 2 + s4 / 1024 + s4 / 256
+    assert bench.algorithmic_bytes("fwd_walk_tc", 1, 128, 256, 1024, 2) == 4 * 128 * 2 + s4 / 256
