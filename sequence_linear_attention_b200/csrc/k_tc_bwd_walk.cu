@@ -18,7 +18,8 @@
 //   MMA 2:  T0 = dP' K
 //   epi 2:  dQ = T0 + lambda^{i+1} T2 -> global;  K <- diag(lambda^{127-j}) K
 //   MMA 3:  T0 = dP'^T Q + V~ R^T  (dK),  T1 = S'^T dO + K~ R  (dV)
-//   epi 3:  dK -> A, dV -> B (TMA stores);  Q <- diag(lambda^{j+1}) Q
+//   epi 3:  Q <- diag(lambda^{j+1}) Q;  then, while MMA 4 runs, dK -> A,
+//           dV -> B (TMA stores)
 //   MMA 4:  R += Q~^T dO          (the state for chunk c - 1)
 //
 // The decays of the dK/dV inter terms ride on the bf16 operands V~ and K~ so
@@ -182,7 +183,10 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_walk_tc(
     bulk_load(sX, src, kTileBytes, &s->ld_p);
   };
 
-  if (tid == 0 && (int64_t)blockIdx.x < nitems) {
+  // thread 32 issues every TMA load and bulk copy (and waits for the stores it
+  // issued); thread 0 issues the MMAs
+  constexpr int kProducer = 32;
+  if (tid == kProducer && (int64_t)blockIdx.x < nitems) {
     const Item first = item_of(blockIdx.x, H, nseg);
     load_kv(first, tiles - 1);
     load_qd(first, tiles - 1);
@@ -236,8 +240,12 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_walk_tc(
       const int64_t c = row0 / kTile;  // chunk index (C = tile)
 
       // the previous chunk's dK/dV stores must have left A and B before epilogue 1
-      if (tid == 0) tma_store_wait_read0();
+      if (tid == kProducer) tma_store_wait_read0();
       __syncthreads();
+      if (s->abort) {
+        stop = true;
+        break;
+      }
 
       // ---- MMA 1
       if (tid == 0) {
@@ -354,8 +362,50 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_walk_tc(
         for (int kk = 0; kk < kD / 16; ++kk) mma_bf16(tmem + T1, kmaj(aK, kk), mnmaj(aX, kk), id_kn, 1);
         mma_commit(&s->c3);
       }
-      // ---- epilogue 3: dK -> A, dV -> B; Q~ = diag(lambda^{j+1}) Q
+      // ---- epilogue 3, first Q~ = diag(lambda^{j+1}) Q so that MMA 4 and the
+      // next chunk's loads can start, then dK -> A, dV -> B
       if (mbar_wait(&s->c3, par, SITE_BWD_MMA)) {
+        tc_fence_after();
+        if (scale) {
+          scale_rows(sQ, s->pw, false, lam, tid);  // lambda^{j+1} = pw[j] * lambda
+          fence_async_smem();
+        }
+      } else {
+        s->abort = 1;
+      }
+      tc_fence_before();
+      __syncthreads();
+      if (s->abort) {
+        stop = true;
+        break;
+      }
+      if (tid == 0) {
+        tc_fence_after();
+        // ---- MMA 4: R += Q~^T dO (TMEM R was pre-scaled by lambda^128 in epilogue 1)
+        for (int kk = 0; kk < kTile / 16; ++kk) mma_bf16(tmem + TR, mnmaj(aQ, kk), mnmaj(aD, kk), id_nn, 1);
+        mma_commit(&s->c4);
+      }
+      if (tid == kProducer) {
+        // next chunk of this CTA's stream: K, V and X were read by MMA 3, Q and dO
+        // are free once MMA 4 is done
+        Item nx = item;
+        int nt = t - 1;
+        bool has_next = true;
+        if (nt < 0) {
+          has_next = w + gridDim.x < nitems;
+          if (has_next) {
+            nx = item_of(w + gridDim.x, H, nseg);
+            nt = tiles - 1;
+          }
+        }
+        if (has_next) {
+          load_kv(nx, nt);
+          load_p(nx, nt);
+          if (mbar_wait(&s->c4, par, SITE_BWD_MMA)) load_qd(nx, nt);
+          else s->abort = 1;
+        }
+      }
+      {
         tc_fence_after();
 #pragma unroll 1
         for (int cc = 2 * half; cc < 2 * half + 2; ++cc) {
@@ -372,49 +422,20 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_walk_tc(
           st_row32_bf16(sA, i, cc * 32, fk);
           st_row32_bf16(sB, i, cc * 32, fv);
         }
-        if (scale) scale_rows(sQ, s->pw, false, lam, tid);  // lambda^{j+1} = pw[j] * lambda
         fence_async_smem();
-      } else {
-        s->abort = 1;
       }
       tc_fence_before();
       __syncthreads();
-      if (s->abort) {
-        stop = true;
-        break;
-      }
-
-      if (tid == 0) {
-        tc_fence_after();
-        // ---- MMA 4: R += Q~^T dO (TMEM R was pre-scaled by lambda^128 in epilogue 1)
-        for (int kk = 0; kk < kTile / 16; ++kk) mma_bf16(tmem + TR, mnmaj(aQ, kk), mnmaj(aD, kk), id_nn, 1);
-        mma_commit(&s->c4);
+      if (tid == kProducer) {
         tma_store_4d(&map_dk, sA, 0, item.h, row0, item.b);
         tma_store_4d(&map_dk, sA + kBox, 64, item.h, row0, item.b);
         tma_store_4d(&map_dv, sB, 0, item.h, row0, item.b);
         tma_store_4d(&map_dv, sB + kBox, 64, item.h, row0, item.b);
         tma_store_commit();
-        // next chunk of this CTA's stream: K, V are free now, Q and dO once MMA 4 is done
-        Item nx = item;
-        int nt = t - 1;
-        bool has_next = true;
-        if (nt < 0) {
-          has_next = w + gridDim.x < nitems;
-          if (has_next) {
-            nx = item_of(w + gridDim.x, H, nseg);
-            nt = tiles - 1;
-          }
-        }
-        if (has_next) {
-          load_kv(nx, nt);
-          load_p(nx, nt);  // X (R) has been read by MMA 3
-          if (mbar_wait(&s->c4, par, SITE_BWD_MMA)) load_qd(nx, nt);
-          else s->abort = 1;
-        }
       }
     }
   }
-  if (tid == 0) tma_store_wait0();
+  if (tid == kProducer) tma_store_wait0();
   tc_fence_before();
   __syncthreads();
   if (warp == 0) tmem_dealloc(tmem, kTmemCols);

@@ -143,7 +143,10 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_walk_tc(const __grid_constant
     tma_load_4d(q + 2 * kTileBytes + kBox, &map_v, &s->load[set], 64, it.h, row, it.b);
   };
 
-  if (tid == 0 && (int64_t)blockIdx.x < nitems) issue_loads(0, item_of(blockIdx.x, H, nseg), 0);
+  // thread 32 issues every TMA load and bulk copy (and waits for the stores it
+  // issued); thread 0 issues the MMAs
+  constexpr int kProducer = 32;
+  if (tid == kProducer && (int64_t)blockIdx.x < nitems) issue_loads(0, item_of(blockIdx.x, H, nseg), 0);
 
   constexpr uint32_t id_kk = idesc_bf16(128, 128, 0, 0);
   constexpr uint32_t id_kn = idesc_bf16(128, 128, 0, 1);
@@ -195,16 +198,9 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_walk_tc(const __grid_constant
       uint8_t* sV = sQ + 2 * kTileBytes;
       const int row0 = item.seg * G + t * kTile;
 
-      if (tid == 0 && cache_bf16) {
-        // the bf16 operand tile of the state entering this chunk, as it sits in
-        // shared memory, is the cache entry the backward pass loads back
-        uint8_t* slot = reinterpret_cast<uint8_t*>(P + (((int64_t)item.b * T + row0 / C) * H + item.h) * kD * kD);
-        bulk_store(slot, sP, kTileBytes);
-        tma_store_commit();
-      }
-      if (tid == 0) {
-        // prefetch the next tile of this CTA's stream into the other set; its
-        // K buffer may still be the source of the previous tile's TMA store
+      if (tid == kProducer) {
+        // prefetch the next tile of this CTA's stream into the other set; its K
+        // buffer is the source of the previous tile's output store
         Item nx = item;
         int nt = t + 1;
         bool has_next = true;
@@ -217,6 +213,15 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_walk_tc(const __grid_constant
           tma_store_wait_read0();
           issue_loads(set ^ 1, nx, nt);
         }
+        if (cache_bf16) {
+          // the bf16 operand tile of the state entering this chunk, as it sits
+          // in shared memory, is the cache entry the backward pass loads back
+          uint8_t* slot = reinterpret_cast<uint8_t*>(P + (((int64_t)item.b * T + row0 / C) * H + item.h) * kD * kD);
+          bulk_store(slot, sP, kTileBytes);
+          tma_store_commit();
+        }
+      }
+      if (tid == 0) {
         // MMA 1: S = Q K^T, O_inter = Q P
         if (mbar_wait(&s->load[set], (it >> 1) & 1u, SITE_OUT_TMA)) {
           tc_fence_after();
@@ -297,7 +302,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_walk_tc(const __grid_constant
       } else {
         s->abort = 1;
       }
-      if (tid == 0 && cache_bf16) tma_store_wait_read0();  // epilogue B rewrites sP
+      if (tid == kProducer && cache_bf16) tma_store_wait_read0();  // epilogue B rewrites sP
       tc_fence_before();
       __syncthreads();
       if (s->abort) {
@@ -357,14 +362,14 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_walk_tc(const __grid_constant
         stop = true;
         break;
       }
-      if (tid == 0) {
+      if (tid == kProducer) {
         tma_store_4d(&map_o, sK, 0, item.h, row0, item.b);
         tma_store_4d(&map_o, sK + kBox, 64, item.h, row0, item.b);
         tma_store_commit();
       }
     }
   }
-  if (tid == 0) tma_store_wait0();
+  if (tid == kProducer) tma_store_wait0();
   tc_fence_before();
   __syncthreads();
   if (warp == 0) tmem_dealloc(tmem, kTmemCols);
