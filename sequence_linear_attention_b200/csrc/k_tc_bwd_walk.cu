@@ -16,15 +16,15 @@
 //           R -> bf16 X (replacing P),  R <- lambda^128 R in TMEM;
 //           V <- diag(lambda^{127-j}) V in place
 //   MMA 2:  T0 = dP' K
-//   epi 2:  dQ = T0 + lambda^{i+1} T2 -> global;  K <- diag(lambda^{127-j}) K
-//   MMA 3:  T0 = dP'^T Q + V~ R^T  (dK),  T1 = S'^T dO + K~ R  (dV)
+//   epi 2:  dQ = T0 + lambda^{i+1} T2 -> global
+//   MMA 3:  T0 = dP'^T Q + V~ R^T  (dK),  T1 = S'^T dO,  T2 = K R
 //   epi 3:  Q <- diag(lambda^{j+1}) Q;  then, while MMA 4 runs, dK -> A,
-//           dV -> B (TMA stores)
+//           dV = T1 + lambda^{127-j} T2 -> B (TMA stores)
 //   MMA 4:  R += Q~^T dO          (the state for chunk c - 1)
 //
-// The decays of the dK/dV inter terms ride on the bf16 operands V~ and K~ so
-// both terms share an accumulator; the dQ inter term keeps its fp32 row
-// scaling. The next chunk's K, V and P are loaded as soon as MMA 3 has read
+// The decay of the dK inter term rides on the bf16 operand V~ so both dK terms
+// share an accumulator (TMEM has no fifth block); the dQ and dV inter terms
+// keep fp32 row scalings. The next chunk's K, V and P are loaded as soon as MMA 3 has read
 // the buffers they replace, its Q and dO once MMA 4 has. R is not stored per
 // chunk: only the segment-level slots of the workspace are used. In every epilogue warp w owns TMEM lanes
 // (rows) 32*(w%4).. and the column half w/4.
@@ -341,7 +341,6 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_walk_tc(
                 make_uint4(pack_bf16(o[0], o[1]), pack_bf16(o[2], o[3]), pack_bf16(o[4], o[5]), pack_bf16(o[6], o[7]));
           }
         }
-        if (scale) scale_rows(sK, s->pw, true, 1.f, tid);  // K~ = diag(lambda^{127-j}) K
         fence_async_smem();
       } else {
         s->abort = 1;
@@ -353,13 +352,13 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_walk_tc(
         break;
       }
 
-      // ---- MMA 3: dK = dP'^T Q + V~ R^T, dV = S'^T dO + K~ R
+      // ---- MMA 3: dK = dP'^T Q + V~ R^T, dV_intra = S'^T dO, dV_inter = K R
       if (tid == 0) {
         tc_fence_after();
         for (int kk = 0; kk < kTile / 16; ++kk) mma_bf16(tmem + T0, mnmaj(aA, kk), mnmaj(aQ, kk), id_nn, kk != 0);
         for (int kk = 0; kk < kD / 16; ++kk) mma_bf16(tmem + T0, kmaj(aV, kk), kmaj(aX, kk), id_kk, 1);
         for (int kk = 0; kk < kTile / 16; ++kk) mma_bf16(tmem + T1, mnmaj(aB, kk), mnmaj(aD, kk), id_nn, kk != 0);
-        for (int kk = 0; kk < kD / 16; ++kk) mma_bf16(tmem + T1, kmaj(aK, kk), mnmaj(aX, kk), id_kn, 1);
+        for (int kk = 0; kk < kD / 16; ++kk) mma_bf16(tmem + T2, kmaj(aK, kk), mnmaj(aX, kk), id_kn, kk != 0);
         mma_commit(&s->c3);
       }
       // ---- epilogue 3, first Q~ = diag(lambda^{j+1}) Q so that MMA 4 and the
@@ -407,17 +406,19 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_walk_tc(
       }
       {
         tc_fence_after();
+        const float wj = decay_pow(l2, (float)(kTile - 1 - i));  // dV inter decay of row j = i
 #pragma unroll 1
         for (int cc = 2 * half; cc < 2 * half + 2; ++cc) {
-          uint32_t ka[32], va[32];
+          uint32_t ka[32], va[32], ve[32];
           tmem_ld32(lane_base + T0 + cc * 32, ka);
           tmem_ld32(lane_base + T1 + cc * 32, va);
+          tmem_ld32(lane_base + T2 + cc * 32, ve);
           tmem_ld_wait();
           float fk[32], fv[32];
 #pragma unroll
           for (int q = 0; q < 32; ++q) {
             fk[q] = __uint_as_float(ka[q]);
-            fv[q] = __uint_as_float(va[q]);
+            fv[q] = fmaf(wj, __uint_as_float(ve[q]), __uint_as_float(va[q]));
           }
           st_row32_bf16(sA, i, cc * 32, fk);
           st_row32_bf16(sB, i, cc * 32, fv);

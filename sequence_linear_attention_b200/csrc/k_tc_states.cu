@@ -3,16 +3,18 @@
 //   M_c = (diag(w) A_c)^T B_c,   A_c, B_c = C x d token tiles of chunk c,
 //   w_t = lambda^{C-1-t} (kind 0, (A, B) = (K, V)) or lambda^{t+1} (kind 1, (Q, dO)).
 //
-// One CTA per (chunk, head, batch), 256 threads. The chunk is consumed in
-// stages of KB tokens (KB = 128, or the largest of 64/32/16 dividing C). Per
+// Persistent CTAs (one per SM, 256 threads) take the (chunk, head, batch)
+// items in turn. A chunk is consumed in stages of KB tokens (KB = 128, or the
+// largest of 64/32/16 dividing C), and the stages of all of a CTA's chunks
+// form one stream. Per
 // stage: TMA brings A and B (KB rows x 128 features, two 64-feature boxes each,
 // 128-byte swizzle) into a shared-memory slot; when lambda != 1 the four warps
 // scale the rows of A by w_t in place (bf16); one thread issues KB/16
 // tcgen05.mma (M = N = 128 features, K = 16 tokens) that accumulate M_c in
 // TMEM. Both operands are MN-major: the tiles arrive token-major with features
 // contiguous, which is exactly A^T and B with the reduced (token) index as the
-// slow one. Up to three slots keep two stages' loads in flight under the
-// current stage's scaling and MMAs. The epilogue reads the 128 x 128 fp32
+// slow one. Three slots keep two stages' loads in flight under the current
+// stage's scaling and MMAs (thread 32 issues the loads, thread 0 the MMAs). The epilogue reads the 128 x 128 fp32
 // accumulator from TMEM (warp w: rows 32*(w%4).., column half w/4) and writes
 // the state row by row.
 #include <algorithm>
@@ -61,24 +63,39 @@ __device__ __forceinline__ void issue_stage(uint8_t* tiles, uint32_t tile_bytes,
   tma_load_4d(bb + tile_bytes / 2, map_b, &s->full[slot], 64, h, row, b);
 }
 
+// Work item n of this CTA (chunk index c, head h, batch b).
+struct Work {
+  int c, h, b;
+};
+__device__ __forceinline__ Work work_of(int64_t n, int T, int H) {
+  const int64_t w = blockIdx.x + n * gridDim.x;
+  Work r;
+  r.c = (int)(w % T);
+  r.h = (int)((w / T) % H);
+  r.b = (int)(w / ((int64_t)T * H));
+  return r;
+}
+
+// Persistent: each CTA takes chunks blockIdx.x, blockIdx.x + gridDim.x, ...
+// and consumes their stages as one stream, so the next chunk's loads are in
+// flight during the current chunk's epilogue.
 __global__ void __launch_bounds__(kThreads, 1) chunk_states_tc(const __grid_constant__ CUtensorMap map_a,
                                                             const __grid_constant__ CUtensorMap map_b,
                                                             const float* decay, float* __restrict__ M, int H,
-                                                            int C, int KB, int kind, int64_t t_out,
-                                                            int slot_stride, int slot_offset) {
+                                                            int C, int KB, int kind, int T, int64_t nitems,
+                                                            int64_t t_out, int slot_stride, int slot_offset) {
   extern __shared__ uint8_t smem_raw[];
   // tiles need 1024-byte alignment for the 128-byte swizzle atoms
   uint8_t* tiles = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   const int nstages = C / KB;
-  const int nslots = nstages < kMaxSlots ? nstages : kMaxSlots;
   const uint32_t tile_bytes = (uint32_t)KB * 256;  // KB rows x 128 features x bf16
-  Smem* s = reinterpret_cast<Smem*>(tiles + nslots * 2 * tile_bytes);
+  Smem* s = reinterpret_cast<Smem*>(tiles + kMaxSlots * 2 * tile_bytes);
+  const int nslots = kMaxSlots;
 
-  const int c = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const float lam = load_decay(decay, h);
-  const float l2 = log2f(lam);
-  const bool scale = lam != 1.0f;
+  constexpr int kProducer = 32;  // issues the TMA loads; thread 0 issues the MMAs
+  const int64_t my_items = nitems > blockIdx.x ? (nitems - 1 - blockIdx.x) / gridDim.x + 1 : 0;
+  const int64_t nstream = my_items * nstages;  // stages this CTA consumes
 
   if (tid == 0) {
     prefetch_tmap(&map_a);
@@ -100,33 +117,43 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_states_tc(const __grid_cons
   tc_fence_after();
   const uint32_t tmem = s->tmem_base;
 
-  if (tid == 0) {
-    for (int k = 0; k < nslots; ++k) issue_stage(tiles, tile_bytes, s, &map_a, &map_b, k, c * C + k * KB, h, b);
-  }
+  auto issue = [&](int64_t g) {
+    const Work wk = work_of(g / nstages, T, H);
+    const int k = (int)(g % nstages);
+    issue_stage(tiles, tile_bytes, s, &map_a, &map_b, (int)(g % nslots), wk.c * C + k * KB, wk.h, wk.b);
+  };
+  if (tid == kProducer)
+    for (int64_t g = 0; g < nslots && g < nstream; ++g) issue(g);
 
   constexpr uint32_t idesc = idesc_bf16(128, 128, 1, 1);
-  for (int k = 0; k < nstages; ++k) {
-    const int slot = k % nslots;
-    const uint32_t par = (uint32_t)(k / nslots) & 1u;
+  for (int64_t g = 0; g < nstream; ++g) {
+    const int slot = (int)(g % nslots);
+    const uint32_t par = (uint32_t)((g / nslots) & 1);
+    const int k = (int)(g % nstages);
+    const int64_t n = g / nstages;
+    const Work wk = work_of(n, T, H);
+    const float lam = load_decay(decay, wk.h);
+    const float l2 = log2f(lam);
     if (!mbar_wait(&s->full[slot], par, SITE_STATES_TMA)) s->abort = 1;
-    if (scale) {
+    if (lam != 1.0f) {
       // scale row r of A by w_{k*KB + r}; the row of a 16-byte chunk is its
       // byte offset / 128 in either 64-feature box, whatever the swizzle
       uint4* a = reinterpret_cast<uint4*>(tiles + (size_t)slot * 2 * tile_bytes);
       const int nchunks = KB * 16;
-      for (int g = tid; g < nchunks; g += kThreads) {
-        const int r = (g % (KB * 8)) / 8;
+      for (int q = tid; q < nchunks; q += kThreads) {
+        const int r = (q % (KB * 8)) / 8;
         const int t = k * KB + r;
         const float w = kind == 0 ? decay_pow(l2, (float)(C - 1 - t)) : decay_pow(l2, (float)(t + 1));
-        uint4 x = a[g];
+        uint4 x = a[q];
         x.x = bf16x2_scale(x.x, w);
         x.y = bf16x2_scale(x.y, w);
         x.z = bf16x2_scale(x.z, w);
         x.w = bf16x2_scale(x.w, w);
-        a[g] = x;
+        a[q] = x;
       }
       fence_async_smem();
     }
+    tc_fence_before();
     __syncthreads();
     if (s->abort) break;
     if (tid == 0) {
@@ -137,38 +164,43 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_states_tc(const __grid_cons
         const uint64_t bd = sw128_desc(b0 + j * 2048, KB * 128, 1024);
         mma_bf16(tmem, ad, bd, idesc, (k | j) != 0);
       }
-      mma_commit(k + 1 < nstages ? &s->empty[slot] : &s->done);
-      // refill the slot of the previous stage (its MMAs were issued one stage
-      // ago), keeping nslots - 1 stages in flight while this one is consumed
-      const int kr = k - 1 + nslots;
-      if (k >= 1 && kr < nstages) {
-        const int pslot = (k - 1) % nslots;
-        if (mbar_wait(&s->empty[pslot], (uint32_t)((k - 1) / nslots) & 1u, SITE_STATES_MMA))
-          issue_stage(tiles, tile_bytes, s, &map_a, &map_b, pslot, c * C + kr * KB, h, b);
-        else
-          s->abort = 1;
-      }
+      mma_commit(&s->empty[slot]);
+      if (k == nstages - 1) mma_commit(&s->done);
     }
-  }
-  __syncthreads();
-  const bool ok = !s->abort && mbar_wait(&s->done, 0, SITE_STATES_MMA);
-  tc_fence_after();
-  if (ok) {
-    // warp w reads TMEM lanes (rows) 32*(w%4).. and the column half w/4
-    const int row = (warp & 3) * 32 + lane, half = warp >> 2;
-    // chunk c's state goes to slot c * slot_stride + slot_offset of an array with t_out slots
-    const int64_t slot = (int64_t)c * slot_stride + slot_offset;
-    float* out = M + ((((int64_t)b * t_out + slot) * H + h) * kD + row) * kD;
-#pragma unroll 1
-    for (int cc = 2 * half; cc < 2 * half + 2; ++cc) {
-      uint32_t r[32];
-      tmem_ld32(tmem + ((uint32_t)((warp & 3) * 32) << 16) + cc * 32, r);
-      tmem_ld_wait();
-      float4* o4 = reinterpret_cast<float4*>(out + cc * 32);
+    if (tid == kProducer && g >= 1 && g - 1 + nslots < nstream) {
+      // refill the slot of the previous stage (its MMAs were issued one step
+      // ago), keeping nslots - 1 stages in flight while this one is consumed
+      const int64_t gp = g - 1;
+      if (mbar_wait(&s->empty[gp % nslots], (uint32_t)((gp / nslots) & 1), SITE_STATES_MMA)) issue(gp + nslots);
+      else s->abort = 1;
+    }
+    if (k == nstages - 1) {
+      // epilogue of this chunk: warp w reads TMEM lanes (rows) 32*(w%4).. and the
+      // column half w/4; the state goes to slot c * slot_stride + slot_offset
+      if (mbar_wait(&s->done, (uint32_t)(n & 1), SITE_STATES_MMA)) {
+        tc_fence_after();
+        const int row = (warp & 3) * 32 + lane, half = warp >> 2;
+        const int64_t oslot = (int64_t)wk.c * slot_stride + slot_offset;
+        float* out = M + ((((int64_t)wk.b * t_out + oslot) * H + wk.h) * kD + row) * kD;
+        uint32_t r0[32], r1[32];
+        tmem_ld32(tmem + ((uint32_t)((warp & 3) * 32) << 16) + (2 * half) * 32, r0);
+        tmem_ld32(tmem + ((uint32_t)((warp & 3) * 32) << 16) + (2 * half + 1) * 32, r1);
+        tmem_ld_wait();
+        float4* o0 = reinterpret_cast<float4*>(out + (2 * half) * 32);
+        float4* o1 = reinterpret_cast<float4*>(out + (2 * half + 1) * 32);
 #pragma unroll
-      for (int q = 0; q < 8; ++q)
-        o4[q] = make_float4(__uint_as_float(r[4 * q]), __uint_as_float(r[4 * q + 1]), __uint_as_float(r[4 * q + 2]),
-                            __uint_as_float(r[4 * q + 3]));
+        for (int q = 0; q < 8; ++q) {
+          __stcs(o0 + q, make_float4(__uint_as_float(r0[4 * q]), __uint_as_float(r0[4 * q + 1]),
+                                     __uint_as_float(r0[4 * q + 2]), __uint_as_float(r0[4 * q + 3])));
+          __stcs(o1 + q, make_float4(__uint_as_float(r1[4 * q]), __uint_as_float(r1[4 * q + 1]),
+                                     __uint_as_float(r1[4 * q + 2]), __uint_as_float(r1[4 * q + 3])));
+        }
+      } else {
+        s->abort = 1;
+      }
+      // the next chunk's first MMA overwrites the accumulator
+      tc_fence_before();
+      __syncthreads();
     }
   }
   tc_fence_before();
@@ -196,12 +228,16 @@ cudaError_t tc_chunk_states_slots(const void* a, const void* bm, const float* de
   CUtensorMap ma, mb;
   if (!make_token_map(&ma, a, B, H, N, d, KB) || !make_token_map(&mb, bm, B, H, N, d, KB))
     return cudaErrorInvalidValue;
-  const int nslots = std::min(C / KB, kMaxSlots);
-  const size_t smem = 1024 + (size_t)nslots * 2 * KB * 256 + sizeof(Smem);
+  const size_t smem = 1024 + (size_t)kMaxSlots * 2 * KB * 256 + sizeof(Smem);
   cudaError_t e = cudaFuncSetAttribute(chunk_states_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  dim3 grid((unsigned)(N / C), H, B);
-  chunk_states_tc<<<grid, kThreads, smem, st>>>(ma, mb, decay, M, H, C, KB, kind, t_out, slot_stride, slot_offset);
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int T = (int)(N / C);
+  const int64_t nitems = (int64_t)B * H * T;
+  const unsigned grid = (unsigned)std::min<int64_t>(nitems, sms);
+  chunk_states_tc<<<grid, kThreads, smem, st>>>(ma, mb, decay, M, H, C, KB, kind, T, nitems, t_out, slot_stride,
+                                               slot_offset);
   return cudaGetLastError();
 }
 
