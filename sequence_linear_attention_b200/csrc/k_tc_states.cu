@@ -13,8 +13,9 @@
 // tcgen05.mma (M = N = 128 features, K = 16 tokens) that accumulate M_c in
 // TMEM. Both operands are MN-major: the tiles arrive token-major with features
 // contiguous, which is exactly A^T and B with the reduced (token) index as the
-// slow one. Three slots keep two stages' loads in flight under the current
-// stage's scaling and MMAs (thread 32 issues the loads, thread 0 the MMAs). The epilogue reads the 128 x 128 fp32
+// slow one. Up to six slots (192 KB) keep all but one stage's loads in flight
+// under the current stage's scaling and MMAs (thread 32 issues the loads,
+// thread 0 the MMAs). The epilogue reads the 128 x 128 fp32
 // accumulator from TMEM (warp w: rows 32*(w%4).., column half w/4) and writes
 // the state row by row.
 #include <algorithm>
@@ -32,7 +33,8 @@ using namespace sm100;
 
 constexpr int kD = 128;           // head dimension handled here
 constexpr int kThreads = 256;
-constexpr int kMaxSlots = 3;
+constexpr int kMaxSlots = 6;
+constexpr size_t kStageBudget = 192 * 1024;  // shared memory for the stage slots
 constexpr uint32_t kTmemCols = 128;  // one 128 x 128 fp32 accumulator
 
 struct Smem {
@@ -82,15 +84,15 @@ __device__ __forceinline__ Work work_of(int64_t n, int T, int H) {
 __global__ void __launch_bounds__(kThreads, 1) chunk_states_tc(const __grid_constant__ CUtensorMap map_a,
                                                             const __grid_constant__ CUtensorMap map_b,
                                                             const float* decay, float* __restrict__ M, int H,
-                                                            int C, int KB, int kind, int T, int64_t nitems,
-                                                            int64_t t_out, int slot_stride, int slot_offset) {
+                                                            int C, int KB, int nslots, int kind, int T,
+                                                            int64_t nitems, int64_t t_out, int slot_stride,
+                                                            int slot_offset) {
   extern __shared__ uint8_t smem_raw[];
   // tiles need 1024-byte alignment for the 128-byte swizzle atoms
   uint8_t* tiles = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   const int nstages = C / KB;
   const uint32_t tile_bytes = (uint32_t)KB * 256;  // KB rows x 128 features x bf16
-  Smem* s = reinterpret_cast<Smem*>(tiles + kMaxSlots * 2 * tile_bytes);
-  const int nslots = kMaxSlots;
+  Smem* s = reinterpret_cast<Smem*>(tiles + nslots * 2 * tile_bytes);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   constexpr int kProducer = 32;  // issues the TMA loads; thread 0 issues the MMAs
@@ -126,14 +128,18 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_states_tc(const __grid_cons
     for (int64_t g = 0; g < nslots && g < nstream; ++g) issue(g);
 
   constexpr uint32_t idesc = idesc_bf16(128, 128, 1, 1);
+  Work wk{0, 0, 0};
+  float lam = 1.f, l2 = 0.f;
   for (int64_t g = 0; g < nstream; ++g) {
     const int slot = (int)(g % nslots);
     const uint32_t par = (uint32_t)((g / nslots) & 1);
     const int k = (int)(g % nstages);
     const int64_t n = g / nstages;
-    const Work wk = work_of(n, T, H);
-    const float lam = load_decay(decay, wk.h);
-    const float l2 = log2f(lam);
+    if (k == 0) {  // a new chunk: its coordinates and decay
+      wk = work_of(n, T, H);
+      lam = load_decay(decay, wk.h);
+      l2 = log2f(lam);
+    }
     if (!mbar_wait(&s->full[slot], par, SITE_STATES_TMA)) s->abort = 1;
     if (lam != 1.0f) {
       // scale row r of A by w_{k*KB + r}; the row of a 16-byte chunk is its
@@ -208,7 +214,10 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_states_tc(const __grid_cons
   if (warp == 0) tmem_dealloc(tmem, kTmemCols);
 }
 
+// Stage rows: 64 for long chunks (more, smaller stages in flight), else the
+// largest of 128/64/32/16 dividing C.
 inline int stage_rows(int C) {
+  if (C >= 256 && C % 64 == 0) return 64;
   for (int kb : {128, 64, 32, 16})
     if (C % kb == 0) return kb;
   return 0;
@@ -228,7 +237,8 @@ cudaError_t tc_chunk_states_slots(const void* a, const void* bm, const float* de
   CUtensorMap ma, mb;
   if (!make_token_map(&ma, a, B, H, N, d, KB) || !make_token_map(&mb, bm, B, H, N, d, KB))
     return cudaErrorInvalidValue;
-  const size_t smem = 1024 + (size_t)kMaxSlots * 2 * KB * 256 + sizeof(Smem);
+  const int nslots = (int)std::min<size_t>(kMaxSlots, kStageBudget / ((size_t)2 * KB * 256));
+  const size_t smem = 1024 + (size_t)nslots * 2 * KB * 256 + sizeof(Smem);
   cudaError_t e = cudaFuncSetAttribute(chunk_states_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   int dev = 0, sms = 148;
@@ -236,8 +246,8 @@ cudaError_t tc_chunk_states_slots(const void* a, const void* bm, const float* de
   const int T = (int)(N / C);
   const int64_t nitems = (int64_t)B * H * T;
   const unsigned grid = (unsigned)std::min<int64_t>(nitems, sms);
-  chunk_states_tc<<<grid, kThreads, smem, st>>>(ma, mb, decay, M, H, C, KB, kind, T, nitems, t_out, slot_stride,
-                                               slot_offset);
+  chunk_states_tc<<<grid, kThreads, smem, st>>>(ma, mb, decay, M, H, C, KB, nslots, kind, T, nitems, t_out,
+                                               slot_stride, slot_offset);
   return cudaGetLastError();
 }
 
