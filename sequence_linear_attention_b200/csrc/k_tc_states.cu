@@ -214,10 +214,8 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_states_tc(const __grid_cons
   if (warp == 0) tmem_dealloc(tmem, kTmemCols);
 }
 
-// Stage rows: 64 for long chunks (more, smaller stages in flight), else the
-// largest of 128/64/32/16 dividing C.
+// Stage rows: the largest of 128/64/32/16 dividing C.
 inline int stage_rows(int C) {
-  if (C >= 256 && C % 64 == 0) return 64;
   for (int kb : {128, 64, 32, 16})
     if (C % kb == 0) return kb;
   return 0;
