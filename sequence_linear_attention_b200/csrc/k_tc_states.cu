@@ -3,21 +3,19 @@
 //   M_c = (diag(w) A_c)^T B_c,   A_c, B_c = C x d token tiles of chunk c,
 //   w_t = lambda^{C-1-t} (kind 0, (A, B) = (K, V)) or lambda^{t+1} (kind 1, (Q, dO)).
 //
-// Persistent CTAs (one per SM, 256 threads) take the (chunk, head, batch)
-// items in turn. A chunk is consumed in stages of KB tokens (KB = 128, or the
-// largest of 64/32/16 dividing C), and the stages of all of a CTA's chunks
-// form one stream. Per
-// stage: TMA brings A and B (KB rows x 128 features, two 64-feature boxes each,
-// 128-byte swizzle) into a shared-memory slot; when lambda != 1 the four warps
-// scale the rows of A by w_t in place (bf16); one thread issues KB/16
-// tcgen05.mma (M = N = 128 features, K = 16 tokens) that accumulate M_c in
-// TMEM. Both operands are MN-major: the tiles arrive token-major with features
-// contiguous, which is exactly A^T and B with the reduced (token) index as the
-// slow one. Up to six slots (192 KB) keep all but one stage's loads in flight
-// under the current stage's scaling and MMAs (thread 32 issues the loads,
-// thread 0 the MMAs). The epilogue reads the 128 x 128 fp32
-// accumulator from TMEM (warp w: rows 32*(w%4).., column half w/4) and writes
-// the state row by row.
+// Persistent, warp-specialized CTAs (one per SM) take the (chunk, head,
+// batch) items in turn. A chunk is consumed in stages of KB tokens (KB = 128,
+// or the largest of 64/32/16 dividing C); the stages of all of a CTA's chunks
+// form one stream through up to six shared-memory slots (192 KB). Per stage:
+// warp 1 brings A and B by TMA (KB rows x 128 features, two 64-feature boxes
+// each, 128-byte swizzle); when lambda != 1 the four worker warps scale the
+// rows of A by w_t in place (bf16); warp 0 issues KB/16 tcgen05.mma (M = N =
+// 128 features, K = 16 tokens) accumulating M_c in TMEM. Both operands are
+// MN-major: the tiles arrive token-major with features contiguous, which is
+// exactly A^T and B with the reduced (token) index as the slow one. Two TMEM
+// accumulators alternate between chunks; the workers read a finished one
+// (warp w: TMEM lanes 32*(w%4)..) and write the state row by row while the
+// next chunk accumulates.
 #include <algorithm>
 
 #include "kernels.h"
@@ -31,16 +29,21 @@ namespace tc_states_detail {
 
 using namespace sm100;
 
-constexpr int kD = 128;           // head dimension handled here
-constexpr int kThreads = 256;
+constexpr int kD = 128;              // head dimension handled here
+constexpr int kThreads = 192;        // warp 0: MMA, warp 1: TMA, warps 2-5: scaling and epilogue
+constexpr int kWorkers = 128;
 constexpr int kMaxSlots = 6;
 constexpr size_t kStageBudget = 192 * 1024;  // shared memory for the stage slots
-constexpr uint32_t kTmemCols = 128;  // one 128 x 128 fp32 accumulator
+constexpr uint32_t kTmemCols = 256;  // two 128 x 128 fp32 accumulators
+
+__device__ __forceinline__ bool aborted(const int* flag) { return *(volatile const int*)flag != 0; }
 
 struct Smem {
-  uint64_t full[kMaxSlots];
-  uint64_t empty[kMaxSlots];
-  uint64_t done;
+  uint64_t full[kMaxSlots];    // TMA bytes of a stage have landed
+  uint64_t scaled[kMaxSlots];  // the workers have scaled a stage's A rows
+  uint64_t empty[kMaxSlots];   // the MMAs reading a stage have completed
+  uint64_t acc_full[2];        // an accumulator holds a finished state
+  uint64_t acc_empty[2];       // the workers have read an accumulator out
   uint32_t tmem_base;
   int abort;
 };
@@ -50,19 +53,6 @@ __device__ __forceinline__ uint32_t bf16x2_scale(uint32_t x, float w) {
   float2 f = __bfloat1622float2(h);
   __nv_bfloat162 r = __floats2bfloat162_rn(f.x * w, f.y * w);
   return *reinterpret_cast<uint32_t*>(&r);
-}
-
-// Issues the four TMA boxes of one stage (A and B, two 64-feature boxes each)
-// into `slot`.
-__device__ __forceinline__ void issue_stage(uint8_t* tiles, uint32_t tile_bytes, Smem* s, const CUtensorMap* map_a,
-                                            const CUtensorMap* map_b, int slot, int row, int h, int b) {
-  uint8_t* a = tiles + (size_t)slot * 2 * tile_bytes;
-  uint8_t* bb = a + tile_bytes;
-  mbar_arrive_expect_tx(&s->full[slot], 2 * tile_bytes);
-  tma_load_4d(a, map_a, &s->full[slot], 0, h, row, b);
-  tma_load_4d(a + tile_bytes / 2, map_a, &s->full[slot], 64, h, row, b);
-  tma_load_4d(bb, map_b, &s->full[slot], 0, h, row, b);
-  tma_load_4d(bb + tile_bytes / 2, map_b, &s->full[slot], 64, h, row, b);
 }
 
 // Work item n of this CTA (chunk index c, head h, batch b).
@@ -78,9 +68,13 @@ __device__ __forceinline__ Work work_of(int64_t n, int T, int H) {
   return r;
 }
 
-// Persistent: each CTA takes chunks blockIdx.x, blockIdx.x + gridDim.x, ...
-// and consumes their stages as one stream, so the next chunk's loads are in
-// flight during the current chunk's epilogue.
+// Persistent and warp-specialized: each CTA takes chunks blockIdx.x,
+// blockIdx.x + gridDim.x, ... and their KB-token stages form one stream that
+// flows through nslots shared-memory slots: warp 1 loads a stage, the four
+// worker warps scale its A rows by the decay weights, warp 0 issues its MMAs
+// into one of two TMEM accumulators; when a chunk's last stage is done the
+// workers read that accumulator out while the next chunk accumulates in the
+// other one. Hand-offs are mbarriers; no CTA-wide barrier in the stream.
 __global__ void __launch_bounds__(kThreads, 1) chunk_states_tc(const __grid_constant__ CUtensorMap map_a,
                                                             const __grid_constant__ CUtensorMap map_b,
                                                             const float* decay, float* __restrict__ M, int H,
@@ -95,18 +89,21 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_states_tc(const __grid_cons
   Smem* s = reinterpret_cast<Smem*>(tiles + nslots * 2 * tile_bytes);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  constexpr int kProducer = 32;  // issues the TMA loads; thread 0 issues the MMAs
   const int64_t my_items = nitems > blockIdx.x ? (nitems - 1 - blockIdx.x) / gridDim.x + 1 : 0;
-  const int64_t nstream = my_items * nstages;  // stages this CTA consumes
+  const int64_t nstream = my_items * nstages;
 
   if (tid == 0) {
     prefetch_tmap(&map_a);
     prefetch_tmap(&map_b);
     for (int q = 0; q < kMaxSlots; ++q) {
       mbar_init(&s->full[q], 1);
+      mbar_init(&s->scaled[q], kWorkers);
       mbar_init(&s->empty[q], 1);
     }
-    mbar_init(&s->done, 1);
+    for (int q = 0; q < 2; ++q) {
+      mbar_init(&s->acc_full[q], 1);
+      mbar_init(&s->acc_empty[q], kWorkers);
+    }
     s->abort = 0;
     fence_mbar_init();
   }
@@ -119,94 +116,127 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_states_tc(const __grid_cons
   tc_fence_after();
   const uint32_t tmem = s->tmem_base;
 
-  auto issue = [&](int64_t g) {
-    const Work wk = work_of(g / nstages, T, H);
-    const int k = (int)(g % nstages);
-    issue_stage(tiles, tile_bytes, s, &map_a, &map_b, (int)(g % nslots), wk.c * C + k * KB, wk.h, wk.b);
-  };
-  if (tid == kProducer)
-    for (int64_t g = 0; g < nslots && g < nstream; ++g) issue(g);
-
-  constexpr uint32_t idesc = idesc_bf16(128, 128, 1, 1);
-  Work wk{0, 0, 0};
-  float lam = 1.f, l2 = 0.f;
-  for (int64_t g = 0; g < nstream; ++g) {
-    const int slot = (int)(g % nslots);
-    const uint32_t par = (uint32_t)((g / nslots) & 1);
-    const int k = (int)(g % nstages);
-    const int64_t n = g / nstages;
-    if (k == 0) {  // a new chunk: its coordinates and decay
-      wk = work_of(n, T, H);
-      lam = load_decay(decay, wk.h);
-      l2 = log2f(lam);
-    }
-    if (!mbar_wait(&s->full[slot], par, SITE_STATES_TMA)) s->abort = 1;
-    if (lam != 1.0f) {
-      // scale row r of A by w_{k*KB + r}; the row of a 16-byte chunk is its
-      // byte offset / 128 in either 64-feature box, whatever the swizzle
-      uint4* a = reinterpret_cast<uint4*>(tiles + (size_t)slot * 2 * tile_bytes);
-      const int nchunks = KB * 16;
-      for (int q = tid; q < nchunks; q += kThreads) {
-        const int r = (q % (KB * 8)) / 8;
-        const int t = k * KB + r;
-        const float w = kind == 0 ? decay_pow(l2, (float)(C - 1 - t)) : decay_pow(l2, (float)(t + 1));
-        uint4 x = a[q];
-        x.x = bf16x2_scale(x.x, w);
-        x.y = bf16x2_scale(x.y, w);
-        x.z = bf16x2_scale(x.z, w);
-        x.w = bf16x2_scale(x.w, w);
-        a[q] = x;
+  if (warp == 1) {
+    // ---------------------------------------------------------------- TMA
+    if (lane == 0) {
+      for (int64_t g = 0; g < nstream && !aborted(&s->abort); ++g) {
+        const int slot = (int)(g % nslots);
+        const int64_t u = g / nslots;
+        if (u > 0 && !mbar_wait(&s->empty[slot], (uint32_t)((u - 1) & 1), SITE_STATES_MMA)) {
+          s->abort = 1;
+          break;
+        }
+        const Work wk = work_of(g / nstages, T, H);
+        const int row = wk.c * C + (int)(g % nstages) * KB;
+        uint8_t* a = tiles + (size_t)slot * 2 * tile_bytes;
+        uint8_t* bb = a + tile_bytes;
+        mbar_arrive_expect_tx(&s->full[slot], 2 * tile_bytes);
+        tma_load_4d(a, &map_a, &s->full[slot], 0, wk.h, row, wk.b);
+        tma_load_4d(a + tile_bytes / 2, &map_a, &s->full[slot], 64, wk.h, row, wk.b);
+        tma_load_4d(bb, &map_b, &s->full[slot], 0, wk.h, row, wk.b);
+        tma_load_4d(bb + tile_bytes / 2, &map_b, &s->full[slot], 64, wk.h, row, wk.b);
       }
-      fence_async_smem();
     }
-    tc_fence_before();
-    __syncthreads();
-    if (s->abort) break;
-    if (tid == 0) {
-      tc_fence_after();
-      const uint32_t a0 = smem_u32(tiles + (size_t)slot * 2 * tile_bytes), b0 = a0 + tile_bytes;
-      for (int j = 0; j < KB / 16; ++j) {
-        const uint64_t ad = sw128_desc(a0 + j * 2048, KB * 128, 1024);
-        const uint64_t bd = sw128_desc(b0 + j * 2048, KB * 128, 1024);
-        mma_bf16(tmem, ad, bd, idesc, (k | j) != 0);
-      }
-      mma_commit(&s->empty[slot]);
-      if (k == nstages - 1) mma_commit(&s->done);
-    }
-    if (tid == kProducer && g >= 1 && g - 1 + nslots < nstream) {
-      // refill the slot of the previous stage (its MMAs were issued one step
-      // ago), keeping nslots - 1 stages in flight while this one is consumed
-      const int64_t gp = g - 1;
-      if (mbar_wait(&s->empty[gp % nslots], (uint32_t)((gp / nslots) & 1), SITE_STATES_MMA)) issue(gp + nslots);
-      else s->abort = 1;
-    }
-    if (k == nstages - 1) {
-      // epilogue of this chunk: warp w reads TMEM lanes (rows) 32*(w%4).. and the
-      // column half w/4; the state goes to slot c * slot_stride + slot_offset
-      if (mbar_wait(&s->done, (uint32_t)(n & 1), SITE_STATES_MMA)) {
+  } else if (warp == 0) {
+    // ---------------------------------------------------------------- MMA
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16(128, 128, 1, 1);
+      for (int64_t g = 0; g < nstream && !aborted(&s->abort); ++g) {
+        const int slot = (int)(g % nslots);
+        const int64_t u = g / nslots;
+        const int k = (int)(g % nstages);
+        const int64_t n = g / nstages;
+        const int acc = (int)(n & 1);
+        if (!mbar_wait(&s->scaled[slot], (uint32_t)(u & 1), SITE_STATES_TMA)) {
+          s->abort = 1;
+          break;
+        }
+        if (k == 0 && n >= 2 && !mbar_wait(&s->acc_empty[acc], (uint32_t)(((n >> 1) - 1) & 1), SITE_STATES_MMA)) {
+          s->abort = 1;
+          break;
+        }
         tc_fence_after();
-        const int row = (warp & 3) * 32 + lane, half = warp >> 2;
+        const uint32_t a0 = smem_u32(tiles + (size_t)slot * 2 * tile_bytes), b0 = a0 + tile_bytes;
+        const uint32_t d = tmem + (uint32_t)acc * 128;
+        for (int j = 0; j < KB / 16; ++j) {
+          const uint64_t ad = sw128_desc(a0 + j * 2048, KB * 128, 1024);
+          const uint64_t bd = sw128_desc(b0 + j * 2048, KB * 128, 1024);
+          mma_bf16(d, ad, bd, idesc, (k | j) != 0);
+        }
+        mma_commit(&s->empty[slot]);
+        if (k == nstages - 1) mma_commit(&s->acc_full[acc]);
+      }
+    }
+  } else {
+    // ------------------------------------------------- workers (warps 2-5)
+    const int wt = tid - 64;             // 0..127
+    const int quad = warp & 3;           // the TMEM lanes this warp may read
+    const int row = quad * 32 + lane;    // accumulator row read by this thread
+    Work wk{0, 0, 0};
+    float lam = 1.f, l2 = 0.f;
+    for (int64_t g = 0; g < nstream; ++g) {
+      const int slot = (int)(g % nslots);
+      const int64_t u = g / nslots;
+      const int k = (int)(g % nstages);
+      const int64_t n = g / nstages;
+      if (k == 0) {
+        wk = work_of(n, T, H);
+        lam = load_decay(decay, wk.h);
+        l2 = log2f(lam);
+      }
+      if (!mbar_wait(&s->full[slot], (uint32_t)(u & 1), SITE_STATES_TMA)) {
+        s->abort = 1;
+        break;
+      }
+      if (lam != 1.0f) {
+        // scale row r of A by w_{k*KB + r}; the row of a 16-byte chunk is its
+        // byte offset / 128 in either 64-feature box, whatever the swizzle
+        uint4* a = reinterpret_cast<uint4*>(tiles + (size_t)slot * 2 * tile_bytes);
+        const int nchunks = KB * 16;
+        for (int q = wt; q < nchunks; q += kWorkers) {
+          const int r = (q % (KB * 8)) / 8;
+          const int t = k * KB + r;
+          const float w = kind == 0 ? decay_pow(l2, (float)(C - 1 - t)) : decay_pow(l2, (float)(t + 1));
+          uint4 x = a[q];
+          x.x = bf16x2_scale(x.x, w);
+          x.y = bf16x2_scale(x.y, w);
+          x.z = bf16x2_scale(x.z, w);
+          x.w = bf16x2_scale(x.w, w);
+          a[q] = x;
+        }
+        fence_async_smem();
+      }
+      mbar_arrive(&s->scaled[slot]);
+      if (k == nstages - 1) {
+        // the chunk's state: accumulator n & 1 -> slot c * slot_stride + slot_offset
+        const int acc = (int)(n & 1);
+        if (!mbar_wait(&s->acc_full[acc], (uint32_t)((n >> 1) & 1), SITE_STATES_MMA)) {
+          s->abort = 1;
+          break;
+        }
+        tc_fence_after();
         const int64_t oslot = (int64_t)wk.c * slot_stride + slot_offset;
         float* out = M + ((((int64_t)wk.b * t_out + oslot) * H + wk.h) * kD + row) * kD;
-        uint32_t r0[32], r1[32];
-        tmem_ld32(tmem + ((uint32_t)((warp & 3) * 32) << 16) + (2 * half) * 32, r0);
-        tmem_ld32(tmem + ((uint32_t)((warp & 3) * 32) << 16) + (2 * half + 1) * 32, r1);
-        tmem_ld_wait();
-        float4* o0 = reinterpret_cast<float4*>(out + (2 * half) * 32);
-        float4* o1 = reinterpret_cast<float4*>(out + (2 * half + 1) * 32);
+        const uint32_t tbase = tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)acc * 128;
+#pragma unroll 1
+        for (int cc = 0; cc < kD / 32; cc += 2) {
+          uint32_t r0[32], r1[32];
+          tmem_ld32(tbase + cc * 32, r0);
+          tmem_ld32(tbase + (cc + 1) * 32, r1);
+          tmem_ld_wait();
+          float4* o0 = reinterpret_cast<float4*>(out + cc * 32);
+          float4* o1 = reinterpret_cast<float4*>(out + (cc + 1) * 32);
 #pragma unroll
-        for (int q = 0; q < 8; ++q) {
-          __stcs(o0 + q, make_float4(__uint_as_float(r0[4 * q]), __uint_as_float(r0[4 * q + 1]),
-                                     __uint_as_float(r0[4 * q + 2]), __uint_as_float(r0[4 * q + 3])));
-          __stcs(o1 + q, make_float4(__uint_as_float(r1[4 * q]), __uint_as_float(r1[4 * q + 1]),
-                                     __uint_as_float(r1[4 * q + 2]), __uint_as_float(r1[4 * q + 3])));
+          for (int q = 0; q < 8; ++q) {
+            __stcs(o0 + q, make_float4(__uint_as_float(r0[4 * q]), __uint_as_float(r0[4 * q + 1]),
+                                       __uint_as_float(r0[4 * q + 2]), __uint_as_float(r0[4 * q + 3])));
+            __stcs(o1 + q, make_float4(__uint_as_float(r1[4 * q]), __uint_as_float(r1[4 * q + 1]),
+                                       __uint_as_float(r1[4 * q + 2]), __uint_as_float(r1[4 * q + 3])));
+          }
         }
-      } else {
-        s->abort = 1;
+        tc_fence_before();
+        mbar_arrive(&s->acc_empty[acc]);
       }
-      // the next chunk's first MMA overwrites the accumulator
-      tc_fence_before();
-      __syncthreads();
     }
   }
   tc_fence_before();
