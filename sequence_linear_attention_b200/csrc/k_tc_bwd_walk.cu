@@ -239,14 +239,6 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_walk_tc(
       const int row0 = item.seg * G + t * kTile;
       const int64_t c = row0 / kTile;  // chunk index (C = tile)
 
-      // the previous chunk's dK/dV stores must have left A and B before epilogue 1
-      if (tid == kProducer) tma_store_wait_read0();
-      __syncthreads();
-      if (s->abort) {
-        stop = true;
-        break;
-      }
-
       // ---- MMA 1
       if (tid == 0) {
         if (mbar_wait(&s->ld_kv, par, SITE_BWD_TMA) && mbar_wait(&s->ld_qd, par, SITE_BWD_TMA) &&
@@ -259,6 +251,15 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_walk_tc(
         } else {
           s->abort = 1;
         }
+      }
+
+      // the previous chunk's dK/dV stores must have left A and B before epilogue 1
+      // writes them (MMA 1 does not touch A or B)
+      if (tid == kProducer) tma_store_wait_read0();
+      __syncthreads();
+      if (s->abort) {
+        stop = true;
+        break;
       }
 
       // ---- epilogue 1
