@@ -8,7 +8,7 @@
 // The sequence is cut into segments of G tokens (a multiple of C and of the
 // 128-token tile). Before this kernel, the segment states and an exclusive
 // prefix over them put P of each segment's first chunk into the state cache.
-// Here one persistent CTA (512 threads) takes segments in turn and walks their
+// Here one persistent CTA (256 threads) takes segments in turn and walks their
 // 128-token tiles in order, holding the state P (fp32) in TMEM:
 //
 //   MMA 1:  S = Q K^T (TMEM S),  O_inter = Q P_bf16 (TMEM I)
@@ -22,8 +22,8 @@
 // entering state (already in shared memory for O_inter) goes to the chunk's
 // cache slot by one bulk copy; the backward walk loads it back as is. Two sets
 // of Q/K/V buffers alternate: while a tile is computed, the next tile's loads
-// (possibly of the next segment) are in flight. The CTA has 16 warps; in every
-// epilogue warp w owns TMEM lanes (rows) 32*(w%4).. and the 32-column quarter w/4.
+// (possibly of the next segment) are in flight. In every epilogue
+// warp w owns TMEM lanes (rows) 32*(w%4).. and the column half w/4.
 #include <algorithm>
 
 #include "kernels.h"
@@ -39,7 +39,7 @@ using namespace sm100;
 
 constexpr int kD = 128;
 constexpr int kTile = 128;
-constexpr int kThreads = 512;
+constexpr int kThreads = 256;
 constexpr uint32_t kTileBytes = kTile * kD * 2;
 constexpr uint32_t kBox = kTileBytes / 2;
 constexpr uint32_t kTmemCols = 512;
@@ -105,7 +105,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_walk_tc(const __grid_constant
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int i = (warp & 3) * 32 + lane;  // the row this thread owns in every epilogue
-  const int part = warp >> 2;            // and the 32-column quarter
+  const int half = warp >> 2;            // and the column half
   const int tiles = G / kTile;
 
   if (tid == 0) {
@@ -165,12 +165,11 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_walk_tc(const __grid_constant
     // entering state of the segment (slot of its first chunk): TMEM P and bf16 operand
     {
       const int64_t slot = ((int64_t)item.seg * G) / C;
-      const float* src = P + ((((int64_t)item.b * T + slot) * H + item.h) * kD + i) * kD + part * 32;
+      const float* src = P + ((((int64_t)item.b * T + slot) * H + item.h) * kD + i) * kD + half * 64;
       const float4* s4 = reinterpret_cast<const float4*>(src);
-      float v[32];
-      uint32_t r[32];
+      float v[64];
 #pragma unroll
-      for (int q = 0; q < 8; ++q) {
+      for (int q = 0; q < 16; ++q) {
         const float4 x = __ldcs(s4 + q);
         v[4 * q] = x.x;
         v[4 * q + 1] = x.y;
@@ -178,9 +177,13 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_walk_tc(const __grid_constant
         v[4 * q + 3] = x.w;
       }
 #pragma unroll
-      for (int q = 0; q < 32; ++q) r[q] = __float_as_uint(v[q]);
-      tmem_st32(lane_base + TP + part * 32, r);
-      st_row32_bf16(sP, i, part * 32, v);
+      for (int c2 = 0; c2 < 2; ++c2) {
+        uint32_t r[32];
+#pragma unroll
+        for (int q = 0; q < 32; ++q) r[q] = __float_as_uint(v[c2 * 32 + q]);
+        tmem_st32(lane_base + TP + half * 64 + c2 * 32, r);
+        st_row32_bf16(sP, i, half * 64 + c2 * 32, v + c2 * 32);
+      }
       tmem_st_wait();
       fence_async_smem();
     }
@@ -234,18 +237,26 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_walk_tc(const __grid_constant
       // ---- epilogue A
       if (mbar_wait(&s->mma1, it & 1u, SITE_OUT_MMA)) {
         tc_fence_after();
-        // S' = Mask . S into the Q buffer (Q has been read by both MMAs)
+        // S' = Mask . S into the Q buffer (Q has been read by both MMAs); both
+        // TMEM loads are in flight before the one wait
         {
-          uint32_t r0[32];
-          tmem_ld32(lane_base + TS + part * 32, r0);
+          uint32_t r0[32], r1[32];
+          tmem_ld32(lane_base + TS + (2 * half) * 32, r0);
+          tmem_ld32(lane_base + TS + (2 * half + 1) * 32, r1);
           tmem_ld_wait();
           float w32[32];
 #pragma unroll
           for (int q = 0; q < 32; ++q) {
-            const int j = part * 32 + q;
+            const int j = 2 * half * 32 + q;
             w32[q] = j <= i ? __uint_as_float(r0[q]) * s->pw[i - j] : 0.f;
           }
-          st_row32_bf16(sQ, i, part * 32, w32);
+          st_row32_bf16(sQ, i, 2 * half * 32, w32);
+#pragma unroll
+          for (int q = 0; q < 32; ++q) {
+            const int j = (2 * half + 1) * 32 + q;
+            w32[q] = j <= i ? __uint_as_float(r1[q]) * s->pw[i - j] : 0.f;
+          }
+          st_row32_bf16(sQ, i, (2 * half + 1) * 32, w32);
         }
         // K~ = diag(lambda^{127-j}) K, in place (K has been read by the S MMA)
         if (scale) {
@@ -265,21 +276,25 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_walk_tc(const __grid_constant
         // the state entering this tile: into the cache at chunk starts, then pre-scaled by lambda^128
         const bool write_cache = !cache_bf16 && t > 0 && (t * kTile) % C == 0;
         if (write_cache || scale) {
-          float* dst = P + ((((int64_t)item.b * T + row0 / C) * H + item.h) * kD + i) * kD + part * 32;
-          uint32_t r[32];
-          tmem_ld32(lane_base + TP + part * 32, r);
+          float* dst = P + ((((int64_t)item.b * T + row0 / C) * H + item.h) * kD + i) * kD + half * 64;
+          uint32_t r[2][32];
+          tmem_ld32(lane_base + TP + half * 64, r[0]);
+          tmem_ld32(lane_base + TP + half * 64 + 32, r[1]);
           tmem_ld_wait();
-          if (write_cache) {
-            float4* d4 = reinterpret_cast<float4*>(dst);
 #pragma unroll
-            for (int q = 0; q < 8; ++q)
-              __stcs(d4 + q, make_float4(__uint_as_float(r[4 * q]), __uint_as_float(r[4 * q + 1]),
-                                         __uint_as_float(r[4 * q + 2]), __uint_as_float(r[4 * q + 3])));
-          }
-          if (scale) {
+          for (int c2 = 0; c2 < 2; ++c2) {
+            if (write_cache) {
+              float4* d4 = reinterpret_cast<float4*>(dst + c2 * 32);
 #pragma unroll
-            for (int q = 0; q < 32; ++q) r[q] = __float_as_uint(__uint_as_float(r[q]) * g_tile);
-            tmem_st32(lane_base + TP + part * 32, r);
+              for (int q = 0; q < 8; ++q)
+                __stcs(d4 + q, make_float4(__uint_as_float(r[c2][4 * q]), __uint_as_float(r[c2][4 * q + 1]),
+                                           __uint_as_float(r[c2][4 * q + 2]), __uint_as_float(r[c2][4 * q + 3])));
+            }
+            if (scale) {
+#pragma unroll
+              for (int q = 0; q < 32; ++q) r[c2][q] = __float_as_uint(__uint_as_float(r[c2][q]) * g_tile);
+              tmem_st32(lane_base + TP + half * 64 + c2 * 32, r[c2]);
+            }
           }
           tmem_st_wait();
         }
@@ -309,19 +324,33 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_walk_tc(const __grid_constant
         tc_fence_after();
         const float wi = decay_pow(l2, (float)(i + 1));
         {
-          // O = O_intra + lambda^{i+1} O_inter; P (after its update) -> bf16 operand
-          uint32_t a0[32], e0[32], p0[32];
-          tmem_ld32(lane_base + TO + part * 32, a0);
-          tmem_ld32(lane_base + TI + part * 32, e0);
-          tmem_ld32(lane_base + TP + part * 32, p0);
+          // O = O_intra + lambda^{i+1} O_inter, both column chunks' loads in flight together
+          uint32_t a0[32], e0[32], a1[32], e1[32];
+          tmem_ld32(lane_base + TO + (2 * half) * 32, a0);
+          tmem_ld32(lane_base + TI + (2 * half) * 32, e0);
+          tmem_ld32(lane_base + TO + (2 * half + 1) * 32, a1);
+          tmem_ld32(lane_base + TI + (2 * half + 1) * 32, e1);
           tmem_ld_wait();
           float o[32];
 #pragma unroll
           for (int q = 0; q < 32; ++q) o[q] = fmaf(wi, __uint_as_float(e0[q]), __uint_as_float(a0[q]));
-          st_row32_bf16(sK, i, part * 32, o);  // output staging over K~
+          st_row32_bf16(sK, i, 2 * half * 32, o);  // output staging over K~
 #pragma unroll
-          for (int q = 0; q < 32; ++q) o[q] = __uint_as_float(p0[q]);
-          st_row32_bf16(sP, i, part * 32, o);
+          for (int q = 0; q < 32; ++q) o[q] = fmaf(wi, __uint_as_float(e1[q]), __uint_as_float(a1[q]));
+          st_row32_bf16(sK, i, (2 * half + 1) * 32, o);
+        }
+        {
+          uint32_t r0[32], r1[32];
+          tmem_ld32(lane_base + TP + (2 * half) * 32, r0);
+          tmem_ld32(lane_base + TP + (2 * half + 1) * 32, r1);
+          tmem_ld_wait();
+          float p[32];
+#pragma unroll
+          for (int q = 0; q < 32; ++q) p[q] = __uint_as_float(r0[q]);
+          st_row32_bf16(sP, i, 2 * half * 32, p);
+#pragma unroll
+          for (int q = 0; q < 32; ++q) p[q] = __uint_as_float(r1[q]);
+          st_row32_bf16(sP, i, (2 * half + 1) * 32, p);
         }
         fence_async_smem();
       } else {
