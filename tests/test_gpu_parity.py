@@ -46,6 +46,8 @@ SMALL = [
     (2, 3, 1536, 128, 256, True, True),  # chunks of two tiles
     (1, 2, 1024, 128, 512, True, False),
     (2, 150, 1024, 128, 128, True, True),  # more segments than SMs: each CTA walks several
+    (2, 3, 1152, 128, 128, True, True),    # three segments of three tiles
+    (1, 4, 2048, 128, 128, True, False),   # walks without decay
 ]
 
 

@@ -1,0 +1,102 @@
+"""The pins catch plausible mistakes: each case plants one error in a copy of
+the oracle's C source (on the CPU, in a temporary directory), loads the broken
+build in place of the real one, and checks that the pin checks below fail.
+The real oracle is restored afterwards."""
+import os
+import subprocess
+import sys
+
+import numpy as np
+import pytest
+
+import oracle
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, HERE)
+import test_oracle_pins as pins  # noqa: E402
+
+SRC = os.path.join(os.path.dirname(HERE), "oracle", "lasp_oracle.c")
+
+# (what the mistake is, exact text in the source, its replacement, occurrence index)
+MUTATIONS = [
+    ("forward state loses its decay",
+     "S[i * d + j] = l * S[i * d + j] + (double)ks[i] * vs[j];\n      for",
+     "S[i * d + j] = S[i * d + j] + (double)ks[i] * vs[j];\n      for", 0),
+    ("forward output reads the state transposed",
+     "acc += (double)qs[i] * S[i * d + j];", "acc += (double)qs[i] * S[j * d + i];", 0),
+    ("forward uses v for k",
+     "S[i * d + j] = l * S[i * d + j] + (double)ks[i] * vs[j];\n      for",
+     "S[i * d + j] = l * S[i * d + j] + (double)vs[i] * vs[j];\n      for", 0),
+    ("dq contracts with dout against the wrong index",
+     "acc += S[i * d + j] * ds[j];", "acc += S[j * d + i] * ds[j];", 0),
+    ("dk uses k instead of v", "acc += G[i * d + j] * vs[j];", "acc += G[i * d + j] * ks[j];", 0),
+    ("dv gradient state misses the current token",
+     "for (int j = r0; j < r1; ++j) G[i * d + j] += (double)qs[i] * ds[j];",
+     "for (int j = r0; j < r1; ++j) G[i * d + j] += 0.0 * qs[i] * ds[j];", 0),
+    ("dv sums over the wrong operand", "acc += (double)ks[i] * G[i * d + j];",
+     "acc += (double)qs[i] * G[i * d + j];", 0),
+    ("chunk-state weight off by one", "pow(l, (double)(C - 1 - t))", "pow(l, (double)(C - t))", 0),
+    ("gradient-state weight off by one", "pow(l, (double)(t + 1))", "pow(l, (double)(t))", 0),
+    ("scan without the chunk decay", "acc[e] = g * acc[e] + Mc[e];", "acc[e] = acc[e] + Mc[e];", 0),
+    ("gradient snapshots decay before adding the token",
+     "S[i * d + j] = l * (S[i * d + j] + (double)as[i] * bs[j]);",
+     "S[i * d + j] = l * S[i * d + j] + (double)as[i] * bs[j];", 0),
+]
+
+
+def _build_mutant(tmp_path, old, new, nth):
+    src = open(SRC).read()
+    idx = -1
+    for _ in range(nth + 1):
+        idx = src.find(old, idx + 1)
+        assert idx >= 0, f"mutation anchor not found: {old!r}"
+    src = src[:idx] + new + src[idx + len(old):]
+    path = tmp_path / "mutant.c"
+    path.write_text(src)
+    so = tmp_path / "libmutant.so"
+    subprocess.run(["gcc", "-O1", "-fopenmp", "-fPIC", "-shared", "-std=c11", str(path), "-o", str(so), "-lm"],
+                   check=True)
+    return str(so)
+
+
+def _pins_pass():
+    """A reduced set of the pins; True when all of them hold."""
+    checks = [
+        pins.test_two_token_worked_example,
+        pins.test_unit_vector_closed_form,
+        lambda: pins.test_recurrence_equals_quadratic_form(True, 1),
+        pins.test_entering_states_equal_quadratic_form,
+        lambda: pins.test_recurrence_equals_chunk_form(8),
+        pins.test_chunk_states_equal_recurrence_run_over_the_chunk,
+        pins.test_state_scan_closed_forms,
+        pins.test_scan_of_chunk_states_equals_recurrence_snapshots,
+    ]
+    for check in checks:
+        try:
+            check()
+        except AssertionError:
+            return False
+    return True
+
+
+@pytest.mark.parametrize("name,old,new,nth", MUTATIONS, ids=[m[0] for m in MUTATIONS])
+def test_pins_catch_the_mistake(tmp_path, name, old, new, nth):
+    import ctypes
+    so = _build_mutant(tmp_path, old, new, nth)
+    real = oracle._load()
+    lib = ctypes.CDLL(so)
+    for f in ("oracle_fwd", "oracle_bwd", "oracle_chunk_states", "oracle_state_scan", "oracle_state_snapshots"):
+        getattr(lib, f).argtypes = getattr(real, f).argtypes
+        getattr(lib, f).restype = None
+    lib.oracle_num_threads.restype = ctypes.c_int
+    oracle._lib = lib
+    try:
+        assert not _pins_pass(), f"the pins did not catch: {name}"
+    finally:
+        oracle._lib = real
+
+
+def test_unmutated_source_passes_the_same_checks():
+    assert _pins_pass()
+    assert np.isfinite(oracle.fwd(np.ones((1, 4, 1, 2), np.float32), np.ones((1, 4, 1, 2), np.float32),
+                                  np.ones((1, 4, 1, 2), np.float32))).all()
