@@ -12,13 +12,12 @@
 // cache as a ready bf16 operand tile. Per chunk c (LASP Eq. 14-23):
 //
 //   MMA 1:  T0 = dO V^T,  T1 = Q K^T,  T2 = dO P^T
-//   epi 1a: dP' = Mask . T0 -> A
-//   MMA 2:  T0 = dP' K                      (runs under epi 1b)
-//   epi 1b: S' = Mask . T1 -> B;  R -> bf16 X (replacing P),
-//           R <- lambda^128 R in TMEM;  V <- diag(lambda^{127-j}) V in place
-//   MMA 3a: T1 = S'^T dO                    (runs under epi 2)
+//   epi 1:  dP' = Mask . T0 -> A,  S' = Mask . T1 -> B;
+//           R -> bf16 X (replacing P),  R <- lambda^128 R in TMEM;
+//           V <- diag(lambda^{127-j}) V in place
+//   MMA 2:  T0 = dP' K
 //   epi 2:  dQ = T0 + lambda^{i+1} T2 -> global
-//   MMA 3b: T0 = dP'^T Q + V~ R^T  (dK),  T2 = K R
+//   MMA 3:  T0 = dP'^T Q + V~ R^T  (dK),  T1 = S'^T dO,  T2 = K R
 //   epi 3:  Q <- diag(lambda^{j+1}) Q;  then, while MMA 4 runs, dK -> A,
 //           dV = T1 + lambda^{127-j} T2 -> B (TMA stores)
 //   MMA 4:  R += Q~^T dO          (the state for chunk c - 1)
@@ -263,26 +262,49 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_walk_tc(
         break;
       }
 
-      // ---- epilogue 1a: dP' -> A, so that MMA 2 can start
+      // ---- epilogue 1
       if (mbar_wait(&s->c1, par, SITE_BWD_MMA)) {
         tc_fence_after();
-        uint32_t r0[32], r1[32];
-        tmem_ld32(lane_base + T0 + (2 * half) * 32, r0);
-        tmem_ld32(lane_base + T0 + (2 * half + 1) * 32, r1);
-        tmem_ld_wait();
-        float f[32];
+#pragma unroll 1
+        for (int cc = 2 * half; cc < 2 * half + 2; ++cc) {
+          uint32_t rp[32], rs[32];
+          tmem_ld32(lane_base + T0 + cc * 32, rp);
+          tmem_ld32(lane_base + T1 + cc * 32, rs);
+          tmem_ld_wait();
+          float fp[32], fs[32];
 #pragma unroll
-        for (int q = 0; q < 32; ++q) {
-          const int j = 2 * half * 32 + q;
-          f[q] = j <= i ? __uint_as_float(r0[q]) * s->pw[i - j] : 0.f;
+          for (int q = 0; q < 32; ++q) {
+            const int j = cc * 32 + q;
+            const float wgt = j <= i ? s->pw[i - j] : 0.f;
+            fp[q] = __uint_as_float(rp[q]) * wgt;
+            fs[q] = __uint_as_float(rs[q]) * wgt;
+          }
+          st_row32_bf16(sA, i, cc * 32, fp);
+          st_row32_bf16(sB, i, cc * 32, fs);
         }
-        st_row32_bf16(sA, i, 2 * half * 32, f);
+        // R of this chunk -> bf16 X (MMA 1 has read P) and pre-scaled by lambda^128 for MMA 4
+        {
+          uint32_t r[2][32];
+          tmem_ld32(lane_base + TR + half * 64, r[0]);
+          tmem_ld32(lane_base + TR + half * 64 + 32, r[1]);
+          tmem_ld_wait();
 #pragma unroll
-        for (int q = 0; q < 32; ++q) {
-          const int j = (2 * half + 1) * 32 + q;
-          f[q] = j <= i ? __uint_as_float(r1[q]) * s->pw[i - j] : 0.f;
+          for (int c2 = 0; c2 < 2; ++c2) {
+            float f[32];
+#pragma unroll
+            for (int q = 0; q < 32; ++q) f[q] = __uint_as_float(r[c2][q]);
+            st_row32_bf16(sX, i, half * 64 + c2 * 32, f);
+            if (scale) {
+#pragma unroll
+              for (int q = 0; q < 32; ++q) r[c2][q] = __float_as_uint(f[q] * g_tile);
+              tmem_st32(lane_base + TR + half * 64 + c2 * 32, r[c2]);
+            }
+          }
         }
-        st_row32_bf16(sA, i, (2 * half + 1) * 32, f);
+        if (scale) {
+          tmem_st_wait();
+          scale_rows(sV, s->pw, true, 1.f, tid);  // V~ = diag(lambda^{127-j}) V
+        }
         fence_async_smem();
       } else {
         s->abort = 1;
@@ -293,66 +315,14 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_walk_tc(
         stop = true;
         break;
       }
-      // ---- MMA 2: dQ_intra = dP' K (T0 has been read)
+
+      // ---- MMA 2: dQ_intra = dP' K
       if (tid == 0) {
         tc_fence_after();
         for (int kk = 0; kk < kTile / 16; ++kk) mma_bf16(tmem + T0, kmaj(aA, kk), mnmaj(aK, kk), id_kn, kk != 0);
         mma_commit(&s->c2);
       }
-
-      // ---- epilogue 1b, under MMA 2: S' -> B; R -> bf16 X (MMA 1 has read P) and
-      // pre-scaled by lambda^128 for MMA 4; V~ = diag(lambda^{127-j}) V
-      {
-        uint32_t r0[32], r1[32];
-        tmem_ld32(lane_base + T1 + (2 * half) * 32, r0);
-        tmem_ld32(lane_base + T1 + (2 * half + 1) * 32, r1);
-        tmem_ld_wait();
-        float f[32];
-#pragma unroll
-        for (int q = 0; q < 32; ++q) {
-          const int j = 2 * half * 32 + q;
-          f[q] = j <= i ? __uint_as_float(r0[q]) * s->pw[i - j] : 0.f;
-        }
-        st_row32_bf16(sB, i, 2 * half * 32, f);
-#pragma unroll
-        for (int q = 0; q < 32; ++q) {
-          const int j = (2 * half + 1) * 32 + q;
-          f[q] = j <= i ? __uint_as_float(r1[q]) * s->pw[i - j] : 0.f;
-        }
-        st_row32_bf16(sB, i, (2 * half + 1) * 32, f);
-      }
-      {
-        uint32_t r[2][32];
-        tmem_ld32(lane_base + TR + half * 64, r[0]);
-        tmem_ld32(lane_base + TR + half * 64 + 32, r[1]);
-        tmem_ld_wait();
-#pragma unroll
-        for (int c2 = 0; c2 < 2; ++c2) {
-          float f[32];
-#pragma unroll
-          for (int q = 0; q < 32; ++q) f[q] = __uint_as_float(r[c2][q]);
-          st_row32_bf16(sX, i, half * 64 + c2 * 32, f);
-          if (scale) {
-#pragma unroll
-            for (int q = 0; q < 32; ++q) r[c2][q] = __float_as_uint(f[q] * g_tile);
-            tmem_st32(lane_base + TR + half * 64 + c2 * 32, r[c2]);
-          }
-        }
-      }
-      if (scale) {
-        tmem_st_wait();
-        scale_rows(sV, s->pw, true, 1.f, tid);
-      }
-      fence_async_smem();
-      tc_fence_before();
-      __syncthreads();
-      // ---- MMA 3a: dV_intra = S'^T dO (T1 has been read)
-      if (tid == 0) {
-        tc_fence_after();
-        for (int kk = 0; kk < kTile / 16; ++kk) mma_bf16(tmem + T1, mnmaj(aB, kk), mnmaj(aD, kk), id_nn, kk != 0);
-      }
-
-      // ---- epilogue 2, under MMA 3a: dQ = T0 + lambda^{i+1} T2 -> global
+      // ---- epilogue 2: dQ
       if (mbar_wait(&s->c2, par, SITE_BWD_MMA)) {
         tc_fence_after();
         const float wi = decay_pow(l2, (float)(i + 1));
@@ -372,6 +342,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_walk_tc(
                 make_uint4(pack_bf16(o[0], o[1]), pack_bf16(o[2], o[3]), pack_bf16(o[4], o[5]), pack_bf16(o[6], o[7]));
           }
         }
+        fence_async_smem();
       } else {
         s->abort = 1;
       }
@@ -382,11 +353,12 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_walk_tc(
         break;
       }
 
-      // ---- MMA 3b: dK = dP'^T Q + V~ R^T, dV_inter = K R (T0 and T2 have been read)
+      // ---- MMA 3: dK = dP'^T Q + V~ R^T, dV_intra = S'^T dO, dV_inter = K R
       if (tid == 0) {
         tc_fence_after();
         for (int kk = 0; kk < kTile / 16; ++kk) mma_bf16(tmem + T0, mnmaj(aA, kk), mnmaj(aQ, kk), id_nn, kk != 0);
         for (int kk = 0; kk < kD / 16; ++kk) mma_bf16(tmem + T0, kmaj(aV, kk), kmaj(aX, kk), id_kk, 1);
+        for (int kk = 0; kk < kTile / 16; ++kk) mma_bf16(tmem + T1, mnmaj(aB, kk), mnmaj(aD, kk), id_nn, kk != 0);
         for (int kk = 0; kk < kD / 16; ++kk) mma_bf16(tmem + T2, kmaj(aK, kk), mnmaj(aX, kk), id_kn, kk != 0);
         mma_commit(&s->c3);
       }
