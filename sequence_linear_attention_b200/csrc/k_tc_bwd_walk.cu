@@ -51,7 +51,7 @@ constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t T0 = 0, T1 = 128, T2 = 256, TR = 384;
 
 struct Smem {
-  uint64_t ld_kv, ld_qd, ld_p;
+  uint64_t ld_kv, ld_qd, ld_p, ld_r;
   uint64_t c1, c2, c3, c4;
   uint32_t tmem_base;
   int abort;
@@ -113,7 +113,8 @@ __device__ __forceinline__ Item item_of(int64_t w, int H, int nseg) {
 __global__ void __launch_bounds__(kThreads, 1) bwd_walk_tc(
     const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
     const __grid_constant__ CUtensorMap map_v, const __grid_constant__ CUtensorMap map_do,
-    const __grid_constant__ CUtensorMap map_dk, const __grid_constant__ CUtensorMap map_dv, const float* decay,
+    const __grid_constant__ CUtensorMap map_dk, const __grid_constant__ CUtensorMap map_dv,
+    const __grid_constant__ CUtensorMap map_state, const float* decay,
     const float* __restrict__ P, float* __restrict__ R, __nv_bfloat16* __restrict__ dq, int H, int64_t N, int T,
     int G, int nseg, int64_t nitems) {
   extern __shared__ uint8_t smem_raw[];
@@ -137,9 +138,11 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_walk_tc(
     prefetch_tmap(&map_k);
     prefetch_tmap(&map_v);
     prefetch_tmap(&map_do);
+    prefetch_tmap(&map_state);
     mbar_init(&s->ld_kv, 1);
     mbar_init(&s->ld_qd, 1);
     mbar_init(&s->ld_p, 1);
+    mbar_init(&s->ld_r, 1);
     mbar_init(&s->c1, 1);
     mbar_init(&s->c2, 1);
     mbar_init(&s->c3, 1);
@@ -199,6 +202,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_walk_tc(
   const uint32_t aQ = smem_u32(sQ), aK = smem_u32(sK), aV = smem_u32(sV), aD = smem_u32(sD);
   const uint32_t aX = smem_u32(sX), aA = smem_u32(sA), aB = smem_u32(sB);
   uint32_t it = 0;
+  uint32_t nseg_done = 0;  // segments started by this CTA
   bool stop = false;
 
   for (int64_t w = blockIdx.x; w < nitems && !stop; w += gridDim.x) {
@@ -211,25 +215,16 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_walk_tc(
     if (it > 0 && !mbar_wait(&s->c4, (it - 1) & 1u, SITE_BWD_MMA)) s->abort = 1;
     tc_fence_after();
     if (tid < kTile) s->pw[tid] = decay_pow(l2, (float)tid);
-    {
-      // R entering the segment's last chunk -> TMEM R
-      const int64_t slot = (int64_t)item.seg * (G / kTile) + tiles - 1;
-      const float4* src = reinterpret_cast<const float4*>(
-          R + ((((int64_t)item.b * T + slot) * H + item.h) * kD + i) * kD + half * 64);
+    if (tid == kProducer) {
+      // R entering the segment's last chunk, as four 32-column fp32 boxes into
+      // A and B (free once the previous chunk's dK/dV stores have read them);
+      // epilogue 1 of the first chunk moves it into TMEM
+      tma_store_wait_read0();
+      const int64_t slot = (int64_t)item.seg * tiles + tiles - 1;
+      const int y = (int)((((int64_t)item.b * T + slot) * H + item.h) * kD);
+      mbar_arrive_expect_tx(&s->ld_r, kD * kD * 4);
 #pragma unroll
-      for (int c2 = 0; c2 < 2; ++c2) {
-        uint32_t r[32];
-#pragma unroll
-        for (int q = 0; q < 8; ++q) {
-          const float4 x = __ldcs(src + c2 * 8 + q);
-          r[4 * q] = __float_as_uint(x.x);
-          r[4 * q + 1] = __float_as_uint(x.y);
-          r[4 * q + 2] = __float_as_uint(x.z);
-          r[4 * q + 3] = __float_as_uint(x.w);
-        }
-        tmem_st32(lane_base + TR + half * 64 + c2 * 32, r);
-      }
-      tmem_st_wait();
+      for (int bx = 0; bx < 4; ++bx) tma_load_2d(sA + bx * kBox, &map_state, &s->ld_r, 32 * bx, y);
     }
     tc_fence_before();
     __syncthreads();
@@ -237,7 +232,6 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_walk_tc(
     for (int t = tiles - 1; t >= 0; --t, ++it) {
       const uint32_t par = it & 1u;
       const int row0 = item.seg * G + t * kTile;
-      const int64_t c = row0 / kTile;  // chunk index (C = tile)
 
       // ---- MMA 1
       if (tid == 0) {
@@ -263,6 +257,36 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_walk_tc(
       }
 
       // ---- epilogue 1
+      if (t == tiles - 1) {
+        // the segment's entering R: A/B -> TMEM R. Row i of a swizzled box has
+        // its 16-byte chunk c at position c ^ (i & 7), so the eight rows of a
+        // quarter-warp read different banks.
+        if (mbar_wait(&s->ld_r, nseg_done & 1u, SITE_BWD_TMA)) {
+          const uint8_t* src = sA + half * 2 * kBox;
+          uint32_t r[2][32];
+#pragma unroll
+          for (int bb = 0; bb < 2; ++bb)
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+              const uint4 x = *reinterpret_cast<const uint4*>(src + bb * kBox + sw128_offset(i, c));
+              r[bb][4 * c] = x.x;
+              r[bb][4 * c + 1] = x.y;
+              r[bb][4 * c + 2] = x.z;
+              r[bb][4 * c + 3] = x.w;
+            }
+          tmem_st32(lane_base + TR + half * 64, r[0]);
+          tmem_st32(lane_base + TR + half * 64 + 32, r[1]);
+          tmem_st_wait();
+        } else {
+          s->abort = 1;
+        }
+        ++nseg_done;
+        __syncthreads();  // all of R is read before A and B are rewritten
+        if (s->abort) {
+          stop = true;
+          break;
+        }
+      }
       if (mbar_wait(&s->c1, par, SITE_BWD_MMA)) {
         tc_fence_after();
 #pragma unroll 1
@@ -398,6 +422,13 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_walk_tc(
             nt = tiles - 1;
           }
         }
+        if (t == (tiles > 1 ? 1 : 0) && w + gridDim.x < nitems) {
+          // the next segment's entering R is read by all threads at the segment
+          // switch; bring it into L2 while this segment's last tiles run
+          const Item ns = item_of(w + gridDim.x, H, nseg);
+          const int64_t slot = (int64_t)ns.seg * tiles + tiles - 1;
+          bulk_prefetch_l2(R + (((int64_t)ns.b * T + slot) * H + ns.h) * kD * kD, kD * kD * sizeof(float));
+        }
         if (has_next) {
           load_kv(nx, nt);
           load_p(nx, nt);
@@ -453,10 +484,11 @@ cudaError_t tc_bwd_walk(const void* q, const void* k, const void* v, const void*
                         const float* P, float* R, void* dq, void* dk, void* dv, int B, int H, int64_t N, int d, int C,
                         int G, int num_sms, cudaStream_t st) {
   using namespace tc_bwd_walk_detail;
-  CUtensorMap mq, mk, mv, mdo, mdk, mdv;
+  CUtensorMap mq, mk, mv, mdo, mdk, mdv, mr;
   if (!make_token_map(&mq, q, B, H, N, d, kTile) || !make_token_map(&mk, k, B, H, N, d, kTile) ||
       !make_token_map(&mv, v, B, H, N, d, kTile) || !make_token_map(&mdo, dout, B, H, N, d, kTile) ||
-      !make_token_map(&mdk, dk, B, H, N, d, kTile) || !make_token_map(&mdv, dv, B, H, N, d, kTile))
+      !make_token_map(&mdk, dk, B, H, N, d, kTile) || !make_token_map(&mdv, dv, B, H, N, d, kTile) ||
+      !make_state_map(&mr, R, (int64_t)B * (N / C) * H, d))
     return cudaErrorInvalidValue;
   const size_t smem = 1024 + 7 * (size_t)kTileBytes + sizeof(Smem);
   cudaError_t e = cudaFuncSetAttribute(bwd_walk_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -464,7 +496,7 @@ cudaError_t tc_bwd_walk(const void* q, const void* k, const void* v, const void*
   const int nseg = (int)(N / G);
   const int64_t nitems = (int64_t)B * H * nseg;
   const unsigned grid = (unsigned)std::min<int64_t>(nitems, num_sms);
-  bwd_walk_tc<<<grid, kThreads, smem, st>>>(mq, mk, mv, mdo, mdk, mdv, decay, P, R, (__nv_bfloat16*)dq, H, N,
+  bwd_walk_tc<<<grid, kThreads, smem, st>>>(mq, mk, mv, mdo, mdk, mdv, mr, decay, P, R, (__nv_bfloat16*)dq, H, N,
                                             (int)(N / C), G, nseg, nitems);
   return cudaGetLastError();
 }

@@ -48,6 +48,7 @@ constexpr uint32_t TS = 0, TI = 128, TO = 256, TP = 384;
 struct Smem {
   uint64_t load[2];
   uint64_t mma1, mma2;
+  uint64_t ld_state;
   uint32_t tmem_base;
   int abort;
   float pw[kTile];
@@ -94,6 +95,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_walk_tc(const __grid_constant
                                                             const __grid_constant__ CUtensorMap map_k,
                                                             const __grid_constant__ CUtensorMap map_v,
                                                             const __grid_constant__ CUtensorMap map_o,
+                                                            const __grid_constant__ CUtensorMap map_state,
                                                             const float* decay, float* __restrict__ P, int H,
                                                             int T, int C, int G, int nseg, int64_t nitems,
                                                             int cache_bf16) {
@@ -117,6 +119,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_walk_tc(const __grid_constant
     mbar_init(&s->load[1], 1);
     mbar_init(&s->mma1, 1);
     mbar_init(&s->mma2, 1);
+    mbar_init(&s->ld_state, 1);
     s->abort = 0;
     fence_mbar_init();
   }
@@ -143,15 +146,33 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_walk_tc(const __grid_constant
     tma_load_4d(q + 2 * kTileBytes + kBox, &map_v, &s->load[set], 64, it.h, row, it.b);
   };
 
+  // the fp32 state entering a segment (the slot of its first chunk) as four
+  // 32-column boxes: boxes 0, 1 into the Q buffer of `set`, boxes 2, 3 into its
+  // V buffer, both free at that point
+  auto issue_state_load = [&](int set, const Item& it) {
+    const int64_t slot = ((int64_t)it.seg * G) / C;
+    const int y = (int)((((int64_t)it.b * T + slot) * H + it.h) * kD);
+    mbar_arrive_expect_tx(&s->ld_state, kD * kD * 4);
+#pragma unroll
+    for (int bx = 0; bx < 4; ++bx)
+      tma_load_2d(bufQ(set) + (bx >> 1) * 2 * kTileBytes + (bx & 1) * kBox, &map_state, &s->ld_state, 32 * bx, y);
+  };
+
   // thread 32 issues every TMA load and bulk copy (and waits for the stores it
   // issued); thread 0 issues the MMAs
   constexpr int kProducer = 32;
-  if (tid == kProducer && (int64_t)blockIdx.x < nitems) issue_loads(0, item_of(blockIdx.x, H, nseg), 0);
+  if (tid == kProducer && (int64_t)blockIdx.x < nitems) {
+    prefetch_tmap(&map_state);
+    const Item first = item_of(blockIdx.x, H, nseg);
+    issue_loads(0, first, 0);
+    issue_state_load(1, first);
+  }
 
   constexpr uint32_t id_kk = idesc_bf16(128, 128, 0, 0);
   constexpr uint32_t id_kn = idesc_bf16(128, 128, 0, 1);
   constexpr uint32_t id_nn = idesc_bf16(128, 128, 1, 1);
   uint32_t it = 0;  // tiles processed by this CTA
+  uint32_t nseg_done = 0;  // segments started by this CTA
   bool stop = false;
 
   for (int64_t w = blockIdx.x; w < nitems && !stop; w += gridDim.x) {
@@ -162,20 +183,23 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_walk_tc(const __grid_constant
     const float g_tile = decay_pow(l2, (float)kTile);
     if (tid < kTile) s->pw[tid] = decay_pow(l2, (float)tid);
 
-    // entering state of the segment (slot of its first chunk): TMEM P and bf16 operand
-    {
-      const int64_t slot = ((int64_t)item.seg * G) / C;
-      const float* src = P + ((((int64_t)item.b * T + slot) * H + item.h) * kD + i) * kD + half * 64;
-      const float4* s4 = reinterpret_cast<const float4*>(src);
+    // entering state of the segment, loaded by TMA into the buffer set the
+    // previous tile used (see issue_state_load): TMEM P and bf16 operand. Row i
+    // of a swizzled box has its 16-byte chunk c at position c ^ (i & 7), so the
+    // eight rows of a quarter-warp read different banks.
+    if (mbar_wait(&s->ld_state, nseg_done & 1u, SITE_OUT_TMA)) {
+      const uint8_t* src = bufQ((it & 1) ^ 1) + half * 2 * kTileBytes;
       float v[64];
 #pragma unroll
-      for (int q = 0; q < 16; ++q) {
-        const float4 x = __ldcs(s4 + q);
-        v[4 * q] = x.x;
-        v[4 * q + 1] = x.y;
-        v[4 * q + 2] = x.z;
-        v[4 * q + 3] = x.w;
-      }
+      for (int bb = 0; bb < 2; ++bb)
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          const float4 x = *reinterpret_cast<const float4*>(src + bb * kBox + sw128_offset(i, c));
+          v[bb * 32 + 4 * c] = x.x;
+          v[bb * 32 + 4 * c + 1] = x.y;
+          v[bb * 32 + 4 * c + 2] = x.z;
+          v[bb * 32 + 4 * c + 3] = x.w;
+        }
 #pragma unroll
       for (int c2 = 0; c2 < 2; ++c2) {
         uint32_t r[32];
@@ -186,10 +210,14 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_walk_tc(const __grid_constant
       }
       tmem_st_wait();
       fence_async_smem();
+    } else {
+      s->abort = 1;
     }
+    ++nseg_done;
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
+    if (s->abort) break;
 
     for (int t = 0; t < tiles; ++t, ++it) {
       const int set = it & 1;
@@ -212,6 +240,14 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_walk_tc(const __grid_constant
         if (has_next) {
           tma_store_wait_read0();
           issue_loads(set ^ 1, nx, nt);
+        }
+        if (t == (tiles > 1 ? tiles - 2 : 0) && w + gridDim.x < nitems) {
+          // the next segment's entering state is read by all threads at the
+          // segment switch; bring it into L2 while this segment's last tiles run
+          const Item ns = item_of(w + gridDim.x, H, nseg);
+          const int64_t slot = ((int64_t)ns.seg * G) / C;
+          const float* src = P + (((int64_t)ns.b * T + slot) * H + ns.h) * kD * kD;
+          bulk_prefetch_l2(src, kD * kD * sizeof(float));
         }
         if (cache_bf16) {
           // the bf16 operand tile of the state entering this chunk, as it sits
@@ -322,6 +358,10 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_walk_tc(const __grid_constant
       // ---- epilogue B
       if (mbar_wait(&s->mma2, it & 1u, SITE_OUT_MMA)) {
         tc_fence_after();
+        // MMA 2 has read this set's Q (S') and V buffers: the next segment's
+        // entering state goes there
+        if (tid == kProducer && t == tiles - 1 && w + gridDim.x < nitems)
+          issue_state_load(set, item_of(w + gridDim.x, H, nseg));
         const float wi = decay_pow(l2, (float)(i + 1));
         {
           // O = O_intra + lambda^{i+1} O_inter, both column chunks' loads in flight together
@@ -392,9 +432,10 @@ int walk_segment_tokens(int64_t N, int C) {
 cudaError_t tc_fwd_walk(const void* q, const void* k, const void* v, const float* decay, float* P, void* o, int B,
                         int H, int64_t N, int d, int C, int G, int num_sms, cudaStream_t st) {
   using namespace tc_fwd_walk_detail;
-  CUtensorMap mq, mk, mv, mo;
+  CUtensorMap mq, mk, mv, mo, mp;
   if (!make_token_map(&mq, q, B, H, N, d, kTile) || !make_token_map(&mk, k, B, H, N, d, kTile) ||
-      !make_token_map(&mv, v, B, H, N, d, kTile) || !make_token_map(&mo, o, B, H, N, d, kTile))
+      !make_token_map(&mv, v, B, H, N, d, kTile) || !make_token_map(&mo, o, B, H, N, d, kTile) ||
+      !make_state_map(&mp, P, (int64_t)B * (N / C) * H, d))
     return cudaErrorInvalidValue;
   const size_t smem = 1024 + 7 * (size_t)kTileBytes + sizeof(Smem);
   cudaError_t e = cudaFuncSetAttribute(fwd_walk_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -405,7 +446,7 @@ cudaError_t tc_fwd_walk(const void* q, const void* k, const void* v, const float
   // with C = 128 the backward walk reads the cache: it gets each chunk's state
   // as the bf16 operand tile; otherwise the cache holds fp32 states
   const int cache_bf16 = C == kTile ? 1 : 0;
-  fwd_walk_tc<<<grid, kThreads, smem, st>>>(mq, mk, mv, mo, decay, P, H, (int)(N / C), C, G, nseg, nitems,
+  fwd_walk_tc<<<grid, kThreads, smem, st>>>(mq, mk, mv, mo, mp, decay, P, H, (int)(N / C), C, G, nseg, nitems,
                                            cache_bf16);
   return cudaGetLastError();
 }
