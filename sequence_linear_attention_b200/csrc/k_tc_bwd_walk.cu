@@ -11,23 +11,29 @@
 // holding R (fp32) in TMEM; P of each chunk comes from the forward walk's
 // cache as a ready bf16 operand tile. Per chunk c (LASP Eq. 14-23):
 //
-//   MMA 1:  T0 = dO V^T,  T1 = Q K^T,  T2 = dO P^T
-//   epi 1:  dP' = Mask . T0 -> A,  S' = Mask . T1 -> B;
+//   MMA 1:  T0 = dO V^T,  T1 = Q K^T  | then T2 = dO P^T
+//   epi 1:  dP' = Mask . T0 -> A,  S' = Mask . T1 -> B;  (T2 done:)
 //           R -> bf16 X (replacing P),  R <- lambda^128 R in TMEM;
 //           V <- diag(lambda^{127-j}) V in place
-//   MMA 2:  T0 = dP' K
+//   MMA 2:  T0 = dP' K                 | then T1 = S'^T dO
 //   epi 2:  dQ = T0 + lambda^{i+1} T2 -> global
-//   MMA 3:  T0 = dP'^T Q + V~ R^T  (dK),  T1 = S'^T dO,  T2 = K R
-//   epi 3:  Q <- diag(lambda^{j+1}) Q;  then, while MMA 4 runs, dK -> A,
-//           dV = T1 + lambda^{127-j} T2 -> B (TMA stores)
+//   MMA 3:  T0 = dP'^T Q               | then T0 += V~ R^T (dK), T2 = K R
+//   epi 3:  Q <- diag(lambda^{j+1}) Q;  then dK = T0,
+//           dV = T1 + lambda^{127-j} T2 -> over Q~ and dO (TMA stores)
 //   MMA 4:  R += Q~^T dO          (the state for chunk c - 1)
+//
+// Each epilogue waits only for the MMAs before the bar; those after it run
+// under the epilogue.
 //
 // The decay of the dK inter term rides on the bf16 operand V~ so both dK terms
 // share an accumulator (TMEM has no fifth block); the dQ and dV inter terms
-// keep fp32 row scalings. The next chunk's K, V and P are loaded as soon as MMA 3 has read
-// the buffers they replace, its Q and dO once MMA 4 has. R is not stored per
-// chunk: only the segment-level slots of the workspace are used. In every epilogue warp w owns TMEM lanes
-// (rows) 32*(w%4).. and the column half w/4.
+// keep fp32 row scalings. Two pairs of tile buffers trade roles from chunk to
+// chunk: one holds the chunk's Q and dO and then its outgoing dK and dV, the
+// other its dP' and S' and then the next chunk's Q and dO, which are loaded as
+// soon as the first part of MMA 3 has read dP'. The next K, V and P follow once
+// all of MMA 3 is done. R is not stored per chunk: only the segment-level slots
+// of the workspace are used. In every epilogue warp w owns TMEM lanes (rows)
+// 32*(w%4).. and the column half w/4.
 #include <algorithm>
 
 #include "kernels.h"
@@ -52,7 +58,7 @@ constexpr uint32_t T0 = 0, T1 = 128, T2 = 256, TR = 384;
 
 struct Smem {
   uint64_t ld_kv, ld_qd, ld_p, ld_r;
-  uint64_t c1, c2, c3, c4;
+  uint64_t c1, c1b, c2, c3a, c3, c4;
   uint32_t tmem_base;
   int abort;
   float pw[kTile];
@@ -114,18 +120,19 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_walk_tc(
     const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
     const __grid_constant__ CUtensorMap map_v, const __grid_constant__ CUtensorMap map_do,
     const __grid_constant__ CUtensorMap map_dk, const __grid_constant__ CUtensorMap map_dv,
-    const __grid_constant__ CUtensorMap map_state, const float* decay,
-    const float* __restrict__ P, float* __restrict__ R, __nv_bfloat16* __restrict__ dq, int H, int64_t N, int T,
-    int G, int nseg, int64_t nitems) {
+    const __grid_constant__ CUtensorMap map_state, const float* decay, const float* __restrict__ P,
+    float* __restrict__ R, __nv_bfloat16* __restrict__ dq, int H, int64_t N, int T, int G, int nseg,
+    int64_t nitems) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-  uint8_t* sQ = base;
   uint8_t* sK = base + 1 * kTileBytes;
   uint8_t* sV = base + 2 * kTileBytes;
-  uint8_t* sD = base + 3 * kTileBytes;
   uint8_t* sX = base + 4 * kTileBytes;  // P, then R (bf16)
-  uint8_t* sA = base + 5 * kTileBytes;  // dP', then dK out
-  uint8_t* sB = base + 6 * kTileBytes;  // S',  then dV out
+  // two buffer pairs trade roles from chunk to chunk: one holds the chunk's Q
+  // and dO (and, once MMA 4 has read them, its dK and dV on their way out), the
+  // other dP' and S' (and, once MMA 3 has read those, the next chunk's Q and dO)
+  // (pair 0: buffers 0 and 3; pair 1: buffers 5 and 6)
+  auto pair = [&](uint32_t p, int m) { return base + (p ? 5 + m : 3 * m) * kTileBytes; };
   Smem* s = reinterpret_cast<Smem*>(base + 7 * kTileBytes);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -144,7 +151,9 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_walk_tc(
     mbar_init(&s->ld_p, 1);
     mbar_init(&s->ld_r, 1);
     mbar_init(&s->c1, 1);
+    mbar_init(&s->c1b, 1);
     mbar_init(&s->c2, 1);
+    mbar_init(&s->c3a, 1);
     mbar_init(&s->c3, 1);
     mbar_init(&s->c4, 1);
     s->abort = 0;
@@ -168,13 +177,15 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_walk_tc(
     tma_load_4d(sV, &map_v, &s->ld_kv, 0, it.h, row, it.b);
     tma_load_4d(sV + kBox, &map_v, &s->ld_kv, 64, it.h, row, it.b);
   };
-  auto load_qd = [&](const Item& it, int t) {
+  auto load_qd = [&](const Item& it, int t, uint32_t p) {
     const int row = it.seg * G + t * kTile;
+    uint8_t* q = pair(p, 0);
+    uint8_t* d = pair(p, 1);
     mbar_arrive_expect_tx(&s->ld_qd, 2 * kTileBytes);
-    tma_load_4d(sQ, &map_q, &s->ld_qd, 0, it.h, row, it.b);
-    tma_load_4d(sQ + kBox, &map_q, &s->ld_qd, 64, it.h, row, it.b);
-    tma_load_4d(sD, &map_do, &s->ld_qd, 0, it.h, row, it.b);
-    tma_load_4d(sD + kBox, &map_do, &s->ld_qd, 64, it.h, row, it.b);
+    tma_load_4d(q, &map_q, &s->ld_qd, 0, it.h, row, it.b);
+    tma_load_4d(q + kBox, &map_q, &s->ld_qd, 64, it.h, row, it.b);
+    tma_load_4d(d, &map_do, &s->ld_qd, 0, it.h, row, it.b);
+    tma_load_4d(d + kBox, &map_do, &s->ld_qd, 64, it.h, row, it.b);
   };
 
   // P of a chunk: the forward walk stored it in the chunk's cache slot as the
@@ -192,15 +203,14 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_walk_tc(
   if (tid == kProducer && (int64_t)blockIdx.x < nitems) {
     const Item first = item_of(blockIdx.x, H, nseg);
     load_kv(first, tiles - 1);
-    load_qd(first, tiles - 1);
+    load_qd(first, tiles - 1, 0);
     load_p(first, tiles - 1);
   }
 
   constexpr uint32_t id_kk = idesc_bf16(128, 128, 0, 0);
   constexpr uint32_t id_kn = idesc_bf16(128, 128, 0, 1);
   constexpr uint32_t id_nn = idesc_bf16(128, 128, 1, 1);
-  const uint32_t aQ = smem_u32(sQ), aK = smem_u32(sK), aV = smem_u32(sV), aD = smem_u32(sD);
-  const uint32_t aX = smem_u32(sX), aA = smem_u32(sA), aB = smem_u32(sB);
+  const uint32_t aK = smem_u32(sK), aV = smem_u32(sV), aX = smem_u32(sX);
   uint32_t it = 0;
   uint32_t nseg_done = 0;  // segments started by this CTA
   bool stop = false;
@@ -217,14 +227,16 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_walk_tc(
     if (tid < kTile) s->pw[tid] = decay_pow(l2, (float)tid);
     if (tid == kProducer) {
       // R entering the segment's last chunk, as four 32-column fp32 boxes into
-      // A and B (free once the previous chunk's dK/dV stores have read them);
-      // epilogue 1 of the first chunk moves it into TMEM
+      // the first chunk's dP'/S' pair (free once the previous chunk's dK/dV
+      // stores have read it); epilogue 1 of that chunk moves it into TMEM
       tma_store_wait_read0();
       const int64_t slot = (int64_t)item.seg * tiles + tiles - 1;
       const int y = (int)((((int64_t)item.b * T + slot) * H + item.h) * kD);
+      const uint32_t ps = (it & 1u) ^ 1u;
       mbar_arrive_expect_tx(&s->ld_r, kD * kD * 4);
 #pragma unroll
-      for (int bx = 0; bx < 4; ++bx) tma_load_2d(sA + bx * kBox, &map_state, &s->ld_r, 32 * bx, y);
+      for (int bx = 0; bx < 4; ++bx)
+        tma_load_2d(pair(ps, bx >> 1) + (bx & 1) * kBox, &map_state, &s->ld_r, 32 * bx, y);
     }
     tc_fence_before();
     __syncthreads();
@@ -232,6 +244,11 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_walk_tc(
     for (int t = tiles - 1; t >= 0; --t, ++it) {
       const uint32_t par = it & 1u;
       const int row0 = item.seg * G + t * kTile;
+      uint8_t* sQ = pair(par, 0);  // Q, then dK out
+      uint8_t* sD = pair(par, 1);  // dO, then dV out
+      uint8_t* sA = pair(par ^ 1u, 0);  // dP'
+      uint8_t* sB = pair(par ^ 1u, 1);  // S'
+      const uint32_t aQ = smem_u32(sQ), aD = smem_u32(sD), aA = smem_u32(sA), aB = smem_u32(sB);
 
       // ---- MMA 1
       if (tid == 0) {
@@ -240,15 +257,17 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_walk_tc(
           tc_fence_after();
           for (int kk = 0; kk < kD / 16; ++kk) mma_bf16(tmem + T0, kmaj(aD, kk), kmaj(aV, kk), id_kk, kk != 0);
           for (int kk = 0; kk < kD / 16; ++kk) mma_bf16(tmem + T1, kmaj(aQ, kk), kmaj(aK, kk), id_kk, kk != 0);
-          for (int kk = 0; kk < kD / 16; ++kk) mma_bf16(tmem + T2, kmaj(aD, kk), kmaj(aX, kk), id_kk, kk != 0);
           mma_commit(&s->c1);
+          // dO P^T runs while epilogue 1 masks dP and S
+          for (int kk = 0; kk < kD / 16; ++kk) mma_bf16(tmem + T2, kmaj(aD, kk), kmaj(aX, kk), id_kk, kk != 0);
+          mma_commit(&s->c1b);
         } else {
           s->abort = 1;
         }
       }
 
-      // the previous chunk's dK/dV stores must have left A and B before epilogue 1
-      // writes them (MMA 1 does not touch A or B)
+      // the previous chunk's dK/dV stores must have left the dP'/S' pair before
+      // epilogue 1 writes it (MMA 1 does not touch it)
       if (tid == kProducer) tma_store_wait_read0();
       __syncthreads();
       if (s->abort) {
@@ -258,11 +277,11 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_walk_tc(
 
       // ---- epilogue 1
       if (t == tiles - 1) {
-        // the segment's entering R: A/B -> TMEM R. Row i of a swizzled box has
-        // its 16-byte chunk c at position c ^ (i & 7), so the eight rows of a
-        // quarter-warp read different banks.
+        // the segment's entering R: dP'/S' pair -> TMEM R. Row i of a swizzled
+        // box has its 16-byte chunk c at position c ^ (i & 7), so the eight rows
+        // of a quarter-warp read different banks.
         if (mbar_wait(&s->ld_r, nseg_done & 1u, SITE_BWD_TMA)) {
-          const uint8_t* src = sA + half * 2 * kBox;
+          const uint8_t* src = pair(par ^ 1u, half);
           uint32_t r[2][32];
 #pragma unroll
           for (int bb = 0; bb < 2; ++bb)
@@ -281,7 +300,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_walk_tc(
           s->abort = 1;
         }
         ++nseg_done;
-        __syncthreads();  // all of R is read before A and B are rewritten
+        __syncthreads();  // all of R is read before the pair is rewritten
         if (s->abort) {
           stop = true;
           break;
@@ -306,7 +325,9 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_walk_tc(
           st_row32_bf16(sA, i, cc * 32, fp);
           st_row32_bf16(sB, i, cc * 32, fs);
         }
-        // R of this chunk -> bf16 X (MMA 1 has read P) and pre-scaled by lambda^128 for MMA 4
+        // R of this chunk -> bf16 X (once dO P^T has read P) and pre-scaled by lambda^128 for MMA 4
+        if (!mbar_wait(&s->c1b, par, SITE_BWD_MMA)) s->abort = 1;
+        tc_fence_after();
         {
           uint32_t r[2][32];
           tmem_ld32(lane_base + TR + half * 64, r[0]);
@@ -345,6 +366,8 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_walk_tc(
         tc_fence_after();
         for (int kk = 0; kk < kTile / 16; ++kk) mma_bf16(tmem + T0, kmaj(aA, kk), mnmaj(aK, kk), id_kn, kk != 0);
         mma_commit(&s->c2);
+        // dV_intra = S'^T dO runs while epilogue 2 drains dQ (TMEM 1 was emptied by epilogue 1)
+        for (int kk = 0; kk < kTile / 16; ++kk) mma_bf16(tmem + T1, mnmaj(aB, kk), mnmaj(aD, kk), id_nn, kk != 0);
       }
       // ---- epilogue 2: dQ
       if (mbar_wait(&s->c2, par, SITE_BWD_MMA)) {
@@ -377,19 +400,33 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_walk_tc(
         break;
       }
 
-      // ---- MMA 3: dK = dP'^T Q + V~ R^T, dV_intra = S'^T dO, dV_inter = K R
+      // ---- MMA 3: dK = dP'^T Q + V~ R^T, dV_inter = K R
       if (tid == 0) {
         tc_fence_after();
         for (int kk = 0; kk < kTile / 16; ++kk) mma_bf16(tmem + T0, mnmaj(aA, kk), mnmaj(aQ, kk), id_nn, kk != 0);
+        mma_commit(&s->c3a);
+        // the rest of MMA 3 runs while Q is rescaled
         for (int kk = 0; kk < kD / 16; ++kk) mma_bf16(tmem + T0, kmaj(aV, kk), kmaj(aX, kk), id_kk, 1);
-        for (int kk = 0; kk < kTile / 16; ++kk) mma_bf16(tmem + T1, mnmaj(aB, kk), mnmaj(aD, kk), id_nn, kk != 0);
         for (int kk = 0; kk < kD / 16; ++kk) mma_bf16(tmem + T2, kmaj(aK, kk), mnmaj(aX, kk), id_kn, kk != 0);
         mma_commit(&s->c3);
       }
-      // ---- epilogue 3, first Q~ = diag(lambda^{j+1}) Q so that MMA 4 and the
-      // next chunk's loads can start, then dK -> A, dV -> B
-      if (mbar_wait(&s->c3, par, SITE_BWD_MMA)) {
+      // the next chunk of this CTA's stream
+      Item nx = item;
+      int nt = t - 1;
+      bool has_next = true;
+      if (nt < 0) {
+        has_next = w + gridDim.x < nitems;
+        if (has_next) {
+          nx = item_of(w + gridDim.x, H, nseg);
+          nt = tiles - 1;
+        }
+      }
+      // ---- epilogue 3, first Q~ = diag(lambda^{j+1}) Q (as soon as dP'^T Q has
+      // read Q) so that MMA 4 can start, then dK, dV out
+      if (mbar_wait(&s->c3a, par, SITE_BWD_MMA)) {
         tc_fence_after();
+        // dP' and S' have been read: the next chunk's Q and dO go into their pair
+        if (tid == kProducer && has_next) load_qd(nx, nt, par ^ 1u);
         if (scale) {
           scale_rows(sQ, s->pw, false, lam, tid);  // lambda^{j+1} = pw[j] * lambda
           fence_async_smem();
@@ -410,37 +447,32 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_walk_tc(
         mma_commit(&s->c4);
       }
       if (tid == kProducer) {
-        // next chunk of this CTA's stream: K, V and X were read by MMA 3, Q and dO
-        // are free once MMA 4 is done
-        Item nx = item;
-        int nt = t - 1;
-        bool has_next = true;
-        if (nt < 0) {
-          has_next = w + gridDim.x < nitems;
-          if (has_next) {
-            nx = item_of(w + gridDim.x, H, nseg);
-            nt = tiles - 1;
-          }
-        }
         if (t == (tiles > 1 ? 1 : 0) && w + gridDim.x < nitems) {
-          // the next segment's entering R is read by all threads at the segment
-          // switch; bring it into L2 while this segment's last tiles run
+          // the next segment's entering R is read at the segment switch; bring
+          // it into L2 while this segment's last chunks run
           const Item ns = item_of(w + gridDim.x, H, nseg);
           const int64_t slot = (int64_t)ns.seg * tiles + tiles - 1;
           bulk_prefetch_l2(R + (((int64_t)ns.b * T + slot) * H + ns.h) * kD * kD, kD * kD * sizeof(float));
         }
+        // K, V and X are free once all of MMA 3 is done
         if (has_next) {
-          load_kv(nx, nt);
-          load_p(nx, nt);
-          if (mbar_wait(&s->c4, par, SITE_BWD_MMA)) load_qd(nx, nt);
-          else s->abort = 1;
+          if (mbar_wait(&s->c3, par, SITE_BWD_MMA)) {
+            load_kv(nx, nt);
+            load_p(nx, nt);
+          } else {
+            s->abort = 1;
+          }
         }
       }
-      {
+      if (mbar_wait(&s->c3, par, SITE_BWD_MMA)) {
         tc_fence_after();
         const float wj = decay_pow(l2, (float)(kTile - 1 - i));  // dV inter decay of row j = i
+        // dK and dV are staged over Q~ and dO once MMA 4 has read them
+        const bool ok4 = mbar_wait(&s->c4, par, SITE_BWD_MMA);
+        if (!ok4) s->abort = 1;
+        tc_fence_after();
 #pragma unroll 1
-        for (int cc = 2 * half; cc < 2 * half + 2; ++cc) {
+        for (int cc = 2 * half; cc < 2 * half + 2 && ok4; ++cc) {
           uint32_t ka[32], va[32], ve[32];
           tmem_ld32(lane_base + T0 + cc * 32, ka);
           tmem_ld32(lane_base + T1 + cc * 32, va);
@@ -452,18 +484,24 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_walk_tc(
             fk[q] = __uint_as_float(ka[q]);
             fv[q] = fmaf(wj, __uint_as_float(ve[q]), __uint_as_float(va[q]));
           }
-          st_row32_bf16(sA, i, cc * 32, fk);
-          st_row32_bf16(sB, i, cc * 32, fv);
+          st_row32_bf16(sQ, i, cc * 32, fk);
+          st_row32_bf16(sD, i, cc * 32, fv);
         }
         fence_async_smem();
+      } else {
+        s->abort = 1;
       }
       tc_fence_before();
       __syncthreads();
+      if (s->abort) {
+        stop = true;
+        break;
+      }
       if (tid == kProducer) {
-        tma_store_4d(&map_dk, sA, 0, item.h, row0, item.b);
-        tma_store_4d(&map_dk, sA + kBox, 64, item.h, row0, item.b);
-        tma_store_4d(&map_dv, sB, 0, item.h, row0, item.b);
-        tma_store_4d(&map_dv, sB + kBox, 64, item.h, row0, item.b);
+        tma_store_4d(&map_dk, sQ, 0, item.h, row0, item.b);
+        tma_store_4d(&map_dk, sQ + kBox, 64, item.h, row0, item.b);
+        tma_store_4d(&map_dv, sD, 0, item.h, row0, item.b);
+        tma_store_4d(&map_dv, sD + kBox, 64, item.h, row0, item.b);
         tma_store_commit();
       }
     }
