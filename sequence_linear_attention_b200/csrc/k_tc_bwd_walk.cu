@@ -49,16 +49,24 @@ using namespace sm100;
 
 constexpr int kD = 128;
 constexpr int kTile = 128;
-constexpr int kThreads = 256;
-constexpr int kWarps = kThreads / 32;
+// warps 0-7 run the epilogues (warp w owns TMEM lanes 32*(w%4).. and column
+// half w/4), warp 8 issues the MMAs, warp 9 the TMA loads and stores
+constexpr int kEpiThreads = 256;
+constexpr int kMmaWarp = 8;
+constexpr int kProducerWarp = 9;
+constexpr int kThreads = 320;
+constexpr uint32_t kEpiBar = 1;  // named barrier of the epilogue warps
 constexpr uint32_t kTileBytes = kTile * kD * 2;
 constexpr uint32_t kBox = kTileBytes / 2;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t T0 = 0, T1 = 128, T2 = 256, TR = 384;
 
 struct Smem {
-  uint64_t ld_kv, ld_qd, ld_p, ld_r;
-  uint64_t c1, c1b, c2, c3a, c3, c4;
+  uint64_t ld_kv, ld_qd, ld_p, ld_r;  // TMA -> MMA warp / epilogue
+  uint64_t c1, c1b, c2, c3a, c3, c4;  // MMA commits -> epilogue / producer
+  uint64_t e1, e2, e3a, e0;           // epilogue -> MMA warp (256 arrivals each)
+  uint64_t staged;                    // epilogue -> producer: dK, dV staged (256 arrivals)
+  uint64_t scratch_free;              // producer -> epilogue: the dP'/S' pair has been stored out
   uint32_t tmem_base;
   int abort;
   float pw[kTile];
@@ -93,7 +101,7 @@ __device__ __forceinline__ uint64_t mnmaj(uint32_t tile, int kk) { return sw128_
 __device__ __forceinline__ void scale_rows(uint8_t* tile, const float* pw, bool flip, float post, int tid) {
   uint4* t4 = reinterpret_cast<uint4*>(tile);
 #pragma unroll 2
-  for (int g = tid; g < kTile * 16; g += kThreads) {
+  for (int g = tid; g < kTile * 16; g += kEpiThreads) {
     const int r = (g & (kTile * 8 - 1)) >> 3;
     const float w = pw[flip ? kTile - 1 - r : r] * post;
     uint4 x = t4[g];
@@ -134,10 +142,9 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_walk_tc(
   // (pair 0: buffers 0 and 3; pair 1: buffers 5 and 6)
   auto pair = [&](uint32_t p, int m) { return base + (p ? 5 + m : 3 * m) * kTileBytes; };
   Smem* s = reinterpret_cast<Smem*>(base + 7 * kTileBytes);
+  const volatile int* abort_flag = &s->abort;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int i = (warp & 3) * 32 + lane;
-  const int half = warp >> 2;
   const int tiles = G / kTile;
 
   if (tid == 0) {
@@ -156,6 +163,12 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_walk_tc(
     mbar_init(&s->c3a, 1);
     mbar_init(&s->c3, 1);
     mbar_init(&s->c4, 1);
+    mbar_init(&s->e1, kEpiThreads);
+    mbar_init(&s->e2, kEpiThreads);
+    mbar_init(&s->e3a, kEpiThreads);
+    mbar_init(&s->e0, kEpiThreads);
+    mbar_init(&s->staged, kEpiThreads);
+    mbar_init(&s->scratch_free, 1);
     s->abort = 0;
     fence_mbar_init();
   }
@@ -167,120 +180,221 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_walk_tc(
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = s->tmem_base;
-  const uint32_t lane_base = tmem + ((uint32_t)((warp & 3) * 32) << 16);
 
-  auto load_kv = [&](const Item& it, int t) {
-    const int row = it.seg * G + t * kTile;
-    mbar_arrive_expect_tx(&s->ld_kv, 2 * kTileBytes);
-    tma_load_4d(sK, &map_k, &s->ld_kv, 0, it.h, row, it.b);
-    tma_load_4d(sK + kBox, &map_k, &s->ld_kv, 64, it.h, row, it.b);
-    tma_load_4d(sV, &map_v, &s->ld_kv, 0, it.h, row, it.b);
-    tma_load_4d(sV + kBox, &map_v, &s->ld_kv, 64, it.h, row, it.b);
-  };
-  auto load_qd = [&](const Item& it, int t, uint32_t p) {
-    const int row = it.seg * G + t * kTile;
-    uint8_t* q = pair(p, 0);
-    uint8_t* d = pair(p, 1);
-    mbar_arrive_expect_tx(&s->ld_qd, 2 * kTileBytes);
-    tma_load_4d(q, &map_q, &s->ld_qd, 0, it.h, row, it.b);
-    tma_load_4d(q + kBox, &map_q, &s->ld_qd, 64, it.h, row, it.b);
-    tma_load_4d(d, &map_do, &s->ld_qd, 0, it.h, row, it.b);
-    tma_load_4d(d + kBox, &map_do, &s->ld_qd, 64, it.h, row, it.b);
-  };
+  if (warp == kProducerWarp) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      auto load_kv = [&](const Item& it, int t) {
+        const int row = it.seg * G + t * kTile;
+        mbar_arrive_expect_tx(&s->ld_kv, 2 * kTileBytes);
+        tma_load_4d(sK, &map_k, &s->ld_kv, 0, it.h, row, it.b);
+        tma_load_4d(sK + kBox, &map_k, &s->ld_kv, 64, it.h, row, it.b);
+        tma_load_4d(sV, &map_v, &s->ld_kv, 0, it.h, row, it.b);
+        tma_load_4d(sV + kBox, &map_v, &s->ld_kv, 64, it.h, row, it.b);
+      };
+      auto load_qd = [&](const Item& it, int t, uint32_t p) {
+        const int row = it.seg * G + t * kTile;
+        uint8_t* q = pair(p, 0);
+        uint8_t* d = pair(p, 1);
+        mbar_arrive_expect_tx(&s->ld_qd, 2 * kTileBytes);
+        tma_load_4d(q, &map_q, &s->ld_qd, 0, it.h, row, it.b);
+        tma_load_4d(q + kBox, &map_q, &s->ld_qd, 64, it.h, row, it.b);
+        tma_load_4d(d, &map_do, &s->ld_qd, 0, it.h, row, it.b);
+        tma_load_4d(d + kBox, &map_do, &s->ld_qd, 64, it.h, row, it.b);
+      };
+      // P of a chunk: the forward walk stored it in the chunk's cache slot as the
+      // bf16 operand tile (128-byte swizzled), so it is copied into X as is
+      auto load_p = [&](const Item& it, int t) {
+        const int64_t c = ((int64_t)it.seg * G + (int64_t)t * kTile) / kTile;
+        const float* src = P + (((int64_t)it.b * T + c) * H + it.h) * kD * kD;
+        mbar_arrive_expect_tx(&s->ld_p, kTileBytes);
+        bulk_load(sX, src, kTileBytes, &s->ld_p);
+      };
+      auto store_dkdv = [&](const Item& it, int row0, uint32_t p) {
+        tma_store_4d(&map_dk, pair(p, 0), 0, it.h, row0, it.b);
+        tma_store_4d(&map_dk, pair(p, 0) + kBox, 64, it.h, row0, it.b);
+        tma_store_4d(&map_dv, pair(p, 1), 0, it.h, row0, it.b);
+        tma_store_4d(&map_dv, pair(p, 1) + kBox, 64, it.h, row0, it.b);
+        tma_store_commit();
+      };
 
-  // P of a chunk: the forward walk stored it in the chunk's cache slot as the
-  // bf16 operand tile (128-byte swizzled), so it is copied into X as is
-  auto load_p = [&](const Item& it, int t) {
-    const int64_t c = ((int64_t)it.seg * G + (int64_t)t * kTile) / kTile;
-    const float* src = P + (((int64_t)it.b * T + c) * H + it.h) * kD * kD;
-    mbar_arrive_expect_tx(&s->ld_p, kTileBytes);
-    bulk_load(sX, src, kTileBytes, &s->ld_p);
-  };
-
-  // thread 32 issues every TMA load and bulk copy (and waits for the stores it
-  // issued); thread 0 issues the MMAs
-  constexpr int kProducer = 32;
-  if (tid == kProducer && (int64_t)blockIdx.x < nitems) {
-    const Item first = item_of(blockIdx.x, H, nseg);
-    load_kv(first, tiles - 1);
-    load_qd(first, tiles - 1, 0);
-    load_p(first, tiles - 1);
-  }
-
-  constexpr uint32_t id_kk = idesc_bf16(128, 128, 0, 0);
-  constexpr uint32_t id_kn = idesc_bf16(128, 128, 0, 1);
-  constexpr uint32_t id_nn = idesc_bf16(128, 128, 1, 1);
-  const uint32_t aK = smem_u32(sK), aV = smem_u32(sV), aX = smem_u32(sX);
-  uint32_t it = 0;
-  uint32_t nseg_done = 0;  // segments started by this CTA
-  bool stop = false;
-
-  for (int64_t w = blockIdx.x; w < nitems && !stop; w += gridDim.x) {
-    const Item item = item_of(w, H, nseg);
-    const float lam = load_decay(decay, item.h);
-    const float l2 = log2f(lam);
-    const bool scale = lam != 1.0f;
-    const float g_tile = decay_pow(l2, (float)kTile);
-    // the previous segment's last MMA 4 writes TMEM R: let it finish before R is replaced
-    if (it > 0 && !mbar_wait(&s->c4, (it - 1) & 1u, SITE_BWD_MMA)) s->abort = 1;
-    tc_fence_after();
-    if (tid < kTile) s->pw[tid] = decay_pow(l2, (float)tid);
-    if (tid == kProducer) {
-      // R entering the segment's last chunk, as four 32-column fp32 boxes into
-      // the first chunk's dP'/S' pair (free once the previous chunk's dK/dV
-      // stores have read it); epilogue 1 of that chunk moves it into TMEM
-      tma_store_wait_read0();
-      const int64_t slot = (int64_t)item.seg * tiles + tiles - 1;
-      const int y = (int)((((int64_t)item.b * T + slot) * H + item.h) * kD);
-      const uint32_t ps = (it & 1u) ^ 1u;
-      mbar_arrive_expect_tx(&s->ld_r, kD * kD * 4);
+      if ((int64_t)blockIdx.x < nitems) {
+        const Item first = item_of(blockIdx.x, H, nseg);
+        load_kv(first, tiles - 1);
+        load_qd(first, tiles - 1, 0);
+        load_p(first, tiles - 1);
+      }
+      uint32_t it = 0;
+      Item prev{0, 0, 0};
+      int prev_row = 0;
+      bool ok = true;
+      for (int64_t w = blockIdx.x; w < nitems && ok; w += gridDim.x) {
+        const Item item = item_of(w, H, nseg);
+        for (int t = tiles - 1; t >= 0 && ok; --t, ++it) {
+          const uint32_t par = it & 1u;
+          const int row0 = item.seg * G + t * kTile;
+          // the previous chunk's dK and dV, staged over its Q~ and dO, go out;
+          // once they have been read, that pair is this chunk's dP'/S' pair
+          if (it > 0) {
+            if (!(ok = mbar_wait_or_abort(&s->staged, (it - 1) & 1u, SITE_BWD_TMA, abort_flag))) break;
+            store_dkdv(prev, prev_row, par ^ 1u);
+          }
+          tma_store_wait_read0();
+          if (t == tiles - 1) {
+            // R entering the segment's last chunk, as four 32-column fp32 boxes
+            // into the dP'/S' pair; epilogue 1 moves it into TMEM
+            const int64_t slot = (int64_t)item.seg * tiles + tiles - 1;
+            const int y = (int)((((int64_t)item.b * T + slot) * H + item.h) * kD);
+            mbar_arrive_expect_tx(&s->ld_r, kD * kD * 4);
 #pragma unroll
-      for (int bx = 0; bx < 4; ++bx)
-        tma_load_2d(pair(ps, bx >> 1) + (bx & 1) * kBox, &map_state, &s->ld_r, 32 * bx, y);
+            for (int bx = 0; bx < 4; ++bx)
+              tma_load_2d(pair(par ^ 1u, bx >> 1) + (bx & 1) * kBox, &map_state, &s->ld_r, 32 * bx, y);
+          }
+          mbar_arrive(&s->scratch_free);
+
+          // the next chunk of this CTA's stream
+          Item nx = item;
+          int nt = t - 1;
+          bool has_next = true;
+          if (nt < 0) {
+            has_next = w + gridDim.x < nitems;
+            if (has_next) {
+              nx = item_of(w + gridDim.x, H, nseg);
+              nt = tiles - 1;
+            }
+          }
+          if (has_next) {
+            // into L2 now, so that the loads issued once this chunk's MMAs have
+            // freed their buffers are short
+            const int nrow = nx.seg * G + nt * kTile;
+            tma_prefetch_4d(&map_q, 0, nx.h, nrow, nx.b);
+            tma_prefetch_4d(&map_q, 64, nx.h, nrow, nx.b);
+            tma_prefetch_4d(&map_do, 0, nx.h, nrow, nx.b);
+            tma_prefetch_4d(&map_do, 64, nx.h, nrow, nx.b);
+            tma_prefetch_4d(&map_k, 0, nx.h, nrow, nx.b);
+            tma_prefetch_4d(&map_k, 64, nx.h, nrow, nx.b);
+            tma_prefetch_4d(&map_v, 0, nx.h, nrow, nx.b);
+            tma_prefetch_4d(&map_v, 64, nx.h, nrow, nx.b);
+            const int64_t c = (int64_t)nrow / kTile;
+            bulk_prefetch_l2(P + (((int64_t)nx.b * T + c) * H + nx.h) * kD * kD, kTileBytes);
+          }
+          if (t == (tiles > 1 ? 1 : 0) && w + gridDim.x < nitems) {
+            // and the next segment's entering R, read at the segment switch
+            const Item ns = item_of(w + gridDim.x, H, nseg);
+            const int64_t slot = (int64_t)ns.seg * tiles + tiles - 1;
+            bulk_prefetch_l2(R + (((int64_t)ns.b * T + slot) * H + ns.h) * kD * kD, kD * kD * sizeof(float));
+          }
+          // dP' and S' have been read once the first part of MMA 3 is done: the
+          // next Q and dO go into their pair; K, V and X are free after all of MMA 3
+          if (!(ok = mbar_wait_or_abort(&s->c3a, par, SITE_BWD_MMA, abort_flag))) break;
+          if (has_next) load_qd(nx, nt, par ^ 1u);
+          if (!(ok = mbar_wait_or_abort(&s->c3, par, SITE_BWD_MMA, abort_flag))) break;
+          if (has_next) {
+            load_kv(nx, nt);
+            load_p(nx, nt);
+          }
+          prev = item;
+          prev_row = row0;
+        }
+      }
+      if (ok && it > 0 && mbar_wait_or_abort(&s->staged, (it - 1) & 1u, SITE_BWD_TMA, abort_flag))
+        store_dkdv(prev, prev_row, (it - 1) & 1u);
+      if (!ok) s->abort = 1;
+      tma_store_wait0();
     }
-    tc_fence_before();
-    __syncthreads();
-
-    for (int t = tiles - 1; t >= 0; --t, ++it) {
-      const uint32_t par = it & 1u;
-      const int row0 = item.seg * G + t * kTile;
-      uint8_t* sQ = pair(par, 0);  // Q, then dK out
-      uint8_t* sD = pair(par, 1);  // dO, then dV out
-      uint8_t* sA = pair(par ^ 1u, 0);  // dP'
-      uint8_t* sB = pair(par ^ 1u, 1);  // S'
-      const uint32_t aQ = smem_u32(sQ), aD = smem_u32(sD), aA = smem_u32(sA), aB = smem_u32(sB);
-
-      // ---- MMA 1
-      if (tid == 0) {
-        if (mbar_wait(&s->ld_kv, par, SITE_BWD_TMA) && mbar_wait(&s->ld_qd, par, SITE_BWD_TMA) &&
-            mbar_wait(&s->ld_p, par, SITE_BWD_TMA)) {
+  } else if (warp == kMmaWarp) {
+    // ------------------------------------------------------------ MMA issue
+    if (lane == 0) {
+      constexpr uint32_t id_kk = idesc_bf16(128, 128, 0, 0);
+      constexpr uint32_t id_kn = idesc_bf16(128, 128, 0, 1);
+      constexpr uint32_t id_nn = idesc_bf16(128, 128, 1, 1);
+      const uint32_t aK = smem_u32(sK), aV = smem_u32(sV), aX = smem_u32(sX);
+      uint32_t it = 0;
+      bool ok = true;
+      for (int64_t w = blockIdx.x; w < nitems && ok; w += gridDim.x) {
+        for (int t = tiles - 1; t >= 0; --t, ++it) {
+          const uint32_t par = it & 1u;
+          const uint32_t aQ = smem_u32(pair(par, 0)), aD = smem_u32(pair(par, 1));
+          const uint32_t aA = smem_u32(pair(par ^ 1u, 0)), aB = smem_u32(pair(par ^ 1u, 1));
+          // MMA 1 needs this chunk's loads, and TMEM 0-2 drained by the previous epilogue 3
+          ok = mbar_wait_or_abort(&s->ld_kv, par, SITE_BWD_TMA, abort_flag) &&
+               mbar_wait_or_abort(&s->ld_qd, par, SITE_BWD_TMA, abort_flag) &&
+               mbar_wait_or_abort(&s->ld_p, par, SITE_BWD_TMA, abort_flag) &&
+               (it == 0 || mbar_wait_or_abort(&s->e0, (it - 1) & 1u, SITE_BWD_MMA, abort_flag));
+          if (!ok) break;
           tc_fence_after();
+          // ---- MMA 1: T0 = dO V^T, T1 = Q K^T | T2 = dO P^T
           for (int kk = 0; kk < kD / 16; ++kk) mma_bf16(tmem + T0, kmaj(aD, kk), kmaj(aV, kk), id_kk, kk != 0);
           for (int kk = 0; kk < kD / 16; ++kk) mma_bf16(tmem + T1, kmaj(aQ, kk), kmaj(aK, kk), id_kk, kk != 0);
           mma_commit(&s->c1);
-          // dO P^T runs while epilogue 1 masks dP and S
           for (int kk = 0; kk < kD / 16; ++kk) mma_bf16(tmem + T2, kmaj(aD, kk), kmaj(aX, kk), id_kk, kk != 0);
           mma_commit(&s->c1b);
-        } else {
-          s->abort = 1;
+          // ---- MMA 2: T0 = dP' K | T1 = S'^T dO
+          if (!(ok = mbar_wait_or_abort(&s->e1, par, SITE_BWD_MMA, abort_flag))) break;
+          tc_fence_after();
+          for (int kk = 0; kk < kTile / 16; ++kk) mma_bf16(tmem + T0, kmaj(aA, kk), mnmaj(aK, kk), id_kn, kk != 0);
+          mma_commit(&s->c2);
+          for (int kk = 0; kk < kTile / 16; ++kk) mma_bf16(tmem + T1, mnmaj(aB, kk), mnmaj(aD, kk), id_nn, kk != 0);
+          // ---- MMA 3: T0 = dP'^T Q | T0 += V~ R^T, T2 = K R
+          if (!(ok = mbar_wait_or_abort(&s->e2, par, SITE_BWD_MMA, abort_flag))) break;
+          tc_fence_after();
+          for (int kk = 0; kk < kTile / 16; ++kk) mma_bf16(tmem + T0, mnmaj(aA, kk), mnmaj(aQ, kk), id_nn, kk != 0);
+          mma_commit(&s->c3a);
+          for (int kk = 0; kk < kD / 16; ++kk) mma_bf16(tmem + T0, kmaj(aV, kk), kmaj(aX, kk), id_kk, 1);
+          for (int kk = 0; kk < kD / 16; ++kk) mma_bf16(tmem + T2, kmaj(aK, kk), mnmaj(aX, kk), id_kn, kk != 0);
+          mma_commit(&s->c3);
+          // ---- MMA 4: R += Q~^T dO (TMEM R was pre-scaled by lambda^128 in epilogue 1)
+          if (!(ok = mbar_wait_or_abort(&s->e3a, par, SITE_BWD_MMA, abort_flag))) break;
+          tc_fence_after();
+          for (int kk = 0; kk < kTile / 16; ++kk) mma_bf16(tmem + TR, mnmaj(aQ, kk), mnmaj(aD, kk), id_nn, 1);
+          mma_commit(&s->c4);
         }
       }
-
-      // the previous chunk's dK/dV stores must have left the dP'/S' pair before
-      // epilogue 1 writes it (MMA 1 does not touch it)
-      if (tid == kProducer) tma_store_wait_read0();
-      __syncthreads();
-      if (s->abort) {
-        stop = true;
-        break;
+      if (!ok) s->abort = 1;
+    }
+  } else {
+    // ------------------------------------------------------------ epilogues
+    const int i = (warp & 3) * 32 + lane;  // the row this thread owns
+    const int half = warp >> 2;            // and the column half
+    const uint32_t lane_base = tmem + ((uint32_t)((warp & 3) * 32) << 16);
+    bool bad = false;
+    // a failed wait stops the other roles too; this thread runs on (on
+    // whatever data) to the next point where all epilogue warps agree to stop
+    auto wait = [&](uint64_t* bar, uint32_t parity, unsigned int site) {
+      if (!bad && !mbar_wait_or_abort(bar, parity, site, abort_flag)) {
+        bad = true;
+        s->abort = 1;
       }
+    };
+    uint32_t it = 0;
+    uint32_t nseg_done = 0;  // segments started by this CTA
+    for (int64_t w = blockIdx.x; w < nitems; w += gridDim.x) {
+      if (named_sync_or(kEpiBar, kEpiThreads, bad)) break;  // every epilogue thread is past the last segment
+      const Item item = item_of(w, H, nseg);
+      const float lam = load_decay(decay, item.h);
+      const float l2 = log2f(lam);
+      const bool scale = lam != 1.0f;
+      const float g_tile = decay_pow(l2, (float)kTile);
+      if (tid < kTile) s->pw[tid] = decay_pow(l2, (float)tid);
+      named_sync(kEpiBar, kEpiThreads);
 
-      // ---- epilogue 1
-      if (t == tiles - 1) {
-        // the segment's entering R: dP'/S' pair -> TMEM R. Row i of a swizzled
-        // box has its 16-byte chunk c at position c ^ (i & 7), so the eight rows
-        // of a quarter-warp read different banks.
-        if (mbar_wait(&s->ld_r, nseg_done & 1u, SITE_BWD_TMA)) {
+      for (int t = tiles - 1; t >= 0; --t, ++it) {
+        const uint32_t par = it & 1u;
+        const int row0 = item.seg * G + t * kTile;
+        uint8_t* sQ = pair(par, 0);       // Q, then dK out
+        uint8_t* sD = pair(par, 1);       // dO, then dV out
+        uint8_t* sA = pair(par ^ 1u, 0);  // dP'
+        uint8_t* sB = pair(par ^ 1u, 1);  // S'
+
+        // ---- epilogue 1
+        if (t == tiles - 1) {
+          // the segment's entering R: dP'/S' pair -> TMEM R, once the previous
+          // chunk's MMA 4 is done with TMEM R. Row i of a swizzled box has its
+          // 16-byte chunk c at position c ^ (i & 7), so the eight rows of a
+          // quarter-warp read different banks.
+          wait(&s->ld_r, nseg_done & 1u, SITE_BWD_TMA);
+          if (it > 0) wait(&s->c4, (it - 1) & 1u, SITE_BWD_MMA);
+          tc_fence_after();
           const uint8_t* src = pair(par ^ 1u, half);
           uint32_t r[2][32];
 #pragma unroll
@@ -296,17 +410,11 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_walk_tc(
           tmem_st32(lane_base + TR + half * 64, r[0]);
           tmem_st32(lane_base + TR + half * 64 + 32, r[1]);
           tmem_st_wait();
-        } else {
-          s->abort = 1;
+          ++nseg_done;
+          named_sync(kEpiBar, kEpiThreads);  // all of R is read before the pair is rewritten
         }
-        ++nseg_done;
-        __syncthreads();  // all of R is read before the pair is rewritten
-        if (s->abort) {
-          stop = true;
-          break;
-        }
-      }
-      if (mbar_wait(&s->c1, par, SITE_BWD_MMA)) {
+        wait(&s->scratch_free, par, SITE_BWD_TMA);  // the previous dK/dV stores have read the pair
+        wait(&s->c1, par, SITE_BWD_MMA);
         tc_fence_after();
 #pragma unroll 1
         for (int cc = 2 * half; cc < 2 * half + 2; ++cc) {
@@ -326,7 +434,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_walk_tc(
           st_row32_bf16(sB, i, cc * 32, fs);
         }
         // R of this chunk -> bf16 X (once dO P^T has read P) and pre-scaled by lambda^128 for MMA 4
-        if (!mbar_wait(&s->c1b, par, SITE_BWD_MMA)) s->abort = 1;
+        wait(&s->c1b, par, SITE_BWD_MMA);
         tc_fence_after();
         {
           uint32_t r[2][32];
@@ -351,164 +459,86 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_walk_tc(
           scale_rows(sV, s->pw, true, 1.f, tid);  // V~ = diag(lambda^{127-j}) V
         }
         fence_async_smem();
-      } else {
-        s->abort = 1;
-      }
-      tc_fence_before();
-      __syncthreads();
-      if (s->abort) {
-        stop = true;
-        break;
-      }
+        tc_fence_before();
+        mbar_arrive(&s->e1);
 
-      // ---- MMA 2: dQ_intra = dP' K
-      if (tid == 0) {
+        // ---- epilogue 2: dQ = T0 + lambda^{i+1} T2
+        wait(&s->c2, par, SITE_BWD_MMA);
         tc_fence_after();
-        for (int kk = 0; kk < kTile / 16; ++kk) mma_bf16(tmem + T0, kmaj(aA, kk), mnmaj(aK, kk), id_kn, kk != 0);
-        mma_commit(&s->c2);
-        // dV_intra = S'^T dO runs while epilogue 2 drains dQ (TMEM 1 was emptied by epilogue 1)
-        for (int kk = 0; kk < kTile / 16; ++kk) mma_bf16(tmem + T1, mnmaj(aB, kk), mnmaj(aD, kk), id_nn, kk != 0);
-      }
-      // ---- epilogue 2: dQ
-      if (mbar_wait(&s->c2, par, SITE_BWD_MMA)) {
-        tc_fence_after();
-        const float wi = decay_pow(l2, (float)(i + 1));
-        __nv_bfloat16* out = dq + (((int64_t)item.b * N + row0 + i) * H + item.h) * kD;
+        {
+          const float wi = decay_pow(l2, (float)(i + 1));
+          __nv_bfloat16* out = dq + (((int64_t)item.b * N + row0 + i) * H + item.h) * kD;
 #pragma unroll 1
-        for (int cc = 2 * half; cc < 2 * half + 2; ++cc) {
-          uint32_t ra[32], re[32];
-          tmem_ld32(lane_base + T0 + cc * 32, ra);
-          tmem_ld32(lane_base + T2 + cc * 32, re);
-          tmem_ld_wait();
+          for (int cc = 2 * half; cc < 2 * half + 2; ++cc) {
+            uint32_t ra[32], re[32];
+            tmem_ld32(lane_base + T0 + cc * 32, ra);
+            tmem_ld32(lane_base + T2 + cc * 32, re);
+            tmem_ld_wait();
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            float o[8];
+            for (int q = 0; q < 4; ++q) {
+              float o[8];
 #pragma unroll
-            for (int u = 0; u < 8; ++u) o[u] = fmaf(wi, __uint_as_float(re[q * 8 + u]), __uint_as_float(ra[q * 8 + u]));
-            *reinterpret_cast<uint4*>(out + cc * 32 + q * 8) =
-                make_uint4(pack_bf16(o[0], o[1]), pack_bf16(o[2], o[3]), pack_bf16(o[4], o[5]), pack_bf16(o[6], o[7]));
+              for (int u = 0; u < 8; ++u)
+                o[u] = fmaf(wi, __uint_as_float(re[q * 8 + u]), __uint_as_float(ra[q * 8 + u]));
+              *reinterpret_cast<uint4*>(out + cc * 32 + q * 8) = make_uint4(
+                  pack_bf16(o[0], o[1]), pack_bf16(o[2], o[3]), pack_bf16(o[4], o[5]), pack_bf16(o[6], o[7]));
+            }
           }
         }
-        fence_async_smem();
-      } else {
-        s->abort = 1;
-      }
-      tc_fence_before();
-      __syncthreads();
-      if (s->abort) {
-        stop = true;
-        break;
-      }
+        tc_fence_before();
+        mbar_arrive(&s->e2);
 
-      // ---- MMA 3: dK = dP'^T Q + V~ R^T, dV_inter = K R
-      if (tid == 0) {
-        tc_fence_after();
-        for (int kk = 0; kk < kTile / 16; ++kk) mma_bf16(tmem + T0, mnmaj(aA, kk), mnmaj(aQ, kk), id_nn, kk != 0);
-        mma_commit(&s->c3a);
-        // the rest of MMA 3 runs while Q is rescaled
-        for (int kk = 0; kk < kD / 16; ++kk) mma_bf16(tmem + T0, kmaj(aV, kk), kmaj(aX, kk), id_kk, 1);
-        for (int kk = 0; kk < kD / 16; ++kk) mma_bf16(tmem + T2, kmaj(aK, kk), mnmaj(aX, kk), id_kn, kk != 0);
-        mma_commit(&s->c3);
-      }
-      // the next chunk of this CTA's stream
-      Item nx = item;
-      int nt = t - 1;
-      bool has_next = true;
-      if (nt < 0) {
-        has_next = w + gridDim.x < nitems;
-        if (has_next) {
-          nx = item_of(w + gridDim.x, H, nseg);
-          nt = tiles - 1;
-        }
-      }
-      // ---- epilogue 3, first Q~ = diag(lambda^{j+1}) Q (as soon as dP'^T Q has
-      // read Q) so that MMA 4 can start, then dK, dV out
-      if (mbar_wait(&s->c3a, par, SITE_BWD_MMA)) {
-        tc_fence_after();
-        // dP' and S' have been read: the next chunk's Q and dO go into their pair
-        if (tid == kProducer && has_next) load_qd(nx, nt, par ^ 1u);
+        // ---- epilogue 3a: Q~ = diag(lambda^{j+1}) Q once dP'^T Q has read Q
+        wait(&s->c3a, par, SITE_BWD_MMA);
         if (scale) {
           scale_rows(sQ, s->pw, false, lam, tid);  // lambda^{j+1} = pw[j] * lambda
           fence_async_smem();
         }
-      } else {
-        s->abort = 1;
-      }
-      tc_fence_before();
-      __syncthreads();
-      if (s->abort) {
-        stop = true;
-        break;
-      }
-      if (tid == 0) {
+        mbar_arrive(&s->e3a);
+
+        // ---- epilogue 3b: dK = T0, dV = T1 + lambda^{127-j} T2, staged over
+        // Q~ and dO once MMA 4 has read them
+        wait(&s->c3, par, SITE_BWD_MMA);
         tc_fence_after();
-        // ---- MMA 4: R += Q~^T dO (TMEM R was pre-scaled by lambda^128 in epilogue 1)
-        for (int kk = 0; kk < kTile / 16; ++kk) mma_bf16(tmem + TR, mnmaj(aQ, kk), mnmaj(aD, kk), id_nn, 1);
-        mma_commit(&s->c4);
-      }
-      if (tid == kProducer) {
-        if (t == (tiles > 1 ? 1 : 0) && w + gridDim.x < nitems) {
-          // the next segment's entering R is read at the segment switch; bring
-          // it into L2 while this segment's last chunks run
-          const Item ns = item_of(w + gridDim.x, H, nseg);
-          const int64_t slot = (int64_t)ns.seg * tiles + tiles - 1;
-          bulk_prefetch_l2(R + (((int64_t)ns.b * T + slot) * H + ns.h) * kD * kD, kD * kD * sizeof(float));
-        }
-        // K, V and X are free once all of MMA 3 is done
-        if (has_next) {
-          if (mbar_wait(&s->c3, par, SITE_BWD_MMA)) {
-            load_kv(nx, nt);
-            load_p(nx, nt);
-          } else {
-            s->abort = 1;
-          }
-        }
-      }
-      if (mbar_wait(&s->c3, par, SITE_BWD_MMA)) {
-        tc_fence_after();
-        const float wj = decay_pow(l2, (float)(kTile - 1 - i));  // dV inter decay of row j = i
-        // dK and dV are staged over Q~ and dO once MMA 4 has read them
-        const bool ok4 = mbar_wait(&s->c4, par, SITE_BWD_MMA);
-        if (!ok4) s->abort = 1;
-        tc_fence_after();
-#pragma unroll 1
-        for (int cc = 2 * half; cc < 2 * half + 2 && ok4; ++cc) {
-          uint32_t ka[32], va[32], ve[32];
-          tmem_ld32(lane_base + T0 + cc * 32, ka);
-          tmem_ld32(lane_base + T1 + cc * 32, va);
-          tmem_ld32(lane_base + T2 + cc * 32, ve);
-          tmem_ld_wait();
-          float fk[32], fv[32];
+        {
+          const float wj = decay_pow(l2, (float)(kTile - 1 - i));  // dV inter decay of row j = i
+          uint32_t pk[2][16], pv[2][16];  // bf16 pairs of dK and dV, held until MMA 4 is done
 #pragma unroll
-          for (int q = 0; q < 32; ++q) {
-            fk[q] = __uint_as_float(ka[q]);
-            fv[q] = fmaf(wj, __uint_as_float(ve[q]), __uint_as_float(va[q]));
+          for (int c2 = 0; c2 < 2; ++c2) {
+            uint32_t ka[32], va[32], ve[32];
+            tmem_ld32(lane_base + T0 + (2 * half + c2) * 32, ka);
+            tmem_ld32(lane_base + T1 + (2 * half + c2) * 32, va);
+            tmem_ld32(lane_base + T2 + (2 * half + c2) * 32, ve);
+            tmem_ld_wait();
+#pragma unroll
+            for (int q = 0; q < 16; ++q) {
+              pk[c2][q] = pack_bf16(__uint_as_float(ka[2 * q]), __uint_as_float(ka[2 * q + 1]));
+              pv[c2][q] = pack_bf16(fmaf(wj, __uint_as_float(ve[2 * q]), __uint_as_float(va[2 * q])),
+                                    fmaf(wj, __uint_as_float(ve[2 * q + 1]), __uint_as_float(va[2 * q + 1])));
+            }
           }
-          st_row32_bf16(sQ, i, cc * 32, fk);
-          st_row32_bf16(sD, i, cc * 32, fv);
+          tc_fence_before();
+          mbar_arrive(&s->e0);  // TMEM 0-2 are free for the next chunk's MMA 1
+          wait(&s->c4, par, SITE_BWD_MMA);
+#pragma unroll
+          for (int c2 = 0; c2 < 2; ++c2)
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              const int col = (2 * half + c2) * 32 + q * 8;
+              st_tile16(sQ, i, col, make_uint4(pk[c2][4 * q], pk[c2][4 * q + 1], pk[c2][4 * q + 2], pk[c2][4 * q + 3]));
+              st_tile16(sD, i, col, make_uint4(pv[c2][4 * q], pv[c2][4 * q + 1], pv[c2][4 * q + 2], pv[c2][4 * q + 3]));
+            }
         }
         fence_async_smem();
-      } else {
-        s->abort = 1;
-      }
-      tc_fence_before();
-      __syncthreads();
-      if (s->abort) {
-        stop = true;
-        break;
-      }
-      if (tid == kProducer) {
-        tma_store_4d(&map_dk, sQ, 0, item.h, row0, item.b);
-        tma_store_4d(&map_dk, sQ + kBox, 64, item.h, row0, item.b);
-        tma_store_4d(&map_dv, sD, 0, item.h, row0, item.b);
-        tma_store_4d(&map_dv, sD + kBox, 64, item.h, row0, item.b);
-        tma_store_commit();
+        mbar_arrive(&s->staged);
       }
     }
+    if (named_sync_or(kEpiBar, kEpiThreads, bad) && tid == 0) s->abort = 1;
   }
-  if (tid == kProducer) tma_store_wait0();
+  __syncwarp();
   tc_fence_before();
   __syncthreads();
+  tc_fence_after();
   if (warp == 0) tmem_dealloc(tmem, kTmemCols);
 }
 

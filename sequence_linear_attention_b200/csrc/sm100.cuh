@@ -57,6 +57,43 @@ __device__ __noinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, unsigned 
   }
 }
 
+// As mbar_wait, but also gives up, without recording anything, once *abort
+// is set by another thread of the CTA (checked on the slow path only).
+__device__ __noinline__ bool mbar_wait_or_abort(uint64_t* bar, uint32_t parity, unsigned int site,
+                                                const volatile int* abort) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const unsigned long long t0 = globaltimer_ns();
+  const unsigned long long limit = g_wait_limit_ns;
+  for (uint32_t it = 1;; ++it) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((it & 63u) == 0u) {
+      if (*abort) return false;
+      if (globaltimer_ns() - t0 > limit) {
+        record_error(LASP_ERR_TIMEOUT, site);
+        return false;
+      }
+    }
+  }
+}
+
+// Named barrier `id` over the first `nthreads` threads (whole warps) of the CTA.
+__device__ __forceinline__ void named_sync(uint32_t id, uint32_t nthreads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+// Named barrier that also returns the OR of `pred` over the participating threads.
+__device__ __forceinline__ bool named_sync_or(uint32_t id, uint32_t nthreads, bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.or.pred q, %2, %3, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}\n"
+      : "=r"(r)
+      : "r"((uint32_t)pred), "r"(id), "r"(nthreads)
+      : "memory");
+  return r != 0;
+}
+
 // ----------------------------------------------------------------------- TMA
 // 4-D tiled load into shared memory, completing bytes on `bar`.
 __device__ __forceinline__ void tma_load_4d(void* dst, const CUtensorMap* map, uint64_t* bar, int c0, int c1,
@@ -93,6 +130,12 @@ __device__ __forceinline__ void bulk_store(void* dst, const void* src, uint32_t 
 // multiple of 16); no completion, nothing lands in shared memory.
 __device__ __forceinline__ void bulk_prefetch_l2(const void* src, uint32_t bytes) {
   asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
+// Prefetch of one box of a 4-D tensor map into L2 (no completion).
+__device__ __forceinline__ void tma_prefetch_4d(const CUtensorMap* map, int c0, int c1, int c2, int c3) {
+  asm volatile("cp.async.bulk.prefetch.tensor.4d.L2.global.tile [%0, {%1, %2, %3, %4}];" ::"l"(map), "r"(c0),
+               "r"(c1), "r"(c2), "r"(c3)
+               : "memory");
 }
 // 4-D tiled store from shared memory (bulk-group completion).
 __device__ __forceinline__ void tma_store_4d(const CUtensorMap* map, const void* src, int c0, int c1, int c2,
