@@ -63,10 +63,10 @@ constexpr uint32_t T0 = 0, T1 = 128, T2 = 256, TR = 384;
 
 struct Smem {
   uint64_t ld_kv, ld_qd, ld_p, ld_r;  // TMA -> MMA warp / epilogue
-  uint64_t c1, c1b, c2, c3a, c3, c4;  // MMA commits -> epilogue / producer
-  uint64_t e1, e2, e3a, e0;           // epilogue -> MMA warp (256 arrivals each)
-  uint64_t staged;                    // epilogue -> producer: dK, dV staged (256 arrivals)
-  uint64_t scratch_free;              // producer -> epilogue: the dP'/S' pair has been stored out
+  uint64_t c1, c1b, c2, c2b, c3a, c3, c4;  // MMA commits -> epilogue / producer
+  uint64_t e1, e2, e3a, e0;  // epilogue -> MMA warp (256 arrivals each); e2 also -> producer: dQ staged
+  uint64_t staged;           // epilogue -> producer: dK, dV staged (256 arrivals)
+  uint64_t free_a, free_b;   // producer -> epilogue: the previous dK / dV stores have read the buffer
   uint32_t tmem_base;
   int abort;
   float pw[kTile];
@@ -127,9 +127,10 @@ __device__ __forceinline__ Item item_of(int64_t w, int H, int nseg) {
 __global__ void __launch_bounds__(kThreads, 1) bwd_walk_tc(
     const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
     const __grid_constant__ CUtensorMap map_v, const __grid_constant__ CUtensorMap map_do,
-    const __grid_constant__ CUtensorMap map_dk, const __grid_constant__ CUtensorMap map_dv,
+    const __grid_constant__ CUtensorMap map_dq, const __grid_constant__ CUtensorMap map_dk,
+    const __grid_constant__ CUtensorMap map_dv,
     const __grid_constant__ CUtensorMap map_state, const float* decay, const float* __restrict__ P,
-    float* __restrict__ R, __nv_bfloat16* __restrict__ dq, int H, int64_t N, int T, int G, int nseg,
+    float* __restrict__ R, int H, int64_t N, int T, int G, int nseg,
     int64_t nitems) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
@@ -160,6 +161,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_walk_tc(
     mbar_init(&s->c1, 1);
     mbar_init(&s->c1b, 1);
     mbar_init(&s->c2, 1);
+    mbar_init(&s->c2b, 1);
     mbar_init(&s->c3a, 1);
     mbar_init(&s->c3, 1);
     mbar_init(&s->c4, 1);
@@ -168,7 +170,8 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_walk_tc(
     mbar_init(&s->e3a, kEpiThreads);
     mbar_init(&s->e0, kEpiThreads);
     mbar_init(&s->staged, kEpiThreads);
-    mbar_init(&s->scratch_free, 1);
+    mbar_init(&s->free_a, 1);
+    mbar_init(&s->free_b, 1);
     s->abort = 0;
     fence_mbar_init();
   }
@@ -210,11 +213,10 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_walk_tc(
         mbar_arrive_expect_tx(&s->ld_p, kTileBytes);
         bulk_load(sX, src, kTileBytes, &s->ld_p);
       };
-      auto store_dkdv = [&](const Item& it, int row0, uint32_t p) {
-        tma_store_4d(&map_dk, pair(p, 0), 0, it.h, row0, it.b);
-        tma_store_4d(&map_dk, pair(p, 0) + kBox, 64, it.h, row0, it.b);
-        tma_store_4d(&map_dv, pair(p, 1), 0, it.h, row0, it.b);
-        tma_store_4d(&map_dv, pair(p, 1) + kBox, 64, it.h, row0, it.b);
+      // one bulk group per tensor, so that the dK buffer frees up first
+      auto store_tile = [&](const CUtensorMap* map, const uint8_t* src, const Item& it, int row0) {
+        tma_store_4d(map, src, 0, it.h, row0, it.b);
+        tma_store_4d(map, src + kBox, 64, it.h, row0, it.b);
         tma_store_commit();
       };
 
@@ -237,7 +239,10 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_walk_tc(
           // once they have been read, that pair is this chunk's dP'/S' pair
           if (it > 0) {
             if (!(ok = mbar_wait_or_abort(&s->staged, (it - 1) & 1u, SITE_BWD_TMA, abort_flag))) break;
-            store_dkdv(prev, prev_row, par ^ 1u);
+            store_tile(&map_dk, pair(par ^ 1u, 0), prev, prev_row);
+            store_tile(&map_dv, pair(par ^ 1u, 1), prev, prev_row);
+            tma_store_wait_read1();
+            mbar_arrive(&s->free_a);
           }
           tma_store_wait_read0();
           if (t == tiles - 1) {
@@ -250,7 +255,8 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_walk_tc(
             for (int bx = 0; bx < 4; ++bx)
               tma_load_2d(pair(par ^ 1u, bx >> 1) + (bx & 1) * kBox, &map_state, &s->ld_r, 32 * bx, y);
           }
-          mbar_arrive(&s->scratch_free);
+          if (it == 0) mbar_arrive(&s->free_a);
+          mbar_arrive(&s->free_b);
 
           // the next chunk of this CTA's stream
           Item nx = item;
@@ -286,7 +292,11 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_walk_tc(
           }
           // dP' and S' have been read once the first part of MMA 3 is done: the
           // next Q and dO go into their pair; K, V and X are free after all of MMA 3
+          // dQ, staged over S' (which MMA 2 has read), goes out
+          if (!(ok = mbar_wait_or_abort(&s->e2, par, SITE_BWD_TMA, abort_flag))) break;
+          store_tile(&map_dq, pair(par ^ 1u, 1), item, row0);
           if (!(ok = mbar_wait_or_abort(&s->c3a, par, SITE_BWD_MMA, abort_flag))) break;
+          tma_store_wait_read0();  // dQ has left the S' buffer
           if (has_next) load_qd(nx, nt, par ^ 1u);
           if (!(ok = mbar_wait_or_abort(&s->c3, par, SITE_BWD_MMA, abort_flag))) break;
           if (has_next) {
@@ -297,8 +307,10 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_walk_tc(
           prev_row = row0;
         }
       }
-      if (ok && it > 0 && mbar_wait_or_abort(&s->staged, (it - 1) & 1u, SITE_BWD_TMA, abort_flag))
-        store_dkdv(prev, prev_row, (it - 1) & 1u);
+      if (ok && it > 0 && mbar_wait_or_abort(&s->staged, (it - 1) & 1u, SITE_BWD_TMA, abort_flag)) {
+        store_tile(&map_dk, pair((it - 1) & 1u, 0), prev, prev_row);
+        store_tile(&map_dv, pair((it - 1) & 1u, 1), prev, prev_row);
+      }
       if (!ok) s->abort = 1;
       tma_store_wait0();
     }
@@ -335,6 +347,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_walk_tc(
           for (int kk = 0; kk < kTile / 16; ++kk) mma_bf16(tmem + T0, kmaj(aA, kk), mnmaj(aK, kk), id_kn, kk != 0);
           mma_commit(&s->c2);
           for (int kk = 0; kk < kTile / 16; ++kk) mma_bf16(tmem + T1, mnmaj(aB, kk), mnmaj(aD, kk), id_nn, kk != 0);
+          mma_commit(&s->c2b);
           // ---- MMA 3: T0 = dP'^T Q | T0 += V~ R^T, T2 = K R
           if (!(ok = mbar_wait_or_abort(&s->e2, par, SITE_BWD_MMA, abort_flag))) break;
           tc_fence_after();
@@ -380,7 +393,6 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_walk_tc(
 
       for (int t = tiles - 1; t >= 0; --t, ++it) {
         const uint32_t par = it & 1u;
-        const int row0 = item.seg * G + t * kTile;
         uint8_t* sQ = pair(par, 0);       // Q, then dK out
         uint8_t* sD = pair(par, 1);       // dO, then dV out
         uint8_t* sA = pair(par ^ 1u, 0);  // dP'
@@ -413,9 +425,14 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_walk_tc(
           ++nseg_done;
           named_sync(kEpiBar, kEpiThreads);  // all of R is read before the pair is rewritten
         }
-        wait(&s->scratch_free, par, SITE_BWD_TMA);  // the previous dK/dV stores have read the pair
+        // V~ = diag(lambda^{127-j}) V once MMA 1 has read V
         wait(&s->c1, par, SITE_BWD_MMA);
         tc_fence_after();
+        if (scale) scale_rows(sV, s->pw, true, 1.f, tid);
+        // dP' = Mask . T0 and S' = Mask . T1 into the buffers the previous
+        // chunk's dK and dV stores have left
+        wait(&s->free_a, par, SITE_BWD_TMA);
+        wait(&s->free_b, par, SITE_BWD_TMA);
 #pragma unroll 1
         for (int cc = 2 * half; cc < 2 * half + 2; ++cc) {
           uint32_t rp[32], rs[32];
@@ -433,7 +450,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_walk_tc(
           st_row32_bf16(sA, i, cc * 32, fp);
           st_row32_bf16(sB, i, cc * 32, fs);
         }
-        // R of this chunk -> bf16 X (once dO P^T has read P) and pre-scaled by lambda^128 for MMA 4
+        // R of this chunk -> bf16 X (once dO P^T has read P), pre-scaled by lambda^128 for MMA 4
         wait(&s->c1b, par, SITE_BWD_MMA);
         tc_fence_after();
         {
@@ -454,38 +471,39 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_walk_tc(
             }
           }
         }
-        if (scale) {
-          tmem_st_wait();
-          scale_rows(sV, s->pw, true, 1.f, tid);  // V~ = diag(lambda^{127-j}) V
-        }
+        tmem_st_wait();
         fence_async_smem();
         tc_fence_before();
         mbar_arrive(&s->e1);
 
-        // ---- epilogue 2: dQ = T0 + lambda^{i+1} T2
+        // ---- epilogue 2: dQ = T0 + lambda^{i+1} T2, staged over S' once
+        // S'^T dO has read it (the TMA warp stores it)
         wait(&s->c2, par, SITE_BWD_MMA);
         tc_fence_after();
         {
           const float wi = decay_pow(l2, (float)(i + 1));
-          __nv_bfloat16* out = dq + (((int64_t)item.b * N + row0 + i) * H + item.h) * kD;
-#pragma unroll 1
-          for (int cc = 2 * half; cc < 2 * half + 2; ++cc) {
+          uint32_t pq[2][16];
+#pragma unroll
+          for (int c2 = 0; c2 < 2; ++c2) {
             uint32_t ra[32], re[32];
-            tmem_ld32(lane_base + T0 + cc * 32, ra);
-            tmem_ld32(lane_base + T2 + cc * 32, re);
+            tmem_ld32(lane_base + T0 + (2 * half + c2) * 32, ra);
+            tmem_ld32(lane_base + T2 + (2 * half + c2) * 32, re);
             tmem_ld_wait();
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              float o[8];
-#pragma unroll
-              for (int u = 0; u < 8; ++u)
-                o[u] = fmaf(wi, __uint_as_float(re[q * 8 + u]), __uint_as_float(ra[q * 8 + u]));
-              *reinterpret_cast<uint4*>(out + cc * 32 + q * 8) = make_uint4(
-                  pack_bf16(o[0], o[1]), pack_bf16(o[2], o[3]), pack_bf16(o[4], o[5]), pack_bf16(o[6], o[7]));
-            }
+            for (int q = 0; q < 16; ++q)
+              pq[c2][q] = pack_bf16(fmaf(wi, __uint_as_float(re[2 * q]), __uint_as_float(ra[2 * q])),
+                                    fmaf(wi, __uint_as_float(re[2 * q + 1]), __uint_as_float(ra[2 * q + 1])));
           }
+          tc_fence_before();
+          wait(&s->c2b, par, SITE_BWD_MMA);
+#pragma unroll
+          for (int c2 = 0; c2 < 2; ++c2)
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+              st_tile16(sB, i, (2 * half + c2) * 32 + q * 8,
+                        make_uint4(pq[c2][4 * q], pq[c2][4 * q + 1], pq[c2][4 * q + 2], pq[c2][4 * q + 3]));
         }
-        tc_fence_before();
+        fence_async_smem();
         mbar_arrive(&s->e2);
 
         // ---- epilogue 3a: Q~ = diag(lambda^{j+1}) Q once dP'^T Q has read Q
@@ -552,10 +570,11 @@ cudaError_t tc_bwd_walk(const void* q, const void* k, const void* v, const void*
                         const float* P, float* R, void* dq, void* dk, void* dv, int B, int H, int64_t N, int d, int C,
                         int G, int num_sms, cudaStream_t st) {
   using namespace tc_bwd_walk_detail;
-  CUtensorMap mq, mk, mv, mdo, mdk, mdv, mr;
+  CUtensorMap mq, mk, mv, mdo, mdq, mdk, mdv, mr;
   if (!make_token_map(&mq, q, B, H, N, d, kTile) || !make_token_map(&mk, k, B, H, N, d, kTile) ||
       !make_token_map(&mv, v, B, H, N, d, kTile) || !make_token_map(&mdo, dout, B, H, N, d, kTile) ||
-      !make_token_map(&mdk, dk, B, H, N, d, kTile) || !make_token_map(&mdv, dv, B, H, N, d, kTile) ||
+      !make_token_map(&mdq, dq, B, H, N, d, kTile) || !make_token_map(&mdk, dk, B, H, N, d, kTile) ||
+      !make_token_map(&mdv, dv, B, H, N, d, kTile) ||
       !make_state_map(&mr, R, (int64_t)B * (N / C) * H, d))
     return cudaErrorInvalidValue;
   const size_t smem = 1024 + 7 * (size_t)kTileBytes + sizeof(Smem);
@@ -564,8 +583,8 @@ cudaError_t tc_bwd_walk(const void* q, const void* k, const void* v, const void*
   const int nseg = (int)(N / G);
   const int64_t nitems = (int64_t)B * H * nseg;
   const unsigned grid = (unsigned)std::min<int64_t>(nitems, num_sms);
-  bwd_walk_tc<<<grid, kThreads, smem, st>>>(mq, mk, mv, mdo, mdk, mdv, mr, decay, P, R, (__nv_bfloat16*)dq, H, N,
-                                            (int)(N / C), G, nseg, nitems);
+  bwd_walk_tc<<<grid, kThreads, smem, st>>>(mq, mk, mv, mdo, mdq, mdk, mdv, mr, decay, P, R, H, N, (int)(N / C), G,
+                                            nseg, nitems);
   return cudaGetLastError();
 }
 
