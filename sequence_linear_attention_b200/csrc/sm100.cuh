@@ -43,9 +43,9 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 
 // Waits for the phase with the given parity to complete. Gives up after the
 // per-device wait limit, records LASP_ERR_TIMEOUT with `site` and returns
-// false; the caller then skips the rest of its work and exits.
-__device__ __noinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, unsigned int site) {
-  if (mbar_try_wait(bar, parity)) return true;
+// false; the caller then skips the rest of its work and exits. The first probe
+// is inline; only a wait that has to spin leaves the caller.
+__device__ __noinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parity, unsigned int site) {
   const unsigned long long t0 = globaltimer_ns();
   const unsigned long long limit = g_wait_limit_ns;
   for (uint32_t it = 1;; ++it) {
@@ -56,12 +56,14 @@ __device__ __noinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, unsigned 
     }
   }
 }
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, unsigned int site) {
+  return mbar_try_wait(bar, parity) || mbar_wait_slow(bar, parity, site);
+}
 
 // As mbar_wait, but also gives up, without recording anything, once *abort
-// is set by another thread of the CTA (checked on the slow path only).
-__device__ __noinline__ bool mbar_wait_or_abort(uint64_t* bar, uint32_t parity, unsigned int site,
-                                                const volatile int* abort) {
-  if (mbar_try_wait(bar, parity)) return true;
+// is set by another thread of the CTA (checked while spinning).
+__device__ __noinline__ bool mbar_wait_or_abort_slow(uint64_t* bar, uint32_t parity, unsigned int site,
+                                                     const volatile int* abort) {
   const unsigned long long t0 = globaltimer_ns();
   const unsigned long long limit = g_wait_limit_ns;
   for (uint32_t it = 1;; ++it) {
@@ -74,6 +76,10 @@ __device__ __noinline__ bool mbar_wait_or_abort(uint64_t* bar, uint32_t parity, 
       }
     }
   }
+}
+__device__ __forceinline__ bool mbar_wait_or_abort(uint64_t* bar, uint32_t parity, unsigned int site,
+                                                   const volatile int* abort) {
+  return mbar_try_wait(bar, parity) || mbar_wait_or_abort_slow(bar, parity, site, abort);
 }
 
 // Named barrier `id` over the first `nthreads` threads (whole warps) of the CTA.
