@@ -7,33 +7,32 @@
 // Before this kernel, the segment gradient states and an exclusive suffix
 // over them put, in the R slot of each segment's last chunk, the gradient
 // state entering that chunk from the tokens after the segment. One persistent
-// CTA (256 threads) takes segments in turn and walks their chunks backward,
-// holding R (fp32) in TMEM; P of each chunk comes from the forward walk's
-// cache as a ready bf16 operand tile. Per chunk c (LASP Eq. 14-23):
+// CTA per SM takes segments in turn and walks their chunks backward, holding R
+// (fp32) in TMEM; P of each chunk comes from the forward walk's cache as a
+// ready bf16 operand tile. Per chunk c (LASP Eq. 14-23), with the MMAs issued
+// by one warp and the epilogues run by eight others:
 //
-//   MMA 1:  T0 = dO V^T,  T1 = Q K^T  | then T2 = dO P^T
-//   epi 1:  dP' = Mask . T0 -> A,  S' = Mask . T1 -> B;  (T2 done:)
-//           R -> bf16 X (replacing P),  R <- lambda^128 R in TMEM;
-//           V <- diag(lambda^{127-j}) V in place
-//   MMA 2:  T0 = dP' K                 | then T1 = S'^T dO
-//   epi 2:  dQ = T0 + lambda^{i+1} T2 -> global
-//   MMA 3:  T0 = dP'^T Q               | then T0 += V~ R^T (dK), T2 = K R
-//   epi 3:  Q <- diag(lambda^{j+1}) Q;  then dK = T0,
-//           dV = T1 + lambda^{127-j} T2 -> over Q~ and dO (TMA stores)
-//   MMA 4:  R += Q~^T dO          (the state for chunk c - 1)
+//   MMA 1:  T0 = dO V^T,  T1 = Q K^T  | T2 = dO P^T
+//   epi 1:  V <- diag(lambda^{127-j}) V;  dP' = Mask . T0 -> A,  S' = Mask . T1 -> B
+//   MMA 2:  T0 = dP' K                 | T1 = S'^T dO
+//   epi 2:  (under MMA 2) R -> bf16 X (replacing P), R <- lambda^128 R in TMEM;
+//           dQ = T0 + lambda^{i+1} T2 -> over S' (TMA store)
+//   MMA 3:  T0 = dP'^T Q + V~ R^T (dK),  T2 = K R
+//   epi 3:  (under MMA 3) dO <- diag(lambda^{j+1}) dO;
+//   MMA 4:  R += Q^T dO~               (the state for chunk c - 1)
+//   epi 3:  dK = T0, dV = T1 + lambda^{127-j} T2 -> over Q and dO~ (TMA stores)
 //
-// Each epilogue waits only for the MMAs before the bar; those after it run
-// under the epilogue.
+// A bar marks a commit the epilogue can start on while the rest runs.
 //
 // The decay of the dK inter term rides on the bf16 operand V~ so both dK terms
 // share an accumulator (TMEM has no fifth block); the dQ and dV inter terms
 // keep fp32 row scalings. Two pairs of tile buffers trade roles from chunk to
 // chunk: one holds the chunk's Q and dO and then its outgoing dK and dV, the
-// other its dP' and S' and then the next chunk's Q and dO, which are loaded as
-// soon as the first part of MMA 3 has read dP'. The next K, V and P follow once
-// all of MMA 3 is done. R is not stored per chunk: only the segment-level slots
-// of the workspace are used. In every epilogue warp w owns TMEM lanes (rows)
-// 32*(w%4).. and the column half w/4.
+// other its dP' and S' (and dQ) and then the next chunk's Q and dO, which are
+// loaded as soon as dQ has left and dP'^T Q is done. The next K, V and P follow
+// once all of MMA 3 is done. R is not stored per chunk: only the segment-level
+// slots of the workspace are used. In every epilogue warp w owns TMEM lanes
+// (rows) 32*(w%4).. and the column half w/4.
 #include <algorithm>
 
 #include "kernels.h"
@@ -235,7 +234,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_walk_tc(
         for (int t = tiles - 1; t >= 0 && ok; --t, ++it) {
           const uint32_t par = it & 1u;
           const int row0 = item.seg * G + t * kTile;
-          // the previous chunk's dK and dV, staged over its Q~ and dO, go out;
+          // the previous chunk's dK and dV, staged over its Q and dO~, go out;
           // once they have been read, that pair is this chunk's dP'/S' pair
           if (it > 0) {
             if (!(ok = mbar_wait_or_abort(&s->staged, (it - 1) & 1u, SITE_BWD_TMA, abort_flag))) break;
@@ -356,7 +355,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_walk_tc(
           for (int kk = 0; kk < kD / 16; ++kk) mma_bf16(tmem + T0, kmaj(aV, kk), kmaj(aX, kk), id_kk, 1);
           for (int kk = 0; kk < kD / 16; ++kk) mma_bf16(tmem + T2, kmaj(aK, kk), mnmaj(aX, kk), id_kn, kk != 0);
           mma_commit(&s->c3);
-          // ---- MMA 4: R += Q~^T dO (TMEM R was pre-scaled by lambda^128 in epilogue 1)
+          // ---- MMA 4: R += Q^T dO~ (TMEM R was pre-scaled by lambda^128 in epilogue 1)
           if (!(ok = mbar_wait_or_abort(&s->e3a, par, SITE_BWD_MMA, abort_flag))) break;
           tc_fence_after();
           for (int kk = 0; kk < kTile / 16; ++kk) mma_bf16(tmem + TR, mnmaj(aQ, kk), mnmaj(aD, kk), id_nn, 1);
@@ -435,22 +434,45 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_walk_tc(
         wait(&s->free_b, par, SITE_BWD_TMA);
 #pragma unroll 1
         for (int cc = 2 * half; cc < 2 * half + 2; ++cc) {
+          if (cc > (warp & 3)) {
+            // the 32 x 32 block lies above the diagonal of this warp's rows
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              st_tile16(sA, i, cc * 32 + q * 8, make_uint4(0u, 0u, 0u, 0u));
+              st_tile16(sB, i, cc * 32 + q * 8, make_uint4(0u, 0u, 0u, 0u));
+            }
+            continue;
+          }
           uint32_t rp[32], rs[32];
           tmem_ld32(lane_base + T0 + cc * 32, rp);
           tmem_ld32(lane_base + T1 + cc * 32, rs);
           tmem_ld_wait();
           float fp[32], fs[32];
+          if (cc < (warp & 3)) {  // below the diagonal: every j < i
 #pragma unroll
-          for (int q = 0; q < 32; ++q) {
-            const int j = cc * 32 + q;
-            const float wgt = j <= i ? s->pw[i - j] : 0.f;
-            fp[q] = __uint_as_float(rp[q]) * wgt;
-            fs[q] = __uint_as_float(rs[q]) * wgt;
+            for (int q = 0; q < 32; ++q) {
+              const float wgt = s->pw[i - cc * 32 - q];
+              fp[q] = __uint_as_float(rp[q]) * wgt;
+              fs[q] = __uint_as_float(rs[q]) * wgt;
+            }
+          } else {
+#pragma unroll
+            for (int q = 0; q < 32; ++q) {
+              const int j = cc * 32 + q;
+              const float wgt = j <= i ? s->pw[i - j] : 0.f;
+              fp[q] = __uint_as_float(rp[q]) * wgt;
+              fs[q] = __uint_as_float(rs[q]) * wgt;
+            }
           }
           st_row32_bf16(sA, i, cc * 32, fp);
           st_row32_bf16(sB, i, cc * 32, fs);
         }
-        // R of this chunk -> bf16 X (once dO P^T has read P), pre-scaled by lambda^128 for MMA 4
+        fence_async_smem();
+        tc_fence_before();
+        mbar_arrive(&s->e1);
+
+        // R of this chunk -> bf16 X (once dO P^T has read P), pre-scaled by
+        // lambda^128 for MMA 4, while MMA 2 runs
         wait(&s->c1b, par, SITE_BWD_MMA);
         tc_fence_after();
         {
@@ -472,9 +494,6 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_walk_tc(
           }
         }
         tmem_st_wait();
-        fence_async_smem();
-        tc_fence_before();
-        mbar_arrive(&s->e1);
 
         // ---- epilogue 2: dQ = T0 + lambda^{i+1} T2, staged over S' once
         // S'^T dO has read it (the TMA warp stores it)
@@ -504,18 +523,18 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_walk_tc(
                         make_uint4(pq[c2][4 * q], pq[c2][4 * q + 1], pq[c2][4 * q + 2], pq[c2][4 * q + 3]));
         }
         fence_async_smem();
+        tc_fence_before();
         mbar_arrive(&s->e2);
 
-        // ---- epilogue 3a: Q~ = diag(lambda^{j+1}) Q once dP'^T Q has read Q
-        wait(&s->c3a, par, SITE_BWD_MMA);
+        // ---- epilogue 3a: dO~ = diag(lambda^{j+1}) dO (S'^T dO has read dO), while MMA 3 runs
         if (scale) {
-          scale_rows(sQ, s->pw, false, lam, tid);  // lambda^{j+1} = pw[j] * lambda
+          scale_rows(sD, s->pw, false, lam, tid);  // lambda^{j+1} = pw[j] * lambda
           fence_async_smem();
         }
         mbar_arrive(&s->e3a);
 
         // ---- epilogue 3b: dK = T0, dV = T1 + lambda^{127-j} T2, staged over
-        // Q~ and dO once MMA 4 has read them
+        // Q and dO~ once MMA 4 has read them
         wait(&s->c3, par, SITE_BWD_MMA);
         tc_fence_after();
         {
