@@ -8,14 +8,15 @@
 // or the largest of 64/32/16 dividing C); the stages of all of a CTA's chunks
 // form one stream through up to six shared-memory slots (192 KB). Per stage:
 // warp 1 brings A and B by TMA (KB rows x 128 features, two 64-feature boxes
-// each, 128-byte swizzle); when lambda != 1 the four worker warps scale the
-// rows of A by w_t in place (bf16); warp 0 issues KB/16 tcgen05.mma (M = N =
-// 128 features, K = 16 tokens) accumulating M_c in TMEM. Both operands are
-// MN-major: the tiles arrive token-major with features contiguous, which is
-// exactly A^T and B with the reduced (token) index as the slow one. Two TMEM
-// accumulators alternate between chunks; the workers read a finished one
-// (warp w: TMEM lanes 32*(w%4)..) and write the state row by row while the
-// next chunk accumulates.
+// each, 128-byte swizzle); when lambda != 1 the eight worker warps scale the
+// rows of A by w_t in place (bf16, one thread per 128-byte row); warp 0 issues
+// KB/16 tcgen05.mma (M = N = 128 features, K = 16 tokens) accumulating M_c in
+// TMEM. Both operands are MN-major: the tiles arrive token-major with features
+// contiguous, which is exactly A^T and B with the reduced (token) index as the
+// slow one. Two TMEM accumulators alternate between chunks; the workers read a
+// finished one (warp w: TMEM lanes 32*(w%4).., one column half) and store it by
+// TMA in 32 x 32 blocks staged in shared memory, while the next chunk
+// accumulates.
 #include <algorithm>
 
 #include "kernels.h"
@@ -30,8 +31,9 @@ namespace tc_states_detail {
 using namespace sm100;
 
 constexpr int kD = 128;              // head dimension handled here
-constexpr int kThreads = 192;        // warp 0: MMA, warp 1: TMA, warps 2-5: scaling and epilogue
-constexpr int kWorkers = 128;
+constexpr int kThreads = 320;        // warp 0: MMA, warp 1: TMA, warps 2-9: scaling and epilogue
+constexpr int kWorkers = 256;
+constexpr uint32_t kStageOutBytes = 32 * 128;  // per worker warp: a 32 x 32 fp32 block of the state
 constexpr int kMaxSlots = 6;
 constexpr size_t kStageBudget = 192 * 1024;  // shared memory for the stage slots
 constexpr uint32_t kTmemCols = 256;  // two 128 x 128 fp32 accumulators
@@ -77,7 +79,8 @@ __device__ __forceinline__ Work work_of(int64_t n, int T, int H) {
 // other one. Hand-offs are mbarriers; no CTA-wide barrier in the stream.
 __global__ void __launch_bounds__(kThreads, 1) chunk_states_tc(const __grid_constant__ CUtensorMap map_a,
                                                             const __grid_constant__ CUtensorMap map_b,
-                                                            const float* decay, float* __restrict__ M, int H,
+                                                            const __grid_constant__ CUtensorMap map_m,
+                                                            const float* decay, int H,
                                                             int C, int KB, int nslots, int kind, int T,
                                                             int64_t nitems, int64_t t_out, int slot_stride,
                                                             int slot_offset) {
@@ -86,7 +89,8 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_states_tc(const __grid_cons
   uint8_t* tiles = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   const int nstages = C / KB;
   const uint32_t tile_bytes = (uint32_t)KB * 256;  // KB rows x 128 features x bf16
-  Smem* s = reinterpret_cast<Smem*>(tiles + nslots * 2 * tile_bytes);
+  uint8_t* out_stage = tiles + nslots * 2 * tile_bytes;  // kStageOutBytes per worker warp
+  Smem* s = reinterpret_cast<Smem*>(out_stage + (kWorkers / 32) * kStageOutBytes);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int64_t my_items = nitems > blockIdx.x ? (nitems - 1 - blockIdx.x) / gridDim.x + 1 : 0;
@@ -95,6 +99,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_states_tc(const __grid_cons
   if (tid == 0) {
     prefetch_tmap(&map_a);
     prefetch_tmap(&map_b);
+    prefetch_tmap(&map_m);
     for (int q = 0; q < kMaxSlots; ++q) {
       mbar_init(&s->full[q], 1);
       mbar_init(&s->scaled[q], kWorkers);
@@ -168,10 +173,11 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_states_tc(const __grid_cons
       }
     }
   } else {
-    // ------------------------------------------------- workers (warps 2-5)
-    const int wt = tid - 64;             // 0..127
-    const int quad = warp & 3;           // the TMEM lanes this warp may read
-    const int row = quad * 32 + lane;    // accumulator row read by this thread
+    // ------------------------------------------------- workers (warps 2-9)
+    const int wt = tid - 64;              // 0..255
+    const int quad = warp & 3;            // the TMEM lanes this warp may read
+    const int colhalf = (warp - 2) >> 2;  // and the half of the columns it writes out
+    uint8_t* stage_out = out_stage + (warp - 2) * kStageOutBytes;
     Work wk{0, 0, 0};
     float lam = 1.f, l2 = 0.f;
     for (int64_t g = 0; g < nstream; ++g) {
@@ -189,26 +195,33 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_states_tc(const __grid_cons
         break;
       }
       if (lam != 1.0f) {
-        // scale row r of A by w_{k*KB + r}; the row of a 16-byte chunk is its
-        // byte offset / 128 in either 64-feature box, whatever the swizzle
-        uint4* a = reinterpret_cast<uint4*>(tiles + (size_t)slot * 2 * tile_bytes);
-        const int nchunks = KB * 16;
-        for (int q = wt; q < nchunks; q += kWorkers) {
-          const int r = (q % (KB * 8)) / 8;
+        // scale row r of A by w_{k*KB + r}: one thread per row of a 64-feature
+        // box (8 chunks of 16 bytes, chunk c of row r stored at position
+        // c ^ (r & 7), so the eight rows of a quarter-warp hit different banks)
+        uint8_t* a = tiles + (size_t)slot * 2 * tile_bytes;
+        for (int q = wt; q < 2 * KB; q += kWorkers) {
+          const int r = q % KB;
           const int t = k * KB + r;
           const float w = kind == 0 ? decay_pow(l2, (float)(C - 1 - t)) : decay_pow(l2, (float)(t + 1));
-          uint4 x = a[q];
-          x.x = bf16x2_scale(x.x, w);
-          x.y = bf16x2_scale(x.y, w);
-          x.z = bf16x2_scale(x.z, w);
-          x.w = bf16x2_scale(x.w, w);
-          a[q] = x;
+          uint8_t* line = a + (q / KB) * (tile_bytes / 2) + r * 128;
+          uint4 x[8];
+#pragma unroll
+          for (int c = 0; c < 8; ++c) x[c] = *reinterpret_cast<const uint4*>(line + ((c ^ (r & 7)) << 4));
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            x[c].x = bf16x2_scale(x[c].x, w);
+            x[c].y = bf16x2_scale(x[c].y, w);
+            x[c].z = bf16x2_scale(x[c].z, w);
+            x[c].w = bf16x2_scale(x[c].w, w);
+            *reinterpret_cast<uint4*>(line + ((c ^ (r & 7)) << 4)) = x[c];
+          }
         }
         fence_async_smem();
       }
       mbar_arrive(&s->scaled[slot]);
       if (k == nstages - 1) {
-        // the chunk's state: accumulator n & 1 -> slot c * slot_stride + slot_offset
+        // the chunk's state: accumulator n & 1 -> slot c * slot_stride + slot_offset,
+        // as 32 x 32 blocks staged in shared memory and stored by TMA
         const int acc = (int)(n & 1);
         if (!mbar_wait(&s->acc_full[acc], (uint32_t)((n >> 1) & 1), SITE_STATES_MMA)) {
           s->abort = 1;
@@ -216,28 +229,35 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_states_tc(const __grid_cons
         }
         tc_fence_after();
         const int64_t oslot = (int64_t)wk.c * slot_stride + slot_offset;
-        float* out = M + ((((int64_t)wk.b * t_out + oslot) * H + wk.h) * kD + row) * kD;
+        const int y = (int)((((int64_t)wk.b * t_out + oslot) * H + wk.h) * kD + quad * 32);
         const uint32_t tbase = tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)acc * 128;
-#pragma unroll 1
-        for (int cc = 0; cc < kD / 32; cc += 2) {
-          uint32_t r0[32], r1[32];
-          tmem_ld32(tbase + cc * 32, r0);
-          tmem_ld32(tbase + (cc + 1) * 32, r1);
-          tmem_ld_wait();
-          float4* o0 = reinterpret_cast<float4*>(out + cc * 32);
-          float4* o1 = reinterpret_cast<float4*>(out + (cc + 1) * 32);
-#pragma unroll
-          for (int q = 0; q < 8; ++q) {
-            __stcs(o0 + q, make_float4(__uint_as_float(r0[4 * q]), __uint_as_float(r0[4 * q + 1]),
-                                       __uint_as_float(r0[4 * q + 2]), __uint_as_float(r0[4 * q + 3])));
-            __stcs(o1 + q, make_float4(__uint_as_float(r1[4 * q]), __uint_as_float(r1[4 * q + 1]),
-                                       __uint_as_float(r1[4 * q + 2]), __uint_as_float(r1[4 * q + 3])));
-          }
-        }
+        uint32_t r0[32], r1[32];
+        tmem_ld32(tbase + (2 * colhalf) * 32, r0);
+        tmem_ld32(tbase + (2 * colhalf + 1) * 32, r1);
+        tmem_ld_wait();
         tc_fence_before();
         mbar_arrive(&s->acc_empty[acc]);
+#pragma unroll
+        for (int cb = 0; cb < 2; ++cb) {
+          // the staging block is free once this warp's previous store has read it
+          if (lane == 0) tma_store_wait_read0();
+          __syncwarp();
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            const uint32_t* v = cb == 0 ? r0 + 4 * c : r1 + 4 * c;
+            *reinterpret_cast<uint4*>(stage_out + lane * 128 + ((c ^ (lane & 7)) << 4)) =
+                make_uint4(v[0], v[1], v[2], v[3]);
+          }
+          fence_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_2d(&map_m, stage_out, (2 * colhalf + cb) * 32, y);
+            tma_store_commit();
+          }
+        }
       }
     }
+    if (lane == 0) tma_store_wait0();
   }
   tc_fence_before();
   __syncthreads();
@@ -262,11 +282,12 @@ cudaError_t tc_chunk_states_slots(const void* a, const void* bm, const float* de
                                   cudaStream_t st) {
   using namespace tc_states_detail;
   const int KB = stage_rows(C);
-  CUtensorMap ma, mb;
-  if (!make_token_map(&ma, a, B, H, N, d, KB) || !make_token_map(&mb, bm, B, H, N, d, KB))
+  CUtensorMap ma, mb, mm;
+  if (!make_token_map(&ma, a, B, H, N, d, KB) || !make_token_map(&mb, bm, B, H, N, d, KB) ||
+      !make_state_map(&mm, M, (int64_t)B * t_out * H, d, 32))
     return cudaErrorInvalidValue;
   const int nslots = (int)std::min<size_t>(kMaxSlots, kStageBudget / ((size_t)2 * KB * 256));
-  const size_t smem = 1024 + (size_t)nslots * 2 * KB * 256 + sizeof(Smem);
+  const size_t smem = 1024 + (size_t)nslots * 2 * KB * 256 + (kWorkers / 32) * kStageOutBytes + sizeof(Smem);
   cudaError_t e = cudaFuncSetAttribute(chunk_states_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   int dev = 0, sms = 148;
@@ -274,7 +295,7 @@ cudaError_t tc_chunk_states_slots(const void* a, const void* bm, const float* de
   const int T = (int)(N / C);
   const int64_t nitems = (int64_t)B * H * T;
   const unsigned grid = (unsigned)std::min<int64_t>(nitems, sms);
-  chunk_states_tc<<<grid, kThreads, smem, st>>>(ma, mb, decay, M, H, C, KB, nslots, kind, T, nitems, t_out,
+  chunk_states_tc<<<grid, kThreads, smem, st>>>(ma, mb, mm, decay, H, C, KB, nslots, kind, T, nitems, t_out,
                                                slot_stride, slot_offset);
   return cudaGetLastError();
 }

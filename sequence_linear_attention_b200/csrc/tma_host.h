@@ -43,15 +43,16 @@ inline bool make_token_map(CUtensorMap* map, const void* base, int B, int H, int
 }
 
 // A 2-D view (d, rows) of an fp32 state array [..., d, d] (rows = number of
-// states x d); one box is 32 columns x 128 rows, stored in shared memory as 128
-// lines of 128 bytes with the 128-byte swizzle, so a d = 128 state is 4 boxes.
-inline bool make_state_map(CUtensorMap* map, const float* base, int64_t nstates, int d) {
+// states x d); one box is 32 columns x box_rows rows, stored in shared memory
+// as lines of 128 bytes with the 128-byte swizzle (a d = 128 state is 4 boxes
+// of 128 rows).
+inline bool make_state_map(CUtensorMap* map, const float* base, int64_t nstates, int d, int box_rows = 128) {
   auto fn = tmap_encode_fn();
   const int64_t rows = nstates * d;
   if (fn == nullptr || rows <= 0 || rows > (int64_t)INT32_MAX) return false;
   cuuint64_t dims[2] = {(cuuint64_t)d, (cuuint64_t)rows};
   cuuint64_t strides[1] = {(cuuint64_t)d * 4};
-  cuuint32_t box[2] = {32, 128};
+  cuuint32_t box[2] = {32, (cuuint32_t)box_rows};
   cuuint32_t estr[2] = {1, 1};
   CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float*>(base), dims, strides, box, estr,
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
