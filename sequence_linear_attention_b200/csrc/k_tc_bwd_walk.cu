@@ -17,7 +17,7 @@
 //   MMA 2:  T0 = dP' K                 | T1 = S'^T dO
 //   epi 2:  (under MMA 2) R -> bf16 X (replacing P), R <- lambda^128 R in TMEM;
 //           dQ = T0 + lambda^{i+1} T2 -> over S' (TMA store)
-//   MMA 3:  T0 = dP'^T Q + V~ R^T (dK),  T2 = K R
+//   MMA 3:  T0 = V~ R^T,  T2 = K R    | T0 += dP'^T Q (dK)
 //   epi 3:  (under MMA 3) dO <- diag(lambda^{j+1}) dO;
 //   MMA 4:  R += Q^T dO~               (the state for chunk c - 1)
 //   epi 3:  dK = T0, dV = T1 + lambda^{127-j} T2 -> over Q and dO~ (TMA stores)
@@ -29,8 +29,8 @@
 // keep fp32 row scalings. Two pairs of tile buffers trade roles from chunk to
 // chunk: one holds the chunk's Q and dO and then its outgoing dK and dV, the
 // other its dP' and S' (and dQ) and then the next chunk's Q and dO, which are
-// loaded as soon as dQ has left and dP'^T Q is done. The next K, V and P follow
-// once all of MMA 3 is done. R is not stored per chunk: only the segment-level
+// loaded as soon as dQ has left and dP'^T Q is done. The next K, V and P go
+// in once the first part of MMA 3 is done. R is not stored per chunk: only the segment-level
 // slots of the workspace are used. In every epilogue warp w owns TMEM lanes
 // (rows) 32*(w%4).. and the column half w/4.
 #include <algorithm>
@@ -289,19 +289,20 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_walk_tc(
             const int64_t slot = (int64_t)ns.seg * tiles + tiles - 1;
             bulk_prefetch_l2(R + (((int64_t)ns.b * T + slot) * H + ns.h) * kD * kD, kD * kD * sizeof(float));
           }
-          // dP' and S' have been read once the first part of MMA 3 is done: the
-          // next Q and dO go into their pair; K, V and X are free after all of MMA 3
           // dQ, staged over S' (which MMA 2 has read), goes out
           if (!(ok = mbar_wait_or_abort(&s->e2, par, SITE_BWD_TMA, abort_flag))) break;
           store_tile(&map_dq, pair(par ^ 1u, 1), item, row0);
+          // K, V and X are free once the first part of MMA 3 is done; the next
+          // Q and dO go into the dP'/S' pair once dP'^T Q has read dP' and dQ
+          // has left
           if (!(ok = mbar_wait_or_abort(&s->c3a, par, SITE_BWD_MMA, abort_flag))) break;
-          tma_store_wait_read0();  // dQ has left the S' buffer
-          if (has_next) load_qd(nx, nt, par ^ 1u);
-          if (!(ok = mbar_wait_or_abort(&s->c3, par, SITE_BWD_MMA, abort_flag))) break;
           if (has_next) {
             load_kv(nx, nt);
             load_p(nx, nt);
           }
+          if (!(ok = mbar_wait_or_abort(&s->c3, par, SITE_BWD_MMA, abort_flag))) break;
+          tma_store_wait_read0();
+          if (has_next) load_qd(nx, nt, par ^ 1u);
           prev = item;
           prev_row = row0;
         }
@@ -347,13 +348,13 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_walk_tc(
           mma_commit(&s->c2);
           for (int kk = 0; kk < kTile / 16; ++kk) mma_bf16(tmem + T1, mnmaj(aB, kk), mnmaj(aD, kk), id_nn, kk != 0);
           mma_commit(&s->c2b);
-          // ---- MMA 3: T0 = dP'^T Q | T0 += V~ R^T, T2 = K R
+          // ---- MMA 3: T0 = V~ R^T, T2 = K R | T0 += dP'^T Q
           if (!(ok = mbar_wait_or_abort(&s->e2, par, SITE_BWD_MMA, abort_flag))) break;
           tc_fence_after();
-          for (int kk = 0; kk < kTile / 16; ++kk) mma_bf16(tmem + T0, mnmaj(aA, kk), mnmaj(aQ, kk), id_nn, kk != 0);
-          mma_commit(&s->c3a);
-          for (int kk = 0; kk < kD / 16; ++kk) mma_bf16(tmem + T0, kmaj(aV, kk), kmaj(aX, kk), id_kk, 1);
+          for (int kk = 0; kk < kD / 16; ++kk) mma_bf16(tmem + T0, kmaj(aV, kk), kmaj(aX, kk), id_kk, kk != 0);
           for (int kk = 0; kk < kD / 16; ++kk) mma_bf16(tmem + T2, kmaj(aK, kk), mnmaj(aX, kk), id_kn, kk != 0);
+          mma_commit(&s->c3a);
+          for (int kk = 0; kk < kTile / 16; ++kk) mma_bf16(tmem + T0, mnmaj(aA, kk), mnmaj(aQ, kk), id_nn, 1);
           mma_commit(&s->c3);
           // ---- MMA 4: R += Q^T dO~ (TMEM R was pre-scaled by lambda^128 in epilogue 1)
           if (!(ok = mbar_wait_or_abort(&s->e3a, par, SITE_BWD_MMA, abort_flag))) break;
