@@ -77,12 +77,14 @@ def flops_per_step(tokens_heads: int, d: int, C: int) -> float:
 # each kernel on this workload, from the ncu capture summarised in profiles/,
 # valid only while the kernel's sources hash to the recorded value.
 MEASURED_TRAFFIC = {
-    "bwd_walk_tc": (["k_tc_bwd_walk.cu", "sm100.cuh", "lasp_common.cuh", "tma_host.h"], "1c16835f9af55e30",
-                    1426244000 + 766284800),
-    "fwd_walk_tc": (["k_tc_fwd_walk.cu", "sm100.cuh", "lasp_common.cuh", "tma_host.h"], "85d238bbe4d332a9",
-                    890644000 + 499181056),
-    "segment_states_tc": (["k_tc_states.cu", "sm100.cuh", "lasp_common.cuh", "tma_host.h"], "76a7468029954420",
-                          537818000 + 53428992),
+    # DRAM bytes per launch at the workload's full size: twice the ncu capture of
+    # the 32768-token case of the same workload (traffic grows with the tokens)
+    "bwd_walk_tc": (["k_tc_bwd_walk.cu", "sm100.cuh", "lasp_common.cuh", "tma_host.h"], "1cf301c58e7839f6",
+                    2 * (723450880 + 368640768)),
+    "fwd_walk_tc": (["k_tc_fwd_walk.cu", "sm100.cuh", "lasp_common.cuh", "tma_host.h"], "458f7f6b3a9f51b1",
+                    2 * (436959744 + 231108352)),
+    "segment_states_tc": (["k_tc_states.cu", "sm100.cuh", "lasp_common.cuh", "tma_host.h"], "0124abcfbf954d17",
+                          2 * (268475136 + 22717184)),
 }
 
 
@@ -214,6 +216,10 @@ def run_gpu(args, rank, world, local):
     dev = torch.device("cuda", local)
     w = lasp_inputs.WORKLOADS[args.workload]
     B, N, H, d, C = w["B"], w["N"], w["H"], w["d"], w["C"]
+    if args.tokens is not None:
+        if args.tokens <= 0 or args.tokens % C:
+            raise ValueError(f"--tokens must be a positive multiple of C = {C}")
+        N = args.tokens
     bf16 = w["bf16"]
     tdtype = torch.bfloat16 if bf16 else torch.float32
     elem = 2 if bf16 else 4
@@ -322,7 +328,7 @@ def run_gpu(args, rank, world, local):
         "tensor_peak_frac": round(tflops / peaks["bf16_sustained"], 4),
         "roofline": {"bound": "hbm", "kernel": top, "achieved": round(achieved, 1), "peak": peaks["hbm"],
                      "unit": "GB/s", "frac": round(achieved / peaks["hbm"], 4),
-                     "traffic": measured_traffic(top, args.workload),
+                     "traffic": measured_traffic(top, args.workload) if args.tokens is None else None,
                      "algorithmic_bytes": algorithmic_bytes(top, th, d, C, G, elem),
                      "peak_source": peaks["source"]},
         "kernels": kernel_table,
@@ -400,6 +406,9 @@ def main(argv=None):
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(lasp_inputs.WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--tokens", type=int, default=None,
+                    help="sequence length N instead of the workload's (a smaller case of the same shape, for "
+                         "profiling); the line is then not the workload's headline number")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
