@@ -47,7 +47,7 @@ constexpr uint32_t TS = 0, TI = 128, TO = 256, TP = 384;
 
 struct Smem {
   uint64_t load[2];
-  uint64_t mma1, mma2;
+  uint64_t mma1, mma2a, mma2;
   uint64_t ld_state;
   uint32_t tmem_base;
   int abort;
@@ -118,6 +118,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_walk_tc(const __grid_constant
     mbar_init(&s->load[0], 1);
     mbar_init(&s->load[1], 1);
     mbar_init(&s->mma1, 1);
+    mbar_init(&s->mma2a, 1);
     mbar_init(&s->mma2, 1);
     mbar_init(&s->ld_state, 1);
     s->abort = 0;
@@ -147,7 +148,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_walk_tc(const __grid_constant
   };
 
   // the fp32 state entering a segment (the slot of its first chunk) as four
-  // 32-column boxes: boxes 0, 1 into the Q buffer of `set`, boxes 2, 3 into its
+  // 32-column boxes: boxes 0, 1 into the K buffer of `set`, boxes 2, 3 into its
   // V buffer, both free at that point
   auto issue_state_load = [&](int set, const Item& it) {
     const int64_t slot = ((int64_t)it.seg * G) / C;
@@ -155,7 +156,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_walk_tc(const __grid_constant
     mbar_arrive_expect_tx(&s->ld_state, kD * kD * 4);
 #pragma unroll
     for (int bx = 0; bx < 4; ++bx)
-      tma_load_2d(bufQ(set) + (bx >> 1) * 2 * kTileBytes + (bx & 1) * kBox, &map_state, &s->ld_state, 32 * bx, y);
+      tma_load_2d(bufQ(set) + (1 + (bx >> 1)) * kTileBytes + (bx & 1) * kBox, &map_state, &s->ld_state, 32 * bx, y);
   };
 
   // thread 32 issues every TMA load and bulk copy (and waits for the stores it
@@ -188,7 +189,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_walk_tc(const __grid_constant
     // of a swizzled box has its 16-byte chunk c at position c ^ (i & 7), so the
     // eight rows of a quarter-warp read different banks.
     if (mbar_wait(&s->ld_state, nseg_done & 1u, SITE_OUT_TMA)) {
-      const uint8_t* src = bufQ((it & 1) ^ 1) + half * 2 * kTileBytes;
+      const uint8_t* src = bufQ((it & 1) ^ 1) + (1 + half) * kTileBytes;
       float v[64];
 #pragma unroll
       for (int bb = 0; bb < 2; ++bb)
@@ -270,46 +271,69 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_walk_tc(const __grid_constant
         }
       }
 
-      // ---- epilogue A
+      // ---- epilogue A1: S' = Mask . S into the Q buffer (Q has been read by
+      // both MMAs); the 32 x 32 blocks above the diagonal are zeros
       if (mbar_wait(&s->mma1, it & 1u, SITE_OUT_MMA)) {
         tc_fence_after();
-        // S' = Mask . S into the Q buffer (Q has been read by both MMAs); both
-        // TMEM loads are in flight before the one wait
-        {
-          uint32_t r0[32], r1[32];
-          tmem_ld32(lane_base + TS + (2 * half) * 32, r0);
-          tmem_ld32(lane_base + TS + (2 * half + 1) * 32, r1);
+#pragma unroll 1
+        for (int cc = 2 * half; cc < 2 * half + 2; ++cc) {
+          if (cc > (warp & 3)) {
+#pragma unroll
+            for (int q = 0; q < 4; ++q) st_tile16(sQ, i, cc * 32 + q * 8, make_uint4(0u, 0u, 0u, 0u));
+            continue;
+          }
+          uint32_t r[32];
+          tmem_ld32(lane_base + TS + cc * 32, r);
           tmem_ld_wait();
           float w32[32];
+          if (cc < (warp & 3)) {
 #pragma unroll
-          for (int q = 0; q < 32; ++q) {
-            const int j = 2 * half * 32 + q;
-            w32[q] = j <= i ? __uint_as_float(r0[q]) * s->pw[i - j] : 0.f;
-          }
-          st_row32_bf16(sQ, i, 2 * half * 32, w32);
+            for (int q = 0; q < 32; ++q) w32[q] = __uint_as_float(r[q]) * s->pw[i - cc * 32 - q];
+          } else {
 #pragma unroll
-          for (int q = 0; q < 32; ++q) {
-            const int j = (2 * half + 1) * 32 + q;
-            w32[q] = j <= i ? __uint_as_float(r1[q]) * s->pw[i - j] : 0.f;
+            for (int q = 0; q < 32; ++q) {
+              const int j = cc * 32 + q;
+              w32[q] = j <= i ? __uint_as_float(r[q]) * s->pw[i - j] : 0.f;
+            }
           }
-          st_row32_bf16(sQ, i, (2 * half + 1) * 32, w32);
+          st_row32_bf16(sQ, i, cc * 32, w32);
         }
-        // K~ = diag(lambda^{127-j}) K, in place (K has been read by the S MMA)
-        if (scale) {
-          uint4* k4 = reinterpret_cast<uint4*>(sK);
+        fence_async_smem();
+      } else {
+        s->abort = 1;
+      }
+      tc_fence_before();
+      __syncthreads();
+      if (s->abort) {
+        stop = true;
+        break;
+      }
+      // ---- MMA 2a: O_intra = S' V (runs under epilogue A2)
+      if (tid == 0) {
+        tc_fence_after();
+        const uint32_t aS = smem_u32(sQ), aV = smem_u32(sV);
+        for (int kk = 0; kk < kTile / 16; ++kk) mma_bf16(tmem + TO, kmaj(aS, kk), mnmaj(aV, kk), id_kn, kk != 0);
+        mma_commit(&s->mma2a);
+      }
+
+      // ---- epilogue A2: K~ = diag(lambda^{127-j}) K in place (K has been read
+      // by the S MMA); the state entering this tile into the cache at chunk
+      // starts (C > 128), then pre-scaled by lambda^128
+      if (scale) {
+        uint4* k4 = reinterpret_cast<uint4*>(sK);
 #pragma unroll 2
-          for (int g = tid; g < kTile * 16; g += kThreads) {
-            const int r = (g & (kTile * 8 - 1)) >> 3;  // row of this 16-byte chunk in its box
-            const float wk = s->pw[kTile - 1 - r];
-            uint4 x = k4[g];
-            x.x = scale_bf16x2(x.x, wk);
-            x.y = scale_bf16x2(x.y, wk);
-            x.z = scale_bf16x2(x.z, wk);
-            x.w = scale_bf16x2(x.w, wk);
-            k4[g] = x;
-          }
+        for (int g = tid; g < kTile * 16; g += kThreads) {
+          const int r = (g & (kTile * 8 - 1)) >> 3;  // row of this 16-byte chunk in its box
+          const float wk = s->pw[kTile - 1 - r];
+          uint4 x = k4[g];
+          x.x = scale_bf16x2(x.x, wk);
+          x.y = scale_bf16x2(x.y, wk);
+          x.z = scale_bf16x2(x.z, wk);
+          x.w = scale_bf16x2(x.w, wk);
+          k4[g] = x;
         }
-        // the state entering this tile: into the cache at chunk starts, then pre-scaled by lambda^128
+      }
+      {
         const bool write_cache = !cache_bf16 && t > 0 && (t * kTile) % C == 0;
         if (write_cache || scale) {
           float* dst = P + ((((int64_t)item.b * T + row0 / C) * H + item.h) * kD + i) * kD + half * 64;
@@ -334,68 +358,62 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_walk_tc(const __grid_constant
           }
           tmem_st_wait();
         }
-        fence_async_smem();
-      } else {
-        s->abort = 1;
       }
+      fence_async_smem();
       if (tid == kProducer && cache_bf16) tma_store_wait_read0();  // epilogue B rewrites sP
       tc_fence_before();
       __syncthreads();
-      if (s->abort) {
-        stop = true;
-        break;
-      }
-
-      // ---- MMA 2: O_intra = S' V, P += K~^T V
+      // ---- MMA 2b: P += K~^T V (runs under epilogue B1)
       if (tid == 0) {
         tc_fence_after();
-        const uint32_t aS = smem_u32(sQ), aK = smem_u32(sK), aV = smem_u32(sV);
-        for (int kk = 0; kk < kTile / 16; ++kk) mma_bf16(tmem + TO, kmaj(aS, kk), mnmaj(aV, kk), id_kn, kk != 0);
+        const uint32_t aK = smem_u32(sK), aV = smem_u32(sV);
         for (int kk = 0; kk < kTile / 16; ++kk) mma_bf16(tmem + TP, mnmaj(aK, kk), mnmaj(aV, kk), id_nn, 1);
         mma_commit(&s->mma2);
       }
 
-      // ---- epilogue B
-      if (mbar_wait(&s->mma2, it & 1u, SITE_OUT_MMA)) {
+      // ---- epilogue B1: O = O_intra + lambda^{i+1} O_inter -> bf16 over S'
+      // (which MMA 2a has read), for the TMA store
+      if (mbar_wait(&s->mma2a, it & 1u, SITE_OUT_MMA)) {
         tc_fence_after();
-        // MMA 2 has read this set's Q (S') and V buffers: the next segment's
-        // entering state goes there
-        if (tid == kProducer && t == tiles - 1 && w + gridDim.x < nitems)
-          issue_state_load(set, item_of(w + gridDim.x, H, nseg));
         const float wi = decay_pow(l2, (float)(i + 1));
-        {
-          // O = O_intra + lambda^{i+1} O_inter, both column chunks' loads in flight together
-          uint32_t a0[32], e0[32], a1[32], e1[32];
-          tmem_ld32(lane_base + TO + (2 * half) * 32, a0);
-          tmem_ld32(lane_base + TI + (2 * half) * 32, e0);
-          tmem_ld32(lane_base + TO + (2 * half + 1) * 32, a1);
-          tmem_ld32(lane_base + TI + (2 * half + 1) * 32, e1);
-          tmem_ld_wait();
-          float o[32];
+        uint32_t a0[32], e0[32], a1[32], e1[32];
+        tmem_ld32(lane_base + TO + (2 * half) * 32, a0);
+        tmem_ld32(lane_base + TI + (2 * half) * 32, e0);
+        tmem_ld32(lane_base + TO + (2 * half + 1) * 32, a1);
+        tmem_ld32(lane_base + TI + (2 * half + 1) * 32, e1);
+        tmem_ld_wait();
+        float o[32];
 #pragma unroll
-          for (int q = 0; q < 32; ++q) o[q] = fmaf(wi, __uint_as_float(e0[q]), __uint_as_float(a0[q]));
-          st_row32_bf16(sK, i, 2 * half * 32, o);  // output staging over K~
+        for (int q = 0; q < 32; ++q) o[q] = fmaf(wi, __uint_as_float(e0[q]), __uint_as_float(a0[q]));
+        st_row32_bf16(sQ, i, 2 * half * 32, o);
 #pragma unroll
-          for (int q = 0; q < 32; ++q) o[q] = fmaf(wi, __uint_as_float(e1[q]), __uint_as_float(a1[q]));
-          st_row32_bf16(sK, i, (2 * half + 1) * 32, o);
-        }
-        {
-          uint32_t r0[32], r1[32];
-          tmem_ld32(lane_base + TP + (2 * half) * 32, r0);
-          tmem_ld32(lane_base + TP + (2 * half + 1) * 32, r1);
-          tmem_ld_wait();
-          float p[32];
-#pragma unroll
-          for (int q = 0; q < 32; ++q) p[q] = __uint_as_float(r0[q]);
-          st_row32_bf16(sP, i, 2 * half * 32, p);
-#pragma unroll
-          for (int q = 0; q < 32; ++q) p[q] = __uint_as_float(r1[q]);
-          st_row32_bf16(sP, i, (2 * half + 1) * 32, p);
-        }
-        fence_async_smem();
+        for (int q = 0; q < 32; ++q) o[q] = fmaf(wi, __uint_as_float(e1[q]), __uint_as_float(a1[q]));
+        st_row32_bf16(sQ, i, (2 * half + 1) * 32, o);
       } else {
         s->abort = 1;
       }
+      // ---- epilogue B2: P -> bf16 operand for the next tile
+      if (mbar_wait(&s->mma2, it & 1u, SITE_OUT_MMA)) {
+        tc_fence_after();
+        // MMA 2b has read this set's K~ and V buffers: the next segment's
+        // entering state goes there
+        if (tid == kProducer && t == tiles - 1 && w + gridDim.x < nitems)
+          issue_state_load(set, item_of(w + gridDim.x, H, nseg));
+        uint32_t r0[32], r1[32];
+        tmem_ld32(lane_base + TP + (2 * half) * 32, r0);
+        tmem_ld32(lane_base + TP + (2 * half + 1) * 32, r1);
+        tmem_ld_wait();
+        float p[32];
+#pragma unroll
+        for (int q = 0; q < 32; ++q) p[q] = __uint_as_float(r0[q]);
+        st_row32_bf16(sP, i, 2 * half * 32, p);
+#pragma unroll
+        for (int q = 0; q < 32; ++q) p[q] = __uint_as_float(r1[q]);
+        st_row32_bf16(sP, i, (2 * half + 1) * 32, p);
+      } else {
+        s->abort = 1;
+      }
+      fence_async_smem();
       tc_fence_before();
       __syncthreads();
       if (s->abort) {
@@ -403,8 +421,8 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_walk_tc(const __grid_constant
         break;
       }
       if (tid == kProducer) {
-        tma_store_4d(&map_o, sK, 0, item.h, row0, item.b);
-        tma_store_4d(&map_o, sK + kBox, 64, item.h, row0, item.b);
+        tma_store_4d(&map_o, sQ, 0, item.h, row0, item.b);
+        tma_store_4d(&map_o, sQ + kBox, 64, item.h, row0, item.b);
         tma_store_commit();
       }
     }
