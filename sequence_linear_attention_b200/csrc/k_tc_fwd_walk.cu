@@ -8,22 +8,28 @@
 // The sequence is cut into segments of G tokens (a multiple of C and of the
 // 128-token tile). Before this kernel, the segment states and an exclusive
 // prefix over them put P of each segment's first chunk into the state cache.
-// Here one persistent CTA (256 threads) takes segments in turn and walks their
-// 128-token tiles in order, holding the state P (fp32) in TMEM:
+// Here one persistent CTA per SM takes segments in turn and walks their
+// 128-token tiles in order, holding the state P (fp32) in TMEM. One warp issues
+// the MMAs, one the TMA loads and stores, eight run the epilogues; they hand
+// work to each other through mbarriers. Per tile:
 //
-//   MMA 1:  S = Q K^T (TMEM S),  O_inter = Q P_bf16 (TMEM I)
-//   epi A:  S' = Mask . S -> bf16 over Q;  K~ = diag(lambda^{127-j}) K in place;
-//           P <- lambda^128 P in TMEM (and, for C > 128, P -> fp32 cache at chunk starts)
-//   MMA 2:  O_intra = S' V (TMEM O);  P += K~^T V (TMEM P)
-//   epi B:  O = O_intra + lambda^{i+1} O_inter -> bf16 over K~ -> TMA store;
-//           P -> bf16 operand for the next tile
+//   MMA 1:  S = Q K^T (TMEM S)  | O_inter = Q P_bf16 (TMEM I)
+//   epi A1: S' = Mask . S -> bf16 over Q (once both parts of MMA 1 have read Q)
+//   MMA 2a: O_intra = S' V (TMEM O), under
+//   epi A2: K~ = diag(lambda^{127-j}) K in place; P <- lambda^128 P in TMEM (and,
+//           for C > 128, P -> fp32 cache at chunk starts)
+//   MMA 2b: P += K~^T V (TMEM P), under
+//   epi B1: O = O_intra + lambda^{i+1} O_inter -> bf16 over S' -> TMA store
+//   epi B2: P -> bf16 operand for the next tile
 //
 // With C = 128 each tile starts a chunk, and the bf16 operand tile of the
 // entering state (already in shared memory for O_inter) goes to the chunk's
 // cache slot by one bulk copy; the backward walk loads it back as is. Two sets
 // of Q/K/V buffers alternate: while a tile is computed, the next tile's loads
-// (possibly of the next segment) are in flight. In every epilogue
-// warp w owns TMEM lanes (rows) 32*(w%4).. and the column half w/4.
+// (possibly of the next segment) are in flight; a segment's fp32 entering state
+// is loaded by TMA into the K and V buffers of the set the previous tile used.
+// In every epilogue warp w owns TMEM lanes (rows) 32*(w%4).. and the column
+// half w/4.
 #include <algorithm>
 
 #include "kernels.h"
@@ -39,16 +45,24 @@ using namespace sm100;
 
 constexpr int kD = 128;
 constexpr int kTile = 128;
-constexpr int kThreads = 256;
+// warps 0-7 run the epilogues (warp w owns TMEM lanes 32*(w%4).. and column
+// half w/4), warp 8 issues the MMAs, warp 9 the TMA loads and stores
+constexpr int kEpiThreads = 256;
+constexpr int kMmaWarp = 8;
+constexpr int kProducerWarp = 9;
+constexpr int kThreads = 320;
+constexpr uint32_t kEpiBar = 1;  // named barrier of the epilogue warps
 constexpr uint32_t kTileBytes = kTile * kD * 2;
 constexpr uint32_t kBox = kTileBytes / 2;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t TS = 0, TI = 128, TO = 256, TP = 384;
 
 struct Smem {
-  uint64_t load[2];
-  uint64_t mma1, mma2a, mma2;
-  uint64_t ld_state;
+  uint64_t load[2], ld_state;            // TMA -> MMA warp / epilogue
+  uint64_t mma1a, mma1, mma2a, mma2[2];  // MMA commits -> epilogue / producer (mma2 per buffer set)
+  uint64_t e_a1, e_a2, e_b1[2], e_b2;    // epilogue -> MMA warp / producer (256 arrivals; e_b1 per set)
+  uint64_t state_read;                   // epilogue -> producer: the entering state has been read
+  uint64_t sp_free;                      // producer -> epilogue: P's operand tile is in the cache
   uint32_t tmem_base;
   int abort;
   float pw[kTile];
@@ -104,10 +118,9 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_walk_tc(const __grid_constant
   uint8_t* sP = base + 6 * kTileBytes;
   Smem* s = reinterpret_cast<Smem*>(base + 7 * kTileBytes);
   auto bufQ = [&](int set) { return base + set * 3 * kTileBytes; };
+  const volatile int* abort_flag = &s->abort;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int i = (warp & 3) * 32 + lane;  // the row this thread owns in every epilogue
-  const int half = warp >> 2;            // and the column half
   const int tiles = G / kTile;
 
   if (tid == 0) {
@@ -115,12 +128,22 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_walk_tc(const __grid_constant
     prefetch_tmap(&map_k);
     prefetch_tmap(&map_v);
     prefetch_tmap(&map_o);
+    prefetch_tmap(&map_state);
     mbar_init(&s->load[0], 1);
     mbar_init(&s->load[1], 1);
+    mbar_init(&s->ld_state, 1);
+    mbar_init(&s->mma1a, 1);
     mbar_init(&s->mma1, 1);
     mbar_init(&s->mma2a, 1);
-    mbar_init(&s->mma2, 1);
-    mbar_init(&s->ld_state, 1);
+    mbar_init(&s->mma2[0], 1);
+    mbar_init(&s->mma2[1], 1);
+    mbar_init(&s->e_a1, kEpiThreads);
+    mbar_init(&s->e_a2, kEpiThreads);
+    mbar_init(&s->e_b1[0], kEpiThreads);
+    mbar_init(&s->e_b1[1], kEpiThreads);
+    mbar_init(&s->e_b2, kEpiThreads);
+    mbar_init(&s->state_read, kEpiThreads);
+    mbar_init(&s->sp_free, 1);
     s->abort = 0;
     fence_mbar_init();
   }
@@ -132,304 +155,361 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_walk_tc(const __grid_constant
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = s->tmem_base;
-  const uint32_t lane_base = tmem + ((uint32_t)((warp & 3) * 32) << 16);
 
-  // loads of one tile (Q, K, V: two 64-feature boxes each) into buffer set `set`
-  auto issue_loads = [&](int set, const Item& it, int t) {
-    uint8_t* q = bufQ(set);
-    const int row = it.seg * G + t * kTile;
-    mbar_arrive_expect_tx(&s->load[set], 3 * kTileBytes);
-    tma_load_4d(q, &map_q, &s->load[set], 0, it.h, row, it.b);
-    tma_load_4d(q + kBox, &map_q, &s->load[set], 64, it.h, row, it.b);
-    tma_load_4d(q + kTileBytes, &map_k, &s->load[set], 0, it.h, row, it.b);
-    tma_load_4d(q + kTileBytes + kBox, &map_k, &s->load[set], 64, it.h, row, it.b);
-    tma_load_4d(q + 2 * kTileBytes, &map_v, &s->load[set], 0, it.h, row, it.b);
-    tma_load_4d(q + 2 * kTileBytes + kBox, &map_v, &s->load[set], 64, it.h, row, it.b);
-  };
-
-  // the fp32 state entering a segment (the slot of its first chunk) as four
-  // 32-column boxes: boxes 0, 1 into the K buffer of `set`, boxes 2, 3 into its
-  // V buffer, both free at that point
-  auto issue_state_load = [&](int set, const Item& it) {
-    const int64_t slot = ((int64_t)it.seg * G) / C;
-    const int y = (int)((((int64_t)it.b * T + slot) * H + it.h) * kD);
-    mbar_arrive_expect_tx(&s->ld_state, kD * kD * 4);
+  if (warp == kProducerWarp) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      // loads of one tile (Q, K, V: two 64-feature boxes each) into buffer set `set`
+      auto issue_loads = [&](int set, const Item& it, int t) {
+        uint8_t* q = bufQ(set);
+        const int row = it.seg * G + t * kTile;
+        mbar_arrive_expect_tx(&s->load[set], 3 * kTileBytes);
+        tma_load_4d(q, &map_q, &s->load[set], 0, it.h, row, it.b);
+        tma_load_4d(q + kBox, &map_q, &s->load[set], 64, it.h, row, it.b);
+        tma_load_4d(q + kTileBytes, &map_k, &s->load[set], 0, it.h, row, it.b);
+        tma_load_4d(q + kTileBytes + kBox, &map_k, &s->load[set], 64, it.h, row, it.b);
+        tma_load_4d(q + 2 * kTileBytes, &map_v, &s->load[set], 0, it.h, row, it.b);
+        tma_load_4d(q + 2 * kTileBytes + kBox, &map_v, &s->load[set], 64, it.h, row, it.b);
+      };
+      // the fp32 state entering a segment (the slot of its first chunk) as four
+      // 32-column boxes: boxes 0, 1 into the K buffer of `set`, boxes 2, 3 into
+      // its V buffer
+      auto issue_state_load = [&](int set, const Item& it) {
+        const int64_t slot = ((int64_t)it.seg * G) / C;
+        const int y = (int)((((int64_t)it.b * T + slot) * H + it.h) * kD);
+        mbar_arrive_expect_tx(&s->ld_state, kD * kD * 4);
 #pragma unroll
-    for (int bx = 0; bx < 4; ++bx)
-      tma_load_2d(bufQ(set) + (1 + (bx >> 1)) * kTileBytes + (bx & 1) * kBox, &map_state, &s->ld_state, 32 * bx, y);
-  };
+        for (int bx = 0; bx < 4; ++bx)
+          tma_load_2d(bufQ(set) + (1 + (bx >> 1)) * kTileBytes + (bx & 1) * kBox, &map_state, &s->ld_state, 32 * bx,
+                      y);
+      };
+      auto store_o = [&](int set, const Item& it, int row0) {
+        tma_store_4d(&map_o, bufQ(set), 0, it.h, row0, it.b);
+        tma_store_4d(&map_o, bufQ(set) + kBox, 64, it.h, row0, it.b);
+        tma_store_commit();
+      };
 
-  // thread 32 issues every TMA load and bulk copy (and waits for the stores it
-  // issued); thread 0 issues the MMAs
-  constexpr int kProducer = 32;
-  if (tid == kProducer && (int64_t)blockIdx.x < nitems) {
-    prefetch_tmap(&map_state);
-    const Item first = item_of(blockIdx.x, H, nseg);
-    issue_loads(0, first, 0);
-    issue_state_load(1, first);
-  }
-
-  constexpr uint32_t id_kk = idesc_bf16(128, 128, 0, 0);
-  constexpr uint32_t id_kn = idesc_bf16(128, 128, 0, 1);
-  constexpr uint32_t id_nn = idesc_bf16(128, 128, 1, 1);
-  uint32_t it = 0;  // tiles processed by this CTA
-  uint32_t nseg_done = 0;  // segments started by this CTA
-  bool stop = false;
-
-  for (int64_t w = blockIdx.x; w < nitems && !stop; w += gridDim.x) {
-    const Item item = item_of(w, H, nseg);
-    const float lam = load_decay(decay, item.h);
-    const float l2 = log2f(lam);
-    const bool scale = lam != 1.0f;
-    const float g_tile = decay_pow(l2, (float)kTile);
-    if (tid < kTile) s->pw[tid] = decay_pow(l2, (float)tid);
-
-    // entering state of the segment, loaded by TMA into the buffer set the
-    // previous tile used (see issue_state_load): TMEM P and bf16 operand. Row i
-    // of a swizzled box has its 16-byte chunk c at position c ^ (i & 7), so the
-    // eight rows of a quarter-warp read different banks.
-    if (mbar_wait(&s->ld_state, nseg_done & 1u, SITE_OUT_TMA)) {
-      const uint8_t* src = bufQ((it & 1) ^ 1) + (1 + half) * kTileBytes;
-      float v[64];
-#pragma unroll
-      for (int bb = 0; bb < 2; ++bb)
-#pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          const float4 x = *reinterpret_cast<const float4*>(src + bb * kBox + sw128_offset(i, c));
-          v[bb * 32 + 4 * c] = x.x;
-          v[bb * 32 + 4 * c + 1] = x.y;
-          v[bb * 32 + 4 * c + 2] = x.z;
-          v[bb * 32 + 4 * c + 3] = x.w;
-        }
-#pragma unroll
-      for (int c2 = 0; c2 < 2; ++c2) {
-        uint32_t r[32];
-#pragma unroll
-        for (int q = 0; q < 32; ++q) r[q] = __float_as_uint(v[c2 * 32 + q]);
-        tmem_st32(lane_base + TP + half * 64 + c2 * 32, r);
-        st_row32_bf16(sP, i, half * 64 + c2 * 32, v + c2 * 32);
+      if ((int64_t)blockIdx.x < nitems) {
+        const Item first = item_of(blockIdx.x, H, nseg);
+        issue_loads(0, first, 0);
+        issue_state_load(1, first);
       }
-      tmem_st_wait();
-      fence_async_smem();
-    } else {
-      s->abort = 1;
+      uint32_t it = 0, nsg = 0;
+      Item prev{0, 0, 0};
+      int prev_row = 0;
+      bool ok = true;
+      for (int64_t w = blockIdx.x; w < nitems && ok; w += gridDim.x) {
+        const Item item = item_of(w, H, nseg);
+        for (int t = 0; t < tiles && ok; ++t, ++it) {
+          const int set = it & 1;
+          const uint32_t par = it & 1u;
+          const int row0 = item.seg * G + t * kTile;
+          // the previous tile's O (staged over its S') goes out; once it has
+          // been read, MMA 2 of that tile is done and (at a segment start) the
+          // entering state has been read, its buffer set takes the next tile
+          // (barriers kept per buffer set never run two phases ahead of a waiter:
+          // their next phase needs the loads this thread issues after the wait)
+          const uint32_t ppar = ((it - 1) >> 1) & 1u;  // phase of the previous tile's set
+          if (it > 0) {
+            if (!(ok = mbar_wait_or_abort(&s->e_b1[set ^ 1], ppar, SITE_OUT_TMA, abort_flag))) break;
+            store_o(set ^ 1, prev, prev_row);
+          }
+          if (t == 0 && !(ok = mbar_wait_or_abort(&s->state_read, nsg & 1u, SITE_OUT_TMA, abort_flag))) break;
+          if (t == 0) ++nsg;
+          Item nx = item;
+          int nt = t + 1;
+          bool has_next = true;
+          if (nt == tiles) {
+            nt = 0;
+            has_next = w + gridDim.x < nitems;
+            if (has_next) nx = item_of(w + gridDim.x, H, nseg);
+          }
+          if (has_next) {
+            if (it > 0 && !(ok = mbar_wait_or_abort(&s->mma2[set ^ 1], ppar, SITE_OUT_MMA, abort_flag))) break;
+            tma_store_wait_read0();
+            issue_loads(set ^ 1, nx, nt);
+          }
+          if (t == (tiles > 1 ? tiles - 2 : 0) && w + gridDim.x < nitems) {
+            // the next segment's entering state, into L2 while this segment's
+            // last tiles run
+            const Item ns = item_of(w + gridDim.x, H, nseg);
+            const int64_t slot = ((int64_t)ns.seg * G) / C;
+            bulk_prefetch_l2(P + (((int64_t)ns.b * T + slot) * H + ns.h) * kD * kD, kD * kD * sizeof(float));
+          }
+          // the bf16 operand tile of the state entering this tile, as it sits in
+          // shared memory, is the cache entry the backward pass loads back
+          if (!(ok = mbar_wait_or_abort(&s->e_b2, par, SITE_OUT_TMA, abort_flag))) break;
+          if (cache_bf16) {
+            uint8_t* slot = reinterpret_cast<uint8_t*>(P + (((int64_t)item.b * T + row0 / C) * H + item.h) * kD * kD);
+            bulk_store(slot, sP, kTileBytes);
+            tma_store_commit();
+            tma_store_wait_read0();
+          }
+          mbar_arrive(&s->sp_free);
+          // at the segment's last tile, once MMA 2 has read K~ and V, the next
+          // segment's entering state goes there
+          if (t == tiles - 1 && w + gridDim.x < nitems) {
+            if (!(ok = mbar_wait_or_abort(&s->mma2[set], (it >> 1) & 1u, SITE_OUT_MMA, abort_flag))) break;
+            issue_state_load(set, item_of(w + gridDim.x, H, nseg));
+          }
+          prev = item;
+          prev_row = row0;
+        }
+      }
+      if (ok && it > 0 && mbar_wait_or_abort(&s->e_b1[(it - 1) & 1], ((it - 1) >> 1) & 1u, SITE_OUT_TMA, abort_flag))
+        store_o((it - 1) & 1, prev, prev_row);
+      if (!ok) s->abort = 1;
+      tma_store_wait0();
     }
-    ++nseg_done;
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    if (s->abort) break;
-
-    for (int t = 0; t < tiles; ++t, ++it) {
-      const int set = it & 1;
-      uint8_t* sQ = bufQ(set);
-      uint8_t* sK = sQ + kTileBytes;
-      uint8_t* sV = sQ + 2 * kTileBytes;
-      const int row0 = item.seg * G + t * kTile;
-
-      if (tid == kProducer) {
-        // prefetch the next tile of this CTA's stream into the other set; its K
-        // buffer is the source of the previous tile's output store
-        Item nx = item;
-        int nt = t + 1;
-        bool has_next = true;
-        if (nt == tiles) {
-          nt = 0;
-          has_next = w + gridDim.x < nitems;
-          if (has_next) nx = item_of(w + gridDim.x, H, nseg);
-        }
-        if (has_next) {
-          tma_store_wait_read0();
-          issue_loads(set ^ 1, nx, nt);
-        }
-        if (t == (tiles > 1 ? tiles - 2 : 0) && w + gridDim.x < nitems) {
-          // the next segment's entering state is read by all threads at the
-          // segment switch; bring it into L2 while this segment's last tiles run
-          const Item ns = item_of(w + gridDim.x, H, nseg);
-          const int64_t slot = ((int64_t)ns.seg * G) / C;
-          const float* src = P + (((int64_t)ns.b * T + slot) * H + ns.h) * kD * kD;
-          bulk_prefetch_l2(src, kD * kD * sizeof(float));
-        }
-        if (cache_bf16) {
-          // the bf16 operand tile of the state entering this chunk, as it sits
-          // in shared memory, is the cache entry the backward pass loads back
-          uint8_t* slot = reinterpret_cast<uint8_t*>(P + (((int64_t)item.b * T + row0 / C) * H + item.h) * kD * kD);
-          bulk_store(slot, sP, kTileBytes);
-          tma_store_commit();
-        }
-      }
-      if (tid == 0) {
-        // MMA 1: S = Q K^T, O_inter = Q P
-        if (mbar_wait(&s->load[set], (it >> 1) & 1u, SITE_OUT_TMA)) {
+  } else if (warp == kMmaWarp) {
+    // ------------------------------------------------------------ MMA issue
+    if (lane == 0) {
+      constexpr uint32_t id_kk = idesc_bf16(128, 128, 0, 0);
+      constexpr uint32_t id_kn = idesc_bf16(128, 128, 0, 1);
+      constexpr uint32_t id_nn = idesc_bf16(128, 128, 1, 1);
+      const uint32_t aP = smem_u32(sP);
+      uint32_t it = 0;
+      bool ok = true;
+      for (int64_t w = blockIdx.x; w < nitems && ok; w += gridDim.x) {
+        for (int t = 0; t < tiles; ++t, ++it) {
+          const int set = it & 1;
+          const uint32_t par = it & 1u;
+          const uint32_t aQ = smem_u32(bufQ(set)), aK = aQ + kTileBytes, aV = aQ + 2 * kTileBytes;
+          // ---- MMA 1a: S = Q K^T (TMEM S was read by the previous epilogue A1)
+          if (!(ok = mbar_wait_or_abort(&s->load[set], (it >> 1) & 1u, SITE_OUT_TMA, abort_flag))) break;
           tc_fence_after();
-          const uint32_t aQ = smem_u32(sQ), aK = smem_u32(sK), aP = smem_u32(sP);
           for (int kk = 0; kk < kD / 16; ++kk) mma_bf16(tmem + TS, kmaj(aQ, kk), kmaj(aK, kk), id_kk, kk != 0);
+          mma_commit(&s->mma1a);
+          // ---- MMA 1b: O_inter = Q P, once P is in shared memory and the
+          // previous epilogue B1 has read TMEM I and O
+          ok = (it == 0 || mbar_wait_or_abort(&s->e_b1[set ^ 1], ((it - 1) >> 1) & 1u, SITE_OUT_MMA, abort_flag)) &&
+               mbar_wait_or_abort(&s->e_b2, par, SITE_OUT_MMA, abort_flag);
+          if (!ok) break;
+          tc_fence_after();
           for (int kk = 0; kk < kD / 16; ++kk) mma_bf16(tmem + TI, kmaj(aQ, kk), mnmaj(aP, kk), id_kn, kk != 0);
           mma_commit(&s->mma1);
-        } else {
-          s->abort = 1;
+          // ---- MMA 2a: O_intra = S' V
+          if (!(ok = mbar_wait_or_abort(&s->e_a1, par, SITE_OUT_MMA, abort_flag))) break;
+          tc_fence_after();
+          for (int kk = 0; kk < kTile / 16; ++kk) mma_bf16(tmem + TO, kmaj(aQ, kk), mnmaj(aV, kk), id_kn, kk != 0);
+          mma_commit(&s->mma2a);
+          // ---- MMA 2b: P += K~^T V (TMEM P pre-scaled by lambda^128 in epilogue A2)
+          if (!(ok = mbar_wait_or_abort(&s->e_a2, par, SITE_OUT_MMA, abort_flag))) break;
+          tc_fence_after();
+          for (int kk = 0; kk < kTile / 16; ++kk) mma_bf16(tmem + TP, mnmaj(aK, kk), mnmaj(aV, kk), id_nn, 1);
+          mma_commit(&s->mma2[set]);
         }
       }
+      if (!ok) s->abort = 1;
+    }
+  } else {
+    // ------------------------------------------------------------ epilogues
+    const int i = (warp & 3) * 32 + lane;  // the row this thread owns
+    const int half = warp >> 2;            // and the column half
+    const uint32_t lane_base = tmem + ((uint32_t)((warp & 3) * 32) << 16);
+    bool bad = false;
+    // a failed wait stops the other roles too; this thread runs on (on
+    // whatever data) to the next point where all epilogue warps agree to stop
+    auto wait = [&](uint64_t* bar, uint32_t parity, unsigned int site) {
+      if (!bad && !mbar_wait_or_abort(bar, parity, site, abort_flag)) {
+        bad = true;
+        s->abort = 1;
+      }
+    };
+    uint32_t it = 0, nsg = 0;
+    for (int64_t w = blockIdx.x; w < nitems; w += gridDim.x) {
+      if (named_sync_or(kEpiBar, kEpiThreads, bad)) break;  // every epilogue thread is past the last segment
+      const Item item = item_of(w, H, nseg);
+      const float lam = load_decay(decay, item.h);
+      const float l2 = log2f(lam);
+      const bool scale = lam != 1.0f;
+      const float g_tile = decay_pow(l2, (float)kTile);
+      if (tid < kTile) s->pw[tid] = decay_pow(l2, (float)tid);
 
-      // ---- epilogue A1: S' = Mask . S into the Q buffer (Q has been read by
-      // both MMAs); the 32 x 32 blocks above the diagonal are zeros
-      if (mbar_wait(&s->mma1, it & 1u, SITE_OUT_MMA)) {
+      // entering state of the segment, loaded by TMA into the K and V buffers
+      // of the set the previous tile used: TMEM P and the bf16 operand. Row i
+      // of a swizzled box has its 16-byte chunk c at position c ^ (i & 7), so
+      // the eight rows of a quarter-warp read different banks.
+      wait(&s->ld_state, nsg & 1u, SITE_OUT_TMA);
+      ++nsg;
+      {
+        const uint8_t* src = bufQ((it & 1) ^ 1) + (1 + half) * kTileBytes;
+        float v[64];
+#pragma unroll
+        for (int bb = 0; bb < 2; ++bb)
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            const float4 x = *reinterpret_cast<const float4*>(src + bb * kBox + sw128_offset(i, c));
+            v[bb * 32 + 4 * c] = x.x;
+            v[bb * 32 + 4 * c + 1] = x.y;
+            v[bb * 32 + 4 * c + 2] = x.z;
+            v[bb * 32 + 4 * c + 3] = x.w;
+          }
         tc_fence_after();
-#pragma unroll 1
-        for (int cc = 2 * half; cc < 2 * half + 2; ++cc) {
+#pragma unroll
+        for (int c2 = 0; c2 < 2; ++c2) {
+          uint32_t r[32];
+#pragma unroll
+          for (int q = 0; q < 32; ++q) r[q] = __float_as_uint(v[c2 * 32 + q]);
+          tmem_st32(lane_base + TP + half * 64 + c2 * 32, r);
+          st_row32_bf16(sP, i, half * 64 + c2 * 32, v + c2 * 32);
+        }
+        tmem_st_wait();
+      }
+      fence_async_smem();
+      tc_fence_before();
+      mbar_arrive(&s->state_read);
+      mbar_arrive(&s->e_b2);  // P of the segment's first tile is in place
+      named_sync(kEpiBar, kEpiThreads);  // the decay table is written
+
+      for (int t = 0; t < tiles; ++t, ++it) {
+        const int set = it & 1;
+        const uint32_t par = it & 1u;
+        uint8_t* sQ = bufQ(set);
+        uint8_t* sK = sQ + kTileBytes;
+
+        // ---- epilogue A1: S' = Mask . S over Q once both MMA 1 parts have read
+        // Q; the 32 x 32 blocks above the diagonal are zeros
+        wait(&s->mma1a, par, SITE_OUT_MMA);
+        tc_fence_after();
+        uint32_t ps[2][16];  // bf16 pairs of S'
+#pragma unroll
+        for (int c2 = 0; c2 < 2; ++c2) {
+          const int cc = 2 * half + c2;
           if (cc > (warp & 3)) {
 #pragma unroll
-            for (int q = 0; q < 4; ++q) st_tile16(sQ, i, cc * 32 + q * 8, make_uint4(0u, 0u, 0u, 0u));
+            for (int q = 0; q < 16; ++q) ps[c2][q] = 0u;
             continue;
           }
           uint32_t r[32];
           tmem_ld32(lane_base + TS + cc * 32, r);
           tmem_ld_wait();
-          float w32[32];
           if (cc < (warp & 3)) {
 #pragma unroll
-            for (int q = 0; q < 32; ++q) w32[q] = __uint_as_float(r[q]) * s->pw[i - cc * 32 - q];
+            for (int q = 0; q < 16; ++q)
+              ps[c2][q] = pack_bf16(__uint_as_float(r[2 * q]) * s->pw[i - cc * 32 - 2 * q],
+                                    __uint_as_float(r[2 * q + 1]) * s->pw[i - cc * 32 - 2 * q - 1]);
           } else {
 #pragma unroll
-            for (int q = 0; q < 32; ++q) {
-              const int j = cc * 32 + q;
-              w32[q] = j <= i ? __uint_as_float(r[q]) * s->pw[i - j] : 0.f;
+            for (int q = 0; q < 16; ++q) {
+              const int j = cc * 32 + 2 * q;
+              ps[c2][q] = pack_bf16(j <= i ? __uint_as_float(r[2 * q]) * s->pw[i - j] : 0.f,
+                                    j + 1 <= i ? __uint_as_float(r[2 * q + 1]) * s->pw[i - j - 1] : 0.f);
             }
           }
-          st_row32_bf16(sQ, i, cc * 32, w32);
+        }
+        tc_fence_before();
+        wait(&s->mma1, par, SITE_OUT_MMA);
+#pragma unroll
+        for (int c2 = 0; c2 < 2; ++c2)
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+            st_tile16(sQ, i, (2 * half + c2) * 32 + q * 8,
+                      make_uint4(ps[c2][4 * q], ps[c2][4 * q + 1], ps[c2][4 * q + 2], ps[c2][4 * q + 3]));
+        fence_async_smem();
+        mbar_arrive(&s->e_a1);
+
+        // ---- epilogue A2 (under MMA 2a): K~ = diag(lambda^{127-j}) K in place;
+        // the state entering this tile into the cache at chunk starts (C > 128),
+        // then pre-scaled by lambda^128
+        if (scale) {
+          uint4* k4 = reinterpret_cast<uint4*>(sK);
+#pragma unroll 2
+          for (int g = tid; g < kTile * 16; g += kEpiThreads) {
+            const int r = (g & (kTile * 8 - 1)) >> 3;  // row of this 16-byte chunk in its box
+            const float wk = s->pw[kTile - 1 - r];
+            uint4 x = k4[g];
+            x.x = scale_bf16x2(x.x, wk);
+            x.y = scale_bf16x2(x.y, wk);
+            x.z = scale_bf16x2(x.z, wk);
+            x.w = scale_bf16x2(x.w, wk);
+            k4[g] = x;
+          }
+        }
+        {
+          const int row0 = item.seg * G + t * kTile;
+          const bool write_cache = !cache_bf16 && t > 0 && (t * kTile) % C == 0;
+          if (write_cache || scale) {
+            float* dst = P + ((((int64_t)item.b * T + row0 / C) * H + item.h) * kD + i) * kD + half * 64;
+            uint32_t r[2][32];
+            tmem_ld32(lane_base + TP + half * 64, r[0]);
+            tmem_ld32(lane_base + TP + half * 64 + 32, r[1]);
+            tmem_ld_wait();
+#pragma unroll
+            for (int c2 = 0; c2 < 2; ++c2) {
+              if (write_cache) {
+                float4* d4 = reinterpret_cast<float4*>(dst + c2 * 32);
+#pragma unroll
+                for (int q = 0; q < 8; ++q)
+                  __stcs(d4 + q, make_float4(__uint_as_float(r[c2][4 * q]), __uint_as_float(r[c2][4 * q + 1]),
+                                             __uint_as_float(r[c2][4 * q + 2]), __uint_as_float(r[c2][4 * q + 3])));
+              }
+              if (scale) {
+#pragma unroll
+                for (int q = 0; q < 32; ++q) r[c2][q] = __float_as_uint(__uint_as_float(r[c2][q]) * g_tile);
+                tmem_st32(lane_base + TP + half * 64 + c2 * 32, r[c2]);
+              }
+            }
+            tmem_st_wait();
+          }
         }
         fence_async_smem();
-      } else {
-        s->abort = 1;
-      }
-      tc_fence_before();
-      __syncthreads();
-      if (s->abort) {
-        stop = true;
-        break;
-      }
-      // ---- MMA 2a: O_intra = S' V (runs under epilogue A2)
-      if (tid == 0) {
-        tc_fence_after();
-        const uint32_t aS = smem_u32(sQ), aV = smem_u32(sV);
-        for (int kk = 0; kk < kTile / 16; ++kk) mma_bf16(tmem + TO, kmaj(aS, kk), mnmaj(aV, kk), id_kn, kk != 0);
-        mma_commit(&s->mma2a);
-      }
+        tc_fence_before();
+        mbar_arrive(&s->e_a2);
 
-      // ---- epilogue A2: K~ = diag(lambda^{127-j}) K in place (K has been read
-      // by the S MMA); the state entering this tile into the cache at chunk
-      // starts (C > 128), then pre-scaled by lambda^128
-      if (scale) {
-        uint4* k4 = reinterpret_cast<uint4*>(sK);
-#pragma unroll 2
-        for (int g = tid; g < kTile * 16; g += kThreads) {
-          const int r = (g & (kTile * 8 - 1)) >> 3;  // row of this 16-byte chunk in its box
-          const float wk = s->pw[kTile - 1 - r];
-          uint4 x = k4[g];
-          x.x = scale_bf16x2(x.x, wk);
-          x.y = scale_bf16x2(x.y, wk);
-          x.z = scale_bf16x2(x.z, wk);
-          x.w = scale_bf16x2(x.w, wk);
-          k4[g] = x;
-        }
-      }
-      {
-        const bool write_cache = !cache_bf16 && t > 0 && (t * kTile) % C == 0;
-        if (write_cache || scale) {
-          float* dst = P + ((((int64_t)item.b * T + row0 / C) * H + item.h) * kD + i) * kD + half * 64;
-          uint32_t r[2][32];
-          tmem_ld32(lane_base + TP + half * 64, r[0]);
-          tmem_ld32(lane_base + TP + half * 64 + 32, r[1]);
+        // ---- epilogue B1 (under MMA 2b): O = O_intra + lambda^{i+1} O_inter ->
+        // bf16 over S' (which MMA 2a has read), stored by the TMA warp
+        wait(&s->mma2a, par, SITE_OUT_MMA);
+        tc_fence_after();
+        {
+          const float wi = decay_pow(l2, (float)(i + 1));
+          uint32_t a0[32], e0[32], a1[32], e1[32];
+          tmem_ld32(lane_base + TO + (2 * half) * 32, a0);
+          tmem_ld32(lane_base + TI + (2 * half) * 32, e0);
+          tmem_ld32(lane_base + TO + (2 * half + 1) * 32, a1);
+          tmem_ld32(lane_base + TI + (2 * half + 1) * 32, e1);
           tmem_ld_wait();
+          float o[32];
 #pragma unroll
-          for (int c2 = 0; c2 < 2; ++c2) {
-            if (write_cache) {
-              float4* d4 = reinterpret_cast<float4*>(dst + c2 * 32);
+          for (int q = 0; q < 32; ++q) o[q] = fmaf(wi, __uint_as_float(e0[q]), __uint_as_float(a0[q]));
+          st_row32_bf16(sQ, i, 2 * half * 32, o);
 #pragma unroll
-              for (int q = 0; q < 8; ++q)
-                __stcs(d4 + q, make_float4(__uint_as_float(r[c2][4 * q]), __uint_as_float(r[c2][4 * q + 1]),
-                                           __uint_as_float(r[c2][4 * q + 2]), __uint_as_float(r[c2][4 * q + 3])));
-            }
-            if (scale) {
-#pragma unroll
-              for (int q = 0; q < 32; ++q) r[c2][q] = __float_as_uint(__uint_as_float(r[c2][q]) * g_tile);
-              tmem_st32(lane_base + TP + half * 64 + c2 * 32, r[c2]);
-            }
-          }
-          tmem_st_wait();
+          for (int q = 0; q < 32; ++q) o[q] = fmaf(wi, __uint_as_float(e1[q]), __uint_as_float(a1[q]));
+          st_row32_bf16(sQ, i, (2 * half + 1) * 32, o);
         }
-      }
-      fence_async_smem();
-      if (tid == kProducer && cache_bf16) tma_store_wait_read0();  // epilogue B rewrites sP
-      tc_fence_before();
-      __syncthreads();
-      // ---- MMA 2b: P += K~^T V (runs under epilogue B1)
-      if (tid == 0) {
-        tc_fence_after();
-        const uint32_t aK = smem_u32(sK), aV = smem_u32(sV);
-        for (int kk = 0; kk < kTile / 16; ++kk) mma_bf16(tmem + TP, mnmaj(aK, kk), mnmaj(aV, kk), id_nn, 1);
-        mma_commit(&s->mma2);
-      }
+        fence_async_smem();
+        tc_fence_before();
+        mbar_arrive(&s->e_b1[set]);
 
-      // ---- epilogue B1: O = O_intra + lambda^{i+1} O_inter -> bf16 over S'
-      // (which MMA 2a has read), for the TMA store
-      if (mbar_wait(&s->mma2a, it & 1u, SITE_OUT_MMA)) {
+        // ---- epilogue B2: P -> bf16 operand for the next tile (the segment's
+        // last tile leaves that to the next segment's entering state)
+        wait(&s->mma2[set], (it >> 1) & 1u, SITE_OUT_MMA);
         tc_fence_after();
-        const float wi = decay_pow(l2, (float)(i + 1));
-        uint32_t a0[32], e0[32], a1[32], e1[32];
-        tmem_ld32(lane_base + TO + (2 * half) * 32, a0);
-        tmem_ld32(lane_base + TI + (2 * half) * 32, e0);
-        tmem_ld32(lane_base + TO + (2 * half + 1) * 32, a1);
-        tmem_ld32(lane_base + TI + (2 * half + 1) * 32, e1);
-        tmem_ld_wait();
-        float o[32];
+        wait(&s->sp_free, par, SITE_OUT_TMA);  // this tile's P has been copied to the cache
+        if (t < tiles - 1) {
+          uint32_t r0[32], r1[32];
+          tmem_ld32(lane_base + TP + (2 * half) * 32, r0);
+          tmem_ld32(lane_base + TP + (2 * half + 1) * 32, r1);
+          tmem_ld_wait();
+          float p[32];
 #pragma unroll
-        for (int q = 0; q < 32; ++q) o[q] = fmaf(wi, __uint_as_float(e0[q]), __uint_as_float(a0[q]));
-        st_row32_bf16(sQ, i, 2 * half * 32, o);
+          for (int q = 0; q < 32; ++q) p[q] = __uint_as_float(r0[q]);
+          st_row32_bf16(sP, i, 2 * half * 32, p);
 #pragma unroll
-        for (int q = 0; q < 32; ++q) o[q] = fmaf(wi, __uint_as_float(e1[q]), __uint_as_float(a1[q]));
-        st_row32_bf16(sQ, i, (2 * half + 1) * 32, o);
-      } else {
-        s->abort = 1;
-      }
-      // ---- epilogue B2: P -> bf16 operand for the next tile
-      if (mbar_wait(&s->mma2, it & 1u, SITE_OUT_MMA)) {
-        tc_fence_after();
-        // MMA 2b has read this set's K~ and V buffers: the next segment's
-        // entering state goes there
-        if (tid == kProducer && t == tiles - 1 && w + gridDim.x < nitems)
-          issue_state_load(set, item_of(w + gridDim.x, H, nseg));
-        uint32_t r0[32], r1[32];
-        tmem_ld32(lane_base + TP + (2 * half) * 32, r0);
-        tmem_ld32(lane_base + TP + (2 * half + 1) * 32, r1);
-        tmem_ld_wait();
-        float p[32];
-#pragma unroll
-        for (int q = 0; q < 32; ++q) p[q] = __uint_as_float(r0[q]);
-        st_row32_bf16(sP, i, 2 * half * 32, p);
-#pragma unroll
-        for (int q = 0; q < 32; ++q) p[q] = __uint_as_float(r1[q]);
-        st_row32_bf16(sP, i, (2 * half + 1) * 32, p);
-      } else {
-        s->abort = 1;
-      }
-      fence_async_smem();
-      tc_fence_before();
-      __syncthreads();
-      if (s->abort) {
-        stop = true;
-        break;
-      }
-      if (tid == kProducer) {
-        tma_store_4d(&map_o, sQ, 0, item.h, row0, item.b);
-        tma_store_4d(&map_o, sQ + kBox, 64, item.h, row0, item.b);
-        tma_store_commit();
+          for (int q = 0; q < 32; ++q) p[q] = __uint_as_float(r1[q]);
+          st_row32_bf16(sP, i, (2 * half + 1) * 32, p);
+          fence_async_smem();
+          tc_fence_before();
+          mbar_arrive(&s->e_b2);
+        }
       }
     }
+    if (named_sync_or(kEpiBar, kEpiThreads, bad) && tid == 0) s->abort = 1;
   }
-  if (tid == kProducer) tma_store_wait0();
+  __syncwarp();
   tc_fence_before();
   __syncthreads();
+  tc_fence_after();
   if (warp == 0) tmem_dealloc(tmem, kTmemCols);
 }
 
