@@ -63,7 +63,8 @@ constexpr uint32_t T0 = 0, T1 = 128, T2 = 256, TR = 384;
 struct Smem {
   uint64_t ld_kv, ld_qd, ld_p, ld_r;  // TMA -> MMA warp / epilogue
   uint64_t c1, c1b, c2, c2b, c3a, c3, c4;  // MMA commits -> epilogue / producer
-  uint64_t e1, e2, e3a, e0;  // epilogue -> MMA warp (256 arrivals each); e2 also -> producer: dQ staged
+  uint64_t e1, e2, e3a, e0;  // epilogue -> MMA warp (256 arrivals each)
+  uint64_t e2q;              // epilogue -> producer: dQ staged (256 arrivals)
   uint64_t staged;           // epilogue -> producer: dK, dV staged (256 arrivals)
   uint64_t free_a, free_b;   // producer -> epilogue: the previous dK / dV stores have read the buffer
   uint32_t tmem_base;
@@ -166,6 +167,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_walk_tc(
     mbar_init(&s->c4, 1);
     mbar_init(&s->e1, kEpiThreads);
     mbar_init(&s->e2, kEpiThreads);
+    mbar_init(&s->e2q, kEpiThreads);
     mbar_init(&s->e3a, kEpiThreads);
     mbar_init(&s->e0, kEpiThreads);
     mbar_init(&s->staged, kEpiThreads);
@@ -290,7 +292,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_walk_tc(
             bulk_prefetch_l2(R + (((int64_t)ns.b * T + slot) * H + ns.h) * kD * kD, kD * kD * sizeof(float));
           }
           // dQ, staged over S' (which MMA 2 has read), goes out
-          if (!(ok = mbar_wait_or_abort(&s->e2, par, SITE_BWD_TMA, abort_flag))) break;
+          if (!(ok = mbar_wait_or_abort(&s->e2q, par, SITE_BWD_TMA, abort_flag))) break;
           store_tile(&map_dq, pair(par ^ 1u, 1), item, row0);
           // K, V and X are free once the first part of MMA 3 is done; the next
           // Q and dO go into the dP'/S' pair once dP'^T Q has read dP' and dQ
@@ -514,7 +516,10 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_walk_tc(
               pq[c2][q] = pack_bf16(fmaf(wi, __uint_as_float(re[2 * q]), __uint_as_float(ra[2 * q])),
                                     fmaf(wi, __uint_as_float(re[2 * q + 1]), __uint_as_float(ra[2 * q + 1])));
           }
+          // TMEM 0 and 2 are read and X holds R: MMA 3 may start
+          fence_async_smem();
           tc_fence_before();
+          mbar_arrive(&s->e2);
           wait(&s->c2b, par, SITE_BWD_MMA);
 #pragma unroll
           for (int c2 = 0; c2 < 2; ++c2)
@@ -524,8 +529,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_walk_tc(
                         make_uint4(pq[c2][4 * q], pq[c2][4 * q + 1], pq[c2][4 * q + 2], pq[c2][4 * q + 3]));
         }
         fence_async_smem();
-        tc_fence_before();
-        mbar_arrive(&s->e2);
+        mbar_arrive(&s->e2q);
 
         // ---- epilogue 3a: dO~ = diag(lambda^{j+1}) dO (S'^T dO has read dO), while MMA 3 runs
         if (scale) {
