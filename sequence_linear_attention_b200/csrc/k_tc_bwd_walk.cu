@@ -451,12 +451,15 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_walk_tc(
           tmem_ld32(lane_base + T1 + cc * 32, rs);
           tmem_ld_wait();
           float fp[32], fs[32];
-          if (cc < (warp & 3)) {  // below the diagonal: every j < i
+          if (cc < (warp & 3)) {
+            // below the diagonal (every j < i): lambda^{i-j} from the smallest
+            // power up, one multiplication by lambda per column
+            float wgt = s->pw[i - cc * 32 - 31];
 #pragma unroll
-            for (int q = 0; q < 32; ++q) {
-              const float wgt = s->pw[i - cc * 32 - q];
+            for (int q = 31; q >= 0; --q) {
               fp[q] = __uint_as_float(rp[q]) * wgt;
               fs[q] = __uint_as_float(rs[q]) * wgt;
+              wgt *= lam;
             }
           } else {
 #pragma unroll

@@ -385,10 +385,17 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_walk_tc(const __grid_constant
           tmem_ld32(lane_base + TS + cc * 32, r);
           tmem_ld_wait();
           if (cc < (warp & 3)) {
+            // below the diagonal (every j < i): lambda^{i-j} from the smallest
+            // power up, one multiplication by lambda per column
+            float wgt = s->pw[i - cc * 32 - 31];
 #pragma unroll
-            for (int q = 0; q < 16; ++q)
-              ps[c2][q] = pack_bf16(__uint_as_float(r[2 * q]) * s->pw[i - cc * 32 - 2 * q],
-                                    __uint_as_float(r[2 * q + 1]) * s->pw[i - cc * 32 - 2 * q - 1]);
+            for (int q = 15; q >= 0; --q) {
+              const float hi = __uint_as_float(r[2 * q + 1]) * wgt;
+              wgt *= lam;
+              const float lo = __uint_as_float(r[2 * q]) * wgt;
+              wgt *= lam;
+              ps[c2][q] = pack_bf16(lo, hi);
+            }
           } else {
 #pragma unroll
             for (int q = 0; q < 16; ++q) {
