@@ -79,12 +79,12 @@ def flops_per_step(tokens_heads: int, d: int, C: int) -> float:
 MEASURED_TRAFFIC = {
     # DRAM bytes per launch at the workload's full size: twice the ncu capture of
     # the 32768-token case of the same workload (traffic grows with the tokens)
-    "bwd_walk_tc": (["k_tc_bwd_walk.cu", "sm100.cuh", "lasp_common.cuh", "tma_host.h"], "1cf301c58e7839f6",
-                    2 * (723450880 + 368640768)),
-    "fwd_walk_tc": (["k_tc_fwd_walk.cu", "sm100.cuh", "lasp_common.cuh", "tma_host.h"], "458f7f6b3a9f51b1",
-                    2 * (436959744 + 231108352)),
+    "bwd_walk_tc": (["k_tc_bwd_walk.cu", "sm100.cuh", "lasp_common.cuh", "tma_host.h"], "20c936251fd30878",
+                    2 * (726024448 + 368554240)),
+    "fwd_walk_tc": (["k_tc_fwd_walk.cu", "sm100.cuh", "lasp_common.cuh", "tma_host.h"], "659ed7f878139615",
+                    2 * (437606656 + 230750464)),
     "segment_states_tc": (["k_tc_states.cu", "sm100.cuh", "lasp_common.cuh", "tma_host.h"], "0124abcfbf954d17",
-                          2 * (268475136 + 22717184)),
+                          2 * (268472064 + 23057408)),
 }
 
 
