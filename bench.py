@@ -47,13 +47,14 @@ def algorithmic_bytes(name: str, tokens_heads: int, d: int, C: int, G: int, elem
       segment_scan:                  read and write s/G                  = 2s/G
       chunk_out_*:                   read q, k, v and P, write o         = 4de + s/C
       fwd_walk_tc:  read q, k, v and the segment's P (s/G), write o and
-                    the cached P of every chunk: bf16 (s/2C) when C = 128,
-                    else fp32 for the other chunks (s/C - s/G)
-                                               = 4de + s/G + s/2C   (C = 128)
+                    the cache: for C <= 128 the bf16 operand tile of the state
+                    entering each 128-token tile (s/256), for C > 128 fp32 P of
+                    the other chunks (s/C - s/G)
+                                               = 4de + s/G + s/256  (C <= 128)
                                                = 4de + s/C          (C > 128)
       chunk_bwd_*:  read q, k, v, dO, P and R, write dq, dk, dv          = 7de + 2s/C
-      bwd_walk_tc:  read q, k, v, dO, the cached bf16 P (s/2C) and the
-                    segment's R (s/G), write dq, dk, dv            = 7de + s/2C + s/G
+      bwd_walk_tc:  read q, k, v, dO, the cached bf16 tiles (s/256) and the
+                    segment's R (s/G), write dq, dk, dv            = 7de + s/256 + s/G
     """
     s = 4 * d * d
     de = d * elem
@@ -61,9 +62,9 @@ def algorithmic_bytes(name: str, tokens_heads: int, d: int, C: int, G: int, elem
         "chunk_states_tc": 2 * de + s / C, "chunk_states_simt": 2 * de + s / C,
         "segment_states_tc": 2 * de + s / G,
         "state_scan": 2 * s / C, "segment_scan": 2 * s / G,
-        "chunk_out_tc": 4 * de + s / C, "chunk_out_simt": 4 * de + s / C, "fwd_walk_tc": 4 * de + (s / G + s / (2 * C) if C == 128 else s / C),
+        "chunk_out_tc": 4 * de + s / C, "chunk_out_simt": 4 * de + s / C, "fwd_walk_tc": 4 * de + (s / G + s / 256 if C <= 128 else s / C),
         "chunk_bwd_tc": 7 * de + 2 * s / C, "chunk_bwd_simt": 7 * de + 2 * s / C,
-        "bwd_walk_tc": 7 * de + s / (2 * C) + s / G,
+        "bwd_walk_tc": 7 * de + s / 256 + s / G,
     }[name]
     return per * tokens_heads
 

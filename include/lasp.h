@@ -80,9 +80,10 @@ typedef enum { LASP_F32 = 0, LASP_BF16 = 1 } lasp_dtype;
  *                 cache of chunk-entering states P_c that lasp_bwd reads (LASP
  *                 section 3.4 "KV State Caching"), one d x d slot per (b, c, h).
  *                 Its encoding inside a slot is internal to the library (fp32
- *                 P_c, or, for bf16 with d = 128 and C = 128, the bf16 operand
- *                 tile of P_c); pass it unchanged to lasp_bwd with the same
- *                 sizes. The per-chunk states themselves are exposed by
+ *                 P_c; or, for bf16 with d = 128, C dividing 128 and N a
+ *                 multiple of 128, the bf16 operand tile of the state entering
+ *                 each 128-token tile, in the slot of the tile's first chunk);
+ *                 pass it unchanged to lasp_bwd with the same sizes. The per-chunk states themselves are exposed by
  *                 lasp_chunk_states + lasp_state_prefix. Required.
  *   init_state:   in,  float [B, H, d, d] or NULL: the state entering token 0
  *                 (the prefix of the shards before this one in the LASP-2

@@ -130,7 +130,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_walk_tc(
     const __grid_constant__ CUtensorMap map_dq, const __grid_constant__ CUtensorMap map_dk,
     const __grid_constant__ CUtensorMap map_dv,
     const __grid_constant__ CUtensorMap map_state, const float* decay, const float* __restrict__ P,
-    float* __restrict__ R, int H, int64_t N, int T, int G, int nseg,
+    float* __restrict__ R, int H, int64_t N, int T, int C, int G, int nseg,
     int64_t nitems) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
@@ -209,7 +209,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_walk_tc(
       // P of a chunk: the forward walk stored it in the chunk's cache slot as the
       // bf16 operand tile (128-byte swizzled), so it is copied into X as is
       auto load_p = [&](const Item& it, int t) {
-        const int64_t c = ((int64_t)it.seg * G + (int64_t)t * kTile) / kTile;
+        const int64_t c = ((int64_t)it.seg * G + (int64_t)t * kTile) / C;  // the tile's first chunk
         const float* src = P + (((int64_t)it.b * T + c) * H + it.h) * kD * kD;
         mbar_arrive_expect_tx(&s->ld_p, kTileBytes);
         bulk_load(sX, src, kTileBytes, &s->ld_p);
@@ -249,7 +249,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_walk_tc(
           if (t == tiles - 1) {
             // R entering the segment's last chunk, as four 32-column fp32 boxes
             // into the dP'/S' pair; epilogue 1 moves it into TMEM
-            const int64_t slot = (int64_t)item.seg * tiles + tiles - 1;
+            const int64_t slot = (int64_t)(item.seg + 1) * (G / C) - 1;  // the segment's last chunk
             const int y = (int)((((int64_t)item.b * T + slot) * H + item.h) * kD);
             mbar_arrive_expect_tx(&s->ld_r, kD * kD * 4);
 #pragma unroll
@@ -282,13 +282,13 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_walk_tc(
             tma_prefetch_4d(&map_k, 64, nx.h, nrow, nx.b);
             tma_prefetch_4d(&map_v, 0, nx.h, nrow, nx.b);
             tma_prefetch_4d(&map_v, 64, nx.h, nrow, nx.b);
-            const int64_t c = (int64_t)nrow / kTile;
+            const int64_t c = (int64_t)nrow / C;
             bulk_prefetch_l2(P + (((int64_t)nx.b * T + c) * H + nx.h) * kD * kD, kTileBytes);
           }
           if (t == (tiles > 1 ? 1 : 0) && w + gridDim.x < nitems) {
             // and the next segment's entering R, read at the segment switch
             const Item ns = item_of(w + gridDim.x, H, nseg);
-            const int64_t slot = (int64_t)ns.seg * tiles + tiles - 1;
+            const int64_t slot = (int64_t)(ns.seg + 1) * (G / C) - 1;
             bulk_prefetch_l2(R + (((int64_t)ns.b * T + slot) * H + ns.h) * kD * kD, kD * kD * sizeof(float));
           }
           // dQ, staged over S' (which MMA 2 has read), goes out
@@ -589,8 +589,12 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_walk_tc(
 
 }  // namespace tc_bwd_walk_detail
 
-bool tc_bwd_walk_ok(int dtype, int d, int64_t C) {
-  return dtype == LASP_BF16 && d == tc_bwd_walk_detail::kD && C == tc_bwd_walk_detail::kTile;
+bool tc_bwd_walk_ok(int dtype, int d, int64_t C, int64_t N) {
+  // chunks that divide the 128-token tile: the forward walk leaves the bf16
+  // operand tile of each tile's entering state in the slot of its first chunk
+  using tc_bwd_walk_detail::kTile;
+  return dtype == LASP_BF16 && d == tc_bwd_walk_detail::kD && C >= 1 && C <= kTile && kTile % C == 0 &&
+         N % kTile == 0;
 }
 
 cudaError_t tc_bwd_walk(const void* q, const void* k, const void* v, const void* dout, const float* decay,
@@ -610,7 +614,7 @@ cudaError_t tc_bwd_walk(const void* q, const void* k, const void* v, const void*
   const int nseg = (int)(N / G);
   const int64_t nitems = (int64_t)B * H * nseg;
   const unsigned grid = (unsigned)std::min<int64_t>(nitems, num_sms);
-  bwd_walk_tc<<<grid, kThreads, smem, st>>>(mq, mk, mv, mdo, mdq, mdk, mdv, mr, decay, P, R, H, N, (int)(N / C), G,
+  bwd_walk_tc<<<grid, kThreads, smem, st>>>(mq, mk, mv, mdo, mdq, mdk, mdv, mr, decay, P, R, H, N, (int)(N / C), C, G,
                                             nseg, nitems);
   return cudaGetLastError();
 }

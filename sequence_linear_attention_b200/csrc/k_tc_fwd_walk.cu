@@ -522,16 +522,22 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_walk_tc(const __grid_constant
 
 }  // namespace tc_fwd_walk_detail
 
-bool tc_fwd_walk_ok(int dtype, int d, int64_t C) {
-  return dtype == LASP_BF16 && d == tc_fwd_walk_detail::kD && C % tc_fwd_walk_detail::kTile == 0;
+bool tc_fwd_walk_ok(int dtype, int d, int64_t C, int64_t N) {
+  // 128-token tiles: chunks that divide a tile or are made of whole tiles
+  using tc_fwd_walk_detail::kTile;
+  if (dtype != LASP_BF16 || d != tc_fwd_walk_detail::kD || C < 1) return false;
+  const int64_t unit = C > kTile ? C : kTile;
+  return (C % kTile == 0 || kTile % C == 0) && N % unit == 0;
 }
 
 int walk_segment_tokens(int64_t N, int C) {
-  // about 1024 tokens per segment: enough tiles per walk to hide the segment's
-  // first load, enough segments to spread over the SMs
-  int m = C >= 1024 ? 1 : 1024 / C;
-  while (m > 1 && N % ((int64_t)C * m) != 0) --m;
-  return C * m;
+  // about 1024 tokens per segment (a multiple of the tile and of the chunk):
+  // enough tiles per walk to hide the segment's first load, enough segments to
+  // spread over the SMs
+  const int unit = C > tc_fwd_walk_detail::kTile ? C : tc_fwd_walk_detail::kTile;
+  int m = unit >= 1024 ? 1 : 1024 / unit;
+  while (m > 1 && N % ((int64_t)unit * m) != 0) --m;
+  return unit * m;
 }
 
 cudaError_t tc_fwd_walk(const void* q, const void* k, const void* v, const float* decay, float* P, void* o, int B,
@@ -548,9 +554,10 @@ cudaError_t tc_fwd_walk(const void* q, const void* k, const void* v, const float
   const int nseg = (int)(N / G);
   const int64_t nitems = (int64_t)B * H * nseg;
   const unsigned grid = (unsigned)std::min<int64_t>(nitems, num_sms);
-  // with C = 128 the backward walk reads the cache: it gets each chunk's state
-  // as the bf16 operand tile; otherwise the cache holds fp32 states
-  const int cache_bf16 = C == kTile ? 1 : 0;
+  // with chunks that divide the tile the backward walk reads the cache: it gets
+  // each tile's entering state as the bf16 operand tile (in the slot of the
+  // tile's first chunk); with longer chunks the cache holds fp32 states
+  const int cache_bf16 = C <= kTile ? 1 : 0;
   fwd_walk_tc<<<grid, kThreads, smem, st>>>(mq, mk, mv, mo, mp, decay, P, H, (int)(N / C), C, G, nseg, nitems,
                                            cache_bf16);
   return cudaGetLastError();

@@ -193,7 +193,7 @@ int lasp_fwd(const void* q, const void* k, const void* v, const float* decay, vo
   if ((s = check_ptrs({q, k, v, o, state_cache}, {decay, init_state}))) return s;
   cudaStream_t st = (cudaStream_t)stream;
   const int T = (int)(N / C);
-  if (tc_fwd_walk_ok(dtype, d, C)) {
+  if (tc_fwd_walk_ok(dtype, d, C, N)) {
     // segments of G tokens: their states go to the slots of their first chunks,
     // the exclusive prefix over segments turns them into P of those chunks, and
     // the walk carries the state through each segment, filling the other slots
@@ -249,7 +249,7 @@ int lasp_bwd(const void* q, const void* k, const void* v, const float* decay, co
     return s;
   cudaStream_t st = (cudaStream_t)stream;
   const int T = (int)(N / C);
-  if (tc_bwd_walk_ok(dtype, d, C)) {
+  if (tc_bwd_walk_ok(dtype, d, C, N)) {
     // segments of G tokens: their gradient states go to the slots of their last
     // chunks, the exclusive suffix over segments turns them into R of those
     // chunks (and gives dinit), and the walk carries R backward through each
@@ -340,7 +340,7 @@ const char* lasp_kernel_name(int id) {
 
 int lasp_segment_tokens(int64_t N, int C, int d, int dtype) {
   if (N <= 0 || C < 1 || N % C != 0) return 0;
-  return tc_fwd_walk_ok(dtype, d, C) ? walk_segment_tokens(N, C) : C;
+  return tc_fwd_walk_ok(dtype, d, C, N) ? walk_segment_tokens(N, C) : C;
 }
 
 int lasp_set_wait_limit_ns(uint64_t limit_ns) {

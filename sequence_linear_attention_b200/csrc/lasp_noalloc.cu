@@ -62,7 +62,7 @@ extern "C" int lasp_bwd_noalloc(const void* q, const void* k, const void* v, con
   cudaStream_t st = (cudaStream_t)stream;
   // the same steps as lasp_bwd, with the workspace in the fixed array; every
   // element of R that is read is written first, so nothing is cleared
-  if (tc_bwd_walk_ok(dtype, d, C)) {
+  if (tc_bwd_walk_ok(dtype, d, C, N)) {
     const int G = walk_segment_tokens(N, C);
     const int stride = G / C;
     if ((s = cuda_status(tc_chunk_states_slots(q, dout, decay, R, B, H, N, d, G, 1, T, stride, stride - 1, st))))

@@ -21,19 +21,23 @@ cudaError_t tc_chunk_states_slots(const void* a, const void* b, const float* dec
                                   cudaStream_t st);
 
 // Forward walk over segments of G tokens with the state on chip (bf16,
-// d = 128, C a multiple of 128, G a multiple of C dividing N). P must hold,
-// in the slot of each segment's first chunk, the state entering that segment;
-// the walk fills the other chunks' slots and writes o.
-bool tc_fwd_walk_ok(int dtype, int d, int64_t C);
+// d = 128, C a multiple of 128 or a divisor of it, N a multiple of max(C, 128),
+// G = walk_segment_tokens(N, C)). P must hold, in the slot of each segment's
+// first chunk, the state entering that segment; the walk writes o and fills the
+// cache: fp32 P_c at the other chunk starts when C > 128, otherwise the bf16
+// operand tile of the state entering each 128-token tile in the slot of the
+// tile's first chunk.
+bool tc_fwd_walk_ok(int dtype, int d, int64_t C, int64_t N);
 int walk_segment_tokens(int64_t N, int C);
 cudaError_t tc_fwd_walk(const void* q, const void* k, const void* v, const float* decay, float* P, void* o, int B,
                         int H, int64_t N, int d, int C, int G, int num_sms, cudaStream_t st);
 
 // Backward walk over segments with the gradient state on chip (bf16, d = 128,
-// C = 128). R must hold, in the slot of each segment's last chunk, the
-// gradient state entering that chunk; the walk fills the other chunks' R
-// slots and writes dq, dk, dv. P is the forward state cache.
-bool tc_bwd_walk_ok(int dtype, int d, int64_t C);
+// C dividing 128, N a multiple of 128). R must hold, in the slot of each
+// segment's last chunk, the gradient state entering that chunk from the tokens
+// after the segment; the walk writes dq, dk, dv (R of the other chunks stays on
+// chip). P is the forward walk's cache of bf16 operand tiles.
+bool tc_bwd_walk_ok(int dtype, int d, int64_t C, int64_t N);
 cudaError_t tc_bwd_walk(const void* q, const void* k, const void* v, const void* dout, const float* decay,
                         const float* P, float* R, void* dq, void* dk, void* dv, int B, int H, int64_t N, int d, int C,
                         int G, int num_sms, cudaStream_t st);

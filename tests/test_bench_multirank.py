@@ -53,3 +53,6 @@ def test_single_rank_needs_no_process_group():
     s4 = 4 * 128 * 128
     assert bench.algorithmic_bytes("fwd_walk_tc", 1, 128, 128, 1024, 2) == 4 * 128 * 2 + s4 / 1024 + s4 / 256
     assert bench.algorithmic_bytes("fwd_walk_tc", 1, 128, 256, 1024, 2) == 4 * 128 * 2 + s4 / 256
+    # chunks inside a tile: one cached bf16 tile per 128 tokens whatever C is
+    assert bench.algorithmic_bytes("fwd_walk_tc", 1, 128, 64, 1024, 2) == 4 * 128 * 2 + s4 / 1024 + s4 / 256
+    assert bench.algorithmic_bytes("bwd_walk_tc", 1, 128, 32, 1024, 2) == 7 * 128 * 2 + s4 / 256 + s4 / 1024

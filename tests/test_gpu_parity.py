@@ -48,6 +48,9 @@ SMALL = [
     (2, 150, 1024, 128, 128, True, True),  # more segments than SMs: each CTA walks several
     (2, 3, 1152, 128, 128, True, True),    # three segments of three tiles
     (1, 4, 2048, 128, 128, True, False),   # walks without decay
+    (1, 3, 2048, 128, 64, True, True),     # walks with chunks that divide the tile
+    (2, 2, 1280, 128, 32, True, True),
+    (1, 2, 384, 128, 16, True, False),
 ]
 
 
@@ -80,10 +83,11 @@ def test_chunk_size_invariance():
     """The output does not depend on the chunk size (it is a regrouping of the
     same sums, LASP Eq. 8 and Eq. 10)."""
     inp = lasp_inputs.make_inputs(1, 512, 4, 128, seed=91, bf16=True, decayed=True)
-    a = run_fwd_bwd(inp, 64)
     b = run_fwd_bwd(inp, 128)
-    for n in ("o", "dq", "dk", "dv"):
-        assert rel_err(to_host(a[n]), to_host(b[n]).astype(np.float64)) <= tol(True), n
+    for C in (32, 64, 256):  # walks with chunks inside a tile; forward walk + per-chunk backward
+        a = run_fwd_bwd(inp, C)
+        for n in ("o", "dq", "dk", "dv"):
+            assert rel_err(to_host(a[n]), to_host(b[n]).astype(np.float64)) <= tol(True), (C, n)
 
 
 def test_no_decay_equals_all_ones_bitwise():

@@ -27,8 +27,18 @@ def test_bf16_d128_c128_runs_the_segment_walks():
                      "segment_states_tc", "segment_scan", "bwd_walk_tc"], names
 
 
-def test_bf16_c64_runs_the_per_chunk_tensor_core_kernels():
-    inp = lasp_inputs.make_inputs(1, 512, 2, 128, seed=202, bf16=True, decayed=True)
+def test_bf16_c64_runs_the_segment_walks():
+    """Chunks that divide the 128-token tile walk too (the cache then holds each
+    tile's entering state in the slot of the tile's first chunk)."""
+    for C in (64, 32, 16):
+        inp = lasp_inputs.make_inputs(1, 512, 2, 128, seed=202 + C, bf16=True, decayed=True)
+        names = _traced_names(inp, C)
+        assert names == ["segment_states_tc", "segment_scan", "fwd_walk_tc",
+                         "segment_states_tc", "segment_scan", "bwd_walk_tc"], (C, names)
+
+
+def test_bf16_c64_with_a_ragged_tile_runs_the_per_chunk_tensor_core_kernels():
+    inp = lasp_inputs.make_inputs(1, 320, 2, 128, seed=202, bf16=True, decayed=True)
     names = _traced_names(inp, 64)
     assert names == ["chunk_states_tc", "state_scan", "chunk_out_tc",
                      "chunk_states_tc", "state_scan", "chunk_bwd_tc"], names
@@ -52,6 +62,8 @@ def test_segment_length():
     import sequence_linear_attention_b200 as lasp
     assert lasp.lasp_segment_tokens(65536, 128, 128, 1) == 1024
     assert lasp.lasp_segment_tokens(1152, 128, 128, 1) == 384   # 9 tiles: three segments of three
-    assert lasp.lasp_segment_tokens(256, 64, 128, 1) == 64      # per-chunk path
+    assert lasp.lasp_segment_tokens(256, 64, 128, 1) == 256     # two tiles of four chunks
+    assert lasp.lasp_segment_tokens(8192, 64, 128, 1) == 1024
+    assert lasp.lasp_segment_tokens(320, 64, 128, 1) == 64      # N not a multiple of 128: per-chunk path
     assert lasp.lasp_segment_tokens(256, 64, 32, 0) == 64
     assert lasp.lasp_segment_tokens(100, 64, 128, 1) == 0       # C does not divide N
