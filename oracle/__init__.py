@@ -19,6 +19,10 @@ it with ctypes. Each wrapper states the passage it follows:
   chunk from LASP Eq. 10 / Eq. 20.
 * :func:`state_snapshots` -- LASP page, section 3.4 "KV State Caching": the
   chunk-boundary states of the recurrences.
+* :func:`bidir_fwd`, :func:`bidir_bwd` -- the bidirectional (unmasked) form:
+  LASP page, section 3.1, Eq. 3 right product Q (K^T V) without Norm; LASP-2
+  review page, "Summary": the unmasked variant gathers all chunk states and
+  every chunk computes Q_t M_{1:T}, and the backward the same with dM.
 
 Inputs are float32 arrays shaped [B, N, H, d] (any strides, feature axis
 contiguous). Values that came from bf16 are exact in float32 and double, so the
@@ -67,9 +71,13 @@ def _load():
             lib.oracle_chunk_states.argtypes = [_P, _P, _L, _L, _L, _P, _P, _I, _L, _I, _I, _L, _I]
             lib.oracle_state_scan.argtypes = [_P, _P, _P, _P, _P, _I, _L, _I, _I, _L, _I]
             lib.oracle_state_snapshots.argtypes = [_P, _P, _L, _L, _L, _P, _P, _P, _I, _L, _I, _I, _L, _I]
+            lib.oracle_bidir_fwd.argtypes = [_P, _P, _P, _L, _L, _L, _P, _L, _L, _L, _P, _I, _L, _I, _I]
+            lib.oracle_bidir_bwd.argtypes = [_P, _P, _P, _P, _L, _L, _L, _P, _P, _P, _L, _L, _L, _P,
+                                             _I, _L, _I, _I]
             lib.oracle_num_threads.restype = _I
             for f in (lib.oracle_fwd, lib.oracle_bwd, lib.oracle_chunk_states,
-                      lib.oracle_state_scan, lib.oracle_state_snapshots):
+                      lib.oracle_state_scan, lib.oracle_state_snapshots, lib.oracle_bidir_fwd,
+                      lib.oracle_bidir_bwd):
                 f.restype = None
             _lib = lib
     return _lib
@@ -207,3 +215,34 @@ def state_snapshots(a, b, lam, C, init=None, kind=0):
     _load().oracle_state_snapshots(pa, b.ctypes.data, sb, sn, sh, pl, pi, P.ctypes.data,
                                    B, N, H, d, C, kind)
     return P
+
+
+def bidir_fwd(q, k, v, want_state=False):
+    """Bidirectional (unmasked) output o_s = q_s M with M = sum_s k_s^T v_s
+    (LASP Eq. 3 right product, no Norm, no decay). Returns o (float64
+    [B, N, H, d]) and, if ``want_state``, M [B, H, d, d]."""
+    B, N, H, d = q.shape
+    pq, sb, sn, sh = _view(q)
+    _view(k, q), _view(v, q)
+    o = np.empty((B, N, H, d), np.float64)
+    M = np.empty((B, H, d, d), np.float64) if want_state else None
+    _load().oracle_bidir_fwd(pq, k.ctypes.data, v.ctypes.data, sb, sn, sh, o.ctypes.data, N * H * d, H * d, d,
+                             _ptr(M), B, N, H, d)
+    return (o, M) if want_state else o
+
+
+def bidir_bwd(q, k, v, do, want_state=False):
+    """Gradients of sum(o * do) for :func:`bidir_fwd`: dq = do M^T,
+    dk = v dM^T, dv = k dM with dM = sum_s q_s^T do_s. Returns dq, dk, dv
+    (float64 [B, N, H, d]) and, if ``want_state``, dM [B, H, d, d]."""
+    B, N, H, d = q.shape
+    pq, sb, sn, sh = _view(q)
+    for t in (k, v, do):
+        _view(t, q)
+    dq = np.empty((B, N, H, d), np.float64)
+    dk = np.empty_like(dq)
+    dv = np.empty_like(dq)
+    dM = np.empty((B, H, d, d), np.float64) if want_state else None
+    _load().oracle_bidir_bwd(pq, k.ctypes.data, v.ctypes.data, do.ctypes.data, sb, sn, sh, dq.ctypes.data,
+                             dk.ctypes.data, dv.ctypes.data, N * H * d, H * d, d, _ptr(dM), B, N, H, d)
+    return (dq, dk, dv, dM) if want_state else (dq, dk, dv)

@@ -311,3 +311,91 @@ int oracle_num_threads(void) {
   return 1;
 #endif
 }
+
+/*
+ * Bidirectional (unmasked) linear attention: LASP Eq. 3 without Norm, the
+ * right product O = Q (K^T V); on the LASP-2 page the unmasked variant sums
+ * all chunk states, M_{1:T} = sum_t M_t, and every chunk computes Q_t M_{1:T}
+ * (no decay).  Per (b, h):
+ *   M[i][j] = sum_s k_s[i] v_s[j];           o_s[j] = sum_i q_s[i] M[i][j].
+ * M_out (optional, [B, H, d, d]) receives M.
+ */
+void oracle_bidir_fwd(const float *q, const float *k, const float *v, long sb, long sn, long sh,
+                      double *o, long ob, long on, long oh, double *M_out, int B, long N, int H, int d) {
+#pragma omp parallel for schedule(dynamic, 1)
+  for (long task = 0; task < (long)B * H; ++task) {
+    int h = (int)(task % H);
+    int b = (int)(task / H);
+    double *M = (double *)calloc((size_t)d * d, sizeof(double));
+    for (long s = 0; s < N; ++s) {
+      const float *ks = tok(k, sb, sn, sh, b, s, h);
+      const float *vs = tok(v, sb, sn, sh, b, s, h);
+      for (int i = 0; i < d; ++i)
+        for (int j = 0; j < d; ++j) M[i * d + j] += (double)ks[i] * vs[j];
+    }
+    for (long s = 0; s < N; ++s) {
+      const float *qs = tok(q, sb, sn, sh, b, s, h);
+      double *os = tokd(o, ob, on, oh, b, s, h);
+      for (int j = 0; j < d; ++j) {
+        double acc = 0.0;
+        for (int i = 0; i < d; ++i) acc += (double)qs[i] * M[i * d + j];
+        os[j] = acc;
+      }
+    }
+    if (M_out) memcpy(st_bh_w(M_out, H, d, b, h), M, sizeof(double) * d * d);
+    free(M);
+  }
+}
+
+/*
+ * Its gradients for L = sum_s o_s . do_s (the unmasked backward of the
+ * LASP-2 page: the gradient state summed over all chunks):
+ *   dM[i][j] = sum_s q_s[i] do_s[j];
+ *   dq_s[i] = sum_j M[i][j] do_s[j];   dk_s[i] = sum_j dM[i][j] v_s[j];
+ *   dv_s[j] = sum_i k_s[i] dM[i][j].
+ * dM_out (optional, [B, H, d, d]) receives dM.
+ */
+void oracle_bidir_bwd(const float *q, const float *k, const float *v, const float *dout, long sb, long sn,
+                      long sh, double *dq, double *dk, double *dv, long gb, long gn, long gh, double *dM_out,
+                      int B, long N, int H, int d) {
+#pragma omp parallel for schedule(dynamic, 1)
+  for (long task = 0; task < (long)B * H; ++task) {
+    int h = (int)(task % H);
+    int b = (int)(task / H);
+    double *M = (double *)calloc((size_t)d * d, sizeof(double));
+    double *G = (double *)calloc((size_t)d * d, sizeof(double));
+    for (long s = 0; s < N; ++s) {
+      const float *qs = tok(q, sb, sn, sh, b, s, h);
+      const float *ks = tok(k, sb, sn, sh, b, s, h);
+      const float *vs = tok(v, sb, sn, sh, b, s, h);
+      const float *ds = tok(dout, sb, sn, sh, b, s, h);
+      for (int i = 0; i < d; ++i)
+        for (int j = 0; j < d; ++j) {
+          M[i * d + j] += (double)ks[i] * vs[j];
+          G[i * d + j] += (double)qs[i] * ds[j];
+        }
+    }
+    for (long s = 0; s < N; ++s) {
+      const float *ks = tok(k, sb, sn, sh, b, s, h);
+      const float *vs = tok(v, sb, sn, sh, b, s, h);
+      const float *ds = tok(dout, sb, sn, sh, b, s, h);
+      double *dqs = tokd(dq, gb, gn, gh, b, s, h);
+      double *dks = tokd(dk, gb, gn, gh, b, s, h);
+      double *dvs = tokd(dv, gb, gn, gh, b, s, h);
+      for (int i = 0; i < d; ++i) {
+        double aq = 0.0, ak = 0.0, av = 0.0;
+        for (int j = 0; j < d; ++j) {
+          aq += M[i * d + j] * ds[j];
+          ak += G[i * d + j] * vs[j];
+          av += (double)ks[j] * G[j * d + i];
+        }
+        dqs[i] = aq;
+        dks[i] = ak;
+        dvs[i] = av;
+      }
+    }
+    if (dM_out) memcpy(st_bh_w(dM_out, H, d, b, h), G, sizeof(double) * d * d);
+    free(M);
+    free(G);
+  }
+}

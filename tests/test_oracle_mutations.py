@@ -41,6 +41,11 @@ MUTATIONS = [
     ("gradient snapshots decay before adding the token",
      "S[i * d + j] = l * (S[i * d + j] + (double)as[i] * bs[j]);",
      "S[i * d + j] = l * S[i * d + j] + (double)as[i] * bs[j];", 0),
+    ("bidirectional state transposed", "M[i * d + j] += (double)ks[i] * vs[j];",
+     "M[i * d + j] += (double)vs[i] * ks[j];", 0),
+    ("bidirectional dk uses dM transposed", "ak += G[i * d + j] * vs[j];", "ak += G[j * d + i] * vs[j];", 0),
+    ("bidirectional dv uses dM transposed", "av += (double)ks[j] * G[j * d + i];",
+     "av += (double)ks[j] * G[i * d + j];", 0),
 ]
 
 
@@ -70,6 +75,7 @@ def _pins_pass():
         pins.test_chunk_states_equal_recurrence_run_over_the_chunk,
         pins.test_state_scan_closed_forms,
         pins.test_scan_of_chunk_states_equals_recurrence_snapshots,
+        pins.test_bidirectional_equals_left_product,
     ]
     for check in checks:
         try:
@@ -85,7 +91,8 @@ def test_pins_catch_the_mistake(tmp_path, name, old, new, nth):
     so = _build_mutant(tmp_path, old, new, nth)
     real = oracle._load()
     lib = ctypes.CDLL(so)
-    for f in ("oracle_fwd", "oracle_bwd", "oracle_chunk_states", "oracle_state_scan", "oracle_state_snapshots"):
+    for f in ("oracle_fwd", "oracle_bwd", "oracle_chunk_states", "oracle_state_scan", "oracle_state_snapshots",
+              "oracle_bidir_fwd", "oracle_bidir_bwd"):
         getattr(lib, f).argtypes = getattr(real, f).argtypes
         getattr(lib, f).restype = None
     lib.oracle_num_threads.restype = ctypes.c_int

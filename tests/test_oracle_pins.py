@@ -379,3 +379,65 @@ def test_results_do_not_depend_on_thread_count():
         outs.append(subprocess.run([sys.executable, "-c", code], env=env, check=True,
                                    capture_output=True, text=True).stdout.strip())
     assert outs[0] == outs[1]
+
+
+# ------------------------------------------- bidirectional (unmasked) variant
+def test_bidirectional_equals_left_product():
+    """LASP Eq. 3: Q (K^T V) equals the left product (Q K^T) V, written with
+    numpy matmuls in the other association; the gradients equal the textbook
+    ones of the left product: dQ = dO V^T K, dK = (dO V^T)^T Q, dV = (Q K^T)^T dO."""
+    q, k, v, do, _ = _problem(31, B=2, N=37, H=3, d=8, decayed=False)
+    o, M = oracle.bidir_fwd(q, k, v, want_state=True)
+    dq, dk, dv, dM = oracle.bidir_bwd(q, k, v, do, want_state=True)
+    for b in range(2):
+        for h in range(3):
+            Q, K, V, D = (x[b, :, h, :].astype(np.float64) for x in (q, k, v, do))
+            S, dP = Q @ K.T, D @ V.T
+            assert _rel(o[b, :, h], S @ V) < 1e-13
+            assert _rel(dq[b, :, h], dP @ K) < 1e-13
+            assert _rel(dk[b, :, h], dP.T @ Q) < 1e-13
+            assert _rel(dv[b, :, h], S.T @ D) < 1e-13
+            assert _rel(M[b, h], K.T @ V) < 1e-13
+            assert _rel(dM[b, h], Q.T @ D) < 1e-13
+
+
+def test_bidirectional_is_causal_plus_anticausal_minus_diagonal():
+    """Unmasked = the causal recurrence (lambda = 1) + the same recurrence run
+    on the reversed sequence, minus the diagonal term counted twice; ties the
+    bidirectional oracle to the token recurrence (LASP Eq. 4-6)."""
+    q, k, v, do, _ = _problem(32, B=1, N=29, H=2, d=8, decayed=False)
+    flip = lambda x: np.ascontiguousarray(x[:, ::-1])
+    causal = oracle.fwd(q, k, v)
+    anti = oracle.fwd(flip(q), flip(k), flip(v))[:, ::-1]
+    diag = np.einsum("bnhi,bnhi->bnh", q.astype(np.float64), k.astype(np.float64))[..., None] * v
+    assert _rel(oracle.bidir_fwd(q, k, v), causal + anti - diag) < 1e-12
+    dq_c, dk_c, dv_c = oracle.bwd(q, k, v, do)
+    dq_a, dk_a, dv_a = (g[:, ::-1] for g in oracle.bwd(flip(q), flip(k), flip(v), flip(do)))
+    qd = q.astype(np.float64)
+    kd, vd, dd = k.astype(np.float64), v.astype(np.float64), do.astype(np.float64)
+    vdo = np.einsum("bnhi,bnhi->bnh", vd, dd)[..., None]   # diagonal term's gradients
+    qk = np.einsum("bnhi,bnhi->bnh", qd, kd)[..., None]
+    dq, dk, dv = oracle.bidir_bwd(q, k, v, do)
+    assert _rel(dq, dq_c + dq_a - vdo * kd) < 1e-12
+    assert _rel(dk, dk_c + dk_a - vdo * qd) < 1e-12
+    assert _rel(dv, dv_c + dv_a - qk * dd) < 1e-12
+
+
+def test_bidirectional_gradients_match_finite_differences():
+    q, k, v, do, _ = _problem(33, B=1, N=20, H=2, d=6, decayed=False, quant=64)
+    dq, dk, dv = oracle.bidir_bwd(q, k, v, do)
+    h = 1.0 / 64
+    rng = np.random.default_rng(34)
+
+    def loss(qq, kk, vv):
+        return float(np.sum(oracle.bidir_fwd(qq, kk, vv) * do))
+
+    for grad, which in ((dq, 0), (dk, 1), (dv, 2)):
+        for _ in range(30):
+            ix = tuple(int(rng.integers(0, s)) for s in q.shape)
+            args_p = [q.copy(), k.copy(), v.copy()]
+            args_m = [q.copy(), k.copy(), v.copy()]
+            args_p[which][ix] += h
+            args_m[which][ix] -= h
+            fd = (loss(*args_p) - loss(*args_m)) / (2 * h)
+            assert abs(fd - grad[ix]) <= 1e-9 * max(1.0, abs(grad[ix])), (which, ix)
