@@ -275,6 +275,46 @@ LASP_API int lasp_wait_probe(void* stream);
 /* Library version, major * 10000 + minor * 100 + patch. */
 LASP_API int lasp_version(void);
 
+/*
+ * Bidirectional (unmasked) linear attention: LASP section 3.1, Eq. 3 as the
+ * right product O = Q (K^T V) (no Norm, no decay, no mask); the LASP-2 review
+ * page ("Summary") gives the unmasked variant as: gather every chunk state
+ * M_t, sum them, M_{1:T} = sum_t M_t, and compute Q_t M_{1:T} in every chunk;
+ * the backward pass sums dM_t = Q_t^T dO_t the same way. Per (b, h):
+ *   M = sum_s k_s^T v_s,  o_s = q_s M;
+ *   dM = sum_s q_s^T do_s,  dq_s = do_s M^T,  dk_s = v_s dM^T,  dv_s = k_s dM.
+ * Supported: bf16, d = 128, N a multiple of 128 (LASP_ERR_UNSUPPORTED
+ * otherwise); N = 0 returns LASP_OK without a launch.
+ *
+ * lasp_bidir_workspace_floats -- floats of the workspace each pass needs (0
+ * for unsupported or invalid sizes). Layout: the segment states (internal),
+ * then at lasp_bidir_state_offset the fp32 total state [B, H, d, d] (M after
+ * lasp_bidir_fwd, dM after lasp_bidir_bwd; element [i][j] = sum k_i v_j, resp.
+ * sum q_i do_j), then its bf16 operand tiles (internal).
+ */
+LASP_API int64_t lasp_bidir_workspace_floats(int B, int H, int64_t N, int d, int dtype);
+LASP_API int64_t lasp_bidir_state_offset(int B, int H, int64_t N, int d, int dtype);
+
+/*
+ * lasp_bidir_fwd -- o = q (k^T v) per (b, h).
+ *   q, k, v:  in,  [B, N, H, d] bf16.      o: out, [B, N, H, d] bf16.
+ *   ws:       out, lasp_bidir_workspace_floats(...) floats (16-byte aligned),
+ *             holding M on return; pass it to lasp_bidir_bwd. Required.
+ */
+LASP_API int lasp_bidir_fwd(const void* q, const void* k, const void* v, void* o, int B, int H, int64_t N, int d,
+                            int dtype, float* ws, void* stream);
+
+/*
+ * lasp_bidir_bwd -- gradients of sum(o * dout) for lasp_bidir_fwd.
+ *   q, k, v, dout:  in,  [B, N, H, d] bf16.   dq, dk, dv: out, [B, N, H, d] bf16.
+ *   ws:             in,  the workspace lasp_bidir_fwd filled for the same k, v.
+ *   dws:            out, a second workspace of the same size, holding dM on
+ *                   return. Required.
+ */
+LASP_API int lasp_bidir_bwd(const void* q, const void* k, const void* v, const void* dout, void* dq, void* dk,
+                            void* dv, int B, int H, int64_t N, int d, int dtype, const float* ws, float* dws,
+                            void* stream);
+
 #ifdef __cplusplus
 }
 #endif

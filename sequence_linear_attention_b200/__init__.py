@@ -22,7 +22,8 @@ __all__ = [
     "lasp_chunk_out", "lasp_chunk_grads", "lasp_bwd_noalloc",
     "lasp_state_prefix", "lasp_check_device_status", "lasp_set_wait_limit_ns", "lasp_wait_probe",
     "lasp_status_string", "lasp_version", "lasp_trace_enable", "lasp_trace_read", "lasp_kernel_name",
-    "lasp_segment_tokens",
+    "lasp_segment_tokens", "lasp_bidir_workspace_floats", "lasp_bidir_state_offset", "lasp_bidir_fwd",
+    "lasp_bidir_bwd",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -73,13 +74,19 @@ def _load():
             lib.lasp_kernel_name.argtypes = [I]
             lib.lasp_kernel_name.restype = ctypes.c_char_p
             lib.lasp_segment_tokens.argtypes = [L, I, I, I]
+            lib.lasp_bidir_workspace_floats.argtypes = [I, I, L, I, I]
+            lib.lasp_bidir_workspace_floats.restype = L
+            lib.lasp_bidir_state_offset.argtypes = [I, I, L, I, I]
+            lib.lasp_bidir_state_offset.restype = L
+            lib.lasp_bidir_fwd.argtypes = [P, P, P, P, I, I, L, I, I, P, P]
+            lib.lasp_bidir_bwd.argtypes = [P, P, P, P, P, P, P, I, I, L, I, I, P, P, P]
             lib.lasp_status_string.argtypes = [I]
             lib.lasp_status_string.restype = ctypes.c_char_p
             for f in (lib.lasp_fwd, lib.lasp_bwd, lib.lasp_chunk_states, lib.lasp_chunk_dstates,
                       lib.lasp_chunk_out, lib.lasp_chunk_grads, lib.lasp_bwd_noalloc,
                       lib.lasp_state_prefix, lib.lasp_check_device_status, lib.lasp_set_wait_limit_ns,
                       lib.lasp_wait_probe, lib.lasp_version, lib.lasp_trace_enable, lib.lasp_trace_read,
-                      lib.lasp_segment_tokens):
+                      lib.lasp_segment_tokens, lib.lasp_bidir_fwd, lib.lasp_bidir_bwd):
                 f.restype = I
             _lib = lib
     return _lib
@@ -188,6 +195,30 @@ def lasp_state_prefix(M, Mprefix, decay, C, init=None, total=None, reverse=False
     _check(_load().lasp_state_prefix(_ptr(M), _ptr(Mprefix), _ptr(decay), _ptr(init), _ptr(total),
                                      B, T, H, d, int(C), int(bool(reverse)), _stream(stream, M)),
            "lasp_state_prefix")
+
+
+def lasp_bidir_workspace_floats(B, H, N, d, dtype=LASP_BF16):
+    """Floats of the workspace lasp_bidir_fwd / lasp_bidir_bwd need (0 if unsupported). See lasp.h."""
+    return int(_load().lasp_bidir_workspace_floats(B, H, N, d, dtype))
+
+
+def lasp_bidir_state_offset(B, H, N, d, dtype=LASP_BF16):
+    """Offset (floats) of the fp32 total state [B, H, d, d] inside the workspace. See lasp.h."""
+    return int(_load().lasp_bidir_state_offset(B, H, N, d, dtype))
+
+
+def lasp_bidir_fwd(q, k, v, o, ws, stream=None):
+    """o = q (k^T v) per (b, h), the bidirectional (unmasked) form; ws receives M. See lasp.h."""
+    B, N, H, d, dt = _tokens(q, k, v, o)
+    _check(_load().lasp_bidir_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), B, H, N, d, dt, _ptr(ws),
+                                  _stream(stream, q)), "lasp_bidir_fwd")
+
+
+def lasp_bidir_bwd(q, k, v, dout, dq, dk, dv, ws, dws, stream=None):
+    """dq, dk, dv of sum(o * dout) for lasp_bidir_fwd; dws receives dM. See lasp.h."""
+    B, N, H, d, dt = _tokens(q, k, v, dout, dq, dk, dv)
+    _check(_load().lasp_bidir_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(dout), _ptr(dq), _ptr(dk), _ptr(dv),
+                                  B, H, N, d, dt, _ptr(ws), _ptr(dws), _stream(stream, q)), "lasp_bidir_bwd")
 
 
 def lasp_check_device_status(stream=None, device=None):

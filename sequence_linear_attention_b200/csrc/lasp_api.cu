@@ -30,6 +30,8 @@ enum KernelId : int {
   K_SEG_STATES = 10,    // segment states (tensor cores)
   K_SEG_SCAN = 11,      // prefix / suffix over segments
   K_PROBE = 12,
+  K_BIDIR_TOTAL = 13,   // bidirectional: sum of the segment states
+  K_BIDIR_APPLY = 14,   // bidirectional: token tiles times the total state
   K_COUNT
 };
 
@@ -334,6 +336,8 @@ const char* lasp_kernel_name(int id) {
     case K_SEG_STATES: return "segment_states_tc";
     case K_SEG_SCAN: return "segment_scan";
     case K_PROBE: return "wait_probe";
+    case K_BIDIR_TOTAL: return "bidir_total";
+    case K_BIDIR_APPLY: return "bidir_apply_tc";
     default: return "unknown";
   }
 }
@@ -357,3 +361,81 @@ int lasp_wait_probe(void* stream) {
 }
 
 }  // extern "C"
+
+// ------------------------------------------------ bidirectional (unmasked) form
+namespace {
+int64_t bidir_segments(int64_t N) { return N / walk_segment_tokens(N, 128); }
+}  // namespace
+
+int64_t lasp_bidir_workspace_floats(int B, int H, int64_t N, int d, int dtype) {
+  using namespace lasp;
+  if (lasp::api_detail::check_sizes(B, H, N, d, 1, dtype) || N == 0 || !tc_bidir_ok(dtype, d, N)) return 0;
+  const int64_t s = (int64_t)d * d;
+  return ((int64_t)B * bidir_segments(N) * H + (int64_t)B * H) * s + (int64_t)B * H * s / 2;
+}
+
+int64_t lasp_bidir_state_offset(int B, int H, int64_t N, int d, int dtype) {
+  using namespace lasp;
+  if (lasp::api_detail::check_sizes(B, H, N, d, 1, dtype) || N == 0 || !tc_bidir_ok(dtype, d, N)) return -1;
+  return (int64_t)B * bidir_segments(N) * H * d * d;
+}
+
+namespace {
+// segment states of (a, b) with lambda = 1 into ws, then their sum (fp32 and
+// the bf16 operand tile) behind them
+int bidir_total_state(const void* a, const void* b, int kind, float* ws, int B, int H, int64_t N, int d,
+                      cudaStream_t st) {
+  using namespace lasp;
+  using namespace lasp::api_detail;
+  const int G = walk_segment_tokens(N, 128);
+  const int nseg = (int)(N / G);
+  const int64_t off = (int64_t)B * nseg * H * d * d;
+  int s;
+  if ((s = cuda_status(traced(K_SEG_STATES, st, [&] {
+         return tc_chunk_states_slots(a, b, nullptr, ws, B, H, N, d, G, kind, nseg, 1, 0, st);
+       }))))
+    return s;
+  return cuda_status(traced(K_BIDIR_TOTAL, st, [&] {
+    return bidir_total(ws, ws + off, ws + off + (int64_t)B * H * d * d, B, H, nseg, st);
+  }));
+}
+}  // namespace
+
+int lasp_bidir_fwd(const void* q, const void* k, const void* v, void* o, int B, int H, int64_t N, int d, int dtype,
+                   float* ws, void* stream) {
+  using namespace lasp;
+  using namespace lasp::api_detail;
+  int s = check_sizes(B, H, N, d, 1, dtype);
+  if (s) return s;
+  if (N == 0) return LASP_OK;
+  if (!tc_bidir_ok(dtype, d, N)) return LASP_ERR_UNSUPPORTED;
+  if ((s = check_ptrs({q, k, v, o, ws}, {}))) return s;
+  cudaStream_t st = (cudaStream_t)stream;
+  if ((s = bidir_total_state(k, v, 0, ws, B, H, N, d, st))) return s;
+  const float* tiles = ws + lasp_bidir_state_offset(B, H, N, d, dtype) + (int64_t)B * H * d * d;
+  const int sms = num_sms_current_device();
+  return cuda_status(traced(K_BIDIR_APPLY, st, [&] { return tc_bidir_apply(q, tiles, o, B, H, N, d, 0, sms, st); }));
+}
+
+int lasp_bidir_bwd(const void* q, const void* k, const void* v, const void* dout, void* dq, void* dk, void* dv, int B,
+                   int H, int64_t N, int d, int dtype, const float* ws, float* dws, void* stream) {
+  using namespace lasp;
+  using namespace lasp::api_detail;
+  int s = check_sizes(B, H, N, d, 1, dtype);
+  if (s) return s;
+  if (N == 0) return LASP_OK;
+  if (!tc_bidir_ok(dtype, d, N)) return LASP_ERR_UNSUPPORTED;
+  if ((s = check_ptrs({q, k, v, dout, dq, dk, dv, ws, dws}, {}))) return s;
+  cudaStream_t st = (cudaStream_t)stream;
+  if ((s = bidir_total_state(q, dout, 1, dws, B, H, N, d, st))) return s;
+  const int64_t toff = lasp_bidir_state_offset(B, H, N, d, dtype) + (int64_t)B * H * d * d;
+  const float* m_tiles = ws + toff;
+  const float* dm_tiles = dws + toff;
+  const int sms = num_sms_current_device();
+  // dQ = dO M^T, dK = V dM^T, dV = K dM
+  if ((s = cuda_status(traced(K_BIDIR_APPLY, st, [&] { return tc_bidir_apply(dout, m_tiles, dq, B, H, N, d, 1, sms, st); }))))
+    return s;
+  if ((s = cuda_status(traced(K_BIDIR_APPLY, st, [&] { return tc_bidir_apply(v, dm_tiles, dk, B, H, N, d, 1, sms, st); }))))
+    return s;
+  return cuda_status(traced(K_BIDIR_APPLY, st, [&] { return tc_bidir_apply(k, dm_tiles, dv, B, H, N, d, 0, sms, st); }));
+}

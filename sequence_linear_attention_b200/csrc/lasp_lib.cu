@@ -8,4 +8,5 @@
 #include "k_tc_fwd_walk.cu"
 #include "k_tc_bwd.cu"
 #include "k_tc_bwd_walk.cu"
+#include "k_tc_bidir.cu"
 #include "lasp_noalloc.cu"

@@ -51,4 +51,13 @@ cudaError_t tc_chunk_bwd(const void* q, const void* k, const void* v, const void
                          const float* P, const float* Rs, void* dq, void* dk, void* dv, int B, int H, int64_t N,
                          int d, int C, cudaStream_t st);
 
+// Bidirectional (unmasked) form, bf16, d = 128, N a multiple of 128
+// (k_tc_bidir.cu): the fp32 sum of nseg segment states of each (b, h) and its
+// bf16 operand tile; and Y = X S (b_kmajor = 0) or X S^T (b_kmajor = 1) per
+// 128-token tile of X with S the (b, h)'s tile.
+bool tc_bidir_ok(int dtype, int d, int64_t N);
+cudaError_t bidir_total(const float* seg, float* total, void* tiles, int B, int H, int nseg, cudaStream_t st);
+cudaError_t tc_bidir_apply(const void* x, const void* stiles, void* y, int B, int H, int64_t N, int d, int b_kmajor,
+                           int num_sms, cudaStream_t st);
+
 }  // namespace lasp

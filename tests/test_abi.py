@@ -115,3 +115,24 @@ def test_binding_marshals_only(lib):
     for forbidden in ("oracle", "einsum", "matmul", "cumsum", "@"):
         assert forbidden not in src.replace("@property", ""), forbidden
     assert ctypes.CDLL(lasp.library_path())
+
+
+def test_bidir_rejects_bad_arguments(lib):
+    f = lib.lasp_bidir_fwd
+    assert f(A, A, A, A, 1, 2, 256, 64, BF16, A, None) == UNSUPPORTED      # d = 64
+    assert f(A, A, A, A, 1, 2, 256, 128, F32, A, None) == UNSUPPORTED      # fp32
+    assert f(A, A, A, A, 1, 2, 200, 128, BF16, A, None) == UNSUPPORTED     # N not a multiple of 128
+    assert f(A, A, A, A, 0, 2, 256, 128, BF16, A, None) == INVALID
+    assert f(A, A, A, A, 1, 2, 0, 128, BF16, None, None) == OK             # nothing to do
+    assert f(A, A, A, A, 1, 2, 256, 128, BF16, None, None) == INVALID      # no workspace
+    assert f(A, A, A + 8, A, 1, 2, 256, 128, BF16, A, None) == MISALIGNED
+    g = lib.lasp_bidir_bwd
+    assert g(A, A, A, A, A, A, A, 1, 2, 256, 128, BF16, A, None, None) == INVALID
+    assert g(A, A, A, A, A, A, A, 1, 2, 256, 32, BF16, A, A, None) == UNSUPPORTED
+    assert lasp.lasp_bidir_workspace_floats(1, 2, 256, 64) == 0
+    assert lasp.lasp_bidir_state_offset(1, 2, 256, 64) == -1
+    # segment states, then the [B, H, d, d] total, then its bf16 tiles
+    n = lasp.lasp_bidir_workspace_floats(2, 3, 2048, 128)
+    off = lasp.lasp_bidir_state_offset(2, 3, 2048, 128)
+    assert off == 2 * 2 * 3 * 128 * 128   # two 1024-token segments
+    assert n == off + 2 * 3 * 128 * 128 + 2 * 3 * 128 * 128 // 2
