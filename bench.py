@@ -65,6 +65,9 @@ def algorithmic_bytes(name: str, tokens_heads: int, d: int, C: int, G: int, elem
         "chunk_out_tc": 4 * de + s / C, "chunk_out_simt": 4 * de + s / C, "fwd_walk_tc": 4 * de + (s / G + s / 256 if C <= 128 else s / C),
         "chunk_bwd_tc": 7 * de + 2 * s / C, "chunk_bwd_simt": 7 * de + 2 * s / C,
         "bwd_walk_tc": 7 * de + s / 256 + s / G,
+        # bidirectional form: the sum of the segment states (s/G; the total and
+        # its tile per (b, h) are negligible), and one token tensor in, one out
+        "bidir_total": s / G, "bidir_apply_tc": 2 * de,
     }[name]
     return per * tokens_heads
 
@@ -351,6 +354,82 @@ def run_gpu(args, rank, world, local):
     return line
 
 
+def run_bidir(args, rank, world, local):
+    """The bidirectional (unmasked) form on the workload's shapes (its decay is
+    not used): a step is lasp_bidir_fwd + lasp_bidir_bwd. Printed as its own
+    line, with its own metric; the default run does not include it."""
+    import torch
+    import sequence_linear_attention_b200 as lasp
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    w = lasp_inputs.WORKLOADS[args.workload]
+    B, N, H, d = w["B"], (args.tokens or w["N"]), w["H"], w["d"]
+    if not w["bf16"] or lasp.lasp_bidir_workspace_floats(B, H, N, d) == 0:
+        raise ValueError("the bidirectional form needs a bf16 workload with d = 128 and N a multiple of 128")
+    inp = lasp_inputs.make_inputs(B, N, H, d, seed=w["seed"] + 7919 * rank, bf16=True, decayed=False)
+    q, k, v, do = (torch.from_numpy(np.ascontiguousarray(inp[n]).view(np.int16)).view(torch.bfloat16).to(dev)
+                   for n in ("q", "k", "v", "do"))
+    o, dq, dk, dv = (torch.empty_like(q) for _ in range(4))
+    ws = torch.empty(lasp.lasp_bidir_workspace_floats(B, H, N, d), dtype=torch.float32, device=dev)
+    dws = torch.empty_like(ws)
+    stream = torch.cuda.current_stream(dev)
+    G = lasp.lasp_segment_tokens(N, 128, d, 1)
+
+    def step():
+        lasp.lasp_bidir_fwd(q, k, v, o, ws)
+        lasp.lasp_bidir_bwd(q, k, v, do, dq, dk, dv, ws, dws)
+
+    for _ in range(args.warmup):
+        step()
+    events = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    torch.cuda.synchronize(dev)
+    barrier(world, dev)
+    with ClockSampler(local) as clk:
+        for i in range(args.steps):
+            events[i][0].record(stream)
+            step()
+            events[i][1].record(stream)
+        torch.cuda.synchronize(dev)
+    barrier(world, dev)
+    tokens = B * N
+    value, t_max = aggregate(tokens * args.steps, sum(a.elapsed_time(b) for a, b in events) / 1e3, world, dev)
+    ksteps = min(args.steps, 200)
+    lasp.lasp_trace_enable(16 * ksteps + 16)
+    for _ in range(ksteps):
+        step()
+    torch.cuda.synchronize(dev)
+    trace = lasp.lasp_trace_read(16 * ksteps + 16)
+    lasp.lasp_trace_enable(0)
+    st, site = lasp.lasp_check_device_status()
+    if st != 0:
+        raise RuntimeError(f"device status {lasp.lasp_status_string(st)} at site {site}")
+    per_kernel = {}
+    for name, ms in trace:
+        per_kernel.setdefault(name, []).append(ms)
+    peaks = load_peaks()
+    th = tokens * H
+    kernel_table = {}
+    for n, ms in per_kernel.items():
+        mean = statistics.mean(ms)
+        gbps = algorithmic_bytes(n, th, d, 128, G, 2) / (mean / 1e3) / 1e9
+        kernel_table[n] = {"launches_per_step": len(ms) / ksteps, "ms": round(mean, 4), "GBps": round(gbps, 1),
+                           "hbm_frac": round(gbps / peaks["hbm"], 4)}
+    top = max(per_kernel, key=lambda n: sum(per_kernel[n]))
+    return {
+        "metric": "bidirectional linear-attn fwd+bwd tokens/s", "impl": "bidirectional",
+        "value": round(value, 1), "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(t_max * 1e3 / args.steps, 4), "higher_is_better": True,
+        "dtype": "bf16", "data": "synthetic (seeded normal q,k,v,dO; no dataset)",
+        "config": {"workload": args.workload, "B": B, "H": H, "N": N, "d": d, "segment": G, "decay": "none"},
+        "roofline": {"bound": "hbm", "kernel": top, "achieved": kernel_table[top]["GBps"], "peak": peaks["hbm"],
+                     "unit": "GB/s", "frac": kernel_table[top]["hbm_frac"], "peak_source": peaks["source"]},
+        "kernels": kernel_table,
+        "gpu_launches": int(round(len(trace) / ksteps * args.steps)),
+        "clocks": clk.summary(),
+    }
+
+
 # ------------------------------------------------------------------ CPU oracle
 def oracle_sample(args, tokens: int):
     """A bounded sample of the workload for the fp64 oracle: all heads, the
@@ -416,6 +495,8 @@ def main(argv=None):
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(lasp_inputs.WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--bidir", action="store_true",
+                    help="time the bidirectional (unmasked) form instead (its own metric and line)")
     ap.add_argument("--tokens", type=int, default=None,
                     help="sequence length N instead of the workload's (a smaller case of the same shape, for "
                          "profiling); the line is then not the workload's headline number")
@@ -426,6 +507,8 @@ def main(argv=None):
     try:
         if args.impl == "reference":
             line = run_reference(args, rank, world)
+        elif args.bidir:
+            line = run_bidir(args, rank, world, local)
         else:
             line = run_gpu(args, rank, world, local)
             if rank == 0 and world == 1 and not args.no_cpu_baseline:

@@ -30,34 +30,44 @@ constexpr uint32_t kTileBytes = kTile * kD * 2;  // 32 KB: two 64-feature boxes
 constexpr uint32_t kBox = kTileBytes / 2;
 
 // ------------------------------------------------------------------ totals
-// One thread per float4 of a d x d state: total = sum over the nseg segment
-// states of (b, h), in segment order, written as fp32 and as the bf16 operand
-// tile (two 64-column boxes of 128 rows, 128-byte swizzled: element (r, c)
-// sits in box c / 64, row r, 16-byte chunk ((c % 64) / 8) ^ (r % 8)).
-constexpr int kTotalThreads = 256;
+// total = sum over the nseg segment states of (b, h), written as fp32 and as
+// the bf16 operand tile (two 64-column boxes of 128 rows, 128-byte swizzled:
+// element (r, c) sits in box c / 64, row r, 16-byte chunk ((c % 64) / 8) ^
+// (r % 8)). A block takes 32 float4s of the state; its four warps sum a
+// quarter of the segments each (eight loads in flight per thread), and the
+// four partial sums are added in a fixed order, so the result does not depend
+// on timing.
+constexpr int kTotalThreads = 128;
+constexpr int kTotalCols = 32;  // float4s of the state per block
 
 __global__ void __launch_bounds__(kTotalThreads) bidir_total(const float4* __restrict__ seg, float4* __restrict__ total,
                                                             uint8_t* __restrict__ tiles, int H, int nseg) {
+  __shared__ float4 part[kTotalThreads / kTotalCols][kTotalCols];
   const int bh = blockIdx.y;  // b * H + h
   const int b = bh / H, h = bh % H;
-  const int e4 = blockIdx.x * kTotalThreads + threadIdx.x;  // float4 index in the state
+  const int col = threadIdx.x % kTotalCols, grp = threadIdx.x / kTotalCols;
+  const int e4 = blockIdx.x * kTotalCols + col;  // float4 index in the state
   constexpr int kPer = kD * kD / 4;
-  if (e4 >= kPer) return;
+  constexpr int kGroups = kTotalThreads / kTotalCols;
   const int64_t step = (int64_t)H * kPer;  // float4s from one segment slot to the next
   const float4* p = seg + ((int64_t)b * nseg * H + h) * kPer + e4;
-  float4 a[4] = {};
-  int g = 0;
-  for (; g + 4 <= nseg; g += 4) {
+  const int per = (nseg + kGroups - 1) / kGroups;
+  const int g0 = grp * per, g1 = g0 + per < nseg ? g0 + per : nseg;
+  float4 a[8] = {};
+  int g = g0;
+  for (; g + 8 <= g1; g += 8) {
+    float4 x[8];
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const float4 x = __ldcs(p + (g + u) * step);
-      a[u].x += x.x;
-      a[u].y += x.y;
-      a[u].z += x.z;
-      a[u].w += x.w;
+    for (int u = 0; u < 8; ++u) x[u] = __ldcs(p + (g + u) * step);
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      a[u].x += x[u].x;
+      a[u].y += x[u].y;
+      a[u].z += x[u].z;
+      a[u].w += x[u].w;
     }
   }
-  for (; g < nseg; ++g) {
+  for (; g < g1; ++g) {
     const float4 x = __ldcs(p + g * step);
     a[0].x += x.x;
     a[0].y += x.y;
@@ -65,10 +75,20 @@ __global__ void __launch_bounds__(kTotalThreads) bidir_total(const float4* __res
     a[0].w += x.w;
   }
   float4 s;
-  s.x = (a[0].x + a[1].x) + (a[2].x + a[3].x);
-  s.y = (a[0].y + a[1].y) + (a[2].y + a[3].y);
-  s.z = (a[0].z + a[1].z) + (a[2].z + a[3].z);
-  s.w = (a[0].w + a[1].w) + (a[2].w + a[3].w);
+  s.x = ((a[0].x + a[1].x) + (a[2].x + a[3].x)) + ((a[4].x + a[5].x) + (a[6].x + a[7].x));
+  s.y = ((a[0].y + a[1].y) + (a[2].y + a[3].y)) + ((a[4].y + a[5].y) + (a[6].y + a[7].y));
+  s.z = ((a[0].z + a[1].z) + (a[2].z + a[3].z)) + ((a[4].z + a[5].z) + (a[6].z + a[7].z));
+  s.w = ((a[0].w + a[1].w) + (a[2].w + a[3].w)) + ((a[4].w + a[5].w) + (a[6].w + a[7].w));
+  part[grp][col] = s;
+  __syncthreads();
+  if (grp != 0) return;
+#pragma unroll
+  for (int q = 1; q < kGroups; ++q) {
+    s.x += part[q][col].x;
+    s.y += part[q][col].y;
+    s.z += part[q][col].z;
+    s.w += part[q][col].w;
+  }
   total[(int64_t)bh * kPer + e4] = s;
   const int r = (e4 * 4) / kD, c = (e4 * 4) % kD;
   const int cb = c & 63;
@@ -285,7 +305,7 @@ bool tc_bidir_ok(int dtype, int d, int64_t N) {
 
 cudaError_t bidir_total(const float* seg, float* total, void* tiles, int B, int H, int nseg, cudaStream_t st) {
   using namespace tc_bidir_detail;
-  dim3 grid((kD * kD / 4 + kTotalThreads - 1) / kTotalThreads, (unsigned)(B * H));
+  dim3 grid(kD * kD / 4 / kTotalCols, (unsigned)(B * H));
   bidir_total<<<grid, kTotalThreads, 0, st>>>(reinterpret_cast<const float4*>(seg), reinterpret_cast<float4*>(total),
                                              static_cast<uint8_t*>(tiles), H, nseg);
   return cudaGetLastError();
