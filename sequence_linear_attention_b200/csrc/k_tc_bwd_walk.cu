@@ -13,10 +13,11 @@
 // by one warp and the epilogues run by eight others:
 //
 //   MMA 1:  T0 = dO V^T,  T1 = Q K^T  | T2 = dO P^T
-//   epi 1:  V <- diag(lambda^{127-j}) V;  dP' = Mask . T0 -> A,  S' = Mask . T1 -> B
+//   epi 1:  dP' = Mask . T0 -> A,  S' = Mask . T1 -> B
 //   MMA 2:  T0 = dP' K                 | T1 = S'^T dO
-//   epi 2:  (under MMA 2) R -> bf16 X (replacing P), R <- lambda^128 R in TMEM;
-//           dQ = T0 + lambda^{i+1} T2 -> over S' (TMA store)
+//   epi 2:  (under MMA 2) V <- diag(lambda^{127-j}) V;  R -> bf16 X (replacing
+//           P), R <- lambda^128 R in TMEM;  dQ = T0 + lambda^{i+1} T2 -> over S'
+//           (TMA store)
 //   MMA 3:  T0 = V~ R^T,  T2 = K R    | T0 += dP'^T Q (dK)
 //   epi 3:  (under MMA 3) dO <- diag(lambda^{j+1}) dO;
 //   MMA 4:  R += Q^T dO~               (the state for chunk c - 1)
@@ -427,14 +428,12 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_walk_tc(
           ++nseg_done;
           named_sync(kEpiBar, kEpiThreads);  // all of R is read before the pair is rewritten
         }
-        // V~ = diag(lambda^{127-j}) V once MMA 1 has read V
-        wait(&s->c1, par, SITE_BWD_MMA);
-        tc_fence_after();
-        if (scale) scale_rows(sV, s->pw, true, 1.f, tid);
         // dP' = Mask . T0 and S' = Mask . T1 into the buffers the previous
         // chunk's dK and dV stores have left
         wait(&s->free_a, par, SITE_BWD_TMA);
         wait(&s->free_b, par, SITE_BWD_TMA);
+        wait(&s->c1, par, SITE_BWD_MMA);
+        tc_fence_after();
 #pragma unroll 1
         for (int cc = 2 * half; cc < 2 * half + 2; ++cc) {
           if (cc > (warp & 3)) {
@@ -477,8 +476,10 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_walk_tc(
         tc_fence_before();
         mbar_arrive(&s->e1);
 
-        // R of this chunk -> bf16 X (once dO P^T has read P), pre-scaled by
-        // lambda^128 for MMA 4, while MMA 2 runs
+        // while MMA 2 runs: V~ = diag(lambda^{127-j}) V (MMA 1 has read V), and R
+        // of this chunk -> bf16 X (once dO P^T has read P), pre-scaled by
+        // lambda^128 for MMA 4
+        if (scale) scale_rows(sV, s->pw, true, 1.f, tid);
         wait(&s->c1b, par, SITE_BWD_MMA);
         tc_fence_after();
         {
