@@ -301,11 +301,13 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_walk_tc(
           if (!(ok = mbar_wait_or_abort(&s->c3a, par, SITE_BWD_MMA, abort_flag))) break;
           if (has_next) {
             load_kv(nx, nt);
-            load_p(nx, nt);
           }
           if (!(ok = mbar_wait_or_abort(&s->c3, par, SITE_BWD_MMA, abort_flag))) break;
           tma_store_wait_read0();
-          if (has_next) load_qd(nx, nt, par ^ 1u);
+          if (has_next) {
+            load_qd(nx, nt, par ^ 1u);
+            load_p(nx, nt);  // last: only the third GEMM of MMA 1 reads it
+          }
           prev = item;
           prev_row = row0;
         }
@@ -334,14 +336,15 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_walk_tc(
           // MMA 1 needs this chunk's loads, and TMEM 0-2 drained by the previous epilogue 3
           ok = mbar_wait_or_abort(&s->ld_kv, par, SITE_BWD_TMA, abort_flag) &&
                mbar_wait_or_abort(&s->ld_qd, par, SITE_BWD_TMA, abort_flag) &&
-               mbar_wait_or_abort(&s->ld_p, par, SITE_BWD_TMA, abort_flag) &&
                (it == 0 || mbar_wait_or_abort(&s->e0, (it - 1) & 1u, SITE_BWD_MMA, abort_flag));
           if (!ok) break;
           tc_fence_after();
-          // ---- MMA 1: T0 = dO V^T, T1 = Q K^T | T2 = dO P^T
+          // ---- MMA 1: T0 = dO V^T, T1 = Q K^T | T2 = dO P^T (P's tile is loaded last)
           for (int kk = 0; kk < kD / 16; ++kk) mma_bf16(tmem + T0, kmaj(aD, kk), kmaj(aV, kk), id_kk, kk != 0);
           for (int kk = 0; kk < kD / 16; ++kk) mma_bf16(tmem + T1, kmaj(aQ, kk), kmaj(aK, kk), id_kk, kk != 0);
           mma_commit(&s->c1);
+          if (!(ok = mbar_wait_or_abort(&s->ld_p, par, SITE_BWD_TMA, abort_flag))) break;
+          tc_fence_after();
           for (int kk = 0; kk < kD / 16; ++kk) mma_bf16(tmem + T2, kmaj(aD, kk), kmaj(aX, kk), id_kk, kk != 0);
           mma_commit(&s->c1b);
           // ---- MMA 2: T0 = dP' K | T1 = S'^T dO
