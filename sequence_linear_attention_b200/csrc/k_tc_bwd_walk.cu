@@ -30,9 +30,9 @@
 // keep fp32 row scalings. Two pairs of tile buffers trade roles from chunk to
 // chunk: one holds the chunk's Q and dO and then its outgoing dK and dV, the
 // other its dP' and S' (and dQ) and then the next chunk's Q and dO, which are
-// loaded as soon as dQ has left and dP'^T Q is done. The next K, V and P go
-// in once the first part of MMA 3 is done. R is not stored per chunk: only the segment-level
-// slots of the workspace are used. In every epilogue warp w owns TMEM lanes
+// loaded as soon as dQ has left and dP'^T Q is done, followed by P's cache
+// tile; the next K and V go in once the first part of MMA 3 is done. R is not
+// stored per chunk: only the segment-level slots of the workspace are used. In every epilogue warp w owns TMEM lanes
 // (rows) 32*(w%4).. and the column half w/4.
 #include <algorithm>
 
