@@ -22,6 +22,13 @@ namespace scan_detail {
 constexpr int kUnroll = 8;
 constexpr int kThreads = 64;  // small blocks spread the work evenly over the SMs
 
+// store that asks L2 to keep the line (the walk reads P next)
+__device__ __forceinline__ void st_keep(float4* p, float4 v, uint64_t policy) {
+  asm volatile("st.global.L2::cache_hint.v4.f32 [%0], {%1, %2, %3, %4}, %5;" ::"l"(p), "f"(v.x), "f"(v.y), "f"(v.z),
+               "f"(v.w), "l"(policy)
+               : "memory");
+}
+
 __device__ __forceinline__ float4 fma4(float g, float4 a, float4 m) {
   return make_float4(fmaf(g, a.x, m.x), fmaf(g, a.y, m.y), fmaf(g, a.z, m.z), fmaf(g, a.w, m.w));
 }
@@ -38,6 +45,8 @@ __global__ void __launch_bounds__(kThreads) state_scan_kernel(const float4* M, f
   const int h = (int)((idx / dd4) % H);
   const int64_t b = idx / ((int64_t)dd4 * H);
   const float g = decay_pow(log2f(load_decay(decay, h)), Cf);
+  uint64_t keep;
+  asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(keep));
   const int64_t bh = b * H + h;
   float4 acc = init ? init[bh * dd4 + e] : make_float4(0.f, 0.f, 0.f, 0.f);
   // scan element c lives in slot c * slot_stride + slot_offset of an array of t_slots states
@@ -62,7 +71,7 @@ __global__ void __launch_bounds__(kThreads) state_scan_kernel(const float4* M, f
     }
 #pragma unroll
     for (int u = 0; u < kUnroll; ++u) {
-      __stcs(P + off + u * step, acc);
+      st_keep(P + off + u * step, acc, keep);
       acc = fma4(g, acc, cur[u]);
     }
     off += kUnroll * step;
@@ -74,7 +83,7 @@ __global__ void __launch_bounds__(kThreads) state_scan_kernel(const float4* M, f
   int n = ngroups * kUnroll;
   for (; n < T; ++n) {
     float4 m = __ldcs(M + off);
-    __stcs(P + off, acc);
+    st_keep(P + off, acc, keep);
     acc = fma4(g, acc, m);
     off += step;
   }

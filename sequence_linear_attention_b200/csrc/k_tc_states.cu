@@ -124,6 +124,9 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_states_tc(const __grid_cons
   if (warp == 1) {
     // ---------------------------------------------------------------- TMA
     if (lane == 0) {
+      // the token tiles stream through once; the states written below stay in
+      // L2 for the scan that reads them next
+      const uint64_t stream_policy = l2_evict_first();
       for (int64_t g = 0; g < nstream && !aborted(&s->abort); ++g) {
         const int slot = (int)(g % nslots);
         const int64_t u = g / nslots;
@@ -136,10 +139,10 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_states_tc(const __grid_cons
         uint8_t* a = tiles + (size_t)slot * 2 * tile_bytes;
         uint8_t* bb = a + tile_bytes;
         mbar_arrive_expect_tx(&s->full[slot], 2 * tile_bytes);
-        tma_load_4d(a, &map_a, &s->full[slot], 0, wk.h, row, wk.b);
-        tma_load_4d(a + tile_bytes / 2, &map_a, &s->full[slot], 64, wk.h, row, wk.b);
-        tma_load_4d(bb, &map_b, &s->full[slot], 0, wk.h, row, wk.b);
-        tma_load_4d(bb + tile_bytes / 2, &map_b, &s->full[slot], 64, wk.h, row, wk.b);
+        tma_load_4d_hint(a, &map_a, &s->full[slot], 0, wk.h, row, wk.b, stream_policy);
+        tma_load_4d_hint(a + tile_bytes / 2, &map_a, &s->full[slot], 64, wk.h, row, wk.b, stream_policy);
+        tma_load_4d_hint(bb, &map_b, &s->full[slot], 0, wk.h, row, wk.b, stream_policy);
+        tma_load_4d_hint(bb + tile_bytes / 2, &map_b, &s->full[slot], 64, wk.h, row, wk.b, stream_policy);
       }
     }
   } else if (warp == 0) {
@@ -251,7 +254,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_states_tc(const __grid_cons
           fence_async_smem();
           __syncwarp();
           if (lane == 0) {
-            tma_store_2d(&map_m, stage_out, (2 * colhalf + cb) * 32, y);
+            tma_store_2d_hint(&map_m, stage_out, (2 * colhalf + cb) * 32, y, l2_evict_last());
             tma_store_commit();
           }
         }
