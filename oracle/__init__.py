@@ -23,6 +23,11 @@ it with ctypes. Each wrapper states the passage it follows:
   LASP page, section 3.1, Eq. 3 right product Q (K^T V) without Norm; LASP-2
   review page, "Summary": the unmasked variant gathers all chunk states and
   every chunk computes Q_t M_{1:T}, and the backward the same with dM.
+* :func:`gla_fwd`, :func:`gla_bwd`, :func:`gla_chunk_states`,
+  :func:`gla_state_scan`, :func:`gla_state_snapshots` -- the gated form (a
+  decay per token and key feature): LASP page, Appendix A.4, Eq. 24 with the
+  GLA / GateLoop row of Table 5 (oscillation g_t 1^T), the gate passed as its
+  natural log; gradients by the chain rule on that recurrence.
 
 Inputs are float32 arrays shaped [B, N, H, d] (any strides, feature axis
 contiguous). Values that came from bf16 are exact in float32 and double, so the
@@ -74,10 +79,18 @@ def _load():
             lib.oracle_bidir_fwd.argtypes = [_P, _P, _P, _L, _L, _L, _P, _L, _L, _L, _P, _I, _L, _I, _I]
             lib.oracle_bidir_bwd.argtypes = [_P, _P, _P, _P, _L, _L, _L, _P, _P, _P, _L, _L, _L, _P,
                                              _I, _L, _I, _I]
+            lib.oracle_gla_fwd.argtypes = [_P, _P, _P, _P, _L, _L, _L, _P, _P, _L, _L, _L, _P, _I, _L, _I, _I]
+            lib.oracle_gla_bwd.argtypes = [_P, _P, _P, _P, _P, _L, _L, _L, _P, _P,
+                                           _P, _P, _P, _P, _L, _L, _L, _P, _I, _L, _I, _I]
+            lib.oracle_gla_chunk_states.argtypes = [_P, _P, _P, _L, _L, _L, _P, _P, _I, _L, _I, _I, _L, _I]
+            lib.oracle_gla_state_scan.argtypes = [_P, _P, _P, _P, _P, _I, _L, _I, _I, _I]
+            lib.oracle_gla_state_snapshots.argtypes = [_P, _P, _P, _L, _L, _L, _P, _P, _I, _L, _I, _I, _L, _I]
             lib.oracle_num_threads.restype = _I
             for f in (lib.oracle_fwd, lib.oracle_bwd, lib.oracle_chunk_states,
                       lib.oracle_state_scan, lib.oracle_state_snapshots, lib.oracle_bidir_fwd,
-                      lib.oracle_bidir_bwd):
+                      lib.oracle_bidir_bwd, lib.oracle_gla_fwd, lib.oracle_gla_bwd,
+                      lib.oracle_gla_chunk_states, lib.oracle_gla_state_scan,
+                      lib.oracle_gla_state_snapshots):
                 f.restype = None
             _lib = lib
     return _lib
@@ -246,3 +259,99 @@ def bidir_bwd(q, k, v, do, want_state=False):
     _load().oracle_bidir_bwd(pq, k.ctypes.data, v.ctypes.data, do.ctypes.data, sb, sn, sh, dq.ctypes.data,
                              dk.ctypes.data, dv.ctypes.data, N * H * d, H * d, d, _ptr(dM), B, N, H, d)
     return (dq, dk, dv, dM) if want_state else (dq, dk, dv)
+
+
+# ------------------------------------------------------------------ gated form
+def gla_fwd(q, k, v, g, init=None, want_final=False):
+    """Gated recurrence (LASP Appendix A.4, Eq. 24; Table 5, GLA / GateLoop):
+    S_s = diag(exp(g_s)) S_{s-1} + k_s^T v_s, o_s = q_s S_s.
+
+    ``g``: float32 [B, N, H, d], the natural log of the gate of each token and
+    key feature (same shape and strides as q). ``init``: [B, H, d, d] or None.
+    Returns o (float64 [B, N, H, d]) and, if ``want_final``, the last state.
+    """
+    B, N, H, d = q.shape
+    pq, sb, sn, sh = _view(q)
+    for t in (k, v, g):
+        _view(t, q)
+    ia, pi = _state(init, (B, H, d, d))
+    o = np.empty((B, N, H, d), np.float64)
+    fin = np.empty((B, H, d, d), np.float64) if want_final else None
+    _load().oracle_gla_fwd(pq, k.ctypes.data, v.ctypes.data, g.ctypes.data, sb, sn, sh, pi,
+                           o.ctypes.data, N * H * d, H * d, d, _ptr(fin), B, N, H, d)
+    return (o, fin) if want_final else o
+
+
+def gla_bwd(q, k, v, g, do, init=None, dstate_in=None, want_dinit=False):
+    """Gradients of sum(o * do) for :func:`gla_fwd` by the chain rule on the
+    recurrence: dq, dk, dv and dg (the gradient with respect to the log-gate),
+    all float64 [B, N, H, d], and, if ``want_dinit``, the gradient with
+    respect to ``init``. ``dstate_in``: [B, H, d, d] gradient with respect to
+    the state after the last token (0 if None).
+    """
+    B, N, H, d = q.shape
+    pq, sb, sn, sh = _view(q)
+    for t in (k, v, g, do):
+        _view(t, q)
+    ia, pi = _state(init, (B, H, d, d))
+    fa, pf = _state(dstate_in, (B, H, d, d))
+    dq = np.empty((B, N, H, d), np.float64)
+    dk = np.empty_like(dq)
+    dv = np.empty_like(dq)
+    dg = np.empty_like(dq)
+    dinit = np.empty((B, H, d, d), np.float64) if want_dinit else None
+    _load().oracle_gla_bwd(pq, k.ctypes.data, v.ctypes.data, g.ctypes.data, do.ctypes.data, sb, sn, sh, pi, pf,
+                           dq.ctypes.data, dk.ctypes.data, dv.ctypes.data, dg.ctypes.data, N * H * d, H * d, d,
+                           _ptr(dinit), B, N, H, d)
+    return (dq, dk, dv, dg, dinit) if want_dinit else (dq, dk, dv, dg)
+
+
+def gla_chunk_states(x, y, g, C, kind=0):
+    """Gated per-chunk states [B, T, H, d, d] and chunk log-gate totals
+    [B, T, H, d], from their definition.
+
+    kind 0, (x, y) = (k, v): M_c = sum_t diag(exp(sum of g over t+1..C-1)) x_t^T y_t.
+    kind 1, (x, y) = (q, do): M_c = sum_t diag(exp(sum of g over 0..t)) x_t^T y_t.
+    """
+    B, N, H, d = x.shape
+    if N % C:
+        raise ValueError("C must divide N")
+    px, sb, sn, sh = _view(x)
+    _view(y, x), _view(g, x)
+    M = np.empty((B, N // C, H, d, d), np.float64)
+    gs = np.empty((B, N // C, H, d), np.float64)
+    _load().oracle_gla_chunk_states(px, y.ctypes.data, g.ctypes.data, sb, sn, sh, M.ctypes.data, gs.ctypes.data,
+                                    B, N, H, d, C, kind)
+    return M, gs
+
+
+def gla_state_scan(M, gsum, init=None, reverse=False):
+    """Exclusive scan over gated chunk states; a step through chunk c scales
+    row i by exp(gsum[c, i]). Returns (P, total) in float64 (see the C file)."""
+    M = np.ascontiguousarray(np.asarray(M, dtype=np.float64))
+    B, T, H, d, _ = M.shape
+    gs = np.ascontiguousarray(np.asarray(gsum, dtype=np.float64))
+    if gs.shape != (B, T, H, d):
+        raise ValueError("gsum must be [B, T, H, d]")
+    ia, pi = _state(init, (B, H, d, d))
+    P = np.empty_like(M)
+    tot = np.empty((B, H, d, d), np.float64)
+    _load().oracle_gla_state_scan(M.ctypes.data, gs.ctypes.data, P.ctypes.data, pi, tot.ctypes.data,
+                                  B, T, H, d, int(bool(reverse)))
+    return P, tot
+
+
+def gla_state_snapshots(x, y, g, C, init=None, kind=0):
+    """Chunk-boundary states of the gated recurrences, [B, T, H, d, d]:
+    kind 0 (k, v): the state entering each chunk; kind 1 (q, do): the gradient
+    state each chunk receives from the tokens after it (``init`` = dstate_in)."""
+    B, N, H, d = x.shape
+    if N % C:
+        raise ValueError("C must divide N")
+    px, sb, sn, sh = _view(x)
+    _view(y, x), _view(g, x)
+    ia, pi = _state(init, (B, H, d, d))
+    P = np.empty((B, N // C, H, d, d), np.float64)
+    _load().oracle_gla_state_snapshots(px, y.ctypes.data, g.ctypes.data, sb, sn, sh, pi, P.ctypes.data,
+                                       B, N, H, d, C, kind)
+    return P

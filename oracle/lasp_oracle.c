@@ -399,3 +399,325 @@ void oracle_bidir_bwd(const float *q, const float *k, const float *v, const floa
     free(G);
   }
 }
+
+/* ------------------------------------------------------------------------
+ * Gated form: a decay that depends on the token and the key feature.
+ * LASP page, Appendix A.4, Eq. 24, m_t = o_t m_{t-1} + e_t i_t^T, with the
+ * GLA / GateLoop row of Table 5: expand state e_t = k_t, input i_t = v_t,
+ * shrink state s_t = q_t, memory k x d, and oscillation g_t 1^T, a gate per
+ * key feature that scales row i of the memory (elementwise product).  The gate
+ * is passed as its natural log a_t[i] (float [B, N, H, d], the same view as
+ * q), so that
+ *     S_s[i][j] = exp(a_s[i]) S_{s-1}[i][j] + k_s[i] v_s[j],
+ *     o_s[j]    = sum_i q_s[i] S_s[i][j].
+ * With a_s[i] = log(lambda) everywhere this is oracle_fwd's recurrence.
+ * Task = (b, h, block of S columns): column j of o only needs column j of S.
+ * init / final_state as in oracle_fwd.
+ */
+void oracle_gla_fwd(const float *q, const float *k, const float *v, const float *a,
+                    long sb, long sn, long sh, const double *init,
+                    double *o, long ob, long on, long oh,
+                    double *final_state, int B, long N, int H, int d) {
+  int nblk = (d + BLK - 1) / BLK;
+  long ntask = (long)B * H * nblk;
+#pragma omp parallel for schedule(dynamic, 1)
+  for (long task = 0; task < ntask; ++task) {
+    int blk = (int)(task % nblk);
+    int h = (int)((task / nblk) % H);
+    int b = (int)(task / ((long)nblk * H));
+    int j0 = blk * BLK, j1 = j0 + BLK < d ? j0 + BLK : d;
+    double *S = (double *)calloc((size_t)d * d, sizeof(double));
+    if (init) memcpy(S, st_bh(init, H, d, b, h), sizeof(double) * d * d);
+    for (long s = 0; s < N; ++s) {
+      const float *qs = tok(q, sb, sn, sh, b, s, h);
+      const float *ks = tok(k, sb, sn, sh, b, s, h);
+      const float *vs = tok(v, sb, sn, sh, b, s, h);
+      const float *gs = tok(a, sb, sn, sh, b, s, h);
+      double *os = tokd(o, ob, on, oh, b, s, h);
+      for (int i = 0; i < d; ++i) {
+        double g = exp((double)gs[i]);
+        for (int j = j0; j < j1; ++j) S[i * d + j] = g * S[i * d + j] + (double)ks[i] * vs[j];
+      }
+      for (int j = j0; j < j1; ++j) {
+        double acc = 0.0;
+        for (int i = 0; i < d; ++i) acc += (double)qs[i] * S[i * d + j];
+        os[j] = acc;
+      }
+    }
+    if (final_state) {
+      double *F = st_bh_w(final_state, H, d, b, h);
+      for (int i = 0; i < d; ++i)
+        for (int j = j0; j < j1; ++j) F[i * d + j] = S[i * d + j];
+    }
+    free(S);
+  }
+}
+
+/* Rows r0..r1-1 of the gated state after token s, from the rows after s-1. */
+static void gla_rows_step(double *Sr, int r0, int r1, int d, const float *ks, const float *vs,
+                          const float *gs) {
+  for (int i = r0; i < r1; ++i) {
+    double g = exp((double)gs[i]);
+    double *row = Sr + (long)(i - r0) * d;
+    for (int j = 0; j < d; ++j) row[j] = g * row[j] + (double)ks[i] * vs[j];
+  }
+}
+
+/*
+ * Gradients of L = sum_s o_s . do_s for oracle_gla_fwd, by the chain rule on
+ * the recurrence (the gated counterpart of LASP Eq. 12-13).  With G_s the
+ * gradient of L with respect to S_s:
+ *   G_{N-1} = q_{N-1}^T do_{N-1} + dstate_in,
+ *   G_s     = q_s^T do_s + diag(exp(a_{s+1})) G_{s+1};
+ *   dq_s[i] = sum_j S_s[i][j] do_s[j]
+ *   dk_s[i] = sum_j G_s[i][j] v_s[j]
+ *   dv_s[j] = sum_i k_s[i] G_s[i][j]
+ *   da_s[i] = exp(a_s[i]) sum_j G_s[i][j] S_{s-1}[i][j]   (S_{-1} = init or 0)
+ *   dinit   = diag(exp(a_0)) G_0.
+ * Tasks (b, h, sweep, block): sweep 0 = dq (rows of S, forward); sweep 1 = dk
+ * and da (rows of G and S, reverse); sweep 2 = dv and dinit (columns of G).
+ * Sweep 1 needs S_{s-1} while it walks backward: it keeps the rows of S every
+ * K tokens (K about sqrt(N)) on the way forward and, for each block of K
+ * tokens, recomputes the rows in between from the kept ones with the same
+ * operations in the same order, so they are the very numbers of the forward.
+ */
+void oracle_gla_bwd(const float *q, const float *k, const float *v, const float *a, const float *dout,
+                    long sb, long sn, long sh, const double *init, const double *dstate_in,
+                    double *dq, double *dk, double *dv, double *da, long gb, long gn, long gh,
+                    double *dinit, int B, long N, int H, int d) {
+  int nblk = (d + BLK - 1) / BLK;
+  long ntask = (long)B * H * 3 * nblk;
+#pragma omp parallel for schedule(dynamic, 1)
+  for (long task = 0; task < ntask; ++task) {
+    int blk = (int)(task % nblk);
+    int sweep = (int)((task / nblk) % 3);
+    int h = (int)((task / (3L * nblk)) % H);
+    int b = (int)(task / (3L * nblk * H));
+    int r0 = blk * BLK, r1 = r0 + BLK < d ? r0 + BLK : d;
+    int nr = r1 - r0;
+    if (sweep == 0) {
+      double *Sr = (double *)calloc((size_t)nr * d, sizeof(double));
+      if (init) memcpy(Sr, st_bh(init, H, d, b, h) + (long)r0 * d, sizeof(double) * nr * d);
+      for (long s = 0; s < N; ++s) {
+        const float *ds = tok(dout, sb, sn, sh, b, s, h);
+        double *dqs = tokd(dq, gb, gn, gh, b, s, h);
+        gla_rows_step(Sr, r0, r1, d, tok(k, sb, sn, sh, b, s, h), tok(v, sb, sn, sh, b, s, h),
+                      tok(a, sb, sn, sh, b, s, h));
+        for (int i = r0; i < r1; ++i) {
+          double acc = 0.0;
+          for (int j = 0; j < d; ++j) acc += Sr[(long)(i - r0) * d + j] * ds[j];
+          dqs[i] = acc;
+        }
+      }
+      free(Sr);
+    } else if (sweep == 1) {
+      long K = (long)ceil(sqrt((double)(N > 0 ? N : 1)));
+      long nck = (N + K - 1) / K;
+      size_t rows = (size_t)nr * d;
+      double *kept = (double *)calloc((size_t)(nck > 0 ? nck : 1) * rows, sizeof(double));
+      double *buf = (double *)calloc((size_t)K * rows, sizeof(double));
+      double *Sr = (double *)calloc(rows, sizeof(double));
+      double *Gr = (double *)calloc(rows, sizeof(double));
+      if (init) memcpy(Sr, st_bh(init, H, d, b, h) + (long)r0 * d, sizeof(double) * rows);
+      for (long s = 0; s < N; ++s) {
+        if (s % K == 0) memcpy(kept + (size_t)(s / K) * rows, Sr, sizeof(double) * rows);
+        gla_rows_step(Sr, r0, r1, d, tok(k, sb, sn, sh, b, s, h), tok(v, sb, sn, sh, b, s, h),
+                      tok(a, sb, sn, sh, b, s, h));
+      }
+      if (dstate_in) memcpy(Gr, st_bh(dstate_in, H, d, b, h) + (long)r0 * d, sizeof(double) * rows);
+      for (long m = nck - 1; m >= 0; --m) {
+        long t0 = m * K, t1 = t0 + K < N ? t0 + K : N;
+        memcpy(Sr, kept + (size_t)m * rows, sizeof(double) * rows);
+        for (long s = t0; s < t1; ++s) {
+          gla_rows_step(Sr, r0, r1, d, tok(k, sb, sn, sh, b, s, h), tok(v, sb, sn, sh, b, s, h),
+                        tok(a, sb, sn, sh, b, s, h));
+          memcpy(buf + (size_t)(s - t0) * rows, Sr, sizeof(double) * rows);
+        }
+        for (long s = t1 - 1; s >= t0; --s) {
+          const double *prev = s > t0 ? buf + (size_t)(s - 1 - t0) * rows : kept + (size_t)m * rows;
+          const float *qs = tok(q, sb, sn, sh, b, s, h);
+          const float *vs = tok(v, sb, sn, sh, b, s, h);
+          const float *gs = tok(a, sb, sn, sh, b, s, h);
+          const float *ds = tok(dout, sb, sn, sh, b, s, h);
+          double *dks = tokd(dk, gb, gn, gh, b, s, h);
+          double *das = tokd(da, gb, gn, gh, b, s, h);
+          for (int i = r0; i < r1; ++i) {
+            double g = exp((double)gs[i]);
+            double *Gi = Gr + (long)(i - r0) * d;
+            const double *Pi = prev + (long)(i - r0) * d;
+            double acck = 0.0, acca = 0.0;
+            for (int j = 0; j < d; ++j) {
+              Gi[j] += (double)qs[i] * ds[j];
+              acck += Gi[j] * vs[j];
+              acca += Gi[j] * Pi[j];
+            }
+            dks[i] = acck;
+            das[i] = g * acca;
+            for (int j = 0; j < d; ++j) Gi[j] *= g;
+          }
+        }
+      }
+      free(kept);
+      free(buf);
+      free(Sr);
+      free(Gr);
+    } else {
+      double *G = (double *)calloc((size_t)d * d, sizeof(double));
+      if (dstate_in) memcpy(G, st_bh(dstate_in, H, d, b, h), sizeof(double) * d * d);
+      for (long s = N - 1; s >= 0; --s) {
+        const float *qs = tok(q, sb, sn, sh, b, s, h);
+        const float *ks = tok(k, sb, sn, sh, b, s, h);
+        const float *gs = tok(a, sb, sn, sh, b, s, h);
+        const float *ds = tok(dout, sb, sn, sh, b, s, h);
+        double *dvs = tokd(dv, gb, gn, gh, b, s, h);
+        for (int i = 0; i < d; ++i)
+          for (int j = r0; j < r1; ++j) G[i * d + j] += (double)qs[i] * ds[j];
+        for (int j = r0; j < r1; ++j) {
+          double acc = 0.0;
+          for (int i = 0; i < d; ++i) acc += (double)ks[i] * G[i * d + j];
+          dvs[j] = acc;
+        }
+        for (int i = 0; i < d; ++i) {
+          double g = exp((double)gs[i]);
+          for (int j = r0; j < r1; ++j) G[i * d + j] *= g;
+        }
+      }
+      if (dinit) {
+        double *D = st_bh_w(dinit, H, d, b, h);
+        for (int i = 0; i < d; ++i)
+          for (int j = r0; j < r1; ++j) D[i * d + j] = G[i * d + j];
+      }
+      free(G);
+    }
+  }
+}
+
+/*
+ * Per-chunk states of the gated form, written out from their definition (the
+ * gated counterparts of LASP Eq. 10 and of Eq. 20's (Lambda Q_t)^T dO_t): with
+ * A_c(t0, t1)[i] = sum_{r=t0}^{t1} a_{cC+r}[i] (0 when t0 > t1),
+ *   kind 0, (x, y) = (k, v):   M_c[i][j] = sum_t exp(A_c(t+1, C-1)[i]) x_t[i] y_t[j]
+ *                              (the gates from token t to the end of the chunk);
+ *   kind 1, (x, y) = (q, do):  M_c[i][j] = sum_t exp(A_c(0, t)[i]) x_t[i] y_t[j]
+ *                              (the gates from the start of the chunk to token t);
+ *   gsum[b, c, h, i] = A_c(0, C-1)[i], the chunk's total log-gate (if gsum is given).
+ * M is [B, T, H, d, d] and gsum [B, T, H, d], T = N / C.
+ */
+void oracle_gla_chunk_states(const float *x, const float *y, const float *a, long sb, long sn, long sh,
+                             double *M, double *gsum, int B, long N, int H, int d, long C, int kind) {
+  long T = N / C;
+  long ntask = (long)B * T * H;
+#pragma omp parallel for schedule(dynamic, 1)
+  for (long task = 0; task < ntask; ++task) {
+    int h = (int)(task % H);
+    long c = (task / H) % T;
+    int b = (int)(task / ((long)H * T));
+    double *Mc = M + st_btc((int)T, H, d, b, c, h);
+    double *w = (double *)malloc(sizeof(double) * d);
+    for (long e = 0; e < (long)d * d; ++e) Mc[e] = 0.0;
+    for (long t = 0; t < C; ++t) {
+      long r0 = kind == 0 ? t + 1 : 0, r1 = kind == 0 ? C - 1 : t;
+      for (int i = 0; i < d; ++i) {
+        double A = 0.0;
+        for (long r = r0; r <= r1; ++r) A += (double)tok(a, sb, sn, sh, b, c * C + r, h)[i];
+        w[i] = exp(A);
+      }
+      const float *xs = tok(x, sb, sn, sh, b, c * C + t, h);
+      const float *ys = tok(y, sb, sn, sh, b, c * C + t, h);
+      for (int i = 0; i < d; ++i)
+        for (int j = 0; j < d; ++j) Mc[i * d + j] += w[i] * (double)xs[i] * ys[j];
+    }
+    if (gsum) {
+      double *gc = gsum + (((long)b * T + c) * H + h) * d;
+      for (int i = 0; i < d; ++i) {
+        double A = 0.0;
+        for (long r = 0; r < C; ++r) A += (double)tok(a, sb, sn, sh, b, c * C + r, h)[i];
+        gc[i] = A;
+      }
+    }
+    free(w);
+  }
+}
+
+/*
+ * Scans over gated chunk states: each step through chunk c scales row i of
+ * the carried state by exp(gsum_c[i]) (the product of the chunk's gates).
+ *   reverse = 0:  P_0 = init (or 0);     P_c = diag(exp(gsum_{c-1})) P_{c-1} + M_{c-1};
+ *                 total = diag(exp(gsum_{T-1})) P_{T-1} + M_{T-1}.
+ *   reverse = 1:  R_{T-1} = init (or 0); R_c = diag(exp(gsum_{c+1})) R_{c+1} + M_{c+1};
+ *                 total = diag(exp(gsum_0)) R_0 + M_0.
+ * M, P: [B, T, H, d, d]; gsum: [B, T, H, d]; init, total: [B, H, d, d].
+ */
+void oracle_gla_state_scan(const double *M, const double *gsum, double *P, const double *init,
+                           double *total, int B, long T, int H, int d, int reverse) {
+  long ntask = (long)B * H;
+#pragma omp parallel for schedule(dynamic, 1)
+  for (long task = 0; task < ntask; ++task) {
+    int h = (int)(task % H);
+    int b = (int)(task / H);
+    double *acc = (double *)calloc((size_t)d * d, sizeof(double));
+    if (init) memcpy(acc, st_bh(init, H, d, b, h), sizeof(double) * d * d);
+    for (long n = 0; n < T; ++n) {
+      long c = reverse ? T - 1 - n : n;
+      const double *Mc = M + st_btc((int)T, H, d, b, c, h);
+      const double *gc = gsum + (((long)b * T + c) * H + h) * d;
+      double *Pc = P + st_btc((int)T, H, d, b, c, h);
+      for (long e = 0; e < (long)d * d; ++e) Pc[e] = acc[e];
+      for (int i = 0; i < d; ++i) {
+        double g = exp(gc[i]);
+        for (int j = 0; j < d; ++j) acc[i * d + j] = g * acc[i * d + j] + Mc[i * d + j];
+      }
+    }
+    if (total) memcpy(st_bh_w(total, H, d, b, h), acc, sizeof(double) * d * d);
+    free(acc);
+  }
+}
+
+/*
+ * State snapshots of the gated recurrences (what the backward pass needs at
+ * chunk boundaries, LASP section 3.4 "KV State Caching"):
+ *   kind 0, (x, y) = (k, v):  P_c = S_{cC-1}, the state entering chunk c
+ *            (S_{-1} = init or 0), run token by token;
+ *   kind 1, (x, y) = (q, do): R_c = X_{(c+1)C-1}, where X_s is the gradient of
+ *            L with respect to S_s carried by the tokens after s:
+ *            X_{N-1} = init (the dstate_in) or 0,
+ *            X_{s-1} = diag(exp(a_s)) (X_s + q_s^T do_s).
+ * P is [B, T, H, d, d].
+ */
+void oracle_gla_state_snapshots(const float *x, const float *y, const float *a, long sb, long sn, long sh,
+                                const double *init, double *P, int B, long N, int H, int d, long C,
+                                int kind) {
+  long T = N / C;
+  long ntask = (long)B * H;
+#pragma omp parallel for schedule(dynamic, 1)
+  for (long task = 0; task < ntask; ++task) {
+    int h = (int)(task % H);
+    int b = (int)(task / H);
+    double *S = (double *)calloc((size_t)d * d, sizeof(double));
+    if (init) memcpy(S, st_bh(init, H, d, b, h), sizeof(double) * d * d);
+    if (kind == 0) {
+      for (long s = 0; s < N; ++s) {
+        if (s % C == 0) memcpy(P + st_btc((int)T, H, d, b, s / C, h), S, sizeof(double) * d * d);
+        const float *xs = tok(x, sb, sn, sh, b, s, h);
+        const float *ys = tok(y, sb, sn, sh, b, s, h);
+        const float *gs = tok(a, sb, sn, sh, b, s, h);
+        for (int i = 0; i < d; ++i) {
+          double g = exp((double)gs[i]);
+          for (int j = 0; j < d; ++j) S[i * d + j] = g * S[i * d + j] + (double)xs[i] * ys[j];
+        }
+      }
+    } else {
+      for (long s = N - 1; s >= 0; --s) {
+        if (s % C == C - 1) memcpy(P + st_btc((int)T, H, d, b, s / C, h), S, sizeof(double) * d * d);
+        const float *xs = tok(x, sb, sn, sh, b, s, h);
+        const float *ys = tok(y, sb, sn, sh, b, s, h);
+        const float *gs = tok(a, sb, sn, sh, b, s, h);
+        for (int i = 0; i < d; ++i) {
+          double g = exp((double)gs[i]);
+          for (int j = 0; j < d; ++j) S[i * d + j] = g * (S[i * d + j] + (double)xs[i] * ys[j]);
+        }
+      }
+    }
+    free(S);
+  }
+}

@@ -13,6 +13,7 @@ import oracle
 
 HERE = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, HERE)
+import test_oracle_gla_pins as gpins  # noqa: E402
 import test_oracle_pins as pins  # noqa: E402
 
 SRC = os.path.join(os.path.dirname(HERE), "oracle", "lasp_oracle.c")
@@ -46,6 +47,33 @@ MUTATIONS = [
     ("bidirectional dk uses dM transposed", "ak += G[i * d + j] * vs[j];", "ak += G[j * d + i] * vs[j];", 0),
     ("bidirectional dv uses dM transposed", "av += (double)ks[j] * G[j * d + i];",
      "av += (double)ks[j] * G[i * d + j];", 0),
+    ("gated forward gates the value feature instead of the key feature",
+     "for (int j = j0; j < j1; ++j) S[i * d + j] = g * S[i * d + j] + (double)ks[i] * vs[j];",
+     "for (int j = j0; j < j1; ++j) S[i * d + j] = exp((double)gs[j]) * S[i * d + j] + (double)ks[i] * vs[j];", 0),
+    ("gated forward gates the token's own outer product too",
+     "for (int j = j0; j < j1; ++j) S[i * d + j] = g * S[i * d + j] + (double)ks[i] * vs[j];",
+     "for (int j = j0; j < j1; ++j) S[i * d + j] = g * (S[i * d + j] + (double)ks[i] * vs[j]);", 0),
+    ("gated dq rows are stepped without the gate",
+     "for (int j = 0; j < d; ++j) row[j] = g * row[j] + (double)ks[i] * vs[j];",
+     "for (int j = 0; j < d; ++j) row[j] = row[j] + (double)ks[i] * vs[j];", 0),
+    ("gated dk gradient state loses its gate", "for (int j = 0; j < d; ++j) Gi[j] *= g;",
+     "for (int j = 0; j < d; ++j) Gi[j] *= 1.0;", 0),
+    ("gated dv gradient state loses its gate", "for (int j = r0; j < r1; ++j) G[i * d + j] *= g;",
+     "for (int j = r0; j < r1; ++j) G[i * d + j] *= 1.0;", 0),
+    ("gate gradient pairs G_s with S_s instead of S_{s-1}",
+     "const double *prev = s > t0 ? buf + (size_t)(s - 1 - t0) * rows : kept + (size_t)m * rows;",
+     "const double *prev = buf + (size_t)(s - t0) * rows;", 0),
+    ("gate gradient misses the gate factor", "das[i] = g * acca;", "das[i] = acca;", 0),
+    ("gated chunk state decays the token by its own gate",
+     "long r0 = kind == 0 ? t + 1 : 0, r1 = kind == 0 ? C - 1 : t;",
+     "long r0 = kind == 0 ? t : 0, r1 = kind == 0 ? C - 1 : t;", 0),
+    ("gated gradient chunk state leaves out the token's own gate",
+     "long r0 = kind == 0 ? t + 1 : 0, r1 = kind == 0 ? C - 1 : t;",
+     "long r0 = kind == 0 ? t + 1 : 0, r1 = kind == 0 ? C - 1 : t - 1;", 0),
+    ("gated scan uses one feature's gate for every row", "double g = exp(gc[i]);", "double g = exp(gc[0]);", 0),
+    ("gated gradient snapshots gate before adding the token",
+     "for (int j = 0; j < d; ++j) S[i * d + j] = g * (S[i * d + j] + (double)xs[i] * ys[j]);",
+     "for (int j = 0; j < d; ++j) S[i * d + j] = g * S[i * d + j] + (double)xs[i] * ys[j];", 0),
 ]
 
 
@@ -76,6 +104,11 @@ def _pins_pass():
         pins.test_state_scan_closed_forms,
         pins.test_scan_of_chunk_states_equals_recurrence_snapshots,
         pins.test_bidirectional_equals_left_product,
+        gpins.test_constant_gate_is_the_decayed_recurrence,
+        lambda: gpins.test_recurrence_equals_quadratic_form(1),
+        gpins.test_gate_gradient_identity,
+        lambda: gpins.test_chunk_states_and_scans_equal_snapshots(4),
+        lambda: gpins.test_recurrence_equals_chunk_form(8),
     ]
     for check in checks:
         try:
@@ -92,7 +125,8 @@ def test_pins_catch_the_mistake(tmp_path, name, old, new, nth):
     real = oracle._load()
     lib = ctypes.CDLL(so)
     for f in ("oracle_fwd", "oracle_bwd", "oracle_chunk_states", "oracle_state_scan", "oracle_state_snapshots",
-              "oracle_bidir_fwd", "oracle_bidir_bwd"):
+              "oracle_bidir_fwd", "oracle_bidir_bwd", "oracle_gla_fwd", "oracle_gla_bwd", "oracle_gla_chunk_states",
+              "oracle_gla_state_scan", "oracle_gla_state_snapshots"):
         getattr(lib, f).argtypes = getattr(real, f).argtypes
         getattr(lib, f).restype = None
     lib.oracle_num_threads.restype = ctypes.c_int
