@@ -315,6 +315,91 @@ LASP_API int lasp_bidir_bwd(const void* q, const void* k, const void* v, const v
                             void* dv, int B, int H, int64_t N, int d, int dtype, const float* ws, float* dws,
                             void* stream);
 
+/* ------------------------------------------------------------------------
+ * Gated form: a decay that depends on the token and the key feature.
+ * Page LASP, Appendix A.4, Eq. 24 (m_t = o_t m_{t-1} + e_t i_t^T), row
+ * GLA / GateLoop of Table 5: expand state e_t = k_t, input i_t = v_t, shrink
+ * state q_t, memory d x d, oscillation g_t 1^T (the gate of key feature i
+ * scales row i of the memory). For every b, h and token s:
+ *     kv_s = diag(exp(g_s)) kv_{s-1} + k_s^T v_s,    o_s = q_s kv_s,
+ * with g_s[i] the natural log of that gate (g <= 0 for a gate in (0, 1]; any
+ * finite value is accepted, but for g > 0 the gate factors can overflow).
+ * With g_s[i] = log(lambda_h) this is lasp_fwd's recurrence.
+ *
+ *   g, dg:  float [B, N, H, d] (always float32, the layout of the token
+ *           tensors), the log-gates and the gradient of sum(o * dout) with
+ *           respect to them.
+ * Chunks: 1 <= C <= 128, C divides N (LASP_ERR_UNSUPPORTED for C > 128). In
+ * chunk c, b_t = sum_{r<=t} g_{cC+r} (from the chunk start) and the chunk's
+ * total log-gate is gsum_c = b_{C-1}. The states of the gated form:
+ *   kind 0, (x, y) = (k, v):   M_c  = sum_t diag(exp(gsum_c - b_t)) k_t^T v_t
+ *   kind 1, (x, y) = (q, do):  dM_c = sum_t diag(exp(b_t)) q_t^T do_t
+ * and the scans step through chunk c with diag(exp(gsum_c)) where lasp_fwd's
+ * use lambda^C (LASP-2 prefix / suffix over the chunk states).
+ * Pointers, streams and errors as for the calls above.
+ */
+
+/* Size, in floats, of the state cache of lasp_gla_fwd / lasp_gla_bwd:
+ * B * (N/C) * H * d * (d + 1). -1 for sizes the gated calls reject. */
+LASP_API int64_t lasp_gla_cache_floats(int B, int H, int64_t N, int d, int C);
+
+/*
+ * lasp_gla_chunk_states -- kind 0: M [B, N/C, H, d, d] from (x, y) = (k, v)
+ * and, if gsum (float [B, N/C, H, d]) is non-NULL, the chunk log-gate totals;
+ * kind 1: dM from (x, y) = (q, dout) (gsum as for kind 0).
+ */
+LASP_API int lasp_gla_chunk_states(const void* x, const void* y, const float* g, float* M, float* gsum, int B,
+                                   int H, int64_t N, int d, int C, int dtype, int kind, void* stream);
+
+/*
+ * lasp_gla_state_prefix -- exclusive scan with a diagonal decay per chunk:
+ *   reverse = 0:  P_0 = init; P_c = diag(exp(gsum_{c-1})) P_{c-1} + M_{c-1};
+ *                 total = diag(exp(gsum_{T-1})) P_{T-1} + M_{T-1}
+ *   reverse = 1:  R_{T-1} = init; R_c = diag(exp(gsum_{c+1})) R_{c+1} + M_{c+1};
+ *                 total = diag(exp(gsum_0)) R_0 + M_0
+ *   M, Mprefix: float [B, T, H, d, d] (may be the same array); gsum: float
+ *   [B, T, H, d]; init, total: float [B, H, d, d] or NULL.
+ */
+LASP_API int lasp_gla_state_prefix(const float* M, float* Mprefix, const float* gsum, const float* init,
+                                   float* total, int B, int T, int H, int d, int reverse, void* stream);
+
+/*
+ * lasp_gla_fwd -- o for the gated recurrence. Steps: states (kind 0) and
+ * gsum into state_cache, the prefix scan in place (P_c), then per chunk
+ *   o_t = (q_t . exp(b_t)) P_c + sum_{s<=t} (sum_i q_t[i] k_s[i] exp(b_t[i] - b_s[i])) v_s.
+ *   state_cache: out, lasp_gla_cache_floats(...) floats; pass it unchanged to
+ *                lasp_gla_bwd. Required.
+ *   init_state:  in, float [B, H, d, d] or NULL, the state entering token 0.
+ */
+LASP_API int lasp_gla_fwd(const void* q, const void* k, const void* v, const float* g, void* o, int B, int H,
+                          int64_t N, int d, int C, int dtype, float* state_cache, const float* init_state,
+                          void* stream);
+
+/*
+ * lasp_gla_bwd -- gradients of sum(o * dout) for lasp_gla_fwd with respect to
+ * q, k, v and g. Steps: gradient states (kind 1) into dstate_ws, the suffix
+ * scan in place (R_c, the gradient of the state leaving chunk c; dinit), then
+ * per chunk, with A_ts = sum_i q_t[i] k_s[i] exp(b_t[i] - b_s[i]) (s <= t):
+ *   dq_t = exp(b_t) . (do_t P_c^T) + sum_{s<=t} (do_t . v_s) k_s . exp(b_t - b_s)
+ *   dk_s = sum_{t>=s} (do_t . v_s) q_t . exp(b_t - b_s) + exp(gsum_c - b_s) . (v_s R_c^T)
+ *   dv_s = sum_{t>=s} A_ts do_t + (k_s . exp(gsum_c - b_s)) R_c
+ *   dg_s = sum_{t>=s in the chunk} (q_t . dq_t - k_t . dk_t) + rowsum(R_c . P_{c+1})
+ * (P_{c+1} the state leaving the chunk), evaluated without the parts that
+ * cancel exactly (each token's s = t pair; the inter part of k . dk for t >= s),
+ * so that dg stays accurate to its own size when the gates are strong.
+ *   state_cache: in, what lasp_gla_fwd wrote for the same q, k, v, g, C and
+ *                init_state. Required.
+ *   dstate_ws:   workspace, B * (N/C) * H * d * d floats. Required.
+ *   dstate_in:   in, float [B, H, d, d] or NULL: gradient with respect to the
+ *                state after the last token.
+ *   dinit_state: out, float [B, H, d, d] or NULL: gradient with respect to
+ *                init_state.
+ */
+LASP_API int lasp_gla_bwd(const void* q, const void* k, const void* v, const float* g, const void* dout, void* dq,
+                          void* dk, void* dv, float* dg, int B, int H, int64_t N, int d, int C, int dtype,
+                          const float* state_cache, float* dstate_ws, const float* dstate_in, float* dinit_state,
+                          void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -80,13 +80,21 @@ def _load():
             lib.lasp_bidir_state_offset.restype = L
             lib.lasp_bidir_fwd.argtypes = [P, P, P, P, I, I, L, I, I, P, P]
             lib.lasp_bidir_bwd.argtypes = [P, P, P, P, P, P, P, I, I, L, I, I, P, P, P]
+            lib.lasp_gla_cache_floats.argtypes = [I, I, L, I, I]
+            lib.lasp_gla_cache_floats.restype = L
+            lib.lasp_gla_chunk_states.argtypes = [P, P, P, P, P, I, I, L, I, I, I, I, P]
+            lib.lasp_gla_state_prefix.argtypes = [P, P, P, P, P, I, I, I, I, I, P]
+            lib.lasp_gla_fwd.argtypes = [P, P, P, P, P, I, I, L, I, I, I, P, P, P]
+            lib.lasp_gla_bwd.argtypes = [P, P, P, P, P, P, P, P, P, I, I, L, I, I, I, P, P, P, P, P]
             lib.lasp_status_string.argtypes = [I]
             lib.lasp_status_string.restype = ctypes.c_char_p
             for f in (lib.lasp_fwd, lib.lasp_bwd, lib.lasp_chunk_states, lib.lasp_chunk_dstates,
                       lib.lasp_chunk_out, lib.lasp_chunk_grads, lib.lasp_bwd_noalloc,
                       lib.lasp_state_prefix, lib.lasp_check_device_status, lib.lasp_set_wait_limit_ns,
                       lib.lasp_wait_probe, lib.lasp_version, lib.lasp_trace_enable, lib.lasp_trace_read,
-                      lib.lasp_segment_tokens, lib.lasp_bidir_fwd, lib.lasp_bidir_bwd):
+                      lib.lasp_segment_tokens, lib.lasp_bidir_fwd, lib.lasp_bidir_bwd,
+                      lib.lasp_gla_chunk_states, lib.lasp_gla_state_prefix, lib.lasp_gla_fwd,
+                      lib.lasp_gla_bwd):
                 f.restype = I
             _lib = lib
     return _lib
@@ -219,6 +227,57 @@ def lasp_bidir_bwd(q, k, v, dout, dq, dk, dv, ws, dws, stream=None):
     B, N, H, d, dt = _tokens(q, k, v, dout, dq, dk, dv)
     _check(_load().lasp_bidir_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(dout), _ptr(dq), _ptr(dk), _ptr(dv),
                                   B, H, N, d, dt, _ptr(ws), _ptr(dws), _stream(stream, q)), "lasp_bidir_bwd")
+
+
+def _gates(like, *gs):
+    """The float32 [B, N, H, d] log-gate tensors of the gated calls."""
+    import torch
+    for g in gs:
+        if g is None:
+            continue
+        if (tuple(g.shape) != tuple(like.shape) or g.dtype != torch.float32 or not g.is_contiguous()
+                or not g.is_cuda):
+            raise ValueError("gate tensors must be contiguous float32 CUDA tensors shaped like q")
+
+
+def lasp_gla_cache_floats(B, H, N, d, C):
+    """Floats of the state cache of the gated calls (-1 if unsupported). See lasp.h."""
+    return int(_load().lasp_gla_cache_floats(B, H, N, d, C))
+
+
+def lasp_gla_chunk_states(x, y, g, M, C, gsum=None, kind=0, stream=None):
+    """Gated chunk states: kind 0 from (k, v), kind 1 from (q, dout); gsum the chunk log-gate totals. See lasp.h."""
+    B, N, H, d, dt = _tokens(x, y)
+    _gates(x, g)
+    _check(_load().lasp_gla_chunk_states(_ptr(x), _ptr(y), _ptr(g), _ptr(M), _ptr(gsum), B, H, N, d, C, dt,
+                                         int(kind), _stream(stream, x)), "lasp_gla_chunk_states")
+
+
+def lasp_gla_state_prefix(M, Mprefix, gsum, init=None, total=None, reverse=False, stream=None):
+    """Exclusive scan over gated chunk states with a diagonal decay exp(gsum_c) per chunk. See lasp.h."""
+    if M.dim() != 5:
+        raise ValueError("M must be [B, T, H, d, d]")
+    B, T, H, d, _ = M.shape
+    _check(_load().lasp_gla_state_prefix(_ptr(M), _ptr(Mprefix), _ptr(gsum), _ptr(init), _ptr(total), B, T, H, d,
+                                         int(bool(reverse)), _stream(stream, M)), "lasp_gla_state_prefix")
+
+
+def lasp_gla_fwd(q, k, v, g, o, C, state_cache, init_state=None, stream=None):
+    """o for the gated recurrence kv_s = diag(exp(g_s)) kv_{s-1} + k_s^T v_s. See lasp.h."""
+    B, N, H, d, dt = _tokens(q, k, v, o)
+    _gates(q, g)
+    _check(_load().lasp_gla_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(o), B, H, N, d, C, dt, _ptr(state_cache),
+                                _ptr(init_state), _stream(stream, q)), "lasp_gla_fwd")
+
+
+def lasp_gla_bwd(q, k, v, g, dout, dq, dk, dv, dg, C, state_cache, dstate_ws, dstate_in=None, dinit_state=None,
+                 stream=None):
+    """dq, dk, dv, dg of sum(o * dout) for lasp_gla_fwd. See lasp.h."""
+    B, N, H, d, dt = _tokens(q, k, v, dout, dq, dk, dv)
+    _gates(q, g, dg)
+    _check(_load().lasp_gla_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(dout), _ptr(dq), _ptr(dk), _ptr(dv),
+                                _ptr(dg), B, H, N, d, C, dt, _ptr(state_cache), _ptr(dstate_ws), _ptr(dstate_in),
+                                _ptr(dinit_state), _stream(stream, q)), "lasp_gla_bwd")
 
 
 def lasp_check_device_status(stream=None, device=None):

@@ -5,6 +5,10 @@
 //   forward:  P_0 = init,     P_c = g P_{c-1} + M_{c-1},  g = lambda^C
 //   reverse:  R_{T-1} = init, R_c = g R_{c+1} + M_{c+1}
 //
+// The gated form (LASP Appendix A.4, Eq. 24 with the GLA row of Table 5)
+// replaces the scalar g by a diagonal: the step through chunk c scales row i
+// by exp(gsum_c[i]), gsum_c being the chunk's total log-gate (kGated).
+//
 // The scan is pure HBM traffic: every state element is read once and written
 // once. One thread owns one float4 of the d*d state of one (b, h) and walks the
 // chunks in order; the loads of a group of kUnroll chunks do not depend on the
@@ -33,10 +37,15 @@ __device__ __forceinline__ float4 fma4(float g, float4 a, float4 m) {
   return make_float4(fmaf(g, a.x, m.x), fmaf(g, a.y, m.y), fmaf(g, a.z, m.z), fmaf(g, a.w, m.w));
 }
 
+constexpr float kLog2e = 1.4426950408889634f;
+
+// gsum (kGated only): [B, t_slots, H, d] log-gate totals, in the same slots as M
+template <bool kGated>
 __global__ void __launch_bounds__(kThreads) state_scan_kernel(const float4* M, float4* P, const float* decay,
+                                                              const float* __restrict__ gsum,
                                                               const float4* __restrict__ init,
                                                               float4* __restrict__ total, int H, int T,
-                                                              int dd4, int64_t n_threads, float Cf,
+                                                              int d, int dd4, int64_t n_threads, float Cf,
                                                               int reverse, int64_t t_slots, int slot_stride,
                                                               int slot_offset) {
   const int64_t idx = (int64_t)blockIdx.x * kThreads + threadIdx.x;
@@ -44,7 +53,7 @@ __global__ void __launch_bounds__(kThreads) state_scan_kernel(const float4* M, f
   const int e = (int)(idx % dd4);
   const int h = (int)((idx / dd4) % H);
   const int64_t b = idx / ((int64_t)dd4 * H);
-  const float g = decay_pow(log2f(load_decay(decay, h)), Cf);
+  const float g = kGated ? 1.f : decay_pow(log2f(load_decay(decay, h)), Cf);
   uint64_t keep;
   asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(keep));
   const int64_t bh = b * H + h;
@@ -54,38 +63,56 @@ __global__ void __launch_bounds__(kThreads) state_scan_kernel(const float4* M, f
   const int64_t base = ((b * t_slots + slot_offset) * H + h) * (int64_t)dd4 + e;
   const int64_t step = reverse ? -cstride : cstride;
   int64_t off = reverse ? base + (int64_t)(T - 1) * cstride : base;
+  // the log-gate total of this thread's state row in scan element c
+  const int64_t gstride = (int64_t)slot_stride * H * d;
+  const int64_t gstep = reverse ? -gstride : gstride;
+  int64_t goff = ((b * t_slots + slot_offset) * H + h) * (int64_t)d + (4 * e) / d;
+  if (reverse) goff += (int64_t)(T - 1) * gstride;
   // software pipeline: the loads of group g + 1 are issued before group g is
   // scanned and stored, so a group's worth of loads is always in flight
   const int ngroups = T / kUnroll;
   float4 cur[kUnroll];
+  float gc[kUnroll];
   if (ngroups > 0) {
 #pragma unroll
-    for (int u = 0; u < kUnroll; ++u) cur[u] = __ldcs(M + off + u * step);
+    for (int u = 0; u < kUnroll; ++u) {
+      cur[u] = __ldcs(M + off + u * step);
+      if (kGated) gc[u] = gsum[goff + u * gstep];
+    }
   }
   for (int gi = 0; gi < ngroups; ++gi) {
     const bool more = gi + 1 < ngroups;
     float4 nxt[kUnroll];
+    float gn[kUnroll];
     if (more) {
 #pragma unroll
-      for (int u = 0; u < kUnroll; ++u) nxt[u] = __ldcs(M + off + (kUnroll + u) * step);
+      for (int u = 0; u < kUnroll; ++u) {
+        nxt[u] = __ldcs(M + off + (kUnroll + u) * step);
+        if (kGated) gn[u] = gsum[goff + (kUnroll + u) * gstep];
+      }
     }
 #pragma unroll
     for (int u = 0; u < kUnroll; ++u) {
       st_keep(P + off + u * step, acc, keep);
-      acc = fma4(g, acc, cur[u]);
+      acc = fma4(kGated ? exp2f(gc[u] * kLog2e) : g, acc, cur[u]);
     }
     off += kUnroll * step;
+    goff += kUnroll * gstep;
     if (more) {
 #pragma unroll
-      for (int u = 0; u < kUnroll; ++u) cur[u] = nxt[u];
+      for (int u = 0; u < kUnroll; ++u) {
+        cur[u] = nxt[u];
+        if (kGated) gc[u] = gn[u];
+      }
     }
   }
   int n = ngroups * kUnroll;
   for (; n < T; ++n) {
     float4 m = __ldcs(M + off);
     st_keep(P + off, acc, keep);
-    acc = fma4(g, acc, m);
+    acc = fma4(kGated ? exp2f(gsum[goff] * kLog2e) : g, acc, m);
     off += step;
+    goff += gstep;
   }
   if (total) total[bh * dd4 + e] = acc;
 }
@@ -98,9 +125,20 @@ cudaError_t launch_state_scan_slots(const float* M, float* P, const float* decay
   const int dd4 = d * d / 4;
   const int64_t n_threads = (int64_t)B * H * dd4;
   const int64_t blocks = (n_threads + scan_detail::kThreads - 1) / scan_detail::kThreads;
-  scan_detail::state_scan_kernel<<<(unsigned)blocks, scan_detail::kThreads, 0, st>>>(
-      (const float4*)M, (float4*)P, decay, (const float4*)init, (float4*)total, H, T, dd4, n_threads,
-      (float)C, reverse, t_slots, slot_stride, slot_offset);
+  scan_detail::state_scan_kernel<false><<<(unsigned)blocks, scan_detail::kThreads, 0, st>>>(
+      (const float4*)M, (float4*)P, decay, nullptr, (const float4*)init, (float4*)total, H, T, d, dd4,
+      n_threads, (float)C, reverse, t_slots, slot_stride, slot_offset);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_gla_scan(const float* M, float* P, const float* gsum, const float* init, float* total, int B,
+                            int T, int H, int d, int reverse, cudaStream_t st) {
+  const int dd4 = d * d / 4;
+  const int64_t n_threads = (int64_t)B * H * dd4;
+  const int64_t blocks = (n_threads + scan_detail::kThreads - 1) / scan_detail::kThreads;
+  scan_detail::state_scan_kernel<true><<<(unsigned)blocks, scan_detail::kThreads, 0, st>>>(
+      (const float4*)M, (float4*)P, nullptr, gsum, (const float4*)init, (float4*)total, H, T, d, dd4, n_threads,
+      1.f, reverse, T, 1, 0);
   return cudaGetLastError();
 }
 

@@ -27,6 +27,20 @@ cudaError_t simt_chunk_bwd(const void* q, const void* k, const void* v, const vo
                            const float* P, const float* Rs, void* dq, void* dk, void* dv, int B, int H,
                            int64_t N, int d, int C, int dtype, cudaStream_t st);
 
+// Gated form (k_gla_simt.cu, k_state_scan.cu): a decay per token and key
+// feature; g is the log-gate [B, N, H, d] (float32), gsum the chunk totals
+// [B, T, H, d]. kind 0: M_c = sum_t diag(e^{b_end - b_t}) k_t^T v_t (and
+// gsum if non-null); kind 1: dM_c = sum_t diag(e^{b_t}) q_t^T do_t.
+cudaError_t gla_simt_chunk_states(const void* x, const void* y, const float* g, float* M, float* gsum, int B, int H,
+                                  int64_t N, int d, int C, int kind, int dtype, cudaStream_t st);
+cudaError_t launch_gla_scan(const float* M, float* P, const float* gsum, const float* init, float* total, int B,
+                            int T, int H, int d, int reverse, cudaStream_t st);
+cudaError_t gla_simt_chunk_out(const void* q, const void* k, const void* v, const float* g, const float* P, void* o,
+                               int B, int H, int64_t N, int d, int C, int dtype, cudaStream_t st);
+cudaError_t gla_simt_chunk_bwd(const void* q, const void* k, const void* v, const void* dout, const float* g,
+                               const float* P, const float* Rs, void* dq, void* dk, void* dv, float* dg, int B, int H,
+                               int64_t N, int d, int C, int dtype, cudaStream_t st);
+
 // One CTA waiting on a barrier nothing completes; ends by the wait limit.
 cudaError_t launch_wait_probe(cudaStream_t st);
 

@@ -32,6 +32,10 @@ enum KernelId : int {
   K_PROBE = 12,
   K_BIDIR_TOTAL = 13,   // bidirectional: sum of the segment states
   K_BIDIR_APPLY = 14,   // bidirectional: token tiles times the total state
+  K_GLA_STATES = 15,    // gated form: per-chunk states and log-gate totals
+  K_GLA_SCAN = 16,      // gated form: prefix / suffix with a diagonal decay
+  K_GLA_OUT = 17,       // gated form: output
+  K_GLA_BWD = 18,       // gated form: dQ/dK/dV and the log-gate gradient
   K_COUNT
 };
 
@@ -338,6 +342,10 @@ const char* lasp_kernel_name(int id) {
     case K_PROBE: return "wait_probe";
     case K_BIDIR_TOTAL: return "bidir_total";
     case K_BIDIR_APPLY: return "bidir_apply_tc";
+    case K_GLA_STATES: return "gla_states_simt";
+    case K_GLA_SCAN: return "gla_scan";
+    case K_GLA_OUT: return "gla_out_simt";
+    case K_GLA_BWD: return "gla_bwd_simt";
     default: return "unknown";
   }
 }

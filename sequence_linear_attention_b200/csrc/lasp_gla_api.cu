@@ -1,0 +1,111 @@
+// C ABI of the gated form (include/lasp.h, "Gated form"): a decay per token
+// and key feature, LASP Appendix A.4, Eq. 24 with the GLA / GateLoop row of
+// Table 5. Host-side validation and dispatch; nothing here allocates.
+//
+// The state cache of lasp_gla_fwd holds, for B x T x H chunk slots, the
+// fp32 entering state P_c (d x d) of every chunk, followed by the chunk
+// log-gate totals gsum_c (d floats per slot): B*T*H*d*(d+1) floats.
+#include "kernels.h"
+#include "lasp_common.cuh"
+
+namespace lasp {
+namespace gla_api_detail {
+
+using namespace api_detail;
+
+int check_gla_sizes(int B, int H, int64_t N, int d, int C, int dtype) {
+  int s = check_sizes(B, H, N, d, C, dtype);
+  if (s) return s;
+  if (C > 128) return LASP_ERR_UNSUPPORTED;  // a chunk's cumulative gates stay in shared memory
+  return LASP_OK;
+}
+
+int states_impl(const void* x, const void* y, const float* g, float* M, float* gsum, int B, int H, int64_t N, int d,
+                int C, int dtype, int kind, cudaStream_t st) {
+  return cuda_status(traced(K_GLA_STATES, st, [&] {
+    return gla_simt_chunk_states(x, y, g, M, gsum, B, H, N, d, C, kind, dtype, st);
+  }));
+}
+
+int scan_impl(const float* M, float* P, const float* gsum, const float* init, float* total, int B, int T, int H,
+              int d, int reverse, cudaStream_t st) {
+  return cuda_status(
+      traced(K_GLA_SCAN, st, [&] { return launch_gla_scan(M, P, gsum, init, total, B, T, H, d, reverse, st); }));
+}
+
+}  // namespace gla_api_detail
+}  // namespace lasp
+
+using namespace lasp;
+using namespace lasp::api_detail;
+using namespace lasp::gla_api_detail;
+
+extern "C" {
+
+int64_t lasp_gla_cache_floats(int B, int H, int64_t N, int d, int C) {
+  if (check_gla_sizes(B, H, N, d, C, LASP_F32)) return -1;
+  return (int64_t)B * (N / C) * H * d * (d + 1);
+}
+
+int lasp_gla_chunk_states(const void* x, const void* y, const float* g, float* M, float* gsum, int B, int H,
+                          int64_t N, int d, int C, int dtype, int kind, void* stream) {
+  int s = check_gla_sizes(B, H, N, d, C, dtype);
+  if (s) return s;
+  if (kind != 0 && kind != 1) return LASP_ERR_INVALID_ARG;
+  if (N == 0) return LASP_OK;
+  if ((s = check_ptrs({x, y, g, M}, {gsum}))) return s;
+  return states_impl(x, y, g, M, gsum, B, H, N, d, C, dtype, kind, (cudaStream_t)stream);
+}
+
+int lasp_gla_state_prefix(const float* M, float* Mprefix, const float* gsum, const float* init, float* total, int B,
+                          int T, int H, int d, int reverse, void* stream) {
+  if (B < 1 || H < 1 || T < 0 || (reverse != 0 && reverse != 1)) return LASP_ERR_INVALID_ARG;
+  if (d != 32 && d != 64 && d != 128) return LASP_ERR_UNSUPPORTED;
+  int s;
+  if (T > 0) {
+    if ((s = check_ptrs({M, Mprefix, gsum}, {init, total}))) return s;
+  } else {
+    if ((s = check_ptrs({}, {init, total}))) return s;
+    if (total == nullptr) return LASP_OK;
+  }
+  return scan_impl(M, Mprefix, gsum, init, total, B, T, H, d, reverse, (cudaStream_t)stream);
+}
+
+int lasp_gla_fwd(const void* q, const void* k, const void* v, const float* g, void* o, int B, int H, int64_t N, int d,
+                 int C, int dtype, float* state_cache, const float* init_state, void* stream) {
+  int s = check_gla_sizes(B, H, N, d, C, dtype);
+  if (s) return s;
+  if (N == 0) return LASP_OK;
+  if ((s = check_ptrs({q, k, v, g, o, state_cache}, {init_state}))) return s;
+  cudaStream_t st = (cudaStream_t)stream;
+  const int T = (int)(N / C);
+  float* gsum = state_cache + (int64_t)B * T * H * d * d;
+  // 1. chunk states M_c and log-gate totals; 2. exclusive prefix in place -> P_c; 3. output
+  if ((s = states_impl(k, v, g, state_cache, gsum, B, H, N, d, C, dtype, 0, st))) return s;
+  if ((s = scan_impl(state_cache, state_cache, gsum, init_state, nullptr, B, T, H, d, 0, st))) return s;
+  return cuda_status(traced(K_GLA_OUT, st, [&] {
+    return gla_simt_chunk_out(q, k, v, g, state_cache, o, B, H, N, d, C, dtype, st);
+  }));
+}
+
+int lasp_gla_bwd(const void* q, const void* k, const void* v, const float* g, const void* dout, void* dq, void* dk,
+                 void* dv, float* dg, int B, int H, int64_t N, int d, int C, int dtype, const float* state_cache,
+                 float* dstate_ws, const float* dstate_in, float* dinit_state, void* stream) {
+  int s = check_gla_sizes(B, H, N, d, C, dtype);
+  if (s) return s;
+  if (N == 0) return LASP_OK;
+  if ((s = check_ptrs({q, k, v, g, dout, dq, dk, dv, dg, state_cache, dstate_ws}, {dstate_in, dinit_state})))
+    return s;
+  cudaStream_t st = (cudaStream_t)stream;
+  const int T = (int)(N / C);
+  const float* gsum = state_cache + (int64_t)B * T * H * d * d;
+  // 1. gradient chunk states dM_c; 2. exclusive suffix in place -> R_c (and
+  // dinit); 3. dQ, dK, dV and the log-gate gradient
+  if ((s = states_impl(q, dout, g, dstate_ws, nullptr, B, H, N, d, C, dtype, 1, st))) return s;
+  if ((s = scan_impl(dstate_ws, dstate_ws, gsum, dstate_in, dinit_state, B, T, H, d, 1, st))) return s;
+  return cuda_status(traced(K_GLA_BWD, st, [&] {
+    return gla_simt_chunk_bwd(q, k, v, dout, g, state_cache, dstate_ws, dq, dk, dv, dg, B, H, N, d, C, dtype, st);
+  }));
+}
+
+}  // extern "C"

@@ -17,6 +17,9 @@ layers with head dimension 128; no data set or trained weight is used):
   the raw 16-bit patterns (``numpy.uint16``).
 * Per-head decay lambda_h = 1 - 2^-(5 + 8h/H), h = 0..H-1, as float32; the
   undecayed workloads use lambda = 1.
+* Gated workloads (a log-gate per token and key feature): g = log(sigmoid(x)) / tau
+  with x i.i.d. standard normal from a fifth stream, tau = 16 by default (gates
+  mostly in 0.9-1.0; tau = 1 gives strong gates), float32 [B, N, H, d].
 """
 from __future__ import annotations
 
@@ -69,6 +72,20 @@ def draw_tensor(seed: int, index: int, shape, scale: float, bf16: bool, threads:
                 for i in range(nblk)]
         for f in futs:
             f.result()
+    return out.reshape(shape)
+
+
+def make_log_gates(B: int, N: int, H: int, d: int, seed: int, tau: float = 16.0) -> np.ndarray:
+    """Log-gates log(sigmoid(x)) / tau, float32 [B, N, H, d], x from stream 4 of ``seed``."""
+    shape = (B, N, H, d)
+    n = int(np.prod(shape))
+    stream = np.random.SeedSequence(seed).spawn(len(_NAMES) + 1)[len(_NAMES)]
+    nblk = (n + _BLOCK - 1) // _BLOCK
+    out = np.empty(n, np.float32)
+    for i, child in enumerate(stream.spawn(nblk)):
+        m = min(_BLOCK, n - i * _BLOCK)
+        x = np.random.Generator(np.random.PCG64(child)).standard_normal(m, dtype=np.float64)
+        out[i * _BLOCK:i * _BLOCK + m] = (-np.logaddexp(0.0, -x) / tau).astype(np.float32)
     return out.reshape(shape)
 
 

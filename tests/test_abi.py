@@ -136,3 +136,27 @@ def test_bidir_rejects_bad_arguments(lib):
     off = lasp.lasp_bidir_state_offset(2, 3, 2048, 128)
     assert off == 2 * 2 * 3 * 128 * 128   # two 1024-token segments
     assert n == off + 2 * 3 * 128 * 128 + 2 * 3 * 128 * 128 // 2
+
+
+def test_gated_calls_reject_bad_arguments(lib):
+    f = lib.lasp_gla_fwd
+    assert f(A, A, A, A, A, 1, 2, 512, 64, 256, BF16, A, None, None) == UNSUPPORTED   # C > 128
+    assert f(A, A, A, A, A, 1, 2, 512, 96, 64, BF16, A, None, None) == UNSUPPORTED    # d = 96
+    assert f(A, A, A, A, A, 1, 2, 500, 64, 64, BF16, A, None, None) == INVALID        # C does not divide N
+    assert f(A, A, A, None, A, 1, 2, 512, 64, 64, BF16, A, None, None) == INVALID     # no gates
+    assert f(A, A, A, A, A, 1, 2, 512, 64, 64, BF16, None, None, None) == INVALID     # no cache
+    assert f(A, A, A, A + 4, A, 1, 2, 512, 64, 64, F32, A, None, None) == MISALIGNED
+    assert f(A, A, A, A, A, 1, 2, 0, 64, 64, F32, None, None, None) == OK             # nothing to do
+    g = lib.lasp_gla_bwd
+    assert g(A, A, A, A, A, A, A, A, None, 1, 2, 512, 64, 64, F32, A, A, None, None, None) == INVALID  # no dg
+    assert g(A, A, A, A, A, A, A, A, A, 1, 2, 512, 64, 64, F32, A, None, None, None, None) == INVALID  # no ws
+    assert g(A, A, A, A, A, A, A, A, A, 1, 2, 512, 64, 256, F32, A, A, None, None, None) == UNSUPPORTED
+    s = lib.lasp_gla_chunk_states
+    assert s(A, A, A, A, None, 1, 2, 512, 64, 64, F32, 2, None) == INVALID             # kind
+    assert s(A, A, A, A, A + 4, 1, 2, 512, 64, 64, F32, 0, None) == MISALIGNED         # gsum
+    p = lib.lasp_gla_state_prefix
+    assert p(A, A, None, None, None, 1, 4, 2, 64, 0, None) == INVALID                  # no gsum
+    assert p(A, A, A, None, None, 1, 4, 2, 64, 2, None) == INVALID                     # reverse
+    assert p(None, None, None, None, None, 1, 0, 2, 64, 0, None) == OK                 # T = 0, no total
+    assert lasp.lasp_gla_cache_floats(2, 3, 512, 64, 64) == 2 * 8 * 3 * 64 * 65
+    assert lasp.lasp_gla_cache_floats(2, 3, 512, 64, 256) == -1
