@@ -36,6 +36,9 @@ enum KernelId : int {
   K_GLA_SCAN = 16,      // gated form: prefix / suffix with a diagonal decay
   K_GLA_OUT = 17,       // gated form: output
   K_GLA_BWD = 18,       // gated form: dQ/dK/dV and the log-gate gradient
+  K_GLA_STATES_TC = 19,  // gated form on the tensor cores: states
+  K_GLA_OUT_TC = 20,     // gated form on the tensor cores: output
+  K_GLA_BWD_TC = 21,     // gated form on the tensor cores: gradients
   K_COUNT
 };
 
@@ -346,6 +349,9 @@ const char* lasp_kernel_name(int id) {
     case K_GLA_SCAN: return "gla_scan";
     case K_GLA_OUT: return "gla_out_simt";
     case K_GLA_BWD: return "gla_bwd_simt";
+    case K_GLA_STATES_TC: return "gla_states_tc";
+    case K_GLA_OUT_TC: return "gla_out_tc";
+    case K_GLA_BWD_TC: return "gla_bwd_tc";
     default: return "unknown";
   }
 }

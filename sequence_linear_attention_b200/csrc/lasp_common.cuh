@@ -29,6 +29,7 @@ enum Site : unsigned int {
   SITE_OUT_MMA = 21,
   SITE_BWD_TMA = 30,
   SITE_BWD_MMA = 31,
+  SITE_GATE_RANGE = 40,  // gated form: a chunk's log-gates span more than the factorized form takes
 };
 
 __device__ __forceinline__ void record_error(int code, unsigned int site) {

@@ -7,6 +7,7 @@
 // log-gate totals gsum_c (d floats per slot): B*T*H*d*(d+1) floats.
 #include "kernels.h"
 #include "lasp_common.cuh"
+#include "tc_kernels.h"
 
 namespace lasp {
 namespace gla_api_detail {
@@ -22,6 +23,10 @@ int check_gla_sizes(int B, int H, int64_t N, int d, int C, int dtype) {
 
 int states_impl(const void* x, const void* y, const float* g, float* M, float* gsum, int B, int H, int64_t N, int d,
                 int C, int dtype, int kind, cudaStream_t st) {
+  if (tc_gla_ok(dtype, d, C))
+    return cuda_status(traced(K_GLA_STATES_TC, st, [&] {
+      return tc_gla_chunk_states(x, y, g, M, gsum, B, H, N, kind, st);
+    }));
   return cuda_status(traced(K_GLA_STATES, st, [&] {
     return gla_simt_chunk_states(x, y, g, M, gsum, B, H, N, d, C, kind, dtype, st);
   }));
@@ -83,6 +88,9 @@ int lasp_gla_fwd(const void* q, const void* k, const void* v, const float* g, vo
   // 1. chunk states M_c and log-gate totals; 2. exclusive prefix in place -> P_c; 3. output
   if ((s = states_impl(k, v, g, state_cache, gsum, B, H, N, d, C, dtype, 0, st))) return s;
   if ((s = scan_impl(state_cache, state_cache, gsum, init_state, nullptr, B, T, H, d, 0, st))) return s;
+  if (tc_gla_ok(dtype, d, C))
+    return cuda_status(
+        traced(K_GLA_OUT_TC, st, [&] { return tc_gla_chunk_out(q, k, v, g, state_cache, o, B, H, N, st); }));
   return cuda_status(traced(K_GLA_OUT, st, [&] {
     return gla_simt_chunk_out(q, k, v, g, state_cache, o, B, H, N, d, C, dtype, st);
   }));

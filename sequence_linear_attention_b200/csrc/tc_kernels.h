@@ -60,4 +60,13 @@ cudaError_t bidir_total(const float* seg, float* total, void* tiles, int B, int 
 cudaError_t tc_bidir_apply(const void* x, const void* stiles, void* y, int B, int H, int64_t N, int d, int b_kmajor,
                            int num_sms, cudaStream_t st);
 
+// Gated form on the tensor cores, bf16, d = 128, C = 128 (k_tc_gla.cu): the
+// chunk states of k_gla_simt.cu (kind 0 from (k, v) with the log-gate totals,
+// kind 1 from (q, do)), the output given P, and the gradients given P and R.
+bool tc_gla_ok(int dtype, int d, int64_t C);
+cudaError_t tc_gla_chunk_states(const void* x, const void* y, const float* g, float* M, float* gsum, int B, int H,
+                                int64_t N, int kind, cudaStream_t st);
+cudaError_t tc_gla_chunk_out(const void* q, const void* k, const void* v, const float* g, const float* P, void* o,
+                             int B, int H, int64_t N, cudaStream_t st);
+
 }  // namespace lasp

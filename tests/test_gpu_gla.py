@@ -179,3 +179,70 @@ def test_rows_chunk_states_and_scans(bf16):
     R_ref, rtot_ref = oracle.gla_state_scan(dM_ref, gs_ref, init=init.astype(np.float64), reverse=True)
     for got, ref in ((P, P_ref), (tot, tot_ref), (R, R_ref), (rtot, rtot_ref)):
         assert rel_err(got.cpu().numpy(), ref) <= tol
+
+
+# ------------------------------------------------ tensor-core path (bf16, d = 128, C = 128)
+@pytest.mark.parametrize("B,N,H,tau,seed", [(2, 1024, 2, 16.0, 2020), (1, 512, 3, 1.0, 2021), (1, 2048, 1, 4.0, 2022)])
+def test_tensor_core_path_matches_oracle(B, N, H, tau, seed):
+    d, C = 128, 128
+    inp = lasp_inputs.make_inputs(B, N, H, d, seed=seed, bf16=True, decayed=False)
+    g = lasp_inputs.make_log_gates(B, N, H, d, seed=seed, tau=tau)
+    rng = np.random.default_rng(seed)
+    init = (rng.standard_normal((B, H, d, d)) * 0.1).astype(np.float32)
+    dsin = (rng.standard_normal((B, H, d, d)) * 0.1).astype(np.float32)
+    got = _run(inp, g, C, init=init, dstate_in=dsin)
+    ref = _reference(inp, g, init=init.astype(np.float64), dstate_in=dsin.astype(np.float64))
+    _compare(got, ref, TOL_BF16)
+
+
+def test_tensor_core_rows_match_oracle():
+    _rows_states(True, 128, 128)
+
+
+def _rows_states(bf16, C, d):
+    import torch
+    import sequence_linear_attention_b200 as lasp
+    B, N, H = 2, 512, 2
+    T = N // C
+    inp = lasp_inputs.make_inputs(B, N, H, d, seed=2023, bf16=bf16, decayed=False)
+    g = lasp_inputs.make_log_gates(B, N, H, d, seed=2023, tau=2.0)
+    q, k, v, do = (to_device(inp[n], bf16) for n in ("q", "k", "v", "do"))
+    gd = _gates_device(g)
+    M = torch.empty((B, T, H, d, d), dtype=torch.float32, device="cuda")
+    dM = torch.empty_like(M)
+    gs = torch.empty((B, T, H, d), dtype=torch.float32, device="cuda")
+    lasp.lasp_gla_chunk_states(k, v, gd, M, C, gsum=gs, kind=0)
+    lasp.lasp_gla_chunk_states(q, do, gd, dM, C, kind=1)
+    status, site = lasp.lasp_check_device_status()
+    assert status == 0, (status, site)
+    qh, kh, vh, doh = (host_f32(inp, n) for n in ("q", "k", "v", "do"))
+    M_ref, gs_ref = oracle.gla_chunk_states(kh, vh, g, C, kind=0)
+    dM_ref, _ = oracle.gla_chunk_states(qh, doh, g, C, kind=1)
+    # the tensor-core states round the gate-weighted operand to bf16
+    assert rel_err(M.cpu().numpy(), M_ref) <= TOL_BF16
+    assert rel_err(dM.cpu().numpy(), dM_ref) <= TOL_BF16
+    assert rel_err(gs.cpu().numpy(), gs_ref) <= 1e-5
+
+
+def test_tensor_core_path_reports_gates_out_of_range():
+    """Log-gates of -2 per token make each 64-token half of a 128-token chunk
+    span e^-128, more than the factorized form takes: the call records
+    LASP_ERR_INVALID_ARG at the gate-range site instead of returning wrong
+    numbers silently (the CUDA-core path, C < 128, takes such gates)."""
+    import torch
+    import sequence_linear_attention_b200 as lasp
+    B, N, H, d, C = 1, 256, 1, 128, 128
+    inp = lasp_inputs.make_inputs(B, N, H, d, seed=2024, bf16=True, decayed=False)
+    q, k, v = (to_device(inp[n], True) for n in ("q", "k", "v"))
+    gd = torch.full((B, N, H, d), -2.0, dtype=torch.float32, device="cuda")
+    cache = torch.empty(lasp.lasp_gla_cache_floats(B, H, N, d, C), dtype=torch.float32, device="cuda")
+    o = torch.empty_like(q)
+    lasp.lasp_gla_fwd(q, k, v, gd, o, C, cache)
+    status, site = lasp.lasp_check_device_status()
+    assert (status, site) == (1, 40)
+    # the same gates through the CUDA-core kernels (C = 64) are fine
+    cache64 = torch.empty(lasp.lasp_gla_cache_floats(B, H, N, d, 64), dtype=torch.float32, device="cuda")
+    lasp.lasp_gla_fwd(q, k, v, gd, o, 64, cache64)
+    assert lasp.lasp_check_device_status() == (0, 0)
+    ref = oracle.gla_fwd(*(host_f32(inp, n) for n in ("q", "k", "v")), gd.cpu().numpy())
+    assert rel_err(to_host(o), ref) <= TOL_BF16
