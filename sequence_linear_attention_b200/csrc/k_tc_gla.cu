@@ -24,9 +24,11 @@
 // CUDA-core kernels have no such limit.
 //
 // Thread layout (256 threads): warp w owns tile rows / TMEM lanes 32*(w%4)..
-// and the column half w/4 of every row-wise step. A row's cumulative log-gates
-// come from a warp-shuffle scan of the loaded gates down the rows (no gate
-// tile in shared memory).
+// and the column half w/4 of every row-wise step. The cumulative log-gates
+// come from a walk down the chunk's rows by warps 0-3, one feature per lane
+// (loads running 32 rows ahead): the state kernel scales its operand as it
+// walks; the others write the sums into an fp32 tile in shared memory that
+// the row-wise steps then read.
 #include "kernels.h"
 #include "lasp_common.cuh"
 #include "sm100.cuh"
@@ -79,66 +81,77 @@ __device__ __forceinline__ void scale_row_half(uint8_t* tile, int row, int half,
   }
 }
 
-// Inclusive cumulative log-gates (natural log) of row t over the 64 columns of
-// `half`: b[u] = sum_{r<=t} g_r[half*64 + u]. g_chunk points at the chunk's
-// first token, rows row_stride floats apart. A shuffle scan down the warp's 32
-// rows, then the totals of the warps above through `tot` ([8][64] floats).
-// All 256 threads call it (it contains a barrier).
-__device__ __forceinline__ void row_cumgates(const float* __restrict__ g_chunk, int64_t row_stride, int t, int half,
-                                             int warp, int lane, float (&b)[64], float* tot) {
-  const float4* gp = reinterpret_cast<const float4*>(g_chunk + (int64_t)t * row_stride + half * 64);
+// The chunk's log-gates g_t[i] for the feature i of this lane (warp w < 4
+// owns features 32w..32w+31), rows in walking order (down, or up if `up`),
+// handed to `step(t, g)`; the loads run one kBlk-row block ahead.
+template <int kBlk = 32, class F>
+__device__ __forceinline__ void walk_gates(const float* __restrict__ g_chunk, int64_t row_stride, int i, bool up,
+                                           F&& step) {
+  const float* gp = g_chunk + i;
+  auto row = [&](int n) { return up ? kTile - 1 - n : n; };
+  float cur[kBlk], nxt[kBlk];
 #pragma unroll
-  for (int u = 0; u < 16; ++u) {
-    const float4 x = __ldcs(gp + u);
-    b[4 * u] = x.x;
-    b[4 * u + 1] = x.y;
-    b[4 * u + 2] = x.z;
-    b[4 * u + 3] = x.w;
-  }
+  for (int u = 0; u < kBlk; ++u) cur[u] = __ldcs(gp + (int64_t)row(u) * row_stride);
 #pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
+  for (int blk = 0; blk < kTile / kBlk; ++blk) {
+    if (blk + 1 < kTile / kBlk) {
 #pragma unroll
-    for (int u = 0; u < 64; ++u) {
-      const float y = __shfl_up_sync(0xffffffffu, b[u], o);
-      if (lane >= o) b[u] += y;
+      for (int u = 0; u < kBlk; ++u) nxt[u] = __ldcs(gp + (int64_t)row((blk + 1) * kBlk + u) * row_stride);
+    }
+#pragma unroll
+    for (int u = 0; u < kBlk; ++u) step(row(blk * kBlk + u), cur[u]);
+    if (blk + 1 < kTile / kBlk) {
+#pragma unroll
+      for (int u = 0; u < kBlk; ++u) cur[u] = nxt[u];
     }
   }
-  if (lane == 31) {
+}
+
+// Element (t, i) of the [128][128] fp32 gate tile: float4 slots XOR-swizzled
+// by the row, so that a warp walking 32 features of one row and a warp reading
+// float4s of 32 different rows both touch every bank once.
+__device__ __forceinline__ int gate_slot(int t, int i) { return t * kD + 4 * ((i >> 2) ^ (t & 7)) + (i & 3); }
+
+// Warps 0-3: b_t[i] = sum_{r<=t} g_r[i] (natural log) into the tile `bt`, and
+// b at the middle row into r[], at the last row into bend[].
+__device__ __forceinline__ void walk_gates_to_tile(const float* __restrict__ g_chunk, int64_t row_stride, int i,
+                                                   float* bt, float* r, float* bend) {
+  float acc = 0.f;
+  walk_gates(g_chunk, row_stride, i, false, [&](int t, float gt) {
+    acc += gt;
+    bt[gate_slot(t, i)] = acc;
+    if (t == kTile / 2 - 1) r[i] = acc;
+  });
+  bend[i] = acc;
+}
+
+// The 64 values of row t, columns half*64.., of the gate tile.
+__device__ __forceinline__ void read_gate_row(const float* bt, int t, int half, float (&b)[64]) {
 #pragma unroll
-    for (int u = 0; u < 64; ++u) tot[warp * 64 + u] = b[u];
-  }
-  named_sync(kBarAll, kThreads);
-  const int wq = warp & 3;
-  for (int w2 = 0; w2 < wq; ++w2) {
-#pragma unroll
-    for (int u = 0; u < 64; ++u) b[u] += tot[(w2 + 4 * half) * 64 + u];
+  for (int q = 0; q < 16; ++q) {
+    const float4 v = *reinterpret_cast<const float4*>(bt + t * kD + 4 * ((half * 16 + q) ^ (t & 7)));
+    b[4 * q] = v.x;
+    b[4 * q + 1] = v.y;
+    b[4 * q + 2] = v.z;
+    b[4 * q + 3] = v.w;
   }
 }
 
-// Publishes row `src_row`'s b (all 128 features) into dst[128] (natural log).
-__device__ __forceinline__ void publish_row(int t, int src_row, int half, const float (&b)[64], float* dst) {
-  if (t == src_row) {
-#pragma unroll
-    for (int u = 0; u < 64; ++u) dst[half * 64 + u] = b[u];
-  }
+// fp32 d x d state rows (global) -> bf16 operand tile, row m scaled by w[u]
+// (m = warp + 8u). Warp w converts rows w, w + 8, ...; lane covers 4 columns.
+__device__ __forceinline__ void put_state_row(uint8_t* tile, int m, int lane, float4 x, float w) {
+  const int col = lane * 4;
+  const uint32_t off = (col >> 6) * kBox + sw128_offset(m, (col & 63) >> 3) + (col & 7) * 2;
+  *reinterpret_cast<uint2*>(tile + off) = make_uint2(pack_bf16(x.x * w, x.y * w), pack_bf16(x.z * w, x.w * w));
 }
-
-// fp32 d x d state rows (global) -> bf16 operand tile, row m scaled by
-// exp2(scale_log2[m]). Warp w converts rows w, w + 8, ...; lane covers 4 columns.
-__device__ __forceinline__ void load_scaled_state(uint8_t* tile, const float* __restrict__ src,
-                                                  const float* scale_log2, int warp, int lane) {
+__device__ __forceinline__ void load_scaled_state(uint8_t* tile, const float* __restrict__ src, const float (&w)[16],
+                                                  int warp, int lane) {
   const float4* p = reinterpret_cast<const float4*>(src);
   float4 x[16];
 #pragma unroll
   for (int u = 0; u < 16; ++u) x[u] = __ldcs(p + (warp + 8 * u) * (kD / 4) + lane);
 #pragma unroll
-  for (int u = 0; u < 16; ++u) {
-    const int m = warp + 8 * u;
-    const float w = exp2f(scale_log2[m]);
-    const int col = lane * 4;
-    const uint32_t off = (col >> 6) * kBox + sw128_offset(m, (col & 63) >> 3) + (col & 7) * 2;
-    *reinterpret_cast<uint2*>(tile + off) = make_uint2(pack_bf16(x[u].x * w, x[u].y * w), pack_bf16(x[u].z * w, x[u].w * w));
-  }
+  for (int u = 0; u < 16; ++u) put_state_row(tile, warp + 8 * u, lane, x[u], w[u]);
 }
 
 // ---------------------------------------------------------------- states
@@ -146,12 +159,13 @@ struct SmemStates {
   uint64_t load, mma;
   uint32_t tmem_base;
   int abort;
-  float tot[8 * 64];
   float bend[kD];
 };
 
-// kind 0: M_c = (k . e^{b_end - b})^T v, gsum_c = b_end; kind 1: dM_c = (q . e^{b})^T do.
-// x, y: the two token operands ((k, v) or (q, do)); the gate factor goes on x.
+// kind 0: M_c = (k . e^{b_end - b})^T v and gsum_c = b_end; kind 1: dM_c =
+// (q . e^{b})^T do. x, y: the two token operands ((k, v) or (q, do)); the gate
+// factor goes on x, scaled in place by the walker warps, the walk for kind 0
+// going up from the last row (e^{b_end - b_t} = e^{sum_{r>t} g_r}).
 __global__ void __launch_bounds__(kThreads, 2) gla_states_tc(const __grid_constant__ CUtensorMap map_x,
                                                              const __grid_constant__ CUtensorMap map_y,
                                                              const float* __restrict__ g, float* __restrict__ M,
@@ -163,7 +177,6 @@ __global__ void __launch_bounds__(kThreads, 2) gla_states_tc(const __grid_consta
   SmemStates* s = reinterpret_cast<SmemStates*>(base + 2 * kTileBytes);
   const int c = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int t = (warp & 3) * 32 + lane, half = warp >> 2;
   const int64_t row0 = (int64_t)c * kTile;
   const int64_t T = N / kTile;
   if (tid == 0) {
@@ -189,16 +202,21 @@ __global__ void __launch_bounds__(kThreads, 2) gla_states_tc(const __grid_consta
     tma_load_4d(sY, &map_y, &s->load, 0, h, (int)row0, b);
     tma_load_4d(sY + kBox, &map_y, &s->load, 64, h, (int)row0, b);
   }
-  float bl[64];
-  row_cumgates(g + ((int64_t)b * N + row0) * H * kD + (int64_t)h * kD, (int64_t)H * kD, t, half, warp, lane, bl,
-               s->tot);
-  publish_row(t, kTile - 1, half, bl, s->bend);
-  named_sync(kBarAll, kThreads);
-  // the gate factor of row t: e^{b_end - b_t} (kind 0) or e^{b_t} (kind 1), in log2 units
-#pragma unroll
-  for (int u = 0; u < 64; ++u) bl[u] = (kind == 0 ? s->bend[half * 64 + u] - bl[u] : bl[u]) * kLog2e;
-  if (!mbar_wait(&s->load, 0, SITE_STATES_TMA)) s->abort = 1;
-  scale_row_half(sX, t, half, bl, 1.f);
+  if (warp < 4) {
+    const int i = tid;
+    const bool ok = mbar_wait(&s->load, 0, SITE_STATES_TMA);
+    if (!ok) s->abort = 1;
+    __nv_bfloat16* col = reinterpret_cast<__nv_bfloat16*>(sX + (i >> 6) * kBox + (i & 7) * 2);
+    float acc = 0.f;
+    walk_gates<16>(g + ((int64_t)b * N + row0) * H * kD + (int64_t)h * kD, (int64_t)H * kD, i, kind == 0,
+               [&](int t, float gt) {
+                 if (kind != 0) acc += gt;
+                 __nv_bfloat16* e = col + sw128_offset(t, (i & 63) >> 3) / 2;
+                 if (ok) *e = __float2bfloat16_rn(__bfloat162float(*e) * exp2f(acc * kLog2e));
+                 if (kind == 0) acc += gt;
+               });
+    s->bend[i] = acc;  // the walk covers every row either way: acc = b_end
+  }
   fence_async_smem();
   tc_fence_before();
   __syncthreads();
@@ -214,7 +232,7 @@ __global__ void __launch_bounds__(kThreads, 2) gla_states_tc(const __grid_consta
   if (mbar_wait(&s->mma, 0, SITE_STATES_MMA)) {
     tc_fence_after();
     // row i of M (TMEM lane i), columns half*64..
-    const int i = t;
+    const int i = (warp & 3) * 32 + lane, half = warp >> 2;
     float* out = M + (((b * T + c) * H + h) * kD + i) * kD + half * 64;
     const uint32_t lane_base = tmem + ((uint32_t)((warp & 3) * 32) << 16);
 #pragma unroll
@@ -237,14 +255,32 @@ cleanup:
   if (warp == 0) tmem_dealloc(tmem, 128);
 }
 
+// Phase 0 of the output and backward kernels: the walk into the gate tile
+// (warps 0-3; b at the middle row into r[], at the last row into bend[]), then,
+// for row t and column half `half` of every thread, the range check and
+// x = (b_t - r) log2 e, returned in x[].
+__device__ __forceinline__ void gate_rows(const float* __restrict__ g, int64_t N, int H, int b, int h, int64_t row0,
+                                          float* bt, float* r, float* bend, int tid, int t, int half, float (&x)[64]) {
+  if (tid < kD)
+    walk_gates_to_tile(g + ((int64_t)b * N + row0) * H * kD + (int64_t)h * kD, (int64_t)H * kD, tid, bt, r, bend);
+  named_sync(kBarAll, kThreads);
+  read_gate_row(bt, t, half, x);
+  bool ok = true;
+#pragma unroll
+  for (int u = 0; u < 64; ++u) {
+    const float y = x[u] - r[half * 64 + u];
+    ok = ok && fabsf(y) <= kMaxSpan;
+    x[u] = y * kLog2e;
+  }
+  if (!ok) record_error(LASP_ERR_INVALID_ARG, SITE_GATE_RANGE);
+}
+
 // ---------------------------------------------------------------- output
 struct SmemOut {
   uint64_t load, mma1, mma2;
   uint32_t tmem_base;
   int abort;
-  float tot[8 * 64];
-  float r[kD];       // b at the middle row (natural log)
-  float rl2[kD];     // the same, times log2 e
+  float r[kD], bend[kD];
 };
 
 __global__ void __launch_bounds__(kThreads, 1) gla_out_tc(const __grid_constant__ CUtensorMap map_q,
@@ -260,7 +296,8 @@ __global__ void __launch_bounds__(kThreads, 1) gla_out_tc(const __grid_constant_
   uint8_t* sV = base + 2 * kTileBytes;
   uint8_t* sX = base + 3 * kTileBytes;  // P'
   uint8_t* sA = base + 4 * kTileBytes;  // A . causal, then O out
-  SmemOut* s = reinterpret_cast<SmemOut*>(base + 5 * kTileBytes);
+  float* bt = reinterpret_cast<float*>(base + 5 * kTileBytes);  // gate tile, 64 KB
+  SmemOut* s = reinterpret_cast<SmemOut*>(base + 7 * kTileBytes);
   const int c = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int t = (warp & 3) * 32 + lane, half = warp >> 2;
@@ -296,28 +333,18 @@ __global__ void __launch_bounds__(kThreads, 1) gla_out_tc(const __grid_constant_
     tma_load_4d(sV, &map_v, &s->load, 0, h, (int)row0, b);
     tma_load_4d(sV + kBox, &map_v, &s->load, 64, h, (int)row0, b);
   }
-  float bl[64];
-  row_cumgates(g + ((int64_t)b * N + row0) * H * kD + (int64_t)h * kD, (int64_t)H * kD, t, half, warp, lane, bl,
-               s->tot);
-  publish_row(t, kTile / 2 - 1, half, bl, s->r);
-  named_sync(kBarAll, kThreads);
+  float x[64];
+  gate_rows(g, N, H, b, h, row0, bt, s->r, s->bend, tid, t, half, x);
+  // P' = diag(e^{r}) P_c into X
   {
-    bool ok = true;
+    float w[16];
 #pragma unroll
-    for (int u = 0; u < 64; ++u) {
-      const float x = bl[u] - s->r[half * 64 + u];
-      ok = ok && fabsf(x) <= kMaxSpan;
-      bl[u] = x * kLog2e;  // log2 E
-    }
-    if (!ok) record_error(LASP_ERR_INVALID_ARG, SITE_GATE_RANGE);
+    for (int u = 0; u < 16; ++u) w[u] = exp2f(s->r[warp + 8 * u] * kLog2e);
+    load_scaled_state(sX, P + ((b * T + c) * H + h) * (int64_t)kD * kD, w, warp, lane);
   }
-  if (tid < kD) s->rl2[tid] = s->r[tid] * kLog2e;
-  named_sync(kBarAll, kThreads);
-  // P' = diag(e^{r}) P_c into X (the global loads overlap the TMA loads)
-  load_scaled_state(sX, P + ((b * T + c) * H + h) * (int64_t)kD * kD, s->rl2, warp, lane);
   if (!mbar_wait(&s->load, 0, SITE_OUT_TMA)) s->abort = 1;
-  scale_row_half(sQ, t, half, bl, 1.f);   // Q^ = q . E
-  scale_row_half(sK, t, half, bl, -1.f);  // K^ = k / E
+  scale_row_half(sQ, t, half, x, 1.f);   // Q^ = q . E
+  scale_row_half(sK, t, half, x, -1.f);  // K^ = k / E
   fence_async_smem();
   tc_fence_before();
   __syncthreads();
@@ -398,6 +425,397 @@ cleanup:
   if (warp == 0) tmem_dealloc(tmem, 256);
 }
 
+// ---------------------------------------------------------------- gradients
+// Scans down the tile's 128 rows, for the 32 columns each thread holds of its
+// row t = 32 (warp % 4) + lane: suf[u] <- sum_{t' >= t}, pre[u] <- sum_{t' < t}.
+// Shuffles inside each warp's 32 rows; the warps' totals through tot[512].
+__device__ __forceinline__ void row_scans(float (&suf)[32], float (&pre)[32], int warp, int lane, int half,
+                                          float* tot) {
+  const int wq = warp & 3;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+#pragma unroll
+    for (int u = 0; u < 32; ++u) {
+      const float ys = __shfl_down_sync(0xffffffffu, suf[u], o);
+      const float yp = __shfl_up_sync(0xffffffffu, pre[u], o);
+      if (lane + o < 32) suf[u] += ys;
+      if (lane >= o) pre[u] += yp;
+    }
+  }
+  // warp totals: the suffix sum at lane 0, the inclusive prefix at lane 31
+  if (lane == 0) {
+#pragma unroll
+    for (int u = 0; u < 32; ++u) tot[((half * 2) * 4 + wq) * 32 + u] = suf[u];
+  }
+  if (lane == 31) {
+#pragma unroll
+    for (int u = 0; u < 32; ++u) tot[((half * 2 + 1) * 4 + wq) * 32 + u] = pre[u];
+  }
+  // inclusive -> exclusive prefix
+#pragma unroll
+  for (int u = 0; u < 32; ++u) {
+    const float y = __shfl_up_sync(0xffffffffu, pre[u], 1);
+    pre[u] = lane == 0 ? 0.f : y;
+  }
+  named_sync(kBarAll, kThreads);
+  for (int w2 = wq + 1; w2 < 4; ++w2) {
+#pragma unroll
+    for (int u = 0; u < 32; ++u) suf[u] += tot[((half * 2) * 4 + w2) * 32 + u];
+  }
+  for (int w2 = 0; w2 < wq; ++w2) {
+#pragma unroll
+    for (int u = 0; u < 32; ++u) pre[u] += tot[((half * 2 + 1) * 4 + w2) * 32 + u];
+  }
+  named_sync(kBarAll, kThreads);  // tot is rewritten by the next call
+}
+
+// 32 bf16 values of a token row (global), from column col0.
+__device__ __forceinline__ void load_row32(const __nv_bfloat16* p, float (&v)[32]) {
+  const uint4* p4 = reinterpret_cast<const uint4*>(p);
+#pragma unroll
+  for (int q4 = 0; q4 < 4; ++q4) {
+    const uint4 w = __ldg(p4 + q4);
+    const uint32_t* e = reinterpret_cast<const uint32_t*>(&w);
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const float2 f = unpack_bf16(e[u]);
+      v[q4 * 8 + 2 * u] = f.x;
+      v[q4 * 8 + 2 * u + 1] = f.y;
+    }
+  }
+}
+
+struct SmemBwd {
+  uint64_t load, mma1a, mma1b, mma2, mma3;
+  uint32_t tmem_base;
+  int abort;
+  float dAd[kTile];  // do_t . v_t, the diagonal of dO V^T
+  float bnd[kD];     // e^{b_end[i]} <R_c[i], P_c[i]>
+};
+
+// One 128-token chunk per CTA. Shared memory: Q^, K^, V, dO, X (P', then R';
+// r and b_end during the gate walk; the scan totals at the end), and the pair
+// sA / sB (the gate tile during the walk; then dA . strict and A . causal;
+// then the dK and dV outputs). TMEM: T0 = dO V^T -> (dA . strict)^T Q^ -> dB;
+// T1 = Q^ K^^T -> dV; T2 = dO P'^T + (dA . strict) K^ -> q . dq'; T3 = log2 E
+// -> V R'^T -> k . dk^inter.
+__global__ void __launch_bounds__(kThreads, 1) gla_bwd_tc(
+    const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
+    const __grid_constant__ CUtensorMap map_v, const __grid_constant__ CUtensorMap map_do,
+    const __grid_constant__ CUtensorMap map_dk, const __grid_constant__ CUtensorMap map_dv,
+    const float* __restrict__ g, const float* __restrict__ P, const float* __restrict__ R,
+    const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k, __nv_bfloat16* __restrict__ dq,
+    float* __restrict__ dg, int H, int64_t N) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* base = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  uint8_t* sQ = base;
+  uint8_t* sK = base + 1 * kTileBytes;
+  uint8_t* sV = base + 2 * kTileBytes;
+  uint8_t* sD = base + 3 * kTileBytes;
+  uint8_t* sX = base + 4 * kTileBytes;
+  uint8_t* sA = base + 5 * kTileBytes;
+  uint8_t* sB = base + 6 * kTileBytes;
+  SmemBwd* s = reinterpret_cast<SmemBwd*>(base + 7 * kTileBytes);
+  float* bt = reinterpret_cast<float*>(sA);  // gate tile over sA and sB during the walk
+  float* sr = reinterpret_cast<float*>(sX);  // r and b_end over X during the walk
+  float* sbend = sr + kD;
+  float* tot = reinterpret_cast<float*>(sX);  // scan totals over X at the end
+  const int c = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int t = (warp & 3) * 32 + lane, half = warp >> 2;
+  const int64_t row0 = (int64_t)c * kTile;
+  const int64_t T = N / kTile;
+  const int64_t slot = ((int64_t)b * T + c) * H + h;
+  const int64_t tok = (((int64_t)b * N + row0 + t) * H + h) * kD;  // row t of every token tensor
+  if (tid == 0) {
+    prefetch_tmap(&map_q);
+    prefetch_tmap(&map_k);
+    prefetch_tmap(&map_v);
+    prefetch_tmap(&map_do);
+    mbar_init(&s->load, 1);
+    mbar_init(&s->mma1a, 1);
+    mbar_init(&s->mma1b, 1);
+    mbar_init(&s->mma2, 1);
+    mbar_init(&s->mma3, 1);
+    s->abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(&s->tmem_base, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = s->tmem_base;
+  const uint32_t lane_base = tmem + ((uint32_t)((warp & 3) * 32) << 16);
+  const uint32_t T0 = 0, T1 = 128, T2 = 256, T3 = 384;
+  if (tid == 0) {
+    mbar_arrive_expect_tx(&s->load, 4 * kTileBytes);
+    tma_load_4d(sQ, &map_q, &s->load, 0, h, (int)row0, b);
+    tma_load_4d(sQ + kBox, &map_q, &s->load, 64, h, (int)row0, b);
+    tma_load_4d(sK, &map_k, &s->load, 0, h, (int)row0, b);
+    tma_load_4d(sK + kBox, &map_k, &s->load, 64, h, (int)row0, b);
+    tma_load_4d(sV, &map_v, &s->load, 0, h, (int)row0, b);
+    tma_load_4d(sV + kBox, &map_v, &s->load, 64, h, (int)row0, b);
+    tma_load_4d(sD, &map_do, &s->load, 0, h, (int)row0, b);
+    tma_load_4d(sD + kBox, &map_do, &s->load, 64, h, (int)row0, b);
+  }
+  // ---- phase 0: gates, Q^, K^, log2 E -> T3, P' -> X
+  float x[64];
+  gate_rows(g, N, H, b, h, row0, bt, sr, sbend, tid, t, half, x);
+  float wr[16], we[16];  // e^{r_m} and e^{b_end_m - r_m} of this thread's state rows m = warp + 8u
+#pragma unroll
+  for (int u = 0; u < 16; ++u) {
+    const int m = warp + 8 * u;
+    wr[u] = exp2f(sr[m] * kLog2e);
+    we[u] = exp2f((sbend[m] - sr[m]) * kLog2e);
+  }
+  named_sync(kBarAll, kThreads);  // r and b_end are read before X is written
+  load_scaled_state(sX, P + slot * kD * kD, wr, warp, lane);
+  if (!mbar_wait(&s->load, 0, SITE_BWD_TMA)) s->abort = 1;
+  scale_row_half(sQ, t, half, x, 1.f);   // Q^ = q . E
+  scale_row_half(sK, t, half, x, -1.f);  // K^ = k / E
+  {
+    uint32_t r0[32], r1[32];
+#pragma unroll
+    for (int u = 0; u < 32; ++u) {
+      r0[u] = __float_as_uint(x[u]);
+      r1[u] = __float_as_uint(x[32 + u]);
+    }
+    tmem_st32(lane_base + T3 + half * 64, r0);
+    tmem_st32(lane_base + T3 + half * 64 + 32, r1);
+    tmem_st_wait();
+  }
+  fence_async_smem();
+  tc_fence_before();
+  __syncthreads();
+  if (s->abort) goto cleanup;
+  {
+    const uint32_t aQ = smem_u32(sQ), aK = smem_u32(sK), aV = smem_u32(sV), aD = smem_u32(sD);
+    const uint32_t aX = smem_u32(sX), aA = smem_u32(sA), aB = smem_u32(sB);
+    constexpr uint32_t id_kk = idesc_bf16(128, 128, 0, 0);
+    constexpr uint32_t id_kn = idesc_bf16(128, 128, 0, 1);
+    constexpr uint32_t id_nn = idesc_bf16(128, 128, 1, 1);
+    // ---- phase 1: T0 = dO V^T, T1 = Q^ K^^T | T2 = dO P'^T
+    if (tid == 0) {
+      tc_fence_after();
+      for (int kk = 0; kk < kD / 16; ++kk) mma_bf16(tmem + T0, kmaj(aD, kk), kmaj(aV, kk), id_kk, kk != 0);
+      for (int kk = 0; kk < kD / 16; ++kk) mma_bf16(tmem + T1, kmaj(aQ, kk), kmaj(aK, kk), id_kk, kk != 0);
+      mma_commit(&s->mma1a);
+      for (int kk = 0; kk < kD / 16; ++kk) mma_bf16(tmem + T2, kmaj(aD, kk), kmaj(aX, kk), id_kk, kk != 0);
+      mma_commit(&s->mma1b);
+    }
+    // R rows (fp32) into registers while the MMAs run
+    const float4* R4 = reinterpret_cast<const float4*>(R + slot * kD * kD);
+    float4 rreg[16];
+#pragma unroll
+    for (int u = 0; u < 16; ++u) rreg[u] = __ldcs(R4 + (warp + 8 * u) * (kD / 4) + lane);
+    // ---- epilogue 1: dA . strict -> sA, A . causal -> sB, the diagonal of dA
+    if (mbar_wait(&s->mma1a, 0, SITE_BWD_MMA)) {
+      tc_fence_after();
+#pragma unroll 1
+      for (int c2 = 0; c2 < 2; ++c2) {
+        const int col0 = half * 64 + c2 * 32;
+        uint32_t ra[32], rs[32];
+        tmem_ld32(lane_base + T0 + col0, ra);
+        tmem_ld32(lane_base + T1 + col0, rs);
+        tmem_ld_wait();
+#pragma unroll
+        for (int u = 0; u < 32; ++u)
+          if (col0 + u == t) s->dAd[t] = __uint_as_float(ra[u]);
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4) {
+          float fa[8], fs[8];
+#pragma unroll
+          for (int u = 0; u < 8; ++u) {
+            const int col = col0 + q4 * 8 + u;
+            fa[u] = col < t ? __uint_as_float(ra[q4 * 8 + u]) : 0.f;
+            fs[u] = col <= t ? __uint_as_float(rs[q4 * 8 + u]) : 0.f;
+          }
+          *tile16(sA, t, col0 + q4 * 8) = make_uint4(pack_bf16(fa[0], fa[1]), pack_bf16(fa[2], fa[3]),
+                                                     pack_bf16(fa[4], fa[5]), pack_bf16(fa[6], fa[7]));
+          *tile16(sB, t, col0 + q4 * 8) = make_uint4(pack_bf16(fs[0], fs[1]), pack_bf16(fs[2], fs[3]),
+                                                     pack_bf16(fs[4], fs[5]), pack_bf16(fs[6], fs[7]));
+        }
+      }
+    } else {
+      s->abort = 1;
+    }
+    // X is free once dO P'^T has read P': R' = diag(e^{b_end - r}) R_c replaces it,
+    // and <R'_m, P'_m> (fp32) = e^{b_end_m} <R_m, P_m> goes to bnd
+    if (mbar_wait(&s->mma1b, 0, SITE_BWD_MMA)) {
+      const float4* P4 = reinterpret_cast<const float4*>(P + slot * kD * kD);
+#pragma unroll
+      for (int u = 0; u < 16; ++u) {
+        const int m = warp + 8 * u;
+        const float4 pv = __ldg(P4 + m * (kD / 4) + lane);
+        float dot = pv.x * rreg[u].x + pv.y * rreg[u].y + pv.z * rreg[u].z + pv.w * rreg[u].w;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
+        if (lane == 0) s->bnd[m] = dot * wr[u] * we[u];
+        put_state_row(sX, m, lane, rreg[u], we[u]);
+      }
+    } else {
+      s->abort = 1;
+    }
+    fence_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    if (s->abort) goto cleanup;
+    // ---- phase 2: T2 += (dA . strict) K^
+    if (tid == 0) {
+      tc_fence_after();
+      for (int kk = 0; kk < kTile / 16; ++kk) mma_bf16(tmem + T2, kmaj(aA, kk), mnmaj(aK, kk), id_kn, 1);
+      mma_commit(&s->mma2);
+    }
+    // ---- epilogue 2: dq' = E . T2; dq = dq' + (do_t . v_t) k_t; q . dq' -> T2
+    float xl[64];  // log2 E of row t, kept for epilogue 3
+    if (mbar_wait(&s->mma2, 0, SITE_BWD_MMA)) {
+      tc_fence_after();
+      {
+        uint32_t r0[32], r1[32];
+        tmem_ld32(lane_base + T3 + half * 64, r0);
+        tmem_ld32(lane_base + T3 + half * 64 + 32, r1);
+        tmem_ld_wait();
+#pragma unroll
+        for (int u = 0; u < 32; ++u) {
+          xl[u] = __uint_as_float(r0[u]);
+          xl[32 + u] = __uint_as_float(r1[u]);
+        }
+      }
+      const float dad = s->dAd[t];
+#pragma unroll
+      for (int c2 = 0; c2 < 2; ++c2) {
+        const int col0 = half * 64 + c2 * 32;
+        uint32_t a[32];
+        tmem_ld32(lane_base + T2 + col0, a);
+        float qv[32], kv[32];
+        load_row32(q + tok + col0, qv);
+        load_row32(k + tok + col0, kv);
+        tmem_ld_wait();
+        uint32_t out[16];
+#pragma unroll
+        for (int u = 0; u < 32; ++u) {
+          const float dqp = exp2f(xl[c2 * 32 + u]) * __uint_as_float(a[u]);
+          const float full = fmaf(dad, kv[u], dqp);
+          if (u & 1)
+            out[u / 2] = pack_bf16(__uint_as_float(out[u / 2]), full);
+          else
+            out[u / 2] = __float_as_uint(full);
+          a[u] = __float_as_uint(qv[u] * dqp);
+        }
+        uint4* dst = reinterpret_cast<uint4*>(dq + tok + col0);
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4) dst[q4] = make_uint4(out[4 * q4], out[4 * q4 + 1], out[4 * q4 + 2], out[4 * q4 + 3]);
+        tmem_st32(lane_base + T2 + col0, a);
+      }
+      tmem_st_wait();
+    } else {
+      s->abort = 1;
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (s->abort) goto cleanup;
+    // ---- phase 3: T0 = (dA . strict)^T Q^, T1 = (A . causal)^T dO + K^ R', T3 = V R'^T
+    if (tid == 0) {
+      tc_fence_after();
+      for (int kk = 0; kk < kTile / 16; ++kk) mma_bf16(tmem + T0, mnmaj(aA, kk), mnmaj(aQ, kk), id_nn, kk != 0);
+      for (int kk = 0; kk < kTile / 16; ++kk) mma_bf16(tmem + T1, mnmaj(aB, kk), mnmaj(aD, kk), id_nn, kk != 0);
+      for (int kk = 0; kk < kD / 16; ++kk) mma_bf16(tmem + T1, kmaj(aK, kk), mnmaj(aX, kk), id_kn, 1);
+      for (int kk = 0; kk < kD / 16; ++kk) mma_bf16(tmem + T3, kmaj(aV, kk), kmaj(aX, kk), id_kk, kk != 0);
+      mma_commit(&s->mma3);
+    }
+    // ---- epilogue 3: dk, dv -> sA, sB; dB = q . dq' - k . dk', k . dk^inter -> T0, T3; dg
+    if (mbar_wait(&s->mma3, 0, SITE_BWD_MMA)) {
+      tc_fence_after();
+      const float dad = s->dAd[t];
+#pragma unroll
+      for (int c2 = 0; c2 < 2; ++c2) {
+        const int col0 = half * 64 + c2 * 32;
+        uint32_t ka[32], kb[32], bq[32];
+        tmem_ld32(lane_base + T0 + col0, ka);
+        tmem_ld32(lane_base + T3 + col0, kb);
+        tmem_ld32(lane_base + T2 + col0, bq);
+        float qv[32], kv[32];
+        load_row32(q + tok + col0, qv);
+        load_row32(k + tok + col0, kv);
+        tmem_ld_wait();
+        uint32_t out[16];
+#pragma unroll
+        for (int u = 0; u < 32; ++u) {
+          const float ei = exp2f(-xl[c2 * 32 + u]);
+          const float dka = ei * __uint_as_float(ka[u]);
+          const float dkb = ei * __uint_as_float(kb[u]);
+          const float full = fmaf(dad, qv[u], dka + dkb);
+          if (u & 1)
+            out[u / 2] = pack_bf16(__uint_as_float(out[u / 2]), full);
+          else
+            out[u / 2] = __float_as_uint(full);
+          ka[u] = __float_as_uint(__uint_as_float(bq[u]) - kv[u] * dka);
+          kb[u] = __float_as_uint(kv[u] * dkb);
+        }
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4)
+          *tile16(sA, t, col0 + q4 * 8) = make_uint4(out[4 * q4], out[4 * q4 + 1], out[4 * q4 + 2], out[4 * q4 + 3]);
+        tmem_st32(lane_base + T0 + col0, ka);
+        tmem_st32(lane_base + T3 + col0, kb);
+        uint32_t dvv[32];
+        tmem_ld32(lane_base + T1 + col0, dvv);
+        tmem_ld_wait();
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4)
+          *tile16(sB, t, col0 + q4 * 8) =
+              make_uint4(pack_bf16(__uint_as_float(dvv[q4 * 8]), __uint_as_float(dvv[q4 * 8 + 1])),
+                         pack_bf16(__uint_as_float(dvv[q4 * 8 + 2]), __uint_as_float(dvv[q4 * 8 + 3])),
+                         pack_bf16(__uint_as_float(dvv[q4 * 8 + 4]), __uint_as_float(dvv[q4 * 8 + 5])),
+                         pack_bf16(__uint_as_float(dvv[q4 * 8 + 6]), __uint_as_float(dvv[q4 * 8 + 7])));
+      }
+      tmem_st_wait();
+      fence_async_smem();
+    } else {
+      s->abort = 1;
+    }
+    // dg_t = sum_{t' >= t} dB_t' + sum_{t' < t} k . dk^inter_t' + e^{b_end} <R_c, P_c>
+#pragma unroll 1
+    for (int c2 = 0; c2 < 2; ++c2) {
+      const int col0 = half * 64 + c2 * 32;
+      uint32_t a[32], e[32];
+      tmem_ld32(lane_base + T0 + col0, a);
+      tmem_ld32(lane_base + T3 + col0, e);
+      tmem_ld_wait();
+      float suf[32], pre[32];
+#pragma unroll
+      for (int u = 0; u < 32; ++u) {
+        suf[u] = __uint_as_float(a[u]);
+        pre[u] = __uint_as_float(e[u]);
+      }
+      row_scans(suf, pre, warp, lane, half, tot);
+      float4* dst = reinterpret_cast<float4*>(dg + tok + col0);
+#pragma unroll
+      for (int q4 = 0; q4 < 8; ++q4) {
+        float o[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) o[u] = suf[4 * q4 + u] + pre[4 * q4 + u] + s->bnd[col0 + 4 * q4 + u];
+        dst[q4] = make_float4(o[0], o[1], o[2], o[3]);
+      }
+    }
+    __syncthreads();
+    if (tid == 0 && !s->abort) {
+      tma_store_4d(&map_dk, sA, 0, h, (int)row0, b);
+      tma_store_4d(&map_dk, sA + kBox, 64, h, (int)row0, b);
+      tma_store_4d(&map_dv, sB, 0, h, (int)row0, b);
+      tma_store_4d(&map_dv, sB + kBox, 64, h, (int)row0, b);
+      tma_store_commit();
+      tma_store_wait_read0();
+    }
+  }
+cleanup:
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) tmem_dealloc(tmem, 512);
+}
+
 }  // namespace tc_gla_detail
 
 bool tc_gla_ok(int dtype, int d, int64_t C) {
@@ -424,10 +842,32 @@ cudaError_t tc_gla_chunk_out(const void* q, const void* k, const void* v, const 
   if (!make_token_map(&mq, q, B, H, N, kD, kTile) || !make_token_map(&mk, k, B, H, N, kD, kTile) ||
       !make_token_map(&mv, v, B, H, N, kD, kTile) || !make_token_map(&mo, o, B, H, N, kD, kTile))
     return cudaErrorInvalidValue;
-  const size_t smem = 1024 + 5 * (size_t)kTileBytes + sizeof(SmemOut);
+  const size_t smem = 1024 + 7 * (size_t)kTileBytes + sizeof(SmemOut);
   cudaError_t e = cudaFuncSetAttribute(gla_out_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   gla_out_tc<<<dim3((unsigned)(N / kTile), H, B), kThreads, smem, st>>>(mq, mk, mv, mo, g, P, H, N);
+  return cudaGetLastError();
+}
+
+}  // namespace lasp
+
+namespace lasp {
+
+cudaError_t tc_gla_chunk_bwd(const void* q, const void* k, const void* v, const void* dout, const float* g,
+                             const float* P, const float* Rs, void* dq, void* dk, void* dv, float* dg, int B, int H,
+                             int64_t N, cudaStream_t st) {
+  using namespace tc_gla_detail;
+  CUtensorMap mq, mk, mv, mdo, mdk, mdv;
+  if (!make_token_map(&mq, q, B, H, N, kD, kTile) || !make_token_map(&mk, k, B, H, N, kD, kTile) ||
+      !make_token_map(&mv, v, B, H, N, kD, kTile) || !make_token_map(&mdo, dout, B, H, N, kD, kTile) ||
+      !make_token_map(&mdk, dk, B, H, N, kD, kTile) || !make_token_map(&mdv, dv, B, H, N, kD, kTile))
+    return cudaErrorInvalidValue;
+  const size_t smem = 1024 + 7 * (size_t)kTileBytes + sizeof(SmemBwd);
+  cudaError_t e = cudaFuncSetAttribute(gla_bwd_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  gla_bwd_tc<<<dim3((unsigned)(N / kTile), H, B), kThreads, smem, st>>>(
+      mq, mk, mv, mdo, mdk, mdv, g, P, Rs, (const __nv_bfloat16*)q, (const __nv_bfloat16*)k, (__nv_bfloat16*)dq, dg,
+      H, N);
   return cudaGetLastError();
 }
 

@@ -111,6 +111,10 @@ int lasp_gla_bwd(const void* q, const void* k, const void* v, const float* g, co
   // dinit); 3. dQ, dK, dV and the log-gate gradient
   if ((s = states_impl(q, dout, g, dstate_ws, nullptr, B, H, N, d, C, dtype, 1, st))) return s;
   if ((s = scan_impl(dstate_ws, dstate_ws, gsum, dstate_in, dinit_state, B, T, H, d, 1, st))) return s;
+  if (tc_gla_ok(dtype, d, C))
+    return cuda_status(traced(K_GLA_BWD_TC, st, [&] {
+      return tc_gla_chunk_bwd(q, k, v, dout, g, state_cache, dstate_ws, dq, dk, dv, dg, B, H, N, st);
+    }));
   return cuda_status(traced(K_GLA_BWD, st, [&] {
     return gla_simt_chunk_bwd(q, k, v, dout, g, state_cache, dstate_ws, dq, dk, dv, dg, B, H, N, d, C, dtype, st);
   }));

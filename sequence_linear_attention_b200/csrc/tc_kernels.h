@@ -68,5 +68,8 @@ cudaError_t tc_gla_chunk_states(const void* x, const void* y, const float* g, fl
                                 int64_t N, int kind, cudaStream_t st);
 cudaError_t tc_gla_chunk_out(const void* q, const void* k, const void* v, const float* g, const float* P, void* o,
                              int B, int H, int64_t N, cudaStream_t st);
+cudaError_t tc_gla_chunk_bwd(const void* q, const void* k, const void* v, const void* dout, const float* g,
+                             const float* P, const float* Rs, void* dq, void* dk, void* dv, float* dg, int B, int H,
+                             int64_t N, cudaStream_t st);
 
 }  // namespace lasp
