@@ -55,6 +55,12 @@ def algorithmic_bytes(name: str, tokens_heads: int, d: int, C: int, G: int, elem
       chunk_bwd_*:  read q, k, v, dO, P and R, write dq, dk, dv          = 7de + 2s/C
       bwd_walk_tc:  read q, k, v, dO, the cached bf16 tiles (s/256) and the
                     segment's R (s/G), write dq, dk, dv            = 7de + s/256 + s/G
+    Gated form (a log-gate per token and key feature, fp32: 4d bytes):
+      gla_states_*: read 2 token rows and the gates, write s/C         = 2de + 4d + s/C
+      gla_scan:     read and write s/C, read the chunk's gate totals   = 2s/C + 4d/C
+      gla_out_*:    read q, k, v, the gates and P, write o             = 4de + 4d + s/C
+      gla_bwd_*:    read q, k, v, dO, the gates, P and R, write dq, dk,
+                    dv and the gate gradient                          = 7de + 8d + 2s/C
     """
     s = 4 * d * d
     de = d * elem
@@ -68,6 +74,10 @@ def algorithmic_bytes(name: str, tokens_heads: int, d: int, C: int, G: int, elem
         # bidirectional form: the sum of the segment states (s/G; the total and
         # its tile per (b, h) are negligible), and one token tensor in, one out
         "bidir_total": s / G, "bidir_apply_tc": 2 * de,
+        "gla_states_tc": 2 * de + 4 * d + s / C, "gla_states_simt": 2 * de + 4 * d + s / C,
+        "gla_scan": 2 * s / C + 4 * d / C,
+        "gla_out_tc": 4 * de + 4 * d + s / C, "gla_out_simt": 4 * de + 4 * d + s / C,
+        "gla_bwd_tc": 7 * de + 8 * d + 2 * s / C, "gla_bwd_simt": 7 * de + 8 * d + 2 * s / C,
     }[name]
     return per * tokens_heads
 
@@ -430,6 +440,86 @@ def run_bidir(args, rank, world, local):
     }
 
 
+def run_gated(args, rank, world, local):
+    """The gated form (a log-gate per token and key feature) on the workload's
+    shapes, C = 128: a step is lasp_gla_fwd + lasp_gla_bwd, gates
+    log(sigmoid(x)) / 16. Printed as its own line, with its own metric; the
+    default run does not include it."""
+    import torch
+    import sequence_linear_attention_b200 as lasp
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    w = lasp_inputs.WORKLOADS[args.workload]
+    B, N, H, d, C = w["B"], (args.tokens or w["N"]), w["H"], w["d"], 128
+    if not w["bf16"] or d != 128 or N % C:
+        raise ValueError("the gated form is timed on a bf16 workload with d = 128 and N a multiple of 128")
+    seed = w["seed"] + 7919 * rank
+    inp = lasp_inputs.make_inputs(B, N, H, d, seed=seed, bf16=True, decayed=False)
+    q, k, v, do = (torch.from_numpy(np.ascontiguousarray(inp[n]).view(np.int16)).view(torch.bfloat16).to(dev)
+                   for n in ("q", "k", "v", "do"))
+    g = torch.from_numpy(lasp_inputs.make_log_gates(B, N, H, d, seed=seed)).to(dev)
+    o, dq, dk, dv = (torch.empty_like(q) for _ in range(4))
+    dg = torch.empty_like(g)
+    cache = torch.empty(lasp.lasp_gla_cache_floats(B, H, N, d, C), dtype=torch.float32, device=dev)
+    ws = torch.empty(B * (N // C) * H * d * d, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        lasp.lasp_gla_fwd(q, k, v, g, o, C, cache)
+        lasp.lasp_gla_bwd(q, k, v, g, do, dq, dk, dv, dg, C, cache, ws)
+
+    for _ in range(args.warmup):
+        step()
+    events = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    torch.cuda.synchronize(dev)
+    barrier(world, dev)
+    with ClockSampler(local) as clk:
+        for i in range(args.steps):
+            events[i][0].record(stream)
+            step()
+            events[i][1].record(stream)
+        torch.cuda.synchronize(dev)
+    barrier(world, dev)
+    tokens = B * N
+    value, t_max = aggregate(tokens * args.steps, sum(a.elapsed_time(b) for a, b in events) / 1e3, world, dev)
+    ksteps = min(args.steps, 200)
+    lasp.lasp_trace_enable(16 * ksteps + 16)
+    for _ in range(ksteps):
+        step()
+    torch.cuda.synchronize(dev)
+    trace = lasp.lasp_trace_read(16 * ksteps + 16)
+    lasp.lasp_trace_enable(0)
+    st, site = lasp.lasp_check_device_status()
+    if st != 0:
+        raise RuntimeError(f"device status {lasp.lasp_status_string(st)} at site {site}")
+    per_kernel = {}
+    for name, ms in trace:
+        per_kernel.setdefault(name, []).append(ms)
+    peaks = load_peaks()
+    th = tokens * H
+    kernel_table = {}
+    for n, ms in per_kernel.items():
+        mean = statistics.mean(ms)
+        gbps = algorithmic_bytes(n, th, d, C, C, 2) / (mean / 1e3) / 1e9
+        kernel_table[n] = {"launches_per_step": len(ms) / ksteps, "ms": round(mean, 4), "GBps": round(gbps, 1),
+                           "hbm_frac": round(gbps / peaks["hbm"], 4)}
+    top = max(per_kernel, key=lambda n: sum(per_kernel[n]))
+    return {
+        "metric": "gated linear-attn fwd+bwd tokens/s", "impl": "gated",
+        "value": round(value, 1), "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(t_max * 1e3 / args.steps, 4), "higher_is_better": True,
+        "dtype": "bf16", "data": "synthetic (seeded normal q,k,v,dO; log-gates log(sigmoid(x))/16; no dataset)",
+        "config": {"workload": args.workload, "B": B, "H": H, "N": N, "d": d, "C": C, "gates": "log(sigmoid(x))/16",
+                   "l2": "inputs larger than L2"},
+        "roofline": {"bound": "hbm", "kernel": top, "achieved": kernel_table[top]["GBps"], "peak": peaks["hbm"],
+                     "unit": "GB/s", "frac": kernel_table[top]["hbm_frac"], "peak_source": peaks["source"]},
+        "kernels": kernel_table,
+        "gpu_launches": int(round(len(trace) / ksteps * args.steps)),
+        "clocks": clk.summary(),
+    }
+
+
 # ------------------------------------------------------------------ CPU oracle
 def oracle_sample(args, tokens: int):
     """A bounded sample of the workload for the fp64 oracle: all heads, the
@@ -497,6 +587,8 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--bidir", action="store_true",
                     help="time the bidirectional (unmasked) form instead (its own metric and line)")
+    ap.add_argument("--gated", action="store_true",
+                    help="time the gated form (a log-gate per token and key feature) instead (its own metric and line)")
     ap.add_argument("--tokens", type=int, default=None,
                     help="sequence length N instead of the workload's (a smaller case of the same shape, for "
                          "profiling); the line is then not the workload's headline number")
@@ -509,6 +601,8 @@ def main(argv=None):
             line = run_reference(args, rank, world)
         elif args.bidir:
             line = run_bidir(args, rank, world, local)
+        elif args.gated:
+            line = run_gated(args, rank, world, local)
         else:
             line = run_gpu(args, rank, world, local)
             if rank == 0 and world == 1 and not args.no_cpu_baseline:
