@@ -93,12 +93,15 @@ def flops_per_step(tokens_heads: int, d: int, C: int) -> float:
 MEASURED_TRAFFIC = {
     # DRAM bytes per launch at the workload's full size: twice the ncu capture of
     # the 32768-token case of the same workload (traffic grows with the tokens)
-    "bwd_walk_tc": (["k_tc_bwd_walk.cu", "sm100.cuh", "lasp_common.cuh", "tma_host.h"], "20c936251fd30878",
-                    2 * (726024448 + 368554240)),
-    "fwd_walk_tc": (["k_tc_fwd_walk.cu", "sm100.cuh", "lasp_common.cuh", "tma_host.h"], "659ed7f878139615",
-                    2 * (437606656 + 230750464)),
-    "segment_states_tc": (["k_tc_states.cu", "sm100.cuh", "lasp_common.cuh", "tma_host.h"], "0124abcfbf954d17",
-                          2 * (268472064 + 23057408)),
+    "bwd_walk_tc": (["k_tc_bwd_walk.cu", "sm100.cuh", "lasp_common.cuh", "tma_host.h"], "abcc9f96a59d67ba",
+                    2 * (723881216 + 367207936)),
+    "fwd_walk_tc": (["k_tc_fwd_walk.cu", "sm100.cuh", "lasp_common.cuh", "tma_host.h"], "4c265c8661c3ab71",
+                    2 * (437796352 + 231188992)),
+    "segment_states_tc": (["k_tc_states.cu", "sm100.cuh", "lasp_common.cuh", "tma_host.h"], "38b8cf4a1ea255d1",
+                          2 * (268475648 + 5562368)),
+    # the gated form (bench.py --gated): four times the capture of the 16384-token case
+    "gla_bwd_tc": (["k_tc_gla.cu", "sm100.cuh", "lasp_common.cuh", "tma_host.h"], "3290bd8ff6500364",
+                   4 * (777136896 + 290975488)),
 }
 
 
@@ -513,7 +516,9 @@ def run_gated(args, rank, world, local):
         "config": {"workload": args.workload, "B": B, "H": H, "N": N, "d": d, "C": C, "gates": "log(sigmoid(x))/16",
                    "l2": "inputs larger than L2"},
         "roofline": {"bound": "hbm", "kernel": top, "achieved": kernel_table[top]["GBps"], "peak": peaks["hbm"],
-                     "unit": "GB/s", "frac": kernel_table[top]["hbm_frac"], "peak_source": peaks["source"]},
+                     "unit": "GB/s", "frac": kernel_table[top]["hbm_frac"],
+                     "traffic": measured_traffic(top, args.workload) if N == w["N"] else None,
+                     "algorithmic_bytes": algorithmic_bytes(top, th, d, C, C, 2), "peak_source": peaks["source"]},
         "kernels": kernel_table,
         "gpu_launches": int(round(len(trace) / ksteps * args.steps)),
         "clocks": clk.summary(),

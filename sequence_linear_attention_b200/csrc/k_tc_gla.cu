@@ -107,34 +107,55 @@ __device__ __forceinline__ void walk_gates(const float* __restrict__ g_chunk, in
   }
 }
 
-// Element (t, i) of the [128][128] fp32 gate tile: float4 slots XOR-swizzled
-// by the row, so that a warp walking 32 features of one row and a warp reading
-// float4s of 32 different rows both touch every bank once.
-__device__ __forceinline__ int gate_slot(int t, int i) { return t * kD + 4 * ((i >> 2) ^ (t & 7)) + (i & 3); }
+// Element (t, i) of a [128][128] fp32 tile as the gate map's TMA loads lay it
+// out: four 32-feature blocks of 128 lines of 128 bytes, 16-byte chunk c of
+// line t at chunk c ^ (t % 8). A warp walking 32 features of one line and a
+// warp reading float4s of 32 different lines both touch every bank once.
+__device__ __forceinline__ int gate_slot(int t, int i) {
+  return (i >> 5) * (kTile * 32) + t * 32 + 4 * (((i & 31) >> 2) ^ (t & 7)) + (i & 3);
+}
 
-// Warps 0-3: b_t[i] = sum_{r<=t} g_r[i] (natural log) into the tile `bt`, and
-// b at the middle row into r[], at the last row into bend[].
-__device__ __forceinline__ void walk_gates_to_tile(const float* __restrict__ g_chunk, int64_t row_stride, int i,
-                                                   float* bt, float* r, float* bend) {
+// Feature i (one per thread of warps 0-3): the log-gates of the tile become
+// b_t[i] = sum_{r<=t} g_r[i] in place; b at the middle row goes to r[], at the
+// last row to bend[].
+__device__ __forceinline__ void walk_tile(float* bt, int i, float* r, float* bend) {
   float acc = 0.f;
-  walk_gates(g_chunk, row_stride, i, false, [&](int t, float gt) {
-    acc += gt;
-    bt[gate_slot(t, i)] = acc;
-    if (t == kTile / 2 - 1) r[i] = acc;
-  });
+#pragma unroll 1
+  for (int t0 = 0; t0 < kTile; t0 += 8) {
+    float v[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) v[u] = bt[gate_slot(t0 + u, i)];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      acc += v[u];
+      bt[gate_slot(t0 + u, i)] = acc;
+      if (t0 + u == kTile / 2 - 1) r[i] = acc;
+    }
+  }
   bend[i] = acc;
 }
 
-// The 64 values of row t, columns half*64.., of the gate tile.
+// The 64 values of row t, columns half*64.., of such a tile.
 __device__ __forceinline__ void read_gate_row(const float* bt, int t, int half, float (&b)[64]) {
 #pragma unroll
-  for (int q = 0; q < 16; ++q) {
-    const float4 v = *reinterpret_cast<const float4*>(bt + t * kD + 4 * ((half * 16 + q) ^ (t & 7)));
-    b[4 * q] = v.x;
-    b[4 * q + 1] = v.y;
-    b[4 * q + 2] = v.z;
-    b[4 * q + 3] = v.w;
-  }
+  for (int cb = 0; cb < 2; ++cb)
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      const float4 v =
+          *reinterpret_cast<const float4*>(bt + (2 * half + cb) * (kTile * 32) + t * 32 + 4 * (q ^ (t & 7)));
+      b[cb * 32 + 4 * q] = v.x;
+      b[cb * 32 + 4 * q + 1] = v.y;
+      b[cb * 32 + 4 * q + 2] = v.z;
+      b[cb * 32 + 4 * q + 3] = v.w;
+    }
+}
+
+// Four TMA loads of the chunk's log-gates (fp32, 64 KB) into the tile.
+__device__ __forceinline__ void load_gate_tile(float* bt, const CUtensorMap* map_g, uint64_t* bar, int h, int row0,
+                                               int b) {
+  mbar_arrive_expect_tx(bar, kTile * kD * 4);
+#pragma unroll
+  for (int cb = 0; cb < 4; ++cb) tma_load_4d(bt + cb * (kTile * 32), map_g, bar, cb * 32, h, row0, b);
 }
 
 // fp32 d x d state rows (global) -> bf16 operand tile, row m scaled by w[u]
@@ -255,14 +276,16 @@ cleanup:
   if (warp == 0) tmem_dealloc(tmem, 128);
 }
 
-// Phase 0 of the output and backward kernels: the walk into the gate tile
-// (warps 0-3; b at the middle row into r[], at the last row into bend[]), then,
-// for row t and column half `half` of every thread, the range check and
-// x = (b_t - r) log2 e, returned in x[].
-__device__ __forceinline__ void gate_rows(const float* __restrict__ g, int64_t N, int H, int b, int h, int64_t row0,
-                                          float* bt, float* r, float* bend, int tid, int t, int half, float (&x)[64]) {
-  if (tid < kD)
-    walk_gates_to_tile(g + ((int64_t)b * N + row0) * H * kD + (int64_t)h * kD, (int64_t)H * kD, tid, bt, r, bend);
+// Phase 0 of the output and backward kernels: once the gate tile has landed
+// (barrier gbar), its walk (warps 0-3; b at the middle row into r[], at the
+// last row into bend[]), then, for row t and column half `half` of every
+// thread, the range check and x = (b_t - r) log2 e, returned in x[].
+__device__ __forceinline__ void gate_rows(float* bt, uint64_t* gbar, int* abort, unsigned int site, float* r,
+                                          float* bend, int tid, int t, int half, float (&x)[64]) {
+  if (tid < kD) {
+    if (!mbar_wait(gbar, 0, site)) *abort = 1;
+    walk_tile(bt, tid, r, bend);
+  }
   named_sync(kBarAll, kThreads);
   read_gate_row(bt, t, half, x);
   bool ok = true;
@@ -277,7 +300,7 @@ __device__ __forceinline__ void gate_rows(const float* __restrict__ g, int64_t N
 
 // ---------------------------------------------------------------- output
 struct SmemOut {
-  uint64_t load, mma1, mma2;
+  uint64_t gload, load, mma1, mma2;
   uint32_t tmem_base;
   int abort;
   float r[kD], bend[kD];
@@ -287,8 +310,8 @@ __global__ void __launch_bounds__(kThreads, 1) gla_out_tc(const __grid_constant_
                                                           const __grid_constant__ CUtensorMap map_k,
                                                           const __grid_constant__ CUtensorMap map_v,
                                                           const __grid_constant__ CUtensorMap map_o,
-                                                          const float* __restrict__ g, const float* __restrict__ P,
-                                                          int H, int64_t N) {
+                                                          const __grid_constant__ CUtensorMap map_g,
+                                                          const float* __restrict__ P, int H, int64_t N) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   uint8_t* sQ = base;                   // Q^
@@ -308,6 +331,8 @@ __global__ void __launch_bounds__(kThreads, 1) gla_out_tc(const __grid_constant_
     prefetch_tmap(&map_k);
     prefetch_tmap(&map_v);
     prefetch_tmap(&map_o);
+    prefetch_tmap(&map_g);
+    mbar_init(&s->gload, 1);
     mbar_init(&s->load, 1);
     mbar_init(&s->mma1, 1);
     mbar_init(&s->mma2, 1);
@@ -325,6 +350,7 @@ __global__ void __launch_bounds__(kThreads, 1) gla_out_tc(const __grid_constant_
   const uint32_t lane_base = tmem + ((uint32_t)((warp & 3) * 32) << 16);
   const uint32_t T0 = 0, T1 = 128;
   if (tid == 0) {
+    load_gate_tile(bt, &map_g, &s->gload, h, (int)row0, b);
     mbar_arrive_expect_tx(&s->load, 3 * kTileBytes);
     tma_load_4d(sQ, &map_q, &s->load, 0, h, (int)row0, b);
     tma_load_4d(sQ + kBox, &map_q, &s->load, 64, h, (int)row0, b);
@@ -334,7 +360,7 @@ __global__ void __launch_bounds__(kThreads, 1) gla_out_tc(const __grid_constant_
     tma_load_4d(sV + kBox, &map_v, &s->load, 64, h, (int)row0, b);
   }
   float x[64];
-  gate_rows(g, N, H, b, h, row0, bt, s->r, s->bend, tid, t, half, x);
+  gate_rows(bt, &s->gload, &s->abort, SITE_OUT_TMA, s->r, s->bend, tid, t, half, x);
   // P' = diag(e^{r}) P_c into X
   {
     float w[16];
@@ -426,49 +452,6 @@ cleanup:
 }
 
 // ---------------------------------------------------------------- gradients
-// Scans down the tile's 128 rows, for the 32 columns each thread holds of its
-// row t = 32 (warp % 4) + lane: suf[u] <- sum_{t' >= t}, pre[u] <- sum_{t' < t}.
-// Shuffles inside each warp's 32 rows; the warps' totals through tot[512].
-__device__ __forceinline__ void row_scans(float (&suf)[32], float (&pre)[32], int warp, int lane, int half,
-                                          float* tot) {
-  const int wq = warp & 3;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-#pragma unroll
-    for (int u = 0; u < 32; ++u) {
-      const float ys = __shfl_down_sync(0xffffffffu, suf[u], o);
-      const float yp = __shfl_up_sync(0xffffffffu, pre[u], o);
-      if (lane + o < 32) suf[u] += ys;
-      if (lane >= o) pre[u] += yp;
-    }
-  }
-  // warp totals: the suffix sum at lane 0, the inclusive prefix at lane 31
-  if (lane == 0) {
-#pragma unroll
-    for (int u = 0; u < 32; ++u) tot[((half * 2) * 4 + wq) * 32 + u] = suf[u];
-  }
-  if (lane == 31) {
-#pragma unroll
-    for (int u = 0; u < 32; ++u) tot[((half * 2 + 1) * 4 + wq) * 32 + u] = pre[u];
-  }
-  // inclusive -> exclusive prefix
-#pragma unroll
-  for (int u = 0; u < 32; ++u) {
-    const float y = __shfl_up_sync(0xffffffffu, pre[u], 1);
-    pre[u] = lane == 0 ? 0.f : y;
-  }
-  named_sync(kBarAll, kThreads);
-  for (int w2 = wq + 1; w2 < 4; ++w2) {
-#pragma unroll
-    for (int u = 0; u < 32; ++u) suf[u] += tot[((half * 2) * 4 + w2) * 32 + u];
-  }
-  for (int w2 = 0; w2 < wq; ++w2) {
-#pragma unroll
-    for (int u = 0; u < 32; ++u) pre[u] += tot[((half * 2 + 1) * 4 + w2) * 32 + u];
-  }
-  named_sync(kBarAll, kThreads);  // tot is rewritten by the next call
-}
-
 // 32 bf16 values of a token row (global), from column col0.
 __device__ __forceinline__ void load_row32(const __nv_bfloat16* p, float (&v)[32]) {
   const uint4* p4 = reinterpret_cast<const uint4*>(p);
@@ -486,24 +469,25 @@ __device__ __forceinline__ void load_row32(const __nv_bfloat16* p, float (&v)[32
 }
 
 struct SmemBwd {
-  uint64_t load, mma1a, mma1b, mma2, mma3;
+  uint64_t gload, load, mma1a, mma1b, mma2, mma3;
   uint32_t tmem_base;
   int abort;
   float dAd[kTile];  // do_t . v_t, the diagonal of dO V^T
   float bnd[kD];     // e^{b_end[i]} <R_c[i], P_c[i]>
 };
 
-// One 128-token chunk per CTA. Shared memory: Q^, K^, V, dO, X (P', then R';
-// r and b_end during the gate walk; the scan totals at the end), and the pair
+// One 128-token chunk per CTA. Shared memory: Q^, K^, V, dO (then, in pairs,
+// the fp32 tiles of dB and k . dk^inter for the log-gate gradient's column
+// sums), X (P', then R'; r and b_end during the gate walk), and the pair
 // sA / sB (the gate tile during the walk; then dA . strict and A . causal;
-// then the dK and dV outputs). TMEM: T0 = dO V^T -> (dA . strict)^T Q^ -> dB;
+// then the dK and dV outputs). TMEM: T0 = dO V^T -> (dA . strict)^T Q^;
 // T1 = Q^ K^^T -> dV; T2 = dO P'^T + (dA . strict) K^ -> q . dq'; T3 = log2 E
-// -> V R'^T -> k . dk^inter.
+// -> V R'^T.
 __global__ void __launch_bounds__(kThreads, 1) gla_bwd_tc(
     const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
     const __grid_constant__ CUtensorMap map_v, const __grid_constant__ CUtensorMap map_do,
     const __grid_constant__ CUtensorMap map_dk, const __grid_constant__ CUtensorMap map_dv,
-    const float* __restrict__ g, const float* __restrict__ P, const float* __restrict__ R,
+    const __grid_constant__ CUtensorMap map_g, const float* __restrict__ P, const float* __restrict__ R,
     const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k, __nv_bfloat16* __restrict__ dq,
     float* __restrict__ dg, int H, int64_t N) {
   extern __shared__ uint8_t smem_raw[];
@@ -519,7 +503,6 @@ __global__ void __launch_bounds__(kThreads, 1) gla_bwd_tc(
   float* bt = reinterpret_cast<float*>(sA);  // gate tile over sA and sB during the walk
   float* sr = reinterpret_cast<float*>(sX);  // r and b_end over X during the walk
   float* sbend = sr + kD;
-  float* tot = reinterpret_cast<float*>(sX);  // scan totals over X at the end
   const int c = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int t = (warp & 3) * 32 + lane, half = warp >> 2;
@@ -532,6 +515,8 @@ __global__ void __launch_bounds__(kThreads, 1) gla_bwd_tc(
     prefetch_tmap(&map_k);
     prefetch_tmap(&map_v);
     prefetch_tmap(&map_do);
+    prefetch_tmap(&map_g);
+    mbar_init(&s->gload, 1);
     mbar_init(&s->load, 1);
     mbar_init(&s->mma1a, 1);
     mbar_init(&s->mma1b, 1);
@@ -551,6 +536,7 @@ __global__ void __launch_bounds__(kThreads, 1) gla_bwd_tc(
   const uint32_t lane_base = tmem + ((uint32_t)((warp & 3) * 32) << 16);
   const uint32_t T0 = 0, T1 = 128, T2 = 256, T3 = 384;
   if (tid == 0) {
+    load_gate_tile(bt, &map_g, &s->gload, h, (int)row0, b);
     mbar_arrive_expect_tx(&s->load, 4 * kTileBytes);
     tma_load_4d(sQ, &map_q, &s->load, 0, h, (int)row0, b);
     tma_load_4d(sQ + kBox, &map_q, &s->load, 64, h, (int)row0, b);
@@ -563,7 +549,7 @@ __global__ void __launch_bounds__(kThreads, 1) gla_bwd_tc(
   }
   // ---- phase 0: gates, Q^, K^, log2 E -> T3, P' -> X
   float x[64];
-  gate_rows(g, N, H, b, h, row0, bt, sr, sbend, tid, t, half, x);
+  gate_rows(bt, &s->gload, &s->abort, SITE_BWD_TMA, sr, sbend, tid, t, half, x);
   float wr[16], we[16];  // e^{r_m} and e^{b_end_m - r_m} of this thread's state rows m = warp + 8u
 #pragma unroll
   for (int u = 0; u < 16; ++u) {
@@ -726,7 +712,10 @@ __global__ void __launch_bounds__(kThreads, 1) gla_bwd_tc(
       for (int kk = 0; kk < kD / 16; ++kk) mma_bf16(tmem + T3, kmaj(aV, kk), kmaj(aX, kk), id_kk, kk != 0);
       mma_commit(&s->mma3);
     }
-    // ---- epilogue 3: dk, dv -> sA, sB; dB = q . dq' - k . dk', k . dk^inter -> T0, T3; dg
+    // ---- epilogue 3: dk, dv -> sA, sB; dB = q . dq' - k . dk' and k . dk^inter
+    // as fp32 tiles over the token buffers (all MMAs have read them)
+    float* fB = reinterpret_cast<float*>(sQ);  // over sQ and sK
+    float* fK = reinterpret_cast<float*>(sV);  // over sV and sD
     if (mbar_wait(&s->mma3, 0, SITE_BWD_MMA)) {
       tc_fence_after();
       const float dad = s->dAd[t];
@@ -742,6 +731,7 @@ __global__ void __launch_bounds__(kThreads, 1) gla_bwd_tc(
         load_row32(k + tok + col0, kv);
         tmem_ld_wait();
         uint32_t out[16];
+        float db[32], kd[32];
 #pragma unroll
         for (int u = 0; u < 32; ++u) {
           const float ei = exp2f(-xl[c2 * 32 + u]);
@@ -752,14 +742,19 @@ __global__ void __launch_bounds__(kThreads, 1) gla_bwd_tc(
             out[u / 2] = pack_bf16(__uint_as_float(out[u / 2]), full);
           else
             out[u / 2] = __float_as_uint(full);
-          ka[u] = __float_as_uint(__uint_as_float(bq[u]) - kv[u] * dka);
-          kb[u] = __float_as_uint(kv[u] * dkb);
+          db[u] = __uint_as_float(bq[u]) - kv[u] * dka;
+          kd[u] = kv[u] * dkb;
         }
 #pragma unroll
         for (int q4 = 0; q4 < 4; ++q4)
           *tile16(sA, t, col0 + q4 * 8) = make_uint4(out[4 * q4], out[4 * q4 + 1], out[4 * q4 + 2], out[4 * q4 + 3]);
-        tmem_st32(lane_base + T0 + col0, ka);
-        tmem_st32(lane_base + T3 + col0, kb);
+#pragma unroll
+        for (int q4 = 0; q4 < 8; ++q4) {
+          *reinterpret_cast<float4*>(fB + gate_slot(t, col0 + 4 * q4)) =
+              make_float4(db[4 * q4], db[4 * q4 + 1], db[4 * q4 + 2], db[4 * q4 + 3]);
+          *reinterpret_cast<float4*>(fK + gate_slot(t, col0 + 4 * q4)) =
+              make_float4(kd[4 * q4], kd[4 * q4 + 1], kd[4 * q4 + 2], kd[4 * q4 + 3]);
+        }
         uint32_t dvv[32];
         tmem_ld32(lane_base + T1 + col0, dvv);
         tmem_ld_wait();
@@ -771,33 +766,54 @@ __global__ void __launch_bounds__(kThreads, 1) gla_bwd_tc(
                          pack_bf16(__uint_as_float(dvv[q4 * 8 + 4]), __uint_as_float(dvv[q4 * 8 + 5])),
                          pack_bf16(__uint_as_float(dvv[q4 * 8 + 6]), __uint_as_float(dvv[q4 * 8 + 7])));
       }
-      tmem_st_wait();
       fence_async_smem();
     } else {
       s->abort = 1;
     }
-    // dg_t = sum_{t' >= t} dB_t' + sum_{t' < t} k . dk^inter_t' + e^{b_end} <R_c, P_c>
+    __syncthreads();
+    // dg_t = sum_{t' >= t} dB_t' + sum_{t' < t} k . dk^inter_t' + e^{b_end} <R_c, P_c>: the
+    // two sums by column walks (threads 0-127 the suffix of dB, 128-255 the
+    // exclusive prefix of k . dk^inter, one feature each), in place
+    {
+      const int i = tid & (kD - 1);
+      float acc = 0.f;
+      if (tid < kD) {
 #pragma unroll 1
-    for (int c2 = 0; c2 < 2; ++c2) {
-      const int col0 = half * 64 + c2 * 32;
-      uint32_t a[32], e[32];
-      tmem_ld32(lane_base + T0 + col0, a);
-      tmem_ld32(lane_base + T3 + col0, e);
-      tmem_ld_wait();
-      float suf[32], pre[32];
+        for (int t0 = kTile - 8; t0 >= 0; t0 -= 8) {
+          float v[8];
 #pragma unroll
-      for (int u = 0; u < 32; ++u) {
-        suf[u] = __uint_as_float(a[u]);
-        pre[u] = __uint_as_float(e[u]);
+          for (int u = 7; u >= 0; --u) v[u] = fB[gate_slot(t0 + u, i)];
+#pragma unroll
+          for (int u = 7; u >= 0; --u) {
+            acc += v[u];
+            fB[gate_slot(t0 + u, i)] = acc;
+          }
+        }
+      } else {
+#pragma unroll 1
+        for (int t0 = 0; t0 < kTile; t0 += 8) {
+          float v[8];
+#pragma unroll
+          for (int u = 0; u < 8; ++u) v[u] = fK[gate_slot(t0 + u, i)];
+#pragma unroll
+          for (int u = 0; u < 8; ++u) {
+            fK[gate_slot(t0 + u, i)] = acc;
+            acc += v[u];
+          }
+        }
       }
-      row_scans(suf, pre, warp, lane, half, tot);
+    }
+    __syncthreads();
+#pragma unroll
+    for (int cb = 0; cb < 2; ++cb) {
+      const int col0 = half * 64 + cb * 32;
       float4* dst = reinterpret_cast<float4*>(dg + tok + col0);
 #pragma unroll
       for (int q4 = 0; q4 < 8; ++q4) {
-        float o[4];
-#pragma unroll
-        for (int u = 0; u < 4; ++u) o[u] = suf[4 * q4 + u] + pre[4 * q4 + u] + s->bnd[col0 + 4 * q4 + u];
-        dst[q4] = make_float4(o[0], o[1], o[2], o[3]);
+        const float4 a = *reinterpret_cast<const float4*>(fB + gate_slot(t, col0 + 4 * q4));
+        const float4 e = *reinterpret_cast<const float4*>(fK + gate_slot(t, col0 + 4 * q4));
+        const float* bn = s->bnd + col0 + 4 * q4;
+        dst[q4] = make_float4(a.x + e.x + bn[0], a.y + e.y + bn[1], a.z + e.z + bn[2], a.w + e.w + bn[3]);
       }
     }
     __syncthreads();
@@ -838,14 +854,15 @@ cudaError_t tc_gla_chunk_states(const void* x, const void* y, const float* g, fl
 cudaError_t tc_gla_chunk_out(const void* q, const void* k, const void* v, const float* g, const float* P, void* o,
                              int B, int H, int64_t N, cudaStream_t st) {
   using namespace tc_gla_detail;
-  CUtensorMap mq, mk, mv, mo;
+  CUtensorMap mq, mk, mv, mo, mg;
   if (!make_token_map(&mq, q, B, H, N, kD, kTile) || !make_token_map(&mk, k, B, H, N, kD, kTile) ||
-      !make_token_map(&mv, v, B, H, N, kD, kTile) || !make_token_map(&mo, o, B, H, N, kD, kTile))
+      !make_token_map(&mv, v, B, H, N, kD, kTile) || !make_token_map(&mo, o, B, H, N, kD, kTile) ||
+      !make_gate_map(&mg, g, B, H, N, kD, kTile))
     return cudaErrorInvalidValue;
   const size_t smem = 1024 + 7 * (size_t)kTileBytes + sizeof(SmemOut);
   cudaError_t e = cudaFuncSetAttribute(gla_out_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  gla_out_tc<<<dim3((unsigned)(N / kTile), H, B), kThreads, smem, st>>>(mq, mk, mv, mo, g, P, H, N);
+  gla_out_tc<<<dim3((unsigned)(N / kTile), H, B), kThreads, smem, st>>>(mq, mk, mv, mo, mg, P, H, N);
   return cudaGetLastError();
 }
 
@@ -857,17 +874,18 @@ cudaError_t tc_gla_chunk_bwd(const void* q, const void* k, const void* v, const 
                              const float* P, const float* Rs, void* dq, void* dk, void* dv, float* dg, int B, int H,
                              int64_t N, cudaStream_t st) {
   using namespace tc_gla_detail;
-  CUtensorMap mq, mk, mv, mdo, mdk, mdv;
+  CUtensorMap mq, mk, mv, mdo, mdk, mdv, mg;
   if (!make_token_map(&mq, q, B, H, N, kD, kTile) || !make_token_map(&mk, k, B, H, N, kD, kTile) ||
       !make_token_map(&mv, v, B, H, N, kD, kTile) || !make_token_map(&mdo, dout, B, H, N, kD, kTile) ||
-      !make_token_map(&mdk, dk, B, H, N, kD, kTile) || !make_token_map(&mdv, dv, B, H, N, kD, kTile))
+      !make_token_map(&mdk, dk, B, H, N, kD, kTile) || !make_token_map(&mdv, dv, B, H, N, kD, kTile) ||
+      !make_gate_map(&mg, g, B, H, N, kD, kTile))
     return cudaErrorInvalidValue;
   const size_t smem = 1024 + 7 * (size_t)kTileBytes + sizeof(SmemBwd);
   cudaError_t e = cudaFuncSetAttribute(gla_bwd_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   gla_bwd_tc<<<dim3((unsigned)(N / kTile), H, B), kThreads, smem, st>>>(
-      mq, mk, mv, mdo, mdk, mdv, g, P, Rs, (const __nv_bfloat16*)q, (const __nv_bfloat16*)k, (__nv_bfloat16*)dq, dg,
-      H, N);
+      mq, mk, mv, mdo, mdk, mdv, mg, P, Rs, (const __nv_bfloat16*)q, (const __nv_bfloat16*)k, (__nv_bfloat16*)dq,
+      dg, H, N);
   return cudaGetLastError();
 }
 

@@ -60,4 +60,21 @@ inline bool make_state_map(CUtensorMap* map, const float* base, int64_t nstates,
   return r == CUDA_SUCCESS;
 }
 
+// A 4-D view (d, H, N, B) of a [B, N, H, d] fp32 tensor (the log-gates of
+// the gated form); one box is 32 features x 1 head x `rows` tokens x 1 batch,
+// stored as `rows` lines of 128 bytes with the 128-byte swizzle (16-byte chunk
+// c of line t lands at chunk c ^ (t % 8)).
+inline bool make_gate_map(CUtensorMap* map, const float* base, int B, int H, int64_t N, int d, int rows) {
+  auto fn = tmap_encode_fn();
+  if (fn == nullptr) return false;
+  cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)H, (cuuint64_t)N, (cuuint64_t)B};
+  cuuint64_t strides[3] = {(cuuint64_t)d * 4, (cuuint64_t)H * d * 4, (cuuint64_t)N * H * d * 4};
+  cuuint32_t box[4] = {32, 1, (cuuint32_t)rows, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, const_cast<float*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 }  // namespace lasp
