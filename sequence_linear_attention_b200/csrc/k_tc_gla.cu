@@ -180,13 +180,16 @@ struct SmemStates {
   uint64_t load, mma;
   uint32_t tmem_base;
   int abort;
-  float bend[kD];
+  float half_tot[2][kD];  // the log-gates of each feature summed over each half of the chunk
 };
 
 // kind 0: M_c = (k . e^{b_end - b})^T v and gsum_c = b_end; kind 1: dM_c =
 // (q . e^{b})^T do. x, y: the two token operands ((k, v) or (q, do)); the gate
-// factor goes on x, scaled in place by the walker warps, the walk for kind 0
-// going up from the last row (e^{b_end - b_t} = e^{sum_{r>t} g_r}).
+// factor goes on x, scaled in place. Thread i of warps 0-3 and thread i of
+// warps 4-7 take feature i in the first and in the second half of the rows:
+// each sums its half's log-gates, then walks it again (down for kind 1, up
+// for kind 0: e^{b_end - b_t} = e^{sum_{r>t} g_r}) starting from the other
+// half's total where that half comes first.
 __global__ void __launch_bounds__(kThreads, 2) gla_states_tc(const __grid_constant__ CUtensorMap map_x,
                                                              const __grid_constant__ CUtensorMap map_y,
                                                              const float* __restrict__ g, float* __restrict__ M,
@@ -223,20 +226,45 @@ __global__ void __launch_bounds__(kThreads, 2) gla_states_tc(const __grid_consta
     tma_load_4d(sY, &map_y, &s->load, 0, h, (int)row0, b);
     tma_load_4d(sY + kBox, &map_y, &s->load, 64, h, (int)row0, b);
   }
-  if (warp < 4) {
-    const int i = tid;
+  {
+    constexpr int kHalf = kTile / 2;
+    const int i = tid & (kD - 1), hf = tid >> 7;
+    const int64_t rs = (int64_t)H * kD;
+    const float* gcol = g + ((int64_t)b * N + row0 + hf * kHalf) * rs + (int64_t)h * kD + i;
+    float tot = 0.f;
+#pragma unroll 1
+    for (int t0 = 0; t0 < kHalf; t0 += 16) {
+      float v[16];
+#pragma unroll
+      for (int u = 0; u < 16; ++u) v[u] = __ldg(gcol + (int64_t)(t0 + u) * rs);
+#pragma unroll
+      for (int u = 0; u < 16; ++u) tot += v[u];
+    }
+    s->half_tot[hf][i] = tot;
     const bool ok = mbar_wait(&s->load, 0, SITE_STATES_TMA);
     if (!ok) s->abort = 1;
+    __syncthreads();
+    // the part of the exponent from the other half: kind 1 sums down from row 0,
+    // kind 0 up from the last row
+    float acc = kind == 0 ? (hf == 0 ? s->half_tot[1][i] : 0.f) : (hf == 1 ? s->half_tot[0][i] : 0.f);
     __nv_bfloat16* col = reinterpret_cast<__nv_bfloat16*>(sX + (i >> 6) * kBox + (i & 7) * 2);
-    float acc = 0.f;
-    walk_gates<16>(g + ((int64_t)b * N + row0) * H * kD + (int64_t)h * kD, (int64_t)H * kD, i, kind == 0,
-               [&](int t, float gt) {
-                 if (kind != 0) acc += gt;
-                 __nv_bfloat16* e = col + sw128_offset(t, (i & 63) >> 3) / 2;
-                 if (ok) *e = __float2bfloat16_rn(__bfloat162float(*e) * exp2f(acc * kLog2e));
-                 if (kind == 0) acc += gt;
-               });
-    s->bend[i] = acc;  // the walk covers every row either way: acc = b_end
+#pragma unroll 1
+    for (int t0 = 0; t0 < kHalf; t0 += 16) {
+      float v[16];
+#pragma unroll
+      for (int u = 0; u < 16; ++u) {
+        const int tl = kind == 0 ? kHalf - 1 - (t0 + u) : t0 + u;
+        v[u] = __ldg(gcol + (int64_t)tl * rs);
+      }
+#pragma unroll
+      for (int u = 0; u < 16; ++u) {
+        const int t = hf * kHalf + (kind == 0 ? kHalf - 1 - (t0 + u) : t0 + u);
+        if (kind != 0) acc += v[u];
+        __nv_bfloat16* e = col + sw128_offset(t, (i & 63) >> 3) / 2;
+        if (ok) *e = __float2bfloat16_rn(__bfloat162float(*e) * exp2f(acc * kLog2e));
+        if (kind == 0) acc += v[u];
+      }
+    }
   }
   fence_async_smem();
   tc_fence_before();
@@ -249,7 +277,8 @@ __global__ void __launch_bounds__(kThreads, 2) gla_states_tc(const __grid_consta
     for (int kk = 0; kk < kTile / 16; ++kk) mma_bf16(tmem, mnmaj(aX, kk), mnmaj(aY, kk), id_nn, kk != 0);
     mma_commit(&s->mma);
   }
-  if (kind == 0 && gsum != nullptr && tid < kD) gsum[((b * T + c) * H + h) * kD + tid] = s->bend[tid];
+  if (kind == 0 && gsum != nullptr && tid < kD)
+    gsum[((b * T + c) * H + h) * kD + tid] = s->half_tot[0][tid] + s->half_tot[1][tid];
   if (mbar_wait(&s->mma, 0, SITE_STATES_MMA)) {
     tc_fence_after();
     // row i of M (TMEM lane i), columns half*64..
@@ -452,22 +481,6 @@ cleanup:
 }
 
 // ---------------------------------------------------------------- gradients
-// 32 bf16 values of a token row (global), from column col0.
-__device__ __forceinline__ void load_row32(const __nv_bfloat16* p, float (&v)[32]) {
-  const uint4* p4 = reinterpret_cast<const uint4*>(p);
-#pragma unroll
-  for (int q4 = 0; q4 < 4; ++q4) {
-    const uint4 w = __ldg(p4 + q4);
-    const uint32_t* e = reinterpret_cast<const uint32_t*>(&w);
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const float2 f = unpack_bf16(e[u]);
-      v[q4 * 8 + 2 * u] = f.x;
-      v[q4 * 8 + 2 * u + 1] = f.y;
-    }
-  }
-}
-
 struct SmemBwd {
   uint64_t gload, load, mma1a, mma1b, mma2, mma3;
   uint32_t tmem_base;
@@ -487,9 +500,8 @@ __global__ void __launch_bounds__(kThreads, 1) gla_bwd_tc(
     const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
     const __grid_constant__ CUtensorMap map_v, const __grid_constant__ CUtensorMap map_do,
     const __grid_constant__ CUtensorMap map_dk, const __grid_constant__ CUtensorMap map_dv,
-    const __grid_constant__ CUtensorMap map_g, const float* __restrict__ P, const float* __restrict__ R,
-    const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k, __nv_bfloat16* __restrict__ dq,
-    float* __restrict__ dg, int H, int64_t N) {
+    const __grid_constant__ CUtensorMap map_g, const __grid_constant__ CUtensorMap map_dg,
+    const float* __restrict__ P, const float* __restrict__ R, __nv_bfloat16* __restrict__ dq, int H, int64_t N) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   uint8_t* sQ = base;
@@ -537,6 +549,9 @@ __global__ void __launch_bounds__(kThreads, 1) gla_bwd_tc(
   const uint32_t T0 = 0, T1 = 128, T2 = 256, T3 = 384;
   if (tid == 0) {
     load_gate_tile(bt, &map_g, &s->gload, h, (int)row0, b);
+    // P and R are read with plain loads later: into L2 now
+    bulk_prefetch_l2(P + slot * kD * kD, kD * kD * 4);
+    bulk_prefetch_l2(R + slot * kD * kD, kD * kD * 4);
     mbar_arrive_expect_tx(&s->load, 4 * kTileBytes);
     tma_load_4d(sQ, &map_q, &s->load, 0, h, (int)row0, b);
     tma_load_4d(sQ + kBox, &map_q, &s->load, 64, h, (int)row0, b);
@@ -655,7 +670,8 @@ __global__ void __launch_bounds__(kThreads, 1) gla_bwd_tc(
       for (int kk = 0; kk < kTile / 16; ++kk) mma_bf16(tmem + T2, kmaj(aA, kk), mnmaj(aK, kk), id_kn, 1);
       mma_commit(&s->mma2);
     }
-    // ---- epilogue 2: dq' = E . T2; dq = dq' + (do_t . v_t) k_t; q . dq' -> T2
+    // ---- epilogue 2: dq' = E . T2; dq = dq' + (do_t . v_t) k_t = E . (T2 + (do_t . v_t) K^_t);
+    // q . dq' = Q^ . T2 -> T2
     float xl[64];  // log2 E of row t, kept for epilogue 3
     if (mbar_wait(&s->mma2, 0, SITE_BWD_MMA)) {
       tc_fence_after();
@@ -676,20 +692,25 @@ __global__ void __launch_bounds__(kThreads, 1) gla_bwd_tc(
         const int col0 = half * 64 + c2 * 32;
         uint32_t a[32];
         tmem_ld32(lane_base + T2 + col0, a);
-        float qv[32], kv[32];
-        load_row32(q + tok + col0, qv);
-        load_row32(k + tok + col0, kv);
+        // Q^ and K^ of row t (bf16, shared memory): q . dq' = Q^ . T2 and k_t = K^_t . E_t
+        uint32_t qh[16], kh[16];
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4) {
+          const uint4 wq = *tile16(sQ, t, col0 + q4 * 8);
+          const uint4 wk = *tile16(sK, t, col0 + q4 * 8);
+          qh[4 * q4] = wq.x, qh[4 * q4 + 1] = wq.y, qh[4 * q4 + 2] = wq.z, qh[4 * q4 + 3] = wq.w;
+          kh[4 * q4] = wk.x, kh[4 * q4 + 1] = wk.y, kh[4 * q4 + 2] = wk.z, kh[4 * q4 + 3] = wk.w;
+        }
         tmem_ld_wait();
         uint32_t out[16];
 #pragma unroll
-        for (int u = 0; u < 32; ++u) {
-          const float dqp = exp2f(xl[c2 * 32 + u]) * __uint_as_float(a[u]);
-          const float full = fmaf(dad, kv[u], dqp);
-          if (u & 1)
-            out[u / 2] = pack_bf16(__uint_as_float(out[u / 2]), full);
-          else
-            out[u / 2] = __float_as_uint(full);
-          a[u] = __float_as_uint(qv[u] * dqp);
+        for (int u2 = 0; u2 < 16; ++u2) {
+          const float2 qf = unpack_bf16(qh[u2]), kf = unpack_bf16(kh[u2]);
+          const float e0 = exp2f(xl[c2 * 32 + 2 * u2]), e1 = exp2f(xl[c2 * 32 + 2 * u2 + 1]);
+          const float t0 = __uint_as_float(a[2 * u2]), t1 = __uint_as_float(a[2 * u2 + 1]);
+          out[u2] = pack_bf16(e0 * fmaf(dad, kf.x, t0), e1 * fmaf(dad, kf.y, t1));
+          a[2 * u2] = __float_as_uint(qf.x * t0);
+          a[2 * u2 + 1] = __float_as_uint(qf.y * t1);
         }
         uint4* dst = reinterpret_cast<uint4*>(dq + tok + col0);
 #pragma unroll
@@ -712,8 +733,10 @@ __global__ void __launch_bounds__(kThreads, 1) gla_bwd_tc(
       for (int kk = 0; kk < kD / 16; ++kk) mma_bf16(tmem + T3, kmaj(aV, kk), kmaj(aX, kk), id_kk, kk != 0);
       mma_commit(&s->mma3);
     }
-    // ---- epilogue 3: dk, dv -> sA, sB; dB = q . dq' - k . dk' and k . dk^inter
-    // as fp32 tiles over the token buffers (all MMAs have read them)
+    // ---- epilogue 3: dk = E^-1 . (T0 + T3 + (do_s . v_s) Q^_s) -> sA, dv = T1 -> sB;
+    // dB = q . dq' - k . dk' = T2 - K^ . T0 and k . dk^inter = K^ . T3 back into
+    // T0 and T3, then (once every thread has read its Q^ and K^ rows) as fp32
+    // tiles over the token buffers for the column sums
     float* fB = reinterpret_cast<float*>(sQ);  // over sQ and sK
     float* fK = reinterpret_cast<float*>(sV);  // over sV and sD
     if (mbar_wait(&s->mma3, 0, SITE_BWD_MMA)) {
@@ -726,35 +749,33 @@ __global__ void __launch_bounds__(kThreads, 1) gla_bwd_tc(
         tmem_ld32(lane_base + T0 + col0, ka);
         tmem_ld32(lane_base + T3 + col0, kb);
         tmem_ld32(lane_base + T2 + col0, bq);
-        float qv[32], kv[32];
-        load_row32(q + tok + col0, qv);
-        load_row32(k + tok + col0, kv);
+        uint32_t qh[16], kh[16];
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4) {
+          const uint4 wq = *tile16(sQ, t, col0 + q4 * 8);
+          const uint4 wk = *tile16(sK, t, col0 + q4 * 8);
+          qh[4 * q4] = wq.x, qh[4 * q4 + 1] = wq.y, qh[4 * q4 + 2] = wq.z, qh[4 * q4 + 3] = wq.w;
+          kh[4 * q4] = wk.x, kh[4 * q4 + 1] = wk.y, kh[4 * q4 + 2] = wk.z, kh[4 * q4 + 3] = wk.w;
+        }
         tmem_ld_wait();
         uint32_t out[16];
-        float db[32], kd[32];
 #pragma unroll
-        for (int u = 0; u < 32; ++u) {
-          const float ei = exp2f(-xl[c2 * 32 + u]);
-          const float dka = ei * __uint_as_float(ka[u]);
-          const float dkb = ei * __uint_as_float(kb[u]);
-          const float full = fmaf(dad, qv[u], dka + dkb);
-          if (u & 1)
-            out[u / 2] = pack_bf16(__uint_as_float(out[u / 2]), full);
-          else
-            out[u / 2] = __float_as_uint(full);
-          db[u] = __uint_as_float(bq[u]) - kv[u] * dka;
-          kd[u] = kv[u] * dkb;
+        for (int u2 = 0; u2 < 16; ++u2) {
+          const float2 qf = unpack_bf16(qh[u2]), kf = unpack_bf16(kh[u2]);
+          const float e0 = exp2f(-xl[c2 * 32 + 2 * u2]), e1 = exp2f(-xl[c2 * 32 + 2 * u2 + 1]);
+          const float a0 = __uint_as_float(ka[2 * u2]), a1 = __uint_as_float(ka[2 * u2 + 1]);
+          const float b0 = __uint_as_float(kb[2 * u2]), b1 = __uint_as_float(kb[2 * u2 + 1]);
+          out[u2] = pack_bf16(e0 * fmaf(dad, qf.x, a0 + b0), e1 * fmaf(dad, qf.y, a1 + b1));
+          ka[2 * u2] = __float_as_uint(__uint_as_float(bq[2 * u2]) - kf.x * a0);
+          ka[2 * u2 + 1] = __float_as_uint(__uint_as_float(bq[2 * u2 + 1]) - kf.y * a1);
+          kb[2 * u2] = __float_as_uint(kf.x * b0);
+          kb[2 * u2 + 1] = __float_as_uint(kf.y * b1);
         }
 #pragma unroll
         for (int q4 = 0; q4 < 4; ++q4)
           *tile16(sA, t, col0 + q4 * 8) = make_uint4(out[4 * q4], out[4 * q4 + 1], out[4 * q4 + 2], out[4 * q4 + 3]);
-#pragma unroll
-        for (int q4 = 0; q4 < 8; ++q4) {
-          *reinterpret_cast<float4*>(fB + gate_slot(t, col0 + 4 * q4)) =
-              make_float4(db[4 * q4], db[4 * q4 + 1], db[4 * q4 + 2], db[4 * q4 + 3]);
-          *reinterpret_cast<float4*>(fK + gate_slot(t, col0 + 4 * q4)) =
-              make_float4(kd[4 * q4], kd[4 * q4 + 1], kd[4 * q4 + 2], kd[4 * q4 + 3]);
-        }
+        tmem_st32(lane_base + T0 + col0, ka);
+        tmem_st32(lane_base + T3 + col0, kb);
         uint32_t dvv[32];
         tmem_ld32(lane_base + T1 + col0, dvv);
         tmem_ld_wait();
@@ -766,9 +787,30 @@ __global__ void __launch_bounds__(kThreads, 1) gla_bwd_tc(
                          pack_bf16(__uint_as_float(dvv[q4 * 8 + 4]), __uint_as_float(dvv[q4 * 8 + 5])),
                          pack_bf16(__uint_as_float(dvv[q4 * 8 + 6]), __uint_as_float(dvv[q4 * 8 + 7])));
       }
+      tmem_st_wait();
       fence_async_smem();
     } else {
       s->abort = 1;
+    }
+    tc_fence_before();
+    __syncthreads();  // every Q^ and K^ row has been read
+    tc_fence_after();
+#pragma unroll
+    for (int c2 = 0; c2 < 2; ++c2) {
+      const int col0 = half * 64 + c2 * 32;
+      uint32_t db[32], kd[32];
+      tmem_ld32(lane_base + T0 + col0, db);
+      tmem_ld32(lane_base + T3 + col0, kd);
+      tmem_ld_wait();
+#pragma unroll
+      for (int q4 = 0; q4 < 8; ++q4) {
+        *reinterpret_cast<float4*>(fB + gate_slot(t, col0 + 4 * q4)) =
+            make_float4(__uint_as_float(db[4 * q4]), __uint_as_float(db[4 * q4 + 1]), __uint_as_float(db[4 * q4 + 2]),
+                        __uint_as_float(db[4 * q4 + 3]));
+        *reinterpret_cast<float4*>(fK + gate_slot(t, col0 + 4 * q4)) =
+            make_float4(__uint_as_float(kd[4 * q4]), __uint_as_float(kd[4 * q4 + 1]), __uint_as_float(kd[4 * q4 + 2]),
+                        __uint_as_float(kd[4 * q4 + 3]));
+      }
     }
     __syncthreads();
     // dg_t = sum_{t' >= t} dB_t' + sum_{t' < t} k . dk^inter_t' + e^{b_end} <R_c, P_c>: the
@@ -804,24 +846,28 @@ __global__ void __launch_bounds__(kThreads, 1) gla_bwd_tc(
       }
     }
     __syncthreads();
+    // dg into the dB tile (the gate map's layout), stored by TMA below
 #pragma unroll
     for (int cb = 0; cb < 2; ++cb) {
       const int col0 = half * 64 + cb * 32;
-      float4* dst = reinterpret_cast<float4*>(dg + tok + col0);
 #pragma unroll
       for (int q4 = 0; q4 < 8; ++q4) {
-        const float4 a = *reinterpret_cast<const float4*>(fB + gate_slot(t, col0 + 4 * q4));
+        float4* pa = reinterpret_cast<float4*>(fB + gate_slot(t, col0 + 4 * q4));
+        const float4 a = *pa;
         const float4 e = *reinterpret_cast<const float4*>(fK + gate_slot(t, col0 + 4 * q4));
         const float* bn = s->bnd + col0 + 4 * q4;
-        dst[q4] = make_float4(a.x + e.x + bn[0], a.y + e.y + bn[1], a.z + e.z + bn[2], a.w + e.w + bn[3]);
+        *pa = make_float4(a.x + e.x + bn[0], a.y + e.y + bn[1], a.z + e.z + bn[2], a.w + e.w + bn[3]);
       }
     }
+    fence_async_smem();
     __syncthreads();
     if (tid == 0 && !s->abort) {
       tma_store_4d(&map_dk, sA, 0, h, (int)row0, b);
       tma_store_4d(&map_dk, sA + kBox, 64, h, (int)row0, b);
       tma_store_4d(&map_dv, sB, 0, h, (int)row0, b);
       tma_store_4d(&map_dv, sB + kBox, 64, h, (int)row0, b);
+#pragma unroll
+      for (int cb = 0; cb < 4; ++cb) tma_store_4d(&map_dg, fB + cb * (kTile * 32), cb * 32, h, (int)row0, b);
       tma_store_commit();
       tma_store_wait_read0();
     }
@@ -874,18 +920,17 @@ cudaError_t tc_gla_chunk_bwd(const void* q, const void* k, const void* v, const 
                              const float* P, const float* Rs, void* dq, void* dk, void* dv, float* dg, int B, int H,
                              int64_t N, cudaStream_t st) {
   using namespace tc_gla_detail;
-  CUtensorMap mq, mk, mv, mdo, mdk, mdv, mg;
+  CUtensorMap mq, mk, mv, mdo, mdk, mdv, mg, mdg;
   if (!make_token_map(&mq, q, B, H, N, kD, kTile) || !make_token_map(&mk, k, B, H, N, kD, kTile) ||
       !make_token_map(&mv, v, B, H, N, kD, kTile) || !make_token_map(&mdo, dout, B, H, N, kD, kTile) ||
       !make_token_map(&mdk, dk, B, H, N, kD, kTile) || !make_token_map(&mdv, dv, B, H, N, kD, kTile) ||
-      !make_gate_map(&mg, g, B, H, N, kD, kTile))
+      !make_gate_map(&mg, g, B, H, N, kD, kTile) || !make_gate_map(&mdg, dg, B, H, N, kD, kTile))
     return cudaErrorInvalidValue;
   const size_t smem = 1024 + 7 * (size_t)kTileBytes + sizeof(SmemBwd);
   cudaError_t e = cudaFuncSetAttribute(gla_bwd_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   gla_bwd_tc<<<dim3((unsigned)(N / kTile), H, B), kThreads, smem, st>>>(
-      mq, mk, mv, mdo, mdk, mdv, mg, P, Rs, (const __nv_bfloat16*)q, (const __nv_bfloat16*)k, (__nv_bfloat16*)dq,
-      dg, H, N);
+      mq, mk, mv, mdo, mdk, mdv, mg, mdg, P, Rs, (__nv_bfloat16*)dq, H, N);
   return cudaGetLastError();
 }
 
