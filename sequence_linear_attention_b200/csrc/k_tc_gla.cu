@@ -380,6 +380,7 @@ __global__ void __launch_bounds__(kThreads, 1) gla_out_tc(const __grid_constant_
   const uint32_t T0 = 0, T1 = 128;
   if (tid == 0) {
     load_gate_tile(bt, &map_g, &s->gload, h, (int)row0, b);
+    bulk_prefetch_l2(P + ((b * T + c) * H + h) * (int64_t)kD * kD, kD * kD * 4);  // read with plain loads later
     mbar_arrive_expect_tx(&s->load, 3 * kTileBytes);
     tma_load_4d(sQ, &map_q, &s->load, 0, h, (int)row0, b);
     tma_load_4d(sQ + kBox, &map_q, &s->load, 64, h, (int)row0, b);
