@@ -329,7 +329,14 @@ LASP_API int lasp_bidir_bwd(const void* q, const void* k, const void* v, const v
  *   g, dg:  float [B, N, H, d] (always float32, the layout of the token
  *           tensors), the log-gates and the gradient of sum(o * dout) with
  *           respect to them.
- * Chunks: 1 <= C <= 128, C divides N (LASP_ERR_UNSUPPORTED for C > 128). In
+ * Chunks: 1 <= C <= 128, C divides N (LASP_ERR_UNSUPPORTED for C > 128).
+ * bf16 with d = 128, C dividing 128 and N a multiple of 128 runs on the tensor
+ * cores, which factor the decay inside each 128-token tile around the tile's
+ * middle token: that needs the log-gates of each 64-token half of a tile to
+ * sum to at least -80 (gates far stronger than any that leave the state
+ * anything to carry); a tile beyond that records LASP_ERR_INVALID_ARG in the
+ * device status. Every other case (fp32 in particular) runs exact CUDA-core
+ * kernels with no such limit. In
  * chunk c, b_t = sum_{r<=t} g_{cC+r} (from the chunk start) and the chunk's
  * total log-gate is gsum_c = b_{C-1}. The states of the gated form:
  *   kind 0, (x, y) = (k, v):   M_c  = sum_t diag(exp(gsum_c - b_t)) k_t^T v_t

@@ -39,7 +39,8 @@ __device__ __forceinline__ float4 fma4(float g, float4 a, float4 m) {
 
 constexpr float kLog2e = 1.4426950408889634f;
 
-// gsum (kGated only): [B, t_slots, H, d] log-gate totals, in the same slots as M
+// gsum (kGated only): [B, t_slots, H, d] log-gate totals, scan element c's at
+// slot c * slot_stride + gsum_offset
 template <bool kGated>
 __global__ void __launch_bounds__(kThreads) state_scan_kernel(const float4* M, float4* P, const float* decay,
                                                               const float* __restrict__ gsum,
@@ -47,7 +48,7 @@ __global__ void __launch_bounds__(kThreads) state_scan_kernel(const float4* M, f
                                                               float4* __restrict__ total, int H, int T,
                                                               int d, int dd4, int64_t n_threads, float Cf,
                                                               int reverse, int64_t t_slots, int slot_stride,
-                                                              int slot_offset) {
+                                                              int slot_offset, int gsum_offset) {
   const int64_t idx = (int64_t)blockIdx.x * kThreads + threadIdx.x;
   if (idx >= n_threads) return;
   const int e = (int)(idx % dd4);
@@ -66,7 +67,7 @@ __global__ void __launch_bounds__(kThreads) state_scan_kernel(const float4* M, f
   // the log-gate total of this thread's state row in scan element c
   const int64_t gstride = (int64_t)slot_stride * H * d;
   const int64_t gstep = reverse ? -gstride : gstride;
-  int64_t goff = ((b * t_slots + slot_offset) * H + h) * (int64_t)d + (4 * e) / d;
+  int64_t goff = ((b * t_slots + gsum_offset) * H + h) * (int64_t)d + (4 * e) / d;
   if (reverse) goff += (int64_t)(T - 1) * gstride;
   // software pipeline: the loads of group g + 1 are issued before group g is
   // scanned and stored, so a group's worth of loads is always in flight
@@ -127,18 +128,19 @@ cudaError_t launch_state_scan_slots(const float* M, float* P, const float* decay
   const int64_t blocks = (n_threads + scan_detail::kThreads - 1) / scan_detail::kThreads;
   scan_detail::state_scan_kernel<false><<<(unsigned)blocks, scan_detail::kThreads, 0, st>>>(
       (const float4*)M, (float4*)P, decay, nullptr, (const float4*)init, (float4*)total, H, T, d, dd4,
-      n_threads, (float)C, reverse, t_slots, slot_stride, slot_offset);
+      n_threads, (float)C, reverse, t_slots, slot_stride, slot_offset, 0);
   return cudaGetLastError();
 }
 
 cudaError_t launch_gla_scan(const float* M, float* P, const float* gsum, const float* init, float* total, int B,
-                            int T, int H, int d, int reverse, cudaStream_t st) {
+                            int T, int H, int d, int reverse, int64_t t_slots, int slot_stride, int slot_offset,
+                            int gsum_offset, cudaStream_t st) {
   const int dd4 = d * d / 4;
   const int64_t n_threads = (int64_t)B * H * dd4;
   const int64_t blocks = (n_threads + scan_detail::kThreads - 1) / scan_detail::kThreads;
   scan_detail::state_scan_kernel<true><<<(unsigned)blocks, scan_detail::kThreads, 0, st>>>(
       (const float4*)M, (float4*)P, nullptr, gsum, (const float4*)init, (float4*)total, H, T, d, dd4, n_threads,
-      1.f, reverse, T, 1, 0);
+      1.f, reverse, t_slots, slot_stride, slot_offset, gsum_offset);
   return cudaGetLastError();
 }
 

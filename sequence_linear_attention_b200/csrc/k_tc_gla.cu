@@ -193,7 +193,8 @@ struct SmemStates {
 __global__ void __launch_bounds__(kThreads, 2) gla_states_tc(const __grid_constant__ CUtensorMap map_x,
                                                              const __grid_constant__ CUtensorMap map_y,
                                                              const float* __restrict__ g, float* __restrict__ M,
-                                                             float* __restrict__ gsum, int H, int64_t N, int kind) {
+                                                             float* __restrict__ gsum, int H, int64_t N, int kind,
+                                                             int64_t t_slots, int stride, int offset) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   uint8_t* sX = base;
@@ -202,7 +203,7 @@ __global__ void __launch_bounds__(kThreads, 2) gla_states_tc(const __grid_consta
   const int c = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int64_t row0 = (int64_t)c * kTile;
-  const int64_t T = N / kTile;
+  const int64_t sl = (int64_t)b * t_slots + (int64_t)c * stride + offset;  // the state slot of this tile
   if (tid == 0) {
     prefetch_tmap(&map_x);
     prefetch_tmap(&map_y);
@@ -278,12 +279,12 @@ __global__ void __launch_bounds__(kThreads, 2) gla_states_tc(const __grid_consta
     mma_commit(&s->mma);
   }
   if (kind == 0 && gsum != nullptr && tid < kD)
-    gsum[((b * T + c) * H + h) * kD + tid] = s->half_tot[0][tid] + s->half_tot[1][tid];
+    gsum[(sl * H + h) * kD + tid] = s->half_tot[0][tid] + s->half_tot[1][tid];
   if (mbar_wait(&s->mma, 0, SITE_STATES_MMA)) {
     tc_fence_after();
     // row i of M (TMEM lane i), columns half*64..
     const int i = (warp & 3) * 32 + lane, half = warp >> 2;
-    float* out = M + (((b * T + c) * H + h) * kD + i) * kD + half * 64;
+    float* out = M + ((sl * H + h) * kD + i) * kD + half * 64;
     const uint32_t lane_base = tmem + ((uint32_t)((warp & 3) * 32) << 16);
 #pragma unroll
     for (int c2 = 0; c2 < 2; ++c2) {
@@ -340,7 +341,8 @@ __global__ void __launch_bounds__(kThreads, 1) gla_out_tc(const __grid_constant_
                                                           const __grid_constant__ CUtensorMap map_v,
                                                           const __grid_constant__ CUtensorMap map_o,
                                                           const __grid_constant__ CUtensorMap map_g,
-                                                          const float* __restrict__ P, int H, int64_t N) {
+                                                          const float* __restrict__ P, int H, int64_t N,
+                                                          int64_t t_slots, int stride) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   uint8_t* sQ = base;                   // Q^
@@ -354,7 +356,7 @@ __global__ void __launch_bounds__(kThreads, 1) gla_out_tc(const __grid_constant_
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int t = (warp & 3) * 32 + lane, half = warp >> 2;
   const int64_t row0 = (int64_t)c * kTile;
-  const int64_t T = N / kTile;
+  const float* Pc = P + (((int64_t)b * t_slots + (int64_t)c * stride) * H + h) * kD * kD;  // P of the tile's first chunk
   if (tid == 0) {
     prefetch_tmap(&map_q);
     prefetch_tmap(&map_k);
@@ -380,7 +382,7 @@ __global__ void __launch_bounds__(kThreads, 1) gla_out_tc(const __grid_constant_
   const uint32_t T0 = 0, T1 = 128;
   if (tid == 0) {
     load_gate_tile(bt, &map_g, &s->gload, h, (int)row0, b);
-    bulk_prefetch_l2(P + ((b * T + c) * H + h) * (int64_t)kD * kD, kD * kD * 4);  // read with plain loads later
+    bulk_prefetch_l2(Pc, kD * kD * 4);  // read with plain loads later
     mbar_arrive_expect_tx(&s->load, 3 * kTileBytes);
     tma_load_4d(sQ, &map_q, &s->load, 0, h, (int)row0, b);
     tma_load_4d(sQ + kBox, &map_q, &s->load, 64, h, (int)row0, b);
@@ -396,7 +398,7 @@ __global__ void __launch_bounds__(kThreads, 1) gla_out_tc(const __grid_constant_
     float w[16];
 #pragma unroll
     for (int u = 0; u < 16; ++u) w[u] = exp2f(s->r[warp + 8 * u] * kLog2e);
-    load_scaled_state(sX, P + ((b * T + c) * H + h) * (int64_t)kD * kD, w, warp, lane);
+    load_scaled_state(sX, Pc, w, warp, lane);
   }
   if (!mbar_wait(&s->load, 0, SITE_OUT_TMA)) s->abort = 1;
   scale_row_half(sQ, t, half, x, 1.f);   // Q^ = q . E
@@ -502,7 +504,8 @@ __global__ void __launch_bounds__(kThreads, 1) gla_bwd_tc(
     const __grid_constant__ CUtensorMap map_v, const __grid_constant__ CUtensorMap map_do,
     const __grid_constant__ CUtensorMap map_dk, const __grid_constant__ CUtensorMap map_dv,
     const __grid_constant__ CUtensorMap map_g, const __grid_constant__ CUtensorMap map_dg,
-    const float* __restrict__ P, const float* __restrict__ R, __nv_bfloat16* __restrict__ dq, int H, int64_t N) {
+    const float* __restrict__ P, const float* __restrict__ R, __nv_bfloat16* __restrict__ dq, int H, int64_t N,
+    int64_t t_slots, int stride) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   uint8_t* sQ = base;
@@ -520,8 +523,9 @@ __global__ void __launch_bounds__(kThreads, 1) gla_bwd_tc(
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int t = (warp & 3) * 32 + lane, half = warp >> 2;
   const int64_t row0 = (int64_t)c * kTile;
-  const int64_t T = N / kTile;
-  const int64_t slot = ((int64_t)b * T + c) * H + h;
+  // P of the tile's first chunk and R of its last
+  const int64_t pslot = ((int64_t)b * t_slots + (int64_t)c * stride) * H + h;
+  const int64_t rslot = pslot + (int64_t)(stride - 1) * H;
   const int64_t tok = (((int64_t)b * N + row0 + t) * H + h) * kD;  // row t of every token tensor
   if (tid == 0) {
     prefetch_tmap(&map_q);
@@ -551,8 +555,8 @@ __global__ void __launch_bounds__(kThreads, 1) gla_bwd_tc(
   if (tid == 0) {
     load_gate_tile(bt, &map_g, &s->gload, h, (int)row0, b);
     // P and R are read with plain loads later: into L2 now
-    bulk_prefetch_l2(P + slot * kD * kD, kD * kD * 4);
-    bulk_prefetch_l2(R + slot * kD * kD, kD * kD * 4);
+    bulk_prefetch_l2(P + pslot * kD * kD, kD * kD * 4);
+    bulk_prefetch_l2(R + rslot * kD * kD, kD * kD * 4);
     mbar_arrive_expect_tx(&s->load, 4 * kTileBytes);
     tma_load_4d(sQ, &map_q, &s->load, 0, h, (int)row0, b);
     tma_load_4d(sQ + kBox, &map_q, &s->load, 64, h, (int)row0, b);
@@ -574,7 +578,7 @@ __global__ void __launch_bounds__(kThreads, 1) gla_bwd_tc(
     we[u] = exp2f((sbend[m] - sr[m]) * kLog2e);
   }
   named_sync(kBarAll, kThreads);  // r and b_end are read before X is written
-  load_scaled_state(sX, P + slot * kD * kD, wr, warp, lane);
+  load_scaled_state(sX, P + pslot * kD * kD, wr, warp, lane);
   if (!mbar_wait(&s->load, 0, SITE_BWD_TMA)) s->abort = 1;
   scale_row_half(sQ, t, half, x, 1.f);   // Q^ = q . E
   scale_row_half(sK, t, half, x, -1.f);  // K^ = k / E
@@ -609,7 +613,7 @@ __global__ void __launch_bounds__(kThreads, 1) gla_bwd_tc(
       mma_commit(&s->mma1b);
     }
     // R rows (fp32) into registers while the MMAs run
-    const float4* R4 = reinterpret_cast<const float4*>(R + slot * kD * kD);
+    const float4* R4 = reinterpret_cast<const float4*>(R + rslot * kD * kD);
     float4 rreg[16];
 #pragma unroll
     for (int u = 0; u < 16; ++u) rreg[u] = __ldcs(R4 + (warp + 8 * u) * (kD / 4) + lane);
@@ -647,7 +651,7 @@ __global__ void __launch_bounds__(kThreads, 1) gla_bwd_tc(
     // X is free once dO P'^T has read P': R' = diag(e^{b_end - r}) R_c replaces it,
     // and <R'_m, P'_m> (fp32) = e^{b_end_m} <R_m, P_m> goes to bnd
     if (mbar_wait(&s->mma1b, 0, SITE_BWD_MMA)) {
-      const float4* P4 = reinterpret_cast<const float4*>(P + slot * kD * kD);
+      const float4* P4 = reinterpret_cast<const float4*>(P + pslot * kD * kD);
 #pragma unroll
       for (int u = 0; u < 16; ++u) {
         const int m = warp + 8 * u;
@@ -881,12 +885,15 @@ cleanup:
 
 }  // namespace tc_gla_detail
 
-bool tc_gla_ok(int dtype, int d, int64_t C) {
-  return dtype == LASP_BF16 && d == tc_gla_detail::kD && C == tc_gla_detail::kTile;
+bool tc_gla_ok(int dtype, int d, int64_t C, int64_t N) {
+  // chunks that divide the 128-token tile: a tile's sums regroup the per-chunk
+  // intra and inter terms, so states are needed only at tile boundaries
+  using tc_gla_detail::kTile;
+  return dtype == LASP_BF16 && d == tc_gla_detail::kD && C >= 1 && C <= kTile && kTile % C == 0 && N % kTile == 0;
 }
 
 cudaError_t tc_gla_chunk_states(const void* x, const void* y, const float* g, float* M, float* gsum, int B, int H,
-                                int64_t N, int kind, cudaStream_t st) {
+                                int64_t N, int kind, int64_t t_slots, int stride, int offset, cudaStream_t st) {
   using namespace tc_gla_detail;
   CUtensorMap mx, my;
   if (!make_token_map(&mx, x, B, H, N, kD, kTile) || !make_token_map(&my, y, B, H, N, kD, kTile))
@@ -894,12 +901,13 @@ cudaError_t tc_gla_chunk_states(const void* x, const void* y, const float* g, fl
   const size_t smem = 1024 + 2 * (size_t)kTileBytes + sizeof(SmemStates);
   cudaError_t e = cudaFuncSetAttribute(gla_states_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  gla_states_tc<<<dim3((unsigned)(N / kTile), H, B), kThreads, smem, st>>>(mx, my, g, M, gsum, H, N, kind);
+  gla_states_tc<<<dim3((unsigned)(N / kTile), H, B), kThreads, smem, st>>>(mx, my, g, M, gsum, H, N, kind, t_slots,
+                                                                          stride, offset);
   return cudaGetLastError();
 }
 
 cudaError_t tc_gla_chunk_out(const void* q, const void* k, const void* v, const float* g, const float* P, void* o,
-                             int B, int H, int64_t N, cudaStream_t st) {
+                             int B, int H, int64_t N, int64_t t_slots, int stride, cudaStream_t st) {
   using namespace tc_gla_detail;
   CUtensorMap mq, mk, mv, mo, mg;
   if (!make_token_map(&mq, q, B, H, N, kD, kTile) || !make_token_map(&mk, k, B, H, N, kD, kTile) ||
@@ -909,7 +917,8 @@ cudaError_t tc_gla_chunk_out(const void* q, const void* k, const void* v, const 
   const size_t smem = 1024 + 7 * (size_t)kTileBytes + sizeof(SmemOut);
   cudaError_t e = cudaFuncSetAttribute(gla_out_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  gla_out_tc<<<dim3((unsigned)(N / kTile), H, B), kThreads, smem, st>>>(mq, mk, mv, mo, mg, P, H, N);
+  gla_out_tc<<<dim3((unsigned)(N / kTile), H, B), kThreads, smem, st>>>(mq, mk, mv, mo, mg, P, H, N, t_slots,
+                                                                       stride);
   return cudaGetLastError();
 }
 
@@ -919,7 +928,7 @@ namespace lasp {
 
 cudaError_t tc_gla_chunk_bwd(const void* q, const void* k, const void* v, const void* dout, const float* g,
                              const float* P, const float* Rs, void* dq, void* dk, void* dv, float* dg, int B, int H,
-                             int64_t N, cudaStream_t st) {
+                             int64_t N, int64_t t_slots, int stride, cudaStream_t st) {
   using namespace tc_gla_detail;
   CUtensorMap mq, mk, mv, mdo, mdk, mdv, mg, mdg;
   if (!make_token_map(&mq, q, B, H, N, kD, kTile) || !make_token_map(&mk, k, B, H, N, kD, kTile) ||
@@ -931,7 +940,7 @@ cudaError_t tc_gla_chunk_bwd(const void* q, const void* k, const void* v, const 
   cudaError_t e = cudaFuncSetAttribute(gla_bwd_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   gla_bwd_tc<<<dim3((unsigned)(N / kTile), H, B), kThreads, smem, st>>>(
-      mq, mk, mv, mdo, mdk, mdv, mg, mdg, P, Rs, (__nv_bfloat16*)dq, H, N);
+      mq, mk, mv, mdo, mdk, mdv, mg, mdg, P, Rs, (__nv_bfloat16*)dq, H, N, t_slots, stride);
   return cudaGetLastError();
 }
 

@@ -33,8 +33,12 @@ cudaError_t simt_chunk_bwd(const void* q, const void* k, const void* v, const vo
 // gsum if non-null); kind 1: dM_c = sum_t diag(e^{b_t}) q_t^T do_t.
 cudaError_t gla_simt_chunk_states(const void* x, const void* y, const float* g, float* M, float* gsum, int B, int H,
                                   int64_t N, int d, int C, int kind, int dtype, cudaStream_t st);
+// The gated scan over T elements held in every slot_stride-th slot (from
+// slot_offset) of an array of t_slots states; element c's log-gate totals in
+// slot c * slot_stride + gsum_offset of gsum.
 cudaError_t launch_gla_scan(const float* M, float* P, const float* gsum, const float* init, float* total, int B,
-                            int T, int H, int d, int reverse, cudaStream_t st);
+                            int T, int H, int d, int reverse, int64_t t_slots, int slot_stride, int slot_offset,
+                            int gsum_offset, cudaStream_t st);
 cudaError_t gla_simt_chunk_out(const void* q, const void* k, const void* v, const float* g, const float* P, void* o,
                                int B, int H, int64_t N, int d, int C, int dtype, cudaStream_t st);
 cudaError_t gla_simt_chunk_bwd(const void* q, const void* k, const void* v, const void* dout, const float* g,

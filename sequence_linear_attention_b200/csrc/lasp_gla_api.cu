@@ -2,9 +2,12 @@
 // and key feature, LASP Appendix A.4, Eq. 24 with the GLA / GateLoop row of
 // Table 5. Host-side validation and dispatch; nothing here allocates.
 //
-// The state cache of lasp_gla_fwd holds, for B x T x H chunk slots, the
-// fp32 entering state P_c (d x d) of every chunk, followed by the chunk
-// log-gate totals gsum_c (d floats per slot): B*T*H*d*(d+1) floats.
+// The state cache of lasp_gla_fwd holds B x T x H chunk slots of fp32 d x d
+// states, followed by B x T x H slots of d log-gate totals: B*T*H*d*(d+1)
+// floats. The CUDA-core path fills every chunk's slot (P_c, gsum_c); the
+// tensor-core path works on 128-token tiles and fills the slots of each tile's
+// first chunk only (P and gsum of the tile), and its gradient states go to
+// the slot of each tile's last chunk of the workspace.
 #include "kernels.h"
 #include "lasp_common.cuh"
 #include "tc_kernels.h"
@@ -23,19 +26,22 @@ int check_gla_sizes(int B, int H, int64_t N, int d, int C, int dtype) {
 
 int states_impl(const void* x, const void* y, const float* g, float* M, float* gsum, int B, int H, int64_t N, int d,
                 int C, int dtype, int kind, cudaStream_t st) {
-  if (tc_gla_ok(dtype, d, C))
+  if (C == 128 && tc_gla_ok(dtype, d, C, N))
     return cuda_status(traced(K_GLA_STATES_TC, st, [&] {
-      return tc_gla_chunk_states(x, y, g, M, gsum, B, H, N, kind, st);
+      return tc_gla_chunk_states(x, y, g, M, gsum, B, H, N, kind, N / C, 1, 0, st);
     }));
   return cuda_status(traced(K_GLA_STATES, st, [&] {
     return gla_simt_chunk_states(x, y, g, M, gsum, B, H, N, d, C, kind, dtype, st);
   }));
 }
 
+// T scan elements in every stride-th slot (from offset) of t_slots slots; the
+// log-gate totals of element c in slot c * stride + goffset
 int scan_impl(const float* M, float* P, const float* gsum, const float* init, float* total, int B, int T, int H,
-              int d, int reverse, cudaStream_t st) {
-  return cuda_status(
-      traced(K_GLA_SCAN, st, [&] { return launch_gla_scan(M, P, gsum, init, total, B, T, H, d, reverse, st); }));
+              int d, int reverse, int64_t t_slots, int stride, int offset, int goffset, cudaStream_t st) {
+  return cuda_status(traced(K_GLA_SCAN, st, [&] {
+    return launch_gla_scan(M, P, gsum, init, total, B, T, H, d, reverse, t_slots, stride, offset, goffset, st);
+  }));
 }
 
 }  // namespace gla_api_detail
@@ -73,7 +79,7 @@ int lasp_gla_state_prefix(const float* M, float* Mprefix, const float* gsum, con
     if ((s = check_ptrs({}, {init, total}))) return s;
     if (total == nullptr) return LASP_OK;
   }
-  return scan_impl(M, Mprefix, gsum, init, total, B, T, H, d, reverse, (cudaStream_t)stream);
+  return scan_impl(M, Mprefix, gsum, init, total, B, T, H, d, reverse, T, 1, 0, 0, (cudaStream_t)stream);
 }
 
 int lasp_gla_fwd(const void* q, const void* k, const void* v, const float* g, void* o, int B, int H, int64_t N, int d,
@@ -85,12 +91,24 @@ int lasp_gla_fwd(const void* q, const void* k, const void* v, const float* g, vo
   cudaStream_t st = (cudaStream_t)stream;
   const int T = (int)(N / C);
   float* gsum = state_cache + (int64_t)B * T * H * d * d;
+  if (tc_gla_ok(dtype, d, C, N)) {
+    // 128-token tiles: their states and log-gate totals into the slots of each
+    // tile's first chunk, the prefix over tiles in place, then the output
+    const int stride = 128 / C;
+    const int tiles = (int)(N / 128);
+    if ((s = cuda_status(traced(K_GLA_STATES_TC, st, [&] {
+           return tc_gla_chunk_states(k, v, g, state_cache, gsum, B, H, N, 0, T, stride, 0, st);
+         }))))
+      return s;
+    if ((s = scan_impl(state_cache, state_cache, gsum, init_state, nullptr, B, tiles, H, d, 0, T, stride, 0, 0, st)))
+      return s;
+    return cuda_status(traced(K_GLA_OUT_TC, st, [&] {
+      return tc_gla_chunk_out(q, k, v, g, state_cache, o, B, H, N, T, stride, st);
+    }));
+  }
   // 1. chunk states M_c and log-gate totals; 2. exclusive prefix in place -> P_c; 3. output
   if ((s = states_impl(k, v, g, state_cache, gsum, B, H, N, d, C, dtype, 0, st))) return s;
-  if ((s = scan_impl(state_cache, state_cache, gsum, init_state, nullptr, B, T, H, d, 0, st))) return s;
-  if (tc_gla_ok(dtype, d, C))
-    return cuda_status(
-        traced(K_GLA_OUT_TC, st, [&] { return tc_gla_chunk_out(q, k, v, g, state_cache, o, B, H, N, st); }));
+  if ((s = scan_impl(state_cache, state_cache, gsum, init_state, nullptr, B, T, H, d, 0, T, 1, 0, 0, st))) return s;
   return cuda_status(traced(K_GLA_OUT, st, [&] {
     return gla_simt_chunk_out(q, k, v, g, state_cache, o, B, H, N, d, C, dtype, st);
   }));
@@ -107,14 +125,27 @@ int lasp_gla_bwd(const void* q, const void* k, const void* v, const float* g, co
   cudaStream_t st = (cudaStream_t)stream;
   const int T = (int)(N / C);
   const float* gsum = state_cache + (int64_t)B * T * H * d * d;
+  if (tc_gla_ok(dtype, d, C, N)) {
+    // 128-token tiles: gradient states into the slots of each tile's last
+    // chunk, the suffix over tiles in place (the tiles' log-gate totals sit in
+    // the cache slots of their first chunks), then the gradients
+    const int stride = 128 / C;
+    const int tiles = (int)(N / 128);
+    if ((s = cuda_status(traced(K_GLA_STATES_TC, st, [&] {
+           return tc_gla_chunk_states(q, dout, g, dstate_ws, nullptr, B, H, N, 1, T, stride, stride - 1, st);
+         }))))
+      return s;
+    if ((s = scan_impl(dstate_ws, dstate_ws, gsum, dstate_in, dinit_state, B, tiles, H, d, 1, T, stride, stride - 1, 0,
+                       st)))
+      return s;
+    return cuda_status(traced(K_GLA_BWD_TC, st, [&] {
+      return tc_gla_chunk_bwd(q, k, v, dout, g, state_cache, dstate_ws, dq, dk, dv, dg, B, H, N, T, stride, st);
+    }));
+  }
   // 1. gradient chunk states dM_c; 2. exclusive suffix in place -> R_c (and
   // dinit); 3. dQ, dK, dV and the log-gate gradient
   if ((s = states_impl(q, dout, g, dstate_ws, nullptr, B, H, N, d, C, dtype, 1, st))) return s;
-  if ((s = scan_impl(dstate_ws, dstate_ws, gsum, dstate_in, dinit_state, B, T, H, d, 1, st))) return s;
-  if (tc_gla_ok(dtype, d, C))
-    return cuda_status(traced(K_GLA_BWD_TC, st, [&] {
-      return tc_gla_chunk_bwd(q, k, v, dout, g, state_cache, dstate_ws, dq, dk, dv, dg, B, H, N, st);
-    }));
+  if ((s = scan_impl(dstate_ws, dstate_ws, gsum, dstate_in, dinit_state, B, T, H, d, 1, T, 1, 0, 0, st))) return s;
   return cuda_status(traced(K_GLA_BWD, st, [&] {
     return gla_simt_chunk_bwd(q, k, v, dout, g, state_cache, dstate_ws, dq, dk, dv, dg, B, H, N, d, C, dtype, st);
   }));

@@ -60,16 +60,19 @@ cudaError_t bidir_total(const float* seg, float* total, void* tiles, int B, int 
 cudaError_t tc_bidir_apply(const void* x, const void* stiles, void* y, int B, int H, int64_t N, int d, int b_kmajor,
                            int num_sms, cudaStream_t st);
 
-// Gated form on the tensor cores, bf16, d = 128, C = 128 (k_tc_gla.cu): the
-// chunk states of k_gla_simt.cu (kind 0 from (k, v) with the log-gate totals,
-// kind 1 from (q, do)), the output given P, and the gradients given P and R.
-bool tc_gla_ok(int dtype, int d, int64_t C);
+// Gated form on the tensor cores, bf16, d = 128, C dividing 128, N a multiple
+// of 128 (k_tc_gla.cu), on 128-token tiles: the states of k_gla_simt.cu per
+// tile (kind 0 from (k, v) with the log-gate totals, kind 1 from (q, do)) into
+// slot tile * stride + offset of an array of t_slots chunk states; the output
+// given P in the slot of each tile's first chunk; the gradients given that P
+// and R in the slot of the tile's last chunk (stride = chunks per tile).
+bool tc_gla_ok(int dtype, int d, int64_t C, int64_t N);
 cudaError_t tc_gla_chunk_states(const void* x, const void* y, const float* g, float* M, float* gsum, int B, int H,
-                                int64_t N, int kind, cudaStream_t st);
+                                int64_t N, int kind, int64_t t_slots, int stride, int offset, cudaStream_t st);
 cudaError_t tc_gla_chunk_out(const void* q, const void* k, const void* v, const float* g, const float* P, void* o,
-                             int B, int H, int64_t N, cudaStream_t st);
+                             int B, int H, int64_t N, int64_t t_slots, int stride, cudaStream_t st);
 cudaError_t tc_gla_chunk_bwd(const void* q, const void* k, const void* v, const void* dout, const float* g,
                              const float* P, const float* Rs, void* dq, void* dk, void* dv, float* dg, int B, int H,
-                             int64_t N, cudaStream_t st);
+                             int64_t N, int64_t t_slots, int stride, cudaStream_t st);
 
 }  // namespace lasp

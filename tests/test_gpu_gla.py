@@ -225,10 +225,11 @@ def _rows_states(bf16, C, d):
 
 
 def test_tensor_core_path_reports_gates_out_of_range():
-    """Log-gates of -2 per token make each 64-token half of a 128-token chunk
+    """Log-gates of -2 per token make each 64-token half of a 128-token tile
     span e^-128, more than the factorized form takes: the call records
     LASP_ERR_INVALID_ARG at the gate-range site instead of returning wrong
-    numbers silently (the CUDA-core path, C < 128, takes such gates)."""
+    numbers silently (the CUDA-core kernels, which fp32 inputs take, accept
+    such gates)."""
     import torch
     import sequence_linear_attention_b200 as lasp
     B, N, H, d, C = 1, 256, 1, 128, 128
@@ -240,9 +241,26 @@ def test_tensor_core_path_reports_gates_out_of_range():
     lasp.lasp_gla_fwd(q, k, v, gd, o, C, cache)
     status, site = lasp.lasp_check_device_status()
     assert (status, site) == (1, 40)
-    # the same gates through the CUDA-core kernels (C = 64) are fine
-    cache64 = torch.empty(lasp.lasp_gla_cache_floats(B, H, N, d, 64), dtype=torch.float32, device="cuda")
-    lasp.lasp_gla_fwd(q, k, v, gd, o, 64, cache64)
+    # the same (bf16-valued) inputs as fp32 through the CUDA-core kernels are fine
+    q32, k32, v32 = (to_device(host_f32(inp, n), False) for n in ("q", "k", "v"))
+    o32 = torch.empty_like(q32)
+    lasp.lasp_gla_fwd(q32, k32, v32, gd, o32, C, cache)
     assert lasp.lasp_check_device_status() == (0, 0)
     ref = oracle.gla_fwd(*(host_f32(inp, n) for n in ("q", "k", "v")), gd.cpu().numpy())
-    assert rel_err(to_host(o), ref) <= TOL_BF16
+    assert rel_err(to_host(o32), ref) <= TOL_F32
+
+
+@pytest.mark.parametrize("C", [16, 32, 64])
+def test_tensor_core_path_chunks_dividing_the_tile(C):
+    """C < 128 on the tensor cores: 128-token tiles span 128/C chunks, with the
+    states at tile boundaries only (in the slots of the tiles' first and last
+    chunks); against the oracle with entering states and dstate_in."""
+    B, N, H, d = 1, 768, 2, 128
+    inp = lasp_inputs.make_inputs(B, N, H, d, seed=2030 + C, bf16=True, decayed=False)
+    g = lasp_inputs.make_log_gates(B, N, H, d, seed=2030 + C, tau=4.0)
+    rng = np.random.default_rng(C)
+    init = (rng.standard_normal((B, H, d, d)) * 0.1).astype(np.float32)
+    dsin = (rng.standard_normal((B, H, d, d)) * 0.1).astype(np.float32)
+    got = _run(inp, g, C, init=init, dstate_in=dsin)
+    ref = _reference(inp, g, init=init.astype(np.float64), dstate_in=dsin.astype(np.float64))
+    _compare(got, ref, TOL_BF16)
