@@ -180,16 +180,16 @@ struct SmemStates {
   uint64_t load, mma;
   uint32_t tmem_base;
   int abort;
-  float half_tot[2][kD];  // the log-gates of each feature summed over each half of the chunk
+  alignas(16) float grp[8][kD];  // the log-gates of each feature summed over each 16-row group (float4 access)
 };
 
 // kind 0: M_c = (k . e^{b_end - b})^T v and gsum_c = b_end; kind 1: dM_c =
 // (q . e^{b})^T do. x, y: the two token operands ((k, v) or (q, do)); the gate
-// factor goes on x, scaled in place. Thread i of warps 0-3 and thread i of
-// warps 4-7 take feature i in the first and in the second half of the rows:
-// each sums its half's log-gates, then walks it again (down for kind 1, up
-// for kind 0: e^{b_end - b_t} = e^{sum_{r>t} g_r}) starting from the other
-// half's total where that half comes first.
+// factor goes on x, scaled in place. Warp w takes rows 16w..16w+15, lane l
+// features 4l..4l+3 (one 512-byte float4 row per warp-wide load): it sums its
+// group's log-gates, the eight groups' sums give each group's offset, and a
+// second pass over the loaded values (down for kind 1, up for kind 0:
+// e^{b_end - b_t} = e^{sum_{r>t} g_r}) scales the tile.
 __global__ void __launch_bounds__(kThreads, 2) gla_states_tc(const __grid_constant__ CUtensorMap map_x,
                                                              const __grid_constant__ CUtensorMap map_y,
                                                              const float* __restrict__ g, float* __restrict__ M,
@@ -228,42 +228,60 @@ __global__ void __launch_bounds__(kThreads, 2) gla_states_tc(const __grid_consta
     tma_load_4d(sY + kBox, &map_y, &s->load, 64, h, (int)row0, b);
   }
   {
-    constexpr int kHalf = kTile / 2;
-    const int i = tid & (kD - 1), hf = tid >> 7;
+    const int f0 = lane * 4;  // features f0..f0+3
     const int64_t rs = (int64_t)H * kD;
-    const float* gcol = g + ((int64_t)b * N + row0 + hf * kHalf) * rs + (int64_t)h * kD + i;
-    float tot = 0.f;
-#pragma unroll 1
-    for (int t0 = 0; t0 < kHalf; t0 += 16) {
-      float v[16];
+    const float4* gp = reinterpret_cast<const float4*>(g + ((int64_t)b * N + row0 + warp * 16) * rs +
+                                                       (int64_t)h * kD + f0);
+    float4 gv[16];
 #pragma unroll
-      for (int u = 0; u < 16; ++u) v[u] = __ldg(gcol + (int64_t)(t0 + u) * rs);
+    for (int u = 0; u < 16; ++u) gv[u] = __ldg(gp + (int64_t)u * (rs / 4));
+    float4 tot = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-      for (int u = 0; u < 16; ++u) tot += v[u];
+    for (int u = 0; u < 16; ++u) {
+      tot.x += gv[u].x;
+      tot.y += gv[u].y;
+      tot.z += gv[u].z;
+      tot.w += gv[u].w;
     }
-    s->half_tot[hf][i] = tot;
+    *reinterpret_cast<float4*>(&s->grp[warp][f0]) = tot;
     const bool ok = mbar_wait(&s->load, 0, SITE_STATES_TMA);
     if (!ok) s->abort = 1;
     __syncthreads();
-    // the part of the exponent from the other half: kind 1 sums down from row 0,
-    // kind 0 up from the last row
-    float acc = kind == 0 ? (hf == 0 ? s->half_tot[1][i] : 0.f) : (hf == 1 ? s->half_tot[0][i] : 0.f);
-    __nv_bfloat16* col = reinterpret_cast<__nv_bfloat16*>(sX + (i >> 6) * kBox + (i & 7) * 2);
-#pragma unroll 1
-    for (int t0 = 0; t0 < kHalf; t0 += 16) {
-      float v[16];
-#pragma unroll
-      for (int u = 0; u < 16; ++u) {
-        const int tl = kind == 0 ? kHalf - 1 - (t0 + u) : t0 + u;
-        v[u] = __ldg(gcol + (int64_t)tl * rs);
+    // the part of the exponent from the other groups: kind 1 sums down from
+    // row 0, kind 0 up from the last row
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int w2 = 0; w2 < 8; ++w2) {
+      if (kind == 0 ? w2 > warp : w2 < warp) {
+        const float4 x = *reinterpret_cast<const float4*>(&s->grp[w2][f0]);
+        acc.x += x.x;
+        acc.y += x.y;
+        acc.z += x.z;
+        acc.w += x.w;
       }
+    }
+    uint8_t* colp = sX + (f0 >> 6) * kBox + (f0 & 7) * 2;
 #pragma unroll
-      for (int u = 0; u < 16; ++u) {
-        const int t = hf * kHalf + (kind == 0 ? kHalf - 1 - (t0 + u) : t0 + u);
-        if (kind != 0) acc += v[u];
-        __nv_bfloat16* e = col + sw128_offset(t, (i & 63) >> 3) / 2;
-        if (ok) *e = __float2bfloat16_rn(__bfloat162float(*e) * exp2f(acc * kLog2e));
-        if (kind == 0) acc += v[u];
+    for (int n = 0; n < 16; ++n) {
+      const int u = kind == 0 ? 15 - n : n;
+      if (kind != 0) {
+        acc.x += gv[u].x;
+        acc.y += gv[u].y;
+        acc.z += gv[u].z;
+        acc.w += gv[u].w;
+      }
+      uint2* e = reinterpret_cast<uint2*>(colp + sw128_offset(warp * 16 + u, (f0 & 63) >> 3));
+      if (ok) {
+        uint2 w = *e;
+        const float2 a = unpack_bf16(w.x), c2 = unpack_bf16(w.y);
+        w.x = pack_bf16(a.x * exp2f(acc.x * kLog2e), a.y * exp2f(acc.y * kLog2e));
+        w.y = pack_bf16(c2.x * exp2f(acc.z * kLog2e), c2.y * exp2f(acc.w * kLog2e));
+        *e = w;
+      }
+      if (kind == 0) {
+        acc.x += gv[u].x;
+        acc.y += gv[u].y;
+        acc.z += gv[u].z;
+        acc.w += gv[u].w;
       }
     }
   }
@@ -278,8 +296,11 @@ __global__ void __launch_bounds__(kThreads, 2) gla_states_tc(const __grid_consta
     for (int kk = 0; kk < kTile / 16; ++kk) mma_bf16(tmem, mnmaj(aX, kk), mnmaj(aY, kk), id_nn, kk != 0);
     mma_commit(&s->mma);
   }
-  if (kind == 0 && gsum != nullptr && tid < kD)
-    gsum[(sl * H + h) * kD + tid] = s->half_tot[0][tid] + s->half_tot[1][tid];
+  if (kind == 0 && gsum != nullptr && tid < kD) {
+    float a = 0.f;
+    for (int w2 = 0; w2 < 8; ++w2) a += s->grp[w2][tid];
+    gsum[(sl * H + h) * kD + tid] = a;
+  }
   if (mbar_wait(&s->mma, 0, SITE_STATES_MMA)) {
     tc_fence_after();
     // row i of M (TMEM lane i), columns half*64..
