@@ -1,10 +1,12 @@
 // Tensor-core kernels of the gated form (a decay per token and key feature;
 // LASP Appendix A.4, Eq. 24 with the GLA / GateLoop row of Table 5), bf16,
-// d = 128, one 128-token chunk per CTA. The chunk equations are those of
-// k_gla_simt.cu (b_t = inclusive cumulative log-gate from the chunk start,
-// b_end its last row).
+// d = 128, one 128-token tile per CTA. A tile spans 128/C chunks (C dividing
+// 128); its masked products regroup the per-chunk intra and inter terms, so it
+// follows the chunk equations of k_gla_simt.cu with the tile as the chunk
+// (b_t = inclusive cumulative log-gate from the tile start, b_end its last
+// row), the states being needed at tile boundaries only.
 //
-// The intra-chunk products need the factor e^{b_t[i] - b_s[i]} inside a
+// The intra-tile products need the factor e^{b_t[i] - b_s[i]} inside a
 // contraction over i, which a single MMA can carry only if it splits into a
 // row factor and a column factor. With r = b_{63}, the middle row, as the
 // reference of each feature:
@@ -19,16 +21,16 @@
 // fp32 so that the log-gate gradient can leave it out, see k_gla_simt.cu.)
 // Every factor of Q^ and K^ is at most e^{|b_t - r|}; the form is exact as
 // long as that stays inside the bf16 / fp32 range, i.e. the log-gates of each
-// half of the chunk sum to at least -kMaxSpan. Each CTA checks this for its
-// chunk and records LASP_ERR_INVALID_ARG (site SITE_GATE_RANGE) if not; the
+// half of the tile sum to at least -kMaxSpan. Each CTA checks this for its
+// tile and records LASP_ERR_INVALID_ARG (site SITE_GATE_RANGE) if not; the
 // CUDA-core kernels have no such limit.
 //
 // Thread layout (256 threads): warp w owns tile rows / TMEM lanes 32*(w%4)..
-// and the column half w/4 of every row-wise step. The cumulative log-gates
-// come from a walk down the chunk's rows by warps 0-3, one feature per lane
-// (loads running 32 rows ahead): the state kernel scales its operand as it
-// walks; the others write the sums into an fp32 tile in shared memory that
-// the row-wise steps then read.
+// and the column half w/4 of every row-wise step. The cumulative log-gates:
+// the state kernel sums them by 16-row groups (a warp per group, float4 loads)
+// and scales its operand in place; the output and backward kernels load the
+// gate tile by TMA and walk it in shared memory, one feature per thread of
+// warps 0-3, before the row-wise steps read it.
 #include "kernels.h"
 #include "lasp_common.cuh"
 #include "sm100.cuh"
@@ -81,32 +83,6 @@ __device__ __forceinline__ void scale_row_half(uint8_t* tile, int row, int half,
   }
 }
 
-// The chunk's log-gates g_t[i] for the feature i of this lane (warp w < 4
-// owns features 32w..32w+31), rows in walking order (down, or up if `up`),
-// handed to `step(t, g)`; the loads run one kBlk-row block ahead.
-template <int kBlk = 32, class F>
-__device__ __forceinline__ void walk_gates(const float* __restrict__ g_chunk, int64_t row_stride, int i, bool up,
-                                           F&& step) {
-  const float* gp = g_chunk + i;
-  auto row = [&](int n) { return up ? kTile - 1 - n : n; };
-  float cur[kBlk], nxt[kBlk];
-#pragma unroll
-  for (int u = 0; u < kBlk; ++u) cur[u] = __ldcs(gp + (int64_t)row(u) * row_stride);
-#pragma unroll
-  for (int blk = 0; blk < kTile / kBlk; ++blk) {
-    if (blk + 1 < kTile / kBlk) {
-#pragma unroll
-      for (int u = 0; u < kBlk; ++u) nxt[u] = __ldcs(gp + (int64_t)row((blk + 1) * kBlk + u) * row_stride);
-    }
-#pragma unroll
-    for (int u = 0; u < kBlk; ++u) step(row(blk * kBlk + u), cur[u]);
-    if (blk + 1 < kTile / kBlk) {
-#pragma unroll
-      for (int u = 0; u < kBlk; ++u) cur[u] = nxt[u];
-    }
-  }
-}
-
 // Element (t, i) of a [128][128] fp32 tile as the gate map's TMA loads lay it
 // out: four 32-feature blocks of 128 lines of 128 bytes, 16-byte chunk c of
 // line t at chunk c ^ (t % 8). A warp walking 32 features of one line and a
@@ -150,7 +126,7 @@ __device__ __forceinline__ void read_gate_row(const float* bt, int t, int half, 
     }
 }
 
-// Four TMA loads of the chunk's log-gates (fp32, 64 KB) into the tile.
+// Four TMA loads of the tile's log-gates (fp32, 64 KB) into the gate tile.
 __device__ __forceinline__ void load_gate_tile(float* bt, const CUtensorMap* map_g, uint64_t* bar, int h, int row0,
                                                int b) {
   mbar_arrive_expect_tx(bar, kTile * kD * 4);
@@ -513,7 +489,7 @@ struct SmemBwd {
   float bnd[kD];     // e^{b_end[i]} <R_c[i], P_c[i]>
 };
 
-// One 128-token chunk per CTA. Shared memory: Q^, K^, V, dO (then, in pairs,
+// One 128-token tile per CTA. Shared memory: Q^, K^, V, dO (then, in pairs,
 // the fp32 tiles of dB and k . dk^inter for the log-gate gradient's column
 // sums), X (P', then R'; r and b_end during the gate walk), and the pair
 // sA / sB (the gate tile during the walk; then dA . strict and A . causal;
