@@ -577,6 +577,41 @@ def cpu_baseline(args):
             "sample": f"fp64 oracle fwd+bwd, batch 0, all heads, first {tokens} positions"}
 
 
+def cpu_baseline_bidir(args):
+    """The oracle's bidirectional fwd+bwd on a bounded sample (all heads, the
+    first 32768 positions of batch 0), for the --bidir line."""
+    import oracle
+    tokens = 32768
+    w = lasp_inputs.WORKLOADS[args.workload]
+    inp = lasp_inputs.make_inputs(1, tokens, w["H"], w["d"], seed=w["seed"], bf16=w["bf16"], decayed=False)
+    q, k, v, do = (lasp_inputs.as_f32(inp[n], w["bf16"]) for n in ("q", "k", "v", "do"))
+    oracle.build()
+    t0 = time.perf_counter()
+    oracle.bidir_fwd(q, k, v)
+    oracle.bidir_bwd(q, k, v, do)
+    value = tokens / (time.perf_counter() - t0)
+    return {"value": round(value, 1), "unit": "tokens/s", "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": f"fp64 oracle bidirectional fwd+bwd, batch 0, all heads, first {tokens} positions"}
+
+
+def cpu_baseline_gated(args):
+    """The oracle's gated fwd+bwd on a bounded sample (all heads, the first
+    32768 positions of batch 0, the bench's gates), for the --gated line."""
+    import oracle
+    tokens = 32768
+    w = lasp_inputs.WORKLOADS[args.workload]
+    inp = lasp_inputs.make_inputs(1, tokens, w["H"], w["d"], seed=w["seed"], bf16=w["bf16"], decayed=False)
+    q, k, v, do = (lasp_inputs.as_f32(inp[n], w["bf16"]) for n in ("q", "k", "v", "do"))
+    g = lasp_inputs.make_log_gates(1, tokens, w["H"], w["d"], seed=w["seed"])
+    oracle.build()
+    t0 = time.perf_counter()
+    oracle.gla_fwd(q, k, v, g)
+    oracle.gla_bwd(q, k, v, g, do)
+    value = tokens / (time.perf_counter() - t0)
+    return {"value": round(value, 1), "unit": "tokens/s", "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": f"fp64 oracle gated fwd+bwd, batch 0, all heads, first {tokens} positions"}
+
+
 def run_reference(args, rank, world):
     if rank != 0:
         return None
@@ -630,8 +665,12 @@ def main(argv=None):
             line = run_reference(args, rank, world)
         elif args.bidir:
             line = run_bidir(args, rank, world, local)
+            if rank == 0 and world == 1 and not args.no_cpu_baseline:
+                line["cpu_baseline"] = cpu_baseline_bidir(args)
         elif args.gated:
             line = run_gated(args, rank, world, local)
+            if rank == 0 and world == 1 and not args.no_cpu_baseline:
+                line["cpu_baseline"] = cpu_baseline_gated(args)
         else:
             line = run_gpu(args, rank, world, local)
             if rank == 0 and world == 1 and not args.no_cpu_baseline:
