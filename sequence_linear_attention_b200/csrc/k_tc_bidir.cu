@@ -119,17 +119,6 @@ struct Smem {
   int abort;
 };
 
-__device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
-  __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
-  return *reinterpret_cast<uint32_t*>(&h);
-}
-__device__ __forceinline__ void st_tile16(uint8_t* tile, int row, int col, uint4 v) {
-  *reinterpret_cast<uint4*>(tile + (col >> 6) * kBox + sw128_offset(row, (col & 63) >> 3)) = v;
-}
-__device__ __forceinline__ uint64_t kmaj(uint32_t tile, int kk) {
-  return sw128_desc(tile + (kk >> 2) * kBox + (kk & 3) * 32, 16, 1024);
-}
-__device__ __forceinline__ uint64_t mnmaj(uint32_t tile, int kk) { return sw128_desc(tile + kk * 2048, kBox, 1024); }
 
 // Y[b, tile rows, h, :] = X[b, tile rows, h, :] S_bh, S_bh the bf16 operand
 // tile of (b, h) used as stored (b_kmajor = 0: Y = X S) or transposed

@@ -51,14 +51,7 @@ struct Smem {
   float pw[kTile];
 };
 
-__device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
-  __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
-  return *reinterpret_cast<uint32_t*>(&h);
-}
 
-__device__ __forceinline__ void st_tile16(uint8_t* tile, int row, int col, uint4 v) {
-  *reinterpret_cast<uint4*>(tile + (col >> 6) * kBox + sw128_offset(row, (col & 63) >> 3)) = v;
-}
 
 // Row r of a d x d fp32 state [m][e], float4 `lane` (columns 4*lane..4*lane+3),
 // written as bf16 into the operand tile (row m, column e).
@@ -79,12 +72,6 @@ __device__ __forceinline__ void load_state_tile(uint8_t* tile, const float* src,
   for (int u = 0; u < kRowsPerWarp; ++u) put_state_row(tile, warp + kWarps * u, lane, x[u]);
 }
 
-// K-major operand descriptor for K step kk (16 elements) of a 128 x 128 tile.
-__device__ __forceinline__ uint64_t kmaj(uint32_t tile, int kk) {
-  return sw128_desc(tile + (kk >> 2) * kBox + (kk & 3) * 32, 16, 1024);
-}
-// MN-major operand descriptor for K step kk (16 rows) of a 128 x 128 tile.
-__device__ __forceinline__ uint64_t mnmaj(uint32_t tile, int kk) { return sw128_desc(tile + kk * 2048, kBox, 1024); }
 
 __global__ void __launch_bounds__(kThreads, 1) chunk_bwd_tc(const __grid_constant__ CUtensorMap map_q,
                                                              const __grid_constant__ CUtensorMap map_k,

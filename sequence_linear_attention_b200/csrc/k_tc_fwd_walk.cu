@@ -68,22 +68,11 @@ struct Smem {
   float pw[kTile];
 };
 
-__device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
-  __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
-  return *reinterpret_cast<uint32_t*>(&h);
-}
 __device__ __forceinline__ uint32_t scale_bf16x2(uint32_t x, float w) {
   __nv_bfloat162 h = *reinterpret_cast<__nv_bfloat162*>(&x);
   float2 f = __bfloat1622float2(h);
   return pack_bf16(f.x * w, f.y * w);
 }
-__device__ __forceinline__ void st_tile16(uint8_t* tile, int row, int col, uint4 v) {
-  *reinterpret_cast<uint4*>(tile + (col >> 6) * kBox + sw128_offset(row, (col & 63) >> 3)) = v;
-}
-__device__ __forceinline__ uint64_t kmaj(uint32_t tile, int kk) {
-  return sw128_desc(tile + (kk >> 2) * kBox + (kk & 3) * 32, 16, 1024);
-}
-__device__ __forceinline__ uint64_t mnmaj(uint32_t tile, int kk) { return sw128_desc(tile + kk * 2048, kBox, 1024); }
 
 // 32 fp32 values of row `row` (columns col..col+31) -> bf16 into a tile.
 __device__ __forceinline__ void st_row32_bf16(uint8_t* tile, int row, int col, const float* v) {

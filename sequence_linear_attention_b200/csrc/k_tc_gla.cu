@@ -51,20 +51,6 @@ constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kMaxSpan = 80.f;  // largest |b_t - r| (natural log) the factorized form takes
 constexpr uint32_t kBarAll = 1;   // named barrier over all 256 threads
 
-__device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
-  __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
-  return *reinterpret_cast<uint32_t*>(&h);
-}
-__device__ __forceinline__ float2 unpack_bf16(uint32_t x) {
-  return __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&x));
-}
-__device__ __forceinline__ uint4* tile16(uint8_t* tile, int row, int col) {
-  return reinterpret_cast<uint4*>(tile + (col >> 6) * kBox + sw128_offset(row, (col & 63) >> 3));
-}
-__device__ __forceinline__ uint64_t kmaj(uint32_t tile, int kk) {
-  return sw128_desc(tile + (kk >> 2) * kBox + (kk & 3) * 32, 16, 1024);
-}
-__device__ __forceinline__ uint64_t mnmaj(uint32_t tile, int kk) { return sw128_desc(tile + kk * 2048, kBox, 1024); }
 
 // Multiplies the 64 bf16 entries of row `row`, columns half*64.., of a tile by
 // exp2(sgn * x[u]) (x in log2 units), in place.

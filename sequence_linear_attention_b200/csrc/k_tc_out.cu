@@ -47,15 +47,7 @@ struct Smem {
 // Writes 8 consecutive bf16 (16 bytes) of row `row`, starting at column
 // `col` (a multiple of 8), into a 128 x 128 tile stored as two 64-column,
 // 128-byte-swizzled boxes.
-__device__ __forceinline__ void st_tile16(uint8_t* tile, int row, int col, uint4 v) {
-  uint8_t* box = tile + (col >> 6) * kBox;
-  *reinterpret_cast<uint4*>(box + sw128_offset(row, (col & 63) >> 3)) = v;
-}
 
-__device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
-  __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
-  return *reinterpret_cast<uint32_t*>(&h);
-}
 
 __global__ void __launch_bounds__(kThreads, 1) chunk_out_tc(const __grid_constant__ CUtensorMap map_q,
                                                              const __grid_constant__ CUtensorMap map_k,

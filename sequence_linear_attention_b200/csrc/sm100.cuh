@@ -3,6 +3,8 @@
 // MMA with TMEM accumulators, TMEM loads/stores). Plain functions; no state.
 #pragma once
 
+#include <cuda_bf16.h>
+
 #include <cuda.h>
 #include <stdint.h>
 
@@ -308,6 +310,34 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, int a_mn, int b_
 // 128-byte-swizzled tile whose rows are 128 bytes and whose base is 1024-aligned.
 __device__ __forceinline__ uint32_t sw128_offset(uint32_t row, uint32_t chunk16) {
   return row * 128u + ((chunk16 ^ (row & 7u)) << 4);
+}
+
+// ---- 128 x 128 bf16 operand tiles, as the tensor-core kernels stage them: two
+// boxes of 64 features x 128 rows (16 KB each, 128-byte swizzle), `box` bytes
+// apart (kOpBox when they are contiguous).
+constexpr uint32_t kOpBox = 128 * 64 * 2;
+
+__device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
+  __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+__device__ __forceinline__ float2 unpack_bf16(uint32_t x) {
+  return __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&x));
+}
+// The 16-byte chunk of row `row` that holds columns col..col+7 (col a multiple of 8).
+__device__ __forceinline__ uint4* tile16(uint8_t* tile, int row, int col, uint32_t box = kOpBox) {
+  return reinterpret_cast<uint4*>(tile + (col >> 6) * box + sw128_offset(row, (col & 63) >> 3));
+}
+__device__ __forceinline__ void st_tile16(uint8_t* tile, int row, int col, uint4 v, uint32_t box = kOpBox) {
+  *tile16(tile, row, col, box) = v;
+}
+// Operand descriptors for K step kk (16 elements of K) of such a tile: K-major
+// (K along the features) and MN-major (K along the rows).
+__device__ __forceinline__ uint64_t kmaj(uint32_t tile, int kk, uint32_t box = kOpBox) {
+  return sw128_desc(tile + (kk >> 2) * box + (kk & 3) * 32, 16, 1024);
+}
+__device__ __forceinline__ uint64_t mnmaj(uint32_t tile, int kk, uint32_t box = kOpBox) {
+  return sw128_desc(tile + kk * 2048, box, 1024);
 }
 
 }  // namespace sm100
