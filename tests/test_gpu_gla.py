@@ -264,3 +264,34 @@ def test_tensor_core_path_chunks_dividing_the_tile(C):
     got = _run(inp, g, C, init=init, dstate_in=dsin)
     ref = _reference(inp, g, init=init.astype(np.float64), dstate_in=dsin.astype(np.float64))
     _compare(got, ref, TOL_BF16)
+
+
+def test_bench_size_sampled_heads():
+    """The gated bench configuration (B1 H16 N65536 d128 C128, bf16, gates
+    log(sigmoid(x))/16) run on the GPU as bench.py times it; two whole heads
+    (every position) of o, dq, dk, dv and dg against the oracle."""
+    import torch
+    import sequence_linear_attention_b200 as lasp
+    w = lasp_inputs.WORKLOADS["decayed_bf16_N64K"]
+    B, N, H, d, C = w["B"], w["N"], w["H"], w["d"], 128
+    inp = lasp_inputs.make_inputs(B, N, H, d, seed=w["seed"], bf16=True, decayed=False)
+    g = lasp_inputs.make_log_gates(B, N, H, d, seed=w["seed"])
+    q, k, v, do = (to_device(inp[n], True) for n in ("q", "k", "v", "do"))
+    gd = _gates_device(g)
+    cache = torch.empty(lasp.lasp_gla_cache_floats(B, H, N, d, C), dtype=torch.float32, device="cuda")
+    ws = torch.empty(B * (N // C) * H * d * d, dtype=torch.float32, device="cuda")
+    o, dq, dk, dv = (torch.empty_like(q) for _ in range(4))
+    dg = torch.empty_like(gd)
+    lasp.lasp_gla_fwd(q, k, v, gd, o, C, cache)
+    lasp.lasp_gla_bwd(q, k, v, gd, do, dq, dk, dv, dg, C, cache, ws)
+    status, site = lasp.lasp_check_device_status()
+    assert status == 0, (status, site)
+    heads = [3, 14]
+    got = {n: to_host(t)[:, :, heads] for n, t in (("o", o), ("dq", dq), ("dk", dk), ("dv", dv))}
+    got["dg"] = dg.cpu().numpy()[:, :, heads]
+    sub = lambda x: np.ascontiguousarray(x[:, :, heads])
+    qh, kh, vh, doh = (sub(host_f32(inp, n)) for n in ("q", "k", "v", "do"))
+    gh = sub(g)
+    ref = {"o": oracle.gla_fwd(qh, kh, vh, gh)}
+    ref["dq"], ref["dk"], ref["dv"], ref["dg"] = oracle.gla_bwd(qh, kh, vh, gh, doh)
+    _compare(got, ref, TOL_BF16, keys=("o", "dq", "dk", "dv", "dg"))
