@@ -93,15 +93,15 @@ def flops_per_step(tokens_heads: int, d: int, C: int) -> float:
 MEASURED_TRAFFIC = {
     # DRAM bytes per launch at the workload's full size: twice the ncu capture of
     # the 32768-token case of the same workload (traffic grows with the tokens)
-    "bwd_walk_tc": (["k_tc_bwd_walk.cu", "sm100.cuh", "lasp_common.cuh", "tma_host.h"], "abcc9f96a59d67ba",
-                    2 * (723881216 + 367207936)),
-    "fwd_walk_tc": (["k_tc_fwd_walk.cu", "sm100.cuh", "lasp_common.cuh", "tma_host.h"], "4c265c8661c3ab71",
-                    2 * (437796352 + 231188992)),
-    "segment_states_tc": (["k_tc_states.cu", "sm100.cuh", "lasp_common.cuh", "tma_host.h"], "38b8cf4a1ea255d1",
-                          2 * (268475648 + 5562368)),
+    "bwd_walk_tc": (["k_tc_bwd_walk.cu", "sm100.cuh", "lasp_common.cuh", "tma_host.h"], "94ed7a7710fac966",
+                    2 * (721036800 + 365295104)),
+    "fwd_walk_tc": (["k_tc_fwd_walk.cu", "sm100.cuh", "lasp_common.cuh", "tma_host.h"], "af6d12c4ff311f6e",
+                    2 * (437424128 + 227407616)),
+    "segment_states_tc": (["k_tc_states.cu", "sm100.cuh", "lasp_common.cuh", "tma_host.h"], "fc6351767f0401ee",
+                          2 * (268477696 + 5350400)),
     # the gated form (bench.py --gated): four times the capture of the 16384-token case
-    "gla_bwd_tc": (["k_tc_gla.cu", "sm100.cuh", "lasp_common.cuh", "tma_host.h"], "d6bbaff4f2a82e85",
-                   4 * (750259456 + 292590848)),
+    "gla_bwd_tc": (["k_tc_gla.cu", "sm100.cuh", "lasp_common.cuh", "tma_host.h"], "11f76e5b0e16c64d",
+                   4 * (750056448 + 291878656)),
 }
 
 
