@@ -595,11 +595,25 @@ __global__ void __launch_bounds__(kThreads, 1) gla_bwd_tc(
       for (int kk = 0; kk < kD / 16; ++kk) mma_bf16(tmem + T2, kmaj(aD, kk), kmaj(aX, kk), id_kk, kk != 0);
       mma_commit(&s->mma1b);
     }
-    // R rows (fp32) into registers while the MMAs run
+    // while the MMAs run: R rows (fp32) into registers, and <R'_m, P'_m> (fp32)
+    // = e^{b_end_m} <R_m, P_m> into bnd, with P's rows read again (from L2)
     const float4* R4 = reinterpret_cast<const float4*>(R + rslot * kD * kD);
     float4 rreg[16];
 #pragma unroll
     for (int u = 0; u < 16; ++u) rreg[u] = __ldcs(R4 + (warp + 8 * u) * (kD / 4) + lane);
+    {
+      const float4* P4 = reinterpret_cast<const float4*>(P + pslot * kD * kD);
+      float4 pv[16];
+#pragma unroll
+      for (int u = 0; u < 16; ++u) pv[u] = __ldg(P4 + (warp + 8 * u) * (kD / 4) + lane);
+#pragma unroll
+      for (int u = 0; u < 16; ++u) {
+        float dot = pv[u].x * rreg[u].x + pv[u].y * rreg[u].y + pv[u].z * rreg[u].z + pv[u].w * rreg[u].w;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
+        if (lane == 0) s->bnd[warp + 8 * u] = dot * wr[u] * we[u];
+      }
+    }
     // ---- epilogue 1: dA . strict -> sA, A . causal -> sB, the diagonal of dA
     if (mbar_wait(&s->mma1a, 0, SITE_BWD_MMA)) {
       tc_fence_after();
@@ -631,20 +645,10 @@ __global__ void __launch_bounds__(kThreads, 1) gla_bwd_tc(
     } else {
       s->abort = 1;
     }
-    // X is free once dO P'^T has read P': R' = diag(e^{b_end - r}) R_c replaces it,
-    // and <R'_m, P'_m> (fp32) = e^{b_end_m} <R_m, P_m> goes to bnd
+    // X is free once dO P'^T has read P': R' = diag(e^{b_end - r}) R_c replaces it
     if (mbar_wait(&s->mma1b, 0, SITE_BWD_MMA)) {
-      const float4* P4 = reinterpret_cast<const float4*>(P + pslot * kD * kD);
 #pragma unroll
-      for (int u = 0; u < 16; ++u) {
-        const int m = warp + 8 * u;
-        const float4 pv = __ldg(P4 + m * (kD / 4) + lane);
-        float dot = pv.x * rreg[u].x + pv.y * rreg[u].y + pv.z * rreg[u].z + pv.w * rreg[u].w;
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
-        if (lane == 0) s->bnd[m] = dot * wr[u] * we[u];
-        put_state_row(sX, m, lane, rreg[u], we[u]);
-      }
+      for (int u = 0; u < 16; ++u) put_state_row(sX, warp + 8 * u, lane, rreg[u], we[u]);
     } else {
       s->abort = 1;
     }
@@ -781,8 +785,15 @@ __global__ void __launch_bounds__(kThreads, 1) gla_bwd_tc(
       s->abort = 1;
     }
     tc_fence_before();
-    __syncthreads();  // every Q^ and K^ row has been read
+    __syncthreads();  // every Q^ and K^ row has been read; dK and dV are staged
     tc_fence_after();
+    if (tid == 0 && !s->abort) {  // dK and dV leave now, under the log-gate gradient's sums
+      tma_store_4d(&map_dk, sA, 0, h, (int)row0, b);
+      tma_store_4d(&map_dk, sA + kBox, 64, h, (int)row0, b);
+      tma_store_4d(&map_dv, sB, 0, h, (int)row0, b);
+      tma_store_4d(&map_dv, sB + kBox, 64, h, (int)row0, b);
+      tma_store_commit();
+    }
 #pragma unroll
     for (int c2 = 0; c2 < 2; ++c2) {
       const int col0 = half * 64 + c2 * 32;
@@ -850,14 +861,10 @@ __global__ void __launch_bounds__(kThreads, 1) gla_bwd_tc(
     fence_async_smem();
     __syncthreads();
     if (tid == 0 && !s->abort) {
-      tma_store_4d(&map_dk, sA, 0, h, (int)row0, b);
-      tma_store_4d(&map_dk, sA + kBox, 64, h, (int)row0, b);
-      tma_store_4d(&map_dv, sB, 0, h, (int)row0, b);
-      tma_store_4d(&map_dv, sB + kBox, 64, h, (int)row0, b);
 #pragma unroll
       for (int cb = 0; cb < 4; ++cb) tma_store_4d(&map_dg, fB + cb * (kTile * 32), cb * 32, h, (int)row0, b);
       tma_store_commit();
-      tma_store_wait_read0();
+      tma_store_wait_read0();  // all stores have read shared memory before the CTA exits
     }
   }
 cleanup:
