@@ -100,8 +100,8 @@ MEASURED_TRAFFIC = {
     "segment_states_tc": (["k_tc_states.cu", "sm100.cuh", "lasp_common.cuh", "tma_host.h"], "fc6351767f0401ee",
                           2 * (268477696 + 5350400)),
     # the gated form (bench.py --gated): four times the capture of the 16384-token case
-    "gla_bwd_tc": (["k_tc_gla.cu", "sm100.cuh", "lasp_common.cuh", "tma_host.h"], "11f76e5b0e16c64d",
-                   4 * (750056448 + 291878656)),
+    "gla_bwd_tc": (["k_tc_gla.cu", "sm100.cuh", "lasp_common.cuh", "tma_host.h"], "58ff562f104f25ca",
+                   4 * (730221312 + 292373248)),
 }
 
 
