@@ -77,13 +77,16 @@ __device__ __forceinline__ int gate_slot(int t, int i) {
   return (i >> 5) * (kTile * 32) + t * 32 + 4 * (((i & 31) >> 2) ^ (t & 7)) + (i & 3);
 }
 
-// Feature i (one per thread of warps 0-3): the log-gates of the tile become
-// b_t[i] = sum_{r<=t} g_r[i] in place; b at the middle row goes to r[], at the
-// last row to bend[].
-__device__ __forceinline__ void walk_tile(float* bt, int i, float* r, float* bend) {
+// Feature i = tid % 128 over the rows of half tid / 128 of the tile (both
+// halves at once, all 256 threads): the log-gates become sums from the half's
+// first row, in place. Rows 0-63 then hold b_t; rows 64-127 hold b_t - r with
+// r = b_63, the middle row. r goes to r[], the second half's total b_end - r
+// to dend[].
+__device__ __forceinline__ void walk_tile(float* bt, int tid, float* r, float* dend) {
+  const int i = tid & (kD - 1), t1 = (tid >> 7) * (kTile / 2);
   float acc = 0.f;
 #pragma unroll 1
-  for (int t0 = 0; t0 < kTile; t0 += 8) {
+  for (int t0 = t1; t0 < t1 + kTile / 2; t0 += 8) {
     float v[8];
 #pragma unroll
     for (int u = 0; u < 8; ++u) v[u] = bt[gate_slot(t0 + u, i)];
@@ -91,10 +94,9 @@ __device__ __forceinline__ void walk_tile(float* bt, int i, float* r, float* ben
     for (int u = 0; u < 8; ++u) {
       acc += v[u];
       bt[gate_slot(t0 + u, i)] = acc;
-      if (t0 + u == kTile / 2 - 1) r[i] = acc;
     }
   }
-  bend[i] = acc;
+  (t1 == 0 ? r : dend)[i] = acc;
 }
 
 // The 64 values of row t, columns half*64.., of such a tile.
@@ -290,21 +292,20 @@ cleanup:
 }
 
 // Phase 0 of the output and backward kernels: once the gate tile has landed
-// (barrier gbar), its walk (warps 0-3; b at the middle row into r[], at the
-// last row into bend[]), then, for row t and column half `half` of every
-// thread, the range check and x = (b_t - r) log2 e, returned in x[].
+// (barrier gbar), its walk (b at the middle row into r[], b_end - r into
+// dend[]), then, for row t and column half `half` of every thread, the range
+// check and x = (b_t - r) log2 e, returned in x[].
 __device__ __forceinline__ void gate_rows(float* bt, uint64_t* gbar, int* abort, unsigned int site, float* r,
-                                          float* bend, int tid, int t, int half, float (&x)[64]) {
-  if (tid < kD) {
-    if (!mbar_wait(gbar, 0, site)) *abort = 1;
-    walk_tile(bt, tid, r, bend);
-  }
+                                          float* dend, int tid, int t, int half, float (&x)[64]) {
+  if (!mbar_wait(gbar, 0, site)) *abort = 1;
+  walk_tile(bt, tid, r, dend);
   named_sync(kBarAll, kThreads);
   read_gate_row(bt, t, half, x);
+  const bool first = t < kTile / 2;  // rows of the second half already hold b_t - r
   bool ok = true;
 #pragma unroll
   for (int u = 0; u < 64; ++u) {
-    const float y = x[u] - r[half * 64 + u];
+    const float y = first ? x[u] - r[half * 64 + u] : x[u];
     ok = ok && fabsf(y) <= kMaxSpan;
     x[u] = y * kLog2e;
   }
@@ -316,7 +317,7 @@ struct SmemOut {
   uint64_t gload, load, mma1, mma2;
   uint32_t tmem_base;
   int abort;
-  float r[kD], bend[kD];
+  float r[kD], dend[kD];
 };
 
 __global__ void __launch_bounds__(kThreads, 1) gla_out_tc(const __grid_constant__ CUtensorMap map_q,
@@ -375,7 +376,7 @@ __global__ void __launch_bounds__(kThreads, 1) gla_out_tc(const __grid_constant_
     tma_load_4d(sV + kBox, &map_v, &s->load, 64, h, (int)row0, b);
   }
   float x[64];
-  gate_rows(bt, &s->gload, &s->abort, SITE_OUT_TMA, s->r, s->bend, tid, t, half, x);
+  gate_rows(bt, &s->gload, &s->abort, SITE_OUT_TMA, s->r, s->dend, tid, t, half, x);
   // P' = diag(e^{r}) P_c into X
   {
     float w[16];
@@ -477,7 +478,7 @@ struct SmemBwd {
 
 // One 128-token tile per CTA. Shared memory: Q^, K^, V, dO (then, in pairs,
 // the fp32 tiles of dB and k . dk^inter for the log-gate gradient's column
-// sums), X (P', then R'; r and b_end during the gate walk), and the pair
+// sums), X (P', then R'; r and b_end - r during the gate walk), and the pair
 // sA / sB (the gate tile during the walk; then dA . strict and A . causal;
 // then the dK and dV outputs). TMEM: T0 = dO V^T -> (dA . strict)^T Q^;
 // T1 = Q^ K^^T -> dV; T2 = dO P'^T + (dA . strict) K^ -> q . dq'; T3 = log2 E
@@ -500,8 +501,8 @@ __global__ void __launch_bounds__(kThreads, 1) gla_bwd_tc(
   uint8_t* sB = base + 6 * kTileBytes;
   SmemBwd* s = reinterpret_cast<SmemBwd*>(base + 7 * kTileBytes);
   float* bt = reinterpret_cast<float*>(sA);  // gate tile over sA and sB during the walk
-  float* sr = reinterpret_cast<float*>(sX);  // r and b_end over X during the walk
-  float* sbend = sr + kD;
+  float* sr = reinterpret_cast<float*>(sX);  // r and b_end - r over X during the walk
+  float* sdend = sr + kD;
   const int c = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int t = (warp & 3) * 32 + lane, half = warp >> 2;
@@ -552,15 +553,15 @@ __global__ void __launch_bounds__(kThreads, 1) gla_bwd_tc(
   }
   // ---- phase 0: gates, Q^, K^, log2 E -> T3, P' -> X
   float x[64];
-  gate_rows(bt, &s->gload, &s->abort, SITE_BWD_TMA, sr, sbend, tid, t, half, x);
+  gate_rows(bt, &s->gload, &s->abort, SITE_BWD_TMA, sr, sdend, tid, t, half, x);
   float wr[16], we[16];  // e^{r_m} and e^{b_end_m - r_m} of this thread's state rows m = warp + 8u
 #pragma unroll
   for (int u = 0; u < 16; ++u) {
     const int m = warp + 8 * u;
     wr[u] = exp2f(sr[m] * kLog2e);
-    we[u] = exp2f((sbend[m] - sr[m]) * kLog2e);
+    we[u] = exp2f(sdend[m] * kLog2e);
   }
-  named_sync(kBarAll, kThreads);  // r and b_end are read before X is written
+  named_sync(kBarAll, kThreads);  // r and b_end - r are read before X is written
   load_scaled_state(sX, P + pslot * kD * kD, wr, warp, lane);
   if (!mbar_wait(&s->load, 0, SITE_BWD_TMA)) s->abort = 1;
   scale_row_half(sQ, t, half, x, 1.f);   // Q^ = q . E
