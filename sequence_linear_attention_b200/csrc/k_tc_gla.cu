@@ -29,8 +29,10 @@
 // and the column half w/4 of every row-wise step. The cumulative log-gates:
 // the state kernel sums them by 16-row groups (a warp per group, float4 loads)
 // and scales its operand in place; the output and backward kernels load the
-// gate tile by TMA and walk it in shared memory, one feature per thread of
-// warps 0-3, before the row-wise steps read it.
+// gate tile by TMA and walk it in shared memory (a feature and half the rows
+// per thread) before the row-wise steps read it.
+#include <algorithm>
+
 #include "kernels.h"
 #include "lasp_common.cuh"
 #include "sm100.cuh"
@@ -292,12 +294,12 @@ cleanup:
 }
 
 // Phase 0 of the output and backward kernels: once the gate tile has landed
-// (barrier gbar), its walk (b at the middle row into r[], b_end - r into
+// (barrier gbar, phase of the given parity), its walk (b at the middle row into r[], b_end - r into
 // dend[]), then, for row t and column half `half` of every thread, the range
 // check and x = (b_t - r) log2 e, returned in x[].
-__device__ __forceinline__ void gate_rows(float* bt, uint64_t* gbar, int* abort, unsigned int site, float* r,
-                                          float* dend, int tid, int t, int half, float (&x)[64]) {
-  if (!mbar_wait(gbar, 0, site)) *abort = 1;
+__device__ __forceinline__ void gate_rows(float* bt, uint64_t* gbar, uint32_t parity, int* abort, unsigned int site,
+                                          float* r, float* dend, int tid, int t, int half, float (&x)[64]) {
+  if (!mbar_wait(gbar, parity, site)) *abort = 1;
   walk_tile(bt, tid, r, dend);
   named_sync(kBarAll, kThreads);
   read_gate_row(bt, t, half, x);
@@ -376,7 +378,7 @@ __global__ void __launch_bounds__(kThreads, 1) gla_out_tc(const __grid_constant_
     tma_load_4d(sV + kBox, &map_v, &s->load, 64, h, (int)row0, b);
   }
   float x[64];
-  gate_rows(bt, &s->gload, &s->abort, SITE_OUT_TMA, s->r, s->dend, tid, t, half, x);
+  gate_rows(bt, &s->gload, 0, &s->abort, SITE_OUT_TMA, s->r, s->dend, tid, t, half, x);
   // P' = diag(e^{r}) P_c into X
   {
     float w[16];
@@ -489,7 +491,7 @@ __global__ void __launch_bounds__(kThreads, 1) gla_bwd_tc(
     const __grid_constant__ CUtensorMap map_dk, const __grid_constant__ CUtensorMap map_dv,
     const __grid_constant__ CUtensorMap map_g, const __grid_constant__ CUtensorMap map_dg,
     const float* __restrict__ P, const float* __restrict__ R, __nv_bfloat16* __restrict__ dq, int H, int64_t N,
-    int64_t t_slots, int stride) {
+    int64_t t_slots, int stride, int ntx, int64_t ntiles) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   uint8_t* sQ = base;
@@ -503,14 +505,20 @@ __global__ void __launch_bounds__(kThreads, 1) gla_bwd_tc(
   float* bt = reinterpret_cast<float*>(sA);  // gate tile over sA and sB during the walk
   float* sr = reinterpret_cast<float*>(sX);  // r and b_end - r over X during the walk
   float* sdend = sr + kD;
-  const int c = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int t = (warp & 3) * 32 + lane, half = warp >> 2;
-  const int64_t row0 = (int64_t)c * kTile;
-  // P of the tile's first chunk and R of its last
-  const int64_t pslot = ((int64_t)b * t_slots + (int64_t)c * stride) * H + h;
-  const int64_t rslot = pslot + (int64_t)(stride - 1) * H;
-  const int64_t tok = (((int64_t)b * N + row0 + t) * H + h) * kD;  // row t of every token tensor
+  // tile w: 128 tokens c * 128.. of head h of sequence b, in launch order
+  auto tile_of = [&](int64_t w, int& c, int& h, int& b) {
+    c = (int)(w % ntx);
+    h = (int)((w / ntx) % H);
+    b = (int)(w / ((int64_t)ntx * H));
+  };
+  // P of a tile's first chunk (R of its last is stride - 1 slots on)
+  auto pslot_of = [&](int c, int h, int b) { return ((int64_t)b * t_slots + (int64_t)c * stride) * H + h; };
+  auto load_tokens = [&](uint8_t* dst, const CUtensorMap* map, int h, int row, int b) {
+    tma_load_4d(dst, map, &s->load, 0, h, row, b);
+    tma_load_4d(dst + kBox, map, &s->load, 64, h, row, b);
+  };
   if (tid == 0) {
     prefetch_tmap(&map_q);
     prefetch_tmap(&map_k);
@@ -536,24 +544,33 @@ __global__ void __launch_bounds__(kThreads, 1) gla_bwd_tc(
   const uint32_t tmem = s->tmem_base;
   const uint32_t lane_base = tmem + ((uint32_t)((warp & 3) * 32) << 16);
   const uint32_t T0 = 0, T1 = 128, T2 = 256, T3 = 384;
-  if (tid == 0) {
-    load_gate_tile(bt, &map_g, &s->gload, h, (int)row0, b);
+  if (tid == 0 && (int64_t)blockIdx.x < ntiles) {
+    // the first tile's loads; a later tile's are issued during the tile before
+    int c, h, b;
+    tile_of(blockIdx.x, c, h, b);
+    const int64_t ps = pslot_of(c, h, b);
+    load_gate_tile(bt, &map_g, &s->gload, h, c * kTile, b);
     // P and R are read with plain loads later: into L2 now
-    bulk_prefetch_l2(P + pslot * kD * kD, kD * kD * 4);
-    bulk_prefetch_l2(R + rslot * kD * kD, kD * kD * 4);
+    bulk_prefetch_l2(P + ps * kD * kD, kD * kD * 4);
+    bulk_prefetch_l2(R + (ps + (int64_t)(stride - 1) * H) * kD * kD, kD * kD * 4);
     mbar_arrive_expect_tx(&s->load, 4 * kTileBytes);
-    tma_load_4d(sQ, &map_q, &s->load, 0, h, (int)row0, b);
-    tma_load_4d(sQ + kBox, &map_q, &s->load, 64, h, (int)row0, b);
-    tma_load_4d(sK, &map_k, &s->load, 0, h, (int)row0, b);
-    tma_load_4d(sK + kBox, &map_k, &s->load, 64, h, (int)row0, b);
-    tma_load_4d(sV, &map_v, &s->load, 0, h, (int)row0, b);
-    tma_load_4d(sV + kBox, &map_v, &s->load, 64, h, (int)row0, b);
-    tma_load_4d(sD, &map_do, &s->load, 0, h, (int)row0, b);
-    tma_load_4d(sD + kBox, &map_do, &s->load, 64, h, (int)row0, b);
+    load_tokens(sQ, &map_q, h, c * kTile, b);
+    load_tokens(sK, &map_k, h, c * kTile, b);
+    load_tokens(sV, &map_v, h, c * kTile, b);
+    load_tokens(sD, &map_do, h, c * kTile, b);
   }
+  uint32_t ph = 0;  // parity of every barrier's phase for this CTA's current tile
+  for (int64_t w = blockIdx.x; w < ntiles; w += gridDim.x, ph ^= 1u) {
+  int c, h, b;
+  tile_of(w, c, h, b);
+  const int64_t row0 = (int64_t)c * kTile;
+  const int64_t pslot = pslot_of(c, h, b);
+  const int64_t rslot = pslot + (int64_t)(stride - 1) * H;
+  const int64_t tok = (((int64_t)b * N + row0 + t) * H + h) * kD;  // row t of every token tensor
+  const int64_t wn = w + gridDim.x;  // this CTA's next tile
   // ---- phase 0: gates, Q^, K^, log2 E -> T3, P' -> X
   float x[64];
-  gate_rows(bt, &s->gload, &s->abort, SITE_BWD_TMA, sr, sdend, tid, t, half, x);
+  gate_rows(bt, &s->gload, ph, &s->abort, SITE_BWD_TMA, sr, sdend, tid, t, half, x);
   float wr[16], we[16];  // e^{r_m} and e^{b_end_m - r_m} of this thread's state rows m = warp + 8u
 #pragma unroll
   for (int u = 0; u < 16; ++u) {
@@ -563,7 +580,7 @@ __global__ void __launch_bounds__(kThreads, 1) gla_bwd_tc(
   }
   named_sync(kBarAll, kThreads);  // r and b_end - r are read before X is written
   load_scaled_state(sX, P + pslot * kD * kD, wr, warp, lane);
-  if (!mbar_wait(&s->load, 0, SITE_BWD_TMA)) s->abort = 1;
+  if (!mbar_wait(&s->load, ph, SITE_BWD_TMA)) s->abort = 1;
   scale_row_half(sQ, t, half, x, 1.f);   // Q^ = q . E
   scale_row_half(sK, t, half, x, -1.f);  // K^ = k / E
   {
@@ -616,7 +633,7 @@ __global__ void __launch_bounds__(kThreads, 1) gla_bwd_tc(
       }
     }
     // ---- epilogue 1: dA . strict -> sA, A . causal -> sB, the diagonal of dA
-    if (mbar_wait(&s->mma1a, 0, SITE_BWD_MMA)) {
+    if (mbar_wait(&s->mma1a, ph, SITE_BWD_MMA)) {
       tc_fence_after();
 #pragma unroll 1
       for (int c2 = 0; c2 < 2; ++c2) {
@@ -647,7 +664,7 @@ __global__ void __launch_bounds__(kThreads, 1) gla_bwd_tc(
       s->abort = 1;
     }
     // X is free once dO P'^T has read P': R' = diag(e^{b_end - r}) R_c replaces it
-    if (mbar_wait(&s->mma1b, 0, SITE_BWD_MMA)) {
+    if (mbar_wait(&s->mma1b, ph, SITE_BWD_MMA)) {
 #pragma unroll
       for (int u = 0; u < 16; ++u) put_state_row(sX, warp + 8 * u, lane, rreg[u], we[u]);
     } else {
@@ -666,7 +683,7 @@ __global__ void __launch_bounds__(kThreads, 1) gla_bwd_tc(
     // ---- epilogue 2: dq' = E . T2; dq = dq' + (do_t . v_t) k_t = E . (T2 + (do_t . v_t) K^_t);
     // q . dq' = Q^ . T2 -> T2
     float xl[64];  // log2 E of row t, kept for epilogue 3
-    if (mbar_wait(&s->mma2, 0, SITE_BWD_MMA)) {
+    if (mbar_wait(&s->mma2, ph, SITE_BWD_MMA)) {
       tc_fence_after();
       {
         uint32_t r0[32], r1[32];
@@ -732,7 +749,7 @@ __global__ void __launch_bounds__(kThreads, 1) gla_bwd_tc(
     // tiles over the token buffers for the column sums
     float* fB = reinterpret_cast<float*>(sQ);  // over sQ and sK
     float* fK = reinterpret_cast<float*>(sV);  // over sV and sD
-    if (mbar_wait(&s->mma3, 0, SITE_BWD_MMA)) {
+    if (mbar_wait(&s->mma3, ph, SITE_BWD_MMA)) {
       tc_fence_after();
       const float dad = s->dAd[t];
 #pragma unroll
@@ -846,6 +863,17 @@ __global__ void __launch_bounds__(kThreads, 1) gla_bwd_tc(
       }
     }
     __syncthreads();
+    if (tid == 0 && wn < ntiles && !s->abort) {
+      // the dK and dV stores have read the gate tile's space: the next tile's
+      // gates go there, its P and R into L2
+      tma_store_wait_read0();
+      int cn, hn, bn;
+      tile_of(wn, cn, hn, bn);
+      const int64_t ps = pslot_of(cn, hn, bn);
+      load_gate_tile(bt, &map_g, &s->gload, hn, cn * kTile, bn);
+      bulk_prefetch_l2(P + ps * kD * kD, kD * kD * 4);
+      bulk_prefetch_l2(R + (ps + (int64_t)(stride - 1) * H) * kD * kD, kD * kD * 4);
+    }
     // dg into the dB tile (the gate map's layout), stored by TMA below
 #pragma unroll
     for (int cb = 0; cb < 2; ++cb) {
@@ -860,13 +888,30 @@ __global__ void __launch_bounds__(kThreads, 1) gla_bwd_tc(
       }
     }
     fence_async_smem();
-    __syncthreads();
-    if (tid == 0 && !s->abort) {
+    __syncthreads();  // fK (over V and dO) has been read; no wait fails after this point
+    const bool stop = s->abort != 0;
+    if (tid == 0) {
+      if (!stop) {
 #pragma unroll
-      for (int cb = 0; cb < 4; ++cb) tma_store_4d(&map_dg, fB + cb * (kTile * 32), cb * 32, h, (int)row0, b);
-      tma_store_commit();
-      tma_store_wait_read0();  // all stores have read shared memory before the CTA exits
+        for (int cb = 0; cb < 4; ++cb) tma_store_4d(&map_dg, fB + cb * (kTile * 32), cb * 32, h, (int)row0, b);
+        tma_store_commit();
+      }
+      const bool next = wn < ntiles && !stop;
+      int cn = 0, hn = 0, bn = 0;
+      if (next) tile_of(wn, cn, hn, bn);
+      if (next) {
+        mbar_arrive_expect_tx(&s->load, 4 * kTileBytes);
+        load_tokens(sV, &map_v, hn, cn * kTile, bn);
+        load_tokens(sD, &map_do, hn, cn * kTile, bn);
+      }
+      tma_store_wait_read0();  // the dg store has read fB (over Q and K); all stores have read shared memory
+      if (next) {
+        load_tokens(sQ, &map_q, hn, cn * kTile, bn);
+        load_tokens(sK, &map_k, hn, cn * kTile, bn);
+      }
     }
+    if (stop) goto cleanup;
+  }
   }
 cleanup:
   tc_fence_before();
@@ -930,8 +975,16 @@ cudaError_t tc_gla_chunk_bwd(const void* q, const void* k, const void* v, const 
   const size_t smem = 1024 + 7 * (size_t)kTileBytes + sizeof(SmemBwd);
   cudaError_t e = cudaFuncSetAttribute(gla_bwd_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  gla_bwd_tc<<<dim3((unsigned)(N / kTile), H, B), kThreads, smem, st>>>(
-      mq, mk, mv, mdo, mdk, mdv, mg, mdg, P, Rs, (__nv_bfloat16*)dq, H, N, t_slots, stride);
+  int dev = 0, sms = 0;
+  if ((e = cudaGetDevice(&dev)) != cudaSuccess ||
+      (e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
+    return e;
+  // one persistent CTA per SM (the kernel holds all of TMEM and most of shared memory)
+  const int ntx = (int)(N / kTile);
+  const int64_t ntiles = (int64_t)B * H * ntx;
+  const unsigned grid = (unsigned)std::min<int64_t>(ntiles, sms);
+  gla_bwd_tc<<<grid, kThreads, smem, st>>>(mq, mk, mv, mdo, mdk, mdv, mg, mdg, P, Rs, (__nv_bfloat16*)dq, H, N, t_slots,
+                                            stride, ntx, ntiles);
   return cudaGetLastError();
 }
 
