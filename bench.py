@@ -45,6 +45,8 @@ def algorithmic_bytes(name: str, tokens_heads: int, d: int, C: int, G: int, elem
       segment_states_tc:             read 2 token rows, write s/G        = 2de + s/G
       state_scan:                    read and write s/C                  = 2s/C
       segment_scan:                  read and write s/G                  = 2s/G
+      state_total:  the decayed total of the segment (or chunk) states,
+                    read only                                            = s/G
       chunk_out_*:                   read q, k, v and P, write o         = 4de + s/C
       fwd_walk_tc:  read q, k, v and the segment's P (s/G), write o and
                     the cache: for C <= 128 the bf16 operand tile of the state
@@ -67,7 +69,7 @@ def algorithmic_bytes(name: str, tokens_heads: int, d: int, C: int, G: int, elem
     per = {
         "chunk_states_tc": 2 * de + s / C, "chunk_states_simt": 2 * de + s / C,
         "segment_states_tc": 2 * de + s / G,
-        "state_scan": 2 * s / C, "segment_scan": 2 * s / G,
+        "state_scan": 2 * s / C, "segment_scan": 2 * s / G, "state_total": s / G,
         "chunk_out_tc": 4 * de + s / C, "chunk_out_simt": 4 * de + s / C, "fwd_walk_tc": 4 * de + (s / G + s / 256 if C <= 128 else s / C),
         "chunk_bwd_tc": 7 * de + 2 * s / C, "chunk_bwd_simt": 7 * de + 2 * s / C,
         "bwd_walk_tc": 7 * de + s / 256 + s / G,
@@ -549,6 +551,119 @@ def run_gated(args, rank, world, local):
     }
 
 
+def run_lasp2(args, rank, world, local):
+    """LASP-2 sequence parallelism: one sequence of the workload split over the
+    ranks, rank r holding tokens [r L, (r + 1) L) with L = N / world; a step is
+    lasp2_fwd + lasp2_bwd, with one AllGather of shard states per direction
+    (NCCL). The sequence is the same at every world size (strong scaling). At
+    one rank the process group has one member and the gather is a copy. Printed
+    as its own line; the default run does not include it."""
+    import tempfile
+
+    import torch
+    import torch.distributed as dist
+
+    import sequence_linear_attention_b200 as lasp
+    from sequence_linear_attention_b200 import lasp2
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    w = lasp_inputs.WORKLOADS[args.workload]
+    B, N, H, d, C = w["B"], (args.tokens or w["N"]), w["H"], w["d"], w["C"]
+    if N % world or (N // world) % C:
+        raise ValueError("the sequence must split into equal shards of whole chunks")
+    L = N // world
+    own_group = None
+    if world == 1:
+        fd, path = tempfile.mkstemp(prefix="lasp2_pg_")
+        os.close(fd)
+        dist.init_process_group("nccl", store=dist.FileStore(path, 1), rank=0, world_size=1)
+        own_group = path
+    inp = lasp_inputs.make_shard_inputs(B, N, H, d, seed=w["seed"], row0=rank * L, rows=L, bf16=w["bf16"],
+                                        decayed=w["decayed"])
+    elem = 2 if w["bf16"] else 4
+    to_dev = ((lambda x: torch.from_numpy(np.ascontiguousarray(x).view(np.int16)).view(torch.bfloat16).to(dev))
+              if w["bf16"] else (lambda x: torch.from_numpy(np.ascontiguousarray(x)).to(dev)))
+    q, k, v, do = (to_dev(inp[n]) for n in ("q", "k", "v", "do"))
+    del inp["q"], inp["k"], inp["v"], inp["do"]
+    decay = None if inp["lam"] is None else torch.from_numpy(inp["lam"]).to(dev)
+    o, dq, dk, dv = (torch.empty_like(q) for _ in range(4))
+    cache = torch.empty((B, L // C, H, d, d), dtype=torch.float32, device=dev)
+    ws = torch.empty_like(cache)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        lasp2.lasp2_fwd(q, k, v, decay, o, C, cache)
+        lasp2.lasp2_bwd(q, k, v, decay, do, dq, dk, dv, C, cache, ws)
+
+    try:
+        for _ in range(args.warmup):
+            step()
+        events = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                  for _ in range(args.steps)]
+        torch.cuda.synchronize(dev)
+        barrier(world, dev)
+        with ClockSampler(local) as clk:
+            for i in range(args.steps):
+                events[i][0].record(stream)
+                step()
+                events[i][1].record(stream)
+            torch.cuda.synchronize(dev)
+        barrier(world, dev)
+        value, t_max = aggregate(B * L * args.steps, sum(a.elapsed_time(b) for a, b in events) / 1e3, world, dev)
+        ksteps = min(args.steps, 50)
+        lasp.lasp_trace_enable(16 * ksteps + 16)
+        for _ in range(ksteps):
+            step()
+        torch.cuda.synchronize(dev)
+        trace = lasp.lasp_trace_read(16 * ksteps + 16)
+        lasp.lasp_trace_enable(0)
+        st, site = lasp.lasp_check_device_status()
+        if st != 0:
+            raise RuntimeError(f"device status {lasp.lasp_status_string(st)} at site {site}")
+    finally:
+        if own_group is not None:
+            dist.destroy_process_group()
+            if os.path.exists(own_group):  # the store may have removed it
+                os.unlink(own_group)
+    per_kernel = {}
+    for name, ms in trace:
+        per_kernel.setdefault(name, []).append(ms)
+    peaks = load_peaks()
+    th = B * L * H
+    G = lasp.lasp_segment_tokens(L, C, d, lasp.LASP_BF16 if w["bf16"] else lasp.LASP_F32)
+
+    def shard_bytes(name):
+        # the scans over the W gathered shard states
+        if name == "state_scan":
+            return 2 * world * B * H * 4 * d * d
+        return algorithmic_bytes(name, th, d, C, G, elem)
+
+    kernel_table = {}
+    for n, ms in per_kernel.items():
+        mean = statistics.mean(ms)
+        gbps = shard_bytes(n) / (mean / 1e3) / 1e9
+        kernel_table[n] = {"launches_per_step": len(ms) / ksteps, "ms": round(mean, 4), "GBps": round(gbps, 1),
+                           "hbm_frac": round(gbps / peaks["hbm"], 4)}
+    top = max(per_kernel, key=lambda n: sum(per_kernel[n]))
+    return {
+        "metric": "LASP-2 sequence-parallel linear-attn fwd+bwd tokens/s", "impl": "lasp2",
+        "value": round(value, 1), "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(t_max * 1e3 / args.steps, 4), "higher_is_better": True,
+        "scaling": "strong", "vs_baseline": None, "dtype": "bf16" if w["bf16"] else "f32",
+        "data": "synthetic (seeded normal q,k,v,dO; no dataset)",
+        "config": {"workload": args.workload, "B": B, "H": H, "N": N, "d": d, "C": C, "shard_tokens": L,
+                   "segment": G, "parallelism": f"sequence x{world} (one AllGather of shard states per direction)",
+                   "l2": "inputs larger than L2"},
+        "roofline": {"bound": "hbm", "kernel": top, "achieved": kernel_table[top]["GBps"], "peak": peaks["hbm"],
+                     "unit": "GB/s", "frac": kernel_table[top]["hbm_frac"], "traffic": None,
+                     "algorithmic_bytes": shard_bytes(top), "peak_source": peaks["source"]},
+        "kernels": kernel_table,
+        "gpu_launches": int(round(len(trace) / ksteps * args.steps)),
+        "clocks": clk.summary(),
+    }
+
+
 # ------------------------------------------------------------------ CPU oracle
 def oracle_sample(args, tokens: int):
     """A bounded sample of the workload for the fp64 oracle: all heads, the
@@ -647,16 +762,22 @@ def main(argv=None):
     ap.add_argument("--steps", type=int, default=1000)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
-    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(lasp_inputs.WORKLOADS))
+    ap.add_argument("--workload", default=None, choices=sorted(lasp_inputs.WORKLOADS),
+                    help=f"workload (default {DEFAULT_WORKLOAD}; with --lasp2, shards_bf16_N2M)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--bidir", action="store_true",
                     help="time the bidirectional (unmasked) form instead (its own metric and line)")
     ap.add_argument("--gated", action="store_true",
                     help="time the gated form (a log-gate per token and key feature) instead (its own metric and line)")
+    ap.add_argument("--lasp2", action="store_true",
+                    help="time LASP-2 sequence parallelism instead: one sequence split over the ranks "
+                         "(its own metric and line)")
     ap.add_argument("--tokens", type=int, default=None,
                     help="sequence length N instead of the workload's (a smaller case of the same shape, for "
                          "profiling); the line is then not the workload's headline number")
     args = ap.parse_args(argv)
+    if args.workload is None:
+        args.workload = "shards_bf16_N2M" if args.lasp2 else DEFAULT_WORKLOAD
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
     rank, world, local = dist_setup()
@@ -667,6 +788,10 @@ def main(argv=None):
             line = run_bidir(args, rank, world, local)
             if rank == 0 and world == 1 and not args.no_cpu_baseline:
                 line["cpu_baseline"] = cpu_baseline_bidir(args)
+        elif args.lasp2:
+            line = run_lasp2(args, rank, world, local)
+            if rank == 0 and world == 1 and not args.no_cpu_baseline:
+                line["cpu_baseline"] = cpu_baseline(args)
         elif args.gated:
             line = run_gated(args, rank, world, local)
             if rank == 0 and world == 1 and not args.no_cpu_baseline:

@@ -192,6 +192,52 @@ LASP_API int lasp_chunk_grads(const void* q, const void* k, const void* v, const
                               int64_t N, int d, int C, int dtype, void* stream);
 
 /*
+ * lasp_fwd_states, lasp_fwd_finish -- lasp_fwd in the two parts that the
+ * LASP-2 exchange separates (LASP-2 "The reading": every shard computes its
+ * memory state M_t, the states are gathered, then each shard takes the prefix
+ * of the earlier shards' states and computes its output). Sizes, dtype and
+ * state_cache as for lasp_fwd; lasp_fwd is lasp_fwd_states (total NULL)
+ * followed by lasp_fwd_finish with the same arguments.
+ *   lasp_fwd_states: the first step of lasp_fwd (the chunk states, or on the
+ *     tensor-core walk path the segment states, into state_cache) and, if
+ *     total (out, float [B, H, d, d]) is non-NULL, the state after the last
+ *     token of a sequence that starts from zero:
+ *       total = sum_s lambda^{N-1-s} k_s^T v_s   (LASP Eq. 10 with C = N),
+ *     the shard state M_t of LASP-2. For N = 0, total is zero.
+ *   lasp_fwd_finish: the rest of lasp_fwd on a cache that lasp_fwd_states
+ *     filled for the same k, v, decay and sizes: the prefix from init_state
+ *     (may be NULL) and the output o.
+ */
+LASP_API int lasp_fwd_states(const void* k, const void* v, const float* decay, int B, int H, int64_t N, int d, int C,
+                             int dtype, float* state_cache, float* total, void* stream);
+LASP_API int lasp_fwd_finish(const void* q, const void* k, const void* v, const float* decay, void* o, int B, int H,
+                             int64_t N, int d, int C, int dtype, float* state_cache, const float* init_state,
+                             void* stream);
+
+/*
+ * lasp_bwd_states, lasp_bwd_finish -- lasp_bwd in the same two parts (LASP-2
+ * backward: gradient states dM_t, gathered, then the suffix over the later
+ * shards and the gradients). Sizes, dtype, state_cache and dstate_ws as for
+ * lasp_bwd; lasp_bwd is lasp_bwd_states (total NULL) followed by
+ * lasp_bwd_finish.
+ *   lasp_bwd_states: the first step of lasp_bwd (the gradient chunk or
+ *     segment states into dstate_ws) and, if total (out, float [B, H, d, d])
+ *     is non-NULL, the gradient state the sequence passes back to the state
+ *     entering its first token when nothing enters from after it:
+ *       total = sum_s lambda^{s+1} q_s^T do_s   (LASP Eq. 20 with C = N),
+ *     the shard gradient state dM_t of LASP-2. For N = 0, total is zero.
+ *   lasp_bwd_finish: the rest of lasp_bwd on a workspace that
+ *     lasp_bwd_states filled for the same q, dout, decay and sizes: the suffix
+ *     from dstate_in (may be NULL), dinit_state (may be NULL), dq, dk, dv.
+ */
+LASP_API int lasp_bwd_states(const void* q, const void* dout, const float* decay, int B, int H, int64_t N, int d,
+                             int C, int dtype, float* dstate_ws, float* total, void* stream);
+LASP_API int lasp_bwd_finish(const void* q, const void* k, const void* v, const float* decay, const void* dout,
+                             void* dq, void* dk, void* dv, int B, int H, int64_t N, int d, int C, int dtype,
+                             const float* state_cache, float* dstate_ws, const float* dstate_in, float* dinit_state,
+                             void* stream);
+
+/*
  * lasp_bwd_noalloc -- lasp_bwd without the caller-provided workspace.
  * The pages have no counterpart to this call; it exists for callers that
  * cannot allocate device memory: a plain C program or plug-in with no device

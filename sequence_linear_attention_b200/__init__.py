@@ -18,12 +18,14 @@ import os
 import threading
 
 __all__ = [
-    "LaspError", "library_path", "lasp_fwd", "lasp_bwd", "lasp_chunk_states", "lasp_chunk_dstates",
+    "LaspError", "library_path", "lasp_fwd", "lasp_bwd", "lasp_fwd_states", "lasp_fwd_finish", "lasp_bwd_states",
+    "lasp_bwd_finish", "lasp_chunk_states", "lasp_chunk_dstates",
     "lasp_chunk_out", "lasp_chunk_grads", "lasp_bwd_noalloc",
     "lasp_state_prefix", "lasp_check_device_status", "lasp_set_wait_limit_ns", "lasp_wait_probe",
     "lasp_status_string", "lasp_version", "lasp_trace_enable", "lasp_trace_read", "lasp_kernel_name",
     "lasp_segment_tokens", "lasp_bidir_workspace_floats", "lasp_bidir_state_offset", "lasp_bidir_fwd",
-    "lasp_bidir_bwd",
+    "lasp_bidir_bwd", "lasp_gla_cache_floats", "lasp_gla_chunk_states", "lasp_gla_state_prefix", "lasp_gla_fwd",
+    "lasp_gla_bwd",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -60,6 +62,10 @@ def _load():
             P, I, L, U64 = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_uint64
             lib.lasp_fwd.argtypes = [P, P, P, P, P, I, I, L, I, I, I, P, P, P]
             lib.lasp_bwd.argtypes = [P, P, P, P, P, P, P, P, I, I, L, I, I, I, P, P, P, P, P, P]
+            lib.lasp_fwd_states.argtypes = [P, P, P, I, I, L, I, I, I, P, P, P]
+            lib.lasp_fwd_finish.argtypes = [P, P, P, P, P, I, I, L, I, I, I, P, P, P]
+            lib.lasp_bwd_states.argtypes = [P, P, P, I, I, L, I, I, I, P, P, P]
+            lib.lasp_bwd_finish.argtypes = [P, P, P, P, P, P, P, P, I, I, L, I, I, I, P, P, P, P, P]
             lib.lasp_chunk_states.argtypes = [P, P, P, P, P, I, I, L, I, I, I, P]
             lib.lasp_chunk_dstates.argtypes = [P, P, P, P, I, I, L, I, I, I, P]
             lib.lasp_bwd_noalloc.argtypes = [P, P, P, P, P, P, P, P, I, I, L, I, I, I, P, P, P, P]
@@ -88,7 +94,8 @@ def _load():
             lib.lasp_gla_bwd.argtypes = [P, P, P, P, P, P, P, P, P, I, I, L, I, I, I, P, P, P, P, P]
             lib.lasp_status_string.argtypes = [I]
             lib.lasp_status_string.restype = ctypes.c_char_p
-            for f in (lib.lasp_fwd, lib.lasp_bwd, lib.lasp_chunk_states, lib.lasp_chunk_dstates,
+            for f in (lib.lasp_fwd, lib.lasp_bwd, lib.lasp_fwd_states, lib.lasp_fwd_finish, lib.lasp_bwd_states,
+                      lib.lasp_bwd_finish, lib.lasp_chunk_states, lib.lasp_chunk_dstates,
                       lib.lasp_chunk_out, lib.lasp_chunk_grads, lib.lasp_bwd_noalloc,
                       lib.lasp_state_prefix, lib.lasp_check_device_status, lib.lasp_set_wait_limit_ns,
                       lib.lasp_wait_probe, lib.lasp_version, lib.lasp_trace_enable, lib.lasp_trace_read,
@@ -154,6 +161,38 @@ def lasp_bwd(q, k, v, decay, dout, dq, dk, dv, C, state_cache, dstate_ws, init_s
     _check(_load().lasp_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(decay), _ptr(dout), _ptr(dq), _ptr(dk), _ptr(dv),
                             B, H, N, d, C, dt, _ptr(state_cache), _ptr(dstate_ws), _ptr(init_state),
                             _ptr(dstate_in), _ptr(dinit_state), _stream(stream, q)), "lasp_bwd")
+
+
+def lasp_fwd_states(k, v, decay, C, state_cache, total=None, stream=None):
+    """First part of lasp_fwd: its states into state_cache and, if given, their
+    decayed total (the LASP-2 shard state). See lasp.h."""
+    B, N, H, d, dt = _tokens(k, v)
+    _check(_load().lasp_fwd_states(_ptr(k), _ptr(v), _ptr(decay), B, H, N, d, C, dt, _ptr(state_cache), _ptr(total),
+                                   _stream(stream, k)), "lasp_fwd_states")
+
+
+def lasp_fwd_finish(q, k, v, decay, o, C, state_cache, init_state=None, stream=None):
+    """Rest of lasp_fwd on a cache lasp_fwd_states filled: prefix from init_state, output. See lasp.h."""
+    B, N, H, d, dt = _tokens(q, k, v, o)
+    _check(_load().lasp_fwd_finish(_ptr(q), _ptr(k), _ptr(v), _ptr(decay), _ptr(o), B, H, N, d, C, dt,
+                                   _ptr(state_cache), _ptr(init_state), _stream(stream, q)), "lasp_fwd_finish")
+
+
+def lasp_bwd_states(q, dout, decay, C, dstate_ws, total=None, stream=None):
+    """First part of lasp_bwd: its gradient states into dstate_ws and, if given,
+    their decayed total (the LASP-2 shard gradient state). See lasp.h."""
+    B, N, H, d, dt = _tokens(q, dout)
+    _check(_load().lasp_bwd_states(_ptr(q), _ptr(dout), _ptr(decay), B, H, N, d, C, dt, _ptr(dstate_ws), _ptr(total),
+                                   _stream(stream, q)), "lasp_bwd_states")
+
+
+def lasp_bwd_finish(q, k, v, decay, dout, dq, dk, dv, C, state_cache, dstate_ws, dstate_in=None, dinit_state=None,
+                    stream=None):
+    """Rest of lasp_bwd on a workspace lasp_bwd_states filled: suffix from dstate_in, dq, dk, dv. See lasp.h."""
+    B, N, H, d, dt = _tokens(q, k, v, dout, dq, dk, dv)
+    _check(_load().lasp_bwd_finish(_ptr(q), _ptr(k), _ptr(v), _ptr(decay), _ptr(dout), _ptr(dq), _ptr(dk), _ptr(dv),
+                                   B, H, N, d, C, dt, _ptr(state_cache), _ptr(dstate_ws), _ptr(dstate_in),
+                                   _ptr(dinit_state), _stream(stream, q)), "lasp_bwd_finish")
 
 
 def lasp_bwd_noalloc(q, k, v, decay, dout, dq, dk, dv, C, state_cache, dstate_in=None, dinit_state=None,

@@ -16,7 +16,9 @@
 // keeping up to 2 * kUnroll * 16 bytes in flight per thread. Consecutive threads own consecutive
 // float4s of one state, so every warp access is a fully coalesced 512-byte run.
 // M and P may be the same array: each element is loaded before it is stored,
-// by the same thread.
+// by the same thread. With P = NULL only the total is written (the LASP-2
+// shard state): the states are then read with plain loads, so that a step that
+// scans them again soon after finds them in L2.
 #include "kernels.h"
 #include "lasp_common.cuh"
 
@@ -72,12 +74,14 @@ __global__ void __launch_bounds__(kThreads) state_scan_kernel(const float4* M, f
   // software pipeline: the loads of group g + 1 are issued before group g is
   // scanned and stored, so a group's worth of loads is always in flight
   const int ngroups = T / kUnroll;
+  const bool write = P != nullptr;
+  auto ld = [&](int64_t i) { return write ? __ldcs(M + i) : __ldg(M + i); };
   float4 cur[kUnroll];
   float gc[kUnroll];
   if (ngroups > 0) {
 #pragma unroll
     for (int u = 0; u < kUnroll; ++u) {
-      cur[u] = __ldcs(M + off + u * step);
+      cur[u] = ld(off + u * step);
       if (kGated) gc[u] = gsum[goff + u * gstep];
     }
   }
@@ -88,13 +92,13 @@ __global__ void __launch_bounds__(kThreads) state_scan_kernel(const float4* M, f
     if (more) {
 #pragma unroll
       for (int u = 0; u < kUnroll; ++u) {
-        nxt[u] = __ldcs(M + off + (kUnroll + u) * step);
+        nxt[u] = ld(off + (kUnroll + u) * step);
         if (kGated) gn[u] = gsum[goff + (kUnroll + u) * gstep];
       }
     }
 #pragma unroll
     for (int u = 0; u < kUnroll; ++u) {
-      st_keep(P + off + u * step, acc, keep);
+      if (write) st_keep(P + off + u * step, acc, keep);
       acc = fma4(kGated ? exp2f(gc[u] * kLog2e) : g, acc, cur[u]);
     }
     off += kUnroll * step;
@@ -109,8 +113,8 @@ __global__ void __launch_bounds__(kThreads) state_scan_kernel(const float4* M, f
   }
   int n = ngroups * kUnroll;
   for (; n < T; ++n) {
-    float4 m = __ldcs(M + off);
-    st_keep(P + off, acc, keep);
+    float4 m = ld(off);
+    if (write) st_keep(P + off, acc, keep);
     acc = fma4(kGated ? exp2f(gsum[goff] * kLog2e) : g, acc, m);
     off += step;
     goff += gstep;

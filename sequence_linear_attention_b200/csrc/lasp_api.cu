@@ -39,6 +39,7 @@ enum KernelId : int {
   K_GLA_STATES_TC = 19,  // gated form on the tensor cores: states
   K_GLA_OUT_TC = 20,     // gated form on the tensor cores: output
   K_GLA_BWD_TC = 21,     // gated form on the tensor cores: gradients
+  K_STATE_TOTAL = 22,    // decayed total of a sequence's states (the LASP-2 shard state)
   K_COUNT
 };
 
@@ -137,6 +138,109 @@ int chunk_grads_impl(const void* q, const void* k, const void* v, const void* do
       K_BWD_SIMT, st, [&] { return simt_chunk_bwd(q, k, v, dout, decay, P, R, dq, dk, dv, B, H, N, d, C, dtype, st); }));
 }
 
+// lasp_fwd in two parts. States: the chunk (or, on the walk path, segment)
+// states into the cache and, if total is non-NULL, their decayed total with a
+// zero start. Finish: the prefix from init and the output.
+int fwd_states_impl(const void* k, const void* v, const float* decay, int B, int H, int64_t N, int d, int C,
+                    int dtype, float* state_cache, float* total, cudaStream_t st) {
+  const int T = (int)(N / C);
+  int s;
+  if (tc_fwd_walk_ok(dtype, d, C, N)) {
+    // segments of G tokens: their states go to the slots of their first chunks
+    const int G = walk_segment_tokens(N, C);
+    const int stride = G / C;
+    if ((s = cuda_status(traced(K_SEG_STATES, st, [&] {
+           return tc_chunk_states_slots(k, v, decay, state_cache, B, H, N, d, G, 0, T, stride, 0, st);
+         }))))
+      return s;
+    if (!total) return LASP_OK;
+    return cuda_status(traced(K_STATE_TOTAL, st, [&] {
+      return launch_state_scan_slots(state_cache, nullptr, decay, nullptr, total, B, (int)(N / G), H, d, G, 0, T,
+                                     stride, 0, st);
+    }));
+  }
+  if ((s = chunk_states_impl(k, v, decay, state_cache, B, H, N, d, C, dtype, 0, st))) return s;
+  return total ? scan_impl(K_STATE_TOTAL, state_cache, nullptr, decay, nullptr, total, B, T, H, d, C, 0, st) : LASP_OK;
+}
+
+int fwd_finish_impl(const void* q, const void* k, const void* v, const float* decay, void* o, int B, int H, int64_t N,
+                    int d, int C, int dtype, float* state_cache, const float* init_state, cudaStream_t st) {
+  const int T = (int)(N / C);
+  int s;
+  if (tc_fwd_walk_ok(dtype, d, C, N)) {
+    // the exclusive prefix over segments turns their states into P of their
+    // first chunks, and the walk carries the state through each segment,
+    // filling the other slots
+    const int G = walk_segment_tokens(N, C);
+    const int stride = G / C;
+    if ((s = cuda_status(traced(K_SEG_SCAN, st, [&] {
+           return launch_state_scan_slots(state_cache, state_cache, decay, init_state, nullptr, B, (int)(N / G), H, d,
+                                          G, 0, T, stride, 0, st);
+         }))))
+      return s;
+    const int sms = num_sms_current_device();
+    return cuda_status(traced(K_FWD_WALK, st, [&] {
+      return tc_fwd_walk(q, k, v, decay, state_cache, o, B, H, N, d, C, G, sms, st);
+    }));
+  }
+  // exclusive prefix in place -> P_c; then the output
+  if ((s = scan_impl(K_SCAN, state_cache, state_cache, decay, init_state, nullptr, B, T, H, d, C, 0, st))) return s;
+  return chunk_out_impl(q, k, v, decay, state_cache, o, B, H, N, d, C, dtype, st);
+}
+
+// lasp_bwd in two parts. States: the gradient chunk (or segment) states into
+// the workspace and, if total is non-NULL, their decayed total with nothing
+// entering from after the sequence. Finish: the suffix from dstate_in (and
+// dinit) and dQ, dK, dV.
+int bwd_states_impl(const void* q, const void* dout, const float* decay, int B, int H, int64_t N, int d, int C,
+                    int dtype, float* dstate_ws, float* total, cudaStream_t st) {
+  const int T = (int)(N / C);
+  int s;
+  if (tc_bwd_walk_ok(dtype, d, C, N)) {
+    // segments of G tokens: their gradient states go to the slots of their last chunks
+    const int G = walk_segment_tokens(N, C);
+    const int stride = G / C;
+    if ((s = cuda_status(traced(K_SEG_STATES, st, [&] {
+           return tc_chunk_states_slots(q, dout, decay, dstate_ws, B, H, N, d, G, 1, T, stride, stride - 1, st);
+         }))))
+      return s;
+    if (!total) return LASP_OK;
+    return cuda_status(traced(K_STATE_TOTAL, st, [&] {
+      return launch_state_scan_slots(dstate_ws, nullptr, decay, nullptr, total, B, (int)(N / G), H, d, G, 1, T,
+                                     stride, stride - 1, st);
+    }));
+  }
+  if ((s = chunk_states_impl(q, dout, decay, dstate_ws, B, H, N, d, C, dtype, 1, st))) return s;
+  return total ? scan_impl(K_STATE_TOTAL, dstate_ws, nullptr, decay, nullptr, total, B, T, H, d, C, 1, st) : LASP_OK;
+}
+
+int bwd_finish_impl(const void* q, const void* k, const void* v, const float* decay, const void* dout, void* dq,
+                    void* dk, void* dv, int B, int H, int64_t N, int d, int C, int dtype, const float* state_cache,
+                    float* dstate_ws, const float* dstate_in, float* dinit_state, cudaStream_t st) {
+  const int T = (int)(N / C);
+  int s;
+  if (tc_bwd_walk_ok(dtype, d, C, N)) {
+    // the exclusive suffix over segments turns their gradient states into R of
+    // their last chunks (and gives dinit), and the walk carries R backward
+    // through each segment
+    const int G = walk_segment_tokens(N, C);
+    const int stride = G / C;
+    if ((s = cuda_status(traced(K_SEG_SCAN, st, [&] {
+           return launch_state_scan_slots(dstate_ws, dstate_ws, decay, dstate_in, dinit_state, B, (int)(N / G), H, d,
+                                          G, 1, T, stride, stride - 1, st);
+         }))))
+      return s;
+    const int sms = num_sms_current_device();
+    return cuda_status(traced(K_BWD_WALK, st, [&] {
+      return tc_bwd_walk(q, k, v, dout, decay, state_cache, dstate_ws, dq, dk, dv, B, H, N, d, C, G, sms, st);
+    }));
+  }
+  // exclusive suffix in place -> R_c (and dinit); then dQ, dK, dV
+  if ((s = scan_impl(K_SCAN, dstate_ws, dstate_ws, decay, dstate_in, dinit_state, B, T, H, d, C, 1, st))) return s;
+  return chunk_grads_impl(q, k, v, dout, decay, state_cache, dstate_ws, dq, dk, dv, B, H, N, d, C, dtype, st);
+}
+
+
 }  // namespace api_detail
 }  // namespace lasp
 
@@ -194,6 +298,29 @@ int lasp_state_prefix(const float* M, float* Mprefix, const float* decay, const 
   return scan_impl(K_SCAN, M, Mprefix, decay, init, total, B, T, H, d, C, reverse, (cudaStream_t)stream);
 }
 
+int lasp_fwd_states(const void* k, const void* v, const float* decay, int B, int H, int64_t N, int d, int C,
+                    int dtype, float* state_cache, float* total, void* stream) {
+  int s = check_sizes(B, H, N, d, C, dtype);
+  if (s) return s;
+  if (N == 0) {
+    if ((s = check_ptrs({}, {decay, total}))) return s;
+    return total ? scan_impl(K_STATE_TOTAL, nullptr, nullptr, decay, nullptr, total, B, 0, H, d, C, 0,
+                             (cudaStream_t)stream)
+                 : LASP_OK;
+  }
+  if ((s = check_ptrs({k, v, state_cache}, {decay, total}))) return s;
+  return fwd_states_impl(k, v, decay, B, H, N, d, C, dtype, state_cache, total, (cudaStream_t)stream);
+}
+
+int lasp_fwd_finish(const void* q, const void* k, const void* v, const float* decay, void* o, int B, int H,
+                    int64_t N, int d, int C, int dtype, float* state_cache, const float* init_state, void* stream) {
+  int s = check_sizes(B, H, N, d, C, dtype);
+  if (s) return s;
+  if (N == 0) return LASP_OK;
+  if ((s = check_ptrs({q, k, v, o, state_cache}, {decay, init_state}))) return s;
+  return fwd_finish_impl(q, k, v, decay, o, B, H, N, d, C, dtype, state_cache, init_state, (cudaStream_t)stream);
+}
+
 int lasp_fwd(const void* q, const void* k, const void* v, const float* decay, void* o, int B, int H, int64_t N,
              int d, int C, int dtype, float* state_cache, const float* init_state, void* stream) {
   int s = check_sizes(B, H, N, d, C, dtype);
@@ -201,31 +328,8 @@ int lasp_fwd(const void* q, const void* k, const void* v, const float* decay, vo
   if (N == 0) return LASP_OK;
   if ((s = check_ptrs({q, k, v, o, state_cache}, {decay, init_state}))) return s;
   cudaStream_t st = (cudaStream_t)stream;
-  const int T = (int)(N / C);
-  if (tc_fwd_walk_ok(dtype, d, C, N)) {
-    // segments of G tokens: their states go to the slots of their first chunks,
-    // the exclusive prefix over segments turns them into P of those chunks, and
-    // the walk carries the state through each segment, filling the other slots
-    const int G = walk_segment_tokens(N, C);
-    const int stride = G / C;
-    if ((s = cuda_status(traced(K_SEG_STATES, st, [&] {
-           return tc_chunk_states_slots(k, v, decay, state_cache, B, H, N, d, G, 0, T, stride, 0, st);
-         }))))
-      return s;
-    if ((s = cuda_status(traced(K_SEG_SCAN, st, [&] {
-           return launch_state_scan_slots(state_cache, state_cache, decay, init_state, nullptr, B, (int)(N / G), H, d,
-                                          G, 0, T, stride, 0, st);
-         }))))
-      return s;
-    const int sms = num_sms_current_device();
-    return cuda_status(traced(K_FWD_WALK, st, [&] {
-      return tc_fwd_walk(q, k, v, decay, state_cache, o, B, H, N, d, C, G, sms, st);
-    }));
-  }
-  // 1. chunk states M_c into the cache; 2. exclusive prefix in place -> P_c; 3. output.
-  if ((s = chunk_states_impl(k, v, decay, state_cache, B, H, N, d, C, dtype, 0, st))) return s;
-  if ((s = scan_impl(K_SCAN, state_cache, state_cache, decay, init_state, nullptr, B, T, H, d, C, 0, st))) return s;
-  return chunk_out_impl(q, k, v, decay, state_cache, o, B, H, N, d, C, dtype, st);
+  if ((s = fwd_states_impl(k, v, decay, B, H, N, d, C, dtype, state_cache, nullptr, st))) return s;
+  return fwd_finish_impl(q, k, v, decay, o, B, H, N, d, C, dtype, state_cache, init_state, st);
 }
 
 int lasp_chunk_out(const void* q, const void* k, const void* v, const float* decay, const float* P, void* o, int B,
@@ -247,6 +351,32 @@ int lasp_chunk_grads(const void* q, const void* k, const void* v, const void* do
   return chunk_grads_impl(q, k, v, dout, decay, P, R, dq, dk, dv, B, H, N, d, C, dtype, (cudaStream_t)stream);
 }
 
+int lasp_bwd_states(const void* q, const void* dout, const float* decay, int B, int H, int64_t N, int d, int C,
+                    int dtype, float* dstate_ws, float* total, void* stream) {
+  int s = check_sizes(B, H, N, d, C, dtype);
+  if (s) return s;
+  if (N == 0) {
+    if ((s = check_ptrs({}, {decay, total}))) return s;
+    return total ? scan_impl(K_STATE_TOTAL, nullptr, nullptr, decay, nullptr, total, B, 0, H, d, C, 1,
+                             (cudaStream_t)stream)
+                 : LASP_OK;
+  }
+  if ((s = check_ptrs({q, dout, dstate_ws}, {decay, total}))) return s;
+  return bwd_states_impl(q, dout, decay, B, H, N, d, C, dtype, dstate_ws, total, (cudaStream_t)stream);
+}
+
+int lasp_bwd_finish(const void* q, const void* k, const void* v, const float* decay, const void* dout, void* dq,
+                    void* dk, void* dv, int B, int H, int64_t N, int d, int C, int dtype, const float* state_cache,
+                    float* dstate_ws, const float* dstate_in, float* dinit_state, void* stream) {
+  int s = check_sizes(B, H, N, d, C, dtype);
+  if (s) return s;
+  if (N == 0) return LASP_OK;
+  if ((s = check_ptrs({q, k, v, dout, dq, dk, dv, state_cache, dstate_ws}, {decay, dstate_in, dinit_state})))
+    return s;
+  return bwd_finish_impl(q, k, v, decay, dout, dq, dk, dv, B, H, N, d, C, dtype, state_cache, dstate_ws, dstate_in,
+                         dinit_state, (cudaStream_t)stream);
+}
+
 int lasp_bwd(const void* q, const void* k, const void* v, const float* decay, const void* dout, void* dq, void* dk,
              void* dv, int B, int H, int64_t N, int d, int C, int dtype, const float* state_cache, float* dstate_ws,
              const float* init_state, const float* dstate_in, float* dinit_state, void* stream) {
@@ -257,32 +387,9 @@ int lasp_bwd(const void* q, const void* k, const void* v, const float* decay, co
   if ((s = check_ptrs({q, k, v, dout, dq, dk, dv, state_cache, dstate_ws}, {decay, init_state, dstate_in, dinit_state})))
     return s;
   cudaStream_t st = (cudaStream_t)stream;
-  const int T = (int)(N / C);
-  if (tc_bwd_walk_ok(dtype, d, C, N)) {
-    // segments of G tokens: their gradient states go to the slots of their last
-    // chunks, the exclusive suffix over segments turns them into R of those
-    // chunks (and gives dinit), and the walk carries R backward through each
-    // segment, filling the other slots
-    const int G = walk_segment_tokens(N, C);
-    const int stride = G / C;
-    if ((s = cuda_status(traced(K_SEG_STATES, st, [&] {
-           return tc_chunk_states_slots(q, dout, decay, dstate_ws, B, H, N, d, G, 1, T, stride, stride - 1, st);
-         }))))
-      return s;
-    if ((s = cuda_status(traced(K_SEG_SCAN, st, [&] {
-           return launch_state_scan_slots(dstate_ws, dstate_ws, decay, dstate_in, dinit_state, B, (int)(N / G), H, d,
-                                          G, 1, T, stride, stride - 1, st);
-         }))))
-      return s;
-    const int sms = num_sms_current_device();
-    return cuda_status(traced(K_BWD_WALK, st, [&] {
-      return tc_bwd_walk(q, k, v, dout, decay, state_cache, dstate_ws, dq, dk, dv, B, H, N, d, C, G, sms, st);
-    }));
-  }
-  // 1. gradient chunk states dM_c; 2. exclusive suffix in place -> R_c; 3. dQ, dK, dV.
-  if ((s = chunk_states_impl(q, dout, decay, dstate_ws, B, H, N, d, C, dtype, 1, st))) return s;
-  if ((s = scan_impl(K_SCAN, dstate_ws, dstate_ws, decay, dstate_in, dinit_state, B, T, H, d, C, 1, st))) return s;
-  return chunk_grads_impl(q, k, v, dout, decay, state_cache, dstate_ws, dq, dk, dv, B, H, N, d, C, dtype, st);
+  if ((s = bwd_states_impl(q, dout, decay, B, H, N, d, C, dtype, dstate_ws, nullptr, st))) return s;
+  return bwd_finish_impl(q, k, v, decay, dout, dq, dk, dv, B, H, N, d, C, dtype, state_cache, dstate_ws, dstate_in,
+                         dinit_state, st);
 }
 
 int lasp_check_device_status(void* stream, int* site) {
@@ -352,6 +459,7 @@ const char* lasp_kernel_name(int id) {
     case K_GLA_STATES_TC: return "gla_states_tc";
     case K_GLA_OUT_TC: return "gla_out_tc";
     case K_GLA_BWD_TC: return "gla_bwd_tc";
+    case K_STATE_TOTAL: return "state_total";
     default: return "unknown";
   }
 }

@@ -75,6 +75,49 @@ def draw_tensor(seed: int, index: int, shape, scale: float, bf16: bool, threads:
     return out.reshape(shape)
 
 
+def draw_tensor_rows(seed: int, index: int, shape, scale: float, bf16: bool, row0: int, rows: int):
+    """Rows row0 .. row0 + rows - 1 (axis 1) of the [B, N, H, d] tensor that
+    :func:`draw_tensor` draws for the same arguments, drawing only the blocks
+    that hold them (a shard of a long sequence without the rest of it)."""
+    B, N, H, d = shape
+    n = B * N * H * d
+    stream = np.random.SeedSequence(seed).spawn(len(_NAMES))[index]
+    children = stream.spawn((n + _BLOCK - 1) // _BLOCK)
+    row = H * d
+    out = np.empty((B, rows * row), np.uint16 if bf16 else np.float32)
+
+    def part(b, i, lo, hi):
+        m = min(_BLOCK, n - i * _BLOCK)
+        blk = np.empty(m, out.dtype)
+        _draw(children[i], m, scale, bf16, blk, 0)
+        a, z = max(lo, i * _BLOCK), min(hi, i * _BLOCK + m)
+        out[b, a - lo:z - lo] = blk[a - i * _BLOCK:z - i * _BLOCK]
+
+    with ThreadPoolExecutor(max_workers=min(32, os.cpu_count() or 1)) as ex:
+        futs = []
+        for b in range(B):
+            lo, hi = (b * N + row0) * row, (b * N + row0 + rows) * row
+            futs += [ex.submit(part, b, i, lo, hi) for i in range(lo // _BLOCK, (hi + _BLOCK - 1) // _BLOCK)]
+        for f in futs:
+            f.result()
+    return out.reshape(B, rows, H, d)
+
+
+def make_shard_inputs(B: int, N: int, H: int, d: int, seed: int, row0: int, rows: int, bf16: bool = True,
+                      decayed: bool = True, with_grad: bool = True) -> dict:
+    """:func:`make_inputs` restricted to the token rows row0 .. row0 + rows - 1
+    of every sequence (one rank's shard in sequence parallelism)."""
+    out = {}
+    for i, name in enumerate(_NAMES):
+        if name == "do" and not with_grad:
+            continue
+        scale = 1.0 if name == "do" else float(d) ** -0.5
+        out[name] = draw_tensor_rows(seed, i, (B, N, H, d), scale, bf16, row0, rows)
+    out["lam"] = decay_rates(H) if decayed else None
+    out["bf16"] = bf16
+    return out
+
+
 def make_log_gates(B: int, N: int, H: int, d: int, seed: int, tau: float = 16.0) -> np.ndarray:
     """Log-gates log(sigmoid(x)) / tau, float32 [B, N, H, d], x from stream 4 of ``seed``."""
     shape = (B, N, H, d)

@@ -6,23 +6,27 @@ of d x d states per direction (LASP-2, "The reading" and its backward pass):
 
 forward
   1. the shard's memory state, M_r = sum_j lambda^{L-1-j} k_j^T v_j
-     (LASP Eq. 10 with the shard as one chunk);
+     (LASP Eq. 10 with the shard as one chunk): the first part of the
+     single-device forward, whose segment states it sums with their decays;
   2. AllGather of M_0 .. M_{W-1};
   3. the state entering the shard, by the decayed prefix over the shards
      before it: E_0 = the sequence's initial state, E_r = lambda^L E_{r-1} + M_{r-1};
-  4. the single-device forward of the shard with E_r as its initial state.
+  4. the rest of the single-device forward of the shard (its prefix over the
+     segment states already in the cache, then the output) from E_r.
 
 backward
   1. the shard's gradient state, dM_r = sum_j lambda^{j+1} q_j^T do_j
-     (LASP Eq. 20 with the shard as one chunk);
+     (LASP Eq. 20 with the shard as one chunk), likewise the first part of the
+     single-device backward;
   2. AllGather of dM_0 .. dM_{W-1};
   3. the gradient state entering the shard's last token from the shards after
      it, by the decayed suffix: G_{W-1} = the gradient w.r.t. the sequence's
      final state, G_r = lambda^L G_{r+1} + dM_{r+1};
-  4. the single-device backward of the shard with G_r as its incoming
-     gradient state.
+  4. the rest of the single-device backward of the shard from G_r.
 
-The scans over the W gathered states run in the library's scan kernel (the
+No state is computed twice: the segment states stay in the state cache
+(forward) or the gradient-state workspace (backward) for the second part. The
+scans over the W gathered states run in the library's scan kernel (the
 gathered [W, B, H, d, d] array is the [1, W, B*H, d, d] chunk-state array of
 one sequence whose B*H "heads" carry the decays of the H heads B times). All
 arithmetic runs in the library's kernels; torch.distributed moves the states.
@@ -39,21 +43,24 @@ from __future__ import annotations
 import torch
 import torch.distributed as dist
 
-from . import lasp_bwd, lasp_chunk_dstates, lasp_chunk_states, lasp_fwd, lasp_state_prefix
+from . import lasp_bwd_finish, lasp_bwd_states, lasp_fwd_finish, lasp_fwd_states, lasp_state_prefix
 
 __all__ = ["DeviceKernels", "lasp2_fwd", "lasp2_bwd"]
 
 
 class DeviceKernels:
-    """The library's kernels, through its C ABI, in the shape this module calls them."""
+    """The library's kernels, through its C ABI, in the shape this module calls
+    them. The shard states are the first parts of the single-device forward and
+    backward calls (their segment states, in the cache or workspace, and the
+    decayed total); the rest of those calls reuses the segment states."""
 
     @staticmethod
-    def shard_state(k, v, decay, M, L):
-        lasp_chunk_states(None, k, v, decay, M, L)
+    def shard_state(k, v, decay, M, C, state_cache):
+        lasp_fwd_states(k, v, decay, C, state_cache, total=M)
 
     @staticmethod
-    def shard_dstate(q, dout, decay, dM, L):
-        lasp_chunk_dstates(q, dout, decay, dM, L)
+    def shard_dstate(q, dout, decay, dM, C, dstate_ws):
+        lasp_bwd_states(q, dout, decay, C, dstate_ws, total=dM)
 
     @staticmethod
     def state_prefix(M, out, decay, L, init, total, reverse):
@@ -61,11 +68,11 @@ class DeviceKernels:
 
     @staticmethod
     def fwd(q, k, v, decay, o, C, state_cache, init_state):
-        lasp_fwd(q, k, v, decay, o, C, state_cache, init_state=init_state)
+        lasp_fwd_finish(q, k, v, decay, o, C, state_cache, init_state=init_state)
 
     @staticmethod
     def bwd(q, k, v, decay, dout, dq, dk, dv, C, state_cache, dstate_ws, dstate_in):
-        lasp_bwd(q, k, v, decay, dout, dq, dk, dv, C, state_cache, dstate_ws, dstate_in=dstate_in)
+        lasp_bwd_finish(q, k, v, decay, dout, dq, dk, dv, C, state_cache, dstate_ws, dstate_in=dstate_in)
 
 
 def _group_shape(x, group):
@@ -126,7 +133,7 @@ def lasp2_fwd(q, k, v, decay, o, C, state_cache, init_state=None, final_state=No
     _check_state(init_state, B, H, d, q, "init_state")
     _check_state(final_state, B, H, d, q, "final_state")
     M = torch.empty((B, 1, H, d, d), dtype=torch.float32, device=q.device)
-    kern.shard_state(k, v, decay, M, L)
+    kern.shard_state(k, v, decay, M.view(B, H, d, d), C, state_cache)
     gathered = torch.empty((W, B, H, d, d), dtype=torch.float32, device=q.device)
     _all_gather(gathered, M.view(B, H, d, d), group)
     entering = _scan_over_shards(kern, gathered, decay, L, init_state, final_state, False)[r]
@@ -151,7 +158,7 @@ def lasp2_bwd(q, k, v, decay, dout, dq, dk, dv, C, state_cache, dstate_ws, dstat
     _check_state(dstate_in, B, H, d, q, "dstate_in")
     _check_state(dinit_state, B, H, d, q, "dinit_state")
     dM = torch.empty((B, 1, H, d, d), dtype=torch.float32, device=q.device)
-    kern.shard_dstate(q, dout, decay, dM, L)
+    kern.shard_dstate(q, dout, decay, dM.view(B, H, d, d), C, dstate_ws)
     gathered = torch.empty((W, B, H, d, d), dtype=torch.float32, device=q.device)
     _all_gather(gathered, dM.view(B, H, d, d), group)
     incoming = _scan_over_shards(kern, gathered, decay, L, dstate_in, dinit_state, True)[r]

@@ -160,3 +160,18 @@ def test_gated_calls_reject_bad_arguments(lib):
     assert p(None, None, None, None, None, 1, 0, 2, 64, 0, None) == OK                 # T = 0, no total
     assert lasp.lasp_gla_cache_floats(2, 3, 512, 64, 64) == 2 * 8 * 3 * 64 * 65
     assert lasp.lasp_gla_cache_floats(2, 3, 512, 64, 256) == -1
+
+
+def test_split_calls_reject_bad_arguments(lib):
+    fs, ff = lib.lasp_fwd_states, lib.lasp_fwd_finish
+    assert fs(A, A, None, 1, 2, 512, 96, 64, BF16, A, None, None) == UNSUPPORTED         # d = 96
+    assert fs(A, A, None, 1, 2, 500, 64, 64, BF16, A, None, None) == INVALID             # C does not divide N
+    assert fs(A, A, None, 1, 2, 512, 64, 64, F32, None, None, None) == INVALID           # no cache
+    assert fs(A, A, None, 1, 2, 512, 64, 64, F32, A, A + 4, None) == MISALIGNED          # total
+    assert fs(None, None, None, 1, 2, 0, 64, 64, F32, None, None, None) == OK            # nothing to do
+    assert ff(A, A, A, None, None, 1, 2, 512, 64, 64, F32, A, None, None) == INVALID     # no output
+    assert ff(A, A, A, None, A, 1, 2, 0, 64, 64, F32, None, None, None) == OK
+    bs, bf = lib.lasp_bwd_states, lib.lasp_bwd_finish
+    assert bs(A, None, None, 1, 2, 512, 64, 64, F32, A, None, None) == INVALID           # no dout
+    assert bf(A, A, A, None, A, A, A, A, 1, 2, 512, 64, 64, F32, A, None, None, None, None) == INVALID  # no ws
+    assert bf(A, A, A, None, A, A, A, A, 1, 2, 512, 64, 64, F32, A, A, A + 4, None, None) == MISALIGNED

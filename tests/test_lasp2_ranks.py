@@ -50,16 +50,18 @@ class _OracleKernels:
         return None if decay is None else decay.double().numpy()
 
     @classmethod
-    def shard_state(cls, k, v, decay, M, L):
+    def shard_state(cls, k, v, decay, M, C, scratch):
         import oracle
         import torch
-        M.copy_(torch.from_numpy(oracle.chunk_states(k.numpy(), v.numpy(), cls._lam(decay), L, 0)))
+        L = k.shape[1]
+        M.copy_(torch.from_numpy(oracle.chunk_states(k.numpy(), v.numpy(), cls._lam(decay), L, 0)[:, 0]))
 
     @classmethod
-    def shard_dstate(cls, q, dout, decay, dM, L):
+    def shard_dstate(cls, q, dout, decay, dM, C, scratch):
         import oracle
         import torch
-        dM.copy_(torch.from_numpy(oracle.chunk_states(q.numpy(), dout.numpy(), cls._lam(decay), L, 1)))
+        L = q.shape[1]
+        dM.copy_(torch.from_numpy(oracle.chunk_states(q.numpy(), dout.numpy(), cls._lam(decay), L, 1)[:, 0]))
 
     @classmethod
     def state_prefix(cls, M, out, decay, L, init, total, reverse):
