@@ -1,6 +1,7 @@
 // Tensor-core kernels of the gated form (a decay per token and key feature;
 // LASP Appendix A.4, Eq. 24 with the GLA / GateLoop row of Table 5), bf16,
-// d = 128, one 128-token tile per CTA. A tile spans 128/C chunks (C dividing
+// d = 128, over 128-token tiles (one per CTA; the backward's persistent CTAs
+// take one after another). A tile spans 128/C chunks (C dividing
 // 128); its masked products regroup the per-chunk intra and inter terms, so it
 // follows the chunk equations of k_gla_simt.cu with the tile as the chunk
 // (b_t = inclusive cumulative log-gate from the tile start, b_end its last
@@ -478,7 +479,9 @@ struct SmemBwd {
   float bnd[kD];     // e^{b_end[i]} <R_c[i], P_c[i]>
 };
 
-// One 128-token tile per CTA. Shared memory: Q^, K^, V, dO (then, in pairs,
+// One persistent CTA per SM, taking 128-token tiles in launch order (tile w,
+// w + grid, ...); the barriers complete once per tile, so their parity flips
+// from tile to tile. Shared memory: Q^, K^, V, dO (then, in pairs,
 // the fp32 tiles of dB and k . dk^inter for the log-gate gradient's column
 // sums), X (P', then R'; r and b_end - r during the gate walk), and the pair
 // sA / sB (the gate tile during the walk; then dA . strict and A . causal;
