@@ -329,7 +329,7 @@ __global__ void __launch_bounds__(kThreads, 1) gla_out_tc(const __grid_constant_
                                                           const __grid_constant__ CUtensorMap map_o,
                                                           const __grid_constant__ CUtensorMap map_g,
                                                           const float* __restrict__ P, int H, int64_t N,
-                                                          int64_t t_slots, int stride) {
+                                                          int64_t t_slots, int stride, int ntx, int64_t ntiles) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   uint8_t* sQ = base;                   // Q^
@@ -339,11 +339,27 @@ __global__ void __launch_bounds__(kThreads, 1) gla_out_tc(const __grid_constant_
   uint8_t* sA = base + 4 * kTileBytes;  // A . causal, then O out
   float* bt = reinterpret_cast<float*>(base + 5 * kTileBytes);  // gate tile, 64 KB
   SmemOut* s = reinterpret_cast<SmemOut*>(base + 7 * kTileBytes);
-  const int c = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int t = (warp & 3) * 32 + lane, half = warp >> 2;
-  const int64_t row0 = (int64_t)c * kTile;
-  const float* Pc = P + (((int64_t)b * t_slots + (int64_t)c * stride) * H + h) * kD * kD;  // P of the tile's first chunk
+  // tile w: 128 tokens c * 128.. of head h of sequence b, in launch order
+  auto tile_of = [&](int64_t w, int& c, int& h, int& b) {
+    c = (int)(w % ntx);
+    h = (int)((w / ntx) % H);
+    b = (int)(w / ((int64_t)ntx * H));
+  };
+  // P of a tile's first chunk
+  auto state_of = [&](int c, int h, int b) {
+    return P + (((int64_t)b * t_slots + (int64_t)c * stride) * H + h) * kD * kD;
+  };
+  auto load_tokens = [&](int h, int row, int b) {
+    mbar_arrive_expect_tx(&s->load, 3 * kTileBytes);
+    tma_load_4d(sQ, &map_q, &s->load, 0, h, row, b);
+    tma_load_4d(sQ + kBox, &map_q, &s->load, 64, h, row, b);
+    tma_load_4d(sK, &map_k, &s->load, 0, h, row, b);
+    tma_load_4d(sK + kBox, &map_k, &s->load, 64, h, row, b);
+    tma_load_4d(sV, &map_v, &s->load, 0, h, row, b);
+    tma_load_4d(sV + kBox, &map_v, &s->load, 64, h, row, b);
+  };
   if (tid == 0) {
     prefetch_tmap(&map_q);
     prefetch_tmap(&map_k);
@@ -367,19 +383,26 @@ __global__ void __launch_bounds__(kThreads, 1) gla_out_tc(const __grid_constant_
   const uint32_t tmem = s->tmem_base;
   const uint32_t lane_base = tmem + ((uint32_t)((warp & 3) * 32) << 16);
   const uint32_t T0 = 0, T1 = 128;
-  if (tid == 0) {
-    load_gate_tile(bt, &map_g, &s->gload, h, (int)row0, b);
-    bulk_prefetch_l2(Pc, kD * kD * 4);  // read with plain loads later
-    mbar_arrive_expect_tx(&s->load, 3 * kTileBytes);
-    tma_load_4d(sQ, &map_q, &s->load, 0, h, (int)row0, b);
-    tma_load_4d(sQ + kBox, &map_q, &s->load, 64, h, (int)row0, b);
-    tma_load_4d(sK, &map_k, &s->load, 0, h, (int)row0, b);
-    tma_load_4d(sK + kBox, &map_k, &s->load, 64, h, (int)row0, b);
-    tma_load_4d(sV, &map_v, &s->load, 0, h, (int)row0, b);
-    tma_load_4d(sV + kBox, &map_v, &s->load, 64, h, (int)row0, b);
+  if (tid == 0 && (int64_t)blockIdx.x < ntiles) {
+    // the first tile's loads; a later tile's are issued during the tile before
+    int c, h, b;
+    tile_of(blockIdx.x, c, h, b);
+    load_gate_tile(bt, &map_g, &s->gload, h, c * kTile, b);
+    bulk_prefetch_l2(state_of(c, h, b), kD * kD * 4);  // read with plain loads later
+    load_tokens(h, c * kTile, b);
   }
+  uint32_t ph = 0;            // parity of every barrier's phase for this CTA's current tile
+  bool gate_ahead = false;    // thread 0: the next tile's gate tile is in flight
+  bool tok_ahead = false;     // thread 0: the next tile's token tiles are in flight
+  for (int64_t w = blockIdx.x; w < ntiles; w += gridDim.x, ph ^= 1u) {
+  int c, h, b;
+  tile_of(w, c, h, b);
+  const int64_t row0 = (int64_t)c * kTile;
+  const float* Pc = state_of(c, h, b);
+  const int64_t wn = w + gridDim.x;  // this CTA's next tile
+  gate_ahead = tok_ahead = false;
   float x[64];
-  gate_rows(bt, &s->gload, 0, &s->abort, SITE_OUT_TMA, s->r, s->dend, tid, t, half, x);
+  gate_rows(bt, &s->gload, ph, &s->abort, SITE_OUT_TMA, s->r, s->dend, tid, t, half, x);
   // P' = diag(e^{r}) P_c into X
   {
     float w[16];
@@ -387,13 +410,21 @@ __global__ void __launch_bounds__(kThreads, 1) gla_out_tc(const __grid_constant_
     for (int u = 0; u < 16; ++u) w[u] = exp2f(s->r[warp + 8 * u] * kLog2e);
     load_scaled_state(sX, Pc, w, warp, lane);
   }
-  if (!mbar_wait(&s->load, 0, SITE_OUT_TMA)) s->abort = 1;
+  if (!mbar_wait(&s->load, ph, SITE_OUT_TMA)) s->abort = 1;
   scale_row_half(sQ, t, half, x, 1.f);   // Q^ = q . E
   scale_row_half(sK, t, half, x, -1.f);  // K^ = k / E
   fence_async_smem();
   tc_fence_before();
-  __syncthreads();
+  __syncthreads();  // every row of the gate tile has been read
   if (s->abort) goto cleanup;
+  if (tid == 0 && wn < ntiles) {
+    // the next tile's gates into the gate tile, its P into L2
+    int cn, hn, bn;
+    tile_of(wn, cn, hn, bn);
+    load_gate_tile(bt, &map_g, &s->gload, hn, cn * kTile, bn);
+    bulk_prefetch_l2(state_of(cn, hn, bn), kD * kD * 4);
+    gate_ahead = true;
+  }
   {
     const uint32_t aQ = smem_u32(sQ), aK = smem_u32(sK), aV = smem_u32(sV), aX = smem_u32(sX), aA = smem_u32(sA);
     constexpr uint32_t id_kk = idesc_bf16(128, 128, 0, 0);
@@ -406,7 +437,7 @@ __global__ void __launch_bounds__(kThreads, 1) gla_out_tc(const __grid_constant_
       for (int kk = 0; kk < kD / 16; ++kk) mma_bf16(tmem + T1, kmaj(aQ, kk), mnmaj(aX, kk), id_kn, kk != 0);
     }
     // A . causal -> sA (row t, column half)
-    if (mbar_wait(&s->mma1, 0, SITE_OUT_MMA)) {
+    if (mbar_wait(&s->mma1, ph, SITE_OUT_MMA)) {
       tc_fence_after();
 #pragma unroll 1
       for (int c2 = 0; c2 < 2; ++c2) {
@@ -436,8 +467,15 @@ __global__ void __launch_bounds__(kThreads, 1) gla_out_tc(const __grid_constant_
       mma_commit(&s->mma2);
     }
     // O -> sA (free once the MMA has read it) -> TMA store
-    if (mbar_wait(&s->mma2, 0, SITE_OUT_MMA)) {
+    if (mbar_wait(&s->mma2, ph, SITE_OUT_MMA)) {
       tc_fence_after();
+      if (tid == 0 && wn < ntiles) {
+        // every MMA has read Q^, K^, V and P': the next tile's tokens go in
+        int cn, hn, bn;
+        tile_of(wn, cn, hn, bn);
+        load_tokens(hn, cn * kTile, bn);
+        tok_ahead = true;
+      }
 #pragma unroll 1
       for (int c2 = 0; c2 < 2; ++c2) {
         const int col0 = half * 64 + c2 * 32;
@@ -457,14 +495,22 @@ __global__ void __launch_bounds__(kThreads, 1) gla_out_tc(const __grid_constant_
       s->abort = 1;
     }
     __syncthreads();
-    if (tid == 0 && !s->abort) {
+    const bool stop = s->abort != 0;
+    if (tid == 0 && !stop) {
       tma_store_4d(&map_o, sA, 0, h, (int)row0, b);
       tma_store_4d(&map_o, sA + kBox, 64, h, (int)row0, b);
       tma_store_commit();
-      tma_store_wait_read0();
+      tma_store_wait_read0();  // sA is free for the next tile's mask
     }
+    if (stop) goto cleanup;
   }
+  }
+  gate_ahead = tok_ahead = false;
 cleanup:
+  // loads issued for a next tile that an abort leaves unused land before the
+  // CTA exits (bounded waits)
+  if (tid == 0 && gate_ahead) mbar_wait(&s->gload, ph ^ 1u, SITE_OUT_TMA);
+  if (tid == 0 && tok_ahead) mbar_wait(&s->load, ph ^ 1u, SITE_OUT_TMA);
   tc_fence_before();
   __syncthreads();
   if (warp == 0) tmem_dealloc(tmem, 256);
@@ -956,8 +1002,15 @@ cudaError_t tc_gla_chunk_out(const void* q, const void* k, const void* v, const 
   const size_t smem = 1024 + 7 * (size_t)kTileBytes + sizeof(SmemOut);
   cudaError_t e = cudaFuncSetAttribute(gla_out_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  gla_out_tc<<<dim3((unsigned)(N / kTile), H, B), kThreads, smem, st>>>(mq, mk, mv, mo, mg, P, H, N, t_slots,
-                                                                       stride);
+  int dev = 0, sms = 0;
+  if ((e = cudaGetDevice(&dev)) != cudaSuccess ||
+      (e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
+    return e;
+  // one persistent CTA per SM (the kernel holds most of shared memory)
+  const int ntx = (int)(N / kTile);
+  const int64_t ntiles = (int64_t)B * H * ntx;
+  const unsigned grid = (unsigned)std::min<int64_t>(ntiles, sms);
+  gla_out_tc<<<grid, kThreads, smem, st>>>(mq, mk, mv, mo, mg, P, H, N, t_slots, stride, ntx, ntiles);
   return cudaGetLastError();
 }
 
