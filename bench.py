@@ -60,9 +60,14 @@ def algorithmic_bytes(name: str, tokens_heads: int, d: int, C: int, G: int, elem
     Gated form (a log-gate per token and key feature, fp32: 4d bytes):
       gla_states_*: read 2 token rows and the gates, write s/C         = 2de + 4d + s/C
       gla_scan:     read and write s/C, read the chunk's gate totals   = 2s/C + 4d/C
-      gla_out_*:    read q, k, v, the gates and P, write o             = 4de + 4d + s/C
-      gla_bwd_*:    read q, k, v, dO, the gates, P and R, write dq, dk,
+      gla_out_simt: read q, k, v, the gates and P, write o             = 4de + 4d + s/C
+      gla_bwd_simt: read q, k, v, dO, the gates, P and R, write dq, dk,
                     dv and the gate gradient                          = 7de + 8d + 2s/C
+      gla_out_tc:   per 128-token tile: read q, k, v, the gates and P
+                    (fp32), write o and the bf16 tile of diag(e^r) P over
+                    P's cache slot                       = 4de + 4d + s/128 + s/256
+      gla_bwd_tc:   read q, k, v, dO, the gates, that bf16 tile and R,
+                    write dq, dk, dv and the gate gradient = 7de + 8d + s/256 + s/128
     """
     s = 4 * d * d
     de = d * elem
@@ -78,8 +83,8 @@ def algorithmic_bytes(name: str, tokens_heads: int, d: int, C: int, G: int, elem
         "bidir_total": s / G, "bidir_apply_tc": 2 * de,
         "gla_states_tc": 2 * de + 4 * d + s / C, "gla_states_simt": 2 * de + 4 * d + s / C,
         "gla_scan": 2 * s / C + 4 * d / C,
-        "gla_out_tc": 4 * de + 4 * d + s / C, "gla_out_simt": 4 * de + 4 * d + s / C,
-        "gla_bwd_tc": 7 * de + 8 * d + 2 * s / C, "gla_bwd_simt": 7 * de + 8 * d + 2 * s / C,
+        "gla_out_tc": 4 * de + 4 * d + s / 128 + s / 256, "gla_out_simt": 4 * de + 4 * d + s / C,
+        "gla_bwd_tc": 7 * de + 8 * d + s / 256 + s / 128, "gla_bwd_simt": 7 * de + 8 * d + 2 * s / C,
     }[name]
     return per * tokens_heads
 

@@ -328,7 +328,7 @@ __global__ void __launch_bounds__(kThreads, 1) gla_out_tc(const __grid_constant_
                                                           const __grid_constant__ CUtensorMap map_v,
                                                           const __grid_constant__ CUtensorMap map_o,
                                                           const __grid_constant__ CUtensorMap map_g,
-                                                          const float* __restrict__ P, int H, int64_t N,
+                                                          float* __restrict__ P, int H, int64_t N,
                                                           int64_t t_slots, int stride, int ntx, int64_t ntiles) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
@@ -398,7 +398,7 @@ __global__ void __launch_bounds__(kThreads, 1) gla_out_tc(const __grid_constant_
   int c, h, b;
   tile_of(w, c, h, b);
   const int64_t row0 = (int64_t)c * kTile;
-  const float* Pc = state_of(c, h, b);
+  float* Pc = state_of(c, h, b);
   const int64_t wn = w + gridDim.x;  // this CTA's next tile
   gate_ahead = tok_ahead = false;
   float x[64];
@@ -415,8 +415,14 @@ __global__ void __launch_bounds__(kThreads, 1) gla_out_tc(const __grid_constant_
   scale_row_half(sK, t, half, x, -1.f);  // K^ = k / E
   fence_async_smem();
   tc_fence_before();
-  __syncthreads();  // every row of the gate tile has been read
+  __syncthreads();  // every row of the gate tile has been read; P' is in X
   if (s->abort) goto cleanup;
+  if (tid == 0) {
+    // P' as the bf16 operand tile replaces P_c in its cache slot: the backward
+    // loads it back as is
+    bulk_store(Pc, sX, kTileBytes);
+    tma_store_commit();
+  }
   if (tid == 0 && wn < ntiles) {
     // the next tile's gates into the gate tile, its P into L2
     int cn, hn, bn;
@@ -511,6 +517,7 @@ cleanup:
   // CTA exits (bounded waits)
   if (tid == 0 && gate_ahead) mbar_wait(&s->gload, ph ^ 1u, SITE_OUT_TMA);
   if (tid == 0 && tok_ahead) mbar_wait(&s->load, ph ^ 1u, SITE_OUT_TMA);
+  if (tid == 0) tma_store_wait_read0();  // no store still reads shared memory
   tc_fence_before();
   __syncthreads();
   if (warp == 0) tmem_dealloc(tmem, 256);
@@ -529,7 +536,7 @@ struct SmemBwd {
 // w + grid, ...); the barriers complete once per tile, so their parity flips
 // from tile to tile. Shared memory: Q^, K^, V, dO (then, in pairs,
 // the fp32 tiles of dB and k . dk^inter for the log-gate gradient's column
-// sums), X (P', then R'; r and b_end - r during the gate walk), and the pair
+// sums), X (P', loaded as the output kernel cached it, then R'), and the pair
 // sA / sB (the gate tile during the walk; then dA . strict and A . causal;
 // then the dK and dV outputs). TMEM: T0 = dO V^T -> (dA . strict)^T Q^;
 // T1 = Q^ K^^T -> dV; T2 = dO P'^T + (dA . strict) K^ -> q . dq'; T3 = log2 E
@@ -552,8 +559,9 @@ __global__ void __launch_bounds__(kThreads, 1) gla_bwd_tc(
   uint8_t* sB = base + 6 * kTileBytes;
   SmemBwd* s = reinterpret_cast<SmemBwd*>(base + 7 * kTileBytes);
   float* bt = reinterpret_cast<float*>(sA);  // gate tile over sA and sB during the walk
-  float* sr = reinterpret_cast<float*>(sX);  // r and b_end - r over X during the walk
-  float* sdend = sr + kD;
+  // r and b_end - r of the gate walk, over arrays first written after phase 0
+  float* sr = s->dAd;
+  float* sdend = s->bnd;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int t = (warp & 3) * 32 + lane, half = warp >> 2;
   // tile w: 128 tokens c * 128.. of head h of sequence b, in launch order
@@ -568,6 +576,9 @@ __global__ void __launch_bounds__(kThreads, 1) gla_bwd_tc(
     tma_load_4d(dst, map, &s->load, 0, h, row, b);
     tma_load_4d(dst + kBox, map, &s->load, 64, h, row, b);
   };
+  // P' = diag(e^{r}) P_c of a tile, as the forward's output kernel left it in
+  // the cache slot (the bf16 operand tile, loaded as is)
+  auto load_pprime = [&](int64_t ps) { bulk_load(sX, P + ps * kD * kD, kTileBytes, &s->load); };
   if (tid == 0) {
     prefetch_tmap(&map_q);
     prefetch_tmap(&map_k);
@@ -599,14 +610,14 @@ __global__ void __launch_bounds__(kThreads, 1) gla_bwd_tc(
     tile_of(blockIdx.x, c, h, b);
     const int64_t ps = pslot_of(c, h, b);
     load_gate_tile(bt, &map_g, &s->gload, h, c * kTile, b);
-    // P and R are read with plain loads later: into L2 now
-    bulk_prefetch_l2(P + ps * kD * kD, kD * kD * 4);
+    // R is read with plain loads later: into L2 now
     bulk_prefetch_l2(R + (ps + (int64_t)(stride - 1) * H) * kD * kD, kD * kD * 4);
-    mbar_arrive_expect_tx(&s->load, 4 * kTileBytes);
+    mbar_arrive_expect_tx(&s->load, 5 * kTileBytes);
     load_tokens(sQ, &map_q, h, c * kTile, b);
     load_tokens(sK, &map_k, h, c * kTile, b);
     load_tokens(sV, &map_v, h, c * kTile, b);
     load_tokens(sD, &map_do, h, c * kTile, b);
+    load_pprime(ps);
   }
   uint32_t ph = 0;  // parity of every barrier's phase for this CTA's current tile
   for (int64_t w = blockIdx.x; w < ntiles; w += gridDim.x, ph ^= 1u) {
@@ -620,15 +631,9 @@ __global__ void __launch_bounds__(kThreads, 1) gla_bwd_tc(
   // ---- phase 0: gates, Q^, K^, log2 E -> T3, P' -> X
   float x[64];
   gate_rows(bt, &s->gload, ph, &s->abort, SITE_BWD_TMA, sr, sdend, tid, t, half, x);
-  float wr[16], we[16];  // e^{r_m} and e^{b_end_m - r_m} of this thread's state rows m = warp + 8u
+  float we[16];  // e^{b_end_m - r_m} of this thread's state rows m = warp + 8u
 #pragma unroll
-  for (int u = 0; u < 16; ++u) {
-    const int m = warp + 8 * u;
-    wr[u] = exp2f(sr[m] * kLog2e);
-    we[u] = exp2f(sdend[m] * kLog2e);
-  }
-  named_sync(kBarAll, kThreads);  // r and b_end - r are read before X is written
-  load_scaled_state(sX, P + pslot * kD * kD, wr, warp, lane);
+  for (int u = 0; u < 16; ++u) we[u] = exp2f(sdend[warp + 8 * u] * kLog2e);
   if (!mbar_wait(&s->load, ph, SITE_BWD_TMA)) s->abort = 1;
   scale_row_half(sQ, t, half, x, 1.f);   // Q^ = q . E
   scale_row_half(sK, t, half, x, -1.f);  // K^ = k / E
@@ -662,23 +667,24 @@ __global__ void __launch_bounds__(kThreads, 1) gla_bwd_tc(
       for (int kk = 0; kk < kD / 16; ++kk) mma_bf16(tmem + T2, kmaj(aD, kk), kmaj(aX, kk), id_kk, kk != 0);
       mma_commit(&s->mma1b);
     }
-    // while the MMAs run: R rows (fp32) into registers, and <R'_m, P'_m> (fp32)
-    // = e^{b_end_m} <R_m, P_m> into bnd, with P's rows read again (from L2)
+    // while the MMAs run: R rows (fp32) into registers, and <R'_m, P'_m> =
+    // e^{b_end_m} <R_m, P_m> into bnd, with the rows of P' read in X (bf16)
     const float4* R4 = reinterpret_cast<const float4*>(R + rslot * kD * kD);
     float4 rreg[16];
 #pragma unroll
     for (int u = 0; u < 16; ++u) rreg[u] = __ldcs(R4 + (warp + 8 * u) * (kD / 4) + lane);
     {
-      const float4* P4 = reinterpret_cast<const float4*>(P + pslot * kD * kD);
-      float4 pv[16];
-#pragma unroll
-      for (int u = 0; u < 16; ++u) pv[u] = __ldg(P4 + (warp + 8 * u) * (kD / 4) + lane);
+      const int col = lane * 4;
 #pragma unroll
       for (int u = 0; u < 16; ++u) {
-        float dot = pv[u].x * rreg[u].x + pv[u].y * rreg[u].y + pv[u].z * rreg[u].z + pv[u].w * rreg[u].w;
+        const int m = warp + 8 * u;
+        const uint2 pw =
+            *reinterpret_cast<const uint2*>(sX + (col >> 6) * kBox + sw128_offset(m, (col & 63) >> 3) + (col & 7) * 2);
+        const float2 p0 = unpack_bf16(pw.x), p1 = unpack_bf16(pw.y);
+        float dot = p0.x * rreg[u].x + p0.y * rreg[u].y + p1.x * rreg[u].z + p1.y * rreg[u].w;
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
-        if (lane == 0) s->bnd[warp + 8 * u] = dot * wr[u] * we[u];
+        if (lane == 0) s->bnd[m] = dot * we[u];
       }
     }
     // ---- epilogue 1: dA . strict -> sA, A . causal -> sB, the diagonal of dA
@@ -920,7 +926,6 @@ __global__ void __launch_bounds__(kThreads, 1) gla_bwd_tc(
       tile_of(wn, cn, hn, bn);
       const int64_t ps = pslot_of(cn, hn, bn);
       load_gate_tile(bt, &map_g, &s->gload, hn, cn * kTile, bn);
-      bulk_prefetch_l2(P + ps * kD * kD, kD * kD * 4);
       bulk_prefetch_l2(R + (ps + (int64_t)(stride - 1) * H) * kD * kD, kD * kD * 4);
     }
     // dg into the dB tile (the gate map's layout), stored by TMA below
@@ -949,9 +954,11 @@ __global__ void __launch_bounds__(kThreads, 1) gla_bwd_tc(
       int cn = 0, hn = 0, bn = 0;
       if (next) tile_of(wn, cn, hn, bn);
       if (next) {
-        mbar_arrive_expect_tx(&s->load, 4 * kTileBytes);
+        // X (R', read by MMA 3) is free too
+        mbar_arrive_expect_tx(&s->load, 5 * kTileBytes);
         load_tokens(sV, &map_v, hn, cn * kTile, bn);
         load_tokens(sD, &map_do, hn, cn * kTile, bn);
+        load_pprime(pslot_of(cn, hn, bn));
       }
       tma_store_wait_read0();  // the dg store has read fB (over Q and K); all stores have read shared memory
       if (next) {
@@ -991,7 +998,7 @@ cudaError_t tc_gla_chunk_states(const void* x, const void* y, const float* g, fl
   return cudaGetLastError();
 }
 
-cudaError_t tc_gla_chunk_out(const void* q, const void* k, const void* v, const float* g, const float* P, void* o,
+cudaError_t tc_gla_chunk_out(const void* q, const void* k, const void* v, const float* g, float* P, void* o,
                              int B, int H, int64_t N, int64_t t_slots, int stride, cudaStream_t st) {
   using namespace tc_gla_detail;
   CUtensorMap mq, mk, mv, mo, mg;

@@ -6,8 +6,10 @@
 // states, followed by B x T x H slots of d log-gate totals: B*T*H*d*(d+1)
 // floats. The CUDA-core path fills every chunk's slot (P_c, gsum_c); the
 // tensor-core path works on 128-token tiles and fills the slots of each tile's
-// first chunk only (P and gsum of the tile), and its gradient states go to
-// the slot of each tile's last chunk of the workspace.
+// first chunk only (P and gsum of the tile); its output kernel then replaces
+// each tile's fp32 P by the bf16 operand tile of diag(e^{r}) P (r the tile's
+// middle-row log-gate sums), which the backward loads back as is. Its gradient
+// states go to the slot of each tile's last chunk of the workspace.
 #include "kernels.h"
 #include "lasp_common.cuh"
 #include "tc_kernels.h"
