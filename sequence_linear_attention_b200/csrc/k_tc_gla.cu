@@ -525,7 +525,7 @@ cleanup:
 
 // ---------------------------------------------------------------- gradients
 struct SmemBwd {
-  uint64_t gload, load, mma1a, mma1b, mma2, mma3;
+  uint64_t gload, load, ldr, mma1a, mma1b, mma2, mma3;
   uint32_t tmem_base;
   int abort;
   float dAd[kTile];  // do_t . v_t, the diagonal of dO V^T
@@ -587,6 +587,7 @@ __global__ void __launch_bounds__(kThreads, 1) gla_bwd_tc(
     prefetch_tmap(&map_g);
     mbar_init(&s->gload, 1);
     mbar_init(&s->load, 1);
+    mbar_init(&s->ldr, 1);
     mbar_init(&s->mma1a, 1);
     mbar_init(&s->mma1b, 1);
     mbar_init(&s->mma2, 1);
@@ -619,7 +620,8 @@ __global__ void __launch_bounds__(kThreads, 1) gla_bwd_tc(
     load_tokens(sD, &map_do, h, c * kTile, b);
     load_pprime(ps);
   }
-  uint32_t ph = 0;  // parity of every barrier's phase for this CTA's current tile
+  uint32_t ph = 0;       // parity of every barrier's phase for this CTA's current tile
+  bool r_ahead = false;  // thread 0: R's load into sA/sB is in flight
   for (int64_t w = blockIdx.x; w < ntiles; w += gridDim.x, ph ^= 1u) {
   int c, h, b;
   tile_of(w, c, h, b);
@@ -631,6 +633,13 @@ __global__ void __launch_bounds__(kThreads, 1) gla_bwd_tc(
   // ---- phase 0: gates, Q^, K^, log2 E -> T3, P' -> X
   float x[64];
   gate_rows(bt, &s->gload, ph, &s->abort, SITE_BWD_TMA, sr, sdend, tid, t, half, x);
+  named_sync(kBarAll, kThreads);  // every row of the gate tile has been read
+  if (tid == 0) {
+    // R_c (fp32) into the gate tile's space while the token tiles arrive
+    mbar_arrive_expect_tx(&s->ldr, kD * kD * 4);
+    bulk_load(bt, R + rslot * kD * kD, kD * kD * 4, &s->ldr);
+    r_ahead = true;
+  }
   float we[16];  // e^{b_end_m - r_m} of this thread's state rows m = warp + 8u
 #pragma unroll
   for (int u = 0; u < 16; ++u) we[u] = exp2f(sdend[warp + 8 * u] * kLog2e);
@@ -667,12 +676,21 @@ __global__ void __launch_bounds__(kThreads, 1) gla_bwd_tc(
       for (int kk = 0; kk < kD / 16; ++kk) mma_bf16(tmem + T2, kmaj(aD, kk), kmaj(aX, kk), id_kk, kk != 0);
       mma_commit(&s->mma1b);
     }
-    // while the MMAs run: R rows (fp32) into registers, and <R'_m, P'_m> =
-    // e^{b_end_m} <R_m, P_m> into bnd, with the rows of P' read in X (bf16)
-    const float4* R4 = reinterpret_cast<const float4*>(R + rslot * kD * kD);
+    // while the MMAs run: R rows (fp32, from sA/sB) into registers, and
+    // <R'_m, P'_m> = e^{b_end_m} <R_m, P_m> into bnd, with the rows of P' read
+    // in X (bf16)
+    {
+      const bool rok = mbar_wait(&s->ldr, ph, SITE_BWD_TMA);
+      if (!rok) s->abort = 1;
+      if (tid == 0 && rok) r_ahead = false;  // else cleanup waits for it once more
+    }
     float4 rreg[16];
+    {
+      const float4* R4 = reinterpret_cast<const float4*>(bt);
 #pragma unroll
-    for (int u = 0; u < 16; ++u) rreg[u] = __ldcs(R4 + (warp + 8 * u) * (kD / 4) + lane);
+      for (int u = 0; u < 16; ++u) rreg[u] = R4[(warp + 8 * u) * (kD / 4) + lane];
+    }
+    named_sync(kBarAll, kThreads);  // every row of R has been read: the masks may overwrite sA/sB
     {
       const int col = lane * 4;
 #pragma unroll
@@ -970,6 +988,7 @@ __global__ void __launch_bounds__(kThreads, 1) gla_bwd_tc(
   }
   }
 cleanup:
+  if (tid == 0 && r_ahead) mbar_wait(&s->ldr, ph, SITE_BWD_TMA);  // an abort leaves R's load unused: it lands first
   tc_fence_before();
   __syncthreads();
   if (warp == 0) tmem_dealloc(tmem, 512);
