@@ -125,21 +125,12 @@ __device__ __forceinline__ void load_gate_tile(float* bt, const CUtensorMap* map
   for (int cb = 0; cb < 4; ++cb) tma_load_4d(bt + cb * (kTile * 32), map_g, bar, cb * 32, h, row0, b);
 }
 
-// fp32 d x d state rows (global) -> bf16 operand tile, row m scaled by w[u]
-// (m = warp + 8u). Warp w converts rows w, w + 8, ...; lane covers 4 columns.
+// Four fp32 entries (columns 4 lane .. 4 lane + 3) of state row m, times w,
+// into the bf16 operand tile. Warp w converts rows w, w + 8, ...
 __device__ __forceinline__ void put_state_row(uint8_t* tile, int m, int lane, float4 x, float w) {
   const int col = lane * 4;
   const uint32_t off = (col >> 6) * kBox + sw128_offset(m, (col & 63) >> 3) + (col & 7) * 2;
   *reinterpret_cast<uint2*>(tile + off) = make_uint2(pack_bf16(x.x * w, x.y * w), pack_bf16(x.z * w, x.w * w));
-}
-__device__ __forceinline__ void load_scaled_state(uint8_t* tile, const float* __restrict__ src, const float (&w)[16],
-                                                  int warp, int lane) {
-  const float4* p = reinterpret_cast<const float4*>(src);
-  float4 x[16];
-#pragma unroll
-  for (int u = 0; u < 16; ++u) x[u] = __ldcs(p + (warp + 8 * u) * (kD / 4) + lane);
-#pragma unroll
-  for (int u = 0; u < 16; ++u) put_state_row(tile, warp + 8 * u, lane, x[u], w[u]);
 }
 
 // ---------------------------------------------------------------- states
@@ -317,7 +308,7 @@ __device__ __forceinline__ void gate_rows(float* bt, uint64_t* gbar, uint32_t pa
 
 // ---------------------------------------------------------------- output
 struct SmemOut {
-  uint64_t gload, load, mma1, mma2;
+  uint64_t gload, load, ldp, mma1, mma2;
   uint32_t tmem_base;
   int abort;
   float r[kD], dend[kD];
@@ -368,6 +359,7 @@ __global__ void __launch_bounds__(kThreads, 1) gla_out_tc(const __grid_constant_
     prefetch_tmap(&map_g);
     mbar_init(&s->gload, 1);
     mbar_init(&s->load, 1);
+    mbar_init(&s->ldp, 1);
     mbar_init(&s->mma1, 1);
     mbar_init(&s->mma2, 1);
     s->abort = 0;
@@ -394,6 +386,7 @@ __global__ void __launch_bounds__(kThreads, 1) gla_out_tc(const __grid_constant_
   uint32_t ph = 0;            // parity of every barrier's phase for this CTA's current tile
   bool gate_ahead = false;    // thread 0: the next tile's gate tile is in flight
   bool tok_ahead = false;     // thread 0: the next tile's token tiles are in flight
+  bool p_ahead = false;       // thread 0: P's load into the gate tile's space is in flight
   for (int64_t w = blockIdx.x; w < ntiles; w += gridDim.x, ph ^= 1u) {
   int c, h, b;
   tile_of(w, c, h, b);
@@ -403,34 +396,23 @@ __global__ void __launch_bounds__(kThreads, 1) gla_out_tc(const __grid_constant_
   gate_ahead = tok_ahead = false;
   float x[64];
   gate_rows(bt, &s->gload, ph, &s->abort, SITE_OUT_TMA, s->r, s->dend, tid, t, half, x);
-  // P' = diag(e^{r}) P_c into X
-  {
-    float w[16];
-#pragma unroll
-    for (int u = 0; u < 16; ++u) w[u] = exp2f(s->r[warp + 8 * u] * kLog2e);
-    load_scaled_state(sX, Pc, w, warp, lane);
+  named_sync(kBarAll, kThreads);  // every row of the gate tile has been read
+  if (tid == 0) {
+    // P_c (fp32) into the gate tile's space while Q^ and K^ are scaled
+    mbar_arrive_expect_tx(&s->ldp, kD * kD * 4);
+    bulk_load(bt, Pc, kD * kD * 4, &s->ldp);
+    p_ahead = true;
   }
+  float wr[16];  // e^{r_m} of this thread's state rows m = warp + 8u
+#pragma unroll
+  for (int u = 0; u < 16; ++u) wr[u] = exp2f(s->r[warp + 8 * u] * kLog2e);
   if (!mbar_wait(&s->load, ph, SITE_OUT_TMA)) s->abort = 1;
   scale_row_half(sQ, t, half, x, 1.f);   // Q^ = q . E
   scale_row_half(sK, t, half, x, -1.f);  // K^ = k / E
   fence_async_smem();
   tc_fence_before();
-  __syncthreads();  // every row of the gate tile has been read; P' is in X
+  __syncthreads();  // Q^ and K^ are in place
   if (s->abort) goto cleanup;
-  if (tid == 0) {
-    // P' as the bf16 operand tile replaces P_c in its cache slot: the backward
-    // loads it back as is
-    bulk_store(Pc, sX, kTileBytes);
-    tma_store_commit();
-  }
-  if (tid == 0 && wn < ntiles) {
-    // the next tile's gates into the gate tile, its P into L2
-    int cn, hn, bn;
-    tile_of(wn, cn, hn, bn);
-    load_gate_tile(bt, &map_g, &s->gload, hn, cn * kTile, bn);
-    bulk_prefetch_l2(state_of(cn, hn, bn), kD * kD * 4);
-    gate_ahead = true;
-  }
   {
     const uint32_t aQ = smem_u32(sQ), aK = smem_u32(sK), aV = smem_u32(sV), aX = smem_u32(sX), aA = smem_u32(sA);
     constexpr uint32_t id_kk = idesc_bf16(128, 128, 0, 0);
@@ -439,7 +421,37 @@ __global__ void __launch_bounds__(kThreads, 1) gla_out_tc(const __grid_constant_
       tc_fence_after();
       for (int kk = 0; kk < kD / 16; ++kk) mma_bf16(tmem + T0, kmaj(aQ, kk), kmaj(aK, kk), id_kk, kk != 0);
       mma_commit(&s->mma1);
+    }
+    // under Q^ K^^T: P' = diag(e^{r}) P_c from the gate tile's space into X
+    {
+      const bool pok = mbar_wait(&s->ldp, ph, SITE_OUT_TMA);
+      if (!pok) s->abort = 1;
+      if (tid == 0 && pok) p_ahead = false;  // else cleanup waits for it once more
+      const float4* P4 = reinterpret_cast<const float4*>(bt);
+      float4 pr[16];
+#pragma unroll
+      for (int u = 0; u < 16; ++u) pr[u] = P4[(warp + 8 * u) * (kD / 4) + lane];
+#pragma unroll
+      for (int u = 0; u < 16; ++u) put_state_row(sX, warp + 8 * u, lane, pr[u], wr[u]);
+    }
+    fence_async_smem();
+    tc_fence_before();
+    __syncthreads();  // P' is in X; P has been read
+    if (tid == 0 && !s->abort) {
+      // P' as the bf16 operand tile replaces P_c in its cache slot: the backward
+      // loads it back as is
+      bulk_store(Pc, sX, kTileBytes);
+      tma_store_commit();
+      if (wn < ntiles) {
+        // the next tile's gates into the gate tile, its P into L2
+        int cn, hn, bn;
+        tile_of(wn, cn, hn, bn);
+        load_gate_tile(bt, &map_g, &s->gload, hn, cn * kTile, bn);
+        bulk_prefetch_l2(state_of(cn, hn, bn), kD * kD * 4);
+        gate_ahead = true;
+      }
       // the inter term does not wait for the mask
+      tc_fence_after();
       for (int kk = 0; kk < kD / 16; ++kk) mma_bf16(tmem + T1, kmaj(aQ, kk), mnmaj(aX, kk), id_kn, kk != 0);
     }
     // A . causal -> sA (row t, column half)
@@ -517,6 +529,7 @@ cleanup:
   // CTA exits (bounded waits)
   if (tid == 0 && gate_ahead) mbar_wait(&s->gload, ph ^ 1u, SITE_OUT_TMA);
   if (tid == 0 && tok_ahead) mbar_wait(&s->load, ph ^ 1u, SITE_OUT_TMA);
+  if (tid == 0 && p_ahead) mbar_wait(&s->ldp, ph, SITE_OUT_TMA);
   if (tid == 0) tma_store_wait_read0();  // no store still reads shared memory
   tc_fence_before();
   __syncthreads();
