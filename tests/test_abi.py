@@ -175,3 +175,34 @@ def test_split_calls_reject_bad_arguments(lib):
     assert bs(A, None, None, 1, 2, 512, 64, 64, F32, A, None, None) == INVALID           # no dout
     assert bf(A, A, A, None, A, A, A, A, 1, 2, 512, 64, 64, F32, A, None, None, None, None) == INVALID  # no ws
     assert bf(A, A, A, None, A, A, A, A, 1, 2, 512, 64, 64, F32, A, A, A + 4, None, None) == MISALIGNED
+
+
+def test_the_header_serves_a_plain_c_program(tmp_path, lib):
+    """include/lasp.h compiles as strict C99, and a C program linked against
+    the library calls it without torch: host-side calls that return before any
+    CUDA call (sizes, validation, names)."""
+    import shutil
+    import subprocess
+    if shutil.which("gcc") is None:
+        pytest.skip("no C compiler")
+    src = tmp_path / "client.c"
+    src.write_text(r"""
+#include <stdio.h>
+#include "lasp.h"
+int main(void) {
+  printf("%d\n", lasp_version() > 0);
+  printf("%s\n", lasp_status_string(LASP_ERR_UNSUPPORTED));
+  printf("%d\n", lasp_fwd(0, 0, 0, 0, 0, 1, 2, 512, 96, 64, LASP_BF16, 0, 0, 0));         /* d = 96 */
+  printf("%d\n", lasp_fwd_states(0, 0, 0, 1, 2, 500, 64, 64, LASP_F32, 0, 0, 0));        /* C does not divide N */
+  printf("%lld\n", (long long)lasp_gla_cache_floats(2, 3, 512, 64, 64));
+  printf("%d\n", lasp_segment_tokens(65536, 128, 128, LASP_BF16));
+  return 0;
+}
+""")
+    exe = tmp_path / "client"
+    libdir = os.path.dirname(lasp.library_path())
+    subprocess.run(["gcc", "-std=c99", "-Wall", "-Wextra", "-Werror", "-pedantic", "-I", os.path.join(ROOT, "include"),
+                    str(src), "-o", str(exe), "-L", libdir, "-llasp", "-Wl,-rpath," + libdir], check=True)
+    out = subprocess.run([str(exe)], check=True, capture_output=True, text=True).stdout.split()
+    assert out == ["1", "LASP_ERR_UNSUPPORTED", str(UNSUPPORTED), str(INVALID), str(2 * 8 * 3 * 64 * 65),
+                   str(lasp.lasp_segment_tokens(65536, 128, 128, BF16))]
