@@ -307,6 +307,11 @@ def run_gpu(args, rank, world, local):
     per_kernel = {}
     for name, ms in trace:
         per_kernel.setdefault(name, []).append(ms)
+    # the forward and backward separately: each step's launches are lasp_fwd's
+    # followed by as many of lasp_bwd's
+    per_step = len(trace) // ksteps
+    fwd_ms = sum(ms for i, (_, ms) in enumerate(trace) if i % per_step < per_step // 2) / ksteps
+    bwd_ms = sum(ms for i, (_, ms) in enumerate(trace) if i % per_step >= per_step // 2) / ksteps
 
     # end to end through the public API: every step copies its inputs (q, k, v,
     # dO) in from pinned host memory and its results (o, dq, dk, dv) back out.
@@ -371,6 +376,10 @@ def run_gpu(args, rank, world, local):
     achieved = kernel_table[top]["GBps"]
     flops = flops_per_step(th, d, C)
     tflops = flops / (ms_per_step / 1e3) / 1e12
+    # the attainable rate of the step: min(tensor peak, arithmetic intensity x
+    # HBM bandwidth), the intensity over the algorithmic bytes of all launches
+    step_bytes = sum(algorithmic_bytes(n, th, d, C, G, elem) * len(per_kernel[n]) / ksteps for n in names)
+    attainable = min(peaks["bf16_sustained"], flops / step_bytes * peaks["hbm"] / 1e3)
     line = {
         "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4),
@@ -382,6 +391,8 @@ def run_gpu(args, rank, world, local):
                    "parallelism": f"replicas x{world} (independent sequences, no collective)"},
         "tflops": round(tflops, 2),
         "tensor_peak_frac": round(tflops / peaks["bf16_sustained"], 4),
+        "attainable_frac": round(tflops / attainable, 4),
+        "fwd_ms": round(fwd_ms, 4), "bwd_ms": round(bwd_ms, 4),
         "roofline": {"bound": "hbm", "kernel": top, "achieved": round(achieved, 1), "peak": peaks["hbm"],
                      "unit": "GB/s", "frac": round(achieved / peaks["hbm"], 4),
                      "traffic": measured_traffic(top, args.workload) if args.tokens is None else None,
