@@ -63,9 +63,12 @@ def algorithmic_bytes(name: str, tokens_heads: int, d: int, C: int, G: int, elem
       gla_out_simt: read q, k, v, the gates and P, write o             = 4de + 4d + s/C
       gla_bwd_simt: read q, k, v, dO, the gates, P and R, write dq, dk,
                     dv and the gate gradient                          = 7de + 8d + 2s/C
-      gla_out_tc:   per 128-token tile: read q, k, v, the gates and P
-                    (fp32), write o and the bf16 tile of diag(e^r) P over
-                    P's cache slot                       = 4de + 4d + s/128 + s/256
+      gla_segment_states_tc: the forward's states per segment of G tokens
+                    (read 2 token rows and the gates, write s/G) = 2de + 4d + s/G
+      gla_segment_scan: read and write s/G, the segments' gate totals = 2s/G + 4d/G
+      gla_out_tc:   the walk through each segment: read q, k, v, the gates
+                    and the segment's P (s/G), write o and the bf16 tile of
+                    diag(e^r) P per 128-token tile     = 4de + 4d + s/G + s/256
       gla_bwd_tc:   read q, k, v, dO, the gates, that bf16 tile and R,
                     write dq, dk, dv and the gate gradient = 7de + 8d + s/256 + s/128
     """
@@ -83,7 +86,8 @@ def algorithmic_bytes(name: str, tokens_heads: int, d: int, C: int, G: int, elem
         "bidir_total": s / G, "bidir_apply_tc": 2 * de,
         "gla_states_tc": 2 * de + 4 * d + s / C, "gla_states_simt": 2 * de + 4 * d + s / C,
         "gla_scan": 2 * s / C + 4 * d / C,
-        "gla_out_tc": 4 * de + 4 * d + s / 128 + s / 256, "gla_out_simt": 4 * de + 4 * d + s / C,
+        "gla_segment_states_tc": 2 * de + 4 * d + s / G, "gla_segment_scan": 2 * s / G + 4 * d / G,
+        "gla_out_tc": 4 * de + 4 * d + s / G + s / 256, "gla_out_simt": 4 * de + 4 * d + s / C,
         "gla_bwd_tc": 7 * de + 8 * d + s / 256 + s / 128, "gla_bwd_simt": 7 * de + 8 * d + 2 * s / C,
     }[name]
     return per * tokens_heads
@@ -544,9 +548,10 @@ def run_gated(args, rank, world, local):
     peaks = load_peaks()
     th = tokens * H
     kernel_table = {}
+    G = lasp.lasp_segment_tokens(N, C, d, lasp.LASP_BF16)  # the forward walk's segment
     for n, ms in per_kernel.items():
         mean = statistics.mean(ms)
-        gbps = algorithmic_bytes(n, th, d, C, C, 2) / (mean / 1e3) / 1e9
+        gbps = algorithmic_bytes(n, th, d, C, G, 2) / (mean / 1e3) / 1e9
         kernel_table[n] = {"launches_per_step": len(ms) / ksteps, "ms": round(mean, 4), "GBps": round(gbps, 1),
                            "hbm_frac": round(gbps / peaks["hbm"], 4)}
     top = max(per_kernel, key=lambda n: sum(per_kernel[n]))
@@ -560,7 +565,7 @@ def run_gated(args, rank, world, local):
         "roofline": {"bound": "hbm", "kernel": top, "achieved": kernel_table[top]["GBps"], "peak": peaks["hbm"],
                      "unit": "GB/s", "frac": kernel_table[top]["hbm_frac"],
                      "traffic": measured_traffic(top, args.workload) if N == w["N"] else None,
-                     "algorithmic_bytes": algorithmic_bytes(top, th, d, C, C, 2), "peak_source": peaks["source"]},
+                     "algorithmic_bytes": algorithmic_bytes(top, th, d, C, G, 2), "peak_source": peaks["source"]},
         "kernels": kernel_table,
         "gpu_launches": int(round(len(trace) / ksteps * args.steps)),
         "clocks": clk.summary(),

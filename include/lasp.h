@@ -393,7 +393,7 @@ LASP_API int lasp_bidir_bwd(const void* q, const void* k, const void* v, const v
  */
 
 /* Size, in floats, of the state cache of lasp_gla_fwd / lasp_gla_bwd:
- * B * (N/C) * H * d * (d + 1). -1 for sizes the gated calls reject. */
+ * B * (N/C) * H * d * (d + 2). -1 for sizes the gated calls reject. */
 LASP_API int64_t lasp_gla_cache_floats(int B, int H, int64_t N, int d, int C);
 
 /*

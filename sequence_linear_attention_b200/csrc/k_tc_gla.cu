@@ -148,20 +148,29 @@ struct SmemStates {
 // group's log-gates, the eight groups' sums give each group's offset, and a
 // second pass over the loaded values (down for kind 1, up for kind 0:
 // e^{b_end - b_t} = e^{sum_{r>t} g_r}) scales the tile.
+//
+// A CTA takes `tiles` consecutive tiles (a segment of the sequence, one state
+// for all of them): kind 0 from the last tile to the first, kind 1 from the
+// first to the last, each thread carrying the log-gate sum of its features
+// over the tiles already done. That sum joins every factor of the next tile,
+// so the tiles' products add up in one TMEM accumulator with no rescaling;
+// every factor stays at most 1 for log-gates <= 0. gsum (kind 0, may be NULL)
+// receives the item's total log-gate in the item's slot; gsum_tile (may be
+// NULL) every tile's own total in the slot of tile c, c * tstride.
 __global__ void __launch_bounds__(kThreads, 2) gla_states_tc(const __grid_constant__ CUtensorMap map_x,
                                                              const __grid_constant__ CUtensorMap map_y,
                                                              const float* __restrict__ g, float* __restrict__ M,
-                                                             float* __restrict__ gsum, int H, int64_t N, int kind,
-                                                             int64_t t_slots, int stride, int offset) {
+                                                             float* __restrict__ gsum, float* __restrict__ gsum_tile,
+                                                             int H, int64_t N, int kind, int64_t t_slots, int stride,
+                                                             int offset, int tiles, int tstride) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   uint8_t* sX = base;
   uint8_t* sY = base + kTileBytes;
   SmemStates* s = reinterpret_cast<SmemStates*>(base + 2 * kTileBytes);
-  const int c = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const int item = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int64_t row0 = (int64_t)c * kTile;
-  const int64_t sl = (int64_t)b * t_slots + (int64_t)c * stride + offset;  // the state slot of this tile
+  const int64_t sl = (int64_t)b * t_slots + (int64_t)item * stride + offset;  // the state slot of this item
   if (tid == 0) {
     prefetch_tmap(&map_x);
     prefetch_tmap(&map_y);
@@ -178,18 +187,23 @@ __global__ void __launch_bounds__(kThreads, 2) gla_states_tc(const __grid_consta
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = s->tmem_base;
-  if (tid == 0) {
-    mbar_arrive_expect_tx(&s->load, 2 * kTileBytes);
-    tma_load_4d(sX, &map_x, &s->load, 0, h, (int)row0, b);
-    tma_load_4d(sX + kBox, &map_x, &s->load, 64, h, (int)row0, b);
-    tma_load_4d(sY, &map_y, &s->load, 0, h, (int)row0, b);
-    tma_load_4d(sY + kBox, &map_y, &s->load, 64, h, (int)row0, b);
-  }
-  {
-    const int f0 = lane * 4;  // features f0..f0+3
+  const int f0 = lane * 4;  // features f0..f0+3
+  float4 off = make_float4(0.f, 0.f, 0.f, 0.f);  // log-gate sum of the tiles already done
+  for (int j = 0; j < tiles; ++j) {
+    const int64_t tile = (int64_t)item * tiles + (kind == 0 ? tiles - 1 - j : j);
+    const int64_t row0 = tile * kTile;
+    const uint32_t par = (uint32_t)j & 1u;
+    if (tid == 0) {
+      // the previous tile's MMA has read sX and sY (waited below)
+      mbar_arrive_expect_tx(&s->load, 2 * kTileBytes);
+      tma_load_4d(sX, &map_x, &s->load, 0, h, (int)row0, b);
+      tma_load_4d(sX + kBox, &map_x, &s->load, 64, h, (int)row0, b);
+      tma_load_4d(sY, &map_y, &s->load, 0, h, (int)row0, b);
+      tma_load_4d(sY + kBox, &map_y, &s->load, 64, h, (int)row0, b);
+    }
     const int64_t rs = (int64_t)H * kD;
-    const float4* gp = reinterpret_cast<const float4*>(g + ((int64_t)b * N + row0 + warp * 16) * rs +
-                                                       (int64_t)h * kD + f0);
+    const float4* gp =
+        reinterpret_cast<const float4*>(g + ((int64_t)b * N + row0 + warp * 16) * rs + (int64_t)h * kD + f0);
     float4 gv[16];
 #pragma unroll
     for (int u = 0; u < 16; ++u) gv[u] = __ldg(gp + (int64_t)u * (rs / 4));
@@ -202,21 +216,32 @@ __global__ void __launch_bounds__(kThreads, 2) gla_states_tc(const __grid_consta
       tot.w += gv[u].w;
     }
     *reinterpret_cast<float4*>(&s->grp[warp][f0]) = tot;
-    const bool ok = mbar_wait(&s->load, 0, SITE_STATES_TMA);
+    const bool ok = mbar_wait(&s->load, par, SITE_STATES_TMA);
     if (!ok) s->abort = 1;
     __syncthreads();
-    // the part of the exponent from the other groups: kind 1 sums down from
-    // row 0, kind 0 up from the last row
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    // the part of the exponent from the other groups (kind 1 sums down from
+    // row 0, kind 0 up from the last row) and from the tiles already done;
+    // the tile's own total joins `off` for the next tile
+    float4 acc = off, all = make_float4(0.f, 0.f, 0.f, 0.f);
     for (int w2 = 0; w2 < 8; ++w2) {
+      const float4 x = *reinterpret_cast<const float4*>(&s->grp[w2][f0]);
+      all.x += x.x;
+      all.y += x.y;
+      all.z += x.z;
+      all.w += x.w;
       if (kind == 0 ? w2 > warp : w2 < warp) {
-        const float4 x = *reinterpret_cast<const float4*>(&s->grp[w2][f0]);
         acc.x += x.x;
         acc.y += x.y;
         acc.z += x.z;
         acc.w += x.w;
       }
     }
+    off.x += all.x;
+    off.y += all.y;
+    off.z += all.z;
+    off.w += all.w;
+    if (gsum_tile != nullptr && warp == 0)
+      *reinterpret_cast<float4*>(gsum_tile + (((int64_t)b * t_slots + tile * tstride) * H + h) * kD + f0) = all;
     uint8_t* colp = sX + (f0 >> 6) * kBox + (f0 & 7) * 2;
 #pragma unroll
     for (int n = 0; n < 16; ++n) {
@@ -242,24 +267,28 @@ __global__ void __launch_bounds__(kThreads, 2) gla_states_tc(const __grid_consta
         acc.w += gv[u].w;
       }
     }
+    fence_async_smem();
+    tc_fence_before();
+    __syncthreads();  // every thread has read grp and scaled its rows
+    if (s->abort) goto cleanup;
+    if (tid == 0) {
+      tc_fence_after();
+      constexpr uint32_t id_nn = idesc_bf16(128, 128, 1, 1);
+      const uint32_t aX = smem_u32(sX), aY = smem_u32(sY);
+      for (int kk = 0; kk < kTile / 16; ++kk) mma_bf16(tmem, mnmaj(aX, kk), mnmaj(aY, kk), id_nn, kk != 0 || j > 0);
+      mma_commit(&s->mma);
+    }
+    if (j + 1 < tiles) {
+      // the MMA has read sX and sY before the next tile's loads go there
+      if (!mbar_wait(&s->mma, par, SITE_STATES_MMA)) s->abort = 1;
+      __syncthreads();
+      if (s->abort) goto cleanup;
+    }
   }
-  fence_async_smem();
-  tc_fence_before();
-  __syncthreads();
-  if (s->abort) goto cleanup;
-  if (tid == 0) {
-    tc_fence_after();
-    constexpr uint32_t id_nn = idesc_bf16(128, 128, 1, 1);
-    const uint32_t aX = smem_u32(sX), aY = smem_u32(sY);
-    for (int kk = 0; kk < kTile / 16; ++kk) mma_bf16(tmem, mnmaj(aX, kk), mnmaj(aY, kk), id_nn, kk != 0);
-    mma_commit(&s->mma);
-  }
-  if (kind == 0 && gsum != nullptr && tid < kD) {
-    float a = 0.f;
-    for (int w2 = 0; w2 < 8; ++w2) a += s->grp[w2][tid];
-    gsum[(sl * H + h) * kD + tid] = a;
-  }
-  if (mbar_wait(&s->mma, 0, SITE_STATES_MMA)) {
+  // the item's total log-gate (kind 0): every warp holds it; warp 0 writes it
+  if (kind == 0 && gsum != nullptr && warp == 0)
+    *reinterpret_cast<float4*>(gsum + (sl * H + h) * kD + f0) = off;
+  if (mbar_wait(&s->mma, (uint32_t)(tiles - 1) & 1u, SITE_STATES_MMA)) {
     tc_fence_after();
     // row i of M (TMEM lane i), columns half*64..
     const int i = (warp & 3) * 32 + lane, half = warp >> 2;
@@ -319,8 +348,10 @@ __global__ void __launch_bounds__(kThreads, 1) gla_out_tc(const __grid_constant_
                                                           const __grid_constant__ CUtensorMap map_v,
                                                           const __grid_constant__ CUtensorMap map_o,
                                                           const __grid_constant__ CUtensorMap map_g,
+                                                          const __grid_constant__ CUtensorMap map_p,
                                                           float* __restrict__ P, int H, int64_t N,
-                                                          int64_t t_slots, int stride, int ntx, int64_t ntiles) {
+                                                          int64_t t_slots, int stride, int ntx, int tiles,
+                                                          int64_t nseg) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   uint8_t* sQ = base;                   // Q^
@@ -328,20 +359,19 @@ __global__ void __launch_bounds__(kThreads, 1) gla_out_tc(const __grid_constant_
   uint8_t* sV = base + 2 * kTileBytes;
   uint8_t* sX = base + 3 * kTileBytes;  // P'
   uint8_t* sA = base + 4 * kTileBytes;  // A . causal, then O out
-  float* bt = reinterpret_cast<float*>(base + 5 * kTileBytes);  // gate tile, 64 KB
+  float* bt = reinterpret_cast<float*>(base + 5 * kTileBytes);  // gate tile, 64 KB (then a segment's P)
   SmemOut* s = reinterpret_cast<SmemOut*>(base + 7 * kTileBytes);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int t = (warp & 3) * 32 + lane, half = warp >> 2;
-  // tile w: 128 tokens c * 128.. of head h of sequence b, in launch order
-  auto tile_of = [&](int64_t w, int& c, int& h, int& b) {
-    c = (int)(w % ntx);
-    h = (int)((w / ntx) % H);
-    b = (int)(w / ((int64_t)ntx * H));
+  const int spq = ntx / tiles;  // segments per sequence
+  // segment sg: tiles cs * tiles .. of head h of sequence b, in launch order
+  auto seg_of = [&](int64_t sg, int& cs, int& h, int& b) {
+    cs = (int)(sg % spq);
+    h = (int)((sg / spq) % H);
+    b = (int)(sg / ((int64_t)spq * H));
   };
-  // P of a tile's first chunk
-  auto state_of = [&](int c, int h, int b) {
-    return P + (((int64_t)b * t_slots + (int64_t)c * stride) * H + h) * kD * kD;
-  };
+  // the cache slot of tile c (the slot of its first chunk)
+  auto slot_of = [&](int c, int h, int b) { return ((int64_t)b * t_slots + (int64_t)c * stride) * H + h; };
   auto load_tokens = [&](int h, int row, int b) {
     mbar_arrive_expect_tx(&s->load, 3 * kTileBytes);
     tma_load_4d(sQ, &map_q, &s->load, 0, h, row, b);
@@ -357,6 +387,7 @@ __global__ void __launch_bounds__(kThreads, 1) gla_out_tc(const __grid_constant_
     prefetch_tmap(&map_v);
     prefetch_tmap(&map_o);
     prefetch_tmap(&map_g);
+    prefetch_tmap(&map_p);
     mbar_init(&s->gload, 1);
     mbar_init(&s->load, 1);
     mbar_init(&s->ldp, 1);
@@ -366,7 +397,7 @@ __global__ void __launch_bounds__(kThreads, 1) gla_out_tc(const __grid_constant_
     fence_mbar_init();
   }
   if (warp == 0) {
-    tmem_alloc(&s->tmem_base, 256);
+    tmem_alloc(&s->tmem_base, 512);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -374,38 +405,55 @@ __global__ void __launch_bounds__(kThreads, 1) gla_out_tc(const __grid_constant_
   tc_fence_after();
   const uint32_t tmem = s->tmem_base;
   const uint32_t lane_base = tmem + ((uint32_t)((warp & 3) * 32) << 16);
-  const uint32_t T0 = 0, T1 = 128;
-  if (tid == 0 && (int64_t)blockIdx.x < ntiles) {
+  const uint32_t T0 = 0, T1 = 128, TP = 256;
+  if (tid == 0 && (int64_t)blockIdx.x < nseg) {
     // the first tile's loads; a later tile's are issued during the tile before
-    int c, h, b;
-    tile_of(blockIdx.x, c, h, b);
-    load_gate_tile(bt, &map_g, &s->gload, h, c * kTile, b);
-    bulk_prefetch_l2(state_of(c, h, b), kD * kD * 4);  // read with plain loads later
-    load_tokens(h, c * kTile, b);
+    int cs, h, b;
+    seg_of(blockIdx.x, cs, h, b);
+    load_gate_tile(bt, &map_g, &s->gload, h, cs * tiles * kTile, b);
+    bulk_prefetch_l2(P + slot_of(cs * tiles, h, b) * kD * kD, kD * kD * 4);  // loaded after the gate walk
+    load_tokens(h, cs * tiles * kTile, b);
   }
-  uint32_t ph = 0;            // parity of every barrier's phase for this CTA's current tile
+  uint32_t ph = 0;            // parity of the per-tile barriers' phase for this CTA's current tile
+  uint32_t pph = 0;           // parity of the P barrier (once per segment)
   bool gate_ahead = false;    // thread 0: the next tile's gate tile is in flight
   bool tok_ahead = false;     // thread 0: the next tile's token tiles are in flight
   bool p_ahead = false;       // thread 0: P's load into the gate tile's space is in flight
-  for (int64_t w = blockIdx.x; w < ntiles; w += gridDim.x, ph ^= 1u) {
-  int c, h, b;
-  tile_of(w, c, h, b);
+  float dprev = 0.f;          // b_end - r of state row t in the tile before (inside a segment)
+  for (int64_t sg = blockIdx.x; sg < nseg; sg += gridDim.x) {
+  for (int j = 0; j < tiles; ++j, ph ^= 1u) {
+  int cs, h, b;
+  seg_of(sg, cs, h, b);
+  const int c = cs * tiles + j;
   const int64_t row0 = (int64_t)c * kTile;
-  float* Pc = state_of(c, h, b);
-  const int64_t wn = w + gridDim.x;  // this CTA's next tile
+  float* Pc = P + slot_of(c, h, b) * kD * kD;
+  // this CTA's next tile
+  const int64_t sgn = j + 1 < tiles ? sg : sg + gridDim.x;
+  const int jn = j + 1 < tiles ? j + 1 : 0;
+  const bool has_next = sgn < nseg;
   gate_ahead = tok_ahead = false;
   float x[64];
   gate_rows(bt, &s->gload, ph, &s->abort, SITE_OUT_TMA, s->r, s->dend, tid, t, half, x);
   named_sync(kBarAll, kThreads);  // every row of the gate tile has been read
-  if (tid == 0) {
-    // P_c (fp32) into the gate tile's space while Q^ and K^ are scaled
+  if (tid == 0 && j == 0) {
+    // the segment's entering state P (fp32) into the gate tile's space: four
+    // boxes of 32 columns with the 128-byte swizzle, so that every thread
+    // reads its own row without bank conflicts
     mbar_arrive_expect_tx(&s->ldp, kD * kD * 4);
-    bulk_load(bt, Pc, kD * kD * 4, &s->ldp);
+    const int y = (int)(slot_of(c, h, b) * kD);
+#pragma unroll
+    for (int bx = 0; bx < 4; ++bx)
+      tma_load_2d(reinterpret_cast<uint8_t*>(bt) + bx * (kTile * 128), &map_p, &s->ldp, 32 * bx, y);
     p_ahead = true;
   }
-  float wr[16];  // e^{r_m} of this thread's state rows m = warp + 8u
-#pragma unroll
-  for (int u = 0; u < 16; ++u) wr[u] = exp2f(s->r[warp + 8 * u] * kLog2e);
+  // the factors of state row t: e^{(b_end - r) of the tile before} carries
+  // the state from that tile into this one (after a segment's first tile),
+  // then e^{r} makes P'. They are applied one after the other: each lies in
+  // [e^{-80}, 1] (the range check bounds both half-tile sums), their product
+  // need not be a normal fp32 number.
+  const float wcarry = exp2f(dprev * kLog2e);
+  const float wrow = exp2f(s->r[t] * kLog2e);
+  const float dnext = s->dend[t];
   if (!mbar_wait(&s->load, ph, SITE_OUT_TMA)) s->abort = 1;
   scale_row_half(sQ, t, half, x, 1.f);   // Q^ = q . E
   scale_row_half(sK, t, half, x, -1.f);  // K^ = k / E
@@ -417,37 +465,80 @@ __global__ void __launch_bounds__(kThreads, 1) gla_out_tc(const __grid_constant_
     const uint32_t aQ = smem_u32(sQ), aK = smem_u32(sK), aV = smem_u32(sV), aX = smem_u32(sX), aA = smem_u32(sA);
     constexpr uint32_t id_kk = idesc_bf16(128, 128, 0, 0);
     constexpr uint32_t id_kn = idesc_bf16(128, 128, 0, 1);
+    constexpr uint32_t id_nn = idesc_bf16(128, 128, 1, 1);
     if (tid == 0) {
       tc_fence_after();
       for (int kk = 0; kk < kD / 16; ++kk) mma_bf16(tmem + T0, kmaj(aQ, kk), kmaj(aK, kk), id_kk, kk != 0);
       mma_commit(&s->mma1);
     }
-    // under Q^ K^^T: P' = diag(e^{r}) P_c from the gate tile's space into X
+    // under Q^ K^^T: P' = diag(e^{r}) P of row t (this thread's TMEM lane),
+    // columns half * 64.., as bf16 into X and (inside a segment) as fp32 into
+    // TMEM, where the state update accumulates onto it
     {
-      const bool pok = mbar_wait(&s->ldp, ph, SITE_OUT_TMA);
-      if (!pok) s->abort = 1;
-      if (tid == 0 && pok) p_ahead = false;  // else cleanup waits for it once more
-      const float4* P4 = reinterpret_cast<const float4*>(bt);
-      float4 pr[16];
+      float v[64];
+      if (j == 0) {
+        const bool pok = mbar_wait(&s->ldp, pph, SITE_OUT_TMA);
+        pph ^= 1u;
+        if (!pok) s->abort = 1;
+        if (tid == 0 && pok) p_ahead = false;  // else cleanup waits for it once more
+        const uint8_t* src = reinterpret_cast<const uint8_t*>(bt) + 2 * half * (kTile * 128);
 #pragma unroll
-      for (int u = 0; u < 16; ++u) pr[u] = P4[(warp + 8 * u) * (kD / 4) + lane];
+        for (int bb = 0; bb < 2; ++bb)
 #pragma unroll
-      for (int u = 0; u < 16; ++u) put_state_row(sX, warp + 8 * u, lane, pr[u], wr[u]);
+          for (int cc = 0; cc < 8; ++cc) {
+            const float4 q4 = *reinterpret_cast<const float4*>(src + bb * (kTile * 128) + sw128_offset(t, cc));
+            v[bb * 32 + 4 * cc] = q4.x;
+            v[bb * 32 + 4 * cc + 1] = q4.y;
+            v[bb * 32 + 4 * cc + 2] = q4.z;
+            v[bb * 32 + 4 * cc + 3] = q4.w;
+          }
+      } else {
+        uint32_t r0[32], r1[32];
+        tmem_ld32(lane_base + TP + half * 64, r0);
+        tmem_ld32(lane_base + TP + half * 64 + 32, r1);
+        tmem_ld_wait();
+#pragma unroll
+        for (int u = 0; u < 32; ++u) {
+          v[u] = __uint_as_float(r0[u]);
+          v[32 + u] = __uint_as_float(r1[u]);
+        }
+      }
+      if (j > 0) {
+#pragma unroll
+        for (int u = 0; u < 64; ++u) v[u] *= wcarry;
+      }
+#pragma unroll
+      for (int u = 0; u < 64; ++u) v[u] *= wrow;
+      if (j + 1 < tiles) {
+#pragma unroll
+        for (int c2 = 0; c2 < 2; ++c2) {
+          uint32_t r[32];
+#pragma unroll
+          for (int u = 0; u < 32; ++u) r[u] = __float_as_uint(v[c2 * 32 + u]);
+          tmem_st32(lane_base + TP + half * 64 + c2 * 32, r);
+        }
+        tmem_st_wait();
+      }
+#pragma unroll
+      for (int q8 = 0; q8 < 8; ++q8)
+        *tile16(sX, t, half * 64 + q8 * 8) =
+            make_uint4(pack_bf16(v[q8 * 8], v[q8 * 8 + 1]), pack_bf16(v[q8 * 8 + 2], v[q8 * 8 + 3]),
+                       pack_bf16(v[q8 * 8 + 4], v[q8 * 8 + 5]), pack_bf16(v[q8 * 8 + 6], v[q8 * 8 + 7]));
     }
     fence_async_smem();
     tc_fence_before();
-    __syncthreads();  // P' is in X; P has been read
+    __syncthreads();  // P' is in X; a segment's P has been read
     if (tid == 0 && !s->abort) {
-      // P' as the bf16 operand tile replaces P_c in its cache slot: the backward
-      // loads it back as is
+      // P' as the bf16 operand tile goes to this tile's cache slot: the
+      // backward loads it back as is
       bulk_store(Pc, sX, kTileBytes);
       tma_store_commit();
-      if (wn < ntiles) {
-        // the next tile's gates into the gate tile, its P into L2
-        int cn, hn, bn;
-        tile_of(wn, cn, hn, bn);
-        load_gate_tile(bt, &map_g, &s->gload, hn, cn * kTile, bn);
-        bulk_prefetch_l2(state_of(cn, hn, bn), kD * kD * 4);
+      if (has_next) {
+        // the next tile's gates into the gate tile (and, at a segment start, its P into L2)
+        int csn, hn, bn;
+        seg_of(sgn, csn, hn, bn);
+        load_gate_tile(bt, &map_g, &s->gload, hn, (csn * tiles + jn) * kTile, bn);
+        if (jn == 0) bulk_prefetch_l2(P + slot_of(csn * tiles, hn, bn) * kD * kD, kD * kD * 4);
         gate_ahead = true;
       }
       // the inter term does not wait for the mask
@@ -482,16 +573,20 @@ __global__ void __launch_bounds__(kThreads, 1) gla_out_tc(const __grid_constant_
     if (tid == 0) {
       tc_fence_after();
       for (int kk = 0; kk < kTile / 16; ++kk) mma_bf16(tmem + T1, kmaj(aA, kk), mnmaj(aV, kk), id_kn, 1);
+      // inside a segment, the state update onto P' in TMEM: + K^^T V (the next
+      // tile's factor e^{b_end - r} turns K^ into k e^{b_end - b})
+      if (j + 1 < tiles)
+        for (int kk = 0; kk < kTile / 16; ++kk) mma_bf16(tmem + TP, mnmaj(aK, kk), mnmaj(aV, kk), id_nn, 1);
       mma_commit(&s->mma2);
     }
     // O -> sA (free once the MMA has read it) -> TMA store
     if (mbar_wait(&s->mma2, ph, SITE_OUT_MMA)) {
       tc_fence_after();
-      if (tid == 0 && wn < ntiles) {
+      if (tid == 0 && has_next) {
         // every MMA has read Q^, K^, V and P': the next tile's tokens go in
-        int cn, hn, bn;
-        tile_of(wn, cn, hn, bn);
-        load_tokens(hn, cn * kTile, bn);
+        int csn, hn, bn;
+        seg_of(sgn, csn, hn, bn);
+        load_tokens(hn, (csn * tiles + jn) * kTile, bn);
         tok_ahead = true;
       }
 #pragma unroll 1
@@ -522,6 +617,8 @@ __global__ void __launch_bounds__(kThreads, 1) gla_out_tc(const __grid_constant_
     }
     if (stop) goto cleanup;
   }
+  dprev = dnext;
+  }
   }
   gate_ahead = tok_ahead = false;
 cleanup:
@@ -529,11 +626,11 @@ cleanup:
   // CTA exits (bounded waits)
   if (tid == 0 && gate_ahead) mbar_wait(&s->gload, ph ^ 1u, SITE_OUT_TMA);
   if (tid == 0 && tok_ahead) mbar_wait(&s->load, ph ^ 1u, SITE_OUT_TMA);
-  if (tid == 0 && p_ahead) mbar_wait(&s->ldp, ph, SITE_OUT_TMA);
+  if (tid == 0 && p_ahead) mbar_wait(&s->ldp, pph, SITE_OUT_TMA);
   if (tid == 0) tma_store_wait_read0();  // no store still reads shared memory
   tc_fence_before();
   __syncthreads();
-  if (warp == 0) tmem_dealloc(tmem, 256);
+  if (warp == 0) tmem_dealloc(tmem, 512);
 }
 
 // ---------------------------------------------------------------- gradients
@@ -1016,8 +1113,9 @@ bool tc_gla_ok(int dtype, int d, int64_t C, int64_t N) {
   return dtype == LASP_BF16 && d == tc_gla_detail::kD && C >= 1 && C <= kTile && kTile % C == 0 && N % kTile == 0;
 }
 
-cudaError_t tc_gla_chunk_states(const void* x, const void* y, const float* g, float* M, float* gsum, int B, int H,
-                                int64_t N, int kind, int64_t t_slots, int stride, int offset, cudaStream_t st) {
+cudaError_t tc_gla_chunk_states(const void* x, const void* y, const float* g, float* M, float* gsum,
+                                float* gsum_tile, int B, int H, int64_t N, int kind, int64_t t_slots, int stride,
+                                int offset, int tiles, int tstride, cudaStream_t st) {
   using namespace tc_gla_detail;
   CUtensorMap mx, my;
   if (!make_token_map(&mx, x, B, H, N, kD, kTile) || !make_token_map(&my, y, B, H, N, kD, kTile))
@@ -1025,18 +1123,21 @@ cudaError_t tc_gla_chunk_states(const void* x, const void* y, const float* g, fl
   const size_t smem = 1024 + 2 * (size_t)kTileBytes + sizeof(SmemStates);
   cudaError_t e = cudaFuncSetAttribute(gla_states_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  gla_states_tc<<<dim3((unsigned)(N / kTile), H, B), kThreads, smem, st>>>(mx, my, g, M, gsum, H, N, kind, t_slots,
-                                                                          stride, offset);
+  if (tiles < 1 || N % ((int64_t)tiles * kTile) != 0) return cudaErrorInvalidValue;
+  gla_states_tc<<<dim3((unsigned)(N / ((int64_t)tiles * kTile)), H, B), kThreads, smem, st>>>(
+      mx, my, g, M, gsum, gsum_tile, H, N, kind, t_slots, stride, offset, tiles, tstride);
   return cudaGetLastError();
 }
 
 cudaError_t tc_gla_chunk_out(const void* q, const void* k, const void* v, const float* g, float* P, void* o,
-                             int B, int H, int64_t N, int64_t t_slots, int stride, cudaStream_t st) {
+                             int B, int H, int64_t N, int64_t t_slots, int stride, int tiles, cudaStream_t st) {
   using namespace tc_gla_detail;
-  CUtensorMap mq, mk, mv, mo, mg;
+  CUtensorMap mq, mk, mv, mo, mg, mp;
+  const int ntx = (int)(N / kTile);
+  if (tiles < 1 || ntx % tiles != 0) return cudaErrorInvalidValue;
   if (!make_token_map(&mq, q, B, H, N, kD, kTile) || !make_token_map(&mk, k, B, H, N, kD, kTile) ||
       !make_token_map(&mv, v, B, H, N, kD, kTile) || !make_token_map(&mo, o, B, H, N, kD, kTile) ||
-      !make_gate_map(&mg, g, B, H, N, kD, kTile))
+      !make_gate_map(&mg, g, B, H, N, kD, kTile) || !make_state_map(&mp, P, (int64_t)B * t_slots * H, kD))
     return cudaErrorInvalidValue;
   const size_t smem = 1024 + 7 * (size_t)kTileBytes + sizeof(SmemOut);
   cudaError_t e = cudaFuncSetAttribute(gla_out_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -1045,17 +1146,12 @@ cudaError_t tc_gla_chunk_out(const void* q, const void* k, const void* v, const 
   if ((e = cudaGetDevice(&dev)) != cudaSuccess ||
       (e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
     return e;
-  // one persistent CTA per SM (the kernel holds most of shared memory)
-  const int ntx = (int)(N / kTile);
-  const int64_t ntiles = (int64_t)B * H * ntx;
-  const unsigned grid = (unsigned)std::min<int64_t>(ntiles, sms);
-  gla_out_tc<<<grid, kThreads, smem, st>>>(mq, mk, mv, mo, mg, P, H, N, t_slots, stride, ntx, ntiles);
+  // one persistent CTA per SM (the kernel holds most of shared memory and all of TMEM)
+  const int64_t nseg = (int64_t)B * H * (ntx / tiles);
+  const unsigned grid = (unsigned)std::min<int64_t>(nseg, sms);
+  gla_out_tc<<<grid, kThreads, smem, st>>>(mq, mk, mv, mo, mg, mp, P, H, N, t_slots, stride, ntx, tiles, nseg);
   return cudaGetLastError();
 }
-
-}  // namespace lasp
-
-namespace lasp {
 
 cudaError_t tc_gla_chunk_bwd(const void* q, const void* k, const void* v, const void* dout, const float* g,
                              const float* P, const float* Rs, void* dq, void* dk, void* dv, float* dg, int B, int H,

@@ -40,6 +40,8 @@ enum KernelId : int {
   K_GLA_OUT_TC = 20,     // gated form on the tensor cores: output
   K_GLA_BWD_TC = 21,     // gated form on the tensor cores: gradients
   K_STATE_TOTAL = 22,    // decayed total of a sequence's states (the LASP-2 shard state)
+  K_GLA_SEG_STATES = 23,  // gated form on the tensor cores: segment states (forward)
+  K_GLA_SEG_SCAN = 24,    // gated form: prefix over segments
   K_COUNT
 };
 
@@ -460,6 +462,8 @@ const char* lasp_kernel_name(int id) {
     case K_GLA_OUT_TC: return "gla_out_tc";
     case K_GLA_BWD_TC: return "gla_bwd_tc";
     case K_STATE_TOTAL: return "state_total";
+    case K_GLA_SEG_STATES: return "gla_segment_states_tc";
+    case K_GLA_SEG_SCAN: return "gla_segment_scan";
     default: return "unknown";
   }
 }

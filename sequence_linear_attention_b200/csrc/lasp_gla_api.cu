@@ -3,13 +3,18 @@
 // Table 5. Host-side validation and dispatch; nothing here allocates.
 //
 // The state cache of lasp_gla_fwd holds B x T x H chunk slots of fp32 d x d
-// states, followed by B x T x H slots of d log-gate totals: B*T*H*d*(d+1)
-// floats. The CUDA-core path fills every chunk's slot (P_c, gsum_c); the
-// tensor-core path works on 128-token tiles and fills the slots of each tile's
-// first chunk only (P and gsum of the tile); its output kernel then replaces
-// each tile's fp32 P by the bf16 operand tile of diag(e^{r}) P (r the tile's
-// middle-row log-gate sums), which the backward loads back as is. Its gradient
-// states go to the slot of each tile's last chunk of the workspace.
+// states, then B x T x H slots of d log-gate totals, then as many again for
+// segment totals: B*T*H*d*(d+2) floats. The CUDA-core path fills every
+// chunk's slot (P_c, gsum_c). The tensor-core path walks segments of about
+// 1024 tokens: their states (the segment state kernel, which also writes each
+// 128-token tile's log-gate total into the slot of the tile's first chunk)
+// and totals go to the slots of each segment's first chunk, the scan over
+// segments turns them into the states entering the segments, and the walk
+// carries the state through each segment's tiles, leaving in the slot of every
+// tile's first chunk the bf16 operand tile of diag(e^{r}) P (r the tile's
+// middle-row log-gate sums) that the backward loads back as is. The backward's
+// gradient states go to the slot of each tile's last chunk of the workspace;
+// its scan over tiles uses the tile totals.
 #include "kernels.h"
 #include "lasp_common.cuh"
 #include "tc_kernels.h"
@@ -30,7 +35,7 @@ int states_impl(const void* x, const void* y, const float* g, float* M, float* g
                 int C, int dtype, int kind, cudaStream_t st) {
   if (C == 128 && tc_gla_ok(dtype, d, C, N))
     return cuda_status(traced(K_GLA_STATES_TC, st, [&] {
-      return tc_gla_chunk_states(x, y, g, M, gsum, B, H, N, kind, N / C, 1, 0, st);
+      return tc_gla_chunk_states(x, y, g, M, gsum, nullptr, B, H, N, kind, N / C, 1, 0, 1, 1, st);
     }));
   return cuda_status(traced(K_GLA_STATES, st, [&] {
     return gla_simt_chunk_states(x, y, g, M, gsum, B, H, N, d, C, kind, dtype, st);
@@ -57,7 +62,7 @@ extern "C" {
 
 int64_t lasp_gla_cache_floats(int B, int H, int64_t N, int d, int C) {
   if (check_gla_sizes(B, H, N, d, C, LASP_F32)) return -1;
-  return (int64_t)B * (N / C) * H * d * (d + 1);
+  return (int64_t)B * (N / C) * H * d * (d + 2);
 }
 
 int lasp_gla_chunk_states(const void* x, const void* y, const float* g, float* M, float* gsum, int B, int H,
@@ -94,18 +99,25 @@ int lasp_gla_fwd(const void* q, const void* k, const void* v, const float* g, vo
   const int T = (int)(N / C);
   float* gsum = state_cache + (int64_t)B * T * H * d * d;
   if (tc_gla_ok(dtype, d, C, N)) {
-    // 128-token tiles: their states and log-gate totals into the slots of each
-    // tile's first chunk, the prefix over tiles in place, then the output
+    // segments of S 128-token tiles: their states and log-gate totals into the
+    // slots of each segment's first chunk (the tiles' own totals into their
+    // slots, for the backward), the prefix over segments in place, then the
+    // walk through each segment's tiles
     const int stride = 128 / C;
-    const int tiles = (int)(N / 128);
-    if ((s = cuda_status(traced(K_GLA_STATES_TC, st, [&] {
-           return tc_gla_chunk_states(k, v, g, state_cache, gsum, B, H, N, 0, T, stride, 0, st);
+    const int S = walk_segment_tokens(N, 128) / 128;
+    const int nseg = (int)(N / 128) / S;
+    float* gseg = gsum + (int64_t)B * T * H * d;
+    if ((s = cuda_status(traced(K_GLA_SEG_STATES, st, [&] {
+           return tc_gla_chunk_states(k, v, g, state_cache, gseg, gsum, B, H, N, 0, T, S * stride, 0, S, stride, st);
          }))))
       return s;
-    if ((s = scan_impl(state_cache, state_cache, gsum, init_state, nullptr, B, tiles, H, d, 0, T, stride, 0, 0, st)))
+    if ((s = cuda_status(traced(K_GLA_SEG_SCAN, st, [&] {
+           return launch_gla_scan(state_cache, state_cache, gseg, init_state, nullptr, B, nseg, H, d, 0, T, S * stride,
+                                  0, 0, st);
+         }))))
       return s;
     return cuda_status(traced(K_GLA_OUT_TC, st, [&] {
-      return tc_gla_chunk_out(q, k, v, g, state_cache, o, B, H, N, T, stride, st);
+      return tc_gla_chunk_out(q, k, v, g, state_cache, o, B, H, N, T, stride, S, st);
     }));
   }
   // 1. chunk states M_c and log-gate totals; 2. exclusive prefix in place -> P_c; 3. output
@@ -134,7 +146,8 @@ int lasp_gla_bwd(const void* q, const void* k, const void* v, const float* g, co
     const int stride = 128 / C;
     const int tiles = (int)(N / 128);
     if ((s = cuda_status(traced(K_GLA_STATES_TC, st, [&] {
-           return tc_gla_chunk_states(q, dout, g, dstate_ws, nullptr, B, H, N, 1, T, stride, stride - 1, st);
+           return tc_gla_chunk_states(q, dout, g, dstate_ws, nullptr, nullptr, B, H, N, 1, T, stride, stride - 1, 1, stride,
+                                      st);
          }))))
       return s;
     if ((s = scan_impl(dstate_ws, dstate_ws, gsum, dstate_in, dinit_state, B, tiles, H, d, 1, T, stride, stride - 1, 0,
