@@ -422,9 +422,9 @@ LASP_API int lasp_gla_state_prefix(const float* M, float* Mprefix, const float* 
  *   o_t = (q_t . exp(b_t)) P_c + sum_{s<=t} (sum_i q_t[i] k_s[i] exp(b_t[i] - b_s[i])) v_s.
  *   state_cache: out, lasp_gla_cache_floats(...) floats; pass it unchanged to
  *                lasp_gla_bwd. Required. Its encoding inside a slot is
- *                internal to the library (on the tensor-core path a tile's
- *                slot ends up holding the bf16 operand tile its backward
- *                loads).
+ *                internal to the library (the tensor-core path keeps states
+ *                per segment of about 1024 tokens, and a tile's slot ends up
+ *                holding the bf16 operand tile its backward loads).
  *   init_state:  in, float [B, H, d, d] or NULL, the state entering token 0.
  */
 LASP_API int lasp_gla_fwd(const void* q, const void* k, const void* v, const float* g, void* o, int B, int H,

@@ -1,11 +1,14 @@
 // Tensor-core kernels of the gated form (a decay per token and key feature;
 // LASP Appendix A.4, Eq. 24 with the GLA / GateLoop row of Table 5), bf16,
-// d = 128, over 128-token tiles (one per CTA; the backward's persistent CTAs
-// take one after another). A tile spans 128/C chunks (C dividing
-// 128); its masked products regroup the per-chunk intra and inter terms, so it
+// d = 128, over 128-token tiles. A tile spans 128/C chunks (C dividing 128);
+// its masked products regroup the per-chunk intra and inter terms, so it
 // follows the chunk equations of k_gla_simt.cu with the tile as the chunk
 // (b_t = inclusive cumulative log-gate from the tile start, b_end its last
-// row), the states being needed at tile boundaries only.
+// row), the states being needed at tile boundaries only. The forward works on
+// segments of tiles: the state kernel sums each segment's tiles into one
+// state, and the output kernel walks each segment's tiles with the state in
+// TMEM. The backward takes one tile at a time (per-tile states; its persistent
+// CTAs take one tile after another).
 //
 // The intra-tile products need the factor e^{b_t[i] - b_s[i]} inside a
 // contraction over i, which a single MMA can carry only if it splits into a
@@ -336,6 +339,15 @@ __device__ __forceinline__ void gate_rows(float* bt, uint64_t* gbar, uint32_t pa
 }
 
 // ---------------------------------------------------------------- output
+// One persistent CTA per SM walks segments of `tiles` tiles (tiles = 1: every
+// tile on its own, its entering state from the cache). At a segment's first
+// tile the state P entering the segment arrives from the cache slot by TMA.
+// Each tile then forms P' = diag(e^{r}) P, the bf16 operand of the inter term
+// (also stored in the tile's cache slot for the backward) and, inside a
+// segment, the fp32 accumulator in TMEM onto which the last MMA adds K^^T V.
+// The next tile multiplies that accumulator by e^{b_end - r} of this tile,
+// which gives its entering state. TMEM: T0 = Q^K^^T, T1 = the output,
+// TP = the state.
 struct SmemOut {
   uint64_t gload, load, ldp, mma1, mma2;
   uint32_t tmem_base;
