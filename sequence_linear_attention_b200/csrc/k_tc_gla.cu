@@ -160,17 +160,20 @@ struct SmemStates {
 // every factor stays at most 1 for log-gates <= 0. gsum (kind 0, may be NULL)
 // receives the item's total log-gate in the item's slot; gsum_tile (may be
 // NULL) every tile's own total in the slot of tile c, c * tstride.
+// kOne: one tile per CTA (tiles = 1 at compile time).
+template <bool kOne>
 __global__ void __launch_bounds__(kThreads, 2) gla_states_tc(const __grid_constant__ CUtensorMap map_x,
                                                              const __grid_constant__ CUtensorMap map_y,
                                                              const float* __restrict__ g, float* __restrict__ M,
                                                              float* __restrict__ gsum, float* __restrict__ gsum_tile,
                                                              int H, int64_t N, int kind, int64_t t_slots, int stride,
-                                                             int offset, int tiles, int tstride) {
+                                                             int offset, int tiles_arg, int tstride) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   uint8_t* sX = base;
   uint8_t* sY = base + kTileBytes;
   SmemStates* s = reinterpret_cast<SmemStates*>(base + 2 * kTileBytes);
+  const int tiles = kOne ? 1 : tiles_arg;
   const int item = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int64_t sl = (int64_t)b * t_slots + (int64_t)item * stride + offset;  // the state slot of this item
@@ -1133,10 +1136,11 @@ cudaError_t tc_gla_chunk_states(const void* x, const void* y, const float* g, fl
   if (!make_token_map(&mx, x, B, H, N, kD, kTile) || !make_token_map(&my, y, B, H, N, kD, kTile))
     return cudaErrorInvalidValue;
   const size_t smem = 1024 + 2 * (size_t)kTileBytes + sizeof(SmemStates);
-  cudaError_t e = cudaFuncSetAttribute(gla_states_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  if (e != cudaSuccess) return e;
   if (tiles < 1 || N % ((int64_t)tiles * kTile) != 0) return cudaErrorInvalidValue;
-  gla_states_tc<<<dim3((unsigned)(N / ((int64_t)tiles * kTile)), H, B), kThreads, smem, st>>>(
+  auto kern = tiles == 1 ? gla_states_tc<true> : gla_states_tc<false>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  kern<<<dim3((unsigned)(N / ((int64_t)tiles * kTile)), H, B), kThreads, smem, st>>>(
       mx, my, g, M, gsum, gsum_tile, H, N, kind, t_slots, stride, offset, tiles, tstride);
   return cudaGetLastError();
 }
