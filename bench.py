@@ -111,8 +111,8 @@ MEASURED_TRAFFIC = {
     "segment_states_tc": (["k_tc_states.cu", "sm100.cuh", "lasp_common.cuh", "tma_host.h"], "fc6351767f0401ee",
                           2 * (268477696 + 5350400)),
     # the gated form (bench.py --gated): four times the capture of the 16384-token case
-    "gla_bwd_tc": (["k_tc_gla.cu", "sm100.cuh", "lasp_common.cuh", "tma_host.h"], "8e102d448d308a2a",
-                   4 * (606502144 + 291366144)),
+    "gla_bwd_tc": (["k_tc_gla.cu", "sm100.cuh", "lasp_common.cuh", "tma_host.h"], "f75bccb6c192eda9",
+                   4 * (606049024 + 294287872)),
 }
 
 
