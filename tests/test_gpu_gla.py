@@ -182,7 +182,11 @@ def test_rows_chunk_states_and_scans(bf16):
 
 
 # ------------------------------------------------ tensor-core path (bf16, d = 128, C = 128)
-@pytest.mark.parametrize("B,N,H,tau,seed", [(2, 1024, 2, 16.0, 2020), (1, 512, 3, 1.0, 2021), (1, 2048, 1, 4.0, 2022)])
+# the forward walks segments of up to 8 tiles: 1024 and 2048 tokens give 8-tile
+# segments (one and two per head), 512 one 4-tile segment, 1152 three 3-tile
+# segments, 1408 (11 tiles) eleven one-tile segments
+@pytest.mark.parametrize("B,N,H,tau,seed", [(2, 1024, 2, 16.0, 2020), (1, 512, 3, 1.0, 2021), (1, 2048, 1, 4.0, 2022),
+                                            (1, 1152, 2, 4.0, 2023), (2, 1408, 1, 2.0, 2024)])
 def test_tensor_core_path_matches_oracle(B, N, H, tau, seed):
     d, C = 128, 128
     inp = lasp_inputs.make_inputs(B, N, H, d, seed=seed, bf16=True, decayed=False)
