@@ -56,3 +56,22 @@ def test_single_rank_needs_no_process_group():
     # chunks inside a tile: one cached bf16 tile per 128 tokens whatever C is
     assert bench.algorithmic_bytes("fwd_walk_tc", 1, 128, 64, 1024, 2) == 4 * 128 * 2 + s4 / 1024 + s4 / 256
     assert bench.algorithmic_bytes("bwd_walk_tc", 1, 128, 32, 1024, 2) == 7 * 128 * 2 + s4 / 256 + s4 / 1024
+
+
+def test_algorithmic_bytes_of_the_segment_kernels():
+    """Bytes per token-head of the kernels that work per segment of G tokens:
+    the state total reads the segment states once; the gated forward's segment
+    states write one state per segment; its walk reads one state per segment
+    and writes a bf16 state tile per 128 tokens."""
+    sys.path.insert(0, ROOT)
+    import bench
+    d, G, e = 128, 1024, 2
+    s = 4 * d * d
+    assert bench.algorithmic_bytes("state_total", 1, d, 128, G, e) == s / G
+    assert bench.algorithmic_bytes("gla_segment_states_tc", 1, d, 128, G, e) == 2 * d * e + 4 * d + s / G
+    assert bench.algorithmic_bytes("gla_segment_scan", 1, d, 128, G, e) == 2 * s / G + 4 * d / G
+    assert bench.algorithmic_bytes("gla_out_tc", 1, d, 128, G, e) == 4 * d * e + 4 * d + s / G + s / 256
+    assert bench.algorithmic_bytes("gla_bwd_tc", 1, d, 128, G, e) == 7 * d * e + 8 * d + s / 256 + s / 128
+    # per-tile kernels do not depend on the segment
+    assert bench.algorithmic_bytes("gla_states_tc", 1, d, 128, G, e) == bench.algorithmic_bytes(
+        "gla_states_tc", 1, d, 128, 128, e)
