@@ -117,7 +117,7 @@ MEASURED_TRAFFIC = {
 
 
 def measured_traffic(kernel: str, workload: str):
-    """Recorded DRAM bytes per launch, or None if not captured for this build."""
+    """Recorded DRAM bytes per launch, or None if not captured for the current kernel sources."""
     import hashlib
     if workload != DEFAULT_WORKLOAD or kernel not in MEASURED_TRAFFIC:
         return None

@@ -57,7 +57,7 @@ extern "C" {
 typedef enum {
   LASP_OK = 0,
   LASP_ERR_INVALID_ARG = 1, /* bad size, NULL required pointer, bad dtype */
-  LASP_ERR_UNSUPPORTED = 2, /* a size this build has no kernel for (e.g. d = 96) */
+  LASP_ERR_UNSUPPORTED = 2, /* a size the library has no kernel for (e.g. d = 96) */
   LASP_ERR_MISALIGNED = 3,  /* a pointer not 16-byte aligned */
   LASP_ERR_CUDA = 4,        /* a CUDA runtime error (launch failure, no device) */
   LASP_ERR_TIMEOUT = 5      /* a device-side wait exceeded its limit */
