@@ -111,8 +111,8 @@ MEASURED_TRAFFIC = {
     "segment_states_tc": (["k_tc_states.cu", "sm100.cuh", "lasp_common.cuh", "tma_host.h"], "fc6351767f0401ee",
                           2 * (268477696 + 5350400)),
     # the gated form (bench.py --gated): four times the capture of the 16384-token case
-    "gla_bwd_tc": (["k_tc_gla.cu", "sm100.cuh", "lasp_common.cuh", "tma_host.h"], "f75bccb6c192eda9",
-                   4 * (606049024 + 294287872)),
+    "gla_bwd_tc": (["k_tc_gla.cu", "sm100.cuh", "lasp_common.cuh", "tma_host.h"], "039f7de455c9c750",
+                   4 * (605879552 + 294130688)),
 }
 
 

@@ -493,9 +493,12 @@ __global__ void __launch_bounds__(kThreads, 1) gla_out_tc(const __grid_constant_
       float v[64];
       if (j == 0) {
         const bool pok = mbar_wait(&s->ldp, pph, SITE_OUT_TMA);
-        pph ^= 1u;
-        if (!pok) s->abort = 1;
-        if (tid == 0 && pok) p_ahead = false;  // else cleanup waits for it once more
+        if (pok) {
+          pph ^= 1u;
+          if (tid == 0) p_ahead = false;
+        } else {
+          s->abort = 1;  // cleanup waits for this phase once more
+        }
         const uint8_t* src = reinterpret_cast<const uint8_t*>(bt) + 2 * half * (kTile * 128);
 #pragma unroll
         for (int bb = 0; bb < 2; ++bb)
