@@ -19,6 +19,8 @@ namespace noalloc_detail {
 // library until the process exits. Enough for B * (N / C) * H <= 512 states
 // of d = 128.
 constexpr size_t kScratchBytes = (size_t)32 << 20;
+static_assert(kScratchBytes == (size_t)LASP_NOALLOC_SCRATCH_BYTES,
+              "the workspace size must equal the limit the header publishes");
 static __device__ __align__(256) float g_bwd_scratch[kScratchBytes / sizeof(float)];
 
 constexpr int kMaxDevices = 64;

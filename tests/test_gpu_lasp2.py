@@ -20,9 +20,11 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 pytestmark = pytest.mark.gpu
 
 # (W, B, L, H, d, C, bf16, decayed): the tensor-core walks (bf16, d = 128) and
-# the CUDA-core path (fp32)
+# the CUDA-core path (fp32); decayed is True (the workloads' per-head rates),
+# or one lambda for every head
 CASES = {
     "bf16_W2": (2, 2, 1024, 4, 128, 128, True, True),
+    "bf16_W2_lam0.5": (2, 1, 1024, 4, 128, 128, True, 0.5),
     "bf16_W3_C64": (3, 1, 512, 2, 128, 64, True, True),
     "f32_W2": (2, 1, 256, 2, 64, 64, False, True),
 }
@@ -38,7 +40,9 @@ def _inputs(name):
     from sequence_linear_attention_b200 import inputs as lasp_inputs
     W, B, L, H, d, C, bf16, decayed = CASES[name]
     inp = lasp_inputs.make_inputs(B, W * L, H, d, seed=3300 + sorted(CASES).index(name), bf16=bf16,
-                                  decayed=decayed)
+                                  decayed=decayed is True)
+    if decayed is not True:
+        inp["lam"] = np.full(H, decayed, np.float32)
     rng = np.random.default_rng(3400 + sorted(CASES).index(name))
     init = (rng.standard_normal((B, H, d, d)) * 0.1).astype(np.float32)
     dsin = (rng.standard_normal((B, H, d, d)) * 0.1).astype(np.float32)
