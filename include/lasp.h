@@ -378,11 +378,13 @@ LASP_API int lasp_bidir_bwd(const void* q, const void* k, const void* v, const v
  * Chunks: 1 <= C <= 128, C divides N (LASP_ERR_UNSUPPORTED for C > 128).
  * bf16 with d = 128, C dividing 128 and N a multiple of 128 runs on the tensor
  * cores, which factor the decay inside each 128-token tile around the tile's
- * middle token: that needs the log-gates of each 64-token half of a tile to
- * sum to at least -80 (gates far stronger than any that leave the state
- * anything to carry); a tile beyond that records LASP_ERR_INVALID_ARG in the
- * device status. Every other case (fp32 in particular) runs exact CUDA-core
- * kernels with no such limit. In
+ * middle token: that holds while the |log-gates| of each 64-token half of a
+ * tile sum to at most 79. lasp_gla_fwd checks every tile on the device; when
+ * one is beyond that (gates far stronger than any that leave the state
+ * anything to carry), the call, and the lasp_gla_bwd given its cache, run the
+ * exact CUDA-core kernels instead (slower, same results; no status is
+ * recorded and the host is not synchronised). Every other case (fp32 in
+ * particular) runs those CUDA-core kernels. In
  * chunk c, b_t = sum_{r<=t} g_{cC+r} (from the chunk start) and the chunk's
  * total log-gate is gsum_c = b_{C-1}. The states of the gated form:
  *   kind 0, (x, y) = (k, v):   M_c  = sum_t diag(exp(gsum_c - b_t)) k_t^T v_t
@@ -393,7 +395,8 @@ LASP_API int lasp_bidir_bwd(const void* q, const void* k, const void* v, const v
  */
 
 /* Size, in floats, of the state cache of lasp_gla_fwd / lasp_gla_bwd:
- * B * (N/C) * H * d * (d + 2). -1 for sizes the gated calls reject. */
+ * B * (N/C) * H * d * (d + 2) + 4 (the last four hold the forward's choice of
+ * kernels, read by the backward). -1 for sizes the gated calls reject. */
 LASP_API int64_t lasp_gla_cache_floats(int B, int H, int64_t N, int d, int C);
 
 /*

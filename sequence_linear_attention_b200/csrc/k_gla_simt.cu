@@ -75,16 +75,19 @@ __device__ __forceinline__ void cumulative_gates(const float* __restrict__ g, fl
 template <typename T, int D>
 __global__ void __launch_bounds__(256) gla_states_simt(const T* __restrict__ x, const T* __restrict__ y,
                                                        const float* __restrict__ g, float* __restrict__ M,
-                                                       float* __restrict__ gsum, int H, int64_t N, int C,
-                                                       int kind) {
+                                                       float* __restrict__ gsum, int B, int H, int64_t N, int C,
+                                                       int kind, RunIf run_if) {
+  if (!runs(run_if)) return;
   constexpr int TB = 32;
   constexpr int R = D * D / 256;
   extern __shared__ float smem[];
   float* cb = smem;       // [C][D]
   float* xs = cb + C * D;  // [TB][D], gate-weighted x
   float* ys = xs + TB * D;  // [TB][D]
-  const int c = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const int64_t nchunks = N / C;
+  const int64_t items = nchunks * H * (int64_t)B;
+  for (int64_t item = blockIdx.x; item < items; item += gridDim.x) {
+  const int c = (int)(item % nchunks), h = (int)((item / nchunks) % H), b = (int)(item / (nchunks * H));
   const int64_t slot = ((int64_t)b * nchunks + c) * H + h;
   cumulative_gates<D>(g, cb, gsum ? gsum + slot * D : nullptr, b, c, h, H, N, C);
   const float* cend = cb + (C - 1) * D;
@@ -119,18 +122,23 @@ __global__ void __launch_bounds__(256) gla_states_simt(const T* __restrict__ x, 
   float* out = M + slot * D * D;
 #pragma unroll
   for (int r = 0; r < R; ++r) out[threadIdx.x + 256 * r] = acc[r];
+  __syncthreads();  // the next item rewrites the shared arrays
+  }
 }
 
 template <typename T, int D>
 __global__ void __launch_bounds__(kWarps * 32) gla_out_simt(const T* __restrict__ q, const T* __restrict__ k,
                                                             const T* __restrict__ v, const float* __restrict__ g,
-                                                            const float* __restrict__ P, T* __restrict__ o, int H,
-                                                            int64_t N, int C) {
+                                                            const float* __restrict__ P, T* __restrict__ o, int B,
+                                                            int H, int64_t N, int C, RunIf run_if) {
+  if (!runs(run_if)) return;
   constexpr int R = D / 32;
   extern __shared__ float cb[];  // [C][D]
-  const int c = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int64_t nchunks = N / C;
+  const int64_t items = nchunks * H * (int64_t)B;
+  for (int64_t item = blockIdx.x; item < items; item += gridDim.x) {
+  const int c = (int)(item % nchunks), h = (int)((item / nchunks) % H), b = (int)(item / (nchunks * H));
   cumulative_gates<D>(g, cb, nullptr, b, c, h, H, N, C);
   const float* Pc = P + (((int64_t)b * nchunks + c) * H + h) * D * D;
   for (int i = warp; i < C; i += kWarps) {
@@ -169,6 +177,8 @@ __global__ void __launch_bounds__(kWarps * 32) gla_out_simt(const T* __restrict_
 #pragma unroll
     for (int r = 0; r < R; ++r) Elem<T>::store(oi + lane + 32 * r, acc[r]);
   }
+  __syncthreads();  // the next item rewrites the cumulative gates
+  }
 }
 
 template <typename T, int D>
@@ -177,15 +187,19 @@ __global__ void __launch_bounds__(kWarps * 32) gla_bwd_simt(const T* __restrict_
                                                             const float* __restrict__ g, const float* __restrict__ P,
                                                             const float* __restrict__ Rs, T* __restrict__ dq,
                                                             T* __restrict__ dk, T* __restrict__ dv,
-                                                            float* __restrict__ dg, int H, int64_t N, int C) {
+                                                            float* __restrict__ dg, int B, int H, int64_t N, int C,
+                                                            RunIf run_if) {
+  if (!runs(run_if)) return;
   constexpr int R = D / 32;
   extern __shared__ float smem[];
   float* cb = smem;          // [C][D] cumulative log-gates (times log2 e)
   float* dB = cb + C * D;    // [C][D] q . dq' - k . dk' of each token
   float* kdi = dB + C * D;   // [C][D] k . dk^inter of each token
-  const int c = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int64_t nchunks = N / C;
+  const int64_t items = nchunks * H * (int64_t)B;
+  for (int64_t item = blockIdx.x; item < items; item += gridDim.x) {
+  const int c = (int)(item % nchunks), h = (int)((item / nchunks) % H), b = (int)(item / (nchunks * H));
   cumulative_gates<D>(g, cb, nullptr, b, c, h, H, N, C);
   const float* cend = cb + (C - 1) * D;
   const float* Pc = P + (((int64_t)b * nchunks + c) * H + h) * D * D;
@@ -313,6 +327,8 @@ __global__ void __launch_bounds__(kWarps * 32) gla_bwd_simt(const T* __restrict_
       dg[(((int64_t)b * N + (int64_t)c * C + t) * H + h) * D + f] = run + kdi[t * D + f] + bnd;
     }
   }
+  __syncthreads();  // the next item rewrites the shared arrays
+  }
 }
 
 template <typename K>
@@ -323,91 +339,92 @@ cudaError_t set_smem(K kernel, size_t bytes) {
 
 template <typename T, int D>
 cudaError_t launch_states_d(const void* x, const void* y, const float* g, float* M, float* gsum, int B, int H,
-                            int64_t N, int C, int kind, cudaStream_t st) {
+                            int64_t N, int C, int kind, cudaStream_t st, RunIf run) {
   const size_t smem = (size_t)(C + 64) * D * sizeof(float);
   cudaError_t e = set_smem(gla_states_simt<T, D>, smem);
   if (e != cudaSuccess) return e;
-  gla_states_simt<T, D><<<dim3((unsigned)(N / C), H, B), 256, smem, st>>>((const T*)x, (const T*)y, g, M, gsum, H,
-                                                                          N, C, kind);
+  gla_states_simt<T, D><<<(unsigned)grid_for(N / C * H * B, run), 256, smem, st>>>((const T*)x, (const T*)y, g, M, gsum, B, H,
+                                                                          N, C, kind, run);
   return cudaGetLastError();
 }
 
 template <typename T, int D>
 cudaError_t launch_out_d(const void* q, const void* k, const void* v, const float* g, const float* P, void* o,
-                         int B, int H, int64_t N, int C, cudaStream_t st) {
+                         int B, int H, int64_t N, int C, cudaStream_t st, RunIf run) {
   const size_t smem = (size_t)C * D * sizeof(float);
   cudaError_t e = set_smem(gla_out_simt<T, D>, smem);
   if (e != cudaSuccess) return e;
-  gla_out_simt<T, D><<<dim3((unsigned)(N / C), H, B), kWarps * 32, smem, st>>>(
-      (const T*)q, (const T*)k, (const T*)v, g, P, (T*)o, H, N, C);
+  gla_out_simt<T, D><<<(unsigned)grid_for(N / C * H * B, run), kWarps * 32, smem, st>>>(
+      (const T*)q, (const T*)k, (const T*)v, g, P, (T*)o, B, H, N, C, run);
   return cudaGetLastError();
 }
 
 template <typename T, int D>
 cudaError_t launch_bwd_d(const void* q, const void* k, const void* v, const void* dout, const float* g,
                          const float* P, const float* Rs, void* dq, void* dk, void* dv, float* dg, int B, int H,
-                         int64_t N, int C, cudaStream_t st) {
+                         int64_t N, int C, cudaStream_t st, RunIf run) {
   const size_t smem = (size_t)3 * C * D * sizeof(float);
   cudaError_t e = set_smem(gla_bwd_simt<T, D>, smem);
   if (e != cudaSuccess) return e;
-  gla_bwd_simt<T, D><<<dim3((unsigned)(N / C), H, B), kWarps * 32, smem, st>>>(
-      (const T*)q, (const T*)k, (const T*)v, (const T*)dout, g, P, Rs, (T*)dq, (T*)dk, (T*)dv, dg, H, N, C);
+  gla_bwd_simt<T, D><<<(unsigned)grid_for(N / C * H * B, run), kWarps * 32, smem, st>>>(
+      (const T*)q, (const T*)k, (const T*)v, (const T*)dout, g, P, Rs, (T*)dq, (T*)dk, (T*)dv, dg, B, H, N, C, run);
   return cudaGetLastError();
 }
 
 template <typename T>
 cudaError_t launch_states(const void* x, const void* y, const float* g, float* M, float* gsum, int B, int H,
-                          int64_t N, int d, int C, int kind, cudaStream_t st) {
+                          int64_t N, int d, int C, int kind, cudaStream_t st, RunIf run) {
   switch (d) {
-    case 32: return launch_states_d<T, 32>(x, y, g, M, gsum, B, H, N, C, kind, st);
-    case 64: return launch_states_d<T, 64>(x, y, g, M, gsum, B, H, N, C, kind, st);
-    default: return launch_states_d<T, 128>(x, y, g, M, gsum, B, H, N, C, kind, st);
+    case 32: return launch_states_d<T, 32>(x, y, g, M, gsum, B, H, N, C, kind, st, run);
+    case 64: return launch_states_d<T, 64>(x, y, g, M, gsum, B, H, N, C, kind, st, run);
+    default: return launch_states_d<T, 128>(x, y, g, M, gsum, B, H, N, C, kind, st, run);
   }
 }
 
 template <typename T>
 cudaError_t launch_out(const void* q, const void* k, const void* v, const float* g, const float* P, void* o, int B,
-                       int H, int64_t N, int d, int C, cudaStream_t st) {
+                       int H, int64_t N, int d, int C, cudaStream_t st, RunIf run) {
   switch (d) {
-    case 32: return launch_out_d<T, 32>(q, k, v, g, P, o, B, H, N, C, st);
-    case 64: return launch_out_d<T, 64>(q, k, v, g, P, o, B, H, N, C, st);
-    default: return launch_out_d<T, 128>(q, k, v, g, P, o, B, H, N, C, st);
+    case 32: return launch_out_d<T, 32>(q, k, v, g, P, o, B, H, N, C, st, run);
+    case 64: return launch_out_d<T, 64>(q, k, v, g, P, o, B, H, N, C, st, run);
+    default: return launch_out_d<T, 128>(q, k, v, g, P, o, B, H, N, C, st, run);
   }
 }
 
 template <typename T>
 cudaError_t launch_bwd(const void* q, const void* k, const void* v, const void* dout, const float* g,
                        const float* P, const float* Rs, void* dq, void* dk, void* dv, float* dg, int B, int H,
-                       int64_t N, int d, int C, cudaStream_t st) {
+                       int64_t N, int d, int C, cudaStream_t st, RunIf run) {
   switch (d) {
-    case 32: return launch_bwd_d<T, 32>(q, k, v, dout, g, P, Rs, dq, dk, dv, dg, B, H, N, C, st);
-    case 64: return launch_bwd_d<T, 64>(q, k, v, dout, g, P, Rs, dq, dk, dv, dg, B, H, N, C, st);
-    default: return launch_bwd_d<T, 128>(q, k, v, dout, g, P, Rs, dq, dk, dv, dg, B, H, N, C, st);
+    case 32: return launch_bwd_d<T, 32>(q, k, v, dout, g, P, Rs, dq, dk, dv, dg, B, H, N, C, st, run);
+    case 64: return launch_bwd_d<T, 64>(q, k, v, dout, g, P, Rs, dq, dk, dv, dg, B, H, N, C, st, run);
+    default: return launch_bwd_d<T, 128>(q, k, v, dout, g, P, Rs, dq, dk, dv, dg, B, H, N, C, st, run);
   }
 }
 
 }  // namespace gla_simt_detail
 
 cudaError_t gla_simt_chunk_states(const void* x, const void* y, const float* g, float* M, float* gsum, int B, int H,
-                                  int64_t N, int d, int C, int kind, int dtype, cudaStream_t st) {
+                                  int64_t N, int d, int C, int kind, int dtype, cudaStream_t st, RunIf run) {
   using namespace gla_simt_detail;
-  return dtype == LASP_F32 ? launch_states<float>(x, y, g, M, gsum, B, H, N, d, C, kind, st)
-                           : launch_states<__nv_bfloat16>(x, y, g, M, gsum, B, H, N, d, C, kind, st);
+  return dtype == LASP_F32 ? launch_states<float>(x, y, g, M, gsum, B, H, N, d, C, kind, st, run)
+                           : launch_states<__nv_bfloat16>(x, y, g, M, gsum, B, H, N, d, C, kind, st, run);
 }
 
 cudaError_t gla_simt_chunk_out(const void* q, const void* k, const void* v, const float* g, const float* P, void* o,
-                               int B, int H, int64_t N, int d, int C, int dtype, cudaStream_t st) {
+                               int B, int H, int64_t N, int d, int C, int dtype, cudaStream_t st, RunIf run) {
   using namespace gla_simt_detail;
-  return dtype == LASP_F32 ? launch_out<float>(q, k, v, g, P, o, B, H, N, d, C, st)
-                           : launch_out<__nv_bfloat16>(q, k, v, g, P, o, B, H, N, d, C, st);
+  return dtype == LASP_F32 ? launch_out<float>(q, k, v, g, P, o, B, H, N, d, C, st, run)
+                           : launch_out<__nv_bfloat16>(q, k, v, g, P, o, B, H, N, d, C, st, run);
 }
 
 cudaError_t gla_simt_chunk_bwd(const void* q, const void* k, const void* v, const void* dout, const float* g,
                                const float* P, const float* Rs, void* dq, void* dk, void* dv, float* dg, int B, int H,
-                               int64_t N, int d, int C, int dtype, cudaStream_t st) {
+                               int64_t N, int d, int C, int dtype, cudaStream_t st, RunIf run) {
   using namespace gla_simt_detail;
-  return dtype == LASP_F32 ? launch_bwd<float>(q, k, v, dout, g, P, Rs, dq, dk, dv, dg, B, H, N, d, C, st)
-                           : launch_bwd<__nv_bfloat16>(q, k, v, dout, g, P, Rs, dq, dk, dv, dg, B, H, N, d, C, st);
+  return dtype == LASP_F32 ? launch_bwd<float>(q, k, v, dout, g, P, Rs, dq, dk, dv, dg, B, H, N, d, C, st, run)
+                           : launch_bwd<__nv_bfloat16>(q, k, v, dout, g, P, Rs, dq, dk, dv, dg, B, H, N, d, C, st,
+                                                       run);
 }
 
 }  // namespace lasp

@@ -50,9 +50,10 @@ __global__ void __launch_bounds__(kThreads) state_scan_kernel(const float4* M, f
                                                               float4* __restrict__ total, int H, int T,
                                                               int d, int dd4, int64_t n_threads, float Cf,
                                                               int reverse, int64_t t_slots, int slot_stride,
-                                                              int slot_offset, int gsum_offset) {
-  const int64_t idx = (int64_t)blockIdx.x * kThreads + threadIdx.x;
-  if (idx >= n_threads) return;
+                                                              int slot_offset, int gsum_offset, RunIf run_if) {
+  if (!runs(run_if)) return;
+  for (int64_t idx = (int64_t)blockIdx.x * kThreads + threadIdx.x; idx < n_threads;
+       idx += (int64_t)gridDim.x * kThreads) {
   const int e = (int)(idx % dd4);
   const int h = (int)((idx / dd4) % H);
   const int64_t b = idx / ((int64_t)dd4 * H);
@@ -120,6 +121,7 @@ __global__ void __launch_bounds__(kThreads) state_scan_kernel(const float4* M, f
     goff += gstep;
   }
   if (total) total[bh * dd4 + e] = acc;
+  }
 }
 
 }  // namespace scan_detail
@@ -132,19 +134,19 @@ cudaError_t launch_state_scan_slots(const float* M, float* P, const float* decay
   const int64_t blocks = (n_threads + scan_detail::kThreads - 1) / scan_detail::kThreads;
   scan_detail::state_scan_kernel<false><<<(unsigned)blocks, scan_detail::kThreads, 0, st>>>(
       (const float4*)M, (float4*)P, decay, nullptr, (const float4*)init, (float4*)total, H, T, d, dd4,
-      n_threads, (float)C, reverse, t_slots, slot_stride, slot_offset, 0);
+      n_threads, (float)C, reverse, t_slots, slot_stride, slot_offset, 0, RunIf{});
   return cudaGetLastError();
 }
 
 cudaError_t launch_gla_scan(const float* M, float* P, const float* gsum, const float* init, float* total, int B,
                             int T, int H, int d, int reverse, int64_t t_slots, int slot_stride, int slot_offset,
-                            int gsum_offset, cudaStream_t st) {
+                            int gsum_offset, cudaStream_t st, RunIf run) {
   const int dd4 = d * d / 4;
   const int64_t n_threads = (int64_t)B * H * dd4;
-  const int64_t blocks = (n_threads + scan_detail::kThreads - 1) / scan_detail::kThreads;
+  const int64_t blocks = grid_for((n_threads + scan_detail::kThreads - 1) / scan_detail::kThreads, run);
   scan_detail::state_scan_kernel<true><<<(unsigned)blocks, scan_detail::kThreads, 0, st>>>(
       (const float4*)M, (float4*)P, nullptr, gsum, (const float4*)init, (float4*)total, H, T, d, dd4, n_threads,
-      1.f, reverse, t_slots, slot_stride, slot_offset, gsum_offset);
+      1.f, reverse, t_slots, slot_stride, slot_offset, gsum_offset, run);
   return cudaGetLastError();
 }
 

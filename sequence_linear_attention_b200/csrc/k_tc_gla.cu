@@ -55,6 +55,10 @@ constexpr uint32_t kTileBytes = kTile * kD * 2;
 constexpr uint32_t kBox = kTileBytes / 2;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kMaxSpan = 80.f;  // largest |b_t - r| (natural log) the factorized form takes
+// the state kernel's bound on a half-tile's sum of |log-gate|: a little under
+// kMaxSpan, so that no rounding of the two different sums lets a tile past it
+// that the output and backward kernels would then reject
+constexpr float kSpanCheck = kMaxSpan - 1.f;
 constexpr uint32_t kBarAll = 1;   // named barrier over all 256 threads
 
 
@@ -142,6 +146,7 @@ struct SmemStates {
   uint32_t tmem_base;
   int abort;
   alignas(16) float grp[8][kD];  // the log-gates of each feature summed over each 16-row group (float4 access)
+  alignas(16) float grp_abs[8][kD];  // the same sums of |log-gate| (the span check)
 };
 
 // kind 0: M_c = (k . e^{b_end - b})^T v and gsum_c = b_end; kind 1: dM_c =
@@ -167,7 +172,9 @@ __global__ void __launch_bounds__(kThreads, 2) gla_states_tc(const __grid_consta
                                                              const float* __restrict__ g, float* __restrict__ M,
                                                              float* __restrict__ gsum, float* __restrict__ gsum_tile,
                                                              int H, int64_t N, int kind, int64_t t_slots, int stride,
-                                                             int offset, int tiles_arg, int tstride) {
+                                                             int offset, int tiles_arg, int tstride,
+                                                             int* __restrict__ span_flag, RunIf run_if) {
+  if (!runs(run_if)) return;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   uint8_t* sX = base;
@@ -222,6 +229,17 @@ __global__ void __launch_bounds__(kThreads, 2) gla_states_tc(const __grid_consta
       tot.w += gv[u].w;
     }
     *reinterpret_cast<float4*>(&s->grp[warp][f0]) = tot;
+    if (span_flag != nullptr) {
+      float4 ab = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+      for (int u = 0; u < 16; ++u) {
+        ab.x += fabsf(gv[u].x);
+        ab.y += fabsf(gv[u].y);
+        ab.z += fabsf(gv[u].z);
+        ab.w += fabsf(gv[u].w);
+      }
+      *reinterpret_cast<float4*>(&s->grp_abs[warp][f0]) = ab;
+    }
     const bool ok = mbar_wait(&s->load, par, SITE_STATES_TMA);
     if (!ok) s->abort = 1;
     __syncthreads();
@@ -246,6 +264,20 @@ __global__ void __launch_bounds__(kThreads, 2) gla_states_tc(const __grid_consta
     off.y += all.y;
     off.z += all.z;
     off.w += all.w;
+    if (span_flag != nullptr && warp < 2) {
+      // warp 0 the tile's first half, warp 1 its second: the sum of |g| over
+      // a half bounds every |b_t - r| of that half in the factorized form of
+      // the output and backward kernels (r = b at the middle row)
+      float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int w2 = 4 * warp; w2 < 4 * warp + 4; ++w2) {
+        const float4 x = *reinterpret_cast<const float4*>(&s->grp_abs[w2][f0]);
+        a.x += x.x;
+        a.y += x.y;
+        a.z += x.z;
+        a.w += x.w;
+      }
+      if (!(fmaxf(fmaxf(a.x, a.y), fmaxf(a.z, a.w)) <= kSpanCheck)) *span_flag = 1;
+    }
     if (gsum_tile != nullptr && warp == 0)
       *reinterpret_cast<float4*>(gsum_tile + (((int64_t)b * t_slots + tile * tstride) * H + h) * kD + f0) = all;
     uint8_t* colp = sX + (f0 >> 6) * kBox + (f0 & 7) * 2;
@@ -324,9 +356,11 @@ cleanup:
 // (barrier gbar, phase of the given parity), its walk (b at the middle row into r[], b_end - r into
 // dend[]), then, for row t and column half `half` of every thread, the range
 // check and x = (b_t - r) log2 e, returned in x[].
-__device__ __forceinline__ void gate_rows(float* bt, uint64_t* gbar, uint32_t parity, int* abort, unsigned int site,
+// Returns whether this thread's wait for the gate tile succeeded.
+__device__ __forceinline__ bool gate_rows(float* bt, uint64_t* gbar, uint32_t parity, int* abort, unsigned int site,
                                           float* r, float* dend, int tid, int t, int half, float (&x)[64]) {
-  if (!mbar_wait(gbar, parity, site)) *abort = 1;
+  const bool landed = mbar_wait(gbar, parity, site);
+  if (!landed) *abort = 1;
   walk_tile(bt, tid, r, dend);
   named_sync(kBarAll, kThreads);
   read_gate_row(bt, t, half, x);
@@ -339,6 +373,7 @@ __device__ __forceinline__ void gate_rows(float* bt, uint64_t* gbar, uint32_t pa
     x[u] = y * kLog2e;
   }
   if (!ok) record_error(LASP_ERR_INVALID_ARG, SITE_GATE_RANGE);
+  return landed;
 }
 
 // ---------------------------------------------------------------- output
@@ -366,7 +401,8 @@ __global__ void __launch_bounds__(kThreads, 1) gla_out_tc(const __grid_constant_
                                                           const __grid_constant__ CUtensorMap map_p,
                                                           float* __restrict__ P, int H, int64_t N,
                                                           int64_t t_slots, int stride, int ntx, int tiles,
-                                                          int64_t nseg) {
+                                                          int64_t nseg, RunIf run_if) {
+  if (!runs(run_if)) return;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   uint8_t* sQ = base;                   // Q^
@@ -431,8 +467,11 @@ __global__ void __launch_bounds__(kThreads, 1) gla_out_tc(const __grid_constant_
   }
   uint32_t ph = 0;            // parity of the per-tile barriers' phase for this CTA's current tile
   uint32_t pph = 0;           // parity of the P barrier (once per segment)
-  bool gate_ahead = false;    // thread 0: the next tile's gate tile is in flight
-  bool tok_ahead = false;     // thread 0: the next tile's token tiles are in flight
+  // thread 0: the phase parity of a gate-tile / token-tile load in flight
+  // (this tile's until its wait succeeds, then the next tile's once issued),
+  // or -1; cleanup waits for it once more, so no load lands after the exit
+  int gate_out = (tid == 0 && (int64_t)blockIdx.x < nseg) ? 0 : -1;
+  int tok_out = gate_out;
   bool p_ahead = false;       // thread 0: P's load into the gate tile's space is in flight
   float dprev = 0.f;          // b_end - r of state row t in the tile before (inside a segment)
   for (int64_t sg = blockIdx.x; sg < nseg; sg += gridDim.x) {
@@ -446,11 +485,11 @@ __global__ void __launch_bounds__(kThreads, 1) gla_out_tc(const __grid_constant_
   const int64_t sgn = j + 1 < tiles ? sg : sg + gridDim.x;
   const int jn = j + 1 < tiles ? j + 1 : 0;
   const bool has_next = sgn < nseg;
-  gate_ahead = tok_ahead = false;
   float x[64];
-  gate_rows(bt, &s->gload, ph, &s->abort, SITE_OUT_TMA, s->r, s->dend, tid, t, half, x);
+  if (gate_rows(bt, &s->gload, ph, &s->abort, SITE_OUT_TMA, s->r, s->dend, tid, t, half, x) && tid == 0)
+    gate_out = -1;
   named_sync(kBarAll, kThreads);  // every row of the gate tile has been read
-  if (tid == 0 && j == 0) {
+  if (tid == 0 && j == 0 && !s->abort) {
     // the segment's entering state P (fp32) into the gate tile's space: four
     // boxes of 32 columns with the 128-byte swizzle, so that every thread
     // reads its own row without bank conflicts
@@ -469,7 +508,10 @@ __global__ void __launch_bounds__(kThreads, 1) gla_out_tc(const __grid_constant_
   const float wcarry = exp2f(dprev * kLog2e);
   const float wrow = exp2f(s->r[t] * kLog2e);
   const float dnext = s->dend[t];
-  if (!mbar_wait(&s->load, ph, SITE_OUT_TMA)) s->abort = 1;
+  if (!mbar_wait(&s->load, ph, SITE_OUT_TMA))
+    s->abort = 1;
+  else if (tid == 0)
+    tok_out = -1;
   scale_row_half(sQ, t, half, x, 1.f);   // Q^ = q . E
   scale_row_half(sK, t, half, x, -1.f);  // K^ = k / E
   fence_async_smem();
@@ -557,7 +599,7 @@ __global__ void __launch_bounds__(kThreads, 1) gla_out_tc(const __grid_constant_
         seg_of(sgn, csn, hn, bn);
         load_gate_tile(bt, &map_g, &s->gload, hn, (csn * tiles + jn) * kTile, bn);
         if (jn == 0) bulk_prefetch_l2(P + slot_of(csn * tiles, hn, bn) * kD * kD, kD * kD * 4);
-        gate_ahead = true;
+        gate_out = (int)(ph ^ 1u);
       }
       // the inter term does not wait for the mask
       tc_fence_after();
@@ -605,7 +647,7 @@ __global__ void __launch_bounds__(kThreads, 1) gla_out_tc(const __grid_constant_
         int csn, hn, bn;
         seg_of(sgn, csn, hn, bn);
         load_tokens(hn, (csn * tiles + jn) * kTile, bn);
-        tok_ahead = true;
+        tok_out = (int)(ph ^ 1u);
       }
 #pragma unroll 1
       for (int c2 = 0; c2 < 2; ++c2) {
@@ -638,12 +680,11 @@ __global__ void __launch_bounds__(kThreads, 1) gla_out_tc(const __grid_constant_
   dprev = dnext;
   }
   }
-  gate_ahead = tok_ahead = false;
 cleanup:
-  // loads issued for a next tile that an abort leaves unused land before the
-  // CTA exits (bounded waits)
-  if (tid == 0 && gate_ahead) mbar_wait(&s->gload, ph ^ 1u, SITE_OUT_TMA);
-  if (tid == 0 && tok_ahead) mbar_wait(&s->load, ph ^ 1u, SITE_OUT_TMA);
+  // loads that an abort leaves unused (the current tile's, after a wait that
+  // gave up, or the next tile's) land before the CTA exits (bounded waits)
+  if (tid == 0 && gate_out >= 0) mbar_wait(&s->gload, (uint32_t)gate_out, SITE_OUT_TMA);
+  if (tid == 0 && tok_out >= 0) mbar_wait(&s->load, (uint32_t)tok_out, SITE_OUT_TMA);
   if (tid == 0 && p_ahead) mbar_wait(&s->ldp, pph, SITE_OUT_TMA);
   if (tid == 0) tma_store_wait_read0();  // no store still reads shared memory
   tc_fence_before();
@@ -675,7 +716,8 @@ __global__ void __launch_bounds__(kThreads, 1) gla_bwd_tc(
     const __grid_constant__ CUtensorMap map_dk, const __grid_constant__ CUtensorMap map_dv,
     const __grid_constant__ CUtensorMap map_g, const __grid_constant__ CUtensorMap map_dg,
     const float* __restrict__ P, const float* __restrict__ R, __nv_bfloat16* __restrict__ dq, int H, int64_t N,
-    int64_t t_slots, int stride, int ntx, int64_t ntiles) {
+    int64_t t_slots, int stride, int ntx, int64_t ntiles, RunIf run_if) {
+  if (!runs(run_if)) return;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   uint8_t* sQ = base;
@@ -1133,7 +1175,7 @@ bool tc_gla_ok(int dtype, int d, int64_t C, int64_t N) {
 
 cudaError_t tc_gla_chunk_states(const void* x, const void* y, const float* g, float* M, float* gsum,
                                 float* gsum_tile, int B, int H, int64_t N, int kind, int64_t t_slots, int stride,
-                                int offset, int tiles, int tstride, cudaStream_t st) {
+                                int offset, int tiles, int tstride, cudaStream_t st, int* span_flag, RunIf run) {
   using namespace tc_gla_detail;
   CUtensorMap mx, my;
   if (!make_token_map(&mx, x, B, H, N, kD, kTile) || !make_token_map(&my, y, B, H, N, kD, kTile))
@@ -1144,12 +1186,13 @@ cudaError_t tc_gla_chunk_states(const void* x, const void* y, const float* g, fl
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   kern<<<dim3((unsigned)(N / ((int64_t)tiles * kTile)), H, B), kThreads, smem, st>>>(
-      mx, my, g, M, gsum, gsum_tile, H, N, kind, t_slots, stride, offset, tiles, tstride);
+      mx, my, g, M, gsum, gsum_tile, H, N, kind, t_slots, stride, offset, tiles, tstride, span_flag, run);
   return cudaGetLastError();
 }
 
 cudaError_t tc_gla_chunk_out(const void* q, const void* k, const void* v, const float* g, float* P, void* o,
-                             int B, int H, int64_t N, int64_t t_slots, int stride, int tiles, cudaStream_t st) {
+                             int B, int H, int64_t N, int64_t t_slots, int stride, int tiles, cudaStream_t st,
+                             RunIf run) {
   using namespace tc_gla_detail;
   CUtensorMap mq, mk, mv, mo, mg, mp;
   const int ntx = (int)(N / kTile);
@@ -1168,13 +1211,13 @@ cudaError_t tc_gla_chunk_out(const void* q, const void* k, const void* v, const 
   // one persistent CTA per SM (the kernel holds most of shared memory and all of TMEM)
   const int64_t nseg = (int64_t)B * H * (ntx / tiles);
   const unsigned grid = (unsigned)std::min<int64_t>(nseg, sms);
-  gla_out_tc<<<grid, kThreads, smem, st>>>(mq, mk, mv, mo, mg, mp, P, H, N, t_slots, stride, ntx, tiles, nseg);
+  gla_out_tc<<<grid, kThreads, smem, st>>>(mq, mk, mv, mo, mg, mp, P, H, N, t_slots, stride, ntx, tiles, nseg, run);
   return cudaGetLastError();
 }
 
 cudaError_t tc_gla_chunk_bwd(const void* q, const void* k, const void* v, const void* dout, const float* g,
                              const float* P, const float* Rs, void* dq, void* dk, void* dv, float* dg, int B, int H,
-                             int64_t N, int64_t t_slots, int stride, cudaStream_t st) {
+                             int64_t N, int64_t t_slots, int stride, cudaStream_t st, RunIf run) {
   using namespace tc_gla_detail;
   CUtensorMap mq, mk, mv, mdo, mdk, mdv, mg, mdg;
   if (!make_token_map(&mq, q, B, H, N, kD, kTile) || !make_token_map(&mk, k, B, H, N, kD, kTile) ||
@@ -1194,7 +1237,7 @@ cudaError_t tc_gla_chunk_bwd(const void* q, const void* k, const void* v, const 
   const int64_t ntiles = (int64_t)B * H * ntx;
   const unsigned grid = (unsigned)std::min<int64_t>(ntiles, sms);
   gla_bwd_tc<<<grid, kThreads, smem, st>>>(mq, mk, mv, mdo, mdk, mdv, mg, mdg, P, Rs, (__nv_bfloat16*)dq, H, N, t_slots,
-                                            stride, ntx, ntiles);
+                                            stride, ntx, ntiles, run);
   return cudaGetLastError();
 }
 

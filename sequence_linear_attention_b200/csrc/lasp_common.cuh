@@ -7,6 +7,7 @@
 #include <stdint.h>
 
 #include "../../include/lasp.h"
+#include "kernels.h"
 
 namespace lasp {
 
@@ -57,6 +58,11 @@ __device__ __forceinline__ float load_decay(const float* decay, int h) {
 // lambda^n as exp2(n * log2(lambda)); exact 1 for lambda = 1 and for n = 0.
 __device__ __forceinline__ float decay_pow(float log2_lambda, float n) {
   return exp2f(n * log2_lambda);
+}
+
+// Whether a kernel given `c` (kernels.h) does its work.
+__device__ __forceinline__ bool runs(RunIf c) {
+  return c.flag == nullptr || ((*reinterpret_cast<const volatile int*>(c.flag) != 0) == (c.want != 0));
 }
 
 template <typename T> struct Elem;

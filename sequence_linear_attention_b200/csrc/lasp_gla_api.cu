@@ -15,6 +15,15 @@
 // middle-row log-gate sums) that the backward loads back as is. The backward's
 // gradient states go to the slot of each tile's last chunk of the workspace;
 // its scan over tiles uses the tile totals.
+//
+// The tensor-core kernels factor the intra-tile gate products around each
+// tile's middle row, which holds while the log-gates of each half-tile span
+// at most 80 (natural log). The forward's segment-state kernel checks every
+// tile and sets a flag word that follows the state arrays in the cache. A call
+// with such a tile then runs, in place of the tensor-core output kernel, the
+// exact CUDA-core sequence (per-chunk states, scan, output), and its backward,
+// reading the same flag, runs the CUDA-core backward; the kernels of the
+// sequence not taken return at once. No host synchronisation decides this.
 #include "kernels.h"
 #include "lasp_common.cuh"
 #include "tc_kernels.h"
@@ -45,11 +54,17 @@ int states_impl(const void* x, const void* y, const float* g, float* M, float* g
 // T scan elements in every stride-th slot (from offset) of t_slots slots; the
 // log-gate totals of element c in slot c * stride + goffset
 int scan_impl(const float* M, float* P, const float* gsum, const float* init, float* total, int B, int T, int H,
-              int d, int reverse, int64_t t_slots, int stride, int offset, int goffset, cudaStream_t st) {
-  return cuda_status(traced(K_GLA_SCAN, st, [&] {
-    return launch_gla_scan(M, P, gsum, init, total, B, T, H, d, reverse, t_slots, stride, offset, goffset, st);
+              int d, int reverse, int64_t t_slots, int stride, int offset, int goffset, cudaStream_t st,
+              RunIf run = {}, int id = K_GLA_SCAN) {
+  return cuda_status(traced(id, st, [&] {
+    return launch_gla_scan(M, P, gsum, init, total, B, T, H, d, reverse, t_slots, stride, offset, goffset, st,
+                           run);
   }));
 }
+
+// the cache's flag word: after the states and the two log-gate total arrays
+constexpr int64_t kFlagFloats = 4;
+int64_t cache_state_floats(int B, int H, int64_t N, int d, int C) { return (int64_t)B * (N / C) * H * d * (d + 2); }
 
 }  // namespace gla_api_detail
 }  // namespace lasp
@@ -62,7 +77,7 @@ extern "C" {
 
 int64_t lasp_gla_cache_floats(int B, int H, int64_t N, int d, int C) {
   if (check_gla_sizes(B, H, N, d, C, LASP_F32)) return -1;
-  return (int64_t)B * (N / C) * H * d * (d + 2);
+  return cache_state_floats(B, H, N, d, C) + kFlagFloats;
 }
 
 int lasp_gla_chunk_states(const void* x, const void* y, const float* g, float* M, float* gsum, int B, int H,
@@ -107,8 +122,11 @@ int lasp_gla_fwd(const void* q, const void* k, const void* v, const float* g, vo
     const int S = walk_segment_tokens(N, 128) / 128;
     const int nseg = (int)(N / 128) / S;
     float* gseg = gsum + (int64_t)B * T * H * d;
+    int* flag = reinterpret_cast<int*>(state_cache + cache_state_floats(B, H, N, d, C));
+    if ((s = cuda_status(cudaMemsetAsync(flag, 0, sizeof(int), st)))) return s;
     if ((s = cuda_status(traced(K_GLA_SEG_STATES, st, [&] {
-           return tc_gla_chunk_states(k, v, g, state_cache, gseg, gsum, B, H, N, 0, T, S * stride, 0, S, stride, st);
+           return tc_gla_chunk_states(k, v, g, state_cache, gseg, gsum, B, H, N, 0, T, S * stride, 0, S, stride, st,
+                                      flag);
          }))))
       return s;
     if ((s = cuda_status(traced(K_GLA_SEG_SCAN, st, [&] {
@@ -116,8 +134,21 @@ int lasp_gla_fwd(const void* q, const void* k, const void* v, const float* g, vo
                                   0, 0, st);
          }))))
       return s;
-    return cuda_status(traced(K_GLA_OUT_TC, st, [&] {
-      return tc_gla_chunk_out(q, k, v, g, state_cache, o, B, H, N, T, stride, S, st);
+    const RunIf tc{flag, 0}, exact{flag, 1};
+    if ((s = cuda_status(traced(K_GLA_OUT_TC, st, [&] {
+           return tc_gla_chunk_out(q, k, v, g, state_cache, o, B, H, N, T, stride, S, st, tc);
+         }))))
+      return s;
+    // the exact sequence, which runs only when the flag is set
+    if ((s = cuda_status(traced(K_GLA_EXACT_STATES, st, [&] {
+           return gla_simt_chunk_states(k, v, g, state_cache, gsum, B, H, N, d, C, 0, dtype, st, exact);
+         }))))
+      return s;
+    if ((s = scan_impl(state_cache, state_cache, gsum, init_state, nullptr, B, T, H, d, 0, T, 1, 0, 0, st, exact,
+                       K_GLA_EXACT_SCAN)))
+      return s;
+    return cuda_status(traced(K_GLA_EXACT_OUT, st, [&] {
+      return gla_simt_chunk_out(q, k, v, g, state_cache, o, B, H, N, d, C, dtype, st, exact);
     }));
   }
   // 1. chunk states M_c and log-gate totals; 2. exclusive prefix in place -> P_c; 3. output
@@ -145,16 +176,33 @@ int lasp_gla_bwd(const void* q, const void* k, const void* v, const float* g, co
     // the cache slots of their first chunks), then the gradients
     const int stride = 128 / C;
     const int tiles = (int)(N / 128);
+    // the forward's choice, in the cache's flag word
+    const int* flag = reinterpret_cast<const int*>(state_cache + cache_state_floats(B, H, N, d, C));
+    const RunIf tc{flag, 0}, exact{flag, 1};
     if ((s = cuda_status(traced(K_GLA_STATES_TC, st, [&] {
-           return tc_gla_chunk_states(q, dout, g, dstate_ws, nullptr, nullptr, B, H, N, 1, T, stride, stride - 1, 1, stride,
-                                      st);
+           return tc_gla_chunk_states(q, dout, g, dstate_ws, nullptr, nullptr, B, H, N, 1, T, stride, stride - 1, 1,
+                                      stride, st, nullptr, tc);
          }))))
       return s;
     if ((s = scan_impl(dstate_ws, dstate_ws, gsum, dstate_in, dinit_state, B, tiles, H, d, 1, T, stride, stride - 1, 0,
-                       st)))
+                       st, tc)))
       return s;
-    return cuda_status(traced(K_GLA_BWD_TC, st, [&] {
-      return tc_gla_chunk_bwd(q, k, v, dout, g, state_cache, dstate_ws, dq, dk, dv, dg, B, H, N, T, stride, st);
+    if ((s = cuda_status(traced(K_GLA_BWD_TC, st, [&] {
+           return tc_gla_chunk_bwd(q, k, v, dout, g, state_cache, dstate_ws, dq, dk, dv, dg, B, H, N, T, stride, st,
+                                   tc);
+         }))))
+      return s;
+    // the exact sequence, which runs only when the forward took it
+    if ((s = cuda_status(traced(K_GLA_EXACT_STATES, st, [&] {
+           return gla_simt_chunk_states(q, dout, g, dstate_ws, nullptr, B, H, N, d, C, 1, dtype, st, exact);
+         }))))
+      return s;
+    if ((s = scan_impl(dstate_ws, dstate_ws, gsum, dstate_in, dinit_state, B, T, H, d, 1, T, 1, 0, 0, st, exact,
+                       K_GLA_EXACT_SCAN)))
+      return s;
+    return cuda_status(traced(K_GLA_EXACT_BWD, st, [&] {
+      return gla_simt_chunk_bwd(q, k, v, dout, g, state_cache, dstate_ws, dq, dk, dv, dg, B, H, N, d, C, dtype, st,
+                                exact);
     }));
   }
   // 1. gradient chunk states dM_c; 2. exclusive suffix in place -> R_c (and

@@ -6,6 +6,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include "kernels.h"
+
 namespace lasp {
 
 // Chunk states on tensor cores: bf16, d = 128, C a multiple of 16. The
@@ -67,13 +69,18 @@ cudaError_t tc_bidir_apply(const void* x, const void* stiles, void* y, int B, in
 // given P in the slot of each tile's first chunk; the gradients given that P
 // and R in the slot of the tile's last chunk (stride = chunks per tile).
 bool tc_gla_ok(int dtype, int d, int64_t C, int64_t N);
+// span_flag (may be NULL): set to 1 when a tile's log-gates span more than the
+// factorized form of the output and backward kernels takes; `run` makes a
+// launch conditional on such a flag (kernels.h).
 cudaError_t tc_gla_chunk_states(const void* x, const void* y, const float* g, float* M, float* gsum,
                                 float* gsum_tile, int B, int H, int64_t N, int kind, int64_t t_slots, int stride,
-                                int offset, int tiles, int tstride, cudaStream_t st);
+                                int offset, int tiles, int tstride, cudaStream_t st, int* span_flag = nullptr,
+                                RunIf run = {});
 cudaError_t tc_gla_chunk_out(const void* q, const void* k, const void* v, const float* g, float* P, void* o,
-                             int B, int H, int64_t N, int64_t t_slots, int stride, int tiles, cudaStream_t st);
+                             int B, int H, int64_t N, int64_t t_slots, int stride, int tiles, cudaStream_t st,
+                             RunIf run = {});
 cudaError_t tc_gla_chunk_bwd(const void* q, const void* k, const void* v, const void* dout, const float* g,
                              const float* P, const float* Rs, void* dq, void* dk, void* dv, float* dg, int B, int H,
-                             int64_t N, int64_t t_slots, int stride, cudaStream_t st);
+                             int64_t N, int64_t t_slots, int stride, cudaStream_t st, RunIf run = {});
 
 }  // namespace lasp

@@ -158,7 +158,7 @@ def test_gated_calls_reject_bad_arguments(lib):
     assert p(A, A, None, None, None, 1, 4, 2, 64, 0, None) == INVALID                  # no gsum
     assert p(A, A, A, None, None, 1, 4, 2, 64, 2, None) == INVALID                     # reverse
     assert p(None, None, None, None, None, 1, 0, 2, 64, 0, None) == OK                 # T = 0, no total
-    assert lasp.lasp_gla_cache_floats(2, 3, 512, 64, 64) == 2 * 8 * 3 * 64 * 66
+    assert lasp.lasp_gla_cache_floats(2, 3, 512, 64, 64) == 2 * 8 * 3 * 64 * 66 + 4
     assert lasp.lasp_gla_cache_floats(2, 3, 512, 64, 256) == -1
 
 
@@ -204,5 +204,5 @@ int main(void) {
     subprocess.run(["gcc", "-std=c99", "-Wall", "-Wextra", "-Werror", "-pedantic", "-I", os.path.join(ROOT, "include"),
                     str(src), "-o", str(exe), "-L", libdir, "-llasp", "-Wl,-rpath," + libdir], check=True)
     out = subprocess.run([str(exe)], check=True, capture_output=True, text=True).stdout.split()
-    assert out == ["1", "LASP_ERR_UNSUPPORTED", str(UNSUPPORTED), str(INVALID), str(2 * 8 * 3 * 64 * 66),
+    assert out == ["1", "LASP_ERR_UNSUPPORTED", str(UNSUPPORTED), str(INVALID), str(2 * 8 * 3 * 64 * 66 + 4),
                    str(lasp.lasp_segment_tokens(65536, 128, 128, BF16))]

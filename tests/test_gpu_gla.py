@@ -228,30 +228,62 @@ def _rows_states(bf16, C, d):
     assert rel_err(gs.cpu().numpy(), gs_ref) <= 1e-5
 
 
-def test_tensor_core_path_reports_gates_out_of_range():
-    """Log-gates of -2 per token make each 64-token half of a 128-token tile
-    span e^-128, more than the factorized form takes: the call records
-    LASP_ERR_INVALID_ARG at the gate-range site instead of returning wrong
-    numbers silently (the CUDA-core kernels, which fp32 inputs take, accept
-    such gates)."""
-    import torch
+def _strong_gates(kind, B, N, H, d, seed):
+    if kind == "const_ln0.1":
+        return np.full((B, N, H, d), np.log(0.1), np.float32)
+    if kind == "logsig_tau1":
+        return lasp_inputs.make_log_gates(B, N, H, d, seed=seed, tau=1.0)
+    # mild gates everywhere but one 128-token tile of the last head, whose
+    # log-gates are -3 per token
+    g = lasp_inputs.make_log_gates(B, N, H, d, seed=seed, tau=16.0)
+    g[:, 256:384, H - 1, :] = -3.0
+    return g
+
+
+@pytest.mark.parametrize("kind", ["const_ln0.1", "logsig_tau1", "one_tile"])
+@pytest.mark.parametrize("C", [128, 64])
+def test_tensor_core_call_with_strong_gates_matches_oracle(kind, C):
+    """bf16 with d = 128 takes the tensor-core path, whose factorized intra-tile
+    form holds while each half-tile's |log-gates| sum to at most 79. Constant
+    gates of 0.1 (64 ln 0.1 = -147 per half-tile), log sigmoid(x) gates at
+    tau = 1 and a single strong tile go beyond that: the forward's state
+    kernel sees it and the call and its backward run the exact CUDA-core
+    kernels instead. The results match the oracle and no status is recorded
+    (LASP Appendix A.4, Eq. 24 defines these inputs like any other)."""
+    B, N, H, d = 1, 512, 2, 128
+    seed = 2040 + C
+    inp = lasp_inputs.make_inputs(B, N, H, d, seed=seed, bf16=True, decayed=False)
+    g = _strong_gates(kind, B, N, H, d, seed)
+    rng = np.random.default_rng(seed)
+    init = (rng.standard_normal((B, H, d, d)) * 0.1).astype(np.float32)
+    dsin = (rng.standard_normal((B, H, d, d)) * 0.1).astype(np.float32)
+    got = _run(inp, g, C, init=init, dstate_in=dsin)  # asserts a clean device status
+    ref = _reference(inp, g, init=init.astype(np.float64), dstate_in=dsin.astype(np.float64))
+    _compare(got, ref, TOL_BF16)
+
+
+def test_mild_gates_leave_the_exact_kernels_idle():
+    """With gates inside the factorized range the exact CUDA-core kernels a
+    tensor-core call also launches return at once: each takes a small part of
+    the tensor-core kernel it stands in for."""
     import sequence_linear_attention_b200 as lasp
-    B, N, H, d, C = 1, 256, 1, 128, 128
-    inp = lasp_inputs.make_inputs(B, N, H, d, seed=2024, bf16=True, decayed=False)
-    q, k, v = (to_device(inp[n], True) for n in ("q", "k", "v"))
-    gd = torch.full((B, N, H, d), -2.0, dtype=torch.float32, device="cuda")
-    cache = torch.empty(lasp.lasp_gla_cache_floats(B, H, N, d, C), dtype=torch.float32, device="cuda")
-    o = torch.empty_like(q)
-    lasp.lasp_gla_fwd(q, k, v, gd, o, C, cache)
-    status, site = lasp.lasp_check_device_status()
-    assert (status, site) == (1, 40)
-    # the same (bf16-valued) inputs as fp32 through the CUDA-core kernels are fine
-    q32, k32, v32 = (to_device(host_f32(inp, n), False) for n in ("q", "k", "v"))
-    o32 = torch.empty_like(q32)
-    lasp.lasp_gla_fwd(q32, k32, v32, gd, o32, C, cache)
-    assert lasp.lasp_check_device_status() == (0, 0)
-    ref = oracle.gla_fwd(*(host_f32(inp, n) for n in ("q", "k", "v")), gd.cpu().numpy())
-    assert rel_err(to_host(o32), ref) <= TOL_F32
+    B, N, H, d, C = 1, 4096, 4, 128, 128
+    inp = lasp_inputs.make_inputs(B, N, H, d, seed=2050, bf16=True, decayed=False)
+    g = lasp_inputs.make_log_gates(B, N, H, d, seed=2050, tau=16.0)
+    _run(inp, g, C)
+    lasp.lasp_trace_enable(64)
+    try:
+        _run(inp, g, C)
+        trace = lasp.lasp_trace_read(64)
+    finally:
+        lasp.lasp_trace_enable(0)
+    ms = dict(trace)
+    names = [n for n, _ in trace]
+    assert names == ["gla_segment_states_tc", "gla_segment_scan", "gla_out_tc", "gla_states_exact",
+                     "gla_scan_exact", "gla_out_exact", "gla_states_tc", "gla_scan", "gla_bwd_tc",
+                     "gla_states_exact", "gla_scan_exact", "gla_bwd_exact"], names
+    assert ms["gla_out_exact"] < 0.5 * ms["gla_out_tc"], trace
+    assert ms["gla_bwd_exact"] < 0.5 * ms["gla_bwd_tc"], trace
 
 
 @pytest.mark.parametrize("C", [16, 32, 64])
