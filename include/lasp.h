@@ -459,6 +459,46 @@ LASP_API int lasp_gla_bwd(const void* q, const void* k, const void* v, const flo
                           const float* state_cache, float* dstate_ws, const float* dstate_in, float* dinit_state,
                           void* stream);
 
+/* ------------------------------------------------------------------------
+ * Softmax attention: the standard attention layers a hybrid model keeps.
+ * Page LASP-2 review, "Summary" and abstract: LASP-2H applies the same
+ * AllGather pattern to standard attention layers, each rank gathering the
+ * keys and values (K_t, V_t) of the ranks before it. A call takes a block of
+ * queries sitting at global positions p_i = q_offset + i (i = 0..Nq-1) and
+ * the keys / values at positions 0..Nk-1 (on one GPU: q_offset = 0 and
+ * Nq = Nk = N; in sequence parallelism: the rank's own queries against the
+ * gathered keys). For every b, h (causal, scale > 0, usually d^-1/2):
+ *     s_ij  = scale (q_i . k_j)                        for j <= p_i
+ *     o_i   = sum_{j <= p_i} exp(s_ij - lse_i) v_j
+ *     lse_i = log sum_{j <= p_i} exp(s_ij)             (natural log)
+ * Supported: bf16, d = 128 (tensor cores); other types and sizes return
+ * LASP_ERR_UNSUPPORTED. Requires q_offset + Nq <= Nk (LASP_ERR_INVALID_ARG).
+ *   q, o, dout, dq:  [B, Nq, H, d];  k, v, dk, dv: [B, Nk, H, d] (bf16)
+ *   lse, delta:      float [B, H, Nq]
+ * Pointers, streams and errors as for the calls above; nothing allocates.
+ */
+
+/*
+ * lasp_softmax_fwd -- o and lse as above (one online-softmax pass over
+ * 128-key tiles per 128-query tile).
+ */
+LASP_API int lasp_softmax_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
+                              int64_t Nq, int64_t Nk, int64_t q_offset, int d, float scale, int dtype, void* stream);
+
+/*
+ * lasp_softmax_bwd -- gradients of sum(o * dout) for lasp_softmax_fwd:
+ *     p_ij = exp(s_ij - lse_i),   ds_ij = p_ij (dout_i . v_j - delta_i),
+ *     dq_i = scale sum_j ds_ij k_j,  dk_j = scale sum_i ds_ij q_i,  dv_j = sum_i p_ij dout_i,
+ * with delta_i = dout_i . o_i (written to `delta`, a workspace the caller
+ * owns). o and lse are lasp_softmax_fwd's for the same inputs. Every row of
+ * dk and dv is written; keys no query reaches get zeros (in sequence
+ * parallelism each rank's dk, dv are summed over the ranks by a
+ * reduce-scatter).
+ */
+LASP_API int lasp_softmax_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                              const void* dout, void* dq, void* dk, void* dv, float* delta, int B, int H, int64_t Nq,
+                              int64_t Nk, int64_t q_offset, int d, float scale, int dtype, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -23,6 +23,11 @@ it with ctypes. Each wrapper states the passage it follows:
   LASP page, section 3.1, Eq. 3 right product Q (K^T V) without Norm; LASP-2
   review page, "Summary": the unmasked variant gathers all chunk states and
   every chunk computes Q_t M_{1:T}, and the backward the same with dM.
+* :func:`softmax_fwd`, :func:`softmax_bwd` -- the softmax-attention layers of
+  the hybrid model: LASP-2 review page, "Summary" (LASP-2H applies the same
+  AllGather pattern to standard attention, gathering K_t and V_t); standard
+  causal softmax attention with a query offset into the gathered keys, and its
+  gradients by the chain rule through the softmax.
 * :func:`gla_fwd`, :func:`gla_bwd`, :func:`gla_chunk_states`,
   :func:`gla_state_scan`, :func:`gla_state_snapshots` -- the gated form (a
   decay per token and key feature): LASP page, Appendix A.4, Eq. 24 with the
@@ -85,12 +90,17 @@ def _load():
             lib.oracle_gla_chunk_states.argtypes = [_P, _P, _P, _L, _L, _L, _P, _P, _I, _L, _I, _I, _L, _I]
             lib.oracle_gla_state_scan.argtypes = [_P, _P, _P, _P, _P, _I, _L, _I, _I, _I]
             lib.oracle_gla_state_snapshots.argtypes = [_P, _P, _P, _L, _L, _L, _P, _P, _I, _L, _I, _I, _L, _I]
+            _D = ctypes.c_double
+            lib.oracle_softmax_fwd.argtypes = [_P, _L, _L, _L, _P, _P, _L, _L, _L, _P, _L, _L, _L, _P,
+                                               _I, _L, _L, _L, _I, _I, _D]
+            lib.oracle_softmax_bwd.argtypes = [_P, _L, _L, _L, _P, _P, _L, _L, _L, _P, _P, _L, _L, _L, _P, _P,
+                                               _L, _L, _L, _I, _L, _L, _L, _I, _I, _D]
             lib.oracle_num_threads.restype = _I
             for f in (lib.oracle_fwd, lib.oracle_bwd, lib.oracle_chunk_states,
                       lib.oracle_state_scan, lib.oracle_state_snapshots, lib.oracle_bidir_fwd,
                       lib.oracle_bidir_bwd, lib.oracle_gla_fwd, lib.oracle_gla_bwd,
                       lib.oracle_gla_chunk_states, lib.oracle_gla_state_scan,
-                      lib.oracle_gla_state_snapshots):
+                      lib.oracle_gla_state_snapshots, lib.oracle_softmax_fwd, lib.oracle_softmax_bwd):
                 f.restype = None
             _lib = lib
     return _lib
@@ -355,3 +365,60 @@ def gla_state_snapshots(x, y, g, C, init=None, kind=0):
     _load().oracle_gla_state_snapshots(px, y.ctypes.data, g.ctypes.data, sb, sn, sh, pi, P.ctypes.data,
                                        B, N, H, d, C, kind)
     return P
+
+
+# ------------------------------------------------------------ softmax attention
+def _tok_view(x: np.ndarray):
+    if x.dtype != np.float32 or x.ndim != 4 or x.strides[3] != 4:
+        raise ValueError("token tensors must be float32 [B, N, H, d] with a contiguous feature axis")
+    sb, sn, sh, _ = (s // 4 for s in x.strides)
+    return x.ctypes.data, sb, sn, sh
+
+
+def softmax_fwd(q, k, v, q_offset=0, scale=None):
+    """Causal softmax attention of queries q [B, Nq, H, d] at global positions
+    q_offset + i against keys / values k, v [B, Nk, H, d] at positions
+    0..Nk-1: o_i = sum_{j <= q_offset + i} softmax_j(scale q_i . k_j) v_j, and
+    lse_i, the natural log of the softmax denominator (with the scores as
+    given, no shift). scale defaults to d^-1/2. Returns o (float64
+    [B, Nq, H, d]) and lse (float64 [B, H, Nq])."""
+    B, Nq, H, d = q.shape
+    Nk = k.shape[1]
+    if k.shape != v.shape or k.strides != v.strides or k.shape[0] != B or k.shape[2:] != (H, d):
+        raise ValueError("k and v must be [B, Nk, H, d] views with the same strides")
+    if q_offset < 0 or q_offset + Nq > Nk:
+        raise ValueError("the queries must sit inside the keys: q_offset + Nq <= Nk")
+    scale = float(d) ** -0.5 if scale is None else float(scale)
+    pq, qb, qn, qh = _tok_view(q)
+    pk, kb, kn, kh = _tok_view(k)
+    pv = _tok_view(v)[0]
+    o = np.empty((B, Nq, H, d), np.float64)
+    lse = np.empty((B, H, Nq), np.float64)
+    _load().oracle_softmax_fwd(pq, qb, qn, qh, pk, pv, kb, kn, kh, o.ctypes.data, Nq * H * d, H * d, d,
+                               lse.ctypes.data, B, Nq, Nk, q_offset, H, d, scale)
+    return o, lse
+
+
+def softmax_bwd(q, k, v, do, q_offset=0, scale=None):
+    """Gradients of sum(o * do) for :func:`softmax_fwd` with respect to q
+    ([B, Nq, H, d]) and k, v ([B, Nk, H, d]; keys no query reaches get zero).
+    do shares q's shape and strides. Returns dq, dk, dv as float64."""
+    B, Nq, H, d = q.shape
+    Nk = k.shape[1]
+    if k.shape != v.shape or k.strides != v.strides or k.shape[0] != B or k.shape[2:] != (H, d):
+        raise ValueError("k and v must be [B, Nk, H, d] views with the same strides")
+    if do.shape != q.shape or do.strides != q.strides:
+        raise ValueError("do must share q's shape and strides")
+    if q_offset < 0 or q_offset + Nq > Nk:
+        raise ValueError("the queries must sit inside the keys: q_offset + Nq <= Nk")
+    scale = float(d) ** -0.5 if scale is None else float(scale)
+    pq, qb, qn, qh = _tok_view(q)
+    pk, kb, kn, kh = _tok_view(k)
+    pv = _tok_view(v)[0]
+    pd = _tok_view(do)[0]
+    dq = np.empty((B, Nq, H, d), np.float64)
+    dk = np.empty((B, Nk, H, d), np.float64)
+    dv = np.empty_like(dk)
+    _load().oracle_softmax_bwd(pq, qb, qn, qh, pk, pv, kb, kn, kh, pd, dq.ctypes.data, Nq * H * d, H * d, d,
+                               dk.ctypes.data, dv.ctypes.data, Nk * H * d, H * d, d, B, Nq, Nk, q_offset, H, d, scale)
+    return dq, dk, dv

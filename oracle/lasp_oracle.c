@@ -721,3 +721,164 @@ void oracle_gla_state_snapshots(const float *x, const float *y, const float *a, 
     free(S);
   }
 }
+
+/* ------------------------------------------------------------------------
+ * Softmax attention, the layers a hybrid model keeps (LASP-2 review page,
+ * "Summary": LASP-2H applies the same AllGather pattern to standard attention
+ * layers, each rank gathering K_t and V_t). Standard causal softmax attention,
+ * per (b, h), with the queries of this call sitting at global positions
+ * p_i = q_offset + i (i = 0..Nq-1) and the keys / values at positions
+ * j = 0..Nk-1 (the gathered K and V):
+ *   s_ij  = scale * (q_i . k_j)                      for j <= p_i
+ *   a_ij  = exp(s_ij) / sum_{j' <= p_i} exp(s_ij')
+ *   o_i   = sum_{j <= p_i} a_ij v_j
+ *   lse_i = log sum_{j <= p_i} exp(s_ij)             (natural log)
+ * The sums over j are taken after subtracting m_i = max_j s_ij (the textbook
+ * way to keep exp in range; it cancels in a_ij). Requires q_offset + Nq <= Nk.
+ * q, o: [B, Nq, H, d] (views qb/qn/qh, ob/on/oh); k, v: [B, Nk, H, d] (views
+ * kb/kn/kh); lse: [B, H, Nq], may be NULL.
+ * Task = (b, h, query row): each output row is one thread's sum, in key order.
+ */
+static double softmax_row_scores(const float *qi, const float *k, long kb, long kn, long kh, int b, int h, long last,
+                                 int d, double scale, double *s) {
+  double m = -INFINITY;
+  for (long j = 0; j <= last; ++j) {
+    const float *kj = tok(k, kb, kn, kh, b, j, h);
+    double acc = 0.0;
+    for (int f = 0; f < d; ++f) acc += (double)qi[f] * kj[f];
+    s[j] = scale * acc;
+    if (s[j] > m) m = s[j];
+  }
+  return m;
+}
+
+void oracle_softmax_fwd(const float *q, long qb, long qn, long qh, const float *k, const float *v, long kb, long kn,
+                        long kh, double *o, long ob, long on, long oh, double *lse, int B, long Nq, long Nk,
+                        long q_offset, int H, int d, double scale) {
+  (void)Nk;
+#pragma omp parallel
+  {
+    double *s = (double *)malloc(sizeof(double) * (size_t)(q_offset + Nq));
+#pragma omp for schedule(dynamic, 16)
+    for (long task = 0; task < (long)B * H * Nq; ++task) {
+      long i = task % Nq;
+      int h = (int)((task / Nq) % H);
+      int b = (int)(task / (Nq * H));
+      long last = q_offset + i;
+      const float *qi = tok(q, qb, qn, qh, b, i, h);
+      double m = softmax_row_scores(qi, k, kb, kn, kh, b, h, last, d, scale, s);
+      double l = 0.0;
+      for (long j = 0; j <= last; ++j) {
+        s[j] = exp(s[j] - m);
+        l += s[j];
+      }
+      double *oi = tokd(o, ob, on, oh, b, i, h);
+      for (int f = 0; f < d; ++f) oi[f] = 0.0;
+      for (long j = 0; j <= last; ++j) {
+        const float *vj = tok(v, kb, kn, kh, b, j, h);
+        double a = s[j] / l;
+        for (int f = 0; f < d; ++f) oi[f] += a * vj[f];
+      }
+      if (lse) lse[((long)b * H + h) * Nq + i] = m + log(l);
+    }
+    free(s);
+  }
+}
+
+/*
+ * Its gradients for L = sum_i o_i . do_i (the chain rule through the softmax):
+ *   dv_j  = sum_{i: p_i >= j} a_ij do_i
+ *   da_ij = do_i . v_j,   ds_ij = a_ij (da_ij - sum_{j'} a_ij' da_ij')
+ *   dq_i  = scale sum_j ds_ij k_j,    dk_j = scale sum_{i: p_i >= j} ds_ij q_i
+ * dq: [B, Nq, H, d] (view gb/gn/gh); dk, dv: [B, Nk, H, d] (view eb/en/eh);
+ * keys no query reaches get zero gradients. Three passes per (b, h): each
+ * query's normaliser and sum_j a_ij da_ij; dq per query; dk and dv per key,
+ * each row one thread's sum, in index order.
+ */
+void oracle_softmax_bwd(const float *q, long qb, long qn, long qh, const float *k, const float *v, long kb, long kn,
+                        long kh, const float *dout, double *dq, long gb, long gn, long gh, double *dk, double *dv,
+                        long eb, long en, long eh, int B, long Nq, long Nk, long q_offset, int H, int d,
+                        double scale) {
+  double *lse = (double *)malloc(sizeof(double) * (size_t)B * H * Nq);
+  double *rs = (double *)malloc(sizeof(double) * (size_t)B * H * Nq); /* sum_j a_ij da_ij */
+#pragma omp parallel
+  {
+    double *s = (double *)malloc(sizeof(double) * (size_t)(q_offset + Nq));
+#pragma omp for schedule(dynamic, 16)
+    for (long task = 0; task < (long)B * H * Nq; ++task) {
+      long i = task % Nq;
+      int h = (int)((task / Nq) % H);
+      int b = (int)(task / (Nq * H));
+      long last = q_offset + i;
+      const float *qi = tok(q, qb, qn, qh, b, i, h);
+      const float *di = tok(dout, qb, qn, qh, b, i, h);
+      double m = softmax_row_scores(qi, k, kb, kn, kh, b, h, last, d, scale, s);
+      double l = 0.0;
+      for (long j = 0; j <= last; ++j) l += exp(s[j] - m);
+      double r = 0.0;
+      for (long j = 0; j <= last; ++j) {
+        const float *vj = tok(v, kb, kn, kh, b, j, h);
+        double da = 0.0;
+        for (int f = 0; f < d; ++f) da += (double)di[f] * vj[f];
+        r += exp(s[j] - m) / l * da;
+      }
+      lse[task] = m + log(l);
+      rs[task] = r;
+    }
+#pragma omp for schedule(dynamic, 16)
+    for (long task = 0; task < (long)B * H * Nq; ++task) {
+      long i = task % Nq;
+      int h = (int)((task / Nq) % H);
+      int b = (int)(task / (Nq * H));
+      long last = q_offset + i;
+      const float *qi = tok(q, qb, qn, qh, b, i, h);
+      const float *di = tok(dout, qb, qn, qh, b, i, h);
+      double *dqi = tokd(dq, gb, gn, gh, b, i, h);
+      for (int f = 0; f < d; ++f) dqi[f] = 0.0;
+      softmax_row_scores(qi, k, kb, kn, kh, b, h, last, d, scale, s);
+      for (long j = 0; j <= last; ++j) {
+        const float *kj = tok(k, kb, kn, kh, b, j, h);
+        const float *vj = tok(v, kb, kn, kh, b, j, h);
+        double da = 0.0;
+        for (int f = 0; f < d; ++f) da += (double)di[f] * vj[f];
+        double a = exp(s[j] - lse[task]);
+        double ds = a * (da - rs[task]);
+        for (int f = 0; f < d; ++f) dqi[f] += scale * ds * kj[f];
+      }
+    }
+#pragma omp for schedule(dynamic, 16)
+    for (long task = 0; task < (long)B * H * Nk; ++task) {
+      long j = task % Nk;
+      int h = (int)((task / Nk) % H);
+      int b = (int)(task / (Nk * H));
+      const float *kj = tok(k, kb, kn, kh, b, j, h);
+      const float *vj = tok(v, kb, kn, kh, b, j, h);
+      double *dkj = tokd(dk, eb, en, eh, b, j, h);
+      double *dvj = tokd(dv, eb, en, eh, b, j, h);
+      for (int f = 0; f < d; ++f) {
+        dkj[f] = 0.0;
+        dvj[f] = 0.0;
+      }
+      long i0 = j > q_offset ? j - q_offset : 0; /* the first query with p_i >= j */
+      for (long i = i0; i < Nq; ++i) {
+        const float *qi = tok(q, qb, qn, qh, b, i, h);
+        const float *di = tok(dout, qb, qn, qh, b, i, h);
+        long row = ((long)b * H + h) * Nq + i;
+        double sij = 0.0, da = 0.0;
+        for (int f = 0; f < d; ++f) {
+          sij += (double)qi[f] * kj[f];
+          da += (double)di[f] * vj[f];
+        }
+        double a = exp(scale * sij - lse[row]);
+        double ds = a * (da - rs[row]);
+        for (int f = 0; f < d; ++f) {
+          dvj[f] += a * di[f];
+          dkj[f] += scale * ds * qi[f];
+        }
+      }
+    }
+    free(s);
+  }
+  free(lse);
+  free(rs);
+}

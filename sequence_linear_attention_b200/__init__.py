@@ -25,7 +25,7 @@ __all__ = [
     "lasp_status_string", "lasp_version", "lasp_trace_enable", "lasp_trace_read", "lasp_kernel_name",
     "lasp_segment_tokens", "lasp_bidir_workspace_floats", "lasp_bidir_state_offset", "lasp_bidir_fwd",
     "lasp_bidir_bwd", "lasp_gla_cache_floats", "lasp_gla_chunk_states", "lasp_gla_state_prefix", "lasp_gla_fwd",
-    "lasp_gla_bwd",
+    "lasp_gla_bwd", "lasp_softmax_fwd", "lasp_softmax_bwd",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -92,6 +92,9 @@ def _load():
             lib.lasp_gla_state_prefix.argtypes = [P, P, P, P, P, I, I, I, I, I, P]
             lib.lasp_gla_fwd.argtypes = [P, P, P, P, P, I, I, L, I, I, I, P, P, P]
             lib.lasp_gla_bwd.argtypes = [P, P, P, P, P, P, P, P, P, I, I, L, I, I, I, P, P, P, P, P]
+            F = ctypes.c_float
+            lib.lasp_softmax_fwd.argtypes = [P, P, P, P, P, I, I, L, L, L, I, F, I, P]
+            lib.lasp_softmax_bwd.argtypes = [P, P, P, P, P, P, P, P, P, P, I, I, L, L, L, I, F, I, P]
             lib.lasp_status_string.argtypes = [I]
             lib.lasp_status_string.restype = ctypes.c_char_p
             for f in (lib.lasp_fwd, lib.lasp_bwd, lib.lasp_fwd_states, lib.lasp_fwd_finish, lib.lasp_bwd_states,
@@ -101,7 +104,7 @@ def _load():
                       lib.lasp_wait_probe, lib.lasp_version, lib.lasp_trace_enable, lib.lasp_trace_read,
                       lib.lasp_segment_tokens, lib.lasp_bidir_fwd, lib.lasp_bidir_bwd,
                       lib.lasp_gla_chunk_states, lib.lasp_gla_state_prefix, lib.lasp_gla_fwd,
-                      lib.lasp_gla_bwd):
+                      lib.lasp_gla_bwd, lib.lasp_softmax_fwd, lib.lasp_softmax_bwd):
                 f.restype = I
             _lib = lib
     return _lib
@@ -368,3 +371,42 @@ def lasp_status_string(status: int) -> str:
 
 def lasp_version() -> int:
     return int(_load().lasp_version())
+
+
+# ------------------------------------------------------------ softmax attention
+def _softmax_shapes(q, k, *rest_q):
+    """(B, H, Nq, Nk, d, dtype) of queries [B, Nq, H, d] against keys [B, Nk, H, d]."""
+    Bq, Nq, Hq, dq_ = _tokens(q, *rest_q)[:4]
+    B, Nk, H, d, dt = _tokens(k)
+    if (Bq, Hq, dq_) != (B, H, d) or q.dtype != k.dtype:
+        raise ValueError("queries and keys must share B, H, d and dtype")
+    return B, H, Nq, Nk, d, dt
+
+
+def _rows(t, B, H, Nq):
+    if t is not None and (tuple(t.shape) != (B, H, Nq) or t.dtype.itemsize != 4 or not t.is_contiguous()):
+        raise ValueError("lse and delta must be contiguous float32 [B, H, Nq]")
+
+
+def lasp_softmax_fwd(q, k, v, o, lse, q_offset=0, scale=None, stream=None):
+    """Causal softmax attention of queries at positions q_offset + i against
+    keys / values at 0..Nk-1; o [B, Nq, H, d], lse [B, H, Nq]. See lasp.h."""
+    B, H, Nq, Nk, d, dt = _softmax_shapes(q, k, o)
+    _tokens(k, v)
+    _rows(lse, B, H, Nq)
+    scale = float(d) ** -0.5 if scale is None else float(scale)
+    _check(_load().lasp_softmax_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, Nq, Nk, q_offset, d,
+                                    scale, dt, _stream(stream, q)), "lasp_softmax_fwd")
+
+
+def lasp_softmax_bwd(q, k, v, o, lse, dout, dq, dk, dv, delta, q_offset=0, scale=None, stream=None):
+    """dq, dk, dv of sum(o * dout) for lasp_softmax_fwd; delta [B, H, Nq] is a
+    workspace. See lasp.h."""
+    B, H, Nq, Nk, d, dt = _softmax_shapes(q, k, o, dout, dq)
+    _tokens(k, v, dk, dv)
+    _rows(lse, B, H, Nq)
+    _rows(delta, B, H, Nq)
+    scale = float(d) ** -0.5 if scale is None else float(scale)
+    _check(_load().lasp_softmax_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(dout), _ptr(dq), _ptr(dk),
+                                    _ptr(dv), _ptr(delta), B, H, Nq, Nk, q_offset, d, scale, dt,
+                                    _stream(stream, q)), "lasp_softmax_bwd")

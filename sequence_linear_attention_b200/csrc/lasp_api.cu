@@ -42,6 +42,17 @@ enum KernelId : int {
   K_STATE_TOTAL = 22,    // decayed total of a sequence's states (the LASP-2 shard state)
   K_GLA_SEG_STATES = 23,  // gated form on the tensor cores: segment states (forward)
   K_GLA_SEG_SCAN = 24,    // gated form: prefix over segments
+  // gated form, the exact CUDA-core sequence a tensor-core call switches to
+  // on the device when a tile's log-gates leave the factorized form's range
+  // (the kernels return at once otherwise)
+  K_GLA_EXACT_STATES = 25,
+  K_GLA_EXACT_SCAN = 26,
+  K_GLA_EXACT_OUT = 27,
+  K_GLA_EXACT_BWD = 28,
+  K_SOFTMAX_FWD = 29,    // softmax attention (hybrid layers): forward
+  K_SOFTMAX_DELTA = 30,  // softmax attention: rowsum(do . o)
+  K_SOFTMAX_DKDV = 31,   // softmax attention: dK, dV per key tile
+  K_SOFTMAX_DQ = 32,     // softmax attention: dQ per query tile
   K_COUNT
 };
 
@@ -464,6 +475,14 @@ const char* lasp_kernel_name(int id) {
     case K_STATE_TOTAL: return "state_total";
     case K_GLA_SEG_STATES: return "gla_segment_states_tc";
     case K_GLA_SEG_SCAN: return "gla_segment_scan";
+    case K_GLA_EXACT_STATES: return "gla_states_exact";
+    case K_GLA_EXACT_SCAN: return "gla_scan_exact";
+    case K_GLA_EXACT_OUT: return "gla_out_exact";
+    case K_GLA_EXACT_BWD: return "gla_bwd_exact";
+    case K_SOFTMAX_FWD: return "softmax_fwd_tc";
+    case K_SOFTMAX_DELTA: return "softmax_delta";
+    case K_SOFTMAX_DKDV: return "softmax_dkdv_tc";
+    case K_SOFTMAX_DQ: return "softmax_dq_tc";
     default: return "unknown";
   }
 }

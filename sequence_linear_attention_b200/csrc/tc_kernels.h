@@ -83,4 +83,19 @@ cudaError_t tc_gla_chunk_bwd(const void* q, const void* k, const void* v, const 
                              const float* P, const float* Rs, void* dq, void* dk, void* dv, float* dg, int B, int H,
                              int64_t N, int64_t t_slots, int stride, cudaStream_t st, RunIf run = {});
 
+// Causal softmax attention, bf16, d = 128 (k_tc_softmax.cu): queries at
+// positions q_offset + i (i < Nq) against keys / values at 0..Nk-1; lse
+// [B, H, Nq] (natural log); delta [B, H, Nq] = rowsum(do . o).
+bool tc_softmax_ok(int dtype, int d);
+cudaError_t tc_softmax_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int64_t Nq,
+                           int64_t Nk, int64_t q_offset, float scale, cudaStream_t st);
+cudaError_t tc_softmax_delta(const void* o, const void* dout, float* delta, int B, int H, int64_t Nq,
+                             cudaStream_t st);
+cudaError_t tc_softmax_dkdv(const void* q, const void* k, const void* v, const float* lse, const void* dout,
+                            void* dk, void* dv, const float* delta, int B, int H, int64_t Nq, int64_t Nk,
+                            int64_t q_offset, float scale, cudaStream_t st);
+cudaError_t tc_softmax_dq(const void* q, const void* k, const void* v, const float* lse, const void* dout, void* dq,
+                          const float* delta, int B, int H, int64_t Nq, int64_t Nk, int64_t q_offset, float scale,
+                          cudaStream_t st);
+
 }  // namespace lasp

@@ -150,6 +150,17 @@ def make_inputs(B: int, N: int, H: int, d: int, seed: int, bf16: bool = True,
     return out
 
 
+def make_attention_inputs(B: int, Nq: int, Nk: int, H: int, d: int, seed: int, bf16: bool = True) -> dict:
+    """Inputs of a softmax-attention layer: q and dO [B, Nq, H, d], k and v
+    [B, Nk, H, d], i.i.d. standard normal (the layer's own scale, d^-1/2 by
+    default, multiplies the scores), drawn like :func:`make_inputs` from the
+    streams of ``seed`` (q, k, v, dO), rounded to bf16 for bf16 workloads."""
+    out = {"q": draw_tensor(seed, 0, (B, Nq, H, d), 1.0, bf16), "k": draw_tensor(seed, 1, (B, Nk, H, d), 1.0, bf16),
+           "v": draw_tensor(seed, 2, (B, Nk, H, d), 1.0, bf16), "do": draw_tensor(seed, 3, (B, Nq, H, d), 1.0, bf16),
+           "bf16": bf16}
+    return out
+
+
 def as_f32(x: np.ndarray, bf16: bool) -> np.ndarray:
     """The float32 values a tensor from :func:`make_inputs` holds."""
     return bf16_bits_to_f32(x) if bf16 else np.ascontiguousarray(x, dtype=np.float32)

@@ -15,6 +15,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, HERE)
 import test_oracle_gla_pins as gpins  # noqa: E402
 import test_oracle_pins as pins  # noqa: E402
+import test_oracle_softmax_pins as spins  # noqa: E402
 
 SRC = os.path.join(os.path.dirname(HERE), "oracle", "lasp_oracle.c")
 
@@ -71,6 +72,19 @@ MUTATIONS = [
      "long r0 = kind == 0 ? t + 1 : 0, r1 = kind == 0 ? C - 1 : t;",
      "long r0 = kind == 0 ? t + 1 : 0, r1 = kind == 0 ? C - 1 : t - 1;", 0),
     ("gated scan uses one feature's gate for every row", "double g = exp(gc[i]);", "double g = exp(gc[0]);", 0),
+    ("softmax scores miss the scale", "s[j] = scale * acc;", "s[j] = acc;", 0),
+    ("softmax dq leaves out the row's softmax correction", "double ds = a * (da - rs[task]);",
+     "double ds = a * da;", 0),
+    ("softmax dk leaves out the row's softmax correction", "double ds = a * (da - rs[row]);",
+     "double ds = a * da;", 0),
+    ("softmax dk misses the scale", "dkj[f] += scale * ds * qi[f];", "dkj[f] += ds * qi[f];", 0),
+    ("softmax dv weighs do by ds instead of the attention weight", "dvj[f] += a * di[f];",
+     "dvj[f] += ds * di[f];", 0),
+    ("softmax key pass skips the query on the diagonal", "long i0 = j > q_offset ? j - q_offset : 0;",
+     "long i0 = j > q_offset ? j - q_offset + 1 : 0;", 0),
+    ("softmax correction term forgets the normaliser", "r += exp(s[j] - m) / l * da;",
+     "r += exp(s[j] - m) * da;", 0),
+    ("softmax output without the normaliser", "double a = s[j] / l;", "double a = s[j];", 0),
     ("gated gradient snapshots gate before adding the token",
      "for (int j = 0; j < d; ++j) S[i * d + j] = g * (S[i * d + j] + (double)xs[i] * ys[j]);",
      "for (int j = 0; j < d; ++j) S[i * d + j] = g * S[i * d + j] + (double)xs[i] * ys[j];", 0),
@@ -109,6 +123,9 @@ def _pins_pass():
         gpins.test_gate_gradient_identity,
         lambda: gpins.test_chunk_states_and_scans_equal_snapshots(4),
         lambda: gpins.test_recurrence_equals_chunk_form(8),
+        spins.test_two_token_worked_example,
+        lambda: spins.test_equals_torch_scaled_dot_product_attention(1, 2, 20, 50, 30, 8, 0.7),
+        spins.test_shards_equal_the_whole_sequence,
     ]
     for check in checks:
         try:
@@ -126,7 +143,7 @@ def test_pins_catch_the_mistake(tmp_path, name, old, new, nth):
     lib = ctypes.CDLL(so)
     for f in ("oracle_fwd", "oracle_bwd", "oracle_chunk_states", "oracle_state_scan", "oracle_state_snapshots",
               "oracle_bidir_fwd", "oracle_bidir_bwd", "oracle_gla_fwd", "oracle_gla_bwd", "oracle_gla_chunk_states",
-              "oracle_gla_state_scan", "oracle_gla_state_snapshots"):
+              "oracle_gla_state_scan", "oracle_gla_state_snapshots", "oracle_softmax_fwd", "oracle_softmax_bwd"):
         getattr(lib, f).argtypes = getattr(real, f).argtypes
         getattr(lib, f).restype = None
     lib.oracle_num_threads.restype = ctypes.c_int
