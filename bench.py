@@ -634,6 +634,123 @@ def run_gated(args, rank, world, local):
     }
 
 
+def softmax_flops(name: str, B: int, H: int, N: int, d: int) -> float:
+    """Tensor-core FLOPs of one launch of the softmax-attention kernels over
+    the causal pairs (j <= i: N (N + 1) / 2 per head), 2 d per pair and
+    product: the forward computes S and P V (4 d per pair); the dK/dV kernel
+    S^T, dP^T, dV and dK (8 d); the dQ kernel S, dP and dQ (6 d, of which S and
+    dP repeat the dK/dV kernel's: the minimal backward is 10 d per pair)."""
+    pairs = B * H * N * (N + 1) / 2
+    return {"softmax_fwd_tc": 4, "softmax_dkdv_tc": 8, "softmax_dq_tc": 6, "softmax_delta": 0}[name] * d * pairs
+
+
+def run_softmax(args, rank, world, local):
+    """The softmax-attention layers of a hybrid model (LASP-2H) on the
+    workload's shapes: a step is lasp_softmax_fwd + lasp_softmax_bwd over one
+    whole sequence (causal, scale d^-1/2), inputs standard normal. Printed as
+    its own line, with its own metric; the default run does not include it."""
+    import torch
+    import sequence_linear_attention_b200 as lasp
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    w = lasp_inputs.WORKLOADS[args.workload]
+    B, N, H, d = w["B"], (args.tokens or w["N"]), w["H"], w["d"]
+    if not w["bf16"] or d != 128:
+        raise ValueError("softmax attention is timed on a bf16 workload with d = 128")
+    inp = lasp_inputs.make_attention_inputs(B, N, N, H, d, seed=w["seed"] + 7919 * rank)
+    q, k, v, do = (torch.from_numpy(np.ascontiguousarray(inp[n]).view(np.int16)).view(torch.bfloat16).to(dev)
+                   for n in ("q", "k", "v", "do"))
+    o, dq, dk, dv = (torch.empty_like(q) for _ in range(4))
+    lse = torch.empty((B, H, N), dtype=torch.float32, device=dev)
+    delta = torch.empty_like(lse)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        lasp.lasp_softmax_fwd(q, k, v, o, lse)
+        lasp.lasp_softmax_bwd(q, k, v, o, lse, do, dq, dk, dv, delta)
+
+    for _ in range(args.warmup):
+        step()
+    events = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    torch.cuda.synchronize(dev)
+    barrier(world, dev)
+    with ClockSampler(local) as clk:
+        for i in range(args.steps):
+            events[i][0].record(stream)
+            step()
+            events[i][1].record(stream)
+        torch.cuda.synchronize(dev)
+    barrier(world, dev)
+    tokens = B * N
+    value, t_max = aggregate(tokens * args.steps, sum(a.elapsed_time(b) for a, b in events) / 1e3, world, dev)
+    ksteps = min(args.steps, 20)
+    lasp.lasp_trace_enable(8 * ksteps + 8)
+    for _ in range(ksteps):
+        step()
+    torch.cuda.synchronize(dev)
+    trace = lasp.lasp_trace_read(8 * ksteps + 8)
+    lasp.lasp_trace_enable(0)
+    st, site = lasp.lasp_check_device_status()
+    if st != 0:
+        raise RuntimeError(f"device status {lasp.lasp_status_string(st)} at site {site}")
+    per_kernel = {}
+    for name, ms in trace:
+        per_kernel.setdefault(name, []).append(ms)
+    peaks = load_peaks()
+    burst = t_max < 1.0
+    peak = peaks["bf16"] if burst else peaks["bf16_sustained"]
+    kernel_table = {}
+    for n, ms in per_kernel.items():
+        mean = statistics.mean(ms)
+        tf = softmax_flops(n, B, H, N, d) / (mean / 1e3) / 1e12
+        kernel_table[n] = {"launches_per_step": len(ms) / ksteps, "ms": round(mean, 4), "TFLOPs": round(tf, 1),
+                           "tensor_frac": round(tf / peak, 4)}
+    top = max(per_kernel, key=lambda n: sum(per_kernel[n]))
+    ms_step = t_max * 1e3 / args.steps
+    # the step at the minimal count: forward 4 d and backward 10 d per causal pair
+    step_tf = 14 * d * B * H * N * (N + 1) / 2 / (ms_step / 1e3) / 1e12
+    return {
+        "metric": "softmax-attention (LASP-2H layer) fwd+bwd tokens/s", "impl": "softmax",
+        "value": round(value, 1), "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms_step, 4), "higher_is_better": True,
+        "dtype": "bf16", "data": "synthetic (seeded standard-normal q, k, v, dO; no dataset)",
+        "config": {"workload": args.workload, "B": B, "H": H, "N": N, "d": d, "causal": True,
+                   "scale": "d^-1/2", "l2": "inputs larger than L2" if 4 * B * N * H * d * 2 > (126 << 20)
+                   else "inputs fit in L2"},
+        "tflops": round(step_tf, 1), "tensor_peak_frac": round(step_tf / peak, 4),
+        "tensor_peak_basis": "burst" if burst else "sustained",
+        "roofline": {"bound": "tensor", "kernel": top, "achieved": kernel_table[top]["TFLOPs"], "peak": peak,
+                     "unit": "TFLOP/s", "frac": kernel_table[top]["tensor_frac"], "traffic": None,
+                     "algorithmic_flops": softmax_flops(top, B, H, N, d), "peak_source": peaks["source"]},
+        "kernels": kernel_table,
+        "gpu_launches": int(round(len(trace) / ksteps * args.steps)),
+        "clocks": clk.summary(),
+    }
+
+
+def cpu_baseline_softmax(args):
+    """The oracle's softmax attention fwd+bwd on a bounded sample: all heads,
+    the first 4096 positions of batch 0. Its cost grows with the square of the
+    length, so the value is the sample's time per token scaled by the ratio of
+    the lengths (the workload's per-token work over the sample's)."""
+    import oracle
+    n = 4096
+    w = lasp_inputs.WORKLOADS[args.workload]
+    N = args.tokens or w["N"]
+    inp = lasp_inputs.make_attention_inputs(1, n, n, w["H"], w["d"], seed=w["seed"], bf16=True)
+    f = {x: lasp_inputs.as_f32(inp[x], True) for x in ("q", "k", "v", "do")}
+    oracle.build()
+    t0 = time.perf_counter()
+    oracle.softmax_fwd(f["q"], f["k"], f["v"])
+    oracle.softmax_bwd(f["q"], f["k"], f["v"], f["do"])
+    dt = time.perf_counter() - t0
+    value = 1.0 / (dt / n * (N / n))
+    return {"value": round(value, 1), "unit": "tokens/s", "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": f"fp64 oracle softmax attention fwd+bwd, batch 0, all heads, first {n} positions "
+                      f"({dt:.1f} s), per-token time scaled by {N}/{n} to the workload's length"}
+
+
 def run_lasp2(args, rank, world, local):
     """LASP-2 sequence parallelism: one sequence of the workload split over the
     ranks, rank r holding tokens [r L, (r + 1) L) with L = N / world; a step is
@@ -852,6 +969,9 @@ def main(argv=None):
                     help="time the bidirectional (unmasked) form instead (its own metric and line)")
     ap.add_argument("--gated", action="store_true",
                     help="time the gated form (a log-gate per token and key feature) instead (its own metric and line)")
+    ap.add_argument("--softmax", action="store_true",
+                    help="time the softmax-attention layers of the hybrid model (LASP-2H) instead "
+                         "(its own metric and line)")
     ap.add_argument("--lasp2", action="store_true",
                     help="time LASP-2 sequence parallelism instead: one sequence split over the ranks "
                          "(its own metric and line)")
@@ -875,6 +995,10 @@ def main(argv=None):
             line = run_lasp2(args, rank, world, local)
             if rank == 0 and world == 1 and not args.no_cpu_baseline:
                 line["cpu_baseline"] = cpu_baseline(args)
+        elif args.softmax:
+            line = run_softmax(args, rank, world, local)
+            if rank == 0 and world == 1 and not args.no_cpu_baseline:
+                line["cpu_baseline"] = cpu_baseline_softmax(args)
         elif args.gated:
             line = run_gated(args, rank, world, local)
             if rank == 0 and world == 1 and not args.no_cpu_baseline:
