@@ -792,9 +792,11 @@ def run_lasp2(args, rank, world, local):
     ws = torch.empty_like(cache)
     stream = torch.cuda.current_stream(dev)
 
+    parts = args.parts or lasp2.default_parts(q, C, world)
+
     def step():
-        lasp2.lasp2_fwd(q, k, v, decay, o, C, cache)
-        lasp2.lasp2_bwd(q, k, v, decay, do, dq, dk, dv, C, cache, ws)
+        lasp2.lasp2_fwd(q, k, v, decay, o, C, cache, parts=parts)
+        lasp2.lasp2_bwd(q, k, v, decay, do, dq, dk, dv, C, cache, ws, parts=parts)
 
     try:
         for _ in range(args.warmup):
@@ -853,7 +855,9 @@ def run_lasp2(args, rank, world, local):
         "scaling": "strong", "vs_baseline": None, "dtype": "bf16" if w["bf16"] else "f32",
         "data": "synthetic (seeded normal q,k,v,dO; no dataset)",
         "config": {"workload": args.workload, "B": B, "H": H, "N": N, "d": d, "C": C, "shard_tokens": L,
-                   "segment": G, "parallelism": f"sequence x{world} (one AllGather of shard states per direction)",
+                   "segment": G, "parts": parts,
+                   "parallelism": f"sequence x{world} (AllGathers of shard states per direction, one per part of "
+                                  f"the (b, h) pairs, each overlapping the next part's work)",
                    "l2": "inputs larger than L2"},
         "roofline": {"bound": "hbm", "kernel": top, "achieved": kernel_table[top]["GBps"], "peak": peaks["hbm"],
                      "unit": "GB/s", "frac": kernel_table[top]["hbm_frac"], "traffic": None,
@@ -975,6 +979,8 @@ def main(argv=None):
     ap.add_argument("--lasp2", action="store_true",
                     help="time LASP-2 sequence parallelism instead: one sequence split over the ranks "
                          "(its own metric and line)")
+    ap.add_argument("--parts", type=int, default=None,
+                    help="with --lasp2: parts of the (b, h) pairs whose exchanges overlap (default: the library's)")
     ap.add_argument("--tokens", type=int, default=None,
                     help="sequence length N instead of the workload's (a smaller case of the same shape, for "
                          "profiling); the line is then not the workload's headline number")

@@ -238,6 +238,37 @@ LASP_API int lasp_bwd_finish(const void* q, const void* k, const void* v, const 
                              void* stream);
 
 /*
+ * lasp_fwd_states_part, lasp_fwd_finish_part, lasp_bwd_states_part,
+ * lasp_bwd_finish_part -- the four split calls above restricted to part `part`
+ * of `nparts` (0 <= part < nparts <= B * H) of the (b, h) pairs, taken in
+ * b-major order: pairs floor(B H part / nparts) .. floor(B H (part + 1) / nparts) - 1.
+ * Calling every part of a step gives exactly the whole call's results; each
+ * part reads and writes only its own pairs' slices of every tensor, and the
+ * state arrays (total, init_state, dstate_in, dinit_state) stay full
+ * [B, H, d, d] arrays of which a part touches its own pairs. This lets LASP-2's
+ * exchange of one part's shard states run while the next part's states, and
+ * the last part's output, are computed (LASP-2 review page, "Core claim": the
+ * AllGather of fixed-size states overlaps computation). nparts = 1 is the
+ * whole call; nparts > 1 needs lasp_parts_ok (LASP_ERR_UNSUPPORTED otherwise).
+ */
+LASP_API int lasp_fwd_states_part(const void* k, const void* v, const float* decay, int B, int H, int64_t N, int d,
+                                  int C, int dtype, float* state_cache, float* total, int part, int nparts,
+                                  void* stream);
+LASP_API int lasp_fwd_finish_part(const void* q, const void* k, const void* v, const float* decay, void* o, int B,
+                                  int H, int64_t N, int d, int C, int dtype, float* state_cache,
+                                  const float* init_state, int part, int nparts, void* stream);
+LASP_API int lasp_bwd_states_part(const void* q, const void* dout, const float* decay, int B, int H, int64_t N, int d,
+                                  int C, int dtype, float* dstate_ws, float* total, int part, int nparts,
+                                  void* stream);
+LASP_API int lasp_bwd_finish_part(const void* q, const void* k, const void* v, const float* decay, const void* dout,
+                                  void* dq, void* dk, void* dv, int B, int H, int64_t N, int d, int C, int dtype,
+                                  const float* state_cache, float* dstate_ws, const float* dstate_in,
+                                  float* dinit_state, int part, int nparts, void* stream);
+/* 1 when the part calls accept nparts > 1 for these sizes (both segment walks
+ * run: bf16, d = 128, C dividing 128, N a multiple of 128), else 0. */
+LASP_API int lasp_parts_ok(int64_t N, int C, int d, int dtype);
+
+/*
  * lasp_bwd_noalloc -- lasp_bwd without the caller-provided workspace.
  * The pages have no counterpart to this call; it exists for callers that
  * cannot allocate device memory: a plain C program or plug-in with no device

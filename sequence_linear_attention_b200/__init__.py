@@ -25,7 +25,8 @@ __all__ = [
     "lasp_status_string", "lasp_version", "lasp_trace_enable", "lasp_trace_read", "lasp_kernel_name",
     "lasp_segment_tokens", "lasp_bidir_workspace_floats", "lasp_bidir_state_offset", "lasp_bidir_fwd",
     "lasp_bidir_bwd", "lasp_gla_cache_floats", "lasp_gla_chunk_states", "lasp_gla_state_prefix", "lasp_gla_fwd",
-    "lasp_gla_bwd", "lasp_softmax_fwd", "lasp_softmax_bwd",
+    "lasp_gla_bwd", "lasp_softmax_fwd", "lasp_softmax_bwd", "lasp_fwd_states_part", "lasp_fwd_finish_part",
+    "lasp_bwd_states_part", "lasp_bwd_finish_part", "lasp_parts_ok",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -92,6 +93,12 @@ def _load():
             lib.lasp_gla_state_prefix.argtypes = [P, P, P, P, P, I, I, I, I, I, P]
             lib.lasp_gla_fwd.argtypes = [P, P, P, P, P, I, I, L, I, I, I, P, P, P]
             lib.lasp_gla_bwd.argtypes = [P, P, P, P, P, P, P, P, P, I, I, L, I, I, I, P, P, P, P, P]
+            lib.lasp_fwd_states_part.argtypes = [P, P, P, I, I, L, I, I, I, P, P, I, I, P]
+            lib.lasp_fwd_finish_part.argtypes = [P, P, P, P, P, I, I, L, I, I, I, P, P, I, I, P]
+            lib.lasp_bwd_states_part.argtypes = [P, P, P, I, I, L, I, I, I, P, P, I, I, P]
+            lib.lasp_bwd_finish_part.argtypes = [P, P, P, P, P, P, P, P, I, I, L, I, I, I, P, P, P, P, I, I, P]
+            lib.lasp_parts_ok.argtypes = [L, I, I, I]
+            lib.lasp_parts_ok.restype = I
             F = ctypes.c_float
             lib.lasp_softmax_fwd.argtypes = [P, P, P, P, P, I, I, L, L, L, I, F, I, P]
             lib.lasp_softmax_bwd.argtypes = [P, P, P, P, P, P, P, P, P, P, I, I, L, L, L, I, F, I, P]
@@ -104,7 +111,8 @@ def _load():
                       lib.lasp_wait_probe, lib.lasp_version, lib.lasp_trace_enable, lib.lasp_trace_read,
                       lib.lasp_segment_tokens, lib.lasp_bidir_fwd, lib.lasp_bidir_bwd,
                       lib.lasp_gla_chunk_states, lib.lasp_gla_state_prefix, lib.lasp_gla_fwd,
-                      lib.lasp_gla_bwd, lib.lasp_softmax_fwd, lib.lasp_softmax_bwd):
+                      lib.lasp_gla_bwd, lib.lasp_softmax_fwd, lib.lasp_softmax_bwd, lib.lasp_fwd_states_part,
+                      lib.lasp_fwd_finish_part, lib.lasp_bwd_states_part, lib.lasp_bwd_finish_part):
                 f.restype = I
             _lib = lib
     return _lib
@@ -196,6 +204,43 @@ def lasp_bwd_finish(q, k, v, decay, dout, dq, dk, dv, C, state_cache, dstate_ws,
     _check(_load().lasp_bwd_finish(_ptr(q), _ptr(k), _ptr(v), _ptr(decay), _ptr(dout), _ptr(dq), _ptr(dk), _ptr(dv),
                                    B, H, N, d, C, dt, _ptr(state_cache), _ptr(dstate_ws), _ptr(dstate_in),
                                    _ptr(dinit_state), _stream(stream, q)), "lasp_bwd_finish")
+
+
+def lasp_fwd_states_part(k, v, decay, C, state_cache, total, part, nparts, stream=None):
+    """lasp_fwd_states for part `part` of `nparts` of the (b, h) pairs. See lasp.h."""
+    B, N, H, d, dt = _tokens(k, v)
+    _check(_load().lasp_fwd_states_part(_ptr(k), _ptr(v), _ptr(decay), B, H, N, d, C, dt, _ptr(state_cache),
+                                        _ptr(total), part, nparts, _stream(stream, k)), "lasp_fwd_states_part")
+
+
+def lasp_fwd_finish_part(q, k, v, decay, o, C, state_cache, init_state, part, nparts, stream=None):
+    """lasp_fwd_finish for part `part` of `nparts` of the (b, h) pairs. See lasp.h."""
+    B, N, H, d, dt = _tokens(q, k, v, o)
+    _check(_load().lasp_fwd_finish_part(_ptr(q), _ptr(k), _ptr(v), _ptr(decay), _ptr(o), B, H, N, d, C, dt,
+                                        _ptr(state_cache), _ptr(init_state), part, nparts, _stream(stream, q)),
+           "lasp_fwd_finish_part")
+
+
+def lasp_bwd_states_part(q, dout, decay, C, dstate_ws, total, part, nparts, stream=None):
+    """lasp_bwd_states for part `part` of `nparts` of the (b, h) pairs. See lasp.h."""
+    B, N, H, d, dt = _tokens(q, dout)
+    _check(_load().lasp_bwd_states_part(_ptr(q), _ptr(dout), _ptr(decay), B, H, N, d, C, dt, _ptr(dstate_ws),
+                                        _ptr(total), part, nparts, _stream(stream, q)), "lasp_bwd_states_part")
+
+
+def lasp_bwd_finish_part(q, k, v, decay, dout, dq, dk, dv, C, state_cache, dstate_ws, dstate_in, dinit_state, part,
+                         nparts, stream=None):
+    """lasp_bwd_finish for part `part` of `nparts` of the (b, h) pairs. See lasp.h."""
+    B, N, H, d, dt = _tokens(q, k, v, dout, dq, dk, dv)
+    _check(_load().lasp_bwd_finish_part(_ptr(q), _ptr(k), _ptr(v), _ptr(decay), _ptr(dout), _ptr(dq), _ptr(dk),
+                                        _ptr(dv), B, H, N, d, C, dt, _ptr(state_cache), _ptr(dstate_ws),
+                                        _ptr(dstate_in), _ptr(dinit_state), part, nparts, _stream(stream, q)),
+           "lasp_bwd_finish_part")
+
+
+def lasp_parts_ok(N, C, d, dtype):
+    """1 when the part calls accept nparts > 1 for these sizes. See lasp.h."""
+    return int(_load().lasp_parts_ok(N, C, d, dtype))
 
 
 def lasp_bwd_noalloc(q, k, v, decay, dout, dq, dk, dv, C, state_cache, dstate_in=None, dinit_state=None,

@@ -50,9 +50,11 @@ __global__ void __launch_bounds__(kThreads) state_scan_kernel(const float4* M, f
                                                               float4* __restrict__ total, int H, int T,
                                                               int d, int dd4, int64_t n_threads, float Cf,
                                                               int reverse, int64_t t_slots, int slot_stride,
-                                                              int slot_offset, int gsum_offset, RunIf run_if) {
+                                                              int slot_offset, int gsum_offset, RunIf run_if,
+                                                              int64_t idx0) {
   if (!runs(run_if)) return;
-  for (int64_t idx = (int64_t)blockIdx.x * kThreads + threadIdx.x; idx < n_threads;
+  // threads idx0 .. idx0 + n_threads - 1 of the whole (b, h, float4) space
+  for (int64_t idx = idx0 + (int64_t)blockIdx.x * kThreads + threadIdx.x; idx < idx0 + n_threads;
        idx += (int64_t)gridDim.x * kThreads) {
   const int e = (int)(idx % dd4);
   const int h = (int)((idx / dd4) % H);
@@ -128,13 +130,15 @@ __global__ void __launch_bounds__(kThreads) state_scan_kernel(const float4* M, f
 
 cudaError_t launch_state_scan_slots(const float* M, float* P, const float* decay, const float* init, float* total,
                                     int B, int T, int H, int d, int64_t C, int reverse, int64_t t_slots,
-                                    int slot_stride, int slot_offset, cudaStream_t st) {
+                                    int slot_stride, int slot_offset, cudaStream_t st, int64_t bh0, int64_t nbh) {
   const int dd4 = d * d / 4;
-  const int64_t n_threads = (int64_t)B * H * dd4;
+  if (nbh < 0) nbh = (int64_t)B * H;
+  const int64_t n_threads = nbh * dd4;
+  if (n_threads == 0) return cudaSuccess;
   const int64_t blocks = (n_threads + scan_detail::kThreads - 1) / scan_detail::kThreads;
   scan_detail::state_scan_kernel<false><<<(unsigned)blocks, scan_detail::kThreads, 0, st>>>(
       (const float4*)M, (float4*)P, decay, nullptr, (const float4*)init, (float4*)total, H, T, d, dd4,
-      n_threads, (float)C, reverse, t_slots, slot_stride, slot_offset, 0, RunIf{});
+      n_threads, (float)C, reverse, t_slots, slot_stride, slot_offset, 0, RunIf{}, bh0 * dd4);
   return cudaGetLastError();
 }
 
@@ -146,7 +150,7 @@ cudaError_t launch_gla_scan(const float* M, float* P, const float* gsum, const f
   const int64_t blocks = grid_for((n_threads + scan_detail::kThreads - 1) / scan_detail::kThreads, run);
   scan_detail::state_scan_kernel<true><<<(unsigned)blocks, scan_detail::kThreads, 0, st>>>(
       (const float4*)M, (float4*)P, nullptr, gsum, (const float4*)init, (float4*)total, H, T, d, dd4, n_threads,
-      1.f, reverse, t_slots, slot_stride, slot_offset, gsum_offset, run);
+      1.f, reverse, t_slots, slot_stride, slot_offset, gsum_offset, run, 0);
   return cudaGetLastError();
 }
 

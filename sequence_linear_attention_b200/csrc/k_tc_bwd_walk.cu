@@ -121,7 +121,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_walk_tc(
     const __grid_constant__ CUtensorMap map_dv,
     const __grid_constant__ CUtensorMap map_state, const float* decay, const float* __restrict__ P,
     float* __restrict__ R, int H, int64_t N, int T, int C, int G, int nseg,
-    int64_t nitems) {
+    int64_t nitems, int64_t item0) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   uint8_t* sK = base + 1 * kTileBytes;
@@ -212,7 +212,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_walk_tc(
       };
 
       if ((int64_t)blockIdx.x < nitems) {
-        const Item first = item_of(blockIdx.x, H, nseg);
+        const Item first = item_of(item0 + blockIdx.x, H, nseg);
         load_kv(first, tiles - 1);
         load_qd(first, tiles - 1, 0);
         load_p(first, tiles - 1);
@@ -222,7 +222,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_walk_tc(
       int prev_row = 0;
       bool ok = true;
       for (int64_t w = blockIdx.x; w < nitems && ok; w += gridDim.x) {
-        const Item item = item_of(w, H, nseg);
+        const Item item = item_of(item0 + w, H, nseg);
         for (int t = tiles - 1; t >= 0 && ok; --t, ++it) {
           const uint32_t par = it & 1u;
           const int row0 = item.seg * G + t * kTile;
@@ -256,7 +256,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_walk_tc(
           if (nt < 0) {
             has_next = w + gridDim.x < nitems;
             if (has_next) {
-              nx = item_of(w + gridDim.x, H, nseg);
+              nx = item_of(item0 + w + gridDim.x, H, nseg);
               nt = tiles - 1;
             }
           }
@@ -277,7 +277,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_walk_tc(
           }
           if (t == (tiles > 1 ? 1 : 0) && w + gridDim.x < nitems) {
             // and the next segment's entering R, read at the segment switch
-            const Item ns = item_of(w + gridDim.x, H, nseg);
+            const Item ns = item_of(item0 + w + gridDim.x, H, nseg);
             const int64_t slot = (int64_t)(ns.seg + 1) * (G / C) - 1;
             bulk_prefetch_l2(R + (((int64_t)ns.b * T + slot) * H + ns.h) * kD * kD, kD * kD * sizeof(float));
           }
@@ -378,7 +378,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_walk_tc(
     uint32_t nseg_done = 0;  // segments started by this CTA
     for (int64_t w = blockIdx.x; w < nitems; w += gridDim.x) {
       if (named_sync_or(kEpiBar, kEpiThreads, bad)) break;  // every epilogue thread is past the last segment
-      const Item item = item_of(w, H, nseg);
+      const Item item = item_of(item0 + w, H, nseg);
       const float lam = load_decay(decay, item.h);
       const float l2 = log2f(lam);
       const bool scale = lam != 1.0f;
@@ -592,7 +592,7 @@ bool tc_bwd_walk_ok(int dtype, int d, int64_t C, int64_t N) {
 
 cudaError_t tc_bwd_walk(const void* q, const void* k, const void* v, const void* dout, const float* decay,
                         const float* P, float* R, void* dq, void* dk, void* dv, int B, int H, int64_t N, int d, int C,
-                        int G, int num_sms, cudaStream_t st) {
+                        int G, int num_sms, cudaStream_t st, int64_t bh0, int64_t nbh) {
   using namespace tc_bwd_walk_detail;
   CUtensorMap mq, mk, mv, mdo, mdq, mdk, mdv, mr;
   if (!make_token_map(&mq, q, B, H, N, d, kTile) || !make_token_map(&mk, k, B, H, N, d, kTile) ||
@@ -605,10 +605,13 @@ cudaError_t tc_bwd_walk(const void* q, const void* k, const void* v, const void*
   cudaError_t e = cudaFuncSetAttribute(bwd_walk_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   const int nseg = (int)(N / G);
-  const int64_t nitems = (int64_t)B * H * nseg;
+  // the segments of (b, h) pairs bh0 .. bh0 + nbh - 1 (items in b, h, segment order)
+  if (nbh < 0) nbh = (int64_t)B * H;
+  const int64_t nitems = nbh * nseg;
+  if (nitems == 0) return cudaSuccess;
   const unsigned grid = (unsigned)std::min<int64_t>(nitems, num_sms);
   bwd_walk_tc<<<grid, kThreads, smem, st>>>(mq, mk, mv, mdo, mdq, mdk, mdv, mr, decay, P, R, H, N, (int)(N / C), C, G,
-                                            nseg, nitems);
+                                            nseg, nitems, bh0 * nseg);
   return cudaGetLastError();
 }
 

@@ -101,7 +101,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_walk_tc(const __grid_constant
                                                             const __grid_constant__ CUtensorMap map_state,
                                                             const float* decay, float* __restrict__ P, int H,
                                                             int T, int C, int G, int nseg, int64_t nitems,
-                                                            int cache_bf16) {
+                                                            int cache_bf16, int64_t item0) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   uint8_t* sP = base + 6 * kTileBytes;
@@ -179,7 +179,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_walk_tc(const __grid_constant
       };
 
       if ((int64_t)blockIdx.x < nitems) {
-        const Item first = item_of(blockIdx.x, H, nseg);
+        const Item first = item_of(item0 + blockIdx.x, H, nseg);
         issue_loads(0, first, 0);
         issue_state_load(1, first);
       }
@@ -188,7 +188,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_walk_tc(const __grid_constant
       int prev_row = 0;
       bool ok = true;
       for (int64_t w = blockIdx.x; w < nitems && ok; w += gridDim.x) {
-        const Item item = item_of(w, H, nseg);
+        const Item item = item_of(item0 + w, H, nseg);
         for (int t = 0; t < tiles && ok; ++t, ++it) {
           const int set = it & 1;
           const uint32_t par = it & 1u;
@@ -211,7 +211,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_walk_tc(const __grid_constant
           if (nt == tiles) {
             nt = 0;
             has_next = w + gridDim.x < nitems;
-            if (has_next) nx = item_of(w + gridDim.x, H, nseg);
+            if (has_next) nx = item_of(item0 + w + gridDim.x, H, nseg);
           }
           if (has_next) {
             if (it > 0 && !(ok = mbar_wait_or_abort(&s->mma2[set ^ 1], ppar, SITE_OUT_MMA, abort_flag))) break;
@@ -221,7 +221,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_walk_tc(const __grid_constant
           if (t == (tiles > 1 ? tiles - 2 : 0) && w + gridDim.x < nitems) {
             // the next segment's entering state, into L2 while this segment's
             // last tiles run
-            const Item ns = item_of(w + gridDim.x, H, nseg);
+            const Item ns = item_of(item0 + w + gridDim.x, H, nseg);
             const int64_t slot = ((int64_t)ns.seg * G) / C;
             bulk_prefetch_l2(P + (((int64_t)ns.b * T + slot) * H + ns.h) * kD * kD, kD * kD * sizeof(float));
           }
@@ -239,7 +239,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_walk_tc(const __grid_constant
           // segment's entering state goes there
           if (t == tiles - 1 && w + gridDim.x < nitems) {
             if (!(ok = mbar_wait_or_abort(&s->mma2[set], (it >> 1) & 1u, SITE_OUT_MMA, abort_flag))) break;
-            issue_state_load(set, item_of(w + gridDim.x, H, nseg));
+            issue_state_load(set, item_of(item0 + w + gridDim.x, H, nseg));
           }
           prev = item;
           prev_row = row0;
@@ -308,7 +308,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_walk_tc(const __grid_constant
     uint32_t it = 0, nsg = 0;
     for (int64_t w = blockIdx.x; w < nitems; w += gridDim.x) {
       if (named_sync_or(kEpiBar, kEpiThreads, bad)) break;  // every epilogue thread is past the last segment
-      const Item item = item_of(w, H, nseg);
+      const Item item = item_of(item0 + w, H, nseg);
       const float lam = load_decay(decay, item.h);
       const float l2 = log2f(lam);
       const bool scale = lam != 1.0f;
@@ -530,7 +530,8 @@ int walk_segment_tokens(int64_t N, int C) {
 }
 
 cudaError_t tc_fwd_walk(const void* q, const void* k, const void* v, const float* decay, float* P, void* o, int B,
-                        int H, int64_t N, int d, int C, int G, int num_sms, cudaStream_t st) {
+                        int H, int64_t N, int d, int C, int G, int num_sms, cudaStream_t st, int64_t bh0,
+                        int64_t nbh) {
   using namespace tc_fwd_walk_detail;
   CUtensorMap mq, mk, mv, mo, mp;
   if (!make_token_map(&mq, q, B, H, N, d, kTile) || !make_token_map(&mk, k, B, H, N, d, kTile) ||
@@ -541,14 +542,17 @@ cudaError_t tc_fwd_walk(const void* q, const void* k, const void* v, const float
   cudaError_t e = cudaFuncSetAttribute(fwd_walk_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   const int nseg = (int)(N / G);
-  const int64_t nitems = (int64_t)B * H * nseg;
+  // the segments of (b, h) pairs bh0 .. bh0 + nbh - 1 (items in b, h, segment order)
+  if (nbh < 0) nbh = (int64_t)B * H;
+  const int64_t nitems = nbh * nseg;
+  if (nitems == 0) return cudaSuccess;
   const unsigned grid = (unsigned)std::min<int64_t>(nitems, num_sms);
   // with chunks that divide the tile the backward walk reads the cache: it gets
   // each tile's entering state as the bf16 operand tile (in the slot of the
   // tile's first chunk); with longer chunks the cache holds fp32 states
   const int cache_bf16 = C <= kTile ? 1 : 0;
   fwd_walk_tc<<<grid, kThreads, smem, st>>>(mq, mk, mv, mo, mp, decay, P, H, (int)(N / C), C, G, nseg, nitems,
-                                           cache_bf16);
+                                           cache_bf16, bh0 * nseg);
   return cudaGetLastError();
 }
 

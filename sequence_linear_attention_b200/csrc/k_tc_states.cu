@@ -61,8 +61,8 @@ __device__ __forceinline__ uint32_t bf16x2_scale(uint32_t x, float w) {
 struct Work {
   int c, h, b;
 };
-__device__ __forceinline__ Work work_of(int64_t n, int T, int H) {
-  const int64_t w = blockIdx.x + n * gridDim.x;
+__device__ __forceinline__ Work work_of(int64_t n, int T, int H, int64_t item0) {
+  const int64_t w = item0 + blockIdx.x + n * gridDim.x;
   Work r;
   r.c = (int)(w % T);
   r.h = (int)((w / T) % H);
@@ -83,7 +83,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_states_tc(const __grid_cons
                                                             const float* decay, int H,
                                                             int C, int KB, int nslots, int kind, int T,
                                                             int64_t nitems, int64_t t_out, int slot_stride,
-                                                            int slot_offset) {
+                                                            int slot_offset, int64_t item0) {
   extern __shared__ uint8_t smem_raw[];
   // tiles need 1024-byte alignment for the 128-byte swizzle atoms
   uint8_t* tiles = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
@@ -134,7 +134,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_states_tc(const __grid_cons
           s->abort = 1;
           break;
         }
-        const Work wk = work_of(g / nstages, T, H);
+        const Work wk = work_of(g / nstages, T, H, item0);
         const int row = wk.c * C + (int)(g % nstages) * KB;
         uint8_t* a = tiles + (size_t)slot * 2 * tile_bytes;
         uint8_t* bb = a + tile_bytes;
@@ -189,7 +189,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_states_tc(const __grid_cons
       const int k = (int)(g % nstages);
       const int64_t n = g / nstages;
       if (k == 0) {
-        wk = work_of(n, T, H);
+        wk = work_of(n, T, H, item0);
         lam = load_decay(decay, wk.h);
         l2 = log2f(lam);
       }
@@ -282,7 +282,7 @@ bool tc_states_ok(int dtype, int d, int64_t C) {
 
 cudaError_t tc_chunk_states_slots(const void* a, const void* bm, const float* decay, float* M, int B, int H,
                                   int64_t N, int d, int C, int kind, int64_t t_out, int slot_stride, int slot_offset,
-                                  cudaStream_t st) {
+                                  cudaStream_t st, int64_t bh0, int64_t nbh) {
   using namespace tc_states_detail;
   const int KB = stage_rows(C);
   CUtensorMap ma, mb, mm;
@@ -296,10 +296,12 @@ cudaError_t tc_chunk_states_slots(const void* a, const void* bm, const float* de
   int dev = 0, sms = 148;
   if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int T = (int)(N / C);
-  const int64_t nitems = (int64_t)B * H * T;
+  if (nbh < 0) nbh = (int64_t)B * H;  // (b, h) pairs bh0 .. bh0 + nbh - 1, in b-major order
+  const int64_t nitems = nbh * T;
+  if (nitems == 0) return cudaSuccess;
   const unsigned grid = (unsigned)std::min<int64_t>(nitems, sms);
   chunk_states_tc<<<grid, kThreads, smem, st>>>(ma, mb, mm, decay, H, C, KB, nslots, kind, T, nitems, t_out,
-                                               slot_stride, slot_offset);
+                                               slot_stride, slot_offset, bh0 * T);
   return cudaGetLastError();
 }
 

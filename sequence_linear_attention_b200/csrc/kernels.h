@@ -33,9 +33,12 @@ cudaError_t launch_state_scan(const float* M, float* P, const float* decay, cons
 
 // The same scan over every slot_stride-th state of an array of t_slots states,
 // starting at slot slot_offset (segment states stored inside a chunk array).
+// bh0, nbh: only the (b, h) pairs bh0 .. bh0 + nbh - 1 (b-major; nbh < 0: all);
+// init and total stay [B, H, d, d] arrays.
 cudaError_t launch_state_scan_slots(const float* M, float* P, const float* decay, const float* init, float* total,
                                     int B, int T, int H, int d, int64_t C, int reverse, int64_t t_slots,
-                                    int slot_stride, int slot_offset, cudaStream_t st);
+                                    int slot_stride, int slot_offset, cudaStream_t st, int64_t bh0 = 0,
+                                    int64_t nbh = -1);
 
 // CUDA-core kernels, any d in {32, 64, 128} and any C (k_simt.cu).
 // kind 0: M_c = sum lambda^{C-1-t} a_t^T b_t ; kind 1: sum lambda^{t+1} a_t^T b_t.

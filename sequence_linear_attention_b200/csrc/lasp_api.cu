@@ -154,8 +154,10 @@ int chunk_grads_impl(const void* q, const void* k, const void* v, const void* do
 // lasp_fwd in two parts. States: the chunk (or, on the walk path, segment)
 // states into the cache and, if total is non-NULL, their decayed total with a
 // zero start. Finish: the prefix from init and the output.
+// bh0, nbh (walk path only): the (b, h) pairs bh0 .. bh0 + nbh - 1; nbh < 0: all.
 int fwd_states_impl(const void* k, const void* v, const float* decay, int B, int H, int64_t N, int d, int C,
-                    int dtype, float* state_cache, float* total, cudaStream_t st) {
+                    int dtype, float* state_cache, float* total, cudaStream_t st, int64_t bh0 = 0,
+                    int64_t nbh = -1) {
   const int T = (int)(N / C);
   int s;
   if (tc_fwd_walk_ok(dtype, d, C, N)) {
@@ -163,13 +165,13 @@ int fwd_states_impl(const void* k, const void* v, const float* decay, int B, int
     const int G = walk_segment_tokens(N, C);
     const int stride = G / C;
     if ((s = cuda_status(traced(K_SEG_STATES, st, [&] {
-           return tc_chunk_states_slots(k, v, decay, state_cache, B, H, N, d, G, 0, T, stride, 0, st);
+           return tc_chunk_states_slots(k, v, decay, state_cache, B, H, N, d, G, 0, T, stride, 0, st, bh0, nbh);
          }))))
       return s;
     if (!total) return LASP_OK;
     return cuda_status(traced(K_STATE_TOTAL, st, [&] {
       return launch_state_scan_slots(state_cache, nullptr, decay, nullptr, total, B, (int)(N / G), H, d, G, 0, T,
-                                     stride, 0, st);
+                                     stride, 0, st, bh0, nbh);
     }));
   }
   if ((s = chunk_states_impl(k, v, decay, state_cache, B, H, N, d, C, dtype, 0, st))) return s;
@@ -177,7 +179,8 @@ int fwd_states_impl(const void* k, const void* v, const float* decay, int B, int
 }
 
 int fwd_finish_impl(const void* q, const void* k, const void* v, const float* decay, void* o, int B, int H, int64_t N,
-                    int d, int C, int dtype, float* state_cache, const float* init_state, cudaStream_t st) {
+                    int d, int C, int dtype, float* state_cache, const float* init_state, cudaStream_t st,
+                    int64_t bh0 = 0, int64_t nbh = -1) {
   const int T = (int)(N / C);
   int s;
   if (tc_fwd_walk_ok(dtype, d, C, N)) {
@@ -188,12 +191,12 @@ int fwd_finish_impl(const void* q, const void* k, const void* v, const float* de
     const int stride = G / C;
     if ((s = cuda_status(traced(K_SEG_SCAN, st, [&] {
            return launch_state_scan_slots(state_cache, state_cache, decay, init_state, nullptr, B, (int)(N / G), H, d,
-                                          G, 0, T, stride, 0, st);
+                                          G, 0, T, stride, 0, st, bh0, nbh);
          }))))
       return s;
     const int sms = num_sms_current_device();
     return cuda_status(traced(K_FWD_WALK, st, [&] {
-      return tc_fwd_walk(q, k, v, decay, state_cache, o, B, H, N, d, C, G, sms, st);
+      return tc_fwd_walk(q, k, v, decay, state_cache, o, B, H, N, d, C, G, sms, st, bh0, nbh);
     }));
   }
   // exclusive prefix in place -> P_c; then the output
@@ -206,7 +209,7 @@ int fwd_finish_impl(const void* q, const void* k, const void* v, const float* de
 // entering from after the sequence. Finish: the suffix from dstate_in (and
 // dinit) and dQ, dK, dV.
 int bwd_states_impl(const void* q, const void* dout, const float* decay, int B, int H, int64_t N, int d, int C,
-                    int dtype, float* dstate_ws, float* total, cudaStream_t st) {
+                    int dtype, float* dstate_ws, float* total, cudaStream_t st, int64_t bh0 = 0, int64_t nbh = -1) {
   const int T = (int)(N / C);
   int s;
   if (tc_bwd_walk_ok(dtype, d, C, N)) {
@@ -214,13 +217,14 @@ int bwd_states_impl(const void* q, const void* dout, const float* decay, int B, 
     const int G = walk_segment_tokens(N, C);
     const int stride = G / C;
     if ((s = cuda_status(traced(K_SEG_STATES, st, [&] {
-           return tc_chunk_states_slots(q, dout, decay, dstate_ws, B, H, N, d, G, 1, T, stride, stride - 1, st);
+           return tc_chunk_states_slots(q, dout, decay, dstate_ws, B, H, N, d, G, 1, T, stride, stride - 1, st, bh0,
+                                        nbh);
          }))))
       return s;
     if (!total) return LASP_OK;
     return cuda_status(traced(K_STATE_TOTAL, st, [&] {
       return launch_state_scan_slots(dstate_ws, nullptr, decay, nullptr, total, B, (int)(N / G), H, d, G, 1, T,
-                                     stride, stride - 1, st);
+                                     stride, stride - 1, st, bh0, nbh);
     }));
   }
   if ((s = chunk_states_impl(q, dout, decay, dstate_ws, B, H, N, d, C, dtype, 1, st))) return s;
@@ -229,7 +233,8 @@ int bwd_states_impl(const void* q, const void* dout, const float* decay, int B, 
 
 int bwd_finish_impl(const void* q, const void* k, const void* v, const float* decay, const void* dout, void* dq,
                     void* dk, void* dv, int B, int H, int64_t N, int d, int C, int dtype, const float* state_cache,
-                    float* dstate_ws, const float* dstate_in, float* dinit_state, cudaStream_t st) {
+                    float* dstate_ws, const float* dstate_in, float* dinit_state, cudaStream_t st,
+                    int64_t bh0 = 0, int64_t nbh = -1) {
   const int T = (int)(N / C);
   int s;
   if (tc_bwd_walk_ok(dtype, d, C, N)) {
@@ -240,12 +245,13 @@ int bwd_finish_impl(const void* q, const void* k, const void* v, const float* de
     const int stride = G / C;
     if ((s = cuda_status(traced(K_SEG_SCAN, st, [&] {
            return launch_state_scan_slots(dstate_ws, dstate_ws, decay, dstate_in, dinit_state, B, (int)(N / G), H, d,
-                                          G, 1, T, stride, stride - 1, st);
+                                          G, 1, T, stride, stride - 1, st, bh0, nbh);
          }))))
       return s;
     const int sms = num_sms_current_device();
     return cuda_status(traced(K_BWD_WALK, st, [&] {
-      return tc_bwd_walk(q, k, v, dout, decay, state_cache, dstate_ws, dq, dk, dv, B, H, N, d, C, G, sms, st);
+      return tc_bwd_walk(q, k, v, dout, decay, state_cache, dstate_ws, dq, dk, dv, B, H, N, d, C, G, sms, st, bh0,
+                         nbh);
     }));
   }
   // exclusive suffix in place -> R_c (and dinit); then dQ, dK, dV
@@ -332,6 +338,82 @@ int lasp_fwd_finish(const void* q, const void* k, const void* v, const float* de
   if (N == 0) return LASP_OK;
   if ((s = check_ptrs({q, k, v, o, state_cache}, {decay, init_state}))) return s;
   return fwd_finish_impl(q, k, v, decay, o, B, H, N, d, C, dtype, state_cache, init_state, (cudaStream_t)stream);
+}
+
+int lasp_parts_ok(int64_t N, int C, int d, int dtype) {
+  return N > 0 && C >= 1 && N % C == 0 && tc_fwd_walk_ok(dtype, d, C, N) && tc_bwd_walk_ok(dtype, d, C, N) ? 1 : 0;
+}
+
+}  // extern "C"
+
+namespace lasp {
+namespace api_detail {
+
+// The (b, h) pairs of part `part` of `nparts`: bh0 .. bh0 + nbh - 1 (b-major),
+// after the same size checks as the whole call; nparts > 1 only where both
+// walks run (lasp_parts_ok).
+int part_range(int B, int H, int64_t N, int d, int C, int dtype, int part, int nparts, int64_t* bh0, int64_t* nbh) {
+  int s = check_sizes(B, H, N, d, C, dtype);
+  if (s) return s;
+  const int64_t bh = (int64_t)B * H;
+  if (nparts < 1 || part < 0 || part >= nparts || nparts > bh) return LASP_ERR_INVALID_ARG;
+  if (nparts > 1 && !lasp_parts_ok(N, C, d, dtype)) return LASP_ERR_UNSUPPORTED;
+  *bh0 = bh * part / nparts;
+  *nbh = bh * (part + 1) / nparts - *bh0;
+  return LASP_OK;
+}
+
+}  // namespace api_detail
+}  // namespace lasp
+
+extern "C" {
+
+int lasp_fwd_states_part(const void* k, const void* v, const float* decay, int B, int H, int64_t N, int d, int C,
+                         int dtype, float* state_cache, float* total, int part, int nparts, void* stream) {
+  int64_t bh0 = 0, nbh = 0;
+  int s = part_range(B, H, N, d, C, dtype, part, nparts, &bh0, &nbh);
+  if (s) return s;
+  if (nparts == 1) return lasp_fwd_states(k, v, decay, B, H, N, d, C, dtype, state_cache, total, stream);
+  if ((s = check_ptrs({k, v, state_cache}, {decay, total}))) return s;
+  return fwd_states_impl(k, v, decay, B, H, N, d, C, dtype, state_cache, total, (cudaStream_t)stream, bh0, nbh);
+}
+
+int lasp_fwd_finish_part(const void* q, const void* k, const void* v, const float* decay, void* o, int B, int H,
+                         int64_t N, int d, int C, int dtype, float* state_cache, const float* init_state, int part,
+                         int nparts, void* stream) {
+  int64_t bh0 = 0, nbh = 0;
+  int s = part_range(B, H, N, d, C, dtype, part, nparts, &bh0, &nbh);
+  if (s) return s;
+  if (nparts == 1) return lasp_fwd_finish(q, k, v, decay, o, B, H, N, d, C, dtype, state_cache, init_state, stream);
+  if ((s = check_ptrs({q, k, v, o, state_cache}, {decay, init_state}))) return s;
+  return fwd_finish_impl(q, k, v, decay, o, B, H, N, d, C, dtype, state_cache, init_state, (cudaStream_t)stream,
+                         bh0, nbh);
+}
+
+int lasp_bwd_states_part(const void* q, const void* dout, const float* decay, int B, int H, int64_t N, int d, int C,
+                         int dtype, float* dstate_ws, float* total, int part, int nparts, void* stream) {
+  int64_t bh0 = 0, nbh = 0;
+  int s = part_range(B, H, N, d, C, dtype, part, nparts, &bh0, &nbh);
+  if (s) return s;
+  if (nparts == 1) return lasp_bwd_states(q, dout, decay, B, H, N, d, C, dtype, dstate_ws, total, stream);
+  if ((s = check_ptrs({q, dout, dstate_ws}, {decay, total}))) return s;
+  return bwd_states_impl(q, dout, decay, B, H, N, d, C, dtype, dstate_ws, total, (cudaStream_t)stream, bh0, nbh);
+}
+
+int lasp_bwd_finish_part(const void* q, const void* k, const void* v, const float* decay, const void* dout, void* dq,
+                         void* dk, void* dv, int B, int H, int64_t N, int d, int C, int dtype,
+                         const float* state_cache, float* dstate_ws, const float* dstate_in, float* dinit_state,
+                         int part, int nparts, void* stream) {
+  int64_t bh0 = 0, nbh = 0;
+  int s = part_range(B, H, N, d, C, dtype, part, nparts, &bh0, &nbh);
+  if (s) return s;
+  if (nparts == 1)
+    return lasp_bwd_finish(q, k, v, decay, dout, dq, dk, dv, B, H, N, d, C, dtype, state_cache, dstate_ws, dstate_in,
+                           dinit_state, stream);
+  if ((s = check_ptrs({q, k, v, dout, dq, dk, dv, state_cache, dstate_ws}, {decay, dstate_in, dinit_state})))
+    return s;
+  return bwd_finish_impl(q, k, v, decay, dout, dq, dk, dv, B, H, N, d, C, dtype, state_cache, dstate_ws, dstate_in,
+                         dinit_state, (cudaStream_t)stream, bh0, nbh);
 }
 
 int lasp_fwd(const void* q, const void* k, const void* v, const float* decay, void* o, int B, int H, int64_t N,

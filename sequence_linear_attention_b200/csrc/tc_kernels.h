@@ -18,9 +18,10 @@ cudaError_t tc_chunk_states(const void* a, const void* b, const float* decay, fl
 
 // The same, writing chunk c's state to slot c * slot_stride + slot_offset of
 // an array of t_out states per (b, h).
+// bh0, nbh: only the (b, h) pairs bh0 .. bh0 + nbh - 1 (b-major; nbh < 0: all).
 cudaError_t tc_chunk_states_slots(const void* a, const void* b, const float* decay, float* M, int B, int H,
                                   int64_t N, int d, int C, int kind, int64_t t_out, int slot_stride, int slot_offset,
-                                  cudaStream_t st);
+                                  cudaStream_t st, int64_t bh0 = 0, int64_t nbh = -1);
 
 // Forward walk over segments of G tokens with the state on chip (bf16,
 // d = 128, C a multiple of 128 or a divisor of it, N a multiple of max(C, 128),
@@ -32,7 +33,8 @@ cudaError_t tc_chunk_states_slots(const void* a, const void* b, const float* dec
 bool tc_fwd_walk_ok(int dtype, int d, int64_t C, int64_t N);
 int walk_segment_tokens(int64_t N, int C);
 cudaError_t tc_fwd_walk(const void* q, const void* k, const void* v, const float* decay, float* P, void* o, int B,
-                        int H, int64_t N, int d, int C, int G, int num_sms, cudaStream_t st);
+                        int H, int64_t N, int d, int C, int G, int num_sms, cudaStream_t st, int64_t bh0 = 0,
+                        int64_t nbh = -1);
 
 // Backward walk over segments with the gradient state on chip (bf16, d = 128,
 // C dividing 128, N a multiple of 128). R must hold, in the slot of each
@@ -42,7 +44,7 @@ cudaError_t tc_fwd_walk(const void* q, const void* k, const void* v, const float
 bool tc_bwd_walk_ok(int dtype, int d, int64_t C, int64_t N);
 cudaError_t tc_bwd_walk(const void* q, const void* k, const void* v, const void* dout, const float* decay,
                         const float* P, float* R, void* dq, void* dk, void* dv, int B, int H, int64_t N, int d, int C,
-                        int G, int num_sms, cudaStream_t st);
+                        int G, int num_sms, cudaStream_t st, int64_t bh0 = 0, int64_t nbh = -1);
 
 bool tc_out_ok(int dtype, int d, int64_t C);
 cudaError_t tc_chunk_out(const void* q, const void* k, const void* v, const float* decay, const float* P, void* o,

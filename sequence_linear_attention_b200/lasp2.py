@@ -33,46 +33,69 @@ arithmetic runs in the library's kernels; torch.distributed moves the states.
 The payload of each AllGather is W * B * H * d * d fp32 values (1 MiB per rank
 at B = 1, H = 16, d = 128), so the exchange is latency-bound on NVLink.
 
+Overlap (LASP-2 review page, "Core claim": the AllGather of fixed-size
+states runs alongside computation). The (b, h) pairs are split into parts
+(two by default, where both segment walks run and there are at least two
+pairs): part p's shard states are gathered asynchronously (NCCL's stream)
+while part p + 1's shard states are computed, and each part's scan over the
+shards and its output start as soon as its own gather lands, so the gather of
+the last part runs under the output of the ones before. No kernel waits on a
+collective inside itself; the streams order them.
+
 Each function takes the same tensors as the single-device call, plus the
 process group (default: the world group). ``kernels`` replaces the device
 kernels by an object with the same five methods (see ``DeviceKernels``); the
-library's own are the default and the only ones used outside tests.
+library's own are the default and the only ones used outside tests. ``parts``
+overrides the number of parts.
 """
 from __future__ import annotations
 
 import torch
 import torch.distributed as dist
 
-from . import lasp_bwd_finish, lasp_bwd_states, lasp_fwd_finish, lasp_fwd_states, lasp_state_prefix
+from . import (LASP_BF16, LASP_F32, lasp_bwd_finish_part, lasp_bwd_states_part, lasp_fwd_finish_part,
+               lasp_fwd_states_part, lasp_parts_ok, lasp_state_prefix)
 
-__all__ = ["DeviceKernels", "lasp2_fwd", "lasp2_bwd"]
+__all__ = ["DeviceKernels", "lasp2_fwd", "lasp2_bwd", "default_parts"]
 
 
 class DeviceKernels:
     """The library's kernels, through its C ABI, in the shape this module calls
     them. The shard states are the first parts of the single-device forward and
     backward calls (their segment states, in the cache or workspace, and the
-    decayed total); the rest of those calls reuses the segment states."""
+    decayed total); the rest of those calls reuses the segment states. Every
+    call works on part `part` of `nparts` of the (b, h) pairs."""
 
     @staticmethod
-    def shard_state(k, v, decay, M, C, state_cache):
-        lasp_fwd_states(k, v, decay, C, state_cache, total=M)
+    def shard_state(k, v, decay, M, C, state_cache, part, nparts):
+        lasp_fwd_states_part(k, v, decay, C, state_cache, M, part, nparts)
 
     @staticmethod
-    def shard_dstate(q, dout, decay, dM, C, dstate_ws):
-        lasp_bwd_states(q, dout, decay, C, dstate_ws, total=dM)
+    def shard_dstate(q, dout, decay, dM, C, dstate_ws, part, nparts):
+        lasp_bwd_states_part(q, dout, decay, C, dstate_ws, dM, part, nparts)
 
     @staticmethod
     def state_prefix(M, out, decay, L, init, total, reverse):
         lasp_state_prefix(M, out, decay, L, init=init, total=total, reverse=reverse)
 
     @staticmethod
-    def fwd(q, k, v, decay, o, C, state_cache, init_state):
-        lasp_fwd_finish(q, k, v, decay, o, C, state_cache, init_state=init_state)
+    def fwd(q, k, v, decay, o, C, state_cache, init_state, part, nparts):
+        lasp_fwd_finish_part(q, k, v, decay, o, C, state_cache, init_state, part, nparts)
 
     @staticmethod
-    def bwd(q, k, v, decay, dout, dq, dk, dv, C, state_cache, dstate_ws, dstate_in):
-        lasp_bwd_finish(q, k, v, decay, dout, dq, dk, dv, C, state_cache, dstate_ws, dstate_in=dstate_in)
+    def bwd(q, k, v, decay, dout, dq, dk, dv, C, state_cache, dstate_ws, dstate_in, part, nparts):
+        lasp_bwd_finish_part(q, k, v, decay, dout, dq, dk, dv, C, state_cache, dstate_ws, dstate_in, None, part,
+                             nparts)
+
+
+def default_parts(q, C, world=2):
+    """Two parts where there is an exchange to hide (more than one rank), both
+    segment walks run on the shard and it has at least two (b, h) pairs; else
+    one (at one rank the split only adds launches and a second wave tail:
+    3.4% slower on the 2M-token workload)."""
+    B, L, H, d = q.shape
+    dt = LASP_BF16 if q.dtype == torch.bfloat16 else LASP_F32
+    return 2 if world > 1 and B * H >= 2 and q.is_cuda and lasp_parts_ok(L, C, d, dt) else 1
 
 
 def _group_shape(x, group):
@@ -84,29 +107,70 @@ def _group_shape(x, group):
     return dist.get_world_size(group), dist.get_rank(group), B, L, H, d
 
 
+class _Done:
+    def wait(self):
+        pass
+
+
 def _all_gather(out, x, group):
-    # NCCL gathers device memory straight into the [W, ...] buffer. Other
-    # backends (gloo) gather host copies into the list of the buffer's W slices.
+    """Gathers x from every rank into the [W, ...] buffer out; returns a handle
+    whose wait() orders later work on the current stream after the gather.
+    NCCL gathers device memory straight into the buffer, asynchronously on its
+    own stream; other backends (gloo) gather host copies, synchronously."""
     if dist.get_backend(group) == "nccl":
-        dist.all_gather_into_tensor(out, x, group=group)
-    elif out.is_cuda:
+        return dist.all_gather_into_tensor(out, x, group=group, async_op=True)
+    if out.is_cuda:
         host = torch.empty(out.shape, dtype=out.dtype)
         dist.all_gather(list(host.unbind(0)), x.cpu(), group=group)
         out.copy_(host)
     else:
         dist.all_gather(list(out.unbind(0)), x, group=group)
+    return _Done()
 
 
-def _scan_over_shards(kern, gathered, decay, L, init, total, reverse):
-    """Exclusive decayed scan over the W gathered [B, H, d, d] states; returns
-    the [W, B, H, d, d] scan, writes the total (if given)."""
-    W, B, H, d, _ = gathered.shape
-    flat = lambda t: None if t is None else t.reshape(1, B * H, d, d)
+def _bounds(B, H, nparts):
+    bh = B * H
+    return [bh * p // nparts for p in range(nparts + 1)]
+
+
+def _pairs(t, bh0, bh1):
+    """Pairs bh0 .. bh1 - 1 of a [B, H, d, d] state (or None), as [1, n, d, d]."""
+    if t is None:
+        return None
+    d = t.shape[-1]
+    return t.reshape(-1, d, d)[bh0:bh1].unsqueeze(0)
+
+
+def _exchange(kern, states_fn, finish_fn, decay, L, init, total, reverse, B, H, d, W, r, nparts, device, group):
+    """The exchange of one direction: per part, the shard states (states_fn),
+    an asynchronous gather, then the scan over the W shards and the rest of the
+    call (finish_fn) once that part's gather has landed. Returns the states
+    entering this shard, [B, H, d, d]."""
+    M = torch.empty((B, H, d, d), dtype=torch.float32, device=device)
+    bounds = _bounds(B, H, nparts)
+    handles, bufs = [], []
+    for p in range(nparts):
+        states_fn(M, p)
+        bh0, bh1 = bounds[p], bounds[p + 1]
+        buf = torch.empty((W, bh1 - bh0, d, d), dtype=torch.float32, device=device)
+        handles.append(_all_gather(buf, M.view(B * H, d, d)[bh0:bh1], group))
+        bufs.append(buf)
+    # the decay of every (b, h) pair; a part's slice is copied, since the ABI
+    # takes 16-byte-aligned pointers only
     rep = None if decay is None else decay.repeat(B)
-    out = torch.empty_like(gathered)
-    kern.state_prefix(gathered.view(1, W, B * H, d, d), out.view(1, W, B * H, d, d), rep, L,
-                      flat(init), flat(total), reverse)
-    return out
+    entering = torch.empty((B, H, d, d), dtype=torch.float32, device=device)
+    for p in range(nparts):
+        handles[p].wait()
+        bh0, bh1 = bounds[p], bounds[p + 1]
+        n = bh1 - bh0
+        out = torch.empty_like(bufs[p])
+        # the W gathered states of these pairs as one sequence of W chunks with n heads
+        kern.state_prefix(bufs[p].view(1, W, n, d, d), out.view(1, W, n, d, d),
+                          None if rep is None else rep[bh0:bh1].clone(), L, _pairs(init, bh0, bh1),
+                          _pairs(total, bh0, bh1), reverse)
+        entering.view(B * H, d, d)[bh0:bh1].copy_(out[r])
+        finish_fn(entering, p)
+    return entering
 
 
 def _check_state(t, B, H, d, like, name):
@@ -117,7 +181,8 @@ def _check_state(t, B, H, d, like, name):
         raise ValueError(f"{name} must be a contiguous float32 [B, H, d, d] tensor on the shard's device")
 
 
-def lasp2_fwd(q, k, v, decay, o, C, state_cache, init_state=None, final_state=None, group=None, kernels=None):
+def lasp2_fwd(q, k, v, decay, o, C, state_cache, init_state=None, final_state=None, group=None, kernels=None,
+              parts=None):
     """Forward pass of this rank's shard (see the module docstring).
 
     q, k, v, o: [B, L, H, d] shard tensors; C, state_cache: as for the
@@ -132,17 +197,14 @@ def lasp2_fwd(q, k, v, decay, o, C, state_cache, init_state=None, final_state=No
     W, r, B, L, H, d = _group_shape(q, group)
     _check_state(init_state, B, H, d, q, "init_state")
     _check_state(final_state, B, H, d, q, "final_state")
-    M = torch.empty((B, 1, H, d, d), dtype=torch.float32, device=q.device)
-    kern.shard_state(k, v, decay, M.view(B, H, d, d), C, state_cache)
-    gathered = torch.empty((W, B, H, d, d), dtype=torch.float32, device=q.device)
-    _all_gather(gathered, M.view(B, H, d, d), group)
-    entering = _scan_over_shards(kern, gathered, decay, L, init_state, final_state, False)[r]
-    kern.fwd(q, k, v, decay, o, C, state_cache, entering)
-    return entering
+    nparts = parts or (default_parts(q, C, W) if kernels is None else 1)
+    return _exchange(kern, lambda M, p: kern.shard_state(k, v, decay, M, C, state_cache, p, nparts),
+                     lambda E, p: kern.fwd(q, k, v, decay, o, C, state_cache, E, p, nparts),
+                     decay, L, init_state, final_state, False, B, H, d, W, r, nparts, q.device, group)
 
 
 def lasp2_bwd(q, k, v, decay, dout, dq, dk, dv, C, state_cache, dstate_ws, dstate_in=None, dinit_state=None,
-              group=None, kernels=None):
+              group=None, kernels=None, parts=None):
     """Backward pass of this rank's shard (see the module docstring): dq, dk, dv
     of sum(o * dout) over the whole sequence, for this shard's tokens.
 
@@ -157,10 +219,7 @@ def lasp2_bwd(q, k, v, decay, dout, dq, dk, dv, C, state_cache, dstate_ws, dstat
     W, r, B, L, H, d = _group_shape(q, group)
     _check_state(dstate_in, B, H, d, q, "dstate_in")
     _check_state(dinit_state, B, H, d, q, "dinit_state")
-    dM = torch.empty((B, 1, H, d, d), dtype=torch.float32, device=q.device)
-    kern.shard_dstate(q, dout, decay, dM.view(B, H, d, d), C, dstate_ws)
-    gathered = torch.empty((W, B, H, d, d), dtype=torch.float32, device=q.device)
-    _all_gather(gathered, dM.view(B, H, d, d), group)
-    incoming = _scan_over_shards(kern, gathered, decay, L, dstate_in, dinit_state, True)[r]
-    kern.bwd(q, k, v, decay, dout, dq, dk, dv, C, state_cache, dstate_ws, incoming)
-    return incoming
+    nparts = parts or (default_parts(q, C, W) if kernels is None else 1)
+    return _exchange(kern, lambda dM, p: kern.shard_dstate(q, dout, decay, dM, C, dstate_ws, p, nparts),
+                     lambda G, p: kern.bwd(q, k, v, decay, dout, dq, dk, dv, C, state_cache, dstate_ws, G, p, nparts),
+                     decay, L, dstate_in, dinit_state, True, B, H, d, W, r, nparts, q.device, group)

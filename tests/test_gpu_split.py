@@ -67,3 +67,46 @@ def test_empty_sequence_gives_zero_totals():
     st, _ = lasp.lasp_check_device_status()
     assert st == 0
     assert not torch.any(tf) and not torch.any(tb)
+
+
+@pytest.mark.parametrize("nparts", [2, 3, 6])
+def test_pair_parts_equal_the_whole_call(nparts):
+    """The four split calls restricted to parts of the (b, h) pairs (b-major),
+    run part after part as LASP-2's overlapped exchange runs them, give the
+    whole calls' results bit for bit, totals included."""
+    import torch
+    import sequence_linear_attention_b200 as lasp
+    B, N, H, d, C = 2, 2048, 3, 128, 128
+    assert lasp.lasp_parts_ok(N, C, d, lasp.LASP_BF16) == 1
+    inp = lasp_inputs.make_inputs(B, N, H, d, seed=4300, bf16=True, decayed=True)
+    q, k, v, do = (to_device(inp[n], True) for n in ("q", "k", "v", "do"))
+    decay = decay_device(inp["lam"])
+    rng = np.random.default_rng(4301)
+    init = torch.from_numpy((rng.standard_normal((B, H, d, d)) * 0.1).astype(np.float32)).cuda()
+    dsin = torch.from_numpy((rng.standard_normal((B, H, d, d)) * 0.1).astype(np.float32)).cuda()
+    shape = (B, N // C, H, d, d)
+    res = []
+    for parts in (1, nparts):
+        o, dq, dk, dv = (torch.full_like(q, float("nan")) for _ in range(4))
+        P, R = torch.empty(shape, device="cuda"), torch.empty(shape, device="cuda")
+        tf, tb, din = (torch.full((B, H, d, d), float("nan"), device="cuda") for _ in range(3))
+        for p in range(parts):
+            lasp.lasp_fwd_states_part(k, v, decay, C, P, tf, p, parts)
+        for p in range(parts):
+            lasp.lasp_fwd_finish_part(q, k, v, decay, o, C, P, init, p, parts)
+        for p in range(parts):
+            lasp.lasp_bwd_states_part(q, do, decay, C, R, tb, p, parts)
+        for p in range(parts):
+            lasp.lasp_bwd_finish_part(q, k, v, decay, do, dq, dk, dv, C, P, R, dsin, din, p, parts)
+        st, _ = lasp.lasp_check_device_status()
+        assert st == 0
+        res.append((o, dq, dk, dv, tf, tb, din))
+    for a, b in zip(*res):
+        assert torch.equal(a, b)
+    # parts beyond the pairs, or on sizes the walks do not take, are refused
+    with pytest.raises(lasp.LaspError):
+        lasp.lasp_fwd_states_part(k, v, decay, C, P, tf, 0, B * H + 1)
+    q32 = torch.zeros((1, 256, 2, 64), device="cuda")
+    with pytest.raises(lasp.LaspError) as e:
+        lasp.lasp_fwd_states_part(q32, q32, None, 64, torch.empty((1, 4, 2, 64, 64), device="cuda"), None, 0, 2)
+    assert e.value.status == 2
