@@ -125,15 +125,12 @@ def flops_per_step(tokens_heads: int, d: int, C: int) -> float:
 MEASURED_TRAFFIC = {
     # DRAM bytes per launch at the workload's full size: twice the ncu capture of
     # the 32768-token case of the same workload (traffic grows with the tokens)
-    "bwd_walk_tc": (["k_tc_bwd_walk.cu", "sm100.cuh", "lasp_common.cuh", "tma_host.h"], "94ed7a7710fac966",
-                    2 * (721036800 + 365295104)),
-    "fwd_walk_tc": (["k_tc_fwd_walk.cu", "sm100.cuh", "lasp_common.cuh", "tma_host.h"], "af6d12c4ff311f6e",
-                    2 * (437424128 + 227407616)),
-    "segment_states_tc": (["k_tc_states.cu", "sm100.cuh", "lasp_common.cuh", "tma_host.h"], "fc6351767f0401ee",
-                          2 * (268477696 + 5350400)),
-    # the gated form (bench.py --gated): four times the capture of the 16384-token case
-    "gla_bwd_tc": (["k_tc_gla.cu", "sm100.cuh", "lasp_common.cuh", "tma_host.h"], "039f7de455c9c750",
-                   4 * (605879552 + 294130688)),
+    "bwd_walk_tc": (["k_tc_bwd_walk.cu", "sm100.cuh", "lasp_common.cuh", "tma_host.h"], "adce30b1fce33512",
+                    2 * (723739136 + 364952576)),
+    "fwd_walk_tc": (["k_tc_fwd_walk.cu", "sm100.cuh", "lasp_common.cuh", "tma_host.h"], "bcb650137196739b",
+                    2 * (437725440 + 226706432)),
+    "segment_states_tc": (["k_tc_states.cu", "sm100.cuh", "lasp_common.cuh", "tma_host.h"], "bfe2712019c7da94",
+                          2 * (268476416 + 5191168)),
 }
 
 
