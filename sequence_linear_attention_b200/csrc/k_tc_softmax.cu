@@ -9,15 +9,17 @@
 //
 // Forward (one CTA per 128-query tile, heaviest tiles first): the softmax is
 // taken online over 128-key tiles. Warp roles, all hand-offs by mbarriers:
-//   warp 4 (one thread): TMA loads of the Q tile and of every key tile's K and
+//   warp 8 (one thread): TMA loads of the Q tile and of every key tile's K and
 //     V into two stages each (K of stage s is refilled once the S MMA that
 //     read it has completed, V once the P V MMA has);
-//   warp 5 (one thread): S_j = Q K_j^T into one of two TMEM buffers, then
+//   warp 9 (one thread): S_j = Q K_j^T into one of two TMEM buffers, then
 //     O += P_{j-1} V_{j-1}, so the next S is on the tensor pipe while the
 //     softmax warps work on the last one;
-//   warps 0-3 (one query row per thread, TMEM lane = row): read S_j from TMEM,
-//     mask, keep the running maximum m (log2 units) and sum l, write
-//     P = exp2(s - m) in bf16 as the A operand of the P V MMA. O in TMEM is
+//   warps 0-7 (two threads per query row: warp w reads TMEM lanes 32 (w % 4)..
+//     and the column half w / 4): read S_j from TMEM, mask, keep the running
+//     maximum m (log2 units; the two halves of a row exchange their tile
+//     maxima through shared memory) and the sum l, write P = exp2(s - m) in
+//     bf16 as the A operand of the P V MMA. O in TMEM is
 //     rescaled only when a row's maximum grows by more than 8 (P stays below
 //     2^8 in between): the final O / l uses the same stale m for both, so the
 //     result is exact; the rescale waits for the P V MMA before it.
@@ -63,13 +65,15 @@ __device__ __forceinline__ float ex2(float x) {
 }
 
 // ------------------------------------------------------------------ forward
-constexpr int kFwdThreads = 192;  // warps 0-3 softmax, 4 TMA, 5 MMA
+constexpr int kFwdThreads = 320;  // warps 0-7 softmax, 8 TMA, 9 MMA
+constexpr int kSoftmaxThreads = 256;
 constexpr uint32_t kBarSoftmax = 1;
 
 struct SmemFwd {
   uint64_t q_full, k_full[2], v_full[2], s_full[2], p_full[2], pv_done[2], drain;
   uint32_t tmem_base;
   int abort;
+  float red[2][kTile];  // each column half's value of a row (tile maximum, then l)
 };
 
 __global__ void __launch_bounds__(kFwdThreads, 1) softmax_fwd_tc(const __grid_constant__ CUtensorMap map_q,
@@ -79,12 +83,13 @@ __global__ void __launch_bounds__(kFwdThreads, 1) softmax_fwd_tc(const __grid_co
                                                                   float* __restrict__ lse, int H, int64_t Nq,
                                                                   int64_t q_offset, float scale_log2, int qtiles) {
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* base = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  // the small struct first, then seven 1024-aligned tiles
+  SmemFwd* s = reinterpret_cast<SmemFwd*>(smem_raw);
+  uint8_t* base = (uint8_t*)(((uintptr_t)(smem_raw + sizeof(SmemFwd)) + 1023) & ~(uintptr_t)1023);
   uint8_t* sQ = base;  // Q, then the output tile
   uint8_t* sK = base + kTileBytes;       // two stages
   uint8_t* sV = base + 3 * kTileBytes;   // two stages
   uint8_t* sP = base + 5 * kTileBytes;   // two P tiles
-  SmemFwd* s = reinterpret_cast<SmemFwd*>(base + 7 * kTileBytes);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int qt = qtiles - 1 - (int)blockIdx.x;  // heaviest (latest) tiles first
   const int h = blockIdx.y, b = blockIdx.z;
@@ -104,7 +109,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1) softmax_fwd_tc(const __grid_co
       mbar_init(&s->k_full[st], 1);
       mbar_init(&s->v_full[st], 1);
       mbar_init(&s->s_full[st], 1);
-      mbar_init(&s->p_full[st], 128);
+      mbar_init(&s->p_full[st], kSoftmaxThreads);
       mbar_init(&s->pv_done[st], 1);
     }
     mbar_init(&s->drain, 1);
@@ -121,7 +126,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1) softmax_fwd_tc(const __grid_co
   const uint32_t tmem = s->tmem_base;
   constexpr uint32_t kColS = 0, kColO = 256;  // S buffers at 0 and 128, O at 256
 
-  if (warp == 4) {
+  if (warp == 8) {
     // ---------------------------------------------------------- TMA producer
     if (lane == 0) {
       bool bad = false;
@@ -158,7 +163,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1) softmax_fwd_tc(const __grid_co
         mbar_wait(&s->v_full[j & 1], (uint32_t)(j >> 1) & 1u, SITE_OUT_TMA);
       mbar_wait(&s->q_full, 0, SITE_OUT_TMA);
     }
-  } else if (warp == 5) {
+  } else if (warp == 9) {
     // ----------------------------------------------------------- MMA issuer
     if (lane == 0) {
       constexpr uint32_t id_kk = idesc_bf16(128, 128, 0, 0);
@@ -199,10 +204,12 @@ __global__ void __launch_bounds__(kFwdThreads, 1) softmax_fwd_tc(const __grid_co
     }
   } else {
     // ------------------------------------------------------ softmax warps
-    const int i = tid;  // query row of the tile = TMEM lane
-    const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
+    const int i = (warp & 3) * 32 + lane;  // query row of the tile = TMEM lane
+    const int half = warp >> 2;            // and the column half of it
+    const int c0 = half * 64;
+    const uint32_t lane_base = tmem + ((uint32_t)((warp & 3) * 32) << 16);
     const int64_t qpos = q_offset + q0 + i;
-    float m_used = -INFINITY, l = 0.f;
+    float m_used = -INFINITY, l = 0.f;  // l: this half's share of the row sum
     bool bad = false;
     for (int j = 0; j < nkv; ++j) {
       const int st = j & 1;
@@ -211,30 +218,36 @@ __global__ void __launch_bounds__(kFwdThreads, 1) softmax_fwd_tc(const __grid_co
       // tcgen05.ld / st are warp-collective: every branch around them is
       // taken by the whole warp
       bad = __any_sync(0xffffffffu, bad);
-      float x[128];
+      float x[64];
       if (!bad) {
         tc_fence_after();
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
+        for (int c = 0; c < 2; ++c) {
           uint32_t r[32];
-          tmem_ld32(lane_base + kColS + st * 128 + c * 32, r);
+          tmem_ld32(lane_base + kColS + st * 128 + c0 + c * 32, r);
           tmem_ld_wait();
 #pragma unroll
           for (int u = 0; u < 32; ++u) x[c * 32 + u] = __uint_as_float(r[u]) * scale_log2;
         }
       } else {
 #pragma unroll
-        for (int u = 0; u < 128; ++u) x[u] = 0.f;
+        for (int u = 0; u < 64; ++u) x[u] = 0.f;
       }
-      const int64_t k0 = (int64_t)j * kTile;
-      if (k0 + kTile - 1 > qpos) {  // the causal edge crosses this tile for this row
+      const int64_t k0 = (int64_t)j * kTile + c0;
+      if (k0 + 63 > qpos) {  // the causal edge crosses this half tile for this row
 #pragma unroll
-        for (int u = 0; u < 128; ++u)
+        for (int u = 0; u < 64; ++u)
           if (k0 + u > qpos) x[u] = -INFINITY;
       }
-      float mt = x[0];
+      float mh = x[0];
 #pragma unroll
-      for (int u = 1; u < 128; ++u) mt = fmaxf(mt, x[u]);
+      for (int u = 1; u < 64; ++u) mh = fmaxf(mh, x[u]);
+      // the row's tile maximum from both halves: write, barrier, read, barrier
+      // (the second keeps the next tile's write from overtaking the read)
+      s->red[half][i] = mh;
+      named_sync(kBarSoftmax, kSoftmaxThreads);
+      const float mt = fmaxf(mh, s->red[half ^ 1][i]);
+      named_sync(kBarSoftmax, kSoftmaxThreads);
       // a new maximum far above the one in use: this row's O and l move to it.
       // The warp rescales together when any of its rows needs it (factor 1
       // for the others), after the last P V MMA has written O.
@@ -248,13 +261,13 @@ __global__ void __launch_bounds__(kFwdThreads, 1) softmax_fwd_tc(const __grid_co
         if (!bad) {
           tc_fence_after();
 #pragma unroll
-          for (int c = 0; c < 4; ++c) {
+          for (int c = 0; c < 2; ++c) {
             uint32_t r[32];
-            tmem_ld32(lane_base + kColO + c * 32, r);
+            tmem_ld32(lane_base + kColO + c0 + c * 32, r);
             tmem_ld_wait();
 #pragma unroll
             for (int u = 0; u < 32; ++u) r[u] = __float_as_uint(__uint_as_float(r[u]) * f);
-            tmem_st32(lane_base + kColO + c * 32, r);
+            tmem_st32(lane_base + kColO + c0 + c * 32, r);
           }
           tmem_st_wait();
         }
@@ -270,14 +283,14 @@ __global__ void __launch_bounds__(kFwdThreads, 1) softmax_fwd_tc(const __grid_co
       uint8_t* pt = sP + st * kTileBytes;
       float rs = 0.f;
 #pragma unroll
-      for (int c8 = 0; c8 < 16; ++c8) {
+      for (int c8 = 0; c8 < 8; ++c8) {
         float p[8];
 #pragma unroll
         for (int u = 0; u < 8; ++u) {
           p[u] = ex2(x[c8 * 8 + u] - m_used);
           rs += p[u];
         }
-        st_tile16(pt, i, c8 * 8,
+        st_tile16(pt, i, c0 + c8 * 8,
                   make_uint4(pack_bf16(p[0], p[1]), pack_bf16(p[2], p[3]), pack_bf16(p[4], p[5]),
                              pack_bf16(p[6], p[7])));
       }
@@ -286,32 +299,36 @@ __global__ void __launch_bounds__(kFwdThreads, 1) softmax_fwd_tc(const __grid_co
       tc_fence_before();
       mbar_arrive(&s->p_full[st]);  // arrives even after a failure, so no waiter is left short
     }
-    // epilogue: O / l, once the last P V MMA has completed
+    // epilogue: O / l, once the last P V MMA has completed; l of the row is
+    // the sum of the two halves'
     const int jl = nkv - 1;
     if (!bad && !mbar_wait_or_abort(&s->pv_done[jl & 1], (uint32_t)(jl >> 1) & 1u, SITE_OUT_MMA, abort_flag))
       bad = true;
     bad = __any_sync(0xffffffffu, bad);
     if (bad) s->abort = 1;
-    const float inv = 1.f / l;
+    s->red[half][i] = l;
+    named_sync(kBarSoftmax, kSoftmaxThreads);
+    const float lr = l + s->red[half ^ 1][i];
+    const float inv = 1.f / lr;
     if (!bad) {
       tc_fence_after();
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
+      for (int c = 0; c < 2; ++c) {
         uint32_t r[32];
-        tmem_ld32(lane_base + kColO + c * 32, r);
+        tmem_ld32(lane_base + kColO + c0 + c * 32, r);
         tmem_ld_wait();
 #pragma unroll
         for (int q8 = 0; q8 < 4; ++q8)
-          st_tile16(sQ, i, c * 32 + q8 * 8,
+          st_tile16(sQ, i, c0 + c * 32 + q8 * 8,
                     make_uint4(pack_bf16(__uint_as_float(r[q8 * 8]) * inv, __uint_as_float(r[q8 * 8 + 1]) * inv),
                                pack_bf16(__uint_as_float(r[q8 * 8 + 2]) * inv, __uint_as_float(r[q8 * 8 + 3]) * inv),
                                pack_bf16(__uint_as_float(r[q8 * 8 + 4]) * inv, __uint_as_float(r[q8 * 8 + 5]) * inv),
                                pack_bf16(__uint_as_float(r[q8 * 8 + 6]) * inv, __uint_as_float(r[q8 * 8 + 7]) * inv)));
       }
-      if (q0 + i < Nq) lse[((int64_t)b * H + h) * Nq + q0 + i] = (m_used + __log2f(l)) * kLn2;
+      if (half == 0 && q0 + i < Nq) lse[((int64_t)b * H + h) * Nq + q0 + i] = (m_used + __log2f(lr)) * kLn2;
     }
     fence_async_smem();
-    named_sync(kBarSoftmax, 128);
+    named_sync(kBarSoftmax, kSoftmaxThreads);
     if (tid == 0 && !s->abort) {
       tma_store_4d(&map_o, sQ, 0, h, (int)q0, b);
       tma_store_4d(&map_o, sQ + kBox, 64, h, (int)q0, b);
@@ -806,7 +823,7 @@ cudaError_t tc_softmax_fwd(const void* q, const void* k, const void* v, void* o,
   if (!make_token_map(&mq, q, B, H, Nq, kD, kTile) || !make_token_map(&mk, k, B, H, Nk, kD, kTile) ||
       !make_token_map(&mv, v, B, H, Nk, kD, kTile) || !make_token_map(&mo, o, B, H, Nq, kD, kTile))
     return cudaErrorInvalidValue;
-  const size_t smem = 1024 + 7 * (size_t)kTileBytes + sizeof(SmemFwd);
+  const size_t smem = sizeof(SmemFwd) + 1023 + 7 * (size_t)kTileBytes;
   cudaError_t e = cudaFuncSetAttribute(softmax_fwd_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   const int qtiles = (int)((Nq + kTile - 1) / kTile);
