@@ -373,11 +373,13 @@ constexpr uint32_t kBarEpi = 1;
 // operand tiles at (row, column). keep(u) says whether column half*64 + u is
 // inside the causal mask and the sequence; lse2 / dl give the column's (or the
 // row's) values through the callbacks.
+// Chunk cc (0 or 1) of the half: columns half * 64 + cc * 32 .. + 31, so that
+// chunk 0 of both halves is the tile's K-steps 0, 1, 4, 5 of the next MMA and
+// chunk 1 its K-steps 2, 3, 6, 7.
 template <class Keep, class Lse, class Dl>
 __device__ __forceinline__ void p_ds_rows(uint32_t lane_base, uint32_t colS, uint32_t colP, int row, int half,
-                                          float c2, uint8_t* tP, uint8_t* tDS, Keep keep, Lse lse2, Dl dl) {
-#pragma unroll 1
-  for (int cc = 0; cc < 2; ++cc) {
+                                          int cc, float c2, uint8_t* tP, uint8_t* tDS, Keep keep, Lse lse2, Dl dl) {
+  {
     const int col0 = half * 64 + cc * 32;
     uint32_t rs[32], rp[32];
     tmem_ld32(lane_base + colS + col0, rs);
@@ -426,7 +428,7 @@ __device__ __forceinline__ void acc_to_tile(uint32_t lane_base, uint32_t col, in
 }
 
 struct SmemDkdv {
-  uint64_t kv_full, full[3], empty[3], ld_full, s_full, p_full, mma2_done, drain;
+  uint64_t kv_full, full[3], empty[3], ld_full, s_full, p_half, p_full, mma2_done, drain;
   uint32_t tmem_base;
   int abort;
   float lse2[kTile], dl[kTile];  // the current query tile's lse (log2 units) and delta
@@ -472,6 +474,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) softmax_dkdv_tc(
     }
     mbar_init(&s->ld_full, 1);
     mbar_init(&s->s_full, 1);
+    mbar_init(&s->p_half, 256);
     mbar_init(&s->p_full, 256);
     mbar_init(&s->mma2_done, 1);
     mbar_init(&s->drain, 1);
@@ -563,15 +566,28 @@ __global__ void __launch_bounds__(kBwdThreads, 1) softmax_dkdv_tc(
         tc_fence_after();
         for (int kk = 0; kk < kD / 16; ++kk) mma_bf16(tmem + kColP, kmaj(aV, kk), kmaj(aO, kk), id_kk, kk > 0);
         mma_commit(&s->s_full);
-        if (!mbar_wait_or_abort(&s->p_full, (uint32_t)i & 1u, SITE_BWD_MMA, abort_flag)) {
+        // dV += P^T dO and dK += dS^T Q over the query columns the epilogue
+        // has finished: K-steps 0, 1, 4, 5 (its first chunk), then 2, 3, 6, 7
+        bool part_ok = true;
+        for (int pc = 0; pc < 2 && part_ok; ++pc) {
+          if (!mbar_wait_or_abort(pc == 0 ? &s->p_half : &s->p_full, (uint32_t)i & 1u, SITE_BWD_MMA, abort_flag)) {
+            part_ok = false;
+            break;
+          }
+          tc_fence_after();
+          for (int q = 0; q < 4; ++q) {
+            const int kk = (q >> 1) * 4 + pc * 2 + (q & 1);
+            mma_bf16(tmem + kColV, kmaj(aP, kk), mnmaj(aO, kk), id_kn, (i > 0 || pc > 0 || q > 0) ? 1u : 0u);
+          }
+          for (int q = 0; q < 4; ++q) {
+            const int kk = (q >> 1) * 4 + pc * 2 + (q & 1);
+            mma_bf16(tmem + kColK, kmaj(aD, kk), mnmaj(aQ, kk), id_kn, (i > 0 || pc > 0 || q > 0) ? 1u : 0u);
+          }
+        }
+        if (!part_ok) {
           bad = true;
           break;
         }
-        tc_fence_after();
-        for (int kk = 0; kk < kTile / 16; ++kk)
-          mma_bf16(tmem + kColV, kmaj(aP, kk), mnmaj(aO, kk), id_kn, (i > 0 || kk > 0) ? 1u : 0u);
-        for (int kk = 0; kk < kTile / 16; ++kk)
-          mma_bf16(tmem + kColK, kmaj(aD, kk), mnmaj(aQ, kk), id_kn, (i > 0 || kk > 0) ? 1u : 0u);
         mma_commit(&s->empty[sq]);
         mma_commit(&s->empty[sd]);
         mma_commit(&s->mma2_done);
@@ -594,17 +610,19 @@ __global__ void __launch_bounds__(kBwdThreads, 1) softmax_dkdv_tc(
       if (i > 0 && !bad && !mbar_wait_or_abort(&s->mma2_done, (uint32_t)(i - 1) & 1u, SITE_BWD_MMA, abort_flag))
         bad = true;
       bad = __any_sync(0xffffffffu, bad);  // the TMEM loads below are warp-collective
-      if (!bad) {
-        tc_fence_after();
-        const float* L = s->lse2;
-        const float* Dl = s->dl;
-        p_ds_rows(lane_base, kColS, kColP, row, half, c2, sPt, sDSt,
-                  [&](int c) { return q0 + c < Nq && q_offset + q0 + c >= kpos; },
-                  [&](int c) { return L[c]; }, [&](int c) { return Dl[c]; });
+      const float* L = s->lse2;
+      const float* Dl = s->dl;
+      auto keep = [&](int c) { return q0 + c < Nq && q_offset + q0 + c >= kpos; };
+      for (int cc = 0; cc < 2; ++cc) {
+        if (!bad) {
+          tc_fence_after();
+          p_ds_rows(lane_base, kColS, kColP, row, half, cc, c2, sPt, sDSt, keep, [&](int c) { return L[c]; },
+                    [&](int c) { return Dl[c]; });
+        }
+        fence_async_smem();
+        tc_fence_before();
+        mbar_arrive(cc == 0 ? &s->p_half : &s->p_full);  // the MMA takes each chunk as it is done
       }
-      fence_async_smem();
-      tc_fence_before();
-      mbar_arrive(&s->p_full);
     }
     if (n > 0 && !bad && !mbar_wait_or_abort(&s->mma2_done, (uint32_t)(n - 1) & 1u, SITE_BWD_MMA, abort_flag))
       bad = true;
@@ -641,7 +659,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) softmax_dkdv_tc(
 }
 
 struct SmemDq {
-  uint64_t qd_full, k_full[2], v_full[2], kv_empty[2], s_full, ds_full, dq_done, drain;
+  uint64_t qd_full, k_full[2], v_full[2], kv_empty[2], s_full, ds_half, ds_full, dq_done, drain;
   uint32_t tmem_base;
   int abort;
 };
@@ -681,6 +699,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) softmax_dq_tc(
       mbar_init(&s->kv_empty[st], 1);
     }
     mbar_init(&s->s_full, 1);
+    mbar_init(&s->ds_half, 256);
     mbar_init(&s->ds_full, 256);
     mbar_init(&s->dq_done, 1);
     mbar_init(&s->drain, 1);
@@ -751,13 +770,24 @@ __global__ void __launch_bounds__(kBwdThreads, 1) softmax_dq_tc(
         tc_fence_after();
         for (int kk = 0; kk < kD / 16; ++kk) mma_bf16(tmem + kColP, kmaj(aO, kk), kmaj(aV, kk), id_kk, kk > 0);
         mma_commit(&s->s_full);
-        if (!mbar_wait_or_abort(&s->ds_full, (uint32_t)j & 1u, SITE_BWD_MMA, abort_flag)) {
+        // dQ += dS K over the key columns the epilogue has finished: K-steps
+        // 0, 1, 4, 5 (its first chunk), then 2, 3, 6, 7
+        bool part_ok = true;
+        for (int pc = 0; pc < 2; ++pc) {
+          if (!mbar_wait_or_abort(pc == 0 ? &s->ds_half : &s->ds_full, (uint32_t)j & 1u, SITE_BWD_MMA, abort_flag)) {
+            part_ok = false;
+            break;
+          }
+          tc_fence_after();
+          for (int q = 0; q < 4; ++q) {
+            const int kk = (q >> 1) * 4 + pc * 2 + (q & 1);
+            mma_bf16(tmem + kColQ, kmaj(aD, kk), mnmaj(aK, kk), id_kn, (j > 0 || pc > 0 || q > 0) ? 1u : 0u);
+          }
+        }
+        if (!part_ok) {
           bad = true;
           break;
         }
-        tc_fence_after();
-        for (int kk = 0; kk < kTile / 16; ++kk)
-          mma_bf16(tmem + kColQ, kmaj(aD, kk), mnmaj(aK, kk), id_kn, (j > 0 || kk > 0) ? 1u : 0u);
         mma_commit(&s->kv_empty[st]);
         mma_commit(&s->dq_done);
       }
@@ -780,16 +810,18 @@ __global__ void __launch_bounds__(kBwdThreads, 1) softmax_dq_tc(
       if (j > 0 && !bad && !mbar_wait_or_abort(&s->dq_done, (uint32_t)(j - 1) & 1u, SITE_BWD_MMA, abort_flag))
         bad = true;  // the last dQ MMA has read dS
       bad = __any_sync(0xffffffffu, bad);  // the TMEM loads below are warp-collective
-      if (!bad) {
-        tc_fence_after();
-        // P is not needed here: its tile is dS's, written twice, the second time with dS
-        p_ds_rows(lane_base, kColS, kColP, row, half, c2, sDS, sDS,
-                  [&](int c) { return in && kb + c <= qpos; }, [&](int) { return lse2; },
-                  [&](int) { return dl; });
+      for (int cc = 0; cc < 2; ++cc) {
+        if (!bad) {
+          tc_fence_after();
+          // P is not needed here: its tile is dS's, written twice, the second time with dS
+          p_ds_rows(lane_base, kColS, kColP, row, half, cc, c2, sDS, sDS,
+                    [&](int c) { return in && kb + c <= qpos; }, [&](int) { return lse2; },
+                    [&](int) { return dl; });
+        }
+        fence_async_smem();
+        tc_fence_before();
+        mbar_arrive(cc == 0 ? &s->ds_half : &s->ds_full);  // the MMA takes each chunk as it is done
       }
-      fence_async_smem();
-      tc_fence_before();
-      mbar_arrive(&s->ds_full);
     }
     if (!bad && !mbar_wait_or_abort(&s->dq_done, (uint32_t)(nkv - 1) & 1u, SITE_BWD_MMA, abort_flag)) bad = true;
     bad = __any_sync(0xffffffffu, bad);
