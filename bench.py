@@ -131,6 +131,9 @@ MEASURED_TRAFFIC = {
                     2 * (437725440 + 226706432)),
     "segment_states_tc": (["k_tc_states.cu", "sm100.cuh", "lasp_common.cuh", "tma_host.h"], "bfe2712019c7da94",
                           2 * (268476416 + 5191168)),
+    # the gated form (bench.py --gated): four times the capture of the 16384-token case
+    "gla_bwd_tc": (["k_tc_gla.cu", "sm100.cuh", "lasp_common.cuh", "tma_host.h"], "ec39fc0de472db0b",
+                   4 * (605854720 + 291032832)),
 }
 
 
@@ -341,7 +344,9 @@ def run_gpu(args, rank, world, local):
     # step i-1's results come out while step i's kernels run (PCIe is full
     # duplex); the device buffers alternate between two sets, ordered by events.
     outs_host = {n: torch.empty_like(host["q"]).pin_memory() for n in ("o", "dq", "dk", "dv")}
-    e2e_steps = max(1, min(args.steps, 5))
+    # enough steps that the pipeline's fill and drain (the first step's inputs
+    # and the last step's results cross alone) do not dominate
+    e2e_steps = max(1, min(args.steps, 30))
     ins = [dv_, {n: torch.empty_like(dv_[n]) for n in dv_}]
     outs = [{"o": o, "dq": dq, "dk": dk, "dv": dvv}, {n: torch.empty_like(q) for n in ("o", "dq", "dk", "dv")}]
     h2d, d2h = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
