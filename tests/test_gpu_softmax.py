@@ -131,3 +131,51 @@ def test_unsupported_and_invalid_sizes():
     with pytest.raises(lasp.LaspError) as e:
         lasp.lasp_softmax_fwd(q, k, k, q, lse)
     assert e.value.status == 1  # the queries reach past the keys
+
+
+def test_bench_size_sampled_rows_and_sums():
+    """The bench configuration (B1 H16 N65536 d128, causal, standard-normal
+    inputs) as bench.py --softmax runs it. The oracle checks sampled query
+    rows of o, lse and dq of two heads (a block of rows at its offset into the
+    keys), and dk, dv for their last 128 keys (every query that sees them lies
+    in the block of the last 128 queries). Over all keys two sums hold exactly:
+    sum_j dv_j = sum_i do_i (each row of attention weights sums to 1) and
+    sum_j dk_j = 0 (each row of ds sums to 0), per head and feature."""
+    import torch
+    import sequence_linear_attention_b200 as lasp
+    w = lasp_inputs.WORKLOADS["decayed_bf16_N64K"]
+    B, N, H, d = w["B"], w["N"], w["H"], w["d"]
+    inp = lasp_inputs.make_attention_inputs(B, N, N, H, d, seed=w["seed"])
+    q, k, v, do = (to_device(inp[n], True) for n in ("q", "k", "v", "do"))
+    o, dq, dk, dv = (torch.empty_like(q) for _ in range(4))
+    lse = torch.empty((B, H, N), dtype=torch.float32, device="cuda")
+    delta = torch.empty_like(lse)
+    lasp.lasp_softmax_fwd(q, k, v, o, lse)
+    lasp.lasp_softmax_bwd(q, k, v, o, lse, do, dq, dk, dv, delta)
+    st, site = lasp.lasp_check_device_status()
+    assert st == 0, (st, site)
+    f = {n: lasp_inputs.as_f32(inp[n], True) for n in ("q", "k", "v", "do")}
+    go, gdq, gdk, gdv = (to_host(t) for t in (o, dq, dk, dv))
+    glse = lse.cpu().numpy()
+    heads = [5, 12]  # two sampled heads for the oracle (its cost grows with N^2 per head)
+    hk, hv = f["k"][:, :, heads], f["v"][:, :, heads]
+    tail = 128
+    # query blocks at the start, in the middle (off the tile grid) and at the end
+    for r0, n in ((0, 96), (30001, 64), (N - tail, tail)):
+        qs = np.ascontiguousarray(f["q"][:, r0:r0 + n][:, :, heads])
+        dos = np.ascontiguousarray(f["do"][:, r0:r0 + n][:, :, heads])
+        ro, rl = oracle.softmax_fwd(qs, hk, hv, q_offset=r0)
+        assert rel_err(go[:, r0:r0 + n][:, :, heads], ro) <= TOL_BF16, r0
+        assert rel_err(glse[:, heads, r0:r0 + n], rl) <= TOL_BF16, r0
+        if r0 == N - tail:
+            rdq, rdk, rdv = oracle.softmax_bwd(qs, hk, hv, dos, q_offset=r0)
+            assert rel_err(gdq[:, r0:][:, :, heads], rdq) <= TOL_BF16
+            assert rel_err(gdk[:, r0:][:, :, heads], rdk[:, r0:]) <= TOL_BF16
+            assert rel_err(gdv[:, r0:][:, :, heads], rdv[:, r0:]) <= TOL_BF16
+    # every head: the sums over all keys
+    sdv = gdv.astype(np.float64).sum(axis=1)
+    sdo = f["do"].astype(np.float64).sum(axis=1)
+    assert rel_err(sdv, sdo) <= TOL_BF16
+    # sum_j dk_j = 0: against the size of the terms it sums
+    sdk = np.abs(gdk.astype(np.float64).sum(axis=1))
+    assert float(sdk.max()) <= TOL_BF16 * float(np.abs(gdk).sum(axis=1).max())
