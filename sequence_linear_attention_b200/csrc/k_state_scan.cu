@@ -53,9 +53,9 @@ __global__ void __launch_bounds__(kThreads) state_scan_kernel(const float4* M, f
                                                               int slot_offset, int gsum_offset, RunIf run_if,
                                                               int64_t idx0) {
   if (!runs(run_if)) return;
-  // threads idx0 .. idx0 + n_threads - 1 of the whole (b, h, float4) space
-  for (int64_t idx = idx0 + (int64_t)blockIdx.x * kThreads + threadIdx.x; idx < idx0 + n_threads;
-       idx += (int64_t)gridDim.x * kThreads) {
+  // thread idx of idx0 .. idx0 + n_threads - 1 of the whole (b, h, float4) space
+  const int64_t idx = idx0 + (int64_t)blockIdx.x * kThreads + threadIdx.x;
+  if (idx >= idx0 + n_threads) return;
   const int e = (int)(idx % dd4);
   const int h = (int)((idx / dd4) % H);
   const int64_t b = idx / ((int64_t)dd4 * H);
@@ -123,7 +123,6 @@ __global__ void __launch_bounds__(kThreads) state_scan_kernel(const float4* M, f
     goff += gstep;
   }
   if (total) total[bh * dd4 + e] = acc;
-  }
 }
 
 }  // namespace scan_detail
@@ -147,7 +146,8 @@ cudaError_t launch_gla_scan(const float* M, float* P, const float* gsum, const f
                             int gsum_offset, cudaStream_t st, RunIf run) {
   const int dd4 = d * d / 4;
   const int64_t n_threads = (int64_t)B * H * dd4;
-  const int64_t blocks = grid_for((n_threads + scan_detail::kThreads - 1) / scan_detail::kThreads, run);
+  // one thread per element: a launch that returns at once still has the full grid
+  const int64_t blocks = (n_threads + scan_detail::kThreads - 1) / scan_detail::kThreads;
   scan_detail::state_scan_kernel<true><<<(unsigned)blocks, scan_detail::kThreads, 0, st>>>(
       (const float4*)M, (float4*)P, nullptr, gsum, (const float4*)init, (float4*)total, H, T, d, dd4, n_threads,
       1.f, reverse, t_slots, slot_stride, slot_offset, gsum_offset, run, 0);
