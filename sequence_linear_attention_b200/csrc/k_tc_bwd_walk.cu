@@ -178,6 +178,14 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_walk_tc(
   if (warp == kProducerWarp) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
+      // the forward's cached bf16 tile of the state entering the tile at row
+      // `row` of the sequence: in the slot of the tile's first chunk, the
+      // second half of that slot for the second tile of a 256-token chunk
+      auto ptile = [&](const Item& it, int64_t row) {
+        const int half_of_chunk = C > kTile ? (int)((row / kTile) % (C / kTile)) : 0;
+        return reinterpret_cast<const uint8_t*>(P + (((int64_t)it.b * T + row / C) * H + it.h) * kD * kD) +
+               (size_t)half_of_chunk * kTileBytes;
+      };
       auto load_kv = [&](const Item& it, int t) {
         const int row = it.seg * G + t * kTile;
         mbar_arrive_expect_tx(&s->ld_kv, 2 * kTileBytes);
@@ -199,10 +207,8 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_walk_tc(
       // P of a chunk: the forward walk stored it in the chunk's cache slot as the
       // bf16 operand tile (128-byte swizzled), so it is copied into X as is
       auto load_p = [&](const Item& it, int t) {
-        const int64_t c = ((int64_t)it.seg * G + (int64_t)t * kTile) / C;  // the tile's first chunk
-        const float* src = P + (((int64_t)it.b * T + c) * H + it.h) * kD * kD;
         mbar_arrive_expect_tx(&s->ld_p, kTileBytes);
-        bulk_load(sX, src, kTileBytes, &s->ld_p);
+        bulk_load(sX, ptile(it, (int64_t)it.seg * G + (int64_t)t * kTile), kTileBytes, &s->ld_p);
       };
       // one bulk group per tensor, so that the dK buffer frees up first
       auto store_tile = [&](const CUtensorMap* map, const uint8_t* src, const Item& it, int row0) {
@@ -272,8 +278,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_walk_tc(
             tma_prefetch_4d(&map_k, 64, nx.h, nrow, nx.b);
             tma_prefetch_4d(&map_v, 0, nx.h, nrow, nx.b);
             tma_prefetch_4d(&map_v, 64, nx.h, nrow, nx.b);
-            const int64_t c = (int64_t)nrow / C;
-            bulk_prefetch_l2(P + (((int64_t)nx.b * T + c) * H + nx.h) * kD * kD, kTileBytes);
+            bulk_prefetch_l2(ptile(nx, nrow), kTileBytes);
           }
           if (t == (tiles > 1 ? 1 : 0) && w + gridDim.x < nitems) {
             // and the next segment's entering R, read at the segment switch
@@ -583,11 +588,14 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_walk_tc(
 }  // namespace tc_bwd_walk_detail
 
 bool tc_bwd_walk_ok(int dtype, int d, int64_t C, int64_t N) {
-  // chunks that divide the 128-token tile: the forward walk leaves the bf16
-  // operand tile of each tile's entering state in the slot of its first chunk
+  // chunks that divide the 128-token tile, or of two tiles: the forward walk
+  // leaves the bf16 operand tile of each tile's entering state in the slot of
+  // its first chunk (C = 256: the two tiles of a chunk in the two halves of its
+  // 64 KB slot)
   using tc_bwd_walk_detail::kTile;
-  return dtype == LASP_BF16 && d == tc_bwd_walk_detail::kD && C >= 1 && C <= kTile && kTile % C == 0 &&
-         N % kTile == 0;
+  if (dtype != LASP_BF16 || d != tc_bwd_walk_detail::kD || C < 1) return false;
+  if (C == 2 * kTile) return N % C == 0;
+  return C <= kTile && kTile % C == 0 && N % kTile == 0;
 }
 
 cudaError_t tc_bwd_walk(const void* q, const void* k, const void* v, const void* dout, const float* decay,

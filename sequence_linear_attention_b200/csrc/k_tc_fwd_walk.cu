@@ -17,14 +17,16 @@
 //   epi A1: S' = Mask . S -> bf16 over Q (once both parts of MMA 1 have read Q)
 //   MMA 2a: O_intra = S' V (TMEM O), under
 //   epi A2: K~ = diag(lambda^{127-j}) K in place; P <- lambda^128 P in TMEM (and,
-//           for C > 128, P -> fp32 cache at chunk starts)
+//           for C > 256, P -> fp32 cache at chunk starts)
 //   MMA 2b: P += K~^T V (TMEM P), under
 //   epi B1: O = O_intra + lambda^{i+1} O_inter -> bf16 over S' -> TMA store
 //   epi B2: P -> bf16 operand for the next tile
 //
 // With C = 128 each tile starts a chunk, and the bf16 operand tile of the
 // entering state (already in shared memory for O_inter) goes to the chunk's
-// cache slot by one bulk copy; the backward walk loads it back as is. Two sets
+// cache slot by one bulk copy; the backward walk loads it back as is. Shorter
+// chunks use the slot of the tile's first chunk; C = 256 puts the two tiles of
+// a chunk in the two halves of its slot. Two sets
 // of Q/K/V buffers alternate: while a tile is computed, the next tile's loads
 // (possibly of the next segment) are in flight; a segment's fp32 entering state
 // is loaded by TMA into the K and V buffers of the set the previous tile used.
@@ -229,7 +231,11 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_walk_tc(const __grid_constant
           // shared memory, is the cache entry the backward pass loads back
           if (!(ok = mbar_wait_or_abort(&s->e_b2, par, SITE_OUT_TMA, abort_flag))) break;
           if (cache_bf16) {
-            uint8_t* slot = reinterpret_cast<uint8_t*>(P + (((int64_t)item.b * T + row0 / C) * H + item.h) * kD * kD);
+            // in the slot of the tile's first chunk; with C = 256 one 64 KB slot
+            // holds the tiles of both halves of its chunk
+            const int half_of_chunk = C > kTile ? (row0 / kTile) % (C / kTile) : 0;
+            uint8_t* slot = reinterpret_cast<uint8_t*>(P + (((int64_t)item.b * T + row0 / C) * H + item.h) * kD * kD) +
+                            (size_t)half_of_chunk * kTileBytes;
             bulk_store(slot, sP, kTileBytes);
             tma_store_commit();
             tma_store_wait_read0();
@@ -547,10 +553,11 @@ cudaError_t tc_fwd_walk(const void* q, const void* k, const void* v, const float
   const int64_t nitems = nbh * nseg;
   if (nitems == 0) return cudaSuccess;
   const unsigned grid = (unsigned)std::min<int64_t>(nitems, num_sms);
-  // with chunks that divide the tile the backward walk reads the cache: it gets
-  // each tile's entering state as the bf16 operand tile (in the slot of the
-  // tile's first chunk); with longer chunks the cache holds fp32 states
-  const int cache_bf16 = C <= kTile ? 1 : 0;
+  // with chunks that divide the tile, or of two tiles, the backward walk reads
+  // the cache: it gets each tile's entering state as the bf16 operand tile (in
+  // the slot of the tile's first chunk, two tiles to a slot when C = 256); with
+  // longer chunks the cache holds fp32 states
+  const int cache_bf16 = (C <= kTile || C == 2 * kTile) ? 1 : 0;
   fwd_walk_tc<<<grid, kThreads, smem, st>>>(mq, mk, mv, mo, mp, decay, P, H, (int)(N / C), C, G, nseg, nitems,
                                            cache_bf16, bh0 * nseg);
   return cudaGetLastError();

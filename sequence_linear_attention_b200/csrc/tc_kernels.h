@@ -27,9 +27,10 @@ cudaError_t tc_chunk_states_slots(const void* a, const void* b, const float* dec
 // d = 128, C a multiple of 128 or a divisor of it, N a multiple of max(C, 128),
 // G = walk_segment_tokens(N, C)). P must hold, in the slot of each segment's
 // first chunk, the state entering that segment; the walk writes o and fills the
-// cache: fp32 P_c at the other chunk starts when C > 128, otherwise the bf16
+// cache: fp32 P_c at the other chunk starts when C > 256, otherwise the bf16
 // operand tile of the state entering each 128-token tile in the slot of the
-// tile's first chunk.
+// tile's first chunk (C = 256: both tiles of a chunk in the two halves of its
+// slot).
 bool tc_fwd_walk_ok(int dtype, int d, int64_t C, int64_t N);
 int walk_segment_tokens(int64_t N, int C);
 cudaError_t tc_fwd_walk(const void* q, const void* k, const void* v, const float* decay, float* P, void* o, int B,
@@ -37,7 +38,7 @@ cudaError_t tc_fwd_walk(const void* q, const void* k, const void* v, const float
                         int64_t nbh = -1);
 
 // Backward walk over segments with the gradient state on chip (bf16, d = 128,
-// C dividing 128, N a multiple of 128). R must hold, in the slot of each
+// C dividing 128 with N a multiple of 128, or C = 256 with N a multiple of 256). R must hold, in the slot of each
 // segment's last chunk, the gradient state entering that chunk from the tokens
 // after the segment; the walk writes dq, dk, dv (R of the other chunks stays on
 // chip). P is the forward walk's cache of bf16 operand tiles.

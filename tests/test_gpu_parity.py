@@ -43,7 +43,8 @@ SMALL = [
     (1, 2, 128, 128, 128, True, True),   # a single chunk
     (2, 2, 64, 64, 1, False, True),      # C = 1: pure inter-chunk
     (1, 2, 2048, 128, 128, True, True),  # forward walk over two 1024-token segments
-    (2, 3, 1536, 128, 256, True, True),  # chunks of two tiles
+    (2, 3, 1536, 128, 256, True, True),  # chunks of two tiles (both walks)
+    (1, 2, 2048, 128, 256, True, False),  # two 1024-token segments of four such chunks
     (1, 2, 1024, 128, 512, True, False),
     (2, 150, 1024, 128, 128, True, True),  # more segments than SMs: each CTA walks several
     (2, 3, 1152, 128, 128, True, True),    # three segments of three tiles

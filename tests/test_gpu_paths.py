@@ -44,9 +44,18 @@ def test_bf16_c64_with_a_ragged_tile_runs_the_per_chunk_tensor_core_kernels():
                      "chunk_states_tc", "state_scan", "chunk_bwd_tc"], names
 
 
-def test_bf16_c256_walks_forward_and_uses_cuda_cores_backward():
+def test_bf16_c256_runs_the_segment_walks():
+    """Chunks of two tiles walk both ways: the forward leaves both tiles'
+    entering states in the two halves of the chunk's cache slot."""
     inp = lasp_inputs.make_inputs(1, 1024, 2, 128, seed=203, bf16=True, decayed=True)
     names = _traced_names(inp, 256)
+    assert names == ["segment_states_tc", "segment_scan", "fwd_walk_tc",
+                     "segment_states_tc", "segment_scan", "bwd_walk_tc"], names
+
+
+def test_bf16_c512_walks_forward_and_uses_cuda_cores_backward():
+    inp = lasp_inputs.make_inputs(1, 1024, 2, 128, seed=203, bf16=True, decayed=True)
+    names = _traced_names(inp, 512)
     assert names[:3] == ["segment_states_tc", "segment_scan", "fwd_walk_tc"], names
     assert names[3:] == ["chunk_states_tc", "state_scan", "chunk_bwd_simt"], names
 

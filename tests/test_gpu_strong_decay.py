@@ -30,7 +30,8 @@ PATHS = {
     "walks_C64": (2, 1024, 128, 64, True),     # walks with chunks that divide the tile
     "per_chunk_tc": (1, 320, 128, 64, True),   # ragged tile: per-chunk tensor-core kernels
     "simt_f32_d64": (1, 256, 64, 64, False),   # CUDA cores, fp32
-    "bf16_C256": (1, 1024, 128, 256, True),    # forward walk, CUDA-core backward
+    "bf16_C256": (1, 1024, 128, 256, True),    # walks with chunks of two tiles
+    "bf16_C512": (1, 1024, 128, 512, True),    # forward walk, CUDA-core backward
 }
 
 
