@@ -1,5 +1,5 @@
 // Backward pass of one 128-token tile on the 5th-generation tensor cores
-// (LASP Eq. 14, 16, 17, 19, 22, 23; Algorithm 3 steps 7-17), bf16, d = 128:
+// (LASP Eq. 14, 16, 17, 19, 22, 23; Algorithm 3 steps 7-17), bf16, d = 128, 64 or 32:
 //   dP = (dO V^T) . Mask,  S = (Q K^T) . Mask,   Mask_ij = lambda^{i-j} (j <= i)
 //   dQ = dP K   + diag(lambda^{i+1})    dO P^T
 //   dK = dP^T Q + diag(lambda^{e-j})    V  R^T
@@ -24,6 +24,12 @@
 //   phase 2:  T3 = dP' K                                     -> epilogue 2 (dQ)
 //   phase 3:  T0 = dP'^T Q, T1 = S'^T dO, T2 = V R^T, T3 = K R -> epilogue 3 (dK, dV)
 // The decay factors of the inter terms are applied in fp32 in the epilogues.
+// With d = 64 or 32 the tiles keep their 128 features: the second 64-feature
+// box of Q, K, V and dO is zero in shared memory instead of loaded (for d = 32
+// the first box's upper 32 features read as zeros: they lie past the tensor's
+// feature extent), P and R fill the top-left d x d block of X, the feature
+// reductions stop at d and only the first d columns of dQ, dK and dV are
+// stored.
 #include "kernels.h"
 #include "lasp_common.cuh"
 #include "sm100.cuh"
@@ -61,13 +67,16 @@ __device__ __forceinline__ void put_state_row(uint8_t* tile, int r, int lane, fl
   *reinterpret_cast<uint2*>(tile + off) = make_uint2(pack_bf16(x.x, x.y), pack_bf16(x.z, x.w));
 }
 
-// fp32 d x d state in global memory -> bf16 tile. Warp w converts rows w,
-// w + 8, ...; all of its loads are in flight together.
-__device__ __forceinline__ void load_state_tile(uint8_t* tile, const float* src, int warp, int lane) {
+// fp32 d x d state in global memory -> bf16 tile (zero outside d x d). Warp w
+// converts rows w, w + 8, ...; all of its loads are in flight together.
+__device__ __forceinline__ void load_state_tile(uint8_t* tile, const float* src, int d, int warp, int lane) {
   const float4* p = reinterpret_cast<const float4*>(src);
   float4 x[kRowsPerWarp];
 #pragma unroll
-  for (int u = 0; u < kRowsPerWarp; ++u) x[u] = __ldcs(p + (warp + kWarps * u) * (kD / 4) + lane);
+  for (int u = 0; u < kRowsPerWarp; ++u) {
+    const int r = warp + kWarps * u;
+    x[u] = r < d && 4 * lane < d ? __ldcs(p + r * (d / 4) + lane) : make_float4(0.f, 0.f, 0.f, 0.f);
+  }
 #pragma unroll
   for (int u = 0; u < kRowsPerWarp; ++u) put_state_row(tile, warp + kWarps * u, lane, x[u]);
 }
@@ -81,8 +90,8 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_bwd_tc(const __grid_constan
                                                              const __grid_constant__ CUtensorMap map_dv,
                                                              const float* decay, const float* __restrict__ P,
                                                              const float* __restrict__ R,
-                                                             __nv_bfloat16* __restrict__ dq, int H, int64_t N,
-                                                             int T, int C) {
+                                                             __nv_bfloat16* __restrict__ dq, int H, int d,
+                                                             int64_t N, int T, int C) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   uint8_t* sQ = base;
@@ -100,7 +109,16 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_bwd_tc(const __grid_constan
   const int last = (int)min((int64_t)kTile, N - row0) - 1;  // last valid row of the tile
   const float lam = load_decay(decay, h);
   const float l2 = log2f(lam);
+  const int nbox = d > 64 ? 2 : 1;  // 64-feature boxes loaded per tile
 
+  if (nbox == 1) {
+    // the second box of Q, K, V and dO stays zero
+    for (int t = 0; t < 4; ++t) {
+      uint4* z = reinterpret_cast<uint4*>(base + t * kTileBytes + kBox);
+      for (uint32_t q = tid; q < kBox / 16; q += kThreads) z[q] = make_uint4(0, 0, 0, 0);
+    }
+    fence_async_smem();
+  }
   if (tid == 0) {
     prefetch_tmap(&map_q);
     prefetch_tmap(&map_k);
@@ -129,25 +147,29 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_bwd_tc(const __grid_constan
   const uint32_t T0 = 0, T1 = 128, T2 = 256, T3 = 384;
 
   if (tid == 0) {
-    mbar_arrive_expect_tx(&s->load, 4 * kTileBytes);
+    mbar_arrive_expect_tx(&s->load, 4 * nbox * kBox);
     tma_load_4d(sQ, &map_q, &s->load, 0, h, row0, b);
-    tma_load_4d(sQ + kBox, &map_q, &s->load, 64, h, row0, b);
     tma_load_4d(sK, &map_k, &s->load, 0, h, row0, b);
-    tma_load_4d(sK + kBox, &map_k, &s->load, 64, h, row0, b);
     tma_load_4d(sV, &map_v, &s->load, 0, h, row0, b);
-    tma_load_4d(sV + kBox, &map_v, &s->load, 64, h, row0, b);
     tma_load_4d(sD, &map_do, &s->load, 0, h, row0, b);
-    tma_load_4d(sD + kBox, &map_do, &s->load, 64, h, row0, b);
+    if (nbox == 2) {
+      tma_load_4d(sQ + kBox, &map_q, &s->load, 64, h, row0, b);
+      tma_load_4d(sK + kBox, &map_k, &s->load, 64, h, row0, b);
+      tma_load_4d(sV + kBox, &map_v, &s->load, 64, h, row0, b);
+      tma_load_4d(sD + kBox, &map_do, &s->load, 64, h, row0, b);
+    }
   }
   const int c_first = row0 / C, c_last = (row0 + last) / C;
   if (tid == 32) {
-    // R of the tile's last chunk, fp32, into the (still unused) dP'/S' space
-    const float* Rc = R + ((((int64_t)b * T + c_last) * H + h) * kD) * kD;
-    mbar_arrive_expect_tx(&s->rload, kD * kD * 4);
-    for (int part = 0; part < 4; ++part)
-      bulk_load(sA + part * (kD * kD), Rc + part * (kD * kD / 4), kD * kD, &s->rload);
+    // R of the tile's last chunk, fp32 [d][d], into the (still unused) dP'/S'
+    // space, in copies of at most 16 KB
+    const float* Rc = R + ((((int64_t)b * T + c_last) * H + h) * d) * d;
+    const uint32_t rbytes = d * d * 4, pb = rbytes < 16384 ? rbytes : 16384;
+    mbar_arrive_expect_tx(&s->rload, rbytes);
+    for (uint32_t part = 0; part < rbytes / pb; ++part)
+      bulk_load(sA + part * pb, Rc + part * (pb / 4), pb, &s->rload);
   }
-  load_state_tile(sX, P + ((((int64_t)b * T + c_first) * H + h) * kD) * kD, warp, lane);
+  load_state_tile(sX, P + ((((int64_t)b * T + c_first) * H + h) * d) * d, d, warp, lane);
   fence_async_smem();
   __syncthreads();
 
@@ -161,10 +183,10 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_bwd_tc(const __grid_constan
   if (tid == 0) {
     if (mbar_wait(&s->load, 0, SITE_BWD_TMA)) {
       tc_fence_after();
-      for (int kk = 0; kk < kD / 16; ++kk) mma_bf16(tmem + T0, kmaj(aD, kk), kmaj(aV, kk), id_kk, kk != 0);
-      for (int kk = 0; kk < kD / 16; ++kk) mma_bf16(tmem + T1, kmaj(aQ, kk), kmaj(aK, kk), id_kk, kk != 0);
+      for (int kk = 0; kk < d / 16; ++kk) mma_bf16(tmem + T0, kmaj(aD, kk), kmaj(aV, kk), id_kk, kk != 0);
+      for (int kk = 0; kk < d / 16; ++kk) mma_bf16(tmem + T1, kmaj(aQ, kk), kmaj(aK, kk), id_kk, kk != 0);
       mma_commit(&s->mma1a);
-      for (int kk = 0; kk < kD / 16; ++kk) mma_bf16(tmem + T2, kmaj(aD, kk), kmaj(aX, kk), id_kk, kk != 0);
+      for (int kk = 0; kk < d / 16; ++kk) mma_bf16(tmem + T2, kmaj(aD, kk), kmaj(aX, kk), id_kk, kk != 0);
       mma_commit(&s->mma1b);
     } else {
       s->abort = 1;
@@ -176,7 +198,10 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_bwd_tc(const __grid_constan
   if (mbar_wait(&s->rload, 0, SITE_BWD_TMA)) {
     const float4* rs4 = reinterpret_cast<const float4*>(sA);
 #pragma unroll
-    for (int u = 0; u < kRowsPerWarp; ++u) rreg[u] = rs4[(warp + kWarps * u) * (kD / 4) + lane];
+    for (int u = 0; u < kRowsPerWarp; ++u) {
+      const int r = warp + kWarps * u;
+      rreg[u] = r < d && 4 * lane < d ? rs4[r * (d / 4) + lane] : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
   } else {
     s->abort = 1;
   }
@@ -236,9 +261,9 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_bwd_tc(const __grid_constan
     tc_fence_after();
     const float wi = decay_pow(l2, (float)(i + 1));
     const bool valid = i <= last;
-    __nv_bfloat16* out = dq + (((int64_t)b * N + row0 + i) * H + h) * kD;
+    __nv_bfloat16* out = dq + (((int64_t)b * N + row0 + i) * H + h) * d;
 #pragma unroll 1
-    for (int cc = 2 * half; cc < 2 * half + 2; ++cc) {
+    for (int cc = 2 * half; cc < 2 * half + 2 && cc * 32 < d; ++cc) {
       uint32_t ra[32], re[32];
       tmem_ld32(lane_base + T3 + cc * 32, ra);
       tmem_ld32(lane_base + T2 + cc * 32, re);
@@ -267,8 +292,8 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_bwd_tc(const __grid_constan
     tc_fence_after();
     for (int kk = 0; kk < kTile / 16; ++kk) mma_bf16(tmem + T0, mnmaj(aA, kk), mnmaj(aQ, kk), id_nn, kk != 0);
     for (int kk = 0; kk < kTile / 16; ++kk) mma_bf16(tmem + T1, mnmaj(aB, kk), mnmaj(aD, kk), id_nn, kk != 0);
-    for (int kk = 0; kk < kD / 16; ++kk) mma_bf16(tmem + T2, kmaj(aV, kk), kmaj(aX, kk), id_kk, kk != 0);
-    for (int kk = 0; kk < kD / 16; ++kk) mma_bf16(tmem + T3, kmaj(aK, kk), mnmaj(aX, kk), id_kn, kk != 0);
+    for (int kk = 0; kk < d / 16; ++kk) mma_bf16(tmem + T2, kmaj(aV, kk), kmaj(aX, kk), id_kk, kk != 0);
+    for (int kk = 0; kk < d / 16; ++kk) mma_bf16(tmem + T3, kmaj(aK, kk), mnmaj(aX, kk), id_kn, kk != 0);
     mma_commit(&s->mma3);
   }
 
@@ -311,9 +336,11 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_bwd_tc(const __grid_constan
   __syncthreads();
   if (tid == 0 && !s->abort) {
     tma_store_4d(&map_dk, sA, 0, h, row0, b);
-    tma_store_4d(&map_dk, sA + kBox, 64, h, row0, b);
     tma_store_4d(&map_dv, sB, 0, h, row0, b);
-    tma_store_4d(&map_dv, sB + kBox, 64, h, row0, b);
+    if (nbox == 2) {
+      tma_store_4d(&map_dk, sA + kBox, 64, h, row0, b);
+      tma_store_4d(&map_dv, sB + kBox, 64, h, row0, b);
+    }
     tma_store_commit();
     tma_store_wait_read0();
   }
@@ -327,7 +354,7 @@ cleanup:
 }  // namespace tc_bwd_detail
 
 bool tc_bwd_ok(int dtype, int d, int64_t C) {
-  return dtype == LASP_BF16 && d == tc_bwd_detail::kD && C <= tc_bwd_detail::kTile && tc_bwd_detail::kTile % C == 0 &&
+  return dtype == LASP_BF16 && (d == 32 || d == 64 || d == tc_bwd_detail::kD) && C <= tc_bwd_detail::kTile && tc_bwd_detail::kTile % C == 0 &&
          C % 16 == 0;
 }
 
@@ -345,7 +372,7 @@ cudaError_t tc_chunk_bwd(const void* q, const void* k, const void* v, const void
   if (e != cudaSuccess) return e;
   const unsigned tiles = (unsigned)((N + kTile - 1) / kTile);
   dim3 grid(tiles, H, B);
-  chunk_bwd_tc<<<grid, kThreads, smem, st>>>(mq, mk, mv, mdo, mdk, mdv, decay, P, Rs, (__nv_bfloat16*)dq, H, N,
+  chunk_bwd_tc<<<grid, kThreads, smem, st>>>(mq, mk, mv, mdo, mdk, mdv, decay, P, Rs, (__nv_bfloat16*)dq, H, d, N,
                                              (int)(N / C), C);
   return cudaGetLastError();
 }

@@ -1,5 +1,5 @@
 // Forward output on the 5th-generation tensor cores (LASP Eq. 7, 9, 11;
-// Algorithm 2 steps 9, 14, 15), for bf16 inputs with d = 128:
+// Algorithm 2 steps 9, 14, 15), for bf16 inputs with d = 128, 64 or 32:
 //   O = [(Q K^T) . Mask] V + Lambda Q P,  Mask_ij = lambda^{i-j} (j <= i), Lambda = diag(lambda^{i+1}),
 // over a tile of 128 tokens that starts at a chunk boundary; P is the state
 // entering the tile (the cached P_c of its first chunk). When C < 128 a tile
@@ -18,6 +18,12 @@
 //  4. thread 0: O_intra = S' V (cols 128..255).
 //  5. all: O = O_intra + lambda^{i+1} O_inter in fp32, bf16 into the Q tile,
 //     then one TMA store of the 128 x 128 tile (rows past N are dropped).
+// With d = 64 or 32 the tiles keep their 128 features: the second 64-feature
+// box of Q, K and V is zero in shared memory instead of loaded (for d = 32 the
+// first box's upper 32 features read as zeros: they lie past the tensor's
+// feature extent), P fills the top-left d x d block of its tile, the feature
+// reductions stop at d and only the first box of the output is stored (its
+// columns past d are dropped).
 #include "kernels.h"
 #include "lasp_common.cuh"
 #include "sm100.cuh"
@@ -54,7 +60,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_out_tc(const __grid_constan
                                                              const __grid_constant__ CUtensorMap map_v,
                                                              const __grid_constant__ CUtensorMap map_o,
                                                              const float* decay, const float* __restrict__ P,
-                                                             int H, int T, int C) {
+                                                             int H, int d, int T, int C) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   uint8_t* sQ = base;                    // Q, later the output tile
@@ -68,7 +74,16 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_out_tc(const __grid_constan
   const int row0 = tile * kTile;
   const float lam = load_decay(decay, h);
   const float l2 = log2f(lam);
+  const int nbox = d > 64 ? 2 : 1;  // 64-feature boxes loaded per tile
 
+  if (nbox == 1) {
+    // the second box of Q, K and V stays zero
+    for (int t = 0; t < 3; ++t) {
+      uint4* z = reinterpret_cast<uint4*>(base + t * kTileBytes + kBox);
+      for (uint32_t q = tid; q < kBox / 16; q += kThreads) z[q] = make_uint4(0, 0, 0, 0);
+    }
+    fence_async_smem();
+  }
   if (tid == 0) {
     prefetch_tmap(&map_q);
     prefetch_tmap(&map_k);
@@ -91,26 +106,32 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_out_tc(const __grid_constan
   const uint32_t tmem = s->tmem_base;
 
   if (tid == 0) {
-    mbar_arrive_expect_tx(&s->load, 3 * kTileBytes);
+    mbar_arrive_expect_tx(&s->load, 3 * nbox * kBox);
     tma_load_4d(sQ, &map_q, &s->load, 0, h, row0, b);
-    tma_load_4d(sQ + kBox, &map_q, &s->load, 64, h, row0, b);
     tma_load_4d(sK, &map_k, &s->load, 0, h, row0, b);
-    tma_load_4d(sK + kBox, &map_k, &s->load, 64, h, row0, b);
     tma_load_4d(sV, &map_v, &s->load, 0, h, row0, b);
-    tma_load_4d(sV + kBox, &map_v, &s->load, 64, h, row0, b);
+    if (nbox == 2) {
+      tma_load_4d(sQ + kBox, &map_q, &s->load, 64, h, row0, b);
+      tma_load_4d(sK + kBox, &map_k, &s->load, 64, h, row0, b);
+      tma_load_4d(sV + kBox, &map_v, &s->load, 64, h, row0, b);
+    }
   }
 
-  // P of the tile's first chunk, fp32 [k][v] -> bf16 operand tile (row k, column v)
+  // P of the tile's first chunk, fp32 [k][v] -> bf16 operand tile (row k,
+  // column v; zero outside d x d)
   {
     const int c0 = row0 / C;
-    const float4* Pc = reinterpret_cast<const float4*>(P + ((((int64_t)b * T + c0) * H + h) * kD) * kD);
+    const float4* Pc = reinterpret_cast<const float4*>(P + ((((int64_t)b * T + c0) * H + h) * d) * d);
     // warp w converts rows w, w + 8, ...: all 16 of its loads are in flight together
     constexpr int kWarps = kThreads / 32, kRows = kD / kWarps;
     const int col = lane * 4;
     {
       float4 x[kRows];
 #pragma unroll
-      for (int u = 0; u < kRows; ++u) x[u] = __ldcs(Pc + (warp + kWarps * u) * (kD / 4) + lane);
+      for (int u = 0; u < kRows; ++u) {
+        const int r = warp + kWarps * u;
+        x[u] = r < d && col < d ? __ldcs(Pc + r * (d / 4) + lane) : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
 #pragma unroll
       for (int u = 0; u < kRows; ++u) {
         const int r = warp + kWarps * u;
@@ -129,13 +150,13 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_out_tc(const __grid_constan
       tc_fence_after();
       const uint32_t q0 = smem_u32(sQ), k0 = smem_u32(sK), p0 = smem_u32(sP);
       // S = Q K^T : K index = feature (16 per MMA), both operands K-major
-      for (int kk = 0; kk < kD / 16; ++kk) {
+      for (int kk = 0; kk < d / 16; ++kk) {
         const uint32_t off = (kk >> 2) * kBox + (kk & 3) * 32;
         mma_bf16(tmem + kColS, sw128_desc(q0 + off, 16, 1024), sw128_desc(k0 + off, 16, 1024), idesc_kk, kk != 0);
       }
       mma_commit(&s->s_done);
       // O_inter = Q P : K index = key feature; P rows are key features (MN-major B)
-      for (int kk = 0; kk < kD / 16; ++kk) {
+      for (int kk = 0; kk < d / 16; ++kk) {
         const uint32_t aoff = (kk >> 2) * kBox + (kk & 3) * 32;
         mma_bf16(tmem + kColInter, sw128_desc(q0 + aoff, 16, 1024), sw128_desc(p0 + kk * 2048, kBox, 1024),
                  idesc_kn, kk != 0);
@@ -215,7 +236,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_out_tc(const __grid_constan
   __syncthreads();
   if (tid == 0 && ok) {
     tma_store_4d(&map_o, sQ, 0, h, row0, b);
-    tma_store_4d(&map_o, sQ + kBox, 64, h, row0, b);
+    if (nbox == 2) tma_store_4d(&map_o, sQ + kBox, 64, h, row0, b);
     tma_store_commit();
     tma_store_wait_read0();
   }
@@ -225,7 +246,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_out_tc(const __grid_constan
 }  // namespace tc_out_detail
 
 bool tc_out_ok(int dtype, int d, int64_t C) {
-  return dtype == LASP_BF16 && d == tc_out_detail::kD && C <= tc_out_detail::kTile && tc_out_detail::kTile % C == 0 &&
+  return dtype == LASP_BF16 && (d == 32 || d == 64 || d == tc_out_detail::kD) && C <= tc_out_detail::kTile && tc_out_detail::kTile % C == 0 &&
          C % 16 == 0;
 }
 
@@ -241,7 +262,7 @@ cudaError_t tc_chunk_out(const void* q, const void* k, const void* v, const floa
   if (e != cudaSuccess) return e;
   const unsigned tiles = (unsigned)((N + kTile - 1) / kTile);
   dim3 grid(tiles, H, B);
-  chunk_out_tc<<<grid, kThreads, smem, st>>>(mq, mk, mv, mo, decay, P, H, (int)(N / C), C);
+  chunk_out_tc<<<grid, kThreads, smem, st>>>(mq, mk, mv, mo, decay, P, H, d, (int)(N / C), C);
   return cudaGetLastError();
 }
 

@@ -8,7 +8,9 @@
 // or the largest of 64/32/16 dividing C); the stages of all of a CTA's chunks
 // form one stream through up to six shared-memory slots (192 KB). Per stage:
 // warp 1 brings A and B by TMA (KB rows x 128 features, two 64-feature boxes
-// each, 128-byte swizzle); when lambda != 1 the eight worker warps scale the
+// each, 128-byte swizzle; with d <= 64 only the first box is loaded (for d =
+// 32 its upper 32 features read as zeros) and the second stays zero, so the
+// MMA shape does not change); when lambda != 1 the eight worker warps scale the
 // rows of A by w_t in place (bf16, one thread per 128-byte row); warp 0 issues
 // KB/16 tcgen05.mma (M = N = 128 features, K = 16 tokens) accumulating M_c in
 // TMEM. Both operands are MN-major: the tiles arrive token-major with features
@@ -16,7 +18,7 @@
 // slow one. Two TMEM accumulators alternate between chunks; the workers read a
 // finished one (warp w: TMEM lanes 32*(w%4).., one column half) and store it by
 // TMA in 32 x 32 blocks staged in shared memory, while the next chunk
-// accumulates.
+// accumulates. Only the d x d block of each accumulator is stored.
 #include <algorithm>
 
 #include "kernels.h"
@@ -30,7 +32,7 @@ namespace tc_states_detail {
 
 using namespace sm100;
 
-constexpr int kD = 128;              // head dimension handled here
+constexpr int kD = 128;              // features per tile (d = 64 fills the first half)
 constexpr int kThreads = 320;        // warp 0: MMA, warp 1: TMA, warps 2-9: scaling and epilogue
 constexpr int kWorkers = 256;
 constexpr uint32_t kStageOutBytes = 32 * 128;  // per worker warp: a 32 x 32 fp32 block of the state
@@ -80,7 +82,7 @@ __device__ __forceinline__ Work work_of(int64_t n, int T, int H, int64_t item0) 
 __global__ void __launch_bounds__(kThreads, 1) chunk_states_tc(const __grid_constant__ CUtensorMap map_a,
                                                             const __grid_constant__ CUtensorMap map_b,
                                                             const __grid_constant__ CUtensorMap map_m,
-                                                            const float* decay, int H,
+                                                            const float* decay, int H, int d,
                                                             int C, int KB, int nslots, int kind, int T,
                                                             int64_t nitems, int64_t t_out, int slot_stride,
                                                             int slot_offset, int64_t item0) {
@@ -95,6 +97,16 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_states_tc(const __grid_cons
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int64_t my_items = nitems > blockIdx.x ? (nitems - 1 - blockIdx.x) / gridDim.x + 1 : 0;
   const int64_t nstream = my_items * nstages;
+  const int nbox = d > 64 ? 2 : 1;  // 64-feature boxes loaded per tile
+
+  if (nbox == 1) {
+    // the second box of every A and B tile stays zero for the whole kernel
+    for (int s2 = 0; s2 < 2 * nslots; ++s2) {
+      uint4* z = reinterpret_cast<uint4*>(tiles + (size_t)s2 * tile_bytes + tile_bytes / 2);
+      for (uint32_t q = threadIdx.x; q < tile_bytes / 32; q += kThreads) z[q] = make_uint4(0, 0, 0, 0);
+    }
+    fence_async_smem();
+  }
 
   if (tid == 0) {
     prefetch_tmap(&map_a);
@@ -138,11 +150,13 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_states_tc(const __grid_cons
         const int row = wk.c * C + (int)(g % nstages) * KB;
         uint8_t* a = tiles + (size_t)slot * 2 * tile_bytes;
         uint8_t* bb = a + tile_bytes;
-        mbar_arrive_expect_tx(&s->full[slot], 2 * tile_bytes);
+        mbar_arrive_expect_tx(&s->full[slot], nbox * tile_bytes);
         tma_load_4d_hint(a, &map_a, &s->full[slot], 0, wk.h, row, wk.b, stream_policy);
-        tma_load_4d_hint(a + tile_bytes / 2, &map_a, &s->full[slot], 64, wk.h, row, wk.b, stream_policy);
         tma_load_4d_hint(bb, &map_b, &s->full[slot], 0, wk.h, row, wk.b, stream_policy);
-        tma_load_4d_hint(bb + tile_bytes / 2, &map_b, &s->full[slot], 64, wk.h, row, wk.b, stream_policy);
+        if (nbox == 2) {
+          tma_load_4d_hint(a + tile_bytes / 2, &map_a, &s->full[slot], 64, wk.h, row, wk.b, stream_policy);
+          tma_load_4d_hint(bb + tile_bytes / 2, &map_b, &s->full[slot], 64, wk.h, row, wk.b, stream_policy);
+        }
       }
     }
   } else if (warp == 0) {
@@ -202,7 +216,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_states_tc(const __grid_cons
         // box (8 chunks of 16 bytes, chunk c of row r stored at position
         // c ^ (r & 7), so the eight rows of a quarter-warp hit different banks)
         uint8_t* a = tiles + (size_t)slot * 2 * tile_bytes;
-        for (int q = wt; q < 2 * KB; q += kWorkers) {
+        for (int q = wt; q < nbox * KB; q += kWorkers) {
           const int r = q % KB;
           const int t = k * KB + r;
           const float w = kind == 0 ? decay_pow(l2, (float)(C - 1 - t)) : decay_pow(l2, (float)(t + 1));
@@ -232,7 +246,9 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_states_tc(const __grid_cons
         }
         tc_fence_after();
         const int64_t oslot = (int64_t)wk.c * slot_stride + slot_offset;
-        const int y = (int)((((int64_t)wk.b * t_out + oslot) * H + wk.h) * kD + quad * 32);
+        const int y = (int)((((int64_t)wk.b * t_out + oslot) * H + wk.h) * d + quad * 32);
+        // this warp's 32 rows x 64 columns of the accumulator, if inside d x d
+        const bool mine = quad * 32 < d && colhalf * 64 < d;
         const uint32_t tbase = tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)acc * 128;
         uint32_t r0[32], r1[32];
         tmem_ld32(tbase + (2 * colhalf) * 32, r0);
@@ -241,7 +257,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_states_tc(const __grid_cons
         tc_fence_before();
         mbar_arrive(&s->acc_empty[acc]);
 #pragma unroll
-        for (int cb = 0; cb < 2; ++cb) {
+        for (int cb = 0; cb < 2 && mine && (2 * colhalf + cb) * 32 < d; ++cb) {
           // the staging block is free once this warp's previous store has read it
           if (lane == 0) tma_store_wait_read0();
           __syncwarp();
@@ -277,7 +293,7 @@ inline int stage_rows(int C) {
 }  // namespace tc_states_detail
 
 bool tc_states_ok(int dtype, int d, int64_t C) {
-  return dtype == LASP_BF16 && d == tc_states_detail::kD && C % 16 == 0;
+  return dtype == LASP_BF16 && (d == 32 || d == 64 || d == tc_states_detail::kD) && C % 16 == 0;
 }
 
 cudaError_t tc_chunk_states_slots(const void* a, const void* bm, const float* decay, float* M, int B, int H,
@@ -300,7 +316,7 @@ cudaError_t tc_chunk_states_slots(const void* a, const void* bm, const float* de
   const int64_t nitems = nbh * T;
   if (nitems == 0) return cudaSuccess;
   const unsigned grid = (unsigned)std::min<int64_t>(nitems, sms);
-  chunk_states_tc<<<grid, kThreads, smem, st>>>(ma, mb, mm, decay, H, C, KB, nslots, kind, T, nitems, t_out,
+  chunk_states_tc<<<grid, kThreads, smem, st>>>(ma, mb, mm, decay, H, d, C, KB, nslots, kind, T, nitems, t_out,
                                                slot_stride, slot_offset, bh0 * T);
   return cudaGetLastError();
 }

@@ -37,8 +37,13 @@ SMALL = [
     (1, 4, 320, 128, 64, True, True),    # N not a multiple of 128
     (3, 5, 256, 128, 32, True, False),   # odd B and H
     (1, 2, 192, 128, 16, True, True),
-    (2, 2, 224, 64, 32, True, True),     # d = 64
-    (1, 3, 96, 32, 16, True, True),      # d = 32
+    (2, 2, 224, 64, 32, True, True),     # d = 64 (per-chunk tensor-core kernels, ragged tile)
+    (2, 3, 640, 64, 128, True, True),    # d = 64, several tiles
+    (1, 2, 512, 64, 64, True, False),    # d = 64, two chunks per tile
+    (1, 2, 512, 64, 256, True, True),    # d = 64, chunks of two tiles (tensor-core states only)
+    (1, 3, 96, 32, 16, True, True),      # d = 32 (per-chunk tensor-core kernels, ragged tile)
+    (2, 2, 384, 32, 64, True, True),     # d = 32, several tiles
+    (1, 3, 256, 32, 128, True, False),
     (1, 2, 96, 64, 24, True, True),      # C not a multiple of 16
     (1, 2, 128, 128, 128, True, True),   # a single chunk
     (2, 2, 64, 64, 1, False, True),      # C = 1: pure inter-chunk

@@ -44,6 +44,23 @@ def test_bf16_c64_with_a_ragged_tile_runs_the_per_chunk_tensor_core_kernels():
                      "chunk_states_tc", "state_scan", "chunk_bwd_tc"], names
 
 
+@pytest.mark.parametrize("d", [64, 32])
+def test_bf16_small_heads_run_the_per_chunk_tensor_core_kernels(d):
+    """d = 64 and 32: the tiles keep 128 features, zero past d."""
+    for N, C in ((512, 128), (512, 64), (224, 32)):
+        inp = lasp_inputs.make_inputs(1, N, 2, d, seed=205 + C + d, bf16=True, decayed=True)
+        names = _traced_names(inp, C)
+        assert names == ["chunk_states_tc", "state_scan", "chunk_out_tc",
+                         "chunk_states_tc", "state_scan", "chunk_bwd_tc"], (d, N, C, names)
+
+
+def test_bf16_chunks_off_the_16_grid_run_on_cuda_cores():
+    inp = lasp_inputs.make_inputs(1, 96, 2, 64, seed=206, bf16=True, decayed=True)
+    names = _traced_names(inp, 24)
+    assert names == ["chunk_states_simt", "state_scan", "chunk_out_simt",
+                     "chunk_states_simt", "state_scan", "chunk_bwd_simt"], names
+
+
 def test_bf16_c256_runs_the_segment_walks():
     """Chunks of two tiles walk both ways: the forward leaves both tiles'
     entering states in the two halves of the chunk's cache slot."""

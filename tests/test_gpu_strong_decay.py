@@ -29,6 +29,8 @@ PATHS = {
     "walks_C128": (1, 2048, 128, 128, True),   # segment walks, two 1024-token segments
     "walks_C64": (2, 1024, 128, 64, True),     # walks with chunks that divide the tile
     "per_chunk_tc": (1, 320, 128, 64, True),   # ragged tile: per-chunk tensor-core kernels
+    "per_chunk_tc_d64": (1, 384, 64, 128, True),  # d = 64 on the per-chunk tensor-core kernels
+    "per_chunk_tc_d32": (1, 256, 32, 64, True),   # d = 32 on the per-chunk tensor-core kernels
     "simt_f32_d64": (1, 256, 64, 64, False),   # CUDA cores, fp32
     "bf16_C256": (1, 1024, 128, 256, True),    # walks with chunks of two tiles
     "bf16_C512": (1, 1024, 128, 512, True),    # forward walk, CUDA-core backward
@@ -84,7 +86,8 @@ def test_strong_decay_without_entering_states(lam_name):
 
 
 @pytest.mark.parametrize("lam_name", sorted(LAMBDAS))
-@pytest.mark.parametrize("bf16,d,C", [(True, 128, 128), (True, 128, 64), (False, 64, 32)])
+@pytest.mark.parametrize("bf16,d,C", [(True, 128, 128), (True, 128, 64), (True, 64, 64), (True, 32, 128),
+                                      (False, 64, 32)])
 def test_state_entry_points_at_strong_decay(lam_name, bf16, d, C):
     """lasp_chunk_states, lasp_chunk_dstates and lasp_state_prefix (with an
     entering state and the total) on their own, against the oracle's

@@ -24,6 +24,8 @@ CASES = [
     (15, 1, 2, 256, 64, 64, False, "workload"),         # per-chunk CUDA-core branch, fp32
     (16, 1, 4, 1024, 128, 128, True, [1.0, 0.99, 0.5, 1e-3]),  # strong decays on the walk
     (17, 1, 2, 1024, 128, 256, True, "workload"),       # walk branch with chunks of two tiles
+    (18, 2, 3, 640, 64, 128, True, "workload"),         # per-chunk tensor-core branch, d = 64
+    (19, 1, 2, 384, 32, 64, True, [0.5, 1e-3]),         # per-chunk tensor-core branch, d = 32, strong decays
 ]
 
 
