@@ -125,12 +125,12 @@ def flops_per_step(tokens_heads: int, d: int, C: int) -> float:
 MEASURED_TRAFFIC = {
     # DRAM bytes per launch at the workload's full size: twice the ncu capture of
     # the 32768-token case of the same workload (traffic grows with the tokens)
-    "bwd_walk_tc": (["k_tc_bwd_walk.cu", "sm100.cuh", "lasp_common.cuh", "tma_host.h"], "adce30b1fce33512",
-                    2 * (723739136 + 364952576)),
-    "fwd_walk_tc": (["k_tc_fwd_walk.cu", "sm100.cuh", "lasp_common.cuh", "tma_host.h"], "bcb650137196739b",
-                    2 * (437725440 + 226706432)),
-    "segment_states_tc": (["k_tc_states.cu", "sm100.cuh", "lasp_common.cuh", "tma_host.h"], "bfe2712019c7da94",
-                          2 * (268476416 + 5191168)),
+    "bwd_walk_tc": (["k_tc_bwd_walk.cu", "sm100.cuh", "lasp_common.cuh", "tma_host.h"], "a8458a2dda72b0b5",
+                    2 * (723464448 + 365351168)),
+    "fwd_walk_tc": (["k_tc_fwd_walk.cu", "sm100.cuh", "lasp_common.cuh", "tma_host.h"], "0ad0edd4699b890d",
+                    2 * (437797120 + 226962944)),
+    "segment_states_tc": (["k_tc_states.cu", "sm100.cuh", "lasp_common.cuh", "tma_host.h"], "48a5dd38bfe5a0ce",
+                          2 * (268479488 + 8521472)),
     # the gated form (bench.py --gated): four times the capture of the 16384-token case
     "gla_bwd_tc": (["k_tc_gla.cu", "sm100.cuh", "lasp_common.cuh", "tma_host.h"], "ec39fc0de472db0b",
                    4 * (605854720 + 291032832)),
