@@ -70,8 +70,10 @@ def algorithmic_bytes(name: str, tokens_heads: int, d: int, C: int, G: int, elem
       gla_out_tc:   the walk through each segment: read q, k, v, the gates
                     and the segment's P (s/G), write o and the bf16 tile of
                     diag(e^r) P per 128-token tile     = 4de + 4d + s/G + s/256
-      gla_bwd_tc:   read q, k, v, dO, the gates, that bf16 tile and R,
-                    write dq, dk, dv and the gate gradient = 7de + 8d + s/256 + s/128
+      gla_bwd_tc:   the walk back through each segment: read q, k, v, dO, the
+                    gates, that bf16 tile and the segment's R (s/G; the states
+                    it forms for the segment's other tiles stay in L2), write
+                    dq, dk, dv and the gate gradient = 7de + 8d + s/256 + s/G
     """
     s = 4 * d * d
     de = d * elem
@@ -89,7 +91,7 @@ def algorithmic_bytes(name: str, tokens_heads: int, d: int, C: int, G: int, elem
         "gla_scan": 2 * s / C + 4 * d / C,
         "gla_segment_states_tc": 2 * de + 4 * d + s / G, "gla_segment_scan": 2 * s / G + 4 * d / G,
         "gla_out_tc": 4 * de + 4 * d + s / G + s / 256, "gla_out_simt": 4 * de + 4 * d + s / C,
-        "gla_bwd_tc": 7 * de + 8 * d + s / 256 + s / 128, "gla_bwd_simt": 7 * de + 8 * d + 2 * s / C,
+        "gla_bwd_tc": 7 * de + 8 * d + s / 256 + s / G, "gla_bwd_simt": 7 * de + 8 * d + 2 * s / C,
         # the exact CUDA-core sequence a tensor-core gated call also launches;
         # it returns at once unless a tile's gates leave the factorized range
         "gla_states_exact": 0.0, "gla_scan_exact": 0.0, "gla_out_exact": 0.0, "gla_bwd_exact": 0.0,
@@ -109,7 +111,7 @@ def cache_bytes(name: str, tokens_heads: int, d: int, C: int, G: int) -> float:
         "fwd_walk_tc": (s / G + s / 256) if C <= 128 else s / C,
         "bwd_walk_tc": s / 256 + s / G,
         "gla_out_tc": s / G + s / 256,
-        "gla_bwd_tc": s / 256 + s / 128,
+        "gla_bwd_tc": s / 256 + s / G,
     }.get(name, 0.0)
     return per * tokens_heads
 
@@ -132,8 +134,8 @@ MEASURED_TRAFFIC = {
     "segment_states_tc": (["k_tc_states.cu", "sm100.cuh", "lasp_common.cuh", "tma_host.h"], "48a5dd38bfe5a0ce",
                           2 * (268479488 + 8521472)),
     # the gated form (bench.py --gated): four times the capture of the 16384-token case
-    "gla_bwd_tc": (["k_tc_gla.cu", "sm100.cuh", "lasp_common.cuh", "tma_host.h"], "ec39fc0de472db0b",
-                   4 * (605854720 + 291032832)),
+    "gla_bwd_tc": (["k_tc_gla.cu", "sm100.cuh", "lasp_common.cuh", "tma_host.h"], "35948c182ff4f718",
+                   4 * (491065088 + 319227392)),
 }
 
 

@@ -61,6 +61,10 @@ constexpr float kMaxSpan = 80.f;  // largest |b_t - r| (natural log) the factori
 constexpr float kSpanCheck = kMaxSpan - 1.f;
 constexpr uint32_t kBarAll = 1;   // named barrier over all 256 threads
 
+// Orders this thread's generic-proxy writes to global memory before later
+// async-proxy (bulk copy) reads of them.
+__device__ __forceinline__ void fence_async_global() { asm volatile("fence.proxy.async.global;" ::: "memory"); }
+
 
 // Multiplies the 64 bf16 entries of row `row`, columns half*64.., of a tile by
 // exp2(sgn * x[u]) (x in log2 units), in place.
@@ -694,16 +698,30 @@ cleanup:
 
 // ---------------------------------------------------------------- gradients
 struct SmemBwd {
-  uint64_t gload, load, ldr, mma1a, mma1b, mma2, mma3;
+  uint64_t gload, load, ldr, mma1a, mma1b, mma2, mma3, mmar;
   uint32_t tmem_base;
   int abort;
-  float dAd[kTile];  // do_t . v_t, the diagonal of dO V^T
-  float bnd[kD];     // e^{b_end[i]} <R_c[i], P_c[i]>
+  alignas(16) float dAd[kTile];  // do_t . v_t, the diagonal of dO V^T
+  alignas(16) float bnd[kD];     // e^{b_end[i]} <R_c[i], P_c[i]>, the sum over the first half of the columns
+  alignas(16) float bnd2[kD];    // ... and over the second half (both read as float4)
 };
 
-// One persistent CTA per SM, taking 128-token tiles in launch order (tile w,
-// w + grid, ...); the barriers complete once per tile, so their parity flips
-// from tile to tile. Shared memory: Q^, K^, V, dO (then, in pairs,
+// One persistent CTA per SM, taking segments of S 128-token tiles in launch
+// order (segment w, w + grid, ...) and walking each from its last tile to its
+// first. The state R_c entering a tile from the right comes, for a segment's
+// last tile, from the scan over segments (the workspace slot of that tile's
+// last chunk); every other tile's is formed on the way, by the tile after it
+// (LASP Appendix A.4: the gated form of the gradient-state recurrence):
+//   R_{c-1} = diag(e^{b_end}) R_c + diag(e^{r}) Q^^T dO     (Q^ = q . e^{b - r})
+// with Q^^T dO an extra MMA of phase 2 into T0 (idle between epilogue 1 and
+// phase 3), combined in fp32 at the start of epilogue 2 with R_c read back
+// from L2, and written to a scratch slot of the segment (the workspace slot
+// of its first chunk), where the next tile's bulk load of R finds it. The
+// scratch is lane-major (float4 group g of state row m at float4 g * 128 + m),
+// so that the threads of a warp, which own consecutive rows, read and write
+// one 512-byte run per access; the scan's slot is row-major. Most
+// barriers complete once per tile, so their parity flips from tile to tile;
+// mmar only on tiles that form a state. Shared memory: Q^, K^, V, dO (then, in pairs,
 // the fp32 tiles of dB and k . dk^inter for the log-gate gradient's column
 // sums), X (P', loaded as the output kernel cached it, then R'), and the pair
 // sA / sB (the gate tile during the walk; then dA . strict and A . causal;
@@ -715,8 +733,8 @@ __global__ void __launch_bounds__(kThreads, 1) gla_bwd_tc(
     const __grid_constant__ CUtensorMap map_v, const __grid_constant__ CUtensorMap map_do,
     const __grid_constant__ CUtensorMap map_dk, const __grid_constant__ CUtensorMap map_dv,
     const __grid_constant__ CUtensorMap map_g, const __grid_constant__ CUtensorMap map_dg,
-    const float* __restrict__ P, const float* __restrict__ R, __nv_bfloat16* __restrict__ dq, int H, int64_t N,
-    int64_t t_slots, int stride, int ntx, int64_t ntiles, RunIf run_if) {
+    const float* __restrict__ P, float* __restrict__ R, __nv_bfloat16* __restrict__ dq, int H, int64_t N,
+    int64_t t_slots, int stride, int ntx, int S, int64_t nitems, RunIf run_if) {
   if (!runs(run_if)) return;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
@@ -734,14 +752,26 @@ __global__ void __launch_bounds__(kThreads, 1) gla_bwd_tc(
   float* sdend = s->bnd;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int t = (warp & 3) * 32 + lane, half = warp >> 2;
-  // tile w: 128 tokens c * 128.. of head h of sequence b, in launch order
-  auto tile_of = [&](int64_t w, int& c, int& h, int& b) {
-    c = (int)(w % ntx);
-    h = (int)((w / ntx) % H);
-    b = (int)(w / ((int64_t)ntx * H));
+  // this CTA's k-th tile: tile j = S - 1 - k % S (128 tokens c * 128.., c =
+  // seg * S + j) of segment item blockIdx.x + (k / S) * grid (segment seg of
+  // head h of sequence b)
+  const int nsg = ntx / S;
+  const int64_t my_items = nitems > (int64_t)blockIdx.x ? (nitems - 1 - blockIdx.x) / gridDim.x + 1 : 0;
+  const int64_t my_tiles = my_items * S;
+  auto tile_of = [&](int64_t k, int& c, int& h, int& b, int& j) {
+    const int64_t w = blockIdx.x + (k / S) * (int64_t)gridDim.x;
+    j = S - 1 - (int)(k % S);
+    c = (int)(w % nsg) * S + j;
+    h = (int)((w / nsg) % H);
+    b = (int)(w / ((int64_t)nsg * H));
   };
   // P of a tile's first chunk (R of its last is stride - 1 slots on)
   auto pslot_of = [&](int c, int h, int b) { return ((int64_t)b * t_slots + (int64_t)c * stride) * H + h; };
+  // the slot R_c of tile c is read from: the scan's (tile's last chunk) for a
+  // segment's last tile, the scratch (segment's first chunk) for the others
+  auto rslot_of = [&](int c, int h, int b, int j) {
+    return j == S - 1 ? pslot_of(c, h, b) + (int64_t)(stride - 1) * H : pslot_of(c - j, h, b);
+  };
   auto load_tokens = [&](uint8_t* dst, const CUtensorMap* map, int h, int row, int b) {
     tma_load_4d(dst, map, &s->load, 0, h, row, b);
     tma_load_4d(dst + kBox, map, &s->load, 64, h, row, b);
@@ -762,6 +792,7 @@ __global__ void __launch_bounds__(kThreads, 1) gla_bwd_tc(
     mbar_init(&s->mma1b, 1);
     mbar_init(&s->mma2, 1);
     mbar_init(&s->mma3, 1);
+    mbar_init(&s->mmar, 1);
     s->abort = 0;
     fence_mbar_init();
   }
@@ -775,14 +806,14 @@ __global__ void __launch_bounds__(kThreads, 1) gla_bwd_tc(
   const uint32_t tmem = s->tmem_base;
   const uint32_t lane_base = tmem + ((uint32_t)((warp & 3) * 32) << 16);
   const uint32_t T0 = 0, T1 = 128, T2 = 256, T3 = 384;
-  if (tid == 0 && (int64_t)blockIdx.x < ntiles) {
+  if (tid == 0 && my_tiles > 0) {
     // the first tile's loads; a later tile's are issued during the tile before
-    int c, h, b;
-    tile_of(blockIdx.x, c, h, b);
+    int c, h, b, j;
+    tile_of(0, c, h, b, j);
     const int64_t ps = pslot_of(c, h, b);
     load_gate_tile(bt, &map_g, &s->gload, h, c * kTile, b);
-    // R is read with plain loads later: into L2 now
-    bulk_prefetch_l2(R + (ps + (int64_t)(stride - 1) * H) * kD * kD, kD * kD * 4);
+    // R is read by a bulk load later: into L2 now
+    bulk_prefetch_l2(R + rslot_of(c, h, b, j) * kD * kD, kD * kD * 4);
     mbar_arrive_expect_tx(&s->load, 5 * kTileBytes);
     load_tokens(sQ, &map_q, h, c * kTile, b);
     load_tokens(sK, &map_k, h, c * kTile, b);
@@ -791,18 +822,21 @@ __global__ void __launch_bounds__(kThreads, 1) gla_bwd_tc(
     load_pprime(ps);
   }
   uint32_t ph = 0;       // parity of every barrier's phase for this CTA's current tile
+  uint32_t rph = 0;      // parity of mmar's next phase
   bool r_ahead = false;  // thread 0: R's load into sA/sB is in flight
-  for (int64_t w = blockIdx.x; w < ntiles; w += gridDim.x, ph ^= 1u) {
-  int c, h, b;
-  tile_of(w, c, h, b);
+  for (int64_t k = 0; k < my_tiles; ++k, ph ^= 1u) {
+  int c, h, b, j;
+  tile_of(k, c, h, b, j);
   const int64_t row0 = (int64_t)c * kTile;
-  const int64_t pslot = pslot_of(c, h, b);
-  const int64_t rslot = pslot + (int64_t)(stride - 1) * H;
+  const int64_t rslot = rslot_of(c, h, b, j);
   const int64_t tok = (((int64_t)b * N + row0 + t) * H + h) * kD;  // row t of every token tensor
-  const int64_t wn = w + gridDim.x;  // this CTA's next tile
+  const bool has_next = k + 1 < my_tiles;  // this CTA's next tile
+  const bool form = j > 0;  // this tile forms R_{c-1} for the tile before it
   // ---- phase 0: gates, Q^, K^, log2 E -> T3, P' -> X
   float x[64];
   gate_rows(bt, &s->gload, ph, &s->abort, SITE_BWD_TMA, sr, sdend, tid, t, half, x);
+  // e^{r}, e^{b_end - r} and e^{b_end} of state row t (feature t)
+  const float er = exp2f(sr[t] * kLog2e), wt = exp2f(sdend[t] * kLog2e), eb = er * wt;
   named_sync(kBarAll, kThreads);  // every row of the gate tile has been read
   if (tid == 0) {
     // R_c (fp32) into the gate tile's space while the token tiles arrive
@@ -810,9 +844,6 @@ __global__ void __launch_bounds__(kThreads, 1) gla_bwd_tc(
     bulk_load(bt, R + rslot * kD * kD, kD * kD * 4, &s->ldr);
     r_ahead = true;
   }
-  float we[16];  // e^{b_end_m - r_m} of this thread's state rows m = warp + 8u
-#pragma unroll
-  for (int u = 0; u < 16; ++u) we[u] = exp2f(sdend[warp + 8 * u] * kLog2e);
   if (!mbar_wait(&s->load, ph, SITE_BWD_TMA)) s->abort = 1;
   scale_row_half(sQ, t, half, x, 1.f);   // Q^ = q . E
   scale_row_half(sK, t, half, x, -1.f);  // K^ = k / E
@@ -846,34 +877,46 @@ __global__ void __launch_bounds__(kThreads, 1) gla_bwd_tc(
       for (int kk = 0; kk < kD / 16; ++kk) mma_bf16(tmem + T2, kmaj(aD, kk), kmaj(aX, kk), id_kk, kk != 0);
       mma_commit(&s->mma1b);
     }
-    // while the MMAs run: R rows (fp32, from sA/sB) into registers, and
-    // <R'_m, P'_m> = e^{b_end_m} <R_m, P_m> into bnd, with the rows of P' read
-    // in X (bf16)
+    // while the MMAs run: row t of R (fp32, from sA/sB; this thread's half of
+    // the columns) into registers, and that half of <R'_t, P'_t> = e^{b_end_t}
+    // <R_t, P_t> into bnd / bnd2, with row t of P' read in X (bf16)
     {
       const bool rok = mbar_wait(&s->ldr, ph, SITE_BWD_TMA);
       if (!rok) s->abort = 1;
       if (tid == 0 && rok) r_ahead = false;  // else cleanup waits for it once more
     }
+    // R_c, row t, columns half * 64.. (float4 groups g = half * 16 + u):
+    // row-major from the scan's slot, lane-major from the scratch
     float4 rreg[16];
     {
+      const bool rlm = j != S - 1;
       const float4* R4 = reinterpret_cast<const float4*>(bt);
 #pragma unroll
-      for (int u = 0; u < 16; ++u) rreg[u] = R4[(warp + 8 * u) * (kD / 4) + lane];
+      for (int u = 0; u < 16; ++u) {
+        const int g = half * 16 + u;
+        rreg[u] = R4[rlm ? g * kD + t : t * (kD / 4) + g];
+      }
+      if (form && !rlm) {
+        // a segment's last tile: R_c into the scratch, lane-major, where this
+        // tile's own forming of R_{c-1} reads it back in one-run accesses
+        float4* rs = reinterpret_cast<float4*>(R + pslot_of(c - j, h, b) * kD * kD);
+#pragma unroll
+        for (int u = 0; u < 16; ++u) rs[(half * 16 + u) * kD + t] = rreg[u];
+      }
     }
     named_sync(kBarAll, kThreads);  // every row of R has been read: the masks may overwrite sA/sB
     {
-      const int col = lane * 4;
+      // e^{b_end - r} <R_t, P'_t> over this thread's half of the columns (P' row t in X, bf16)
+      float dot = 0.f;
 #pragma unroll
-      for (int u = 0; u < 16; ++u) {
-        const int m = warp + 8 * u;
-        const uint2 pw =
-            *reinterpret_cast<const uint2*>(sX + (col >> 6) * kBox + sw128_offset(m, (col & 63) >> 3) + (col & 7) * 2);
-        const float2 p0 = unpack_bf16(pw.x), p1 = unpack_bf16(pw.y);
-        float dot = p0.x * rreg[u].x + p0.y * rreg[u].y + p1.x * rreg[u].z + p1.y * rreg[u].w;
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
-        if (lane == 0) s->bnd[m] = dot * we[u];
+      for (int q8 = 0; q8 < 8; ++q8) {
+        const uint4 pw = *tile16(sX, t, half * 64 + q8 * 8);
+        const float2 p0 = unpack_bf16(pw.x), p1 = unpack_bf16(pw.y), p2 = unpack_bf16(pw.z), p3 = unpack_bf16(pw.w);
+        const float4 a = rreg[2 * q8], b2 = rreg[2 * q8 + 1];
+        dot += p0.x * a.x + p0.y * a.y + p1.x * a.z + p1.y * a.w + p2.x * b2.x + p2.y * b2.y + p3.x * b2.z +
+               p3.y * b2.w;
       }
+      (half ? s->bnd2 : s->bnd)[t] = dot * wt;
     }
     // ---- epilogue 1: dA . strict -> sA, A . causal -> sB, the diagonal of dA
     if (mbar_wait(&s->mma1a, ph, SITE_BWD_MMA)) {
@@ -909,7 +952,12 @@ __global__ void __launch_bounds__(kThreads, 1) gla_bwd_tc(
     // X is free once dO P'^T has read P': R' = diag(e^{b_end - r}) R_c replaces it
     if (mbar_wait(&s->mma1b, ph, SITE_BWD_MMA)) {
 #pragma unroll
-      for (int u = 0; u < 16; ++u) put_state_row(sX, warp + 8 * u, lane, rreg[u], we[u]);
+      for (int q8 = 0; q8 < 8; ++q8) {
+        const float4 a = rreg[2 * q8], b2 = rreg[2 * q8 + 1];
+        st_tile16(sX, t, half * 64 + q8 * 8,
+                  make_uint4(pack_bf16(a.x * wt, a.y * wt), pack_bf16(a.z * wt, a.w * wt),
+                             pack_bf16(b2.x * wt, b2.y * wt), pack_bf16(b2.z * wt, b2.w * wt)));
+      }
     } else {
       s->abort = 1;
     }
@@ -917,11 +965,15 @@ __global__ void __launch_bounds__(kThreads, 1) gla_bwd_tc(
     tc_fence_before();
     __syncthreads();
     if (s->abort) goto cleanup;
-    // ---- phase 2: T2 += (dA . strict) K^
+    // ---- phase 2: T2 += (dA . strict) K^ | T0 = Q^^T dO (when this tile forms R_{c-1})
     if (tid == 0) {
       tc_fence_after();
       for (int kk = 0; kk < kTile / 16; ++kk) mma_bf16(tmem + T2, kmaj(aA, kk), mnmaj(aK, kk), id_kn, 1);
       mma_commit(&s->mma2);
+      if (form) {
+        for (int kk = 0; kk < kTile / 16; ++kk) mma_bf16(tmem + T0, mnmaj(aQ, kk), mnmaj(aD, kk), id_nn, kk != 0);
+        mma_commit(&s->mmar);
+      }
     }
     // ---- epilogue 2: dq' = E . T2; dq = dq' + (do_t . v_t) k_t = E . (T2 + (do_t . v_t) K^_t);
     // q . dq' = Q^ . T2 -> T2
@@ -977,13 +1029,56 @@ __global__ void __launch_bounds__(kThreads, 1) gla_bwd_tc(
     tc_fence_before();
     __syncthreads();
     if (s->abort) goto cleanup;
-    // ---- phase 3: T0 = (dA . strict)^T Q^, T1 = (A . causal)^T dO + K^ R', T3 = V R'^T
+    // ---- phase 3: T1 = (A . causal)^T dO + K^ R', T3 = V R'^T while the
+    // threads form R_{c-1} from T0, then T0 = (dA . strict)^T Q^
     if (tid == 0) {
       tc_fence_after();
-      for (int kk = 0; kk < kTile / 16; ++kk) mma_bf16(tmem + T0, mnmaj(aA, kk), mnmaj(aQ, kk), id_nn, kk != 0);
       for (int kk = 0; kk < kTile / 16; ++kk) mma_bf16(tmem + T1, mnmaj(aB, kk), mnmaj(aD, kk), id_nn, kk != 0);
       for (int kk = 0; kk < kD / 16; ++kk) mma_bf16(tmem + T1, kmaj(aK, kk), mnmaj(aX, kk), id_kn, 1);
       for (int kk = 0; kk < kD / 16; ++kk) mma_bf16(tmem + T3, kmaj(aV, kk), kmaj(aX, kk), id_kk, kk != 0);
+    }
+    // ---- R_{c-1} = e^{b_end} R_c + e^{r} T0 (row t, columns half * 64..), R_c
+    // read back from the scratch in L2 (this thread's elements only, so the
+    // slot is both source and destination; float4 group g of row t at g * 128 + t)
+    if (form) {
+      float4* rn = reinterpret_cast<float4*>(R + pslot_of(c - j, h, b) * kD * kD);
+      float4 rv[8];  // 32 columns of R_c at a time, the next chunk's in flight under this one's math
+#pragma unroll
+      for (int q4 = 0; q4 < 8; ++q4) rv[q4] = rn[(half * 16 + q4) * kD + t];
+      if (mbar_wait(&s->mmar, rph, SITE_BWD_MMA)) {
+        tc_fence_after();
+#pragma unroll 1
+        for (int c2 = 0; c2 < 2; ++c2) {
+          uint32_t a[32];
+          tmem_ld32(lane_base + T0 + half * 64 + c2 * 32, a);
+          tmem_ld_wait();
+          float4 o4[8];
+#pragma unroll
+          for (int q4 = 0; q4 < 8; ++q4)
+            o4[q4] = make_float4(fmaf(eb, rv[q4].x, er * __uint_as_float(a[4 * q4])),
+                                 fmaf(eb, rv[q4].y, er * __uint_as_float(a[4 * q4 + 1])),
+                                 fmaf(eb, rv[q4].z, er * __uint_as_float(a[4 * q4 + 2])),
+                                 fmaf(eb, rv[q4].w, er * __uint_as_float(a[4 * q4 + 3])));
+          if (c2 == 0) {
+#pragma unroll
+            for (int q4 = 0; q4 < 8; ++q4) rv[q4] = rn[(half * 16 + 8 + q4) * kD + t];
+          }
+#pragma unroll
+          for (int q4 = 0; q4 < 8; ++q4) rn[(half * 16 + c2 * 8 + q4) * kD + t] = o4[q4];
+        }
+        fence_async_global();  // the next tile's bulk load of R reads these stores
+      } else {
+        s->abort = 1;
+      }
+      rph ^= 1u;
+    }
+    if (form) {
+      tc_fence_before();
+      named_sync(kBarAll, kThreads);  // every thread has read its rows of T0
+    }
+    if (tid == 0) {
+      tc_fence_after();
+      for (int kk = 0; kk < kTile / 16; ++kk) mma_bf16(tmem + T0, mnmaj(aA, kk), mnmaj(aQ, kk), id_nn, kk != 0);
       mma_commit(&s->mma3);
     }
     // ---- epilogue 3: dk = E^-1 . (T0 + T3 + (do_s . v_s) Q^_s) -> sA, dv = T1 -> sB;
@@ -1106,15 +1201,14 @@ __global__ void __launch_bounds__(kThreads, 1) gla_bwd_tc(
       }
     }
     __syncthreads();
-    if (tid == 0 && wn < ntiles && !s->abort) {
+    if (tid == 0 && has_next && !s->abort) {
       // the dK and dV stores have read the gate tile's space: the next tile's
-      // gates go there, its P and R into L2
+      // gates go there; a segment's entering R into L2 (a formed one is there)
       tma_store_wait_read0();
-      int cn, hn, bn;
-      tile_of(wn, cn, hn, bn);
-      const int64_t ps = pslot_of(cn, hn, bn);
+      int cn, hn, bn, jn;
+      tile_of(k + 1, cn, hn, bn, jn);
       load_gate_tile(bt, &map_g, &s->gload, hn, cn * kTile, bn);
-      bulk_prefetch_l2(R + (ps + (int64_t)(stride - 1) * H) * kD * kD, kD * kD * 4);
+      if (jn == S - 1) bulk_prefetch_l2(R + rslot_of(cn, hn, bn, jn) * kD * kD, kD * kD * 4);
     }
     // dg into the dB tile (the gate map's layout), stored by TMA below
 #pragma unroll
@@ -1125,8 +1219,10 @@ __global__ void __launch_bounds__(kThreads, 1) gla_bwd_tc(
         float4* pa = reinterpret_cast<float4*>(fB + gate_slot(t, col0 + 4 * q4));
         const float4 a = *pa;
         const float4 e = *reinterpret_cast<const float4*>(fK + gate_slot(t, col0 + 4 * q4));
-        const float* bn = s->bnd + col0 + 4 * q4;
-        *pa = make_float4(a.x + e.x + bn[0], a.y + e.y + bn[1], a.z + e.z + bn[2], a.w + e.w + bn[3]);
+        const float4 bn = *reinterpret_cast<const float4*>(s->bnd + col0 + 4 * q4);
+        const float4 bn2 = *reinterpret_cast<const float4*>(s->bnd2 + col0 + 4 * q4);
+        *pa = make_float4(a.x + e.x + (bn.x + bn2.x), a.y + e.y + (bn.y + bn2.y), a.z + e.z + (bn.z + bn2.z),
+                          a.w + e.w + (bn.w + bn2.w));
       }
     }
     fence_async_smem();
@@ -1138,9 +1234,9 @@ __global__ void __launch_bounds__(kThreads, 1) gla_bwd_tc(
         for (int cb = 0; cb < 4; ++cb) tma_store_4d(&map_dg, fB + cb * (kTile * 32), cb * 32, h, (int)row0, b);
         tma_store_commit();
       }
-      const bool next = wn < ntiles && !stop;
-      int cn = 0, hn = 0, bn = 0;
-      if (next) tile_of(wn, cn, hn, bn);
+      const bool next = has_next && !stop;
+      int cn = 0, hn = 0, bn = 0, jn = 0;
+      if (next) tile_of(k + 1, cn, hn, bn, jn);
       if (next) {
         // X (R', read by MMA 3) is free too
         mbar_arrive_expect_tx(&s->load, 5 * kTileBytes);
@@ -1216,8 +1312,8 @@ cudaError_t tc_gla_chunk_out(const void* q, const void* k, const void* v, const 
 }
 
 cudaError_t tc_gla_chunk_bwd(const void* q, const void* k, const void* v, const void* dout, const float* g,
-                             const float* P, const float* Rs, void* dq, void* dk, void* dv, float* dg, int B, int H,
-                             int64_t N, int64_t t_slots, int stride, cudaStream_t st, RunIf run) {
+                             const float* P, float* Rs, void* dq, void* dk, void* dv, float* dg, int B, int H,
+                             int64_t N, int64_t t_slots, int stride, int tiles, cudaStream_t st, RunIf run) {
   using namespace tc_gla_detail;
   CUtensorMap mq, mk, mv, mdo, mdk, mdv, mg, mdg;
   if (!make_token_map(&mq, q, B, H, N, kD, kTile) || !make_token_map(&mk, k, B, H, N, kD, kTile) ||
@@ -1232,12 +1328,14 @@ cudaError_t tc_gla_chunk_bwd(const void* q, const void* k, const void* v, const 
   if ((e = cudaGetDevice(&dev)) != cudaSuccess ||
       (e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
     return e;
-  // one persistent CTA per SM (the kernel holds all of TMEM and most of shared memory)
+  // one persistent CTA per SM (the kernel holds all of TMEM and most of shared
+  // memory), taking segments of `tiles` 128-token tiles
   const int ntx = (int)(N / kTile);
-  const int64_t ntiles = (int64_t)B * H * ntx;
-  const unsigned grid = (unsigned)std::min<int64_t>(ntiles, sms);
+  if (tiles < 1 || ntx % tiles != 0) return cudaErrorInvalidValue;
+  const int64_t nitems = (int64_t)B * H * (ntx / tiles);
+  const unsigned grid = (unsigned)std::min<int64_t>(nitems, sms);
   gla_bwd_tc<<<grid, kThreads, smem, st>>>(mq, mk, mv, mdo, mdk, mdv, mg, mdg, P, Rs, (__nv_bfloat16*)dq, H, N, t_slots,
-                                            stride, ntx, ntiles, run);
+                                            stride, ntx, tiles, nitems, run);
   return cudaGetLastError();
 }
 

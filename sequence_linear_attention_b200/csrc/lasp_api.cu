@@ -40,8 +40,8 @@ enum KernelId : int {
   K_GLA_OUT_TC = 20,     // gated form on the tensor cores: output
   K_GLA_BWD_TC = 21,     // gated form on the tensor cores: gradients
   K_STATE_TOTAL = 22,    // decayed total of a sequence's states (the LASP-2 shard state)
-  K_GLA_SEG_STATES = 23,  // gated form on the tensor cores: segment states (forward)
-  K_GLA_SEG_SCAN = 24,    // gated form: prefix over segments
+  K_GLA_SEG_STATES = 23,  // gated form on the tensor cores: segment states (both directions)
+  K_GLA_SEG_SCAN = 24,    // gated form: prefix / suffix over segments
   // gated form, the exact CUDA-core sequence a tensor-core call switches to
   // on the device when a tile's log-gates leave the factorized form's range
   // (the kernels return at once otherwise)

@@ -12,9 +12,13 @@
 // segments turns them into the states entering the segments, and the walk
 // carries the state through each segment's tiles, leaving in the slot of every
 // tile's first chunk the bf16 operand tile of diag(e^{r}) P (r the tile's
-// middle-row log-gate sums) that the backward loads back as is. The backward's
-// gradient states go to the slot of each tile's last chunk of the workspace;
-// its scan over tiles uses the tile totals.
+// middle-row log-gate sums) that the backward loads back as is. The backward
+// takes the same segments: their gradient states go to the workspace slot of
+// each segment's last chunk, the scan over segments (with the forward's
+// segment totals) turns them into the states entering the segments from the
+// right, and the gradient kernel walks each segment's tiles backward, forming
+// every other tile's entering state on the way (in the slot of the segment's
+// first chunk).
 //
 // The tensor-core kernels factor the intra-tile gate products around each
 // tile's middle row, which holds while the log-gates of each half-tile span
@@ -171,24 +175,27 @@ int lasp_gla_bwd(const void* q, const void* k, const void* v, const float* g, co
   const int T = (int)(N / C);
   const float* gsum = state_cache + (int64_t)B * T * H * d * d;
   if (tc_gla_ok(dtype, d, C, N)) {
-    // 128-token tiles: gradient states into the slots of each tile's last
-    // chunk, the suffix over tiles in place (the tiles' log-gate totals sit in
-    // the cache slots of their first chunks), then the gradients
+    // the forward's segments of S 128-token tiles: gradient states into the
+    // slots of each segment's last chunk, the suffix over segments in place
+    // (the segments' log-gate totals sit in the cache's third array, in the
+    // slots of their first chunks), then the gradients, walking each segment
     const int stride = 128 / C;
-    const int tiles = (int)(N / 128);
+    const int S = walk_segment_tokens(N, 128) / 128;
+    const int nseg = (int)(N / 128) / S;
+    const float* gseg = gsum + (int64_t)B * T * H * d;
     // the forward's choice, in the cache's flag word
     const int* flag = reinterpret_cast<const int*>(state_cache + cache_state_floats(B, H, N, d, C));
     const RunIf tc{flag, 0}, exact{flag, 1};
-    if ((s = cuda_status(traced(K_GLA_STATES_TC, st, [&] {
-           return tc_gla_chunk_states(q, dout, g, dstate_ws, nullptr, nullptr, B, H, N, 1, T, stride, stride - 1, 1,
-                                      stride, st, nullptr, tc);
+    if ((s = cuda_status(traced(K_GLA_SEG_STATES, st, [&] {
+           return tc_gla_chunk_states(q, dout, g, dstate_ws, nullptr, nullptr, B, H, N, 1, T, S * stride,
+                                      S * stride - 1, S, stride, st, nullptr, tc);
          }))))
       return s;
-    if ((s = scan_impl(dstate_ws, dstate_ws, gsum, dstate_in, dinit_state, B, tiles, H, d, 1, T, stride, stride - 1, 0,
-                       st, tc)))
+    if ((s = scan_impl(dstate_ws, dstate_ws, gseg, dstate_in, dinit_state, B, nseg, H, d, 1, T, S * stride,
+                       S * stride - 1, 0, st, tc, K_GLA_SEG_SCAN)))
       return s;
     if ((s = cuda_status(traced(K_GLA_BWD_TC, st, [&] {
-           return tc_gla_chunk_bwd(q, k, v, dout, g, state_cache, dstate_ws, dq, dk, dv, dg, B, H, N, T, stride, st,
+           return tc_gla_chunk_bwd(q, k, v, dout, g, state_cache, dstate_ws, dq, dk, dv, dg, B, H, N, T, stride, S, st,
                                    tc);
          }))))
       return s;

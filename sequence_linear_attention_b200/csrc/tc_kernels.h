@@ -70,7 +70,10 @@ cudaError_t tc_bidir_apply(const void* x, const void* stiles, void* y, int B, in
 // tile (kind 0 from (k, v) with the log-gate totals, kind 1 from (q, do)) into
 // slot tile * stride + offset of an array of t_slots chunk states; the output
 // given P in the slot of each tile's first chunk; the gradients given that P
-// and R in the slot of the tile's last chunk (stride = chunks per tile).
+// and, for segments of `tiles` tiles, the R entering each segment in the slot
+// of its last chunk (stride = chunks per tile): the kernel forms every other
+// tile's R on its walk through the segment, in the slot of the segment's first
+// chunk, which it overwrites.
 bool tc_gla_ok(int dtype, int d, int64_t C, int64_t N);
 // span_flag (may be NULL): set to 1 when a tile's log-gates span more than the
 // factorized form of the output and backward kernels takes; `run` makes a
@@ -83,8 +86,8 @@ cudaError_t tc_gla_chunk_out(const void* q, const void* k, const void* v, const 
                              int B, int H, int64_t N, int64_t t_slots, int stride, int tiles, cudaStream_t st,
                              RunIf run = {});
 cudaError_t tc_gla_chunk_bwd(const void* q, const void* k, const void* v, const void* dout, const float* g,
-                             const float* P, const float* Rs, void* dq, void* dk, void* dv, float* dg, int B, int H,
-                             int64_t N, int64_t t_slots, int stride, cudaStream_t st, RunIf run = {});
+                             const float* P, float* Rs, void* dq, void* dk, void* dv, float* dg, int B, int H,
+                             int64_t N, int64_t t_slots, int stride, int tiles, cudaStream_t st, RunIf run = {});
 
 // Causal softmax attention, bf16, d = 128 (k_tc_softmax.cu): queries at
 // positions q_offset + i (i < Nq) against keys / values at 0..Nk-1; lse

@@ -60,9 +60,10 @@ def test_single_rank_needs_no_process_group():
 
 def test_algorithmic_bytes_of_the_segment_kernels():
     """Bytes per token-head of the kernels that work per segment of G tokens:
-    the state total reads the segment states once; the gated forward's segment
-    states write one state per segment; its walk reads one state per segment
-    and writes a bf16 state tile per 128 tokens."""
+    the state total reads the segment states once; the gated segment states
+    write one state per segment; the forward walk reads one state per segment
+    and writes a bf16 state tile per 128 tokens, which the backward walk reads
+    back with one gradient state per segment."""
     sys.path.insert(0, ROOT)
     import bench
     d, G, e = 128, 1024, 2
@@ -71,7 +72,7 @@ def test_algorithmic_bytes_of_the_segment_kernels():
     assert bench.algorithmic_bytes("gla_segment_states_tc", 1, d, 128, G, e) == 2 * d * e + 4 * d + s / G
     assert bench.algorithmic_bytes("gla_segment_scan", 1, d, 128, G, e) == 2 * s / G + 4 * d / G
     assert bench.algorithmic_bytes("gla_out_tc", 1, d, 128, G, e) == 4 * d * e + 4 * d + s / G + s / 256
-    assert bench.algorithmic_bytes("gla_bwd_tc", 1, d, 128, G, e) == 7 * d * e + 8 * d + s / 256 + s / 128
+    assert bench.algorithmic_bytes("gla_bwd_tc", 1, d, 128, G, e) == 7 * d * e + 8 * d + s / 256 + s / G
     # per-tile kernels do not depend on the segment
     assert bench.algorithmic_bytes("gla_states_tc", 1, d, 128, G, e) == bench.algorithmic_bytes(
         "gla_states_tc", 1, d, 128, 128, e)

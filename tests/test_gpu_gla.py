@@ -199,6 +199,20 @@ def test_tensor_core_path_matches_oracle(B, N, H, tau, seed):
     _compare(got, ref, TOL_BF16)
 
 
+def test_tensor_core_path_with_more_segments_than_sms():
+    """150 one-segment heads: the first CTAs walk a second segment after their
+    first, so the backward's walk passes from a segment's first tile to the
+    next segment's last (whose entering state comes from the scan again)."""
+    B, N, H, d, C = 1, 1024, 150, 128, 128
+    inp = lasp_inputs.make_inputs(B, N, H, d, seed=2025, bf16=True, decayed=False)
+    g = lasp_inputs.make_log_gates(B, N, H, d, seed=2025, tau=4.0)
+    rng = np.random.default_rng(2025)
+    dsin = (rng.standard_normal((B, H, d, d)) * 0.1).astype(np.float32)
+    got = _run(inp, g, C, dstate_in=dsin)
+    ref = _reference(inp, g, dstate_in=dsin.astype(np.float64))
+    _compare(got, ref, TOL_BF16)
+
+
 def test_tensor_core_rows_match_oracle():
     _rows_states(True, 128, 128)
 
@@ -280,7 +294,7 @@ def test_mild_gates_leave_the_exact_kernels_idle():
     ms = dict(trace)
     names = [n for n, _ in trace]
     assert names == ["gla_segment_states_tc", "gla_segment_scan", "gla_out_tc", "gla_states_exact",
-                     "gla_scan_exact", "gla_out_exact", "gla_states_tc", "gla_scan", "gla_bwd_tc",
+                     "gla_scan_exact", "gla_out_exact", "gla_segment_states_tc", "gla_segment_scan", "gla_bwd_tc",
                      "gla_states_exact", "gla_scan_exact", "gla_bwd_exact"], names
     assert ms["gla_out_exact"] < 0.5 * ms["gla_out_tc"], trace
     assert ms["gla_bwd_exact"] < 0.5 * ms["gla_bwd_tc"], trace
