@@ -479,7 +479,10 @@ LASP_API int lasp_gla_fwd(const void* q, const void* k, const void* v, const flo
  * so that dg stays accurate to its own size when the gates are strong.
  *   state_cache: in, what lasp_gla_fwd wrote for the same q, k, v, g, C and
  *                init_state. Required.
- *   dstate_ws:   workspace, B * (N/C) * H * d * d floats. Required.
+ *   dstate_ws:   workspace, B * (N/C) * H * d * d floats. Required. Its
+ *                contents afterwards are internal (the tensor-core path keeps
+ *                one gradient state per segment and a scratch state per
+ *                segment; the CUDA-core path R_c per chunk).
  *   dstate_in:   in, float [B, H, d, d] or NULL: gradient with respect to the
  *                state after the last token.
  *   dinit_state: out, float [B, H, d, d] or NULL: gradient with respect to

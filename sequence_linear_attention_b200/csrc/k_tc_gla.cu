@@ -7,8 +7,9 @@
 // row), the states being needed at tile boundaries only. The forward works on
 // segments of tiles: the state kernel sums each segment's tiles into one
 // state, and the output kernel walks each segment's tiles with the state in
-// TMEM. The backward takes one tile at a time (per-tile states; its persistent
-// CTAs take one tile after another).
+// TMEM. The backward works on the same segments: one gradient state per
+// segment, and a walk back through each segment's tiles that forms every
+// tile's entering gradient state from the one after it.
 //
 // The intra-tile products need the factor e^{b_t[i] - b_s[i]} inside a
 // contraction over i, which a single MMA can carry only if it splits into a
