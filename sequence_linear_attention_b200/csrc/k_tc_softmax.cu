@@ -31,12 +31,14 @@
 //   dv_j = sum_i p_ij do_i,  dk_j = scale sum_i ds_ij q_i,  dq_i = scale sum_j ds_ij k_j.
 // softmax_delta: delta per query row. softmax_dkdv_tc: one CTA per 128-key
 // tile walks the query tiles that see it: S^T = K Q^T and dP^T = V dO^T into
-// TMEM, then (eight epilogue warps) P^T and dS^T in bf16, then dV += P^T dO
-// and dK += dS^T Q; Q and dO stream through a three-slot ring so that the next
-// Q tile loads during the current tile. softmax_dq_tc: one CTA per 128-query
-// tile walks its key tiles: S = Q K^T, dP = dO V^T, dS, dQ += dS K. The two
-// gradient kernels recompute P separately, so no atomics are needed and the
-// results do not depend on scheduling.
+// TMEM, then (sixteen epilogue warps, 32 query columns each) P^T and dS^T in
+// bf16, then dV += P^T dO and dK += dS^T Q; Q and dO stream through a
+// three-slot ring so that the next Q tile loads during the current tile.
+// softmax_dq_tc: one CTA per 128-query tile walks its key tiles, each in two
+// halves of 64 keys: S = Q K^T, dP = dO V^T, dS, dQ += dS K. Only the tiles
+// on the causal diagonal mask element by element. The two gradient kernels
+// recompute P separately, so no atomics are needed and the results do not
+// depend on scheduling.
 #include <algorithm>
 
 #include "kernels.h"
@@ -364,8 +366,20 @@ __global__ void __launch_bounds__(256) softmax_delta(const __nv_bfloat16* __rest
   }
 }
 
-constexpr int kBwdThreads = 320;  // warps 0-7 epilogue, 8 TMA, 9 MMA
-constexpr uint32_t kBarEpi = 1;
+constexpr uint32_t kBarEpi = 1;  // named barrier of the gradient kernels' epilogue warps
+constexpr int kDqThreads = 576;   // softmax_dq_tc: warps 0-15 epilogue, 16 TMA, 17 MMA
+constexpr int kDqEpi = 512;  // epilogue threads of both gradient kernels
+constexpr int kDkdvThreads = 576;  // softmax_dkdv_tc: warps 0-15 epilogue, 16 TMA, 17 MMA
+
+// 16 consecutive fp32 columns of this thread's TMEM lane (warp-collective).
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]),
+        "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+}
 
 // Reads the S-type and dP-type accumulators of this thread's row (TMEM lane)
 // and column half, forms p = exp2(s c - lse2) (0 where masked) and
@@ -375,54 +389,49 @@ constexpr uint32_t kBarEpi = 1;
 // row's) values through the callbacks.
 // Chunk cc (0 or 1) of the half: columns half * 64 + cc * 32 .. + 31, so that
 // chunk 0 of both halves is the tile's K-steps 0, 1, 4, 5 of the next MMA and
-// chunk 1 its K-steps 2, 3, 6, 7.
+// chunk 1 its K-steps 2, 3, 6, 7. visible = 1 (every column of the chunk inside
+// the mask) or 0 (none) skips the per-column test.
 template <class Keep, class Lse, class Dl>
 __device__ __forceinline__ void p_ds_rows(uint32_t lane_base, uint32_t colS, uint32_t colP, int row, int half,
-                                          int cc, float c2, uint8_t* tP, uint8_t* tDS, Keep keep, Lse lse2, Dl dl) {
-  {
-    const int col0 = half * 64 + cc * 32;
-    uint32_t rs[32], rp[32];
-    tmem_ld32(lane_base + colS + col0, rs);
-    tmem_ld32(lane_base + colP + col0, rp);
+                                          int cc, float c2, uint8_t* tP, uint8_t* tDS, Keep keep, Lse lse2, Dl dl,
+                                          int visible = -1) {
+  const int col0 = half * 64 + cc * 32;
+  // in two passes of 16 columns, so that the values of one pass stay in registers
+#pragma unroll 1
+  for (int ps = 0; ps < 2; ++ps) {
+    const int cb = col0 + ps * 16;
+    uint32_t rs[16], rp[16];
+    tmem_ld16(lane_base + colS + cb, rs);
+    tmem_ld16(lane_base + colP + cb, rp);
     tmem_ld_wait();
-    float p[32], ds[32];
+    float p[16], ds[16];
+    if (visible == 1) {  // every column of the chunk is inside the mask
 #pragma unroll
-    for (int u = 0; u < 32; ++u) {
-      const int c = col0 + u;
-      const float e = ex2(__uint_as_float(rs[u]) * c2 - lse2(c));
-      p[u] = keep(c) ? e : 0.f;
-      ds[u] = p[u] * (__uint_as_float(rp[u]) - dl(c));
+      for (int u = 0; u < 16; ++u) {
+        const int c = cb + u;
+        p[u] = ex2(__uint_as_float(rs[u]) * c2 - lse2(c));
+        ds[u] = p[u] * (__uint_as_float(rp[u]) - dl(c));
+      }
+    } else if (visible == 0) {  // none is
+#pragma unroll
+      for (int u = 0; u < 16; ++u) p[u] = ds[u] = 0.f;
+    } else {
+#pragma unroll
+      for (int u = 0; u < 16; ++u) {
+        const int c = cb + u;
+        const float e = ex2(__uint_as_float(rs[u]) * c2 - lse2(c));
+        p[u] = keep(c) ? e : 0.f;
+        ds[u] = p[u] * (__uint_as_float(rp[u]) - dl(c));
+      }
     }
 #pragma unroll
-    for (int q8 = 0; q8 < 4; ++q8) {
-      st_tile16(tP, row, col0 + q8 * 8,
+    for (int q8 = 0; q8 < 2; ++q8) {
+      st_tile16(tP, row, cb + q8 * 8,
                 make_uint4(pack_bf16(p[q8 * 8], p[q8 * 8 + 1]), pack_bf16(p[q8 * 8 + 2], p[q8 * 8 + 3]),
                            pack_bf16(p[q8 * 8 + 4], p[q8 * 8 + 5]), pack_bf16(p[q8 * 8 + 6], p[q8 * 8 + 7])));
-      st_tile16(tDS, row, col0 + q8 * 8,
+      st_tile16(tDS, row, cb + q8 * 8,
                 make_uint4(pack_bf16(ds[q8 * 8], ds[q8 * 8 + 1]), pack_bf16(ds[q8 * 8 + 2], ds[q8 * 8 + 3]),
                            pack_bf16(ds[q8 * 8 + 4], ds[q8 * 8 + 5]), pack_bf16(ds[q8 * 8 + 6], ds[q8 * 8 + 7])));
-    }
-  }
-}
-
-// Row `row`, column half `half` of a 128-column fp32 accumulator, times f, as
-// bf16 into the tile (the staging of a TMA store).
-__device__ __forceinline__ void acc_to_tile(uint32_t lane_base, uint32_t col, int row, int half, float f,
-                                            uint8_t* tile) {
-#pragma unroll 1
-  for (int cc = 0; cc < 2; ++cc) {
-    const int col0 = half * 64 + cc * 32;
-    uint32_t r[32];
-    tmem_ld32(lane_base + col + col0, r);
-    tmem_ld_wait();
-#pragma unroll
-    for (int q8 = 0; q8 < 4; ++q8) {
-      float v[8];
-#pragma unroll
-      for (int u = 0; u < 8; ++u) v[u] = __uint_as_float(r[q8 * 8 + u]) * f;
-      st_tile16(tile, row, col0 + q8 * 8,
-                make_uint4(pack_bf16(v[0], v[1]), pack_bf16(v[2], v[3]), pack_bf16(v[4], v[5]),
-                           pack_bf16(v[6], v[7])));
     }
   }
 }
@@ -434,7 +443,7 @@ struct SmemDkdv {
   float lse2[kTile], dl[kTile];  // the current query tile's lse (log2 units) and delta
 };
 
-__global__ void __launch_bounds__(kBwdThreads, 1) softmax_dkdv_tc(
+__global__ void __launch_bounds__(kDkdvThreads, 1) softmax_dkdv_tc(
     const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
     const __grid_constant__ CUtensorMap map_v, const __grid_constant__ CUtensorMap map_do,
     const __grid_constant__ CUtensorMap map_dk, const __grid_constant__ CUtensorMap map_dv,
@@ -491,7 +500,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) softmax_dkdv_tc(
   const uint32_t tmem = s->tmem_base;
   constexpr uint32_t kColS = 0, kColP = 128, kColV = 256, kColK = 384;
 
-  if (warp == 8) {
+  if (warp == 16) {
     // ---------------------------------------------------------- TMA producer
     bool bad = false;
     int issued = 0;  // ring loads issued
@@ -517,9 +526,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1) softmax_dkdv_tc(
           ++issued;
         }
       }
+      // the last tile's epilogue has read lse and delta (both chunk groups)
       if (lane == 0 && !bad && (x & 1) == 0 && i > 0 &&
-          !mbar_wait_or_abort(&s->p_full, (uint32_t)(i - 1) & 1u, SITE_BWD_MMA, abort_flag))
-        bad = true;  // the last tile's epilogue has read lse and delta
+          (!mbar_wait_or_abort(&s->p_half, (uint32_t)(i - 1) & 1u, SITE_BWD_MMA, abort_flag) ||
+           !mbar_wait_or_abort(&s->p_full, (uint32_t)(i - 1) & 1u, SITE_BWD_MMA, abort_flag)))
+        bad = true;
       bad = __shfl_sync(0xffffffffu, bad, 0);
       if (!bad && (x & 1) == 0) {
         // the tile's lse and delta, by the whole warp; their loads run under
@@ -542,7 +553,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) softmax_dkdv_tc(
         mbar_wait(&s->full[x % 3], (uint32_t)(x / 3) & 1u, SITE_BWD_TMA);
       if (n > 0) mbar_wait(&s->kv_full, 0, SITE_BWD_TMA);
     }
-  } else if (warp == 9) {
+  } else if (warp == 17) {
     // ----------------------------------------------------------- MMA issuer
     if (lane == 0 && n > 0) {
       constexpr uint32_t id_kk = idesc_bf16(128, 128, 0, 0);
@@ -597,8 +608,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1) softmax_dkdv_tc(
       mbar_wait(&s->drain, 0, SITE_BWD_MMA);
     }
   } else {
-    // --------------------------------------------- epilogue warps (0-7)
-    const int row = (warp & 3) * 32 + lane, half = warp >> 2;  // key row of the tile, query-column half
+    // --------------------------------------------- epilogue warps (0-15)
+    // key row of the tile; this thread's 32 query columns sub * 32.., which
+    // are chunk cc = sub & 1 of column half sub >> 1 (the p_half / p_full split)
+    const int row = (warp & 3) * 32 + lane, sub = warp >> 2;
+    const int half = sub >> 1, cc = sub & 1;
     const uint32_t lane_base = tmem + ((uint32_t)((warp & 3) * 32) << 16);
     const int64_t kpos = k0 + row;
     bool bad = false;
@@ -613,16 +627,18 @@ __global__ void __launch_bounds__(kBwdThreads, 1) softmax_dkdv_tc(
       const float* L = s->lse2;
       const float* Dl = s->dl;
       auto keep = [&](int c) { return q0 + c < Nq && q_offset + q0 + c >= kpos; };
-      for (int cc = 0; cc < 2; ++cc) {
-        if (!bad) {
-          tc_fence_after();
-          p_ds_rows(lane_base, kColS, kColP, row, half, cc, c2, sPt, sDSt, keep, [&](int c) { return L[c]; },
-                    [&](int c) { return Dl[c]; });
-        }
-        fence_async_smem();
-        tc_fence_before();
-        mbar_arrive(cc == 0 ? &s->p_half : &s->p_full);  // the MMA takes each chunk as it is done
+      // the chunk's columns c = sub * 32 .. + 31: all inside the mask, none, or some
+      const int64_t cfirst = q0 + sub * 32, clast = cfirst + 31;
+      const int visible = (clast < Nq && q_offset + cfirst >= kpos) ? 1
+                          : (cfirst >= Nq || q_offset + clast < kpos) ? 0 : -1;
+      if (!bad) {
+        tc_fence_after();
+        p_ds_rows(lane_base, kColS, kColP, row, half, cc, c2, sPt, sDSt, keep, [&](int c) { return L[c]; },
+                  [&](int c) { return Dl[c]; }, visible);
       }
+      fence_async_smem();
+      tc_fence_before();
+      mbar_arrive(cc == 0 ? &s->p_half : &s->p_full);  // the MMA takes each chunk as it is done
     }
     if (n > 0 && !bad && !mbar_wait_or_abort(&s->mma2_done, (uint32_t)(n - 1) & 1u, SITE_BWD_MMA, abort_flag))
       bad = true;
@@ -630,20 +646,35 @@ __global__ void __launch_bounds__(kBwdThreads, 1) softmax_dkdv_tc(
     if (bad) s->abort = 1;
     if (!bad) {
       if (n > 0) {
+        // dK (times scale) and dV, columns sub * 32.. of row `row`, into the P^T and dS^T tiles
         tc_fence_after();
-        acc_to_tile(lane_base, kColK, row, half, scale, sPt);
-        acc_to_tile(lane_base, kColV, row, half, 1.f, sDSt);
+#pragma unroll 1
+        for (int t2 = 0; t2 < 2; ++t2) {
+          uint32_t r[32];
+          tmem_ld32(lane_base + (t2 == 0 ? kColK : kColV) + sub * 32, r);
+          tmem_ld_wait();
+          const float f = t2 == 0 ? scale : 1.f;
+#pragma unroll
+          for (int q8 = 0; q8 < 4; ++q8) {
+            float v[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) v[u] = __uint_as_float(r[q8 * 8 + u]) * f;
+            st_tile16(t2 == 0 ? sPt : sDSt, row, sub * 32 + q8 * 8,
+                      make_uint4(pack_bf16(v[0], v[1]), pack_bf16(v[2], v[3]), pack_bf16(v[4], v[5]),
+                                 pack_bf16(v[6], v[7])));
+          }
+        }
       } else {
         // no query sees these keys: their gradients are zero
 #pragma unroll
-        for (int c8 = 0; c8 < 8; ++c8) {
-          st_tile16(sPt, row, half * 64 + c8 * 8, make_uint4(0u, 0u, 0u, 0u));
-          st_tile16(sDSt, row, half * 64 + c8 * 8, make_uint4(0u, 0u, 0u, 0u));
+        for (int c8 = 0; c8 < 4; ++c8) {
+          st_tile16(sPt, row, sub * 32 + c8 * 8, make_uint4(0u, 0u, 0u, 0u));
+          st_tile16(sDSt, row, sub * 32 + c8 * 8, make_uint4(0u, 0u, 0u, 0u));
         }
       }
     }
     fence_async_smem();
-    named_sync(kBarEpi, 256);
+    named_sync(kBarEpi, kDqEpi);
     if (tid == 0 && !s->abort) {
       tma_store_4d(&map_dk, sPt, 0, h, (int)k0, b);
       tma_store_4d(&map_dk, sPt + kBox, 64, h, (int)k0, b);
@@ -658,13 +689,31 @@ __global__ void __launch_bounds__(kBwdThreads, 1) softmax_dkdv_tc(
   if (warp == 0) tmem_dealloc(tmem, 512);
 }
 
+// softmax_dq_tc works on each key tile in two halves of 64 keys, so that the
+// epilogue of one half runs while the tensor pipe computes the other half's S
+// and dP and the previous half's dQ update. TMEM: S_h at 128 h, dP_h at
+// 128 h + 64 (h = 0, 1), dQ at 256. Per key tile j the MMA thread issues
+//   S_0, dP_0 (once the epilogue has read half 0 of tile j - 1)
+//   dQ += dS_1 K_{j-1,1}  (once half 1 of tile j - 1 is written)
+//   S_1, dP_1 (once the epilogue has read half 1 of tile j - 1)
+//   dQ += dS_0 K_{j,0}    (once half 0 of tile j is written)
+// and the epilogue takes the halves in order: dS_h of tile j goes into
+// columns 64 h.. of the dS tile once the dQ MMA of tile j - 1 has read them.
+// Sixteen epilogue warps (four per TMEM lane quarter, 16 columns of a half
+// each) keep the exponentials' latency covered; only the tile on the causal
+// diagonal masks element by element.
 struct SmemDq {
-  uint64_t qd_full, k_full[2], v_full[2], kv_empty[2], s_full, ds_half, ds_full, dq_done, drain;
+  uint64_t qd_full, k_full[2], v_full[2], kv_empty[2];
+  uint64_t s_full[2];    // MMA -> epilogue: S_h and dP_h are in TMEM
+  uint64_t t_free[2];    // epilogue -> MMA: TMEM half h has been read (512 arrivals)
+  uint64_t ds_ready[2];  // epilogue -> MMA: dS_h is in shared memory (512 arrivals)
+  uint64_t ds_free[2];   // MMA -> epilogue: the dQ MMA has read dS_h
+  uint64_t drain;
   uint32_t tmem_base;
   int abort;
 };
 
-__global__ void __launch_bounds__(kBwdThreads, 1) softmax_dq_tc(
+__global__ void __launch_bounds__(kDqThreads, 1) softmax_dq_tc(
     const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
     const __grid_constant__ CUtensorMap map_v, const __grid_constant__ CUtensorMap map_do,
     const __grid_constant__ CUtensorMap map_dq, const float* __restrict__ lse, const float* __restrict__ delta,
@@ -675,7 +724,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) softmax_dq_tc(
   uint8_t* sO = base + kTileBytes;      // dO
   uint8_t* sK = base + 2 * kTileBytes;  // two stages
   uint8_t* sV = base + 4 * kTileBytes;  // two stages
-  uint8_t* sDS = base + 6 * kTileBytes;
+  uint8_t* sDS = base + 6 * kTileBytes;  // dS: keys 0-63 in the first box, 64-127 in the second
   SmemDq* s = reinterpret_cast<SmemDq*>(base + 7 * kTileBytes);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int qt = qtiles - 1 - (int)blockIdx.x;  // heaviest tiles first
@@ -685,6 +734,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) softmax_dq_tc(
   const int nkv = (int)(last_pos / kTile) + 1;
   const volatile int* abort_flag = &s->abort;
   const float c2 = scale * kLog2e;
+  constexpr uint32_t kHalfRows = 64 * 128;  // byte offset of row 64 in a 128-byte-swizzled box
 
   if (tid == 0) {
     prefetch_tmap(&map_q);
@@ -697,11 +747,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1) softmax_dq_tc(
       mbar_init(&s->k_full[st], 1);
       mbar_init(&s->v_full[st], 1);
       mbar_init(&s->kv_empty[st], 1);
+      mbar_init(&s->s_full[st], 1);
+      mbar_init(&s->t_free[st], kDqEpi);
+      mbar_init(&s->ds_ready[st], kDqEpi);
+      mbar_init(&s->ds_free[st], 1);
     }
-    mbar_init(&s->s_full, 1);
-    mbar_init(&s->ds_half, 256);
-    mbar_init(&s->ds_full, 256);
-    mbar_init(&s->dq_done, 1);
     mbar_init(&s->drain, 1);
     s->abort = 0;
     fence_mbar_init();
@@ -714,9 +764,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1) softmax_dq_tc(
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = s->tmem_base;
-  constexpr uint32_t kColS = 0, kColP = 128, kColQ = 256;
+  constexpr uint32_t kColQ = 256;  // S_h at 128 h, dP_h at 128 h + 64
 
-  if (warp == 8) {
+  if (warp == 16) {
     if (lane == 0) {
       bool bad = false;
       mbar_arrive_expect_tx(&s->qd_full, 2 * kTileBytes);
@@ -747,56 +797,55 @@ __global__ void __launch_bounds__(kBwdThreads, 1) softmax_dq_tc(
       }
       mbar_wait(&s->qd_full, 0, SITE_BWD_TMA);
     }
-  } else if (warp == 9) {
+  } else if (warp == 17) {
     if (lane == 0) {
-      constexpr uint32_t id_kk = idesc_bf16(128, 128, 0, 0);
-      constexpr uint32_t id_kn = idesc_bf16(128, 128, 0, 1);
+      constexpr uint32_t id_s = idesc_bf16(128, 64, 0, 0);   // S_h, dP_h: 64 keys
+      constexpr uint32_t id_q = idesc_bf16(128, 128, 0, 1);  // dQ += dS_h K_h: K = 64 keys
       const uint32_t aQ = smem_u32(sQ), aO = smem_u32(sO), aD = smem_u32(sDS);
       bool bad = !mbar_wait_or_abort(&s->qd_full, 0, SITE_BWD_TMA, abort_flag);
+      // dQ += dS_hh K_{jj,hh}, once the epilogue has written dS_hh of key tile jj
+      auto dq_mma = [&](int jj, int hh) {
+        if (!mbar_wait_or_abort(&s->ds_ready[hh], (uint32_t)jj & 1u, SITE_BWD_MMA, abort_flag)) return false;
+        tc_fence_after();
+        const uint32_t aKh = smem_u32(sK + (jj & 1) * kTileBytes) + hh * kHalfRows;
+        for (int kk = 0; kk < 4; ++kk)
+          mma_bf16(tmem + kColQ, kmaj(aD + hh * kBox, kk), mnmaj(aKh, kk), id_q, (jj > 0 || hh > 0 || kk > 0) ? 1u : 0u);
+        mma_commit(&s->ds_free[hh]);
+        if (hh == 1) mma_commit(&s->kv_empty[jj & 1]);  // K_jj and V_jj are read
+        return true;
+      };
       for (int j = 0; j < nkv && !bad; ++j) {
         const int st = j & 1;
         const uint32_t use = (uint32_t)(j >> 1) & 1u;
         const uint32_t aK = smem_u32(sK + st * kTileBytes), aV = smem_u32(sV + st * kTileBytes);
-        if (!mbar_wait_or_abort(&s->k_full[st], use, SITE_BWD_TMA, abort_flag)) {
+        if (!mbar_wait_or_abort(&s->k_full[st], use, SITE_BWD_TMA, abort_flag) ||
+            !mbar_wait_or_abort(&s->v_full[st], use, SITE_BWD_TMA, abort_flag)) {
           bad = true;
           break;
         }
-        tc_fence_after();
-        for (int kk = 0; kk < kD / 16; ++kk) mma_bf16(tmem + kColS, kmaj(aQ, kk), kmaj(aK, kk), id_kk, kk > 0);
-        if (!mbar_wait_or_abort(&s->v_full[st], use, SITE_BWD_TMA, abort_flag)) {
-          bad = true;
-          break;
-        }
-        tc_fence_after();
-        for (int kk = 0; kk < kD / 16; ++kk) mma_bf16(tmem + kColP, kmaj(aO, kk), kmaj(aV, kk), id_kk, kk > 0);
-        mma_commit(&s->s_full);
-        // dQ += dS K over the key columns the epilogue has finished: K-steps
-        // 0, 1, 4, 5 (its first chunk), then 2, 3, 6, 7
-        bool part_ok = true;
-        for (int pc = 0; pc < 2; ++pc) {
-          if (!mbar_wait_or_abort(pc == 0 ? &s->ds_half : &s->ds_full, (uint32_t)j & 1u, SITE_BWD_MMA, abort_flag)) {
-            part_ok = false;
+        for (int hh = 0; hh < 2 && !bad; ++hh) {
+          if (j > 0 && !mbar_wait_or_abort(&s->t_free[hh], (uint32_t)(j - 1) & 1u, SITE_BWD_MMA, abort_flag)) {
+            bad = true;
             break;
           }
           tc_fence_after();
-          for (int q = 0; q < 4; ++q) {
-            const int kk = (q >> 1) * 4 + pc * 2 + (q & 1);
-            mma_bf16(tmem + kColQ, kmaj(aD, kk), mnmaj(aK, kk), id_kn, (j > 0 || pc > 0 || q > 0) ? 1u : 0u);
-          }
+          const uint32_t colS = (uint32_t)hh * 128;
+          for (int kk = 0; kk < kD / 16; ++kk)
+            mma_bf16(tmem + colS, kmaj(aQ, kk), kmaj(aK + hh * kHalfRows, kk), id_s, kk > 0);
+          for (int kk = 0; kk < kD / 16; ++kk)
+            mma_bf16(tmem + colS + 64, kmaj(aO, kk), kmaj(aV + hh * kHalfRows, kk), id_s, kk > 0);
+          mma_commit(&s->s_full[hh]);
+          if (hh == 0 ? (j > 0 && !dq_mma(j - 1, 1)) : !dq_mma(j, 0)) bad = true;
         }
-        if (!part_ok) {
-          bad = true;
-          break;
-        }
-        mma_commit(&s->kv_empty[st]);
-        mma_commit(&s->dq_done);
       }
+      if (!bad && nkv > 0 && !dq_mma(nkv - 1, 1)) bad = true;
       if (bad) s->abort = 1;
       mma_commit(&s->drain);
       mbar_wait(&s->drain, 0, SITE_BWD_MMA);
     }
   } else {
-    const int row = (warp & 3) * 32 + lane, half = warp >> 2;  // query row of the tile, key-column half
+    // query row `row` of the tile; this thread's 16 key columns sub * 16.. of each half
+    const int row = (warp & 3) * 32 + lane, sub = warp >> 2;
     const uint32_t lane_base = tmem + ((uint32_t)((warp & 3) * 32) << 16);
     const int64_t qi = q0 + row;
     const int64_t qpos = q_offset + qi;
@@ -805,33 +854,74 @@ __global__ void __launch_bounds__(kBwdThreads, 1) softmax_dq_tc(
     const float dl = in ? delta[((int64_t)b * H + h) * Nq + qi] : 0.f;
     bool bad = false;
     for (int j = 0; j < nkv; ++j) {
-      const int64_t kb = (int64_t)j * kTile;
-      if (!bad && !mbar_wait_or_abort(&s->s_full, (uint32_t)j & 1u, SITE_BWD_MMA, abort_flag)) bad = true;
-      if (j > 0 && !bad && !mbar_wait_or_abort(&s->dq_done, (uint32_t)(j - 1) & 1u, SITE_BWD_MMA, abort_flag))
-        bad = true;  // the last dQ MMA has read dS
-      bad = __any_sync(0xffffffffu, bad);  // the TMEM loads below are warp-collective
-      for (int cc = 0; cc < 2; ++cc) {
+      for (int hh = 0; hh < 2; ++hh) {
+        const int64_t kc = (int64_t)j * kTile + hh * 64 + sub * 16;  // key of this thread's first column
+        // columns u <= lim are inside the causal mask (lim >= 15: all, < 0: none)
+        const int64_t lim64 = in ? qpos - kc : -1;
+        const int lim = lim64 < -1 ? -1 : (lim64 > 15 ? 15 : (int)lim64);
+        if (!bad && !mbar_wait_or_abort(&s->s_full[hh], (uint32_t)j & 1u, SITE_BWD_MMA, abort_flag)) bad = true;
+        // dS_hh's columns are free once the dQ MMA of the last key tile has read them
+        if (j > 0 && !bad && !mbar_wait_or_abort(&s->ds_free[hh], (uint32_t)(j - 1) & 1u, SITE_BWD_MMA, abort_flag))
+          bad = true;
+        bad = __any_sync(0xffffffffu, bad);  // the TMEM loads below are warp-collective
+        uint32_t rs[16], rp[16];
         if (!bad) {
           tc_fence_after();
-          // P is not needed here: its tile is dS's, written twice, the second time with dS
-          p_ds_rows(lane_base, kColS, kColP, row, half, cc, c2, sDS, sDS,
-                    [&](int c) { return in && kb + c <= qpos; }, [&](int) { return lse2; },
-                    [&](int) { return dl; });
+          tmem_ld16(lane_base + hh * 128 + sub * 16, rs);
+          tmem_ld16(lane_base + hh * 128 + 64 + sub * 16, rp);
+          tmem_ld_wait();
+        }
+        tc_fence_before();
+        mbar_arrive(&s->t_free[hh]);  // the MMA may refill this TMEM half
+        if (!bad) {
+          float ds[16];
+          if (lim >= 15) {
+#pragma unroll
+            for (int u = 0; u < 16; ++u)
+              ds[u] = ex2(__uint_as_float(rs[u]) * c2 - lse2) * (__uint_as_float(rp[u]) - dl);
+          } else if (lim < 0) {
+#pragma unroll
+            for (int u = 0; u < 16; ++u) ds[u] = 0.f;
+          } else {
+#pragma unroll
+            for (int u = 0; u < 16; ++u) {
+              const float p = u <= lim ? ex2(__uint_as_float(rs[u]) * c2 - lse2) : 0.f;
+              ds[u] = p * (__uint_as_float(rp[u]) - dl);
+            }
+          }
+#pragma unroll
+          for (int q8 = 0; q8 < 2; ++q8)
+            st_tile16(sDS, row, hh * 64 + sub * 16 + q8 * 8,
+                      make_uint4(pack_bf16(ds[q8 * 8], ds[q8 * 8 + 1]), pack_bf16(ds[q8 * 8 + 2], ds[q8 * 8 + 3]),
+                                 pack_bf16(ds[q8 * 8 + 4], ds[q8 * 8 + 5]),
+                                 pack_bf16(ds[q8 * 8 + 6], ds[q8 * 8 + 7])));
         }
         fence_async_smem();
-        tc_fence_before();
-        mbar_arrive(cc == 0 ? &s->ds_half : &s->ds_full);  // the MMA takes each chunk as it is done
+        mbar_arrive(&s->ds_ready[hh]);
       }
     }
-    if (!bad && !mbar_wait_or_abort(&s->dq_done, (uint32_t)(nkv - 1) & 1u, SITE_BWD_MMA, abort_flag)) bad = true;
+    // the last dQ MMA (half 1 of the last key tile) follows every other
+    if (!bad && !mbar_wait_or_abort(&s->ds_free[1], (uint32_t)(nkv - 1) & 1u, SITE_BWD_MMA, abort_flag)) bad = true;
     bad = __any_sync(0xffffffffu, bad);
     if (bad) s->abort = 1;
     if (!bad) {
+      // dQ (every MMA that read Q is done): columns sub * 32.. of row `row`, times scale, into the Q tile
       tc_fence_after();
-      acc_to_tile(lane_base, kColQ, row, half, scale, sQ);  // every MMA that read Q is done
+      uint32_t r[32];
+      tmem_ld32(lane_base + kColQ + sub * 32, r);
+      tmem_ld_wait();
+#pragma unroll
+      for (int q8 = 0; q8 < 4; ++q8) {
+        float v[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) v[u] = __uint_as_float(r[q8 * 8 + u]) * scale;
+        st_tile16(sQ, row, sub * 32 + q8 * 8,
+                  make_uint4(pack_bf16(v[0], v[1]), pack_bf16(v[2], v[3]), pack_bf16(v[4], v[5]),
+                             pack_bf16(v[6], v[7])));
+      }
     }
     fence_async_smem();
-    named_sync(kBarEpi, 256);
+    named_sync(kBarEpi, kDqEpi);
     if (tid == 0 && !s->abort) {
       tma_store_4d(&map_dq, sQ, 0, h, (int)q0, b);
       tma_store_4d(&map_dq, sQ + kBox, 64, h, (int)q0, b);
@@ -891,7 +981,7 @@ cudaError_t tc_softmax_dkdv(const void* q, const void* k, const void* v, const f
   const size_t smem = sizeof(SmemDkdv) + 1023 + 7 * (size_t)kTileBytes;
   cudaError_t e = cudaFuncSetAttribute(softmax_dkdv_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  softmax_dkdv_tc<<<dim3((unsigned)ktiles, H, B), kBwdThreads, smem, st>>>(mq, mk, mv, mdo, mdk, mdv, lse, delta, H,
+  softmax_dkdv_tc<<<dim3((unsigned)ktiles, H, B), kDkdvThreads, smem, st>>>(mq, mk, mv, mdo, mdk, mdv, lse, delta, H,
                                                                           Nq, q_offset, scale, qtiles);
   return cudaGetLastError();
 }
@@ -909,7 +999,7 @@ cudaError_t tc_softmax_dq(const void* q, const void* k, const void* v, const flo
   const size_t smem = 1024 + 7 * (size_t)kTileBytes + sizeof(SmemDq);
   cudaError_t e = cudaFuncSetAttribute(softmax_dq_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  softmax_dq_tc<<<dim3((unsigned)qtiles, H, B), kBwdThreads, smem, st>>>(mq, mk, mv, mdo, mdq, lse, delta, H, Nq,
+  softmax_dq_tc<<<dim3((unsigned)qtiles, H, B), kDqThreads, smem, st>>>(mq, mk, mv, mdo, mdq, lse, delta, H, Nq,
                                                                         q_offset, scale, qtiles);
   return cudaGetLastError();
 }
