@@ -62,6 +62,15 @@ constexpr float kMaxSpan = 80.f;  // largest |b_t - r| (natural log) the factori
 constexpr float kSpanCheck = kMaxSpan - 1.f;
 constexpr uint32_t kBarAll = 1;   // named barrier over all 256 threads
 
+// 2^x by the hardware's approximate exponential (relative error near 2^-22;
+// results below 2^-126 flush to zero). Every exponent here is a difference of
+// log-gate sums within the factorized range, or a gate factor at most 1.
+__device__ __forceinline__ float ex2a(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 // Orders this thread's generic-proxy writes to global memory before later
 // async-proxy (bulk copy) reads of them.
 __device__ __forceinline__ void fence_async_global() { asm volatile("fence.proxy.async.global;" ::: "memory"); }
@@ -78,7 +87,7 @@ __device__ __forceinline__ void scale_row_half(uint8_t* tile, int row, int half,
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
       const float2 f = unpack_bf16(e[u]);
-      e[u] = pack_bf16(f.x * exp2f(sgn * x[c8 * 8 + 2 * u]), f.y * exp2f(sgn * x[c8 * 8 + 2 * u + 1]));
+      e[u] = pack_bf16(f.x * ex2a(sgn * x[c8 * 8 + 2 * u]), f.y * ex2a(sgn * x[c8 * 8 + 2 * u + 1]));
     }
     *p = w;
   }
@@ -299,8 +308,8 @@ __global__ void __launch_bounds__(kThreads, 2) gla_states_tc(const __grid_consta
       if (ok) {
         uint2 w = *e;
         const float2 a = unpack_bf16(w.x), c2 = unpack_bf16(w.y);
-        w.x = pack_bf16(a.x * exp2f(acc.x * kLog2e), a.y * exp2f(acc.y * kLog2e));
-        w.y = pack_bf16(c2.x * exp2f(acc.z * kLog2e), c2.y * exp2f(acc.w * kLog2e));
+        w.x = pack_bf16(a.x * ex2a(acc.x * kLog2e), a.y * ex2a(acc.y * kLog2e));
+        w.y = pack_bf16(c2.x * ex2a(acc.z * kLog2e), c2.y * ex2a(acc.w * kLog2e));
         *e = w;
       }
       if (kind == 0) {
@@ -510,8 +519,8 @@ __global__ void __launch_bounds__(kThreads, 1) gla_out_tc(const __grid_constant_
   // then e^{r} makes P'. They are applied one after the other: each lies in
   // [e^{-80}, 1] (the range check bounds both half-tile sums), their product
   // need not be a normal fp32 number.
-  const float wcarry = exp2f(dprev * kLog2e);
-  const float wrow = exp2f(s->r[t] * kLog2e);
+  const float wcarry = ex2a(dprev * kLog2e);
+  const float wrow = ex2a(s->r[t] * kLog2e);
   const float dnext = s->dend[t];
   if (!mbar_wait(&s->load, ph, SITE_OUT_TMA))
     s->abort = 1;
@@ -837,7 +846,7 @@ __global__ void __launch_bounds__(kThreads, 1) gla_bwd_tc(
   float x[64];
   gate_rows(bt, &s->gload, ph, &s->abort, SITE_BWD_TMA, sr, sdend, tid, t, half, x);
   // e^{r}, e^{b_end - r} and e^{b_end} of state row t (feature t)
-  const float er = exp2f(sr[t] * kLog2e), wt = exp2f(sdend[t] * kLog2e), eb = er * wt;
+  const float er = ex2a(sr[t] * kLog2e), wt = ex2a(sdend[t] * kLog2e), eb = er * wt;
   named_sync(kBarAll, kThreads);  // every row of the gate tile has been read
   if (tid == 0) {
     // R_c (fp32) into the gate tile's space while the token tiles arrive
@@ -1012,7 +1021,7 @@ __global__ void __launch_bounds__(kThreads, 1) gla_bwd_tc(
 #pragma unroll
         for (int u2 = 0; u2 < 16; ++u2) {
           const float2 qf = unpack_bf16(qh[u2]), kf = unpack_bf16(kh[u2]);
-          const float e0 = exp2f(xl[c2 * 32 + 2 * u2]), e1 = exp2f(xl[c2 * 32 + 2 * u2 + 1]);
+          const float e0 = ex2a(xl[c2 * 32 + 2 * u2]), e1 = ex2a(xl[c2 * 32 + 2 * u2 + 1]);
           const float t0 = __uint_as_float(a[2 * u2]), t1 = __uint_as_float(a[2 * u2 + 1]);
           out[u2] = pack_bf16(e0 * fmaf(dad, kf.x, t0), e1 * fmaf(dad, kf.y, t1));
           a[2 * u2] = __float_as_uint(qf.x * t0);
@@ -1111,7 +1120,7 @@ __global__ void __launch_bounds__(kThreads, 1) gla_bwd_tc(
 #pragma unroll
         for (int u2 = 0; u2 < 16; ++u2) {
           const float2 qf = unpack_bf16(qh[u2]), kf = unpack_bf16(kh[u2]);
-          const float e0 = exp2f(-xl[c2 * 32 + 2 * u2]), e1 = exp2f(-xl[c2 * 32 + 2 * u2 + 1]);
+          const float e0 = ex2a(-xl[c2 * 32 + 2 * u2]), e1 = ex2a(-xl[c2 * 32 + 2 * u2 + 1]);
           const float a0 = __uint_as_float(ka[2 * u2]), a1 = __uint_as_float(ka[2 * u2 + 1]);
           const float b0 = __uint_as_float(kb[2 * u2]), b1 = __uint_as_float(kb[2 * u2 + 1]);
           out[u2] = pack_bf16(e0 * fmaf(dad, qf.x, a0 + b0), e1 * fmaf(dad, qf.y, a1 + b1));
@@ -1175,29 +1184,42 @@ __global__ void __launch_bounds__(kThreads, 1) gla_bwd_tc(
     {
       const int i = tid & (kD - 1);
       float acc = 0.f;
+      // blocks of 8 rows; the next block's loads go out before this block's
+      // stores (other rows), so each block waits for one load latency only
+      float v[8], w[8];
       if (tid < kD) {
+#pragma unroll
+        for (int u = 0; u < 8; ++u) v[u] = fB[gate_slot(kTile - 8 + u, i)];
 #pragma unroll 1
         for (int t0 = kTile - 8; t0 >= 0; t0 -= 8) {
-          float v[8];
+          if (t0 >= 8) {
 #pragma unroll
-          for (int u = 7; u >= 0; --u) v[u] = fB[gate_slot(t0 + u, i)];
+            for (int u = 0; u < 8; ++u) w[u] = fB[gate_slot(t0 - 8 + u, i)];
+          }
 #pragma unroll
           for (int u = 7; u >= 0; --u) {
             acc += v[u];
             fB[gate_slot(t0 + u, i)] = acc;
           }
+#pragma unroll
+          for (int u = 0; u < 8; ++u) v[u] = w[u];
         }
       } else {
+#pragma unroll
+        for (int u = 0; u < 8; ++u) v[u] = fK[gate_slot(u, i)];
 #pragma unroll 1
         for (int t0 = 0; t0 < kTile; t0 += 8) {
-          float v[8];
+          if (t0 + 8 < kTile) {
 #pragma unroll
-          for (int u = 0; u < 8; ++u) v[u] = fK[gate_slot(t0 + u, i)];
+            for (int u = 0; u < 8; ++u) w[u] = fK[gate_slot(t0 + 8 + u, i)];
+          }
 #pragma unroll
           for (int u = 0; u < 8; ++u) {
             fK[gate_slot(t0 + u, i)] = acc;
             acc += v[u];
           }
+#pragma unroll
+          for (int u = 0; u < 8; ++u) v[u] = w[u];
         }
       }
     }
