@@ -6,9 +6,8 @@
 // states, then B x T x H slots of d log-gate totals, then as many again for
 // segment totals: B*T*H*d*(d+2) floats. The CUDA-core path fills every
 // chunk's slot (P_c, gsum_c). The tensor-core path walks segments of about
-// 1024 tokens: their states (the segment state kernel, which also writes each
-// 128-token tile's log-gate total into the slot of the tile's first chunk)
-// and totals go to the slots of each segment's first chunk, the scan over
+// 1024 tokens: their states and log-gate totals (the segment state kernel) go
+// to the slots of each segment's first chunk, the scan over
 // segments turns them into the states entering the segments, and the walk
 // carries the state through each segment's tiles, leaving in the slot of every
 // tile's first chunk the bf16 operand tile of diag(e^{r}) P (r the tile's
@@ -129,7 +128,7 @@ int lasp_gla_fwd(const void* q, const void* k, const void* v, const float* g, vo
     int* flag = reinterpret_cast<int*>(state_cache + cache_state_floats(B, H, N, d, C));
     if ((s = cuda_status(cudaMemsetAsync(flag, 0, sizeof(int), st)))) return s;
     if ((s = cuda_status(traced(K_GLA_SEG_STATES, st, [&] {
-           return tc_gla_chunk_states(k, v, g, state_cache, gseg, gsum, B, H, N, 0, T, S * stride, 0, S, stride, st,
+           return tc_gla_chunk_states(k, v, g, state_cache, gseg, nullptr, B, H, N, 0, T, S * stride, 0, S, stride, st,
                                       flag);
          }))))
       return s;
