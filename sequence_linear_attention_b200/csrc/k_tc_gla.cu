@@ -724,18 +724,20 @@ struct SmemBwd {
 // (LASP Appendix A.4: the gated form of the gradient-state recurrence):
 //   R_{c-1} = diag(e^{b_end}) R_c + diag(e^{r}) Q^^T dO     (Q^ = q . e^{b - r})
 // with Q^^T dO an extra MMA of phase 2 into T0 (idle between epilogue 1 and
-// phase 3), combined in fp32 at the start of epilogue 2 with R_c read back
-// from L2, and written to a scratch slot of the segment (the workspace slot
-// of its first chunk), where the next tile's bulk load of R finds it. The
-// scratch is lane-major (float4 group g of state row m at float4 g * 128 + m),
-// so that the threads of a warp, which own consecutive rows, read and write
-// one 512-byte run per access; the scan's slot is row-major. Most
+// phase 3), combined in fp32 with R_c while phase 3's first MMAs run, and
+// written to a scratch slot of the segment (the workspace slot of its first
+// chunk), where the next tile's bulk load of R finds it. The scratch is
+// lane-major (float4 group g of state row m at float4 g * 128 + m), so that
+// the threads of a warp, which own consecutive rows, read and write one
+// 512-byte run per access; the scan's slot is row-major, so a segment's last
+// tile first copies its R_c into the scratch, and the combination always reads
+// R_c from there (L2). Most
 // barriers complete once per tile, so their parity flips from tile to tile;
 // mmar only on tiles that form a state. Shared memory: Q^, K^, V, dO (then, in pairs,
 // the fp32 tiles of dB and k . dk^inter for the log-gate gradient's column
 // sums), X (P', loaded as the output kernel cached it, then R'), and the pair
 // sA / sB (the gate tile during the walk; then dA . strict and A . causal;
-// then the dK and dV outputs). TMEM: T0 = dO V^T -> (dA . strict)^T Q^;
+// then the dK and dV outputs). TMEM: T0 = dO V^T -> Q^^T dO -> (dA . strict)^T Q^;
 // T1 = Q^ K^^T -> dV; T2 = dO P'^T + (dA . strict) K^ -> q . dq'; T3 = log2 E
 // -> V R'^T.
 __global__ void __launch_bounds__(kThreads, 1) gla_bwd_tc(
