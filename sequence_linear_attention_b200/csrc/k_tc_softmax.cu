@@ -34,9 +34,9 @@
 // TMEM, then (sixteen epilogue warps, 32 query columns each) P^T and dS^T in
 // bf16, then dV += P^T dO and dK += dS^T Q; Q and dO stream through a
 // three-slot ring so that the next Q tile loads during the current tile.
-// softmax_dq_tc: one CTA per 128-query tile walks its key tiles, each in two
-// halves of 64 keys: S = Q K^T, dP = dO V^T, dS, dQ += dS K. Only the tiles
-// on the causal diagonal mask element by element. The two gradient kernels
+// softmax_dq_tc: one CTA per 128-query tile walks its key tiles: S = Q K^T,
+// dP = dO V^T, dS (sixteen epilogue warps), dQ += dS K. Only the tiles on the
+// causal diagonal mask element by element. The two gradient kernels
 // recompute P separately, so no atomics are needed and the results do not
 // depend on scheduling.
 #include <algorithm>
@@ -689,26 +689,14 @@ __global__ void __launch_bounds__(kDkdvThreads, 1) softmax_dkdv_tc(
   if (warp == 0) tmem_dealloc(tmem, 512);
 }
 
-// softmax_dq_tc works on each key tile in two halves of 64 keys, so that the
-// epilogue of one half runs while the tensor pipe computes the other half's S
-// and dP and the previous half's dQ update. TMEM: S_h at 128 h, dP_h at
-// 128 h + 64 (h = 0, 1), dQ at 256. Per key tile j the MMA thread issues
-//   S_0, dP_0 (once the epilogue has read half 0 of tile j - 1)
-//   dQ += dS_1 K_{j-1,1}  (once half 1 of tile j - 1 is written)
-//   S_1, dP_1 (once the epilogue has read half 1 of tile j - 1)
-//   dQ += dS_0 K_{j,0}    (once half 0 of tile j is written)
-// and the epilogue takes the halves in order: dS_h of tile j goes into
-// columns 64 h.. of the dS tile once the dQ MMA of tile j - 1 has read them.
-// Sixteen epilogue warps (four per TMEM lane quarter, 16 columns of a half
-// each) keep the exponentials' latency covered; only the tile on the causal
+// softmax_dq_tc: per key tile j, S = Q K_j^T and dP = dO V_j^T (N = 128) into
+// TMEM, the epilogue's sixteen warps (four per TMEM lane quarter, 32 key
+// columns each: chunk sub & 1 of column half sub >> 1) turn them into dS in
+// bf16, and dQ += dS K_j takes the K-steps 0, 1, 4, 5 once the first chunks are
+// written and 2, 3, 6, 7 once the second ones are. Only the tile on the causal
 // diagonal masks element by element.
 struct SmemDq {
-  uint64_t qd_full, k_full[2], v_full[2], kv_empty[2];
-  uint64_t s_full[2];    // MMA -> epilogue: S_h and dP_h are in TMEM
-  uint64_t t_free[2];    // epilogue -> MMA: TMEM half h has been read (512 arrivals)
-  uint64_t ds_ready[2];  // epilogue -> MMA: dS_h is in shared memory (512 arrivals)
-  uint64_t ds_free[2];   // MMA -> epilogue: the dQ MMA has read dS_h
-  uint64_t drain;
+  uint64_t qd_full, k_full[2], v_full[2], kv_empty[2], s_full, ds_half, ds_full, dq_done, drain;
   uint32_t tmem_base;
   int abort;
 };
@@ -724,7 +712,7 @@ __global__ void __launch_bounds__(kDqThreads, 1) softmax_dq_tc(
   uint8_t* sO = base + kTileBytes;      // dO
   uint8_t* sK = base + 2 * kTileBytes;  // two stages
   uint8_t* sV = base + 4 * kTileBytes;  // two stages
-  uint8_t* sDS = base + 6 * kTileBytes;  // dS: keys 0-63 in the first box, 64-127 in the second
+  uint8_t* sDS = base + 6 * kTileBytes;
   SmemDq* s = reinterpret_cast<SmemDq*>(base + 7 * kTileBytes);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int qt = qtiles - 1 - (int)blockIdx.x;  // heaviest tiles first
@@ -734,7 +722,6 @@ __global__ void __launch_bounds__(kDqThreads, 1) softmax_dq_tc(
   const int nkv = (int)(last_pos / kTile) + 1;
   const volatile int* abort_flag = &s->abort;
   const float c2 = scale * kLog2e;
-  constexpr uint32_t kHalfRows = 64 * 128;  // byte offset of row 64 in a 128-byte-swizzled box
 
   if (tid == 0) {
     prefetch_tmap(&map_q);
@@ -747,11 +734,11 @@ __global__ void __launch_bounds__(kDqThreads, 1) softmax_dq_tc(
       mbar_init(&s->k_full[st], 1);
       mbar_init(&s->v_full[st], 1);
       mbar_init(&s->kv_empty[st], 1);
-      mbar_init(&s->s_full[st], 1);
-      mbar_init(&s->t_free[st], kDqEpi);
-      mbar_init(&s->ds_ready[st], kDqEpi);
-      mbar_init(&s->ds_free[st], 1);
     }
+    mbar_init(&s->s_full, 1);
+    mbar_init(&s->ds_half, kDqEpi / 2);
+    mbar_init(&s->ds_full, kDqEpi / 2);
+    mbar_init(&s->dq_done, 1);
     mbar_init(&s->drain, 1);
     s->abort = 0;
     fence_mbar_init();
@@ -764,7 +751,7 @@ __global__ void __launch_bounds__(kDqThreads, 1) softmax_dq_tc(
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = s->tmem_base;
-  constexpr uint32_t kColQ = 256;  // S_h at 128 h, dP_h at 128 h + 64
+  constexpr uint32_t kColS = 0, kColP = 128, kColQ = 256;
 
   if (warp == 16) {
     if (lane == 0) {
@@ -799,53 +786,56 @@ __global__ void __launch_bounds__(kDqThreads, 1) softmax_dq_tc(
     }
   } else if (warp == 17) {
     if (lane == 0) {
-      constexpr uint32_t id_s = idesc_bf16(128, 64, 0, 0);   // S_h, dP_h: 64 keys
-      constexpr uint32_t id_q = idesc_bf16(128, 128, 0, 1);  // dQ += dS_h K_h: K = 64 keys
+      constexpr uint32_t id_kk = idesc_bf16(128, 128, 0, 0);
+      constexpr uint32_t id_kn = idesc_bf16(128, 128, 0, 1);
       const uint32_t aQ = smem_u32(sQ), aO = smem_u32(sO), aD = smem_u32(sDS);
       bool bad = !mbar_wait_or_abort(&s->qd_full, 0, SITE_BWD_TMA, abort_flag);
-      // dQ += dS_hh K_{jj,hh}, once the epilogue has written dS_hh of key tile jj
-      auto dq_mma = [&](int jj, int hh) {
-        if (!mbar_wait_or_abort(&s->ds_ready[hh], (uint32_t)jj & 1u, SITE_BWD_MMA, abort_flag)) return false;
-        tc_fence_after();
-        const uint32_t aKh = smem_u32(sK + (jj & 1) * kTileBytes) + hh * kHalfRows;
-        for (int kk = 0; kk < 4; ++kk)
-          mma_bf16(tmem + kColQ, kmaj(aD + hh * kBox, kk), mnmaj(aKh, kk), id_q, (jj > 0 || hh > 0 || kk > 0) ? 1u : 0u);
-        mma_commit(&s->ds_free[hh]);
-        if (hh == 1) mma_commit(&s->kv_empty[jj & 1]);  // K_jj and V_jj are read
-        return true;
-      };
       for (int j = 0; j < nkv && !bad; ++j) {
         const int st = j & 1;
         const uint32_t use = (uint32_t)(j >> 1) & 1u;
         const uint32_t aK = smem_u32(sK + st * kTileBytes), aV = smem_u32(sV + st * kTileBytes);
-        if (!mbar_wait_or_abort(&s->k_full[st], use, SITE_BWD_TMA, abort_flag) ||
-            !mbar_wait_or_abort(&s->v_full[st], use, SITE_BWD_TMA, abort_flag)) {
+        if (!mbar_wait_or_abort(&s->k_full[st], use, SITE_BWD_TMA, abort_flag)) {
           bad = true;
           break;
         }
-        for (int hh = 0; hh < 2 && !bad; ++hh) {
-          if (j > 0 && !mbar_wait_or_abort(&s->t_free[hh], (uint32_t)(j - 1) & 1u, SITE_BWD_MMA, abort_flag)) {
-            bad = true;
+        tc_fence_after();
+        for (int kk = 0; kk < kD / 16; ++kk) mma_bf16(tmem + kColS, kmaj(aQ, kk), kmaj(aK, kk), id_kk, kk > 0);
+        if (!mbar_wait_or_abort(&s->v_full[st], use, SITE_BWD_TMA, abort_flag)) {
+          bad = true;
+          break;
+        }
+        tc_fence_after();
+        for (int kk = 0; kk < kD / 16; ++kk) mma_bf16(tmem + kColP, kmaj(aO, kk), kmaj(aV, kk), id_kk, kk > 0);
+        mma_commit(&s->s_full);
+        // dQ += dS K over the key columns the epilogue has finished: K-steps
+        // 0, 1, 4, 5 (the first chunks), then 2, 3, 6, 7
+        bool part_ok = true;
+        for (int pc = 0; pc < 2; ++pc) {
+          if (!mbar_wait_or_abort(pc == 0 ? &s->ds_half : &s->ds_full, (uint32_t)j & 1u, SITE_BWD_MMA, abort_flag)) {
+            part_ok = false;
             break;
           }
           tc_fence_after();
-          const uint32_t colS = (uint32_t)hh * 128;
-          for (int kk = 0; kk < kD / 16; ++kk)
-            mma_bf16(tmem + colS, kmaj(aQ, kk), kmaj(aK + hh * kHalfRows, kk), id_s, kk > 0);
-          for (int kk = 0; kk < kD / 16; ++kk)
-            mma_bf16(tmem + colS + 64, kmaj(aO, kk), kmaj(aV + hh * kHalfRows, kk), id_s, kk > 0);
-          mma_commit(&s->s_full[hh]);
-          if (hh == 0 ? (j > 0 && !dq_mma(j - 1, 1)) : !dq_mma(j, 0)) bad = true;
+          for (int q = 0; q < 4; ++q) {
+            const int kk = (q >> 1) * 4 + pc * 2 + (q & 1);
+            mma_bf16(tmem + kColQ, kmaj(aD, kk), mnmaj(aK, kk), id_kn, (j > 0 || pc > 0 || q > 0) ? 1u : 0u);
+          }
         }
+        if (!part_ok) {
+          bad = true;
+          break;
+        }
+        mma_commit(&s->kv_empty[st]);
+        mma_commit(&s->dq_done);
       }
-      if (!bad && nkv > 0 && !dq_mma(nkv - 1, 1)) bad = true;
       if (bad) s->abort = 1;
       mma_commit(&s->drain);
       mbar_wait(&s->drain, 0, SITE_BWD_MMA);
     }
   } else {
-    // query row `row` of the tile; this thread's 16 key columns sub * 16.. of each half
+    // query row `row` of the tile; key columns sub * 32 .. + 31 (two passes of 16)
     const int row = (warp & 3) * 32 + lane, sub = warp >> 2;
+    const int cc = sub & 1;
     const uint32_t lane_base = tmem + ((uint32_t)((warp & 3) * 32) << 16);
     const int64_t qi = q0 + row;
     const int64_t qpos = q_offset + qi;
@@ -854,54 +844,52 @@ __global__ void __launch_bounds__(kDqThreads, 1) softmax_dq_tc(
     const float dl = in ? delta[((int64_t)b * H + h) * Nq + qi] : 0.f;
     bool bad = false;
     for (int j = 0; j < nkv; ++j) {
-      for (int hh = 0; hh < 2; ++hh) {
-        const int64_t kc = (int64_t)j * kTile + hh * 64 + sub * 16;  // key of this thread's first column
-        // columns u <= lim are inside the causal mask (lim >= 15: all, < 0: none)
-        const int64_t lim64 = in ? qpos - kc : -1;
-        const int lim = lim64 < -1 ? -1 : (lim64 > 15 ? 15 : (int)lim64);
-        if (!bad && !mbar_wait_or_abort(&s->s_full[hh], (uint32_t)j & 1u, SITE_BWD_MMA, abort_flag)) bad = true;
-        // dS_hh's columns are free once the dQ MMA of the last key tile has read them
-        if (j > 0 && !bad && !mbar_wait_or_abort(&s->ds_free[hh], (uint32_t)(j - 1) & 1u, SITE_BWD_MMA, abort_flag))
-          bad = true;
-        bad = __any_sync(0xffffffffu, bad);  // the TMEM loads below are warp-collective
-        uint32_t rs[16], rp[16];
-        if (!bad) {
-          tc_fence_after();
-          tmem_ld16(lane_base + hh * 128 + sub * 16, rs);
-          tmem_ld16(lane_base + hh * 128 + 64 + sub * 16, rp);
+      const int64_t kc = (int64_t)j * kTile + sub * 32;  // key of this thread's first column
+      // columns u <= lim are inside the causal mask (lim >= 31: all, < 0: none)
+      const int64_t lim64 = in ? qpos - kc : -1;
+      const int lim = lim64 < -1 ? -1 : (lim64 > 31 ? 31 : (int)lim64);
+      if (!bad && !mbar_wait_or_abort(&s->s_full, (uint32_t)j & 1u, SITE_BWD_MMA, abort_flag)) bad = true;
+      if (j > 0 && !bad && !mbar_wait_or_abort(&s->dq_done, (uint32_t)(j - 1) & 1u, SITE_BWD_MMA, abort_flag))
+        bad = true;  // the last dQ MMA has read dS
+      bad = __any_sync(0xffffffffu, bad);  // the TMEM loads below are warp-collective
+      if (!bad) {
+        tc_fence_after();
+#pragma unroll 1
+        for (int ps = 0; ps < 2; ++ps) {
+          const int cb = sub * 32 + ps * 16;
+          uint32_t rs[16], rp[16];
+          tmem_ld16(lane_base + kColS + cb, rs);
+          tmem_ld16(lane_base + kColP + cb, rp);
           tmem_ld_wait();
-        }
-        tc_fence_before();
-        mbar_arrive(&s->t_free[hh]);  // the MMA may refill this TMEM half
-        if (!bad) {
+          const int lp = lim - ps * 16;  // this pass's columns u <= lp are inside the mask
           float ds[16];
-          if (lim >= 15) {
+          if (lp >= 15) {
 #pragma unroll
             for (int u = 0; u < 16; ++u)
               ds[u] = ex2(__uint_as_float(rs[u]) * c2 - lse2) * (__uint_as_float(rp[u]) - dl);
-          } else if (lim < 0) {
+          } else if (lp < 0) {
 #pragma unroll
             for (int u = 0; u < 16; ++u) ds[u] = 0.f;
           } else {
 #pragma unroll
             for (int u = 0; u < 16; ++u) {
-              const float p = u <= lim ? ex2(__uint_as_float(rs[u]) * c2 - lse2) : 0.f;
+              const float p = u <= lp ? ex2(__uint_as_float(rs[u]) * c2 - lse2) : 0.f;
               ds[u] = p * (__uint_as_float(rp[u]) - dl);
             }
           }
 #pragma unroll
           for (int q8 = 0; q8 < 2; ++q8)
-            st_tile16(sDS, row, hh * 64 + sub * 16 + q8 * 8,
+            st_tile16(sDS, row, cb + q8 * 8,
                       make_uint4(pack_bf16(ds[q8 * 8], ds[q8 * 8 + 1]), pack_bf16(ds[q8 * 8 + 2], ds[q8 * 8 + 3]),
                                  pack_bf16(ds[q8 * 8 + 4], ds[q8 * 8 + 5]),
                                  pack_bf16(ds[q8 * 8 + 6], ds[q8 * 8 + 7])));
         }
-        fence_async_smem();
-        mbar_arrive(&s->ds_ready[hh]);
       }
+      fence_async_smem();
+      tc_fence_before();
+      mbar_arrive(cc == 0 ? &s->ds_half : &s->ds_full);  // the MMA takes each chunk group as it is done
     }
-    // the last dQ MMA (half 1 of the last key tile) follows every other
-    if (!bad && !mbar_wait_or_abort(&s->ds_free[1], (uint32_t)(nkv - 1) & 1u, SITE_BWD_MMA, abort_flag)) bad = true;
+    if (!bad && !mbar_wait_or_abort(&s->dq_done, (uint32_t)(nkv - 1) & 1u, SITE_BWD_MMA, abort_flag)) bad = true;
     bad = __any_sync(0xffffffffu, bad);
     if (bad) s->abort = 1;
     if (!bad) {
