@@ -428,10 +428,7 @@ def run_gpu(args, rank, world, local):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "bf16" if bf16 else "f32", "data": "synthetic (seeded normal q,k,v,dO; no dataset)",
-        "config": {"workload": args.workload, "B": B, "H": H, "N": N, "d": d, "C": C, "segment": G,
-                   "decay": "per-head 1-2^-(5+8h/H)" if w["decayed"] else "none",
-                   "l2": "inputs larger than L2 (q, k, v, dO are 4 x %d MiB)" % (B * N * H * d * elem >> 20),
-                   "parallelism": f"replicas x{world} (independent sequences, no collective)"},
+        "config": dict(workload_config(args.workload, w, N, world), segment=G),
         "tflops": round(tflops, 2),
         "tensor_peak_frac": round(tflops / (peaks["bf16"] if burst else peaks["bf16_sustained"]), 4),
         "tensor_peak_basis": "burst" if burst else "sustained",
@@ -935,6 +932,16 @@ def cpu_baseline_gated(args):
             "sample": f"fp64 oracle gated fwd+bwd, batch 0, all heads, first {tokens} positions"}
 
 
+def workload_config(name: str, w: dict, N: int, world: int) -> dict:
+    """The `config` of the main line and of the reference arm: the workload,
+    its shape and decay, how the inputs relate to L2, and the multi-GPU mode."""
+    elem = 2 if w["bf16"] else 4
+    return {"workload": name, "B": w["B"], "H": w["H"], "N": N, "d": w["d"], "C": w["C"],
+            "decay": "per-head 1-2^-(5+8h/H)" if w["decayed"] else "none",
+            "l2": "inputs larger than L2 (q, k, v, dO are 4 x %d MiB)" % (w["B"] * N * w["H"] * w["d"] * elem >> 20),
+            "parallelism": f"replicas x{world} (independent sequences, no collective)"}
+
+
 def run_reference(args, rank, world):
     if rank != 0:
         return None
@@ -956,8 +963,7 @@ def run_reference(args, rank, world):
         "impl": "reference", "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(dt * 1e3 / args.steps, 3),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-        "data": "synthetic", "config": {"workload": args.workload, "B": w["B"], "H": w["H"], "N": w["N"],
-                                         "d": w["d"], "C": w["C"]},
+        "data": "synthetic", "config": workload_config(args.workload, w, w["N"], world),
         "cpu_baseline": {"value": round(value, 1), "unit": "tokens/s", "kind": "oracle",
                          "cores": __import__("oracle").num_threads(), "sample": sample},
         "e2e": {"value": round(value, 1), "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
