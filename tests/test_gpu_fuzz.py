@@ -114,3 +114,19 @@ def test_random_gated_shapes_against_oracle(i):
     ref = _reference(inp, g, init=None if c["init"] is None else c["init"].astype(np.float64),
                      dstate_in=None if c["din"] is None else c["din"].astype(np.float64))
     _compare(got, ref, tol(c["bf16"]))
+
+
+# ---------------------------------------------------------------- bidirectional form
+def _bidir_draw(i: int):
+    rng = np.random.default_rng([20261205, i])
+    return int(rng.integers(1, 3)), int(rng.integers(1, 6)), 128 * int(rng.integers(1, 33)), 6000 + i
+
+
+@pytest.mark.parametrize("i", range(12), ids=lambda i: "{}-B{}H{}N{}".format(i, *_bidir_draw(i)[:3]))
+def test_random_bidirectional_shapes_against_oracle(i):
+    """The unmasked form (bf16, d = 128) on random batch, head and token counts
+    (one to thirty-two 128-token tiles: one or several segments)."""
+    from test_gpu_bidir import _check, _run
+    B, H, N, seed = _bidir_draw(i)
+    inp = lasp_inputs.make_inputs(B, N, H, 128, seed=seed, bf16=True, decayed=False)
+    _check(_run(inp), inp)
