@@ -30,8 +30,9 @@
 // tile and records LASP_ERR_INVALID_ARG (site SITE_GATE_RANGE) if not; the
 // CUDA-core kernels have no such limit.
 //
-// Thread layout (256 threads): warp w owns tile rows / TMEM lanes 32*(w%4)..
-// and the column half w/4 of every row-wise step. The cumulative log-gates:
+// Thread layout (256 threads; 512 in the gradient kernel): warp w owns tile
+// rows / TMEM lanes 32*(w%4).. and the column half (quarter) w/4 of every
+// row-wise step. The cumulative log-gates:
 // the state kernel sums them by 16-row groups (a warp per group, float4 loads)
 // and scales its operand in place; the output and backward kernels load the
 // gate tile by TMA and walk it in shared memory (a feature and half the rows
@@ -60,7 +61,7 @@ constexpr float kMaxSpan = 80.f;  // largest |b_t - r| (natural log) the factori
 // kMaxSpan, so that no rounding of the two different sums lets a tile past it
 // that the output and backward kernels would then reject
 constexpr float kSpanCheck = kMaxSpan - 1.f;
-constexpr uint32_t kBarAll = 1;   // named barrier over all 256 threads
+constexpr uint32_t kBarAll = 1;   // named barrier over all threads of the CTA
 
 // 2^x by the hardware's approximate exponential (relative error near 2^-22;
 // results below 2^-126 flush to zero). Every exponent here is a difference of
@@ -706,14 +707,95 @@ cleanup:
   if (warp == 0) tmem_dealloc(tmem, 512);
 }
 
+constexpr int kBwdThreads = 512;  // the gradient kernel: four warps per TMEM lane quadrant
+
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]),
+        "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+}
+
+__device__ __forceinline__ void tmem_ld8(uint32_t taddr, uint32_t (&r)[8]) {
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
+               : "r"(taddr));
+}
+
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&r)[8]) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"r"(taddr),
+               "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+               : "memory");
+}
+
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+      "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]),
+      "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+      : "memory");
+}
+
+// Multiplies the 32 bf16 entries of row `row`, columns qt*32.., of a tile by
+// exp2(sgn * x[u]) (x in log2 units), in place.
+__device__ __forceinline__ void scale_row_quarter(uint8_t* tile, int row, int qt, const float (&x)[32], float sgn) {
+#pragma unroll
+  for (int c8 = 0; c8 < 4; ++c8) {
+    uint4* p = tile16(tile, row, qt * 32 + c8 * 8);
+    uint4 w = *p;
+    uint32_t* e = reinterpret_cast<uint32_t*>(&w);
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const float2 f = unpack_bf16(e[u]);
+      e[u] = pack_bf16(f.x * ex2a(sgn * x[c8 * 8 + 2 * u]), f.y * ex2a(sgn * x[c8 * 8 + 2 * u + 1]));
+    }
+    *p = w;
+  }
+}
+
+// gate_rows for the gradient kernel's 512 threads: threads 0-255 walk the gate
+// tile (as walk_tile), then every thread takes row t, columns qt*32.., with
+// the same range check, and returns x = (b_t - r) log2 e for them.
+__device__ __forceinline__ bool gate_rows_quarter(float* bt, uint64_t* gbar, uint32_t parity, int* abort,
+                                                  unsigned int site, float* r, float* dend, int tid, int t, int qt,
+                                                  float (&x)[32]) {
+  const bool landed = mbar_wait(gbar, parity, site);
+  if (!landed) *abort = 1;
+  if (tid < 2 * kD) walk_tile(bt, tid, r, dend);
+  named_sync(kBarAll, kBwdThreads);
+#pragma unroll
+  for (int q = 0; q < 8; ++q) {
+    const float4 v = *reinterpret_cast<const float4*>(bt + qt * (kTile * 32) + t * 32 + 4 * (q ^ (t & 7)));
+    x[4 * q] = v.x;
+    x[4 * q + 1] = v.y;
+    x[4 * q + 2] = v.z;
+    x[4 * q + 3] = v.w;
+  }
+  const bool first = t < kTile / 2;  // rows of the second half already hold b_t - r
+  bool ok = true;
+#pragma unroll
+  for (int u = 0; u < 32; ++u) {
+    const float y = first ? x[u] - r[qt * 32 + u] : x[u];
+    ok = ok && fabsf(y) <= kMaxSpan;
+    x[u] = y * kLog2e;
+  }
+  if (!ok) record_error(LASP_ERR_INVALID_ARG, SITE_GATE_RANGE);
+  return landed;
+}
+
 // ---------------------------------------------------------------- gradients
 struct SmemBwd {
   uint64_t gload, load, ldr, mma1a, mma1b, mma2, mma3, mmar;
   uint32_t tmem_base;
   int abort;
-  alignas(16) float dAd[kTile];  // do_t . v_t, the diagonal of dO V^T
-  alignas(16) float bnd[kD];     // e^{b_end[i]} <R_c[i], P_c[i]>, the sum over the first half of the columns
-  alignas(16) float bnd2[kD];    // ... and over the second half (both read as float4)
+  // do_t . v_t, the diagonal of dO V^T (epilogues 1-3); then, per feature,
+  // the sum of dB over rows 64-127 plus bnd (the column walks' carry)
+  alignas(16) float dAd[kTile];
+  alignas(16) float bnd[kD];  // e^{b_end[i]} <R_c[i], P_c[i]>
+  alignas(16) float cK[kD];   // per feature, the sum of k . dk^inter over rows 0-63 (the other carry)
 };
 
 // One persistent CTA per SM, taking segments of S 128-token tiles in launch
@@ -740,7 +822,11 @@ struct SmemBwd {
 // then the dK and dV outputs). TMEM: T0 = dO V^T -> Q^^T dO -> (dA . strict)^T Q^;
 // T1 = Q^ K^^T -> dV; T2 = dO P'^T + (dA . strict) K^ -> q . dq'; T3 = log2 E
 // -> V R'^T.
-__global__ void __launch_bounds__(kThreads, 1) gla_bwd_tc(
+//
+// 512 threads: warp w owns tile rows / TMEM lanes 32*(w%4).. and the column
+// quarter w/4 (32 columns) of every row-wise step; the column walks give each
+// feature four threads (two sums, each over two halves of the rows).
+__global__ void __launch_bounds__(kBwdThreads, 1) gla_bwd_tc(
     const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
     const __grid_constant__ CUtensorMap map_v, const __grid_constant__ CUtensorMap map_do,
     const __grid_constant__ CUtensorMap map_dk, const __grid_constant__ CUtensorMap map_dv,
@@ -763,7 +849,7 @@ __global__ void __launch_bounds__(kThreads, 1) gla_bwd_tc(
   float* sr = s->dAd;
   float* sdend = s->bnd;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int t = (warp & 3) * 32 + lane, half = warp >> 2;
+  const int t = (warp & 3) * 32 + lane, qt = warp >> 2, cq = qt * 32;
   // this CTA's k-th tile: tile j = S - 1 - k % S (128 tokens c * 128.., c =
   // seg * S + j) of segment item blockIdx.x + (k / S) * grid (segment seg of
   // head h of sequence b)
@@ -836,6 +922,9 @@ __global__ void __launch_bounds__(kThreads, 1) gla_bwd_tc(
   uint32_t ph = 0;       // parity of every barrier's phase for this CTA's current tile
   uint32_t rph = 0;      // parity of mmar's next phase
   bool r_ahead = false;  // thread 0: R's load into sA/sB is in flight
+  // thread 0: the parity of the gate tile's and the token tiles' loads still
+  // in flight (issued, not yet waited for), or -1; cleanup waits for them
+  int gate_out = my_tiles > 0 ? 0 : -1, tok_out = gate_out;
   for (int64_t k = 0; k < my_tiles; ++k, ph ^= 1u) {
   int c, h, b, j;
   tile_of(k, c, h, b, j);
@@ -845,29 +934,30 @@ __global__ void __launch_bounds__(kThreads, 1) gla_bwd_tc(
   const bool has_next = k + 1 < my_tiles;  // this CTA's next tile
   const bool form = j > 0;  // this tile forms R_{c-1} for the tile before it
   // ---- phase 0: gates, Q^, K^, log2 E -> T3, P' -> X
-  float x[64];
-  gate_rows(bt, &s->gload, ph, &s->abort, SITE_BWD_TMA, sr, sdend, tid, t, half, x);
+  float x[32];
+  if (gate_rows_quarter(bt, &s->gload, ph, &s->abort, SITE_BWD_TMA, sr, sdend, tid, t, qt, x) && tid == 0)
+    gate_out = -1;
   // e^{r}, e^{b_end - r} and e^{b_end} of state row t (feature t)
   const float er = ex2a(sr[t] * kLog2e), wt = ex2a(sdend[t] * kLog2e), eb = er * wt;
-  named_sync(kBarAll, kThreads);  // every row of the gate tile has been read
+  named_sync(kBarAll, kBwdThreads);  // every row of the gate tile has been read
   if (tid == 0) {
     // R_c (fp32) into the gate tile's space while the token tiles arrive
     mbar_arrive_expect_tx(&s->ldr, kD * kD * 4);
     bulk_load(bt, R + rslot * kD * kD, kD * kD * 4, &s->ldr);
     r_ahead = true;
   }
-  if (!mbar_wait(&s->load, ph, SITE_BWD_TMA)) s->abort = 1;
-  scale_row_half(sQ, t, half, x, 1.f);   // Q^ = q . E
-  scale_row_half(sK, t, half, x, -1.f);  // K^ = k / E
+  if (mbar_wait(&s->load, ph, SITE_BWD_TMA)) {
+    if (tid == 0) tok_out = -1;
+  } else {
+    s->abort = 1;
+  }
+  scale_row_quarter(sQ, t, qt, x, 1.f);   // Q^ = q . E
+  scale_row_quarter(sK, t, qt, x, -1.f);  // K^ = k / E
   {
-    uint32_t r0[32], r1[32];
+    uint32_t r0[32];
 #pragma unroll
-    for (int u = 0; u < 32; ++u) {
-      r0[u] = __float_as_uint(x[u]);
-      r1[u] = __float_as_uint(x[32 + u]);
-    }
-    tmem_st32(lane_base + T3 + half * 64, r0);
-    tmem_st32(lane_base + T3 + half * 64 + 32, r1);
+    for (int u = 0; u < 32; ++u) r0[u] = __float_as_uint(x[u]);
+    tmem_st32(lane_base + T3 + cq, r0);
     tmem_st_wait();
   }
   fence_async_smem();
@@ -880,32 +970,33 @@ __global__ void __launch_bounds__(kThreads, 1) gla_bwd_tc(
     constexpr uint32_t id_kk = idesc_bf16(128, 128, 0, 0);
     constexpr uint32_t id_kn = idesc_bf16(128, 128, 0, 1);
     constexpr uint32_t id_nn = idesc_bf16(128, 128, 1, 1);
-    // ---- phase 1: T0 = dO V^T, T1 = Q^ K^^T | T2 = dO P'^T
+    // ---- phase 1: T2 = dO P'^T | T0 = dO V^T, T1 = Q^ K^^T (P' first, so that
+    // X takes R' while the other two run)
     if (tid == 0) {
       tc_fence_after();
+      for (int kk = 0; kk < kD / 16; ++kk) mma_bf16(tmem + T2, kmaj(aD, kk), kmaj(aX, kk), id_kk, kk != 0);
+      mma_commit(&s->mma1b);
       for (int kk = 0; kk < kD / 16; ++kk) mma_bf16(tmem + T0, kmaj(aD, kk), kmaj(aV, kk), id_kk, kk != 0);
       for (int kk = 0; kk < kD / 16; ++kk) mma_bf16(tmem + T1, kmaj(aQ, kk), kmaj(aK, kk), id_kk, kk != 0);
       mma_commit(&s->mma1a);
-      for (int kk = 0; kk < kD / 16; ++kk) mma_bf16(tmem + T2, kmaj(aD, kk), kmaj(aX, kk), id_kk, kk != 0);
-      mma_commit(&s->mma1b);
     }
-    // while the MMAs run: row t of R (fp32, from sA/sB; this thread's half of
-    // the columns) into registers, and that half of <R'_t, P'_t> = e^{b_end_t}
-    // <R_t, P_t> into bnd / bnd2, with row t of P' read in X (bf16)
+    // while the MMAs run: row t of R (fp32, from sA/sB; this thread's quarter
+    // of the columns) into registers, and that quarter of <R'_t, P'_t> =
+    // e^{b_end_t} <R_t, P_t>, with row t of P' read in X (bf16)
     {
       const bool rok = mbar_wait(&s->ldr, ph, SITE_BWD_TMA);
       if (!rok) s->abort = 1;
       if (tid == 0 && rok) r_ahead = false;  // else cleanup waits for it once more
     }
-    // R_c, row t, columns half * 64.. (float4 groups g = half * 16 + u):
-    // row-major from the scan's slot, lane-major from the scratch
-    float4 rreg[16];
+    // R_c, row t, columns cq.. (float4 groups g = qt * 8 + u): row-major from
+    // the scan's slot, lane-major from the scratch
+    float4 rreg[8];
     {
       const bool rlm = j != S - 1;
       const float4* R4 = reinterpret_cast<const float4*>(bt);
 #pragma unroll
-      for (int u = 0; u < 16; ++u) {
-        const int g = half * 16 + u;
+      for (int u = 0; u < 8; ++u) {
+        const int g = qt * 8 + u;
         rreg[u] = R4[rlm ? g * kD + t : t * (kD / 4) + g];
       }
       if (form && !rlm) {
@@ -913,38 +1004,56 @@ __global__ void __launch_bounds__(kThreads, 1) gla_bwd_tc(
         // tile's own forming of R_{c-1} reads it back in one-run accesses
         float4* rs = reinterpret_cast<float4*>(R + pslot_of(c - j, h, b) * kD * kD);
 #pragma unroll
-        for (int u = 0; u < 16; ++u) rs[(half * 16 + u) * kD + t] = rreg[u];
+        for (int u = 0; u < 8; ++u) rs[(qt * 8 + u) * kD + t] = rreg[u];
       }
     }
-    named_sync(kBarAll, kThreads);  // every row of R has been read: the masks may overwrite sA/sB
+    named_sync(kBarAll, kBwdThreads);  // every row of R has been read: sA/sB are free
     {
-      // e^{b_end - r} <R_t, P'_t> over this thread's half of the columns (P' row t in X, bf16)
+      // e^{b_end - r} <R_t, P'_t> over this thread's quarter of the columns (P'
+      // row t in X, bf16); the four quarters' sums meet in sA, one thread per
+      // feature adds them into bnd before the masks overwrite sA
       float dot = 0.f;
 #pragma unroll
-      for (int q8 = 0; q8 < 8; ++q8) {
-        const uint4 pw = *tile16(sX, t, half * 64 + q8 * 8);
+      for (int q8 = 0; q8 < 4; ++q8) {
+        const uint4 pw = *tile16(sX, t, cq + q8 * 8);
         const float2 p0 = unpack_bf16(pw.x), p1 = unpack_bf16(pw.y), p2 = unpack_bf16(pw.z), p3 = unpack_bf16(pw.w);
         const float4 a = rreg[2 * q8], b2 = rreg[2 * q8 + 1];
         dot += p0.x * a.x + p0.y * a.y + p1.x * a.z + p1.y * a.w + p2.x * b2.x + p2.y * b2.y + p3.x * b2.z +
                p3.y * b2.w;
       }
-      (half ? s->bnd2 : s->bnd)[t] = dot * wt;
+      float* part = reinterpret_cast<float*>(sA);
+      part[qt * kD + t] = dot * wt;
+      named_sync(kBarAll, kBwdThreads);
+      if (tid < kD) s->bnd[tid] = (part[tid] + part[kD + tid]) + (part[2 * kD + tid] + part[3 * kD + tid]);
+      named_sync(kBarAll, kBwdThreads);
+    }
+    // X is free once dO P'^T has read P': R' = diag(e^{b_end - r}) R_c replaces it
+    if (mbar_wait(&s->mma1b, ph, SITE_BWD_MMA)) {
+#pragma unroll
+      for (int q8 = 0; q8 < 4; ++q8) {
+        const float4 a = rreg[2 * q8], b2 = rreg[2 * q8 + 1];
+        st_tile16(sX, t, cq + q8 * 8,
+                  make_uint4(pack_bf16(a.x * wt, a.y * wt), pack_bf16(a.z * wt, a.w * wt),
+                             pack_bf16(b2.x * wt, b2.y * wt), pack_bf16(b2.z * wt, b2.w * wt)));
+      }
+    } else {
+      s->abort = 1;
     }
     // ---- epilogue 1: dA . strict -> sA, A . causal -> sB, the diagonal of dA
     if (mbar_wait(&s->mma1a, ph, SITE_BWD_MMA)) {
       tc_fence_after();
 #pragma unroll 1
       for (int c2 = 0; c2 < 2; ++c2) {
-        const int col0 = half * 64 + c2 * 32;
-        uint32_t ra[32], rs[32];
-        tmem_ld32(lane_base + T0 + col0, ra);
-        tmem_ld32(lane_base + T1 + col0, rs);
+        const int col0 = cq + c2 * 16;
+        uint32_t ra[16], rs[16];
+        tmem_ld16(lane_base + T0 + col0, ra);
+        tmem_ld16(lane_base + T1 + col0, rs);
         tmem_ld_wait();
 #pragma unroll
-        for (int u = 0; u < 32; ++u)
+        for (int u = 0; u < 16; ++u)
           if (col0 + u == t) s->dAd[t] = __uint_as_float(ra[u]);
 #pragma unroll
-        for (int q4 = 0; q4 < 4; ++q4) {
+        for (int q4 = 0; q4 < 2; ++q4) {
           float fa[8], fs[8];
 #pragma unroll
           for (int u = 0; u < 8; ++u) {
@@ -957,18 +1066,6 @@ __global__ void __launch_bounds__(kThreads, 1) gla_bwd_tc(
           *tile16(sB, t, col0 + q4 * 8) = make_uint4(pack_bf16(fs[0], fs[1]), pack_bf16(fs[2], fs[3]),
                                                      pack_bf16(fs[4], fs[5]), pack_bf16(fs[6], fs[7]));
         }
-      }
-    } else {
-      s->abort = 1;
-    }
-    // X is free once dO P'^T has read P': R' = diag(e^{b_end - r}) R_c replaces it
-    if (mbar_wait(&s->mma1b, ph, SITE_BWD_MMA)) {
-#pragma unroll
-      for (int q8 = 0; q8 < 8; ++q8) {
-        const float4 a = rreg[2 * q8], b2 = rreg[2 * q8 + 1];
-        st_tile16(sX, t, half * 64 + q8 * 8,
-                  make_uint4(pack_bf16(a.x * wt, a.y * wt), pack_bf16(a.z * wt, a.w * wt),
-                             pack_bf16(b2.x * wt, b2.y * wt), pack_bf16(b2.z * wt, b2.w * wt)));
       }
     } else {
       s->abort = 1;
@@ -989,50 +1086,46 @@ __global__ void __launch_bounds__(kThreads, 1) gla_bwd_tc(
     }
     // ---- epilogue 2: dq' = E . T2; dq = dq' + (do_t . v_t) k_t = E . (T2 + (do_t . v_t) K^_t);
     // q . dq' = Q^ . T2 -> T2
-    float xl[64];  // log2 E of row t, kept for epilogue 3
+    float xl[32];  // log2 E of row t, columns cq.., kept for epilogue 3
     if (mbar_wait(&s->mma2, ph, SITE_BWD_MMA)) {
       tc_fence_after();
       {
-        uint32_t r0[32], r1[32];
-        tmem_ld32(lane_base + T3 + half * 64, r0);
-        tmem_ld32(lane_base + T3 + half * 64 + 32, r1);
+        uint32_t r0[32];
+        tmem_ld32(lane_base + T3 + cq, r0);
         tmem_ld_wait();
 #pragma unroll
-        for (int u = 0; u < 32; ++u) {
-          xl[u] = __uint_as_float(r0[u]);
-          xl[32 + u] = __uint_as_float(r1[u]);
-        }
+        for (int u = 0; u < 32; ++u) xl[u] = __uint_as_float(r0[u]);
       }
       const float dad = s->dAd[t];
 #pragma unroll
       for (int c2 = 0; c2 < 2; ++c2) {
-        const int col0 = half * 64 + c2 * 32;
-        uint32_t a[32];
-        tmem_ld32(lane_base + T2 + col0, a);
+        const int col0 = cq + c2 * 16;
+        uint32_t a[16];
+        tmem_ld16(lane_base + T2 + col0, a);
         // Q^ and K^ of row t (bf16, shared memory): q . dq' = Q^ . T2 and k_t = K^_t . E_t
-        uint32_t qh[16], kh[16];
+        uint32_t qh[8], kh[8];
 #pragma unroll
-        for (int q4 = 0; q4 < 4; ++q4) {
+        for (int q4 = 0; q4 < 2; ++q4) {
           const uint4 wq = *tile16(sQ, t, col0 + q4 * 8);
           const uint4 wk = *tile16(sK, t, col0 + q4 * 8);
           qh[4 * q4] = wq.x, qh[4 * q4 + 1] = wq.y, qh[4 * q4 + 2] = wq.z, qh[4 * q4 + 3] = wq.w;
           kh[4 * q4] = wk.x, kh[4 * q4 + 1] = wk.y, kh[4 * q4 + 2] = wk.z, kh[4 * q4 + 3] = wk.w;
         }
         tmem_ld_wait();
-        uint32_t out[16];
+        uint32_t out[8];
 #pragma unroll
-        for (int u2 = 0; u2 < 16; ++u2) {
+        for (int u2 = 0; u2 < 8; ++u2) {
           const float2 qf = unpack_bf16(qh[u2]), kf = unpack_bf16(kh[u2]);
-          const float e0 = ex2a(xl[c2 * 32 + 2 * u2]), e1 = ex2a(xl[c2 * 32 + 2 * u2 + 1]);
+          const float e0 = ex2a(xl[c2 * 16 + 2 * u2]), e1 = ex2a(xl[c2 * 16 + 2 * u2 + 1]);
           const float t0 = __uint_as_float(a[2 * u2]), t1 = __uint_as_float(a[2 * u2 + 1]);
           out[u2] = pack_bf16(e0 * fmaf(dad, kf.x, t0), e1 * fmaf(dad, kf.y, t1));
           a[2 * u2] = __float_as_uint(qf.x * t0);
           a[2 * u2 + 1] = __float_as_uint(qf.y * t1);
         }
         uint4* dst = reinterpret_cast<uint4*>(dq + tok + col0);
-#pragma unroll
-        for (int q4 = 0; q4 < 4; ++q4) dst[q4] = make_uint4(out[4 * q4], out[4 * q4 + 1], out[4 * q4 + 2], out[4 * q4 + 3]);
-        tmem_st32(lane_base + T2 + col0, a);
+        dst[0] = make_uint4(out[0], out[1], out[2], out[3]);
+        dst[1] = make_uint4(out[4], out[5], out[6], out[7]);
+        tmem_st16(lane_base + T2 + col0, a);
       }
       tmem_st_wait();
     } else {
@@ -1049,34 +1142,34 @@ __global__ void __launch_bounds__(kThreads, 1) gla_bwd_tc(
       for (int kk = 0; kk < kD / 16; ++kk) mma_bf16(tmem + T1, kmaj(aK, kk), mnmaj(aX, kk), id_kn, 1);
       for (int kk = 0; kk < kD / 16; ++kk) mma_bf16(tmem + T3, kmaj(aV, kk), kmaj(aX, kk), id_kk, kk != 0);
     }
-    // ---- R_{c-1} = e^{b_end} R_c + e^{r} T0 (row t, columns half * 64..), R_c
-    // read back from the scratch in L2 (this thread's elements only, so the
-    // slot is both source and destination; float4 group g of row t at g * 128 + t)
+    // ---- R_{c-1} = e^{b_end} R_c + e^{r} T0 (row t, columns cq..), R_c read
+    // back from the scratch in L2 (this thread's elements only, so the slot is
+    // both source and destination; float4 group g of row t at g * 128 + t)
     if (form) {
       float4* rn = reinterpret_cast<float4*>(R + pslot_of(c - j, h, b) * kD * kD);
-      float4 rv[8];  // 32 columns of R_c at a time, the next chunk's in flight under this one's math
+      float4 rv[4];  // 16 columns of R_c at a time, the next pass's in flight under this one's math
 #pragma unroll
-      for (int q4 = 0; q4 < 8; ++q4) rv[q4] = rn[(half * 16 + q4) * kD + t];
+      for (int q4 = 0; q4 < 4; ++q4) rv[q4] = rn[(qt * 8 + q4) * kD + t];
       if (mbar_wait(&s->mmar, rph, SITE_BWD_MMA)) {
         tc_fence_after();
 #pragma unroll 1
         for (int c2 = 0; c2 < 2; ++c2) {
-          uint32_t a[32];
-          tmem_ld32(lane_base + T0 + half * 64 + c2 * 32, a);
+          uint32_t a[16];
+          tmem_ld16(lane_base + T0 + cq + c2 * 16, a);
           tmem_ld_wait();
-          float4 o4[8];
+          float4 o4[4];
 #pragma unroll
-          for (int q4 = 0; q4 < 8; ++q4)
+          for (int q4 = 0; q4 < 4; ++q4)
             o4[q4] = make_float4(fmaf(eb, rv[q4].x, er * __uint_as_float(a[4 * q4])),
                                  fmaf(eb, rv[q4].y, er * __uint_as_float(a[4 * q4 + 1])),
                                  fmaf(eb, rv[q4].z, er * __uint_as_float(a[4 * q4 + 2])),
                                  fmaf(eb, rv[q4].w, er * __uint_as_float(a[4 * q4 + 3])));
           if (c2 == 0) {
 #pragma unroll
-            for (int q4 = 0; q4 < 8; ++q4) rv[q4] = rn[(half * 16 + 8 + q4) * kD + t];
+            for (int q4 = 0; q4 < 4; ++q4) rv[q4] = rn[(qt * 8 + 4 + q4) * kD + t];
           }
 #pragma unroll
-          for (int q4 = 0; q4 < 8; ++q4) rn[(half * 16 + c2 * 8 + q4) * kD + t] = o4[q4];
+          for (int q4 = 0; q4 < 4; ++q4) rn[(qt * 8 + c2 * 4 + q4) * kD + t] = o4[q4];
         }
         fence_async_global();  // the next tile's bulk load of R reads these stores
       } else {
@@ -1086,7 +1179,7 @@ __global__ void __launch_bounds__(kThreads, 1) gla_bwd_tc(
     }
     if (form) {
       tc_fence_before();
-      named_sync(kBarAll, kThreads);  // every thread has read its rows of T0
+      named_sync(kBarAll, kBwdThreads);  // every thread has read its rows of T0
     }
     if (tid == 0) {
       tc_fence_after();
@@ -1103,26 +1196,20 @@ __global__ void __launch_bounds__(kThreads, 1) gla_bwd_tc(
       tc_fence_after();
       const float dad = s->dAd[t];
 #pragma unroll
-      for (int c2 = 0; c2 < 2; ++c2) {
-        const int col0 = half * 64 + c2 * 32;
-        uint32_t ka[32], kb[32], bq[32];
-        tmem_ld32(lane_base + T0 + col0, ka);
-        tmem_ld32(lane_base + T3 + col0, kb);
-        tmem_ld32(lane_base + T2 + col0, bq);
-        uint32_t qh[16], kh[16];
-#pragma unroll
-        for (int q4 = 0; q4 < 4; ++q4) {
-          const uint4 wq = *tile16(sQ, t, col0 + q4 * 8);
-          const uint4 wk = *tile16(sK, t, col0 + q4 * 8);
-          qh[4 * q4] = wq.x, qh[4 * q4 + 1] = wq.y, qh[4 * q4 + 2] = wq.z, qh[4 * q4 + 3] = wq.w;
-          kh[4 * q4] = wk.x, kh[4 * q4 + 1] = wk.y, kh[4 * q4 + 2] = wk.z, kh[4 * q4 + 3] = wk.w;
-        }
+      for (int c2 = 0; c2 < 4; ++c2) {
+        const int col0 = cq + c2 * 8;
+        uint32_t ka[8], kb[8], bq[8];
+        tmem_ld8(lane_base + T0 + col0, ka);
+        tmem_ld8(lane_base + T3 + col0, kb);
+        tmem_ld8(lane_base + T2 + col0, bq);
+        const uint4 wq = *tile16(sQ, t, col0), wk = *tile16(sK, t, col0);
+        const uint32_t qh[4] = {wq.x, wq.y, wq.z, wq.w}, kh[4] = {wk.x, wk.y, wk.z, wk.w};
         tmem_ld_wait();
-        uint32_t out[16];
+        uint32_t out[4];
 #pragma unroll
-        for (int u2 = 0; u2 < 16; ++u2) {
+        for (int u2 = 0; u2 < 4; ++u2) {
           const float2 qf = unpack_bf16(qh[u2]), kf = unpack_bf16(kh[u2]);
-          const float e0 = ex2a(-xl[c2 * 32 + 2 * u2]), e1 = ex2a(-xl[c2 * 32 + 2 * u2 + 1]);
+          const float e0 = ex2a(-xl[c2 * 8 + 2 * u2]), e1 = ex2a(-xl[c2 * 8 + 2 * u2 + 1]);
           const float a0 = __uint_as_float(ka[2 * u2]), a1 = __uint_as_float(ka[2 * u2 + 1]);
           const float b0 = __uint_as_float(kb[2 * u2]), b1 = __uint_as_float(kb[2 * u2 + 1]);
           out[u2] = pack_bf16(e0 * fmaf(dad, qf.x, a0 + b0), e1 * fmaf(dad, qf.y, a1 + b1));
@@ -1131,17 +1218,17 @@ __global__ void __launch_bounds__(kThreads, 1) gla_bwd_tc(
           kb[2 * u2] = __float_as_uint(kf.x * b0);
           kb[2 * u2 + 1] = __float_as_uint(kf.y * b1);
         }
-#pragma unroll
-        for (int q4 = 0; q4 < 4; ++q4)
-          *tile16(sA, t, col0 + q4 * 8) = make_uint4(out[4 * q4], out[4 * q4 + 1], out[4 * q4 + 2], out[4 * q4 + 3]);
-        tmem_st32(lane_base + T0 + col0, ka);
-        tmem_st32(lane_base + T3 + col0, kb);
+        *tile16(sA, t, col0) = make_uint4(out[0], out[1], out[2], out[3]);
+        tmem_st8(lane_base + T0 + col0, ka);
+        tmem_st8(lane_base + T3 + col0, kb);
+      }
+      {
         uint32_t dvv[32];
-        tmem_ld32(lane_base + T1 + col0, dvv);
+        tmem_ld32(lane_base + T1 + cq, dvv);
         tmem_ld_wait();
 #pragma unroll
         for (int q4 = 0; q4 < 4; ++q4)
-          *tile16(sB, t, col0 + q4 * 8) =
+          *tile16(sB, t, cq + q4 * 8) =
               make_uint4(pack_bf16(__uint_as_float(dvv[q4 * 8]), __uint_as_float(dvv[q4 * 8 + 1])),
                          pack_bf16(__uint_as_float(dvv[q4 * 8 + 2]), __uint_as_float(dvv[q4 * 8 + 3])),
                          pack_bf16(__uint_as_float(dvv[q4 * 8 + 4]), __uint_as_float(dvv[q4 * 8 + 5])),
@@ -1162,39 +1249,42 @@ __global__ void __launch_bounds__(kThreads, 1) gla_bwd_tc(
       tma_store_4d(&map_dv, sB + kBox, 64, h, (int)row0, b);
       tma_store_commit();
     }
-#pragma unroll
-    for (int c2 = 0; c2 < 2; ++c2) {
-      const int col0 = half * 64 + c2 * 32;
+    {
       uint32_t db[32], kd[32];
-      tmem_ld32(lane_base + T0 + col0, db);
-      tmem_ld32(lane_base + T3 + col0, kd);
+      tmem_ld32(lane_base + T0 + cq, db);
+      tmem_ld32(lane_base + T3 + cq, kd);
       tmem_ld_wait();
 #pragma unroll
       for (int q4 = 0; q4 < 8; ++q4) {
-        *reinterpret_cast<float4*>(fB + gate_slot(t, col0 + 4 * q4)) =
+        *reinterpret_cast<float4*>(fB + gate_slot(t, cq + 4 * q4)) =
             make_float4(__uint_as_float(db[4 * q4]), __uint_as_float(db[4 * q4 + 1]), __uint_as_float(db[4 * q4 + 2]),
                         __uint_as_float(db[4 * q4 + 3]));
-        *reinterpret_cast<float4*>(fK + gate_slot(t, col0 + 4 * q4)) =
+        *reinterpret_cast<float4*>(fK + gate_slot(t, cq + 4 * q4)) =
             make_float4(__uint_as_float(kd[4 * q4]), __uint_as_float(kd[4 * q4 + 1]), __uint_as_float(kd[4 * q4 + 2]),
                         __uint_as_float(kd[4 * q4 + 3]));
       }
     }
     __syncthreads();
     // dg_t = sum_{t' >= t} dB_t' + sum_{t' < t} k . dk^inter_t' + e^{b_end} <R_c, P_c>: the
-    // two sums by column walks (threads 0-127 the suffix of dB, 128-255 the
-    // exclusive prefix of k . dk^inter, one feature each), in place
+    // two sums by column walks, in place, four threads per feature i: the
+    // suffix of dB over rows 64-127 (starting from bnd, so that it reaches
+    // every row) and over rows 0-63, the exclusive prefix of k . dk^inter over
+    // rows 0-63 and over rows 64-127; the walks of rows 0-63 of dB and 64-127
+    // of k . dk^inter leave out the other half's total (the carries dAd and
+    // cK), which the combination below adds
     {
-      const int i = tid & (kD - 1);
-      float acc = 0.f;
+      const int i = tid & (kD - 1), role = tid >> 7;
       // blocks of 8 rows; the next block's loads go out before this block's
       // stores (other rows), so each block waits for one load latency only
       float v[8], w[8];
-      if (tid < kD) {
+      if (role < 2) {
+        const int top = role == 0 ? kTile : kTile / 2;  // rows top - 64 .. top - 1, walked down
+        float acc = role == 0 ? s->bnd[i] : 0.f;
 #pragma unroll
-        for (int u = 0; u < 8; ++u) v[u] = fB[gate_slot(kTile - 8 + u, i)];
+        for (int u = 0; u < 8; ++u) v[u] = fB[gate_slot(top - 8 + u, i)];
 #pragma unroll 1
-        for (int t0 = kTile - 8; t0 >= 0; t0 -= 8) {
-          if (t0 >= 8) {
+        for (int t0 = top - 8; t0 >= top - kTile / 2; t0 -= 8) {
+          if (t0 - 8 >= top - kTile / 2) {
 #pragma unroll
             for (int u = 0; u < 8; ++u) w[u] = fB[gate_slot(t0 - 8 + u, i)];
           }
@@ -1206,12 +1296,15 @@ __global__ void __launch_bounds__(kThreads, 1) gla_bwd_tc(
 #pragma unroll
           for (int u = 0; u < 8; ++u) v[u] = w[u];
         }
+        if (role == 0) s->dAd[i] = acc;
       } else {
+        const int bot = role == 2 ? 0 : kTile / 2;  // rows bot .. bot + 63, walked up
+        float acc = 0.f;
 #pragma unroll
-        for (int u = 0; u < 8; ++u) v[u] = fK[gate_slot(u, i)];
+        for (int u = 0; u < 8; ++u) v[u] = fK[gate_slot(bot + u, i)];
 #pragma unroll 1
-        for (int t0 = 0; t0 < kTile; t0 += 8) {
-          if (t0 + 8 < kTile) {
+        for (int t0 = bot; t0 < bot + kTile / 2; t0 += 8) {
+          if (t0 + 8 < bot + kTile / 2) {
 #pragma unroll
             for (int u = 0; u < 8; ++u) w[u] = fK[gate_slot(t0 + 8 + u, i)];
           }
@@ -1223,6 +1316,7 @@ __global__ void __launch_bounds__(kThreads, 1) gla_bwd_tc(
 #pragma unroll
           for (int u = 0; u < 8; ++u) v[u] = w[u];
         }
+        if (role == 2) s->cK[i] = acc;
       }
     }
     __syncthreads();
@@ -1233,21 +1327,21 @@ __global__ void __launch_bounds__(kThreads, 1) gla_bwd_tc(
       int cn, hn, bn, jn;
       tile_of(k + 1, cn, hn, bn, jn);
       load_gate_tile(bt, &map_g, &s->gload, hn, cn * kTile, bn);
+      gate_out = (int)(ph ^ 1u);
       if (jn == S - 1) bulk_prefetch_l2(R + rslot_of(cn, hn, bn, jn) * kD * kD, kD * kD * 4);
     }
-    // dg into the dB tile (the gate map's layout), stored by TMA below
-#pragma unroll
-    for (int cb = 0; cb < 2; ++cb) {
-      const int col0 = half * 64 + cb * 32;
+    // dg into the dB tile (the gate map's layout), stored by TMA below: rows
+    // 0-63 take dB's carry (the sum over rows 64-127, bnd included), rows
+    // 64-127 the prefix's (the sum of k . dk^inter over rows 0-63)
+    {
+      const float* carry = t < kTile / 2 ? s->dAd : s->cK;
 #pragma unroll
       for (int q4 = 0; q4 < 8; ++q4) {
-        float4* pa = reinterpret_cast<float4*>(fB + gate_slot(t, col0 + 4 * q4));
+        float4* pa = reinterpret_cast<float4*>(fB + gate_slot(t, cq + 4 * q4));
         const float4 a = *pa;
-        const float4 e = *reinterpret_cast<const float4*>(fK + gate_slot(t, col0 + 4 * q4));
-        const float4 bn = *reinterpret_cast<const float4*>(s->bnd + col0 + 4 * q4);
-        const float4 bn2 = *reinterpret_cast<const float4*>(s->bnd2 + col0 + 4 * q4);
-        *pa = make_float4(a.x + e.x + (bn.x + bn2.x), a.y + e.y + (bn.y + bn2.y), a.z + e.z + (bn.z + bn2.z),
-                          a.w + e.w + (bn.w + bn2.w));
+        const float4 e = *reinterpret_cast<const float4*>(fK + gate_slot(t, cq + 4 * q4));
+        const float4 cy = *reinterpret_cast<const float4*>(carry + cq + 4 * q4);
+        *pa = make_float4(a.x + e.x + cy.x, a.y + e.y + cy.y, a.z + e.z + cy.z, a.w + e.w + cy.w);
       }
     }
     fence_async_smem();
@@ -1268,6 +1362,7 @@ __global__ void __launch_bounds__(kThreads, 1) gla_bwd_tc(
         load_tokens(sV, &map_v, hn, cn * kTile, bn);
         load_tokens(sD, &map_do, hn, cn * kTile, bn);
         load_pprime(pslot_of(cn, hn, bn));
+        tok_out = (int)(ph ^ 1u);
       }
       tma_store_wait_read0();  // the dg store has read fB (over Q and K); all stores have read shared memory
       if (next) {
@@ -1279,7 +1374,11 @@ __global__ void __launch_bounds__(kThreads, 1) gla_bwd_tc(
   }
   }
 cleanup:
-  if (tid == 0 && r_ahead) mbar_wait(&s->ldr, ph, SITE_BWD_TMA);  // an abort leaves R's load unused: it lands first
+  // an abort leaves loads unused: they land first
+  if (tid == 0 && r_ahead) mbar_wait(&s->ldr, ph, SITE_BWD_TMA);
+  if (tid == 0 && gate_out >= 0) mbar_wait(&s->gload, (uint32_t)gate_out, SITE_BWD_TMA);
+  if (tid == 0 && tok_out >= 0) mbar_wait(&s->load, (uint32_t)tok_out, SITE_BWD_TMA);
+  if (tid == 0) tma_store_wait_read0();  // no store still reads shared memory
   tc_fence_before();
   __syncthreads();
   if (warp == 0) tmem_dealloc(tmem, 512);
@@ -1359,7 +1458,7 @@ cudaError_t tc_gla_chunk_bwd(const void* q, const void* k, const void* v, const 
   if (tiles < 1 || ntx % tiles != 0) return cudaErrorInvalidValue;
   const int64_t nitems = (int64_t)B * H * (ntx / tiles);
   const unsigned grid = (unsigned)std::min<int64_t>(nitems, sms);
-  gla_bwd_tc<<<grid, kThreads, smem, st>>>(mq, mk, mv, mdo, mdk, mdv, mg, mdg, P, Rs, (__nv_bfloat16*)dq, H, N, t_slots,
+  gla_bwd_tc<<<grid, kBwdThreads, smem, st>>>(mq, mk, mv, mdo, mdk, mdv, mg, mdg, P, Rs, (__nv_bfloat16*)dq, H, N, t_slots,
                                             stride, ntx, tiles, nitems, run);
   return cudaGetLastError();
 }
