@@ -718,6 +718,17 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
       : "r"(taddr));
 }
 
+// D (TMEM) += A (TMEM) B (shared memory descriptor), kind::f16.
+__device__ __forceinline__ void mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                            uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
 __device__ __forceinline__ void tmem_ld8(uint32_t taddr, uint32_t (&r)[8]) {
   asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
                : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
@@ -788,14 +799,11 @@ __device__ __forceinline__ bool gate_rows_quarter(float* bt, uint64_t* gbar, uin
 
 // ---------------------------------------------------------------- gradients
 struct SmemBwd {
-  uint64_t gload, load, ldr, mma1a, mma1b, mma2, mma3, mmar;
+  uint64_t gload, load, ldr, mma1a, mma1b, mma2, mma3, mmar, mmag;
   uint32_t tmem_base;
   int abort;
-  // do_t . v_t, the diagonal of dO V^T (epilogues 1-3); then, per feature,
-  // the sum of dB over rows 64-127 plus bnd (the column walks' carry)
-  alignas(16) float dAd[kTile];
-  alignas(16) float bnd[kD];  // e^{b_end[i]} <R_c[i], P_c[i]>
-  alignas(16) float cK[kD];   // per feature, the sum of k . dk^inter over rows 0-63 (the other carry)
+  alignas(16) float dAd[kTile];  // do_t . v_t, the diagonal of dO V^T (epilogues 1-3)
+  alignas(16) float bnd[kD];     // e^{b_end[i]} <R_c[i], P_c[i]>
 };
 
 // One persistent CTA per SM, taking segments of S 128-token tiles in launch
@@ -813,19 +821,26 @@ struct SmemBwd {
 // the threads of a warp, which own consecutive rows, read and write one
 // 512-byte run per access; the scan's slot is row-major, so a segment's last
 // tile first copies its R_c into the scratch, and the combination always reads
-// R_c from there (L2). Most
-// barriers complete once per tile, so their parity flips from tile to tile;
-// mmar only on tiles that form a state. Shared memory: Q^, K^, V, dO (then, in pairs,
-// the fp32 tiles of dB and k . dk^inter for the log-gate gradient's column
-// sums), X (P', loaded as the output kernel cached it, then R'), and the pair
-// sA / sB (the gate tile during the walk; then dA . strict and A . causal;
-// then the dK and dV outputs). TMEM: T0 = dO V^T -> Q^^T dO -> (dA . strict)^T Q^;
-// T1 = Q^ K^^T -> dV; T2 = dO P'^T + (dA . strict) K^ -> q . dq'; T3 = log2 E
-// -> V R'^T.
+// R_c from there (L2).
+//
+// The log-gate gradient's column sums over the tile's rows,
+//   dg_t = sum_{s >= t} dB_s + sum_{s < t} (k . dk^inter)_s + e^{b_end} <R_c, P_c>,
+// are two products with triangular 0/1 matrices, U_ts = [s >= t] and L_ts =
+// [s < t], held in TMEM as the A operand; dB and k . dk^inter enter as B in
+// two bf16 parts each (x = hi + lo, about 16 bits of mantissa), so the sums
+// keep nearly fp32 precision.
+//
+// Most barriers complete once per tile, so their parity flips from tile to
+// tile; mmar only on tiles that form a state. Shared memory: Q^, K^, V, dO, X
+// (P', loaded as the output kernel cached it, then R'), and the pair sA / sB
+// (the gate tile during the walk; then dA . strict and A . causal; then the
+// dK and dV outputs); after the last gradient MMA, V, dO, X and K^ hold the
+// sums' B operands and Q^ / K^ the fp32 dg tile. TMEM: T0 = dO V^T -> Q^^T dO
+// -> (dA . strict)^T Q^ -> dg; T1 = Q^ K^^T -> dV; T2 = dO P'^T + (dA .
+// strict) K^ -> q . dq' -> U and L; T3 = log2 E -> V R'^T.
 //
 // 512 threads: warp w owns tile rows / TMEM lanes 32*(w%4).. and the column
-// quarter w/4 (32 columns) of every row-wise step; the column walks give each
-// feature four threads (two sums, each over two halves of the rows).
+// quarter w/4 (32 columns) of every row-wise step.
 __global__ void __launch_bounds__(kBwdThreads, 1) gla_bwd_tc(
     const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
     const __grid_constant__ CUtensorMap map_v, const __grid_constant__ CUtensorMap map_do,
@@ -891,6 +906,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) gla_bwd_tc(
     mbar_init(&s->mma2, 1);
     mbar_init(&s->mma3, 1);
     mbar_init(&s->mmar, 1);
+    mbar_init(&s->mmag, 1);
     s->abort = 0;
     fence_mbar_init();
   }
@@ -1187,11 +1203,17 @@ __global__ void __launch_bounds__(kBwdThreads, 1) gla_bwd_tc(
       mma_commit(&s->mma3);
     }
     // ---- epilogue 3: dk = E^-1 . (T0 + T3 + (do_s . v_s) Q^_s) -> sA, dv = T1 -> sB;
-    // dB = q . dq' - k . dk' = T2 - K^ . T0 and k . dk^inter = K^ . T3 back into
-    // T0 and T3, then (once every thread has read its Q^ and K^ rows) as fp32
-    // tiles over the token buffers for the column sums
-    float* fB = reinterpret_cast<float*>(sQ);  // over sQ and sK
-    float* fK = reinterpret_cast<float*>(sV);  // over sV and sD
+    // dB = q . dq' - k . dk' = T2 - K^ . T0 and k . dk^inter = K^ . T3, each in
+    // two bf16 parts (x = hi + lo, hi = bf16(x), lo = bf16(x - hi)), as the
+    // operand tiles of the log-gate gradient's column sums: dB over V and dO,
+    // k . dk^inter over X and K^ (each thread overwrites only the K^ entries it
+    // has read). The masks of those sums go into TMEM, over this thread's
+    // columns of T2 once it has read them: U_ts = [s >= t] and L_ts = [s < t],
+    // the rows' K steps 2 qt and 2 qt + 1 at T2 + cq (U) and T2 + cq + 16 (L).
+    uint8_t* sBh = sV;
+    uint8_t* sBl = sD;
+    uint8_t* sKh = sX;
+    uint8_t* sKl = sK;
     if (mbar_wait(&s->mma3, ph, SITE_BWD_MMA)) {
       tc_fence_after();
       const float dad = s->dAd[t];
@@ -1205,7 +1227,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) gla_bwd_tc(
         const uint4 wq = *tile16(sQ, t, col0), wk = *tile16(sK, t, col0);
         const uint32_t qh[4] = {wq.x, wq.y, wq.z, wq.w}, kh[4] = {wk.x, wk.y, wk.z, wk.w};
         tmem_ld_wait();
-        uint32_t out[4];
+        uint32_t out[4], dbh[4], dbl[4], kdh[4], kdl[4];
 #pragma unroll
         for (int u2 = 0; u2 < 4; ++u2) {
           const float2 qf = unpack_bf16(qh[u2]), kf = unpack_bf16(kh[u2]);
@@ -1213,14 +1235,19 @@ __global__ void __launch_bounds__(kBwdThreads, 1) gla_bwd_tc(
           const float a0 = __uint_as_float(ka[2 * u2]), a1 = __uint_as_float(ka[2 * u2 + 1]);
           const float b0 = __uint_as_float(kb[2 * u2]), b1 = __uint_as_float(kb[2 * u2 + 1]);
           out[u2] = pack_bf16(e0 * fmaf(dad, qf.x, a0 + b0), e1 * fmaf(dad, qf.y, a1 + b1));
-          ka[2 * u2] = __float_as_uint(__uint_as_float(bq[2 * u2]) - kf.x * a0);
-          ka[2 * u2 + 1] = __float_as_uint(__uint_as_float(bq[2 * u2 + 1]) - kf.y * a1);
-          kb[2 * u2] = __float_as_uint(kf.x * b0);
-          kb[2 * u2 + 1] = __float_as_uint(kf.y * b1);
+          const float d0 = __uint_as_float(bq[2 * u2]) - kf.x * a0, d1 = __uint_as_float(bq[2 * u2 + 1]) - kf.y * a1;
+          const float g0 = kf.x * b0, g1 = kf.y * b1;
+          dbh[u2] = pack_bf16(d0, d1);
+          kdh[u2] = pack_bf16(g0, g1);
+          const float2 dh = unpack_bf16(dbh[u2]), gh = unpack_bf16(kdh[u2]);
+          dbl[u2] = pack_bf16(d0 - dh.x, d1 - dh.y);
+          kdl[u2] = pack_bf16(g0 - gh.x, g1 - gh.y);
         }
         *tile16(sA, t, col0) = make_uint4(out[0], out[1], out[2], out[3]);
-        tmem_st8(lane_base + T0 + col0, ka);
-        tmem_st8(lane_base + T3 + col0, kb);
+        *tile16(sBh, t, col0) = make_uint4(dbh[0], dbh[1], dbh[2], dbh[3]);
+        *tile16(sBl, t, col0) = make_uint4(dbl[0], dbl[1], dbl[2], dbl[3]);
+        *tile16(sKh, t, col0) = make_uint4(kdh[0], kdh[1], kdh[2], kdh[3]);
+        *tile16(sKl, t, col0) = make_uint4(kdl[0], kdl[1], kdl[2], kdl[3]);
       }
       {
         uint32_t dvv[32];
@@ -1234,118 +1261,68 @@ __global__ void __launch_bounds__(kBwdThreads, 1) gla_bwd_tc(
                          pack_bf16(__uint_as_float(dvv[q4 * 8 + 4]), __uint_as_float(dvv[q4 * 8 + 5])),
                          pack_bf16(__uint_as_float(dvv[q4 * 8 + 6]), __uint_as_float(dvv[q4 * 8 + 7])));
       }
+      {
+        // U and L rows t, K elements cq.. (bf16 1 = 0x3f80; element 2w in the low half of word w)
+        uint32_t um[16], lm[16];
+#pragma unroll
+        for (int w = 0; w < 16; ++w) {
+          const int s0 = cq + 2 * w;
+          um[w] = (s0 >= t ? 0x3f80u : 0u) | (s0 + 1 >= t ? 0x3f800000u : 0u);
+          lm[w] = (s0 < t ? 0x3f80u : 0u) | (s0 + 1 < t ? 0x3f800000u : 0u);
+        }
+        tmem_st16(lane_base + T2 + cq, um);
+        tmem_st16(lane_base + T2 + cq + 16, lm);
+      }
       tmem_st_wait();
       fence_async_smem();
     } else {
       s->abort = 1;
     }
     tc_fence_before();
-    __syncthreads();  // every Q^ and K^ row has been read; dK and dV are staged
+    __syncthreads();  // dK, dV and the sums' operands are staged
     tc_fence_after();
-    if (tid == 0 && !s->abort) {  // dK and dV leave now, under the log-gate gradient's sums
+    if (s->abort) goto cleanup;
+    if (tid == 0) {
+      // dK and dV leave now; the sums: T0 = U (dB_hi + dB_lo) + L (kdk_hi + kdk_lo)
       tma_store_4d(&map_dk, sA, 0, h, (int)row0, b);
       tma_store_4d(&map_dk, sA + kBox, 64, h, (int)row0, b);
       tma_store_4d(&map_dv, sB, 0, h, (int)row0, b);
       tma_store_4d(&map_dv, sB + kBox, 64, h, (int)row0, b);
       tma_store_commit();
+      const uint32_t aBh = smem_u32(sBh), aBl = smem_u32(sBl), aKh = smem_u32(sKh), aKl = smem_u32(sKl);
+      const uint32_t tu = tmem + T2;
+      for (int kk = 0; kk < kTile / 16; ++kk)
+        mma_bf16_ts(tmem + T0, tu + 32 * (kk >> 1) + 8 * (kk & 1), mnmaj(aBh, kk), id_kn, kk != 0);
+      for (int kk = 0; kk < kTile / 16; ++kk)
+        mma_bf16_ts(tmem + T0, tu + 32 * (kk >> 1) + 8 * (kk & 1), mnmaj(aBl, kk), id_kn, 1);
+      for (int kk = 0; kk < kTile / 16; ++kk)
+        mma_bf16_ts(tmem + T0, tu + 32 * (kk >> 1) + 16 + 8 * (kk & 1), mnmaj(aKh, kk), id_kn, 1);
+      for (int kk = 0; kk < kTile / 16; ++kk)
+        mma_bf16_ts(tmem + T0, tu + 32 * (kk >> 1) + 16 + 8 * (kk & 1), mnmaj(aKl, kk), id_kn, 1);
+      mma_commit(&s->mmag);
     }
-    {
-      uint32_t db[32], kd[32];
-      tmem_ld32(lane_base + T0 + cq, db);
-      tmem_ld32(lane_base + T3 + cq, kd);
+    // dg_t = sum_{t' >= t} dB_t' + sum_{t' < t} k . dk^inter_t' + e^{b_end} <R_c, P_c>:
+    // T0 plus bnd, into an fp32 tile over Q^ and K^ (the gate map's layout),
+    // stored by TMA below
+    float* fB = reinterpret_cast<float*>(sQ);
+    if (mbar_wait(&s->mmag, ph, SITE_BWD_MMA)) {
+      tc_fence_after();
+      uint32_t dgv[32];
+      tmem_ld32(lane_base + T0 + cq, dgv);
       tmem_ld_wait();
 #pragma unroll
       for (int q4 = 0; q4 < 8; ++q4) {
+        const float4 bn = *reinterpret_cast<const float4*>(s->bnd + cq + 4 * q4);
         *reinterpret_cast<float4*>(fB + gate_slot(t, cq + 4 * q4)) =
-            make_float4(__uint_as_float(db[4 * q4]), __uint_as_float(db[4 * q4 + 1]), __uint_as_float(db[4 * q4 + 2]),
-                        __uint_as_float(db[4 * q4 + 3]));
-        *reinterpret_cast<float4*>(fK + gate_slot(t, cq + 4 * q4)) =
-            make_float4(__uint_as_float(kd[4 * q4]), __uint_as_float(kd[4 * q4 + 1]), __uint_as_float(kd[4 * q4 + 2]),
-                        __uint_as_float(kd[4 * q4 + 3]));
+            make_float4(__uint_as_float(dgv[4 * q4]) + bn.x, __uint_as_float(dgv[4 * q4 + 1]) + bn.y,
+                        __uint_as_float(dgv[4 * q4 + 2]) + bn.z, __uint_as_float(dgv[4 * q4 + 3]) + bn.w);
       }
-    }
-    __syncthreads();
-    // dg_t = sum_{t' >= t} dB_t' + sum_{t' < t} k . dk^inter_t' + e^{b_end} <R_c, P_c>: the
-    // two sums by column walks, in place, four threads per feature i: the
-    // suffix of dB over rows 64-127 (starting from bnd, so that it reaches
-    // every row) and over rows 0-63, the exclusive prefix of k . dk^inter over
-    // rows 0-63 and over rows 64-127; the walks of rows 0-63 of dB and 64-127
-    // of k . dk^inter leave out the other half's total (the carries dAd and
-    // cK), which the combination below adds
-    {
-      const int i = tid & (kD - 1), role = tid >> 7;
-      // blocks of 8 rows; the next block's loads go out before this block's
-      // stores (other rows), so each block waits for one load latency only
-      float v[8], w[8];
-      if (role < 2) {
-        const int top = role == 0 ? kTile : kTile / 2;  // rows top - 64 .. top - 1, walked down
-        float acc = role == 0 ? s->bnd[i] : 0.f;
-#pragma unroll
-        for (int u = 0; u < 8; ++u) v[u] = fB[gate_slot(top - 8 + u, i)];
-#pragma unroll 1
-        for (int t0 = top - 8; t0 >= top - kTile / 2; t0 -= 8) {
-          if (t0 - 8 >= top - kTile / 2) {
-#pragma unroll
-            for (int u = 0; u < 8; ++u) w[u] = fB[gate_slot(t0 - 8 + u, i)];
-          }
-#pragma unroll
-          for (int u = 7; u >= 0; --u) {
-            acc += v[u];
-            fB[gate_slot(t0 + u, i)] = acc;
-          }
-#pragma unroll
-          for (int u = 0; u < 8; ++u) v[u] = w[u];
-        }
-        if (role == 0) s->dAd[i] = acc;
-      } else {
-        const int bot = role == 2 ? 0 : kTile / 2;  // rows bot .. bot + 63, walked up
-        float acc = 0.f;
-#pragma unroll
-        for (int u = 0; u < 8; ++u) v[u] = fK[gate_slot(bot + u, i)];
-#pragma unroll 1
-        for (int t0 = bot; t0 < bot + kTile / 2; t0 += 8) {
-          if (t0 + 8 < bot + kTile / 2) {
-#pragma unroll
-            for (int u = 0; u < 8; ++u) w[u] = fK[gate_slot(t0 + 8 + u, i)];
-          }
-#pragma unroll
-          for (int u = 0; u < 8; ++u) {
-            fK[gate_slot(t0 + u, i)] = acc;
-            acc += v[u];
-          }
-#pragma unroll
-          for (int u = 0; u < 8; ++u) v[u] = w[u];
-        }
-        if (role == 2) s->cK[i] = acc;
-      }
-    }
-    __syncthreads();
-    if (tid == 0 && has_next && !s->abort) {
-      // the dK and dV stores have read the gate tile's space: the next tile's
-      // gates go there; a segment's entering R into L2 (a formed one is there)
-      tma_store_wait_read0();
-      int cn, hn, bn, jn;
-      tile_of(k + 1, cn, hn, bn, jn);
-      load_gate_tile(bt, &map_g, &s->gload, hn, cn * kTile, bn);
-      gate_out = (int)(ph ^ 1u);
-      if (jn == S - 1) bulk_prefetch_l2(R + rslot_of(cn, hn, bn, jn) * kD * kD, kD * kD * 4);
-    }
-    // dg into the dB tile (the gate map's layout), stored by TMA below: rows
-    // 0-63 take dB's carry (the sum over rows 64-127, bnd included), rows
-    // 64-127 the prefix's (the sum of k . dk^inter over rows 0-63)
-    {
-      const float* carry = t < kTile / 2 ? s->dAd : s->cK;
-#pragma unroll
-      for (int q4 = 0; q4 < 8; ++q4) {
-        float4* pa = reinterpret_cast<float4*>(fB + gate_slot(t, cq + 4 * q4));
-        const float4 a = *pa;
-        const float4 e = *reinterpret_cast<const float4*>(fK + gate_slot(t, cq + 4 * q4));
-        const float4 cy = *reinterpret_cast<const float4*>(carry + cq + 4 * q4);
-        *pa = make_float4(a.x + e.x + cy.x, a.y + e.y + cy.y, a.z + e.z + cy.z, a.w + e.w + cy.w);
-      }
+    } else {
+      s->abort = 1;
     }
     fence_async_smem();
-    __syncthreads();  // fK (over V and dO) has been read; no wait fails after this point
+    tc_fence_before();
+    __syncthreads();  // every thread has read T0 and written its dg; no wait fails after this point
     const bool stop = s->abort != 0;
     if (tid == 0) {
       if (!stop) {
@@ -1357,15 +1334,20 @@ __global__ void __launch_bounds__(kBwdThreads, 1) gla_bwd_tc(
       int cn = 0, hn = 0, bn = 0, jn = 0;
       if (next) tile_of(k + 1, cn, hn, bn, jn);
       if (next) {
-        // X (R', read by MMA 3) is free too
+        // the sums' operand tiles (V, dO, X) have been read by their MMAs
         mbar_arrive_expect_tx(&s->load, 5 * kTileBytes);
         load_tokens(sV, &map_v, hn, cn * kTile, bn);
         load_tokens(sD, &map_do, hn, cn * kTile, bn);
         load_pprime(pslot_of(cn, hn, bn));
         tok_out = (int)(ph ^ 1u);
       }
-      tma_store_wait_read0();  // the dg store has read fB (over Q and K); all stores have read shared memory
+      tma_store_wait_read0();  // the dK, dV and dg stores have read sA / sB and fB (over Q and K)
       if (next) {
+        // the next tile's gates into the gate tile's space; a segment's
+        // entering R into L2 (a formed one is there)
+        load_gate_tile(bt, &map_g, &s->gload, hn, cn * kTile, bn);
+        gate_out = (int)(ph ^ 1u);
+        if (jn == S - 1) bulk_prefetch_l2(R + rslot_of(cn, hn, bn, jn) * kD * kD, kD * kD * 4);
         load_tokens(sQ, &map_q, hn, cn * kTile, bn);
         load_tokens(sK, &map_k, hn, cn * kTile, bn);
       }
