@@ -19,7 +19,7 @@
 //     and the column half w / 4): read S_j from TMEM, mask, keep the running
 //     maximum m (log2 units; the two halves of a row exchange their tile
 //     maxima through shared memory) and the sum l, write P = exp2(s - m) in
-//     bf16 as the A operand of the P V MMA. O in TMEM is
+//     bf16 into TMEM as the A operand of the P V MMA. O in TMEM is
 //     rescaled only when a row's maximum grows by more than 8 (P stays below
 //     2^8 in between): the final O / l uses the same stale m for both, so the
 //     result is exact; the rescale waits for the P V MMA before it.
@@ -32,11 +32,15 @@
 // softmax_delta: delta per query row. softmax_dkdv_tc: one CTA per 128-key
 // tile walks the query tiles that see it: S^T = K Q^T and dP^T = V dO^T into
 // TMEM, then (sixteen epilogue warps, 32 query columns each) P^T and dS^T in
-// bf16, then dV += P^T dO and dK += dS^T Q; Q and dO stream through a
-// three-slot ring so that the next Q tile loads during the current tile.
+// bf16 back into TMEM over the columns they came from, then dV += P^T dO and
+// dK += dS^T Q; Q and dO stream through a three-slot ring so that the next Q
+// tile loads during the current tile.
 // softmax_dq_tc: one CTA per 128-query tile walks its key tiles: S = Q K^T,
-// dP = dO V^T, dS (sixteen epilogue warps), dQ += dS K. Only the tiles on the
-// causal diagonal mask element by element. The two gradient kernels
+// dP = dO V^T, dS (sixteen epilogue warps, into TMEM), dQ += dS K. Only the
+// tiles on the causal diagonal mask element by element.
+// The operands that the epilogues produce (P, P^T, dS^T, dS) stay in TMEM as
+// the A operand of the MMA that consumes them: an MMA whose operands both
+// come from shared memory takes nearly all of its bandwidth at N = 128. The two gradient kernels
 // recompute P separately, so no atomics are needed and the results do not
 // depend on scheduling.
 #include <algorithm>
@@ -66,6 +70,23 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&r)[8]) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"r"(taddr),
+               "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+               : "memory");
+}
+
+// D (TMEM) += A (TMEM) B (shared memory descriptor), kind::f16.
+__device__ __forceinline__ void mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                            uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
 // ------------------------------------------------------------------ forward
 constexpr int kFwdThreads = 320;  // warps 0-7 softmax, 8 TMA, 9 MMA
 constexpr int kSoftmaxThreads = 256;
@@ -91,7 +112,6 @@ __global__ void __launch_bounds__(kFwdThreads, 1) softmax_fwd_tc(const __grid_co
   uint8_t* sQ = base;  // Q, then the output tile
   uint8_t* sK = base + kTileBytes;       // two stages
   uint8_t* sV = base + 3 * kTileBytes;   // two stages
-  uint8_t* sP = base + 5 * kTileBytes;   // two P tiles
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int qt = qtiles - 1 - (int)blockIdx.x;  // heaviest (latest) tiles first
   const int h = blockIdx.y, b = blockIdx.z;
@@ -126,7 +146,11 @@ __global__ void __launch_bounds__(kFwdThreads, 1) softmax_fwd_tc(const __grid_co
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = s->tmem_base;
-  constexpr uint32_t kColS = 0, kColO = 256;  // S buffers at 0 and 128, O at 256
+  // S buffers at 0 and 128, O at 256; P in bf16 (the P V MMA's A operand) in
+  // two buffers of 64 columns at 384 and 448: K-step kk of buffer st in the 8
+  // columns kColP + 64 st + 8 kk, two bf16 per column, the lower K index in
+  // the low half
+  constexpr uint32_t kColS = 0, kColO = 256, kColP = 384;
 
   if (warp == 8) {
     // ---------------------------------------------------------- TMA producer
@@ -179,9 +203,10 @@ __global__ void __launch_bounds__(kFwdThreads, 1) softmax_fwd_tc(const __grid_co
             !mbar_wait_or_abort(&s->v_full[sp], up, SITE_OUT_TMA, abort_flag))
           return false;
         tc_fence_after();
-        const uint32_t aP = smem_u32(sP + sp * kTileBytes), aV = smem_u32(sV + sp * kTileBytes);
+        const uint32_t aV = smem_u32(sV + sp * kTileBytes);
         for (int kk = 0; kk < kTile / 16; ++kk)
-          mma_bf16(tmem + kColO, kmaj(aP, kk), mnmaj(aV, kk), id_kn, (jp > 0 || kk > 0) ? 1u : 0u);
+          mma_bf16_ts(tmem + kColO, tmem + kColP + 64 * sp + 8 * kk, mnmaj(aV, kk), id_kn,
+                      (jp > 0 || kk > 0) ? 1u : 0u);
         mma_commit(&s->pv_done[sp]);
         return true;
       };
@@ -278,26 +303,22 @@ __global__ void __launch_bounds__(kFwdThreads, 1) softmax_fwd_tc(const __grid_co
         l *= f;
         m_used = mt;
       }
-      // P into this stage's tile once the P V MMA of two tiles ago has read it
+      // P into this stage's TMEM buffer (this thread's 64 columns: K-steps 4
+      // half .. 4 half + 3) once the P V MMA of two tiles ago has read it
       if (j >= 2 && !bad &&
           !mbar_wait_or_abort(&s->pv_done[st], (uint32_t)((j - 2) >> 1) & 1u, SITE_OUT_MMA, abort_flag))
         bad = true;
-      uint8_t* pt = sP + st * kTileBytes;
       float rs = 0.f;
+      uint32_t pw[32];
 #pragma unroll
-      for (int c8 = 0; c8 < 8; ++c8) {
-        float p[8];
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          p[u] = ex2(x[c8 * 8 + u] - m_used);
-          rs += p[u];
-        }
-        st_tile16(pt, i, c0 + c8 * 8,
-                  make_uint4(pack_bf16(p[0], p[1]), pack_bf16(p[2], p[3]), pack_bf16(p[4], p[5]),
-                             pack_bf16(p[6], p[7])));
+      for (int u = 0; u < 32; ++u) {
+        const float p0 = ex2(x[2 * u] - m_used), p1 = ex2(x[2 * u + 1] - m_used);
+        rs += p0 + p1;
+        pw[u] = pack_bf16(p0, p1);
       }
+      tmem_st32(lane_base + kColP + 64 * st + 32 * half, pw);
+      tmem_st_wait();
       l += rs;
-      fence_async_smem();
       tc_fence_before();
       mbar_arrive(&s->p_full[st]);  // arrives even after a failure, so no waiter is left short
     }
@@ -382,21 +403,22 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
 }
 
 // Reads the S-type and dP-type accumulators of this thread's row (TMEM lane)
-// and column half, forms p = exp2(s c - lse2) (0 where masked) and
-// ds = p (dp - delta) per column, and stores both in bf16 into the two
-// operand tiles at (row, column). keep(u) says whether column half*64 + u is
-// inside the causal mask and the sequence; lse2 / dl give the column's (or the
-// row's) values through the callbacks.
-// Chunk cc (0 or 1) of the half: columns half * 64 + cc * 32 .. + 31, so that
-// chunk 0 of both halves is the tile's K-steps 0, 1, 4, 5 of the next MMA and
-// chunk 1 its K-steps 2, 3, 6, 7. visible = 1 (every column of the chunk inside
-// the mask) or 0 (none) skips the per-column test.
+// over the 32 columns of chunk cc of column half `half` (half * 64 + cc * 32
+// ..), forms p = exp2(s c - lse2) (0 where masked) and ds = p (dp - delta) per
+// column, and writes both back into TMEM in bf16, over the accumulator
+// columns this thread has just read, as the A operand of the next MMAs: the
+// 16 columns of pass ps (K-step kk = 2 sub + ps of those MMAs, sub = 2 half +
+// cc) into the 8 columns colS + 32 sub + 8 ps (P) and colP + 32 sub + 8 ps
+// (dS), two bf16 per column, the lower K index in the low half. Chunk 0 of
+// both halves is the MMAs' K-steps 0, 1, 4, 5, chunk 1 their K-steps 2, 3, 6,
+// 7. keep(c) says whether column c is inside the causal mask and the
+// sequence; lse2 / dl give the column's values through the callbacks;
+// visible = 1 (every column of the chunk inside the mask) or 0 (none) skips
+// the per-column test.
 template <class Keep, class Lse, class Dl>
-__device__ __forceinline__ void p_ds_rows(uint32_t lane_base, uint32_t colS, uint32_t colP, int row, int half,
-                                          int cc, float c2, uint8_t* tP, uint8_t* tDS, Keep keep, Lse lse2, Dl dl,
-                                          int visible = -1) {
+__device__ __forceinline__ void p_ds_rows_tmem(uint32_t lane_base, uint32_t colS, uint32_t colP, int half, int cc,
+                                               float c2, Keep keep, Lse lse2, Dl dl, int visible) {
   const int col0 = half * 64 + cc * 32;
-  // in two passes of 16 columns, so that the values of one pass stay in registers
 #pragma unroll 1
   for (int ps = 0; ps < 2; ++ps) {
     const int cb = col0 + ps * 16;
@@ -405,14 +427,14 @@ __device__ __forceinline__ void p_ds_rows(uint32_t lane_base, uint32_t colS, uin
     tmem_ld16(lane_base + colP + cb, rp);
     tmem_ld_wait();
     float p[16], ds[16];
-    if (visible == 1) {  // every column of the chunk is inside the mask
+    if (visible == 1) {
 #pragma unroll
       for (int u = 0; u < 16; ++u) {
         const int c = cb + u;
         p[u] = ex2(__uint_as_float(rs[u]) * c2 - lse2(c));
         ds[u] = p[u] * (__uint_as_float(rp[u]) - dl(c));
       }
-    } else if (visible == 0) {  // none is
+    } else if (visible == 0) {
 #pragma unroll
       for (int u = 0; u < 16; ++u) p[u] = ds[u] = 0.f;
     } else {
@@ -424,20 +446,20 @@ __device__ __forceinline__ void p_ds_rows(uint32_t lane_base, uint32_t colS, uin
         ds[u] = p[u] * (__uint_as_float(rp[u]) - dl(c));
       }
     }
+    uint32_t wp[8], wd[8];
 #pragma unroll
-    for (int q8 = 0; q8 < 2; ++q8) {
-      st_tile16(tP, row, cb + q8 * 8,
-                make_uint4(pack_bf16(p[q8 * 8], p[q8 * 8 + 1]), pack_bf16(p[q8 * 8 + 2], p[q8 * 8 + 3]),
-                           pack_bf16(p[q8 * 8 + 4], p[q8 * 8 + 5]), pack_bf16(p[q8 * 8 + 6], p[q8 * 8 + 7])));
-      st_tile16(tDS, row, cb + q8 * 8,
-                make_uint4(pack_bf16(ds[q8 * 8], ds[q8 * 8 + 1]), pack_bf16(ds[q8 * 8 + 2], ds[q8 * 8 + 3]),
-                           pack_bf16(ds[q8 * 8 + 4], ds[q8 * 8 + 5]), pack_bf16(ds[q8 * 8 + 6], ds[q8 * 8 + 7])));
+    for (int u = 0; u < 8; ++u) {
+      wp[u] = pack_bf16(p[2 * u], p[2 * u + 1]);
+      wd[u] = pack_bf16(ds[2 * u], ds[2 * u + 1]);
     }
+    tmem_st8(lane_base + colS + col0 + 8 * ps, wp);
+    tmem_st8(lane_base + colP + col0 + 8 * ps, wd);
   }
+  tmem_st_wait();
 }
 
 struct SmemDkdv {
-  uint64_t kv_full, full[3], empty[3], ld_full, s_full, p_half, p_full, mma2_done, drain;
+  uint64_t kv_full, full[3], empty[3], ld_full, s_full, p_half, p_full, dv_done, mma2_done, drain;
   uint32_t tmem_base;
   int abort;
   float lse2[kTile], dl[kTile];  // the current query tile's lse (log2 units) and delta
@@ -457,8 +479,8 @@ __global__ void __launch_bounds__(kDkdvThreads, 1) softmax_dkdv_tc(
   uint8_t* sK = base;
   uint8_t* sV = base + kTileBytes;
   uint8_t* ring = base + 2 * kTileBytes;  // three slots: Q_0, dO_0, Q_1, dO_1, ...
-  uint8_t* sPt = base + 5 * kTileBytes;   // P^T, then dK out
-  uint8_t* sDSt = base + 6 * kTileBytes;  // dS^T, then dV out
+  uint8_t* sPt = base + 5 * kTileBytes;   // dK out
+  uint8_t* sDSt = base + 6 * kTileBytes;  // dV out
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int kt = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const int64_t k0 = (int64_t)kt * kTile;
@@ -485,6 +507,7 @@ __global__ void __launch_bounds__(kDkdvThreads, 1) softmax_dkdv_tc(
     mbar_init(&s->s_full, 1);
     mbar_init(&s->p_half, 256);
     mbar_init(&s->p_full, 256);
+    mbar_init(&s->dv_done, 1);
     mbar_init(&s->mma2_done, 1);
     mbar_init(&s->drain, 1);
     s->abort = 0;
@@ -498,6 +521,8 @@ __global__ void __launch_bounds__(kDkdvThreads, 1) softmax_dkdv_tc(
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = s->tmem_base;
+  // S^T, then P^T (bf16, the dV MMA's A operand) over its first 64 columns;
+  // dP^T, then dS^T (the dK MMA's) likewise; the dV and dK accumulators
   constexpr uint32_t kColS = 0, kColP = 128, kColV = 256, kColK = 384;
 
   if (warp == 16) {
@@ -558,7 +583,7 @@ __global__ void __launch_bounds__(kDkdvThreads, 1) softmax_dkdv_tc(
     if (lane == 0 && n > 0) {
       constexpr uint32_t id_kk = idesc_bf16(128, 128, 0, 0);
       constexpr uint32_t id_kn = idesc_bf16(128, 128, 0, 1);
-      const uint32_t aK = smem_u32(sK), aV = smem_u32(sV), aP = smem_u32(sPt), aD = smem_u32(sDSt);
+      const uint32_t aK = smem_u32(sK), aV = smem_u32(sV);
       bool bad = !mbar_wait_or_abort(&s->kv_full, 0, SITE_BWD_TMA, abort_flag);
       for (int i = 0; i < n && !bad; ++i) {
         const int xq = 2 * i, xd = 2 * i + 1;
@@ -568,9 +593,20 @@ __global__ void __launch_bounds__(kDkdvThreads, 1) softmax_dkdv_tc(
           bad = true;
           break;
         }
+        // S^T overwrites P^T: the last tile's dV MMAs have read it (its dK
+        // MMAs are still running, so the wait costs little tensor time)
+        if (i > 0 && !mbar_wait_or_abort(&s->dv_done, (uint32_t)(i - 1) & 1u, SITE_BWD_MMA, abort_flag)) {
+          bad = true;
+          break;
+        }
         tc_fence_after();
         for (int kk = 0; kk < kD / 16; ++kk) mma_bf16(tmem + kColS, kmaj(aK, kk), kmaj(aQ, kk), id_kk, kk > 0);
         if (!mbar_wait_or_abort(&s->full[sd], (uint32_t)(xd / 3) & 1u, SITE_BWD_TMA, abort_flag)) {
+          bad = true;
+          break;
+        }
+        // dP^T overwrites dS^T: the last tile's dK MMAs have read it (under S^T)
+        if (i > 0 && !mbar_wait_or_abort(&s->mma2_done, (uint32_t)(i - 1) & 1u, SITE_BWD_MMA, abort_flag)) {
           bad = true;
           break;
         }
@@ -586,13 +622,17 @@ __global__ void __launch_bounds__(kDkdvThreads, 1) softmax_dkdv_tc(
             break;
           }
           tc_fence_after();
+          // K-step kk's A operand: 8 TMEM columns at 32 (kk / 2) + 8 (kk % 2)
           for (int q = 0; q < 4; ++q) {
             const int kk = (q >> 1) * 4 + pc * 2 + (q & 1);
-            mma_bf16(tmem + kColV, kmaj(aP, kk), mnmaj(aO, kk), id_kn, (i > 0 || pc > 0 || q > 0) ? 1u : 0u);
+            mma_bf16_ts(tmem + kColV, tmem + kColS + 32 * (kk >> 1) + 8 * (kk & 1), mnmaj(aO, kk), id_kn,
+                        (i > 0 || pc > 0 || q > 0) ? 1u : 0u);
           }
+          if (pc == 1) mma_commit(&s->dv_done);
           for (int q = 0; q < 4; ++q) {
             const int kk = (q >> 1) * 4 + pc * 2 + (q & 1);
-            mma_bf16(tmem + kColK, kmaj(aD, kk), mnmaj(aQ, kk), id_kn, (i > 0 || pc > 0 || q > 0) ? 1u : 0u);
+            mma_bf16_ts(tmem + kColK, tmem + kColP + 32 * (kk >> 1) + 8 * (kk & 1), mnmaj(aQ, kk), id_kn,
+                        (i > 0 || pc > 0 || q > 0) ? 1u : 0u);
           }
         }
         if (!part_ok) {
@@ -620,9 +660,8 @@ __global__ void __launch_bounds__(kDkdvThreads, 1) softmax_dkdv_tc(
       const int64_t q0 = (int64_t)(qt0 + i) * kTile;
       if (!bad && !mbar_wait_or_abort(&s->s_full, (uint32_t)i & 1u, SITE_BWD_MMA, abort_flag)) bad = true;
       if (!bad && !mbar_wait_or_abort(&s->ld_full, (uint32_t)i & 1u, SITE_BWD_TMA, abort_flag)) bad = true;
-      // P^T and dS^T are free once the last tile's dV and dK MMAs have read them
-      if (i > 0 && !bad && !mbar_wait_or_abort(&s->mma2_done, (uint32_t)(i - 1) & 1u, SITE_BWD_MMA, abort_flag))
-        bad = true;
+      // (the last tile's dV and dK MMAs, which read P^T and dS^T from TMEM,
+      // completed before this tile's S^T and dP^T were issued)
       bad = __any_sync(0xffffffffu, bad);  // the TMEM loads below are warp-collective
       const float* L = s->lse2;
       const float* Dl = s->dl;
@@ -633,10 +672,9 @@ __global__ void __launch_bounds__(kDkdvThreads, 1) softmax_dkdv_tc(
                           : (cfirst >= Nq || q_offset + clast < kpos) ? 0 : -1;
       if (!bad) {
         tc_fence_after();
-        p_ds_rows(lane_base, kColS, kColP, row, half, cc, c2, sPt, sDSt, keep, [&](int c) { return L[c]; },
-                  [&](int c) { return Dl[c]; }, visible);
+        p_ds_rows_tmem(lane_base, kColS, kColP, half, cc, c2, keep, [&](int c) { return L[c]; },
+                       [&](int c) { return Dl[c]; }, visible);
       }
-      fence_async_smem();
       tc_fence_before();
       mbar_arrive(cc == 0 ? &s->p_half : &s->p_full);  // the MMA takes each chunk as it is done
     }
@@ -712,7 +750,6 @@ __global__ void __launch_bounds__(kDqThreads, 1) softmax_dq_tc(
   uint8_t* sO = base + kTileBytes;      // dO
   uint8_t* sK = base + 2 * kTileBytes;  // two stages
   uint8_t* sV = base + 4 * kTileBytes;  // two stages
-  uint8_t* sDS = base + 6 * kTileBytes;
   SmemDq* s = reinterpret_cast<SmemDq*>(base + 7 * kTileBytes);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int qt = qtiles - 1 - (int)blockIdx.x;  // heaviest tiles first
@@ -751,7 +788,10 @@ __global__ void __launch_bounds__(kDqThreads, 1) softmax_dq_tc(
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = s->tmem_base;
-  constexpr uint32_t kColS = 0, kColP = 128, kColQ = 256;
+  // S, dP, the dQ accumulator; dS in bf16 (the dQ MMA's A operand: K-step kk
+  // in the 8 columns kColD + 8 kk, two bf16 per column, the lower K index in
+  // the low half)
+  constexpr uint32_t kColS = 0, kColP = 128, kColQ = 256, kColD = 384;
 
   if (warp == 16) {
     if (lane == 0) {
@@ -788,7 +828,7 @@ __global__ void __launch_bounds__(kDqThreads, 1) softmax_dq_tc(
     if (lane == 0) {
       constexpr uint32_t id_kk = idesc_bf16(128, 128, 0, 0);
       constexpr uint32_t id_kn = idesc_bf16(128, 128, 0, 1);
-      const uint32_t aQ = smem_u32(sQ), aO = smem_u32(sO), aD = smem_u32(sDS);
+      const uint32_t aQ = smem_u32(sQ), aO = smem_u32(sO);
       bool bad = !mbar_wait_or_abort(&s->qd_full, 0, SITE_BWD_TMA, abort_flag);
       for (int j = 0; j < nkv && !bad; ++j) {
         const int st = j & 1;
@@ -818,7 +858,8 @@ __global__ void __launch_bounds__(kDqThreads, 1) softmax_dq_tc(
           tc_fence_after();
           for (int q = 0; q < 4; ++q) {
             const int kk = (q >> 1) * 4 + pc * 2 + (q & 1);
-            mma_bf16(tmem + kColQ, kmaj(aD, kk), mnmaj(aK, kk), id_kn, (j > 0 || pc > 0 || q > 0) ? 1u : 0u);
+            mma_bf16_ts(tmem + kColQ, tmem + kColD + 8 * kk, mnmaj(aK, kk), id_kn,
+                        (j > 0 || pc > 0 || q > 0) ? 1u : 0u);
           }
         }
         if (!part_ok) {
@@ -850,7 +891,7 @@ __global__ void __launch_bounds__(kDqThreads, 1) softmax_dq_tc(
       const int lim = lim64 < -1 ? -1 : (lim64 > 31 ? 31 : (int)lim64);
       if (!bad && !mbar_wait_or_abort(&s->s_full, (uint32_t)j & 1u, SITE_BWD_MMA, abort_flag)) bad = true;
       if (j > 0 && !bad && !mbar_wait_or_abort(&s->dq_done, (uint32_t)(j - 1) & 1u, SITE_BWD_MMA, abort_flag))
-        bad = true;  // the last dQ MMA has read dS
+        bad = true;  // the last dQ MMAs have read dS
       bad = __any_sync(0xffffffffu, bad);  // the TMEM loads below are warp-collective
       if (!bad) {
         tc_fence_after();
@@ -877,15 +918,13 @@ __global__ void __launch_bounds__(kDqThreads, 1) softmax_dq_tc(
               ds[u] = p * (__uint_as_float(rp[u]) - dl);
             }
           }
+          uint32_t w[8];
 #pragma unroll
-          for (int q8 = 0; q8 < 2; ++q8)
-            st_tile16(sDS, row, cb + q8 * 8,
-                      make_uint4(pack_bf16(ds[q8 * 8], ds[q8 * 8 + 1]), pack_bf16(ds[q8 * 8 + 2], ds[q8 * 8 + 3]),
-                                 pack_bf16(ds[q8 * 8 + 4], ds[q8 * 8 + 5]),
-                                 pack_bf16(ds[q8 * 8 + 6], ds[q8 * 8 + 7])));
+          for (int u = 0; u < 8; ++u) w[u] = pack_bf16(ds[2 * u], ds[2 * u + 1]);
+          tmem_st8(lane_base + kColD + 16 * sub + 8 * ps, w);  // K-step 2 sub + ps
         }
+        tmem_st_wait();
       }
-      fence_async_smem();
       tc_fence_before();
       mbar_arrive(cc == 0 ? &s->ds_half : &s->ds_full);  // the MMA takes each chunk group as it is done
     }
