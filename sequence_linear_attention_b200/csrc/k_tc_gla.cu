@@ -814,14 +814,14 @@ struct SmemBwd {
 // (LASP Appendix A.4: the gated form of the gradient-state recurrence):
 //   R_{c-1} = diag(e^{b_end}) R_c + diag(e^{r}) Q^^T dO     (Q^ = q . e^{b - r})
 // with Q^^T dO an extra MMA of phase 2 into T0 (idle between epilogue 1 and
-// phase 3), combined in fp32 with R_c while phase 3's first MMAs run, and
-// written to a scratch slot of the segment (the workspace slot of its first
-// chunk), where the next tile's bulk load of R finds it. The scratch is
-// lane-major (float4 group g of state row m at float4 g * 128 + m), so that
-// the threads of a warp, which own consecutive rows, read and write one
-// 512-byte run per access; the scan's slot is row-major, so a segment's last
-// tile first copies its R_c into the scratch, and the combination always reads
-// R_c from there (L2).
+// phase 3), combined in fp32 with each thread's share of R_c (kept in
+// registers since phase 1 read it) while the T1 products run, and written to
+// a scratch slot of the segment (the workspace slot of its first chunk),
+// where the next tile's bulk load of R finds it. The scratch is lane-major
+// (float4 group g of state row m at float4 g * 128 + m), so that the threads
+// of a warp, which own consecutive rows, write one 512-byte run per access;
+// phase 1 reads R row-major from the scan's slot (a segment's last tile) or
+// lane-major from the scratch.
 //
 // The log-gate gradient's column sums over the tile's rows,
 //   dg_t = sum_{s >= t} dB_s + sum_{s < t} (k . dk^inter)_s + e^{b_end} <R_c, P_c>,
@@ -1015,13 +1015,6 @@ __global__ void __launch_bounds__(kBwdThreads, 1) gla_bwd_tc(
         const int g = qt * 8 + u;
         rreg[u] = R4[rlm ? g * kD + t : t * (kD / 4) + g];
       }
-      if (form && !rlm) {
-        // a segment's last tile: R_c into the scratch, lane-major, where this
-        // tile's own forming of R_{c-1} reads it back in one-run accesses
-        float4* rs = reinterpret_cast<float4*>(R + pslot_of(c - j, h, b) * kD * kD);
-#pragma unroll
-        for (int u = 0; u < 8; ++u) rs[(qt * 8 + u) * kD + t] = rreg[u];
-      }
     }
     named_sync(kBarAll, kBwdThreads);  // every row of R has been read: sA/sB are free
     {
@@ -1059,29 +1052,26 @@ __global__ void __launch_bounds__(kBwdThreads, 1) gla_bwd_tc(
     if (mbar_wait(&s->mma1a, ph, SITE_BWD_MMA)) {
       tc_fence_after();
 #pragma unroll 1
-      for (int c2 = 0; c2 < 2; ++c2) {
-        const int col0 = cq + c2 * 16;
-        uint32_t ra[16], rs[16];
-        tmem_ld16(lane_base + T0 + col0, ra);
-        tmem_ld16(lane_base + T1 + col0, rs);
+      for (int c2 = 0; c2 < 4; ++c2) {
+        const int col0 = cq + c2 * 8;
+        uint32_t ra[8], rs[8];
+        tmem_ld8(lane_base + T0 + col0, ra);
+        tmem_ld8(lane_base + T1 + col0, rs);
         tmem_ld_wait();
 #pragma unroll
-        for (int u = 0; u < 16; ++u)
+        for (int u = 0; u < 8; ++u)
           if (col0 + u == t) s->dAd[t] = __uint_as_float(ra[u]);
+        float fa[8], fs[8];
 #pragma unroll
-        for (int q4 = 0; q4 < 2; ++q4) {
-          float fa[8], fs[8];
-#pragma unroll
-          for (int u = 0; u < 8; ++u) {
-            const int col = col0 + q4 * 8 + u;
-            fa[u] = col < t ? __uint_as_float(ra[q4 * 8 + u]) : 0.f;
-            fs[u] = col <= t ? __uint_as_float(rs[q4 * 8 + u]) : 0.f;
-          }
-          *tile16(sA, t, col0 + q4 * 8) = make_uint4(pack_bf16(fa[0], fa[1]), pack_bf16(fa[2], fa[3]),
-                                                     pack_bf16(fa[4], fa[5]), pack_bf16(fa[6], fa[7]));
-          *tile16(sB, t, col0 + q4 * 8) = make_uint4(pack_bf16(fs[0], fs[1]), pack_bf16(fs[2], fs[3]),
-                                                     pack_bf16(fs[4], fs[5]), pack_bf16(fs[6], fs[7]));
+        for (int u = 0; u < 8; ++u) {
+          const int col = col0 + u;
+          fa[u] = col < t ? __uint_as_float(ra[u]) : 0.f;
+          fs[u] = col <= t ? __uint_as_float(rs[u]) : 0.f;
         }
+        *tile16(sA, t, col0) = make_uint4(pack_bf16(fa[0], fa[1]), pack_bf16(fa[2], fa[3]), pack_bf16(fa[4], fa[5]),
+                                          pack_bf16(fa[6], fa[7]));
+        *tile16(sB, t, col0) = make_uint4(pack_bf16(fs[0], fs[1]), pack_bf16(fs[2], fs[3]), pack_bf16(fs[4], fs[5]),
+                                          pack_bf16(fs[6], fs[7]));
       }
     } else {
       s->abort = 1;
@@ -1090,7 +1080,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1) gla_bwd_tc(
     tc_fence_before();
     __syncthreads();
     if (s->abort) goto cleanup;
-    // ---- phase 2: T2 += (dA . strict) K^ | T0 = Q^^T dO (when this tile forms R_{c-1})
+    // ---- phase 2: T2 += (dA . strict) K^ | T0 = Q^^T dO (when this tile forms
+    // R_{c-1}) | T1 = (A . causal)^T dO + K^ R' (phase 1's masks and R' are in
+    // place; T1 was read by epilogue 1)
     if (tid == 0) {
       tc_fence_after();
       for (int kk = 0; kk < kTile / 16; ++kk) mma_bf16(tmem + T2, kmaj(aA, kk), mnmaj(aK, kk), id_kn, 1);
@@ -1099,6 +1091,38 @@ __global__ void __launch_bounds__(kBwdThreads, 1) gla_bwd_tc(
         for (int kk = 0; kk < kTile / 16; ++kk) mma_bf16(tmem + T0, mnmaj(aQ, kk), mnmaj(aD, kk), id_nn, kk != 0);
         mma_commit(&s->mmar);
       }
+      for (int kk = 0; kk < kTile / 16; ++kk) mma_bf16(tmem + T1, mnmaj(aB, kk), mnmaj(aD, kk), id_nn, kk != 0);
+      for (int kk = 0; kk < kD / 16; ++kk) mma_bf16(tmem + T1, kmaj(aK, kk), mnmaj(aX, kk), id_kn, 1);
+    }
+    // ---- R_{c-1} = e^{b_end} R_c + e^{r} T0 (row t, columns cq..; R_c from
+    // this thread's registers, read in phase 1), under the T1 products, before
+    // epilogue 2 takes its registers; into the segment's scratch slot, lane-major
+    // (float4 group g of row t at g * 128 + t), where the next tile's bulk load
+    // of R finds it
+    if (form) {
+      float4* rn = reinterpret_cast<float4*>(R + pslot_of(c - j, h, b) * kD * kD);
+      if (mbar_wait(&s->mmar, rph, SITE_BWD_MMA)) {
+        tc_fence_after();
+#pragma unroll
+        for (int c2 = 0; c2 < 2; ++c2) {
+          uint32_t a[16];
+          tmem_ld16(lane_base + T0 + cq + c2 * 16, a);
+          tmem_ld_wait();
+#pragma unroll
+          for (int q4 = 0; q4 < 4; ++q4) {
+            const float4 r4 = rreg[c2 * 4 + q4];
+            rn[(qt * 8 + c2 * 4 + q4) * kD + t] =
+                make_float4(fmaf(eb, r4.x, er * __uint_as_float(a[4 * q4])),
+                            fmaf(eb, r4.y, er * __uint_as_float(a[4 * q4 + 1])),
+                            fmaf(eb, r4.z, er * __uint_as_float(a[4 * q4 + 2])),
+                            fmaf(eb, r4.w, er * __uint_as_float(a[4 * q4 + 3])));
+          }
+        }
+        fence_async_global();  // the next tile's bulk load of R reads these stores
+      } else {
+        s->abort = 1;
+      }
+      rph ^= 1u;
     }
     // ---- epilogue 2: dq' = E . T2; dq = dq' + (do_t . v_t) k_t = E . (T2 + (do_t . v_t) K^_t);
     // q . dq' = Q^ . T2 -> T2
@@ -1150,55 +1174,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1) gla_bwd_tc(
     tc_fence_before();
     __syncthreads();
     if (s->abort) goto cleanup;
-    // ---- phase 3: T1 = (A . causal)^T dO + K^ R', T3 = V R'^T while the
-    // threads form R_{c-1} from T0, then T0 = (dA . strict)^T Q^
+    // ---- phase 3: T3 = V R'^T, then T0 = (dA . strict)^T Q^ (every thread has
+    // read T0 for R_{c-1} before the barrier above)
     if (tid == 0) {
       tc_fence_after();
-      for (int kk = 0; kk < kTile / 16; ++kk) mma_bf16(tmem + T1, mnmaj(aB, kk), mnmaj(aD, kk), id_nn, kk != 0);
-      for (int kk = 0; kk < kD / 16; ++kk) mma_bf16(tmem + T1, kmaj(aK, kk), mnmaj(aX, kk), id_kn, 1);
       for (int kk = 0; kk < kD / 16; ++kk) mma_bf16(tmem + T3, kmaj(aV, kk), kmaj(aX, kk), id_kk, kk != 0);
-    }
-    // ---- R_{c-1} = e^{b_end} R_c + e^{r} T0 (row t, columns cq..), R_c read
-    // back from the scratch in L2 (this thread's elements only, so the slot is
-    // both source and destination; float4 group g of row t at g * 128 + t)
-    if (form) {
-      float4* rn = reinterpret_cast<float4*>(R + pslot_of(c - j, h, b) * kD * kD);
-      float4 rv[4];  // 16 columns of R_c at a time, the next pass's in flight under this one's math
-#pragma unroll
-      for (int q4 = 0; q4 < 4; ++q4) rv[q4] = rn[(qt * 8 + q4) * kD + t];
-      if (mbar_wait(&s->mmar, rph, SITE_BWD_MMA)) {
-        tc_fence_after();
-#pragma unroll 1
-        for (int c2 = 0; c2 < 2; ++c2) {
-          uint32_t a[16];
-          tmem_ld16(lane_base + T0 + cq + c2 * 16, a);
-          tmem_ld_wait();
-          float4 o4[4];
-#pragma unroll
-          for (int q4 = 0; q4 < 4; ++q4)
-            o4[q4] = make_float4(fmaf(eb, rv[q4].x, er * __uint_as_float(a[4 * q4])),
-                                 fmaf(eb, rv[q4].y, er * __uint_as_float(a[4 * q4 + 1])),
-                                 fmaf(eb, rv[q4].z, er * __uint_as_float(a[4 * q4 + 2])),
-                                 fmaf(eb, rv[q4].w, er * __uint_as_float(a[4 * q4 + 3])));
-          if (c2 == 0) {
-#pragma unroll
-            for (int q4 = 0; q4 < 4; ++q4) rv[q4] = rn[(qt * 8 + 4 + q4) * kD + t];
-          }
-#pragma unroll
-          for (int q4 = 0; q4 < 4; ++q4) rn[(qt * 8 + c2 * 4 + q4) * kD + t] = o4[q4];
-        }
-        fence_async_global();  // the next tile's bulk load of R reads these stores
-      } else {
-        s->abort = 1;
-      }
-      rph ^= 1u;
-    }
-    if (form) {
-      tc_fence_before();
-      named_sync(kBarAll, kBwdThreads);  // every thread has read its rows of T0
-    }
-    if (tid == 0) {
-      tc_fence_after();
       for (int kk = 0; kk < kTile / 16; ++kk) mma_bf16(tmem + T0, mnmaj(aA, kk), mnmaj(aQ, kk), id_nn, kk != 0);
       mma_commit(&s->mma3);
     }
