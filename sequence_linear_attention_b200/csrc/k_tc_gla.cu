@@ -1280,6 +1280,17 @@ __global__ void __launch_bounds__(kBwdThreads, 1) gla_bwd_tc(
       for (int kk = 0; kk < kTile / 16; ++kk)
         mma_bf16_ts(tmem + T0, tu + 32 * (kk >> 1) + 16 + 8 * (kk & 1), mnmaj(aKl, kk), id_kn, 1);
       mma_commit(&s->mmag);
+      if (has_next) {
+        // once the dK and dV stores have read sA / sB (the only bulk stores in
+        // flight), the next tile's gates go there, under the sums; a segment's
+        // entering R into L2 (a formed one is there)
+        tma_store_wait_read0();
+        int cn, hn, bn, jn;
+        tile_of(k + 1, cn, hn, bn, jn);
+        load_gate_tile(bt, &map_g, &s->gload, hn, cn * kTile, bn);
+        gate_out = (int)(ph ^ 1u);
+        if (jn == S - 1) bulk_prefetch_l2(R + rslot_of(cn, hn, bn, jn) * kD * kD, kD * kD * 4);
+      }
     }
     // dg_t = sum_{t' >= t} dB_t' + sum_{t' < t} k . dk^inter_t' + e^{b_end} <R_c, P_c>:
     // T0 plus bnd, into an fp32 tile over Q^ and K^ (the gate map's layout),
@@ -1321,13 +1332,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1) gla_bwd_tc(
         load_pprime(pslot_of(cn, hn, bn));
         tok_out = (int)(ph ^ 1u);
       }
-      tma_store_wait_read0();  // the dK, dV and dg stores have read sA / sB and fB (over Q and K)
+      tma_store_wait_read0();  // the dg store has read fB (over Q and K)
       if (next) {
-        // the next tile's gates into the gate tile's space; a segment's
-        // entering R into L2 (a formed one is there)
-        load_gate_tile(bt, &map_g, &s->gload, hn, cn * kTile, bn);
-        gate_out = (int)(ph ^ 1u);
-        if (jn == S - 1) bulk_prefetch_l2(R + rslot_of(cn, hn, bn, jn) * kD * kD, kD * kD * 4);
         load_tokens(sQ, &map_q, hn, cn * kTile, bn);
         load_tokens(sK, &map_k, hn, cn * kTile, bn);
       }
