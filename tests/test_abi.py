@@ -177,6 +177,38 @@ def test_split_calls_reject_bad_arguments(lib):
     assert bf(A, A, A, None, A, A, A, A, 1, 2, 512, 64, 64, F32, A, A, A + 4, None, None) == MISALIGNED
 
 
+def test_softmax_calls_reject_bad_arguments(lib):
+    """LASP-2H's softmax-attention calls validate on the host: types and sizes
+    the tensor cores do not take, a query without its own key (q_offset + Nq >
+    Nk), a scale that is not a positive finite number, missing or misaligned
+    buffers; and calls with nothing to do return before any launch."""
+    inf, nan = float("inf"), float("nan")
+    f = lib.lasp_softmax_fwd
+    #      q  k  v  o  lse  B  H  Nq   Nk   off  d    scale  dtype
+    assert f(A, A, A, A, A, 1, 2, 256, 256, 0, 64, 0.125, BF16, None) == UNSUPPORTED   # d = 64
+    assert f(A, A, A, A, A, 1, 2, 256, 256, 0, 128, 0.125, F32, None) == UNSUPPORTED   # fp32
+    assert f(A, A, A, A, A, 1, 2, 256, 256, 0, 128, 0.125, 7, None) == INVALID         # no such type
+    assert f(A, A, A, A, A, 0, 2, 256, 256, 0, 128, 0.125, BF16, None) == INVALID      # B = 0
+    assert f(A, A, A, A, A, 1, 2, 256, 200, 0, 128, 0.125, BF16, None) == INVALID      # keys short
+    assert f(A, A, A, A, A, 1, 2, 128, 256, 129, 128, 0.125, BF16, None) == INVALID    # offset past Nk
+    assert f(A, A, A, A, A, 1, 2, 128, 256, -1, 128, 0.125, BF16, None) == INVALID     # negative offset
+    for bad in (0.0, -0.125, inf, nan):
+        assert f(A, A, A, A, A, 1, 2, 256, 256, 0, 128, bad, BF16, None) == INVALID, bad
+    assert f(A, A, A, A, None, 1, 2, 256, 256, 0, 128, 0.125, BF16, None) == INVALID   # no lse
+    assert f(A, A + 8, A, A, A, 1, 2, 256, 256, 0, 128, 0.125, BF16, None) == MISALIGNED
+    assert f(None, None, None, None, None, 1, 2, 0, 256, 0, 128, 0.125, BF16, None) == OK  # no query
+    g = lib.lasp_softmax_bwd
+    #      q  k  v  o  lse dout dq dk dv delta  B  H  Nq   Nk   off  d    scale  dtype
+    assert g(A, A, A, A, A, A, A, A, A, A, 1, 2, 256, 256, 0, 64, 0.125, BF16, None) == UNSUPPORTED
+    assert g(A, A, A, A, A, A, A, A, A, A, 1, 2, 256, 200, 0, 128, 0.125, BF16, None) == INVALID
+    assert g(A, A, A, A, A, A, A, None, A, A, 1, 2, 256, 256, 0, 128, 0.125, BF16, None) == INVALID  # no dk
+    assert g(A, A, A, A, A, A, A, A, A, None, 1, 2, 256, 256, 0, 128, 0.125, BF16, None) == INVALID  # no delta
+    assert g(A, A, A, A, A, A, A, A, A + 4, A, 1, 2, 256, 256, 0, 128, 0.125, BF16, None) == MISALIGNED
+    assert g(A, A, A, A, A, A, A, A, A, A, 1, 2, 256, 256, 0, 128, nan, BF16, None) == INVALID
+    # no key and no query: nothing to write
+    assert g(None, A, A, None, None, None, None, A, A, None, 1, 2, 0, 0, 0, 128, 0.125, BF16, None) == OK
+
+
 def test_the_header_serves_a_plain_c_program(tmp_path, lib):
     """include/lasp.h compiles as strict C99, and a C program linked against
     the library calls it without torch: host-side calls that return before any
