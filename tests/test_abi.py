@@ -209,6 +209,88 @@ def test_softmax_calls_reject_bad_arguments(lib):
     assert g(None, A, A, None, None, None, None, A, A, None, 1, 2, 0, 0, 0, 128, 0.125, BF16, None) == OK
 
 
+def test_per_chunk_calls_reject_bad_arguments(lib):
+    """lasp_chunk_out (row a3 on given states) and lasp_chunk_grads (row a6)."""
+    f = lib.lasp_chunk_out
+    #        q  k  v  decay  P     o  B  H  N    d   C   dtype
+    assert f(A, A, A, None, A, A, 1, 2, 512, 96, 64, BF16, None) == UNSUPPORTED        # d = 96
+    assert f(A, A, A, None, A, A, 1, 2, 500, 64, 64, BF16, None) == INVALID            # C does not divide N
+    assert f(A, A, A, None, A, A, 1, 2, 512, 64, 64, 9, None) == INVALID               # no such type
+    assert f(A, A, A, None, None, A, 1, 2, 512, 64, 64, BF16, None) == INVALID         # no states
+    assert f(A, A, A, A + 4, A, A, 1, 2, 512, 64, 64, BF16, None) == MISALIGNED        # decay
+    assert f(None, None, None, None, None, None, 1, 2, 0, 64, 64, BF16, None) == OK    # empty
+    g = lib.lasp_chunk_grads
+    #        q  k  v  dout decay P  R     dq dk dv     B  H  N    d   C   dtype
+    assert g(A, A, A, A, None, A, None, A, A, A, 1, 2, 512, 64, 64, BF16, None) == INVALID     # no R
+    assert g(A, A, A, A, None, A, A, A, A, A + 8, 1, 2, 512, 64, 64, BF16, None) == MISALIGNED
+    assert g(A, A, A, A, None, A, A, A, A, A, 0, 2, 512, 64, 64, BF16, None) == INVALID        # B = 0
+    assert g(None, None, None, None, None, None, None, None, None, None, 1, 2, 0, 64, 64, F32, None) == OK
+
+
+def test_noalloc_backward_rejects_on_the_host(lib):
+    """lasp_bwd_noalloc checks sizes, pointers and its fixed workspace's limit
+    (B (N / C) H d^2 4 bytes within LASP_NOALLOC_SCRATCH_BYTES) before it looks
+    up the workspace on the device."""
+    f = lib.lasp_bwd_noalloc
+    #      q  k  v  decay dout dq dk dv  B  H  N     d    C    dtype cache dstate_in dinit
+    assert f(A, A, A, None, A, A, A, A, 1, 2, 512, 96, 64, BF16, A, None, None, None) == UNSUPPORTED
+    assert f(A, A, A, None, A, A, A, A, 1, 2, 500, 64, 64, BF16, A, None, None, None) == INVALID
+    assert f(A, A, A, None, A, A, A, A, 1, 2, 512, 64, 64, BF16, None, None, None, None) == INVALID  # no cache
+    assert f(A, A, A, None, A, A, A, A, 1, 2, 512, 64, 64, BF16, A, A + 4, None, None) == MISALIGNED
+    # 1 x 16 heads x 64 chunks of 128 x 128 fp32 states: 64 MiB, beyond the array
+    assert f(A, A, A, None, A, A, A, A, 1, 16, 8192, 128, 128, BF16, A, None, None, None) == UNSUPPORTED
+    assert f(None, None, None, None, None, None, None, None, 1, 2, 0, 64, 64, BF16, None, None, None,
+             None) == OK
+
+
+def test_part_calls_reject_bad_arguments(lib):
+    """The split calls restricted to part `part` of `nparts` of the (b, h)
+    pairs: 0 <= part < nparts <= B H, and nparts > 1 only where both walks run
+    (lasp_parts_ok)."""
+    ok = lib.lasp_parts_ok
+    assert ok(65536, 128, 128, BF16) == 1
+    assert ok(1024, 64, 128, BF16) == 1          # chunks that divide the tile
+    assert ok(1024, 128, 64, BF16) == 0          # d = 64: per-chunk kernels
+    assert ok(1024, 128, 128, F32) == 0
+    assert ok(320, 64, 128, BF16) == 0           # a ragged tile
+    assert ok(0, 128, 128, BF16) == 0
+    fs = lib.lasp_fwd_states_part
+    #         k  v  decay B  H  N     d    C    dtype cache total part nparts
+    assert fs(A, A, None, 1, 4, 1024, 128, 128, BF16, A, None, 0, 0, None) == INVALID      # nparts = 0
+    assert fs(A, A, None, 1, 4, 1024, 128, 128, BF16, A, None, 4, 4, None) == INVALID      # part = nparts
+    assert fs(A, A, None, 1, 4, 1024, 128, 128, BF16, A, None, -1, 2, None) == INVALID
+    assert fs(A, A, None, 1, 4, 1024, 128, 128, BF16, A, None, 0, 5, None) == INVALID      # nparts > B H
+    assert fs(A, A, None, 1, 4, 1024, 64, 128, BF16, A, None, 0, 2, None) == UNSUPPORTED   # not parts_ok
+    assert fs(A, A, None, 1, 4, 1024, 128, 128, BF16, None, None, 0, 2, None) == INVALID   # no cache
+    assert fs(A, A, None, 1, 4, 1024, 128, 128, BF16, A, A + 4, 1, 2, None) == MISALIGNED  # total
+    bf = lib.lasp_bwd_finish_part
+    #         q  k  v  decay dout dq dk dv  B  H  N     d    C    dtype cache ws   din   dinit part nparts
+    assert bf(A, A, A, None, A, A, A, A, 1, 4, 1024, 128, 128, BF16, A, None, None, None, 0, 2,
+              None) == INVALID                                                           # no workspace
+    assert bf(A, A, A, None, A, A, A, A, 1, 4, 1024, 128, 128, BF16, A, A, None, A + 8, 1, 2,
+              None) == MISALIGNED                                                        # dinit_state
+    assert bf(A, A, A, None, A, A, A, A, 1, 4, 1024, 128, 128, BF16, A, A, None, None, 2, 2,
+              None) == INVALID                                                           # part = nparts
+
+
+def test_kernel_names_and_segment_length(lib):
+    """The trace's kernel names are stable (bench.py keys its byte model on
+    them), and lasp_segment_tokens is host arithmetic: about 1024 tokens, a
+    multiple of the tile and of the chunk that divides N, or C off the walks."""
+    names = {lasp.lasp_kernel_name(i) for i in range(64)}
+    for n in ("segment_states_tc", "segment_scan", "fwd_walk_tc", "bwd_walk_tc", "state_scan", "chunk_states_tc",
+              "chunk_out_tc", "chunk_bwd_tc", "gla_bwd_tc", "softmax_dkdv_tc", "softmax_dq_tc", "softmax_fwd_tc"):
+        assert n in names, n
+    assert lasp.lasp_kernel_name(-1) == "unknown"
+    seg = lasp.lasp_segment_tokens
+    assert seg(65536, 128, 128, BF16) == 1024
+    assert seg(1152, 128, 128, BF16) == 384      # nine tiles: three segments of three
+    assert seg(256, 64, 128, BF16) == 256
+    assert seg(320, 64, 128, BF16) == 64         # not a multiple of the tile: per chunk
+    assert seg(256, 64, 32, F32) == 64
+    assert seg(100, 64, 128, BF16) == 0          # C does not divide N
+
+
 def test_the_header_serves_a_plain_c_program(tmp_path, lib):
     """include/lasp.h compiles as strict C99, and a C program linked against
     the library calls it without torch: host-side calls that return before any
