@@ -134,7 +134,7 @@ MEASURED_TRAFFIC = {
     "segment_states_tc": (["k_tc_states.cu", "sm100.cuh", "lasp_common.cuh", "tma_host.h"], "48a5dd38bfe5a0ce",
                           2 * (268479488 + 8521472)),
     # the gated form (bench.py --gated): four times the capture of the 16384-token case
-    "gla_bwd_tc": (["k_tc_gla.cu", "sm100.cuh", "lasp_common.cuh", "tma_host.h"], "1148561c16afbc45",
+    "gla_bwd_tc": (["k_tc_gla.cu", "sm100.cuh", "lasp_common.cuh", "tma_host.h"], "0ccaa17fdf1decfe",
                    4 * (491264256 + 320168704)),
 }
 

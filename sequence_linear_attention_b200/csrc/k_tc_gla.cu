@@ -147,14 +147,6 @@ __device__ __forceinline__ void load_gate_tile(float* bt, const CUtensorMap* map
   for (int cb = 0; cb < 4; ++cb) tma_load_4d(bt + cb * (kTile * 32), map_g, bar, cb * 32, h, row0, b);
 }
 
-// Four fp32 entries (columns 4 lane .. 4 lane + 3) of state row m, times w,
-// into the bf16 operand tile. Warp w converts rows w, w + 8, ...
-__device__ __forceinline__ void put_state_row(uint8_t* tile, int m, int lane, float4 x, float w) {
-  const int col = lane * 4;
-  const uint32_t off = (col >> 6) * kBox + sw128_offset(m, (col & 63) >> 3) + (col & 7) * 2;
-  *reinterpret_cast<uint2*>(tile + off) = make_uint2(pack_bf16(x.x * w, x.y * w), pack_bf16(x.z * w, x.w * w));
-}
-
 // ---------------------------------------------------------------- states
 struct SmemStates {
   uint64_t load, mma;
@@ -733,12 +725,6 @@ __device__ __forceinline__ void tmem_ld8(uint32_t taddr, uint32_t (&r)[8]) {
   asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
                : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
                : "r"(taddr));
-}
-
-__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&r)[8]) {
-  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"r"(taddr),
-               "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
-               : "memory");
 }
 
 __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
